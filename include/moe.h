@@ -1,0 +1,208 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) routed-MoE SwiGLU expert forward.
+ *
+ * The path: router softmax/top-k -> permute of every (token, expert) route
+ * into expert-contiguous rows -> gate/up grouped GEMM with SwiGLU fused into
+ * its epilogue -> down-projection grouped GEMM -> probability-weighted
+ * combine accumulated in fp32 in ascending expert-id order.  All work is
+ * bounded by a live-row count that lives in device memory, so one CUDA-graph
+ * capture serves every step.
+ *
+ * Sources (page title, section):
+ *   [P1] Megatron-LM PR #7830 ("flashinfer_mega" backend): "1. Mega backend
+ *        for generation" -- kernel weight layout rebuilt into a caller-owned
+ *        buffer on refit (refresh_mega_weights), canonical expert-id order
+ *        before the combine, MXFP8 quantisation per block of 32.
+ *   [P2] Megatron-LM PR #7798 (moe_training_matches_inference): "Background"
+ *        (activation fused into FC1's epilogue, probabilities applied after
+ *        FC2) and "What is changed" (a token's routes summed as fp32 fused
+ *        multiply-adds of probability and row, from zero, in a fixed order).
+ *   [P3] Megatron-LM PR #8367 ("bound the FlashInfer MoE expert kernels by
+ *        token count"): "Problem" -- the live token count is known only on
+ *        the device; results are returned in fp32.
+ *   [P4] core.transformer.moe.training_matches_inference API doc: `_route`
+ *        ([tokens, topk] probs and ids) and `expert_value_pass` (rows sorted
+ *        by local expert).
+ *   [P5] cudnn-frontend PR #448 (MoeEp API): MXFP8 uses 32-element blocks.
+ *
+ * Conventions for every entry point:
+ *   - Every pointer named *_dev or described as "device" is a device pointer
+ *     the caller allocated; the library never allocates or frees device
+ *     memory and never synchronises the stream, except where stated
+ *     (moe_get_device_status).
+ *   - `stream` is a cudaStream_t (CUstream) passed as void*; NULL is the
+ *     legacy default stream.
+ *   - bf16 tensors are passed as void* to 16-bit bfloat16 elements.
+ *   - Row-major layouts, dense, no padding between rows unless an ld_* stride
+ *     is given.
+ *   - Host-detectable errors (null pointers, bad sizes, misalignment, a too
+ *     small buffer) return a status before anything is launched.  Conditions
+ *     found on the device set bits in a status word inside the workspace
+ *     (MOE_DEV_*) and never trap, fault or hang.
+ *   - moe_forward, moe_route_topk and mxfp8_quantize_block32 enqueue work
+ *     only, so they may be captured into a CUDA graph.
+ *   - A plan is immutable after creation and may be shared by threads; use
+ *     one workspace per concurrently running stream.
+ */
+#ifndef ROUTED_MOE_SWIGLU_B200_MOE_H
+#define ROUTED_MOE_SWIGLU_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,          /* null pointer, negative size, bad enum   */
+    MOE_ERR_UNSUPPORTED = 2,          /* shape outside the supported envelope    */
+    MOE_ERR_ALIGNMENT = 3,            /* pointer or stride not 16-byte aligned   */
+    MOE_ERR_WORKSPACE_TOO_SMALL = 4,  /* workspace / weight buffer too small     */
+    MOE_ERR_CUDA = 5,                 /* a CUDA runtime call failed              */
+    MOE_ERR_NOT_PREPARED = 6          /* reserved: weight buffer not prepared    */
+} moe_status;
+
+typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1 } moe_precision;
+
+/* Device status bits (sticky until moe_clear_device_status). */
+#define MOE_DEV_LIVE_CLAMPED 0x1u  /* live count < 0 or > max live rows: clamped    */
+#define MOE_DEV_BAD_ROUTE 0x2u     /* caller ids out of [0,E) or repeated in a token:
+                                      that token's output row is all zeros          */
+#define MOE_DEV_TIMEOUT 0x4u       /* a bounded on-device wait gave up; outputs of
+                                      that call are not valid                       */
+
+typedef struct {
+    int hidden;              /* H: model width (K of the gate/up GEMM)            */
+    int ffn;                 /* F: expert intermediate width (K of the down GEMM) */
+    int num_experts;         /* E                                                 */
+    int top_k;               /* k: routes per token                               */
+    long long capacity;      /* rows of the caller's preallocated token buffers   */
+    long long max_live_rows; /* largest live count a call will pass (<= capacity);
+                                0 means capacity.  The workspace is sized for it;
+                                larger live counts are clamped and flagged.       */
+    moe_precision precision; /* MOE_BF16 or MOE_MXFP8                             */
+} moe_desc;
+
+typedef struct moe_plan moe_plan; /* opaque, host memory only */
+
+/* Validate `desc` and build a host-side plan (no device work, no device
+ * allocation).  Rejected (MOE_ERR_UNSUPPORTED): H or F not a multiple of 8
+ * (bf16) or of 32 (MXFP8); k < 1, k > 16 or k > E; E < 1 or E > 1024;
+ * capacity < 1 or > 2^24 rows; max_live_rows < 0 or > capacity;
+ * H > 16384 or F > 16384. */
+moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out);
+void moe_plan_destroy(moe_plan* plan);
+/* Copy of the descriptor the plan was made from (max_live_rows resolved). */
+moe_status moe_plan_get_desc(const moe_plan* plan, moe_desc* desc_out);
+
+/* Bytes of the caller-owned kernel-layout weight buffer and of the
+ * per-stream workspace (routes, permutation, tile list, intermediate rows,
+ * status word).  Both buffers must be 256-byte aligned. */
+size_t moe_weight_buffer_bytes(const moe_plan* plan);
+size_t moe_workspace_bytes(const moe_plan* plan);
+
+/* Rebuild the kernel-layout weight buffer in place from the experts' bf16
+ * weights ([P1] "refresh_mega_weights": a refit rewrites the same buffer; no
+ * allocation, no teardown).  Inputs (device, bf16, row-major):
+ *   w_gate [E, F, H], w_up [E, F, H]  (gate and up projections)
+ *   w_down [E, H, F]                  (down projection)
+ * In MXFP8 the weights are quantised here (blocks of 32 along each GEMM's K:
+ * H for gate/up, F for down).  Enqueued on `stream`; forwards enqueued later
+ * on the same stream see the new weights, forwards enqueued earlier finish
+ * with the old ones.  Returns MOE_ERR_WORKSPACE_TOO_SMALL if buf_bytes <
+ * moe_weight_buffer_bytes. */
+moe_status moe_prepare_weights(const moe_plan* plan, const void* w_gate, const void* w_up,
+                               const void* w_down, void* kernel_buf, size_t buf_bytes,
+                               void* stream);
+
+/* MXFP8 quantisation ([P1], [P5]; OCP MX v1.0): each row of `in` (bf16,
+ * [rows, cols], row stride ld_in elements) is cut into blocks of 32; each
+ * block gets the E8M0 scale byte floor(log2(amax)) - 8 + 127 (clamped to
+ * [0, 254]; 0 for an all-zero block) and E4M3 codes of value/scale rounded
+ * to nearest-even, saturating to +-448, sign kept.
+ *   q      [rows, cols] uint8 codes (row stride cols)
+ *   scales [rows, cols/32] uint8 E8M0 bytes (row stride cols/32)
+ * live_rows_dev: nullable device int32; when given, only rows
+ * [0, min(max(*live_rows_dev,0), rows)) are written.
+ * cols must be a positive multiple of 32, ld_in >= cols and a multiple of 8,
+ * `in` 16-byte aligned. */
+moe_status mxfp8_quantize_block32(const void* in, long long rows, int cols, long long ld_in,
+                                  uint8_t* q, uint8_t* scales, const int* live_rows_dev,
+                                  void* stream);
+
+/* Router ([P4] `_route`): for each live row t of logits (fp32 [capacity, E]),
+ * softmax over the E experts, the k largest (ties: lower expert id), the k
+ * probabilities renormalised to sum to 1; written in ascending expert id
+ * ([P1] canonical order).  ids int32 [capacity, k], probs fp32 [capacity, k];
+ * rows >= the live count are not read or written.  live_count_dev: device
+ * int32, clamped to [0, max_live_rows] (no status word here: no workspace). */
+moe_status moe_route_topk(const moe_plan* plan, const float* logits, const int* live_count_dev,
+                          int* ids, float* probs, void* stream);
+
+/* The routed SwiGLU expert forward.
+ *   x        bf16 [capacity, H]: token rows; only rows < live count are read.
+ *   logits   fp32 [capacity, E] or NULL: routed here as moe_route_topk does;
+ *   ids      int32 [capacity, k] and probs fp32 [capacity, k], or both NULL:
+ *            an outside router's routes in any order; they are put in
+ *            ascending id order with their probabilities, not renormalised.
+ *            Exactly one of `logits` or (`ids`, `probs`) must be given.
+ *   kernel_buf  the buffer moe_prepare_weights filled.
+ *   live_count_dev  device int32 live row count (clamped, flagged).
+ *   out      fp32 [capacity, H]: row t < live count gets
+ *            sum over its routes j in ascending expert id of
+ *            p_j * y_j as fp32 FMAs from 0.0f, where
+ *            y_j = W_down[e_j] . (silu(W_gate[e_j] . x_t) * (W_up[e_j] . x_t))
+ *            with the SwiGLU row rounded to bf16 (or re-quantised to MXFP8)
+ *            and y_j kept in fp32.  Rows >= live count are not written.
+ *   workspace  moe_workspace_bytes(plan) bytes, 256-byte aligned.
+ * Each token's output is bitwise independent of the live count and of the
+ * other tokens in the launch. */
+moe_status moe_forward(const moe_plan* plan, const void* x, const float* logits, const int* ids,
+                       const float* probs, const void* kernel_buf, const int* live_count_dev,
+                       float* out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Views into a workspace after a forward (device pointers into it), for
+ * tests and diagnostics:
+ *   route_ids/route_probs [max_live, k]: canonical routes of the last forward
+ *   offsets int32 [E+1]: first row of each expert in the permuted order
+ *   perm    int32 [routes]: permuted row r holds route t*k + j
+ *   inv     int32 [max_live, k]: padded intermediate row of route (t, j)
+ *   pad_offsets int32 [E+1]: first padded intermediate row of each expert
+ *   h       intermediate rows (bf16 [rows_padded, F], or E4M3 codes)
+ *   h_scales E8M0 scale bytes of h in the GEMM's scale layout (MXFP8) or NULL
+ *   xq / xq_scales permuted quantised x rows (MXFP8) or NULL */
+typedef struct {
+    const int* route_ids;
+    const float* route_probs;
+    const int* offsets;
+    const int* perm;
+    const int* inv;
+    const int* pad_offsets;
+    const void* h;
+    const uint8_t* h_scales;
+    const void* xq;
+    const uint8_t* xq_scales;
+    long long rows_padded; /* rows of the padded intermediate buffers */
+    const unsigned* status; /* device status word */
+} moe_workspace_views;
+moe_status moe_get_workspace_views(const moe_plan* plan, const void* workspace,
+                                   moe_workspace_views* views);
+
+/* Copy the workspace's device status word to *flags_host.  Synchronises
+ * `stream` (the only call that does). */
+moe_status moe_get_device_status(const void* workspace, unsigned* flags_host, void* stream);
+/* Zero the status word (enqueued on `stream`). */
+moe_status moe_clear_device_status(void* workspace, void* stream);
+
+/* Static string for a status code. */
+const char* moe_status_string(moe_status s);
+
+/* Library version, e.g. "0.1.0". */
+const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ROUTED_MOE_SWIGLU_B200_MOE_H */

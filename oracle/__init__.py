@@ -1,0 +1,201 @@
+"""CPU oracle for the routed-MoE SwiGLU expert forward (test infrastructure).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It wraps ``moe_oracle.c`` (plain C,
+fp64 sums, one token at a time) through ctypes and numpy; it shares no code
+with the CUDA library and never imports it.  Each function cites the page
+and section it follows in ``moe_oracle.c``.
+
+Parity pins: every function here is checked in ``tests/test_oracle_pins.py``
+against closed forms, library special cases or brute force (see the header
+of that file for which pin covers which mistake).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libmoe_oracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c into oracle/libmoe_oracle.so (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=gnu11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+               "-shared", "-fPIC", "-o", _LIB_PATH + ".tmp", _SRC, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(_LIB_PATH + ".tmp", _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB_PATH)
+    P = ctypes.c_void_p
+    I64 = ctypes.c_int64
+    I = ctypes.c_int
+    lib.oracle_threads.restype = I
+    lib.oracle_e4m3_value.restype = ctypes.c_double
+    lib.oracle_e4m3_value.argtypes = [I]
+    lib.oracle_mxfp8_quantize.argtypes = [P, I64, I64, P, P]
+    lib.oracle_mxfp8_quantize_bf16.argtypes = [P, I64, I64, P, P]
+    lib.oracle_mxfp8_dequantize.argtypes = [P, P, I64, I64, P]
+    lib.oracle_route.argtypes = [P, I64, I, I, P, P]
+    lib.oracle_permute.argtypes = [P, I64, I, I, P, P, P]
+    lib.oracle_forward_bf16.argtypes = [P, P, P, P, P, P, I64, I, I, I, I, P, I64, P, P]
+    lib.oracle_forward_mxfp8.argtypes = [P, P, P, P, P, P, P, P, P, I64, I, I, I, I, P, I64, P, P, P, P]
+    for name in ("oracle_mxfp8_quantize", "oracle_mxfp8_quantize_bf16", "oracle_mxfp8_dequantize",
+                 "oracle_route", "oracle_permute", "oracle_forward_bf16", "oracle_forward_mxfp8"):
+        getattr(lib, name).restype = I
+    _lib = lib
+    return lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle buffers must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise RuntimeError(f"oracle {what} failed with code {rc}")
+
+
+def _bf16_bits(a) -> np.ndarray:
+    """Accept a torch bf16 tensor or a uint16 numpy array of bf16 bit patterns."""
+    if isinstance(a, np.ndarray):
+        assert a.dtype == np.uint16
+        return np.ascontiguousarray(a)
+    import torch  # plain CPU tensor handling only
+
+    assert a.dtype == torch.bfloat16
+    return np.ascontiguousarray(a.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def threads() -> int:
+    return int(_load().oracle_threads())
+
+
+def e4m3_value(code: int) -> float:
+    return float(_load().oracle_e4m3_value(int(code)))
+
+
+def route(logits: np.ndarray, k: int):
+    """Top-k routing of fp32 logits [T, E] -> (ids int32 [T,k] ascending, probs fp32 [T,k])."""
+    lg = np.ascontiguousarray(logits, dtype=np.float32)
+    T, E = lg.shape
+    ids = np.empty((T, k), np.int32)
+    probs = np.empty((T, k), np.float32)
+    _check(_load().oracle_route(_ptr(lg), T, E, k, _ptr(ids), _ptr(probs)), "route")
+    return ids, probs
+
+
+def permute(ids: np.ndarray, num_experts: int):
+    """Stable expert permutation -> (offsets int64 [E+1], perm int32 [R], inv int32 [T,k])."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, k = ids.shape
+    offsets = np.empty(num_experts + 1, np.int64)
+    perm = np.empty(T * k, np.int32)
+    inv = np.empty((T, k), np.int32)
+    _check(_load().oracle_permute(_ptr(ids), T, num_experts, k, _ptr(offsets), _ptr(perm), _ptr(inv)),
+           "permute")
+    return offsets, perm, inv
+
+
+def mxfp8_quantize(values: np.ndarray):
+    """fp32 [rows, cols] (cols % 32 == 0) -> (codes uint8 [rows, cols], scales uint8 [rows, cols/32])."""
+    v = np.ascontiguousarray(values, dtype=np.float32)
+    rows, cols = v.shape
+    q = np.empty((rows, cols), np.uint8)
+    s = np.empty((rows, cols // 32), np.uint8)
+    _check(_load().oracle_mxfp8_quantize(_ptr(v), rows, cols, _ptr(q), _ptr(s)), "mxfp8_quantize")
+    return q, s
+
+
+def mxfp8_quantize_bf16(bits) -> tuple[np.ndarray, np.ndarray]:
+    """bf16 (torch tensor or uint16 bits) [..., cols] -> codes [..., cols], scales [..., cols/32]."""
+    b = _bf16_bits(bits)
+    shape = b.shape
+    cols = shape[-1]
+    rows = int(np.prod(shape[:-1])) if len(shape) > 1 else 1
+    q = np.empty(shape, np.uint8)
+    s = np.empty(shape[:-1] + (cols // 32,), np.uint8)
+    _check(_load().oracle_mxfp8_quantize_bf16(_ptr(b), rows, cols, _ptr(q), _ptr(s)), "mxfp8_quantize_bf16")
+    return q, s
+
+
+def mxfp8_dequantize(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    s = np.ascontiguousarray(s, dtype=np.uint8)
+    cols = q.shape[-1]
+    rows = int(np.prod(q.shape[:-1])) if q.ndim > 1 else 1
+    out = np.empty(q.shape, np.float32)
+    _check(_load().oracle_mxfp8_dequantize(_ptr(q), _ptr(s), rows, cols, _ptr(out)), "mxfp8_dequantize")
+    return out
+
+
+def forward_bf16(x, ids, probs, w_gate, w_up, w_down, tokens=None, want_h=False):
+    """bf16 routed SwiGLU forward for `tokens` (default: all rows of ids).
+
+    x [T,H] bf16, ids/probs [T,k], w_gate/w_up [E,F,H] bf16, w_down [E,H,F] bf16.
+    Returns out fp32 [ntok, H] (and h fp32 [ntok, k, F] when want_h)."""
+    xb = _bf16_bits(x)
+    gb, ub, db = _bf16_bits(w_gate), _bf16_bits(w_up), _bf16_bits(w_down)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    probs = np.ascontiguousarray(probs, dtype=np.float32)
+    T, k = ids.shape
+    E, F, H = gb.shape
+    assert xb.shape[1] == H and db.shape == (E, H, F)
+    toks = np.arange(T, dtype=np.int64) if tokens is None else np.ascontiguousarray(tokens, dtype=np.int64)
+    out = np.empty((toks.size, H), np.float32)
+    h = np.empty((toks.size, k, F), np.float32) if want_h else None
+    _check(_load().oracle_forward_bf16(_ptr(xb), _ptr(ids), _ptr(probs), _ptr(gb), _ptr(ub), _ptr(db),
+                                       xb.shape[0], H, F, E, k, _ptr(toks), toks.size, _ptr(out), _ptr(h)),
+           "forward_bf16")
+    return (out, h) if want_h else out
+
+
+def quantize_weights_mxfp8(w_gate, w_up, w_down):
+    """Quantise the bf16 expert weights with the oracle's MXFP8 rule:
+    gate/up in blocks along H (their last axis), down in blocks along F."""
+    gq, gs = mxfp8_quantize_bf16(w_gate)
+    uq, us = mxfp8_quantize_bf16(w_up)
+    dq, ds = mxfp8_quantize_bf16(w_down)
+    return gq, gs, uq, us, dq, ds
+
+
+def forward_mxfp8(x, ids, probs, wq, tokens=None, want_h=False):
+    """MXFP8 routed SwiGLU forward; `wq` = quantize_weights_mxfp8(...) output.
+
+    Returns out fp32 [ntok, H] and, when want_h, (h codes [ntok,k,F],
+    h scales [ntok,k,F/32], h pre-quantisation fp32 [ntok,k,F])."""
+    xb = _bf16_bits(x)
+    gq, gs, uq, us, dq, ds = wq
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    probs = np.ascontiguousarray(probs, dtype=np.float32)
+    T, k = ids.shape
+    E, F, H = gq.shape
+    toks = np.arange(T, dtype=np.int64) if tokens is None else np.ascontiguousarray(tokens, dtype=np.int64)
+    out = np.empty((toks.size, H), np.float32)
+    hq = hs = hf = None
+    if want_h:
+        hq = np.empty((toks.size, k, F), np.uint8)
+        hs = np.empty((toks.size, k, F // 32), np.uint8)
+        hf = np.empty((toks.size, k, F), np.float32)
+    _check(_load().oracle_forward_mxfp8(_ptr(xb), _ptr(ids), _ptr(probs), _ptr(gq), _ptr(gs), _ptr(uq),
+                                        _ptr(us), _ptr(dq), _ptr(ds), xb.shape[0], H, F, E, k, _ptr(toks),
+                                        toks.size, _ptr(out), _ptr(hq), _ptr(hs), _ptr(hf)),
+           "forward_mxfp8")
+    return (out, (hq, hs, hf)) if want_h else out

@@ -1,0 +1,483 @@
+/*
+ * moe_oracle.c -- the CPU oracle for the routed-MoE SwiGLU expert forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: only the tests, the package's smoke check and the CPU
+ * baseline leg of the benchmark do.  It shares no source, header, table or
+ * helper with the CUDA library; it is written from the pages' description
+ * of what the method computes, one token at a time, in double precision
+ * wherever the pages do not fix a narrower type.
+ *
+ * What each function follows (page title, section):
+ *   oracle_route       -- "core.transformer.moe.training_matches_inference"
+ *                         API doc, `_route` (top-k probs and ids per token),
+ *                         and Megatron-LM PR #7830 "Mega backend for
+ *                         generation" (expert ids put in a canonical sorted
+ *                         order before the combine).  Softmax over the
+ *                         experts, top-k, the k probabilities renormalised to
+ *                         sum to one; ties go to the lower expert id.
+ *   oracle_permute     -- same API doc, `expert_value_pass` ("each row is one
+ *                         route, sorted by local expert"); rows stable by
+ *                         token inside an expert.
+ *   oracle_mxfp8_*     -- Megatron-LM PR #7830 (mxfp8_quantize_per_block_32)
+ *                         and cudnn-frontend PR #448 review of the MXFP8
+ *                         block contract (32-element blocks): E4M3 elements,
+ *                         one E8M0 power-of-two scale per 32 elements along
+ *                         K, the OCP MX rule scale = 2^(floor(log2 amax)-8),
+ *                         round-to-nearest-even, saturating to +-448.
+ *   oracle_forward_*   -- Megatron-LM PR #7798, "Background" (activation
+ *                         fused into FC1, probabilities applied after FC2)
+ *                         and "What is changed" (a token's routes summed as
+ *                         fp32 fused multiply-adds of probability and row,
+ *                         starting from zero, in the listed order); PR #8367
+ *                         "Problem" (the result is returned in fp32, no bf16
+ *                         downcast).  SwiGLU: h = silu(gate . x) * (up . x).
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   - probabilities are renormalised over the k chosen experts in every
+ *     configuration;
+ *   - the combine order is ascending expert id;
+ *   - the expert output row y stays fp32 (the FC2 accumulator) before the
+ *     combine, and the combine output is not rounded to bf16;
+ *   - the SwiGLU intermediate is computed in double, rounded to fp32, then to
+ *     bf16 (round-to-nearest-even) or re-quantised to MXFP8 exactly as the
+ *     kernel path does;
+ *   - an all-zero MXFP8 block gets scale byte 0 (2^-127); negative values
+ *     that round to zero keep their sign (code 0x80).
+ *
+ * Build: gcc -O2 -fopenmp -shared -fPIC (no -ffast-math: fmaf and the
+ * double sums must keep IEEE semantics).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_EINVAL 1
+#define ORACLE_ENOMEM 2
+
+/* ------------------------------------------------------------------ */
+/* Number formats                                                      */
+/* ------------------------------------------------------------------ */
+
+/* bf16 bit pattern -> float (exact: bf16 is the top half of an fp32). */
+static float bf16_bits_to_float(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* float -> bf16 with round-to-nearest-even on the 16 dropped bits.  The
+ * inputs here are finite; a NaN stays a quiet NaN. */
+static uint16_t float_to_bf16_bits_rne(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu)) {
+        return (uint16_t)((u >> 16) | 0x0040u);
+    }
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7fffu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/* E4M3 (OCP FP8, "fn" flavour: no infinities, S.1111.111 is NaN).
+ * Value of a code from the format definition: bias 7, subnormals when the
+ * exponent field is zero with step 2^-9. */
+static double e4m3_code_value(int code) {
+    int sign = (code >> 7) & 1;
+    int ef = (code >> 3) & 15;
+    int mf = code & 7;
+    double mag;
+    if (ef == 15 && mf == 7) return NAN;
+    if (ef == 0)
+        mag = ldexp((double)mf, -9);
+    else
+        mag = ldexp(1.0 + mf / 8.0, ef - 7);
+    return sign ? -mag : mag;
+}
+
+/* The 127 finite non-negative codes 0x00..0x7e have strictly increasing
+ * values, so the nearest grid point of a magnitude is found by bisection
+ * over this table. */
+static double g_e4m3_mag[127];
+static double g_e4m3_all[256];
+static double g_pow2[256]; /* g_pow2[b] = 2^(b-127), the E8M0 scale value */
+static int g_tables_ready = 0;
+
+static void build_tables(void) {
+    if (g_tables_ready) return;
+    for (int c = 0; c < 127; ++c) g_e4m3_mag[c] = e4m3_code_value(c);
+    for (int c = 0; c < 256; ++c) g_e4m3_all[c] = e4m3_code_value(c);
+    for (int b = 0; b < 256; ++b) g_pow2[b] = ldexp(1.0, b - 127);
+    g_tables_ready = 1;
+}
+
+/* Round a real value onto the E4M3 grid: nearest code, ties to the code
+ * with an even mantissa LSB, magnitudes beyond 448 saturate to 448, the
+ * sign is kept (so -tiny -> 0x80). */
+static uint8_t e4m3_encode_rne_sat(double v) {
+    int neg = signbit(v) ? 1 : 0;
+    double a = fabs(v);
+    int code;
+    if (a >= g_e4m3_mag[126]) {
+        code = 126; /* 448: saturate */
+    } else {
+        /* largest lo with mag[lo] <= a */
+        int lo = 0, hi = 126;
+        while (hi - lo > 1) {
+            int mid = (lo + hi) / 2;
+            if (g_e4m3_mag[mid] <= a) lo = mid; else hi = mid;
+        }
+        double dlo = a - g_e4m3_mag[lo];
+        double dhi = g_e4m3_mag[hi] - a;
+        if (dlo < dhi) code = lo;
+        else if (dhi < dlo) code = hi;
+        else code = (lo & 1) ? hi : lo; /* tie: even mantissa */
+    }
+    return (uint8_t)(code | (neg << 7));
+}
+
+/* OCP MX shared-scale exponent of one block from its largest magnitude:
+ * floor(log2(amax)) - emax(E4M3)=8, clamped to the E8M0 range; an all-zero
+ * block gets the smallest scale.  Returns the biased byte. */
+static uint8_t e8m0_block_scale(double amax) {
+    int s;
+    if (amax == 0.0) {
+        s = -127;
+    } else {
+        int ex;
+        (void)frexp(amax, &ex);      /* amax = m * 2^ex, m in [0.5, 1) */
+        s = (ex - 1) - 8;            /* floor(log2 amax) - 8 */
+        if (s < -127) s = -127;
+        if (s > 127) s = 127;
+    }
+    return (uint8_t)(s + 127);
+}
+
+/* Quantise n values (n <= 32, one block) into codes + one scale byte. */
+static void mxfp8_block(const double* v, int n, uint8_t* q, uint8_t* sbyte) {
+    double amax = 0.0;
+    for (int i = 0; i < n; ++i) {
+        double a = fabs(v[i]);
+        if (a > amax) amax = a;
+    }
+    uint8_t sb = e8m0_block_scale(amax);
+    double inv = ldexp(1.0, -((int)sb - 127)); /* exact power of two */
+    for (int i = 0; i < n; ++i) q[i] = e4m3_encode_rne_sat(v[i] * inv);
+    *sbyte = sb;
+}
+
+/* ------------------------------------------------------------------ */
+/* Public entry points (called through ctypes by the tests)           */
+/* ------------------------------------------------------------------ */
+
+int oracle_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+double oracle_e4m3_value(int code) { return e4m3_code_value(code & 255); }
+
+/* MXFP8 quantisation of a row-major fp32 matrix [rows, cols] (values are
+ * exact bf16 or fp32 numbers), blocks of 32 along each row.  cols must be a
+ * multiple of 32.  q: [rows, cols] codes; s: [rows, cols/32] E8M0 bytes. */
+int oracle_mxfp8_quantize(const float* in, int64_t rows, int64_t cols,
+                          uint8_t* q, uint8_t* s) {
+    if (!in || !q || !s || rows < 0 || cols <= 0 || (cols % 32) != 0) return ORACLE_EINVAL;
+    build_tables();
+    const int64_t nb = cols / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        double v[32];
+        for (int64_t b = 0; b < nb; ++b) {
+            for (int i = 0; i < 32; ++i) v[i] = (double)in[r * cols + b * 32 + i];
+            mxfp8_block(v, 32, q + r * cols + b * 32, s + r * nb + b);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Same, for a matrix given as bf16 bit patterns. */
+int oracle_mxfp8_quantize_bf16(const uint16_t* in, int64_t rows, int64_t cols,
+                               uint8_t* q, uint8_t* s) {
+    if (!in || !q || !s || rows < 0 || cols <= 0 || (cols % 32) != 0) return ORACLE_EINVAL;
+    build_tables();
+    const int64_t nb = cols / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        double v[32];
+        for (int64_t b = 0; b < nb; ++b) {
+            for (int i = 0; i < 32; ++i) v[i] = (double)bf16_bits_to_float(in[r * cols + b * 32 + i]);
+            mxfp8_block(v, 32, q + r * cols + b * 32, s + r * nb + b);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Dequantise: out[r,c] = value(q[r,c]) * 2^(s[r,c/32]-127), in fp32 (exact
+ * for every code/scale pair that a bf16 input can produce). */
+int oracle_mxfp8_dequantize(const uint8_t* q, const uint8_t* s, int64_t rows, int64_t cols,
+                            float* out) {
+    if (!q || !s || !out || rows < 0 || cols <= 0 || (cols % 32) != 0) return ORACLE_EINVAL;
+    build_tables();
+    const int64_t nb = cols / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            out[r * cols + c] = (float)(g_e4m3_all[q[r * cols + c]] * g_pow2[s[r * nb + c / 32]]);
+    return ORACLE_OK;
+}
+
+/* Router: per token, top-k of the E logits by value (ties: lower id first),
+ * probabilities = softmax over all E experts renormalised over the chosen k,
+ * which equals exp(l_j - m) / sum_{i in topk} exp(l_i - m); evaluated in
+ * double and rounded once to fp32.  Output ids ascending, probs matching. */
+int oracle_route(const float* logits, int64_t T, int E, int k,
+                 int32_t* ids, float* probs) {
+    if (!logits || !ids || !probs || T < 0 || E <= 0 || E > 1024 || k <= 0 || k > E) return ORACLE_EINVAL;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        const float* l = logits + t * E;
+        int chosen_id[1024];
+        char taken[1024];
+        memset(taken, 0, (size_t)E);
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || l[e] > l[best]) best = e; /* strict: lower id wins ties */
+            }
+            taken[best] = 1;
+            chosen_id[j] = best;
+        }
+        double m = (double)l[chosen_id[0]];
+        double w[1024];
+        double z = 0.0;
+        for (int j = 0; j < k; ++j) {
+            w[j] = exp((double)l[chosen_id[j]] - m);
+            z += w[j];
+        }
+        /* canonical order: ascending expert id (insertion sort on k items) */
+        for (int a = 1; a < k; ++a) {
+            int id = chosen_id[a];
+            double ww = w[a];
+            int b = a - 1;
+            while (b >= 0 && chosen_id[b] > id) {
+                chosen_id[b + 1] = chosen_id[b];
+                w[b + 1] = w[b];
+                --b;
+            }
+            chosen_id[b + 1] = id;
+            w[b + 1] = ww;
+        }
+        for (int j = 0; j < k; ++j) {
+            ids[t * k + j] = chosen_id[j];
+            probs[t * k + j] = (float)(w[j] / z);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Permute: counts per expert, exclusive prefix sum -> offsets[E+1]; route
+ * (t, j) with expert e goes to row offsets[e] + (number of earlier tokens
+ * routed to e).  perm[row] = t*k + j, inv[t*k + j] = row. */
+int oracle_permute(const int32_t* ids, int64_t T, int E, int k,
+                   int64_t* offsets, int32_t* perm, int32_t* inv) {
+    if (!ids || !offsets || !perm || !inv || T < 0 || E <= 0 || k <= 0) return ORACLE_EINVAL;
+    int64_t* seen = (int64_t*)calloc((size_t)E, sizeof(int64_t));
+    if (!seen) return ORACLE_ENOMEM;
+    for (int e = 0; e <= E; ++e) offsets[e] = 0;
+    for (int64_t i = 0; i < T * k; ++i) {
+        int e = ids[i];
+        if (e < 0 || e >= E) { free(seen); return ORACLE_EINVAL; }
+        offsets[e + 1] += 1;
+    }
+    for (int e = 0; e < E; ++e) offsets[e + 1] += offsets[e];
+    for (int64_t t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int e = ids[t * k + j];
+            int64_t row = offsets[e] + seen[e];
+            seen[e] += 1;
+            perm[row] = (int32_t)(t * k + j);
+            inv[t * k + j] = (int32_t)row;
+        }
+    }
+    free(seen);
+    return ORACLE_OK;
+}
+
+static double silu_d(double z) { return z / (1.0 + exp(-z)); }
+
+/* Canonical order of one token's routes: ascending expert id, carrying the
+ * probability with its id. */
+static void sort_routes(const int32_t* ids_in, const float* p_in, int k, int* ids, float* p) {
+    for (int j = 0; j < k; ++j) { ids[j] = ids_in[j]; p[j] = p_in[j]; }
+    for (int a = 1; a < k; ++a) {
+        int id = ids[a];
+        float pp = p[a];
+        int b = a - 1;
+        while (b >= 0 && ids[b] > id) { ids[b + 1] = ids[b]; p[b + 1] = p[b]; --b; }
+        ids[b + 1] = id;
+        p[b + 1] = pp;
+    }
+}
+
+/* bf16 forward for a list of tokens.
+ *   x      [T, H]    bf16 bits          w_gate, w_up [E, F, H] bf16 bits
+ *   ids    [T, k]    int32              w_down       [E, H, F] bf16 bits
+ *   probs  [T, k]    fp32
+ *   toks   [ntok]    token indices to evaluate
+ *   out    [ntok, H] fp32
+ *   h_out  [ntok, k, F] fp32 (nullable): the bf16-rounded SwiGLU row of each
+ *          route, in canonical (ascending id) order.
+ * Per route: g_f = sum_c Wg[e,f,c] x_c and u_f likewise (double);
+ * h_f = bf16(fp32(silu(g_f) * u_f)); y_c = fp32(sum_f Wd[e,c,f] h_f);
+ * out_c = fmaf(p_j, y_c, out_c) over j in ascending id, from 0.0f. */
+int oracle_forward_bf16(const uint16_t* x, const int32_t* ids, const float* probs,
+                        const uint16_t* w_gate, const uint16_t* w_up, const uint16_t* w_down,
+                        int64_t T, int H, int F, int E, int k,
+                        const int64_t* toks, int64_t ntok, float* out, float* h_out) {
+    if (!x || !ids || !probs || !w_gate || !w_up || !w_down || !toks || !out) return ORACLE_EINVAL;
+    if (H <= 0 || F <= 0 || E <= 0 || k <= 0 || k > 64 || ntok < 0) return ORACLE_EINVAL;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t i = 0; i < ntok; ++i) {
+        int64_t t = toks[i];
+        if (t < 0 || t >= T) { bad = 1; continue; }
+        double* xd = (double*)malloc(sizeof(double) * (size_t)H);
+        double* hd = (double*)malloc(sizeof(double) * (size_t)F);
+        float* acc = out + i * H;
+        int sid[64];
+        float sp[64];
+        if (!xd || !hd) { free(xd); free(hd); bad = 1; continue; }
+        for (int c = 0; c < H; ++c) xd[c] = (double)bf16_bits_to_float(x[t * H + c]);
+        for (int c = 0; c < H; ++c) acc[c] = 0.0f;
+        sort_routes(ids + t * k, probs + t * k, k, sid, sp);
+        for (int j = 0; j < k; ++j) {
+            int e = sid[j];
+            if (e < 0 || e >= E) { bad = 1; break; }
+            const uint16_t* wg = w_gate + (int64_t)e * F * H;
+            const uint16_t* wu = w_up + (int64_t)e * F * H;
+            const uint16_t* wd = w_down + (int64_t)e * H * F;
+            for (int f = 0; f < F; ++f) {
+                double g = 0.0, u = 0.0;
+                for (int c = 0; c < H; ++c) {
+                    g += (double)bf16_bits_to_float(wg[(int64_t)f * H + c]) * xd[c];
+                    u += (double)bf16_bits_to_float(wu[(int64_t)f * H + c]) * xd[c];
+                }
+                float hf = (float)(silu_d(g) * u);
+                float hb = bf16_bits_to_float(float_to_bf16_bits_rne(hf));
+                hd[f] = (double)hb;
+                if (h_out) h_out[(i * k + j) * F + f] = hb;
+            }
+            for (int c = 0; c < H; ++c) {
+                double y = 0.0;
+                for (int f = 0; f < F; ++f) y += (double)bf16_bits_to_float(wd[(int64_t)c * F + f]) * hd[f];
+                acc[c] = fmaf(sp[j], (float)y, acc[c]);
+            }
+        }
+        free(xd);
+        free(hd);
+    }
+    return bad ? ORACLE_EINVAL : ORACLE_OK;
+}
+
+/* MXFP8 forward for a list of tokens.  The weights arrive already quantised
+ * (codes + E8M0 bytes, as oracle_mxfp8_quantize_bf16 makes them from the
+ * bf16 weights):
+ *   wg_q, wu_q [E, F, H] codes, wg_s, wu_s [E, F, H/32]  (blocks along H)
+ *   wd_q       [E, H, F] codes, wd_s       [E, H, F/32]  (blocks along F)
+ * x rows are quantised here from their bf16 values (blocks along H).  The
+ * GEMMs use the dequantised operands exactly; h is formed as in the bf16
+ * path up to its fp32 value, then quantised (blocks of 32 along F) and the
+ * dequantised h enters the down GEMM.
+ *   h_q_out [ntok, k, F] codes and h_s_out [ntok, k, F/32] (nullable),
+ *   h_f32_out [ntok, k, F] pre-quantisation fp32 h (nullable). */
+int oracle_forward_mxfp8(const uint16_t* x, const int32_t* ids, const float* probs,
+                         const uint8_t* wg_q, const uint8_t* wg_s,
+                         const uint8_t* wu_q, const uint8_t* wu_s,
+                         const uint8_t* wd_q, const uint8_t* wd_s,
+                         int64_t T, int H, int F, int E, int k,
+                         const int64_t* toks, int64_t ntok, float* out,
+                         uint8_t* h_q_out, uint8_t* h_s_out, float* h_f32_out) {
+    if (!x || !ids || !probs || !wg_q || !wg_s || !wu_q || !wu_s || !wd_q || !wd_s || !toks || !out)
+        return ORACLE_EINVAL;
+    if (H <= 0 || F <= 0 || (H % 32) || (F % 32) || E <= 0 || k <= 0 || k > 64 || ntok < 0)
+        return ORACLE_EINVAL;
+    build_tables();
+    const int nbh = H / 32, nbf = F / 32;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t i = 0; i < ntok; ++i) {
+        int64_t t = toks[i];
+        if (t < 0 || t >= T) { bad = 1; continue; }
+        double* xv = (double*)malloc(sizeof(double) * (size_t)H);
+        double* xd = (double*)malloc(sizeof(double) * (size_t)H);
+        double* hv = (double*)malloc(sizeof(double) * (size_t)F);
+        double* hd = (double*)malloc(sizeof(double) * (size_t)F);
+        uint8_t* qb = (uint8_t*)malloc((size_t)(H > F ? H : F));
+        float* acc = out + i * H;
+        int sid[64];
+        float sp[64];
+        if (!xv || !xd || !hv || !hd || !qb) {
+            free(xv); free(xd); free(hv); free(hd); free(qb);
+            bad = 1;
+            continue;
+        }
+        /* x: bf16 -> MXFP8 along H -> dequantised values */
+        for (int c = 0; c < H; ++c) xv[c] = (double)bf16_bits_to_float(x[t * H + c]);
+        for (int b = 0; b < nbh; ++b) {
+            uint8_t sb;
+            mxfp8_block(xv + b * 32, 32, qb + b * 32, &sb);
+            for (int c = 0; c < 32; ++c) xd[b * 32 + c] = g_e4m3_all[qb[b * 32 + c]] * g_pow2[sb];
+        }
+        for (int c = 0; c < H; ++c) acc[c] = 0.0f;
+        sort_routes(ids + t * k, probs + t * k, k, sid, sp);
+        for (int j = 0; j < k; ++j) {
+            int e = sid[j];
+            if (e < 0 || e >= E) { bad = 1; break; }
+            const uint8_t* gq = wg_q + (int64_t)e * F * H;
+            const uint8_t* gs = wg_s + (int64_t)e * F * nbh;
+            const uint8_t* uq = wu_q + (int64_t)e * F * H;
+            const uint8_t* us = wu_s + (int64_t)e * F * nbh;
+            const uint8_t* dq = wd_q + (int64_t)e * H * F;
+            const uint8_t* ds = wd_s + (int64_t)e * H * nbf;
+            for (int f = 0; f < F; ++f) {
+                double g = 0.0, u = 0.0;
+                for (int c = 0; c < H; ++c) {
+                    double wgv = g_e4m3_all[gq[(int64_t)f * H + c]] * g_pow2[gs[(int64_t)f * nbh + c / 32]];
+                    double wuv = g_e4m3_all[uq[(int64_t)f * H + c]] * g_pow2[us[(int64_t)f * nbh + c / 32]];
+                    g += wgv * xd[c];
+                    u += wuv * xd[c];
+                }
+                float hf = (float)(silu_d(g) * u);
+                hv[f] = (double)hf;
+                if (h_f32_out) h_f32_out[(i * k + j) * F + f] = hf;
+            }
+            for (int b = 0; b < nbf; ++b) {
+                uint8_t sb;
+                mxfp8_block(hv + b * 32, 32, qb + b * 32, &sb);
+                for (int c = 0; c < 32; ++c) hd[b * 32 + c] = g_e4m3_all[qb[b * 32 + c]] * g_pow2[sb];
+                if (h_s_out) h_s_out[(i * k + j) * nbf + b] = sb;
+            }
+            if (h_q_out) memcpy(h_q_out + (i * k + j) * F, qb, (size_t)F);
+            for (int c = 0; c < H; ++c) {
+                double y = 0.0;
+                for (int f = 0; f < F; ++f)
+                    y += g_e4m3_all[dq[(int64_t)c * F + f]] * g_pow2[ds[(int64_t)c * nbf + f / 32]] * hd[f];
+                acc[c] = fmaf(sp[j], (float)y, acc[c]);
+            }
+        }
+        free(xv); free(xd); free(hv); free(hd); free(qb);
+    }
+    return bad ? ORACLE_EINVAL : ORACLE_OK;
+}

@@ -1,0 +1,407 @@
+"""Pins of the CPU oracle to things other than itself (no GPU needed).
+
+Which plausible mistake each pin catches:
+  route      brute-force ranking (wrong comparison, wrong tie rule, wrong
+             output order); k=1 gives p=1 exactly; k=E equals the library
+             softmax (dropped exp, wrong max shift); k=2 equals the logistic
+             closed form (wrong sign in the exponent).
+  permute    a stable library argsort of (expert, token) (wrong rank, not
+             stable, off-by-one offsets); bijection invariants.
+  mxfp8      the E4M3 code table equals torch's float8_e4m3fn decode; every
+             finite bf16 value in blocks of four different amax binades
+             equals an independent quantiser (numpy log2 scale + torch's RNE
+             cast with a clamp to +-448); closed forms: scale rule, grid
+             round-trips, ties to even, saturation, sign of zero.
+  forward    E=1, k=1, p=1 equals a dense SwiGLU MLP from torch float64
+             matmuls (transposed operand, swapped gate/up, wrong silu);
+             zero gate or zero up weights give exact zeros; doubling p
+             doubles the output exactly; the combine is the fp32 FMA chain
+             in ascending expert id (checked against exact rational
+             arithmetic); token order and duplication invariance;
+             MXFP8 E=1 dense check with the independent quantiser.
+"""
+from __future__ import annotations
+
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+import workloads
+
+# ---------------------------------------------------------------- helpers
+
+
+def f32_round_exact(q: Fraction) -> np.float32:
+    """Round an exact rational to the nearest float32 (ties to even)."""
+    approx = np.float32(float(q))
+    best = None
+    for cand in (np.nextafter(approx, np.float32(-np.inf)), approx, np.nextafter(approx, np.float32(np.inf))):
+        d = abs(Fraction(float(cand)) - q)
+        if best is None or d < best[0] or (d == best[0] and (int(np.float32(cand).view(np.uint32)) & 1) == 0):
+            best = (d, cand)
+    return np.float32(best[1])
+
+
+def fmaf_exact(a, b, c) -> np.float32:
+    return f32_round_exact(Fraction(float(a)) * Fraction(float(b)) + Fraction(float(c)))
+
+
+def indep_mxfp8(v: np.ndarray):
+    """Independent MXFP8 quantiser: numpy for the shared exponent, torch's
+    float8_e4m3fn cast (round-to-nearest-even) after a clamp to +-448.
+    v: float64 [rows, cols], cols % 32 == 0.  Returns codes, scale bytes."""
+    rows, cols = v.shape
+    blocks = v.reshape(rows, cols // 32, 32)
+    amax = np.abs(blocks).max(axis=2)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(amax > 0, amax, 1.0)))
+    s = np.where(amax > 0, np.clip(e - 8, -127, 127), -127).astype(np.int64)
+    scaled = blocks * np.exp2(-s.astype(np.float64))[:, :, None]
+    scaled32 = torch.from_numpy(np.clip(scaled, -448.0, 448.0).astype(np.float32))
+    codes = scaled32.to(torch.float8_e4m3fn).view(torch.uint8).numpy().reshape(rows, cols)
+    return codes, (s + 127).astype(np.uint8)
+
+
+def torch_e4m3_table() -> np.ndarray:
+    return torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def indep_dequant(codes: np.ndarray, sbytes: np.ndarray) -> np.ndarray:
+    tab = torch_e4m3_table()
+    rows, cols = codes.shape
+    return (tab[codes].reshape(rows, cols // 32, 32) * np.exp2(sbytes.astype(np.float64) - 127)[:, :, None]
+            ).reshape(rows, cols)
+
+
+def bf16_round(a64: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(a64.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def rand_bf16(gen, shape, std=1.0):
+    return (torch.randn(shape, generator=gen) * std).to(torch.bfloat16)
+
+
+# ---------------------------------------------------------------- route
+
+
+def _brute_topk(row: np.ndarray, k: int) -> np.ndarray:
+    order = np.lexsort((np.arange(row.size), -row.astype(np.float64)))
+    return np.sort(order[:k])
+
+
+def test_route_ids_match_brute_force_tiny():
+    w = workloads.WORKLOADS["tiny"]
+    _, logits = workloads.make_activations(w)
+    lg = logits.numpy()
+    ids, probs = oracle.route(lg, w.top_k)
+    for t in range(lg.shape[0]):
+        assert np.array_equal(ids[t], _brute_topk(lg[t], w.top_k))
+    assert np.all(np.diff(ids, axis=1) > 0)
+
+
+def test_route_ties_go_to_lower_id():
+    rng = np.random.default_rng(5)
+    lg = rng.integers(-3, 3, size=(200, 16)).astype(np.float32)  # many exact ties
+    for k in (1, 3, 8, 16):
+        ids, _ = oracle.route(lg, k)
+        for t in range(lg.shape[0]):
+            assert np.array_equal(ids[t], _brute_topk(lg[t], k))
+
+
+def test_route_k1_prob_is_one():
+    rng = np.random.default_rng(1)
+    lg = rng.standard_normal((300, 128)).astype(np.float32)
+    ids, probs = oracle.route(lg, 1)
+    assert np.all(probs == 1.0)
+    assert np.array_equal(ids[:, 0], np.argmax(lg, axis=1))
+
+
+def test_route_k_equals_e_is_softmax():
+    rng = np.random.default_rng(2)
+    lg = (rng.standard_normal((100, 8)) * 3).astype(np.float32)
+    ids, probs = oracle.route(lg, 8)
+    ref = scipy.special.softmax(lg.astype(np.float64), axis=1).astype(np.float32)
+    assert np.array_equal(ids, np.tile(np.arange(8), (100, 1)))
+    ulp = np.spacing(np.abs(ref))
+    assert np.all(np.abs(probs - ref) <= ulp)
+
+
+def test_route_k2_is_logistic():
+    rng = np.random.default_rng(3)
+    lg = rng.standard_normal((200, 32)).astype(np.float32)
+    ids, probs = oracle.route(lg, 2)
+    for t in range(200):
+        a, b = ids[t]
+        pa = scipy.special.expit(float(lg[t, a]) - float(lg[t, b]))
+        assert abs(probs[t, 0] - np.float32(pa)) <= np.spacing(np.float32(pa))
+        assert abs(probs[t, 1] - np.float32(1 - pa)) <= np.spacing(np.float32(1 - pa))
+
+
+def test_route_probs_sum_to_one():
+    rng = np.random.default_rng(4)
+    lg = rng.standard_normal((500, 128)).astype(np.float32)
+    _, probs = oracle.route(lg, 8)
+    assert np.all(np.abs(probs.astype(np.float64).sum(1) - 1.0) <= 8 * 2.0 ** -24)
+
+
+# ---------------------------------------------------------------- permute
+
+
+@pytest.mark.parametrize("T,E,k", [(64, 8, 2), (1000, 128, 8), (7, 4, 4), (1, 128, 6)])
+def test_permute_matches_stable_argsort(T, E, k):
+    rng = np.random.default_rng(T + E + k)
+    ids = np.stack([np.sort(rng.choice(E, size=k, replace=False)) for _ in range(T)]).astype(np.int32)
+    offsets, perm, inv = oracle.permute(ids, E)
+    flat_e = ids.reshape(-1).astype(np.int64)
+    tok = np.repeat(np.arange(T), k)
+    order = np.argsort(flat_e * T + tok, kind="stable")
+    assert np.array_equal(perm, order.astype(np.int32))
+    assert np.array_equal(offsets, np.concatenate([[0], np.cumsum(np.bincount(flat_e, minlength=E))]))
+    assert offsets[-1] == T * k
+    assert np.array_equal(np.sort(perm), np.arange(T * k))
+    assert np.array_equal(inv.reshape(-1)[perm], np.arange(T * k))
+
+
+def test_permute_empty_experts():
+    ids = np.array([[0, 3], [0, 3], [3, 5]], np.int32)
+    offsets, perm, inv = oracle.permute(ids, 8)
+    assert offsets.tolist() == [0, 2, 2, 2, 5, 5, 6, 6, 6]
+    assert perm.tolist() == [0, 2, 1, 3, 4, 5]
+
+
+# ---------------------------------------------------------------- mxfp8
+
+
+def test_e4m3_table_matches_torch_decode():
+    tab = torch_e4m3_table()
+    for c in range(256):
+        v = oracle.e4m3_value(c)
+        if math.isnan(tab[c]):
+            assert math.isnan(v), c
+        else:
+            assert v == tab[c], c
+    assert oracle.e4m3_value(0x7E) == 448.0
+    assert oracle.e4m3_value(0x01) == 2.0 ** -9
+
+
+def _all_finite_bf16() -> np.ndarray:
+    bits = np.arange(65536, dtype=np.uint32)
+    vals = (bits << 16).view(np.float32)
+    return vals[np.isfinite(vals)]
+
+
+@pytest.mark.parametrize("anchor", [0.0, 1.0, 2.0 ** 20, 2.0 ** -20, 3.0])
+def test_mxfp8_exhaustive_bf16_sweep(anchor):
+    vals = _all_finite_bf16().astype(np.float32)
+    blocks = np.zeros((vals.size, 32), np.float32)
+    blocks[:, 0] = vals
+    blocks[:, 1] = anchor
+    blocks[:, 7] = -vals * 0.5  # a second in-block value, exactly representable
+    q, s = oracle.mxfp8_quantize(blocks)
+    q2, s2 = indep_mxfp8(blocks.astype(np.float64))
+    assert np.array_equal(s[:, 0], s2[:, 0])
+    assert np.array_equal(q, q2)
+
+
+def test_mxfp8_closed_forms():
+    # scale = 2^(floor(log2 amax) - 8): amax 1.0 -> s=-8; amax 3.0 -> s=-7; amax 0.5 -> -9
+    for amax, s_exp in [(1.0, -8), (3.0, -7), (0.5, -9), (448.0, 0), (2.0 ** 100, 92), (1.5 * 2.0 ** -130, -127)]:
+        blk = np.zeros((1, 32), np.float32)
+        blk[0, 3] = amax
+        q, s = oracle.mxfp8_quantize(blk)
+        assert int(s[0, 0]) - 127 == s_exp, (amax, s)
+    # all-zero block -> byte 0, codes 0
+    q, s = oracle.mxfp8_quantize(np.zeros((1, 32), np.float32))
+    assert s[0, 0] == 0 and np.all(q == 0)
+    # grid values k * 2^s round-trip exactly
+    s_val = -4
+    grid = np.array([oracle.e4m3_value(c) for c in range(127)])
+    blk = np.zeros((4, 32), np.float32)
+    chosen = np.concatenate([[448.0], grid[[1, 2, 9, 40, 77, 100, 120]]])
+    for r in range(4):
+        blk[r, :8] = chosen * 2.0 ** s_val * (1 if r % 2 == 0 else -1)
+    q, s = oracle.mxfp8_quantize(blk)
+    deq = oracle.mxfp8_dequantize(q, s)
+    assert np.array_equal(deq, blk)
+    # a scaled value of 500 saturates to 448 when amax already fixes the scale (amax scaled = 500)
+    blk = np.zeros((1, 32), np.float32)
+    blk[0, 0] = 500.0
+    blk[0, 1] = -500.0
+    q, s = oracle.mxfp8_quantize(blk)
+    assert s[0, 0] == 127 and q[0, 0] == 0x7E and q[0, 1] == 0xFE
+    # midpoint between 1.0 (0x38) and 1.125 (0x39) -> even code 0x38; 1.1875 -> 0x3A (1.25 even)
+    blk = np.zeros((1, 32), np.float32)
+    blk[0, 0] = 256.0  # fixes s = 0
+    blk[0, 1] = 1.0625
+    blk[0, 2] = 1.1875
+    blk[0, 3] = -1e-30  # rounds to zero, keeps its sign
+    q, s = oracle.mxfp8_quantize(blk)
+    assert s[0, 0] == 127
+    assert q[0, 1] == 0x38 and q[0, 2] == 0x3A and q[0, 3] == 0x80
+
+
+def test_mxfp8_bf16_entry_matches_float_entry():
+    gen = torch.Generator().manual_seed(9)
+    x = rand_bf16(gen, (33, 256), 3.0)
+    q1, s1 = oracle.mxfp8_quantize_bf16(x)
+    q2, s2 = oracle.mxfp8_quantize(x.float().numpy())
+    assert np.array_equal(q1, q2) and np.array_equal(s1, s2)
+
+
+# ---------------------------------------------------------------- forward (bf16)
+
+
+def _dense_swiglu_ref(x, wg, wu, wd):
+    """torch float64 dense SwiGLU MLP with the intermediate rounded to fp32 then bf16."""
+    x64 = x.to(torch.float64)
+    g = x64 @ wg.to(torch.float64).T
+    u = x64 @ wu.to(torch.float64).T
+    h = (torch.nn.functional.silu(g) * u).to(torch.float32).to(torch.bfloat16).to(torch.float64)
+    return (h @ wd.to(torch.float64).T).to(torch.float32), h
+
+
+def test_forward_k1_single_expert_is_dense_mlp():
+    gen = torch.Generator().manual_seed(11)
+    T, H, F = 24, 96, 160  # H != F: a transposed operand cannot pass
+    x = rand_bf16(gen, (T, H))
+    wg = rand_bf16(gen, (1, F, H), H ** -0.5)
+    wu = rand_bf16(gen, (1, F, H), H ** -0.5)
+    wd = rand_bf16(gen, (1, H, F), F ** -0.5)
+    ids = np.zeros((T, 1), np.int32)
+    probs = np.ones((T, 1), np.float32)
+    out, h = oracle.forward_bf16(x, ids, probs, wg, wu, wd, want_h=True)
+    ref, href = _dense_swiglu_ref(x, wg[0], wu[0], wd[0])
+    # h may differ by a bf16 rounding flip where the double sums differ in the last bit
+    hflip = np.mean(h[:, 0, :] != href.numpy().astype(np.float32))
+    assert hflip < 1e-3
+    rms = float(np.sqrt(np.mean(ref.numpy().astype(np.float64) ** 2)))
+    assert np.max(np.abs(out - ref.numpy())) <= 1e-3 * rms
+    if hflip == 0:
+        assert np.max(np.abs(out - ref.numpy())) <= 1e-6 * rms
+
+
+def test_forward_zero_gate_or_up_gives_zero():
+    gen = torch.Generator().manual_seed(12)
+    T, H, F, E, k = 10, 64, 64, 4, 2
+    x = rand_bf16(gen, (T, H))
+    wg = rand_bf16(gen, (E, F, H), 0.1)
+    wu = rand_bf16(gen, (E, F, H), 0.1)
+    wd = rand_bf16(gen, (E, H, F), 0.1)
+    ids, probs = oracle.route(np.random.default_rng(0).standard_normal((T, E)).astype(np.float32), k)
+    out = oracle.forward_bf16(x, ids, probs, torch.zeros_like(wg), wu, wd)
+    assert np.all(out == 0.0)
+    out = oracle.forward_bf16(x, ids, probs, wg, torch.zeros_like(wu), wd)
+    assert np.all(out == 0.0)
+
+
+def _small_problem(seed, T=12, H=64, F=96, E=6, k=3):
+    gen = torch.Generator().manual_seed(seed)
+    x = rand_bf16(gen, (T, H))
+    wg = rand_bf16(gen, (E, F, H), H ** -0.5)
+    wu = rand_bf16(gen, (E, F, H), H ** -0.5)
+    wd = rand_bf16(gen, (E, H, F), F ** -0.5)
+    ids, probs = oracle.route(np.random.default_rng(seed).standard_normal((T, E)).astype(np.float32), k)
+    return x, wg, wu, wd, ids, probs
+
+
+def test_forward_doubling_probs_doubles_output():
+    x, wg, wu, wd, ids, probs = _small_problem(13)
+    a = oracle.forward_bf16(x, ids, probs, wg, wu, wd)
+    b = oracle.forward_bf16(x, ids, probs * 2, wg, wu, wd)
+    assert np.array_equal(b, a * 2)
+
+
+def test_forward_combine_is_ascending_fma_chain():
+    x, wg, wu, wd, ids, probs = _small_problem(14, T=5, k=3)
+    T, k = ids.shape
+    # per-route expert rows y_e(t) via k=1, p=1 calls
+    ys = {}
+    for j in range(k):
+        ys[j] = oracle.forward_bf16(x, ids[:, j:j + 1].copy(), np.ones((T, 1), np.float32), wg, wu, wd)
+    # hand the routes over in a scrambled order: the oracle must sort them
+    scr = ids[:, ::-1].copy()
+    pscr = probs[:, ::-1].copy()
+    out = oracle.forward_bf16(x, scr, pscr, wg, wu, wd)
+    for t in range(T):
+        for c in range(0, out.shape[1], 7):
+            acc = np.float32(0.0)
+            for j in range(k):  # ids are ascending along j
+                acc = fmaf_exact(probs[t, j], ys[j][t, c], acc)
+            assert out[t, c] == acc
+
+
+def test_forward_identical_experts_half_probs_is_identity():
+    x, wg, wu, wd, ids, probs = _small_problem(15, E=2, k=2)
+    wg = torch.stack([wg[0], wg[0]])
+    wu = torch.stack([wu[0], wu[0]])
+    wd = torch.stack([wd[0], wd[0]])
+    T = ids.shape[0]
+    ids = np.tile(np.array([[0, 1]], np.int32), (T, 1))
+    half = np.full((T, 2), 0.5, np.float32)
+    out = oracle.forward_bf16(x, ids, half, wg, wu, wd)
+    one = oracle.forward_bf16(x, ids[:, :1].copy(), np.ones((T, 1), np.float32), wg, wu, wd)
+    assert np.array_equal(out, one)
+
+
+def test_forward_token_order_and_duplication_invariance():
+    x, wg, wu, wd, ids, probs = _small_problem(16, T=9)
+    out = oracle.forward_bf16(x, ids, probs, wg, wu, wd)
+    p = np.random.default_rng(0).permutation(9)
+    out_p = oracle.forward_bf16(x[torch.from_numpy(p)], ids[p].copy(), probs[p].copy(), wg, wu, wd)
+    assert np.array_equal(out_p, out[p])
+    dup = np.concatenate([np.arange(9), np.arange(9)])
+    out_d = oracle.forward_bf16(x, ids, probs, wg, wu, wd, tokens=dup)
+    assert np.array_equal(out_d[:9], out_d[9:]) and np.array_equal(out_d[:9], out)
+
+
+# ---------------------------------------------------------------- forward (mxfp8)
+
+
+def test_forward_mxfp8_k1_single_expert_is_dense_mlp():
+    gen = torch.Generator().manual_seed(21)
+    T, H, F = 16, 128, 96
+    x = rand_bf16(gen, (T, H))
+    wg = rand_bf16(gen, (1, F, H), H ** -0.5)
+    wu = rand_bf16(gen, (1, F, H), H ** -0.5)
+    wd = rand_bf16(gen, (1, H, F), F ** -0.5)
+    wq = oracle.quantize_weights_mxfp8(wg, wu, wd)
+    ids = np.zeros((T, 1), np.int32)
+    probs = np.ones((T, 1), np.float32)
+    out, (hq, hs, hf) = oracle.forward_mxfp8(x, ids, probs, wq, want_h=True)
+    # independent pipeline: numpy scales + torch e4m3 cast
+    xq = indep_dequant(*indep_mxfp8(x.double().numpy()))
+    g_w = indep_dequant(*indep_mxfp8(wg[0].double().numpy()))
+    u_w = indep_dequant(*indep_mxfp8(wu[0].double().numpy()))
+    d_w = indep_dequant(*indep_mxfp8(wd[0].double().numpy()))
+    g = xq @ g_w.T
+    u = xq @ u_w.T
+    h32 = (scipy.special.expit(g) * g * u).astype(np.float32)
+    assert np.mean(h32 != hf[:, 0, :]) < 2e-2  # double-sum order may flip a last fp32 bit
+    hc, hsc = indep_mxfp8(hf[:, 0, :].astype(np.float64))  # quantiser consistency on the oracle's own h
+    assert np.array_equal(hc, hq[:, 0, :]) and np.array_equal(hsc, hs[:, 0, :])
+    ref = (indep_dequant(*indep_mxfp8(h32.astype(np.float64))) @ d_w.T).astype(np.float32)
+    rms = float(np.sqrt(np.mean(ref.astype(np.float64) ** 2)))
+    assert np.max(np.abs(out - ref)) <= 5e-2 * rms
+    assert np.mean(np.abs(out - ref)) <= 2e-3 * np.mean(np.abs(ref))
+
+
+def test_forward_mxfp8_zero_gate_gives_zero():
+    x, wg, wu, wd, ids, probs = _small_problem(22, H=64, F=64)
+    wq = oracle.quantize_weights_mxfp8(torch.zeros_like(wg), wu, wd)
+    out = oracle.forward_mxfp8(x, ids, probs, wq)
+    assert np.all(out == 0.0)
+
+
+def test_forward_mxfp8_close_to_bf16():
+    """MXFP8 and bf16 forwards of the same problem differ by a few percent
+    (the pages report ~4% relative distance for MXFP8 MoE layers)."""
+    x, wg, wu, wd, ids, probs = _small_problem(23, T=32, H=256, F=128, E=4, k=2)
+    a = oracle.forward_bf16(x, ids, probs, wg, wu, wd).astype(np.float64)
+    b = oracle.forward_mxfp8(x, ids, probs, oracle.quantize_weights_mxfp8(wg, wu, wd)).astype(np.float64)
+    d = np.linalg.norm(b - a) / np.linalg.norm(a)
+    assert 0.005 < d < 0.12
