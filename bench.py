@@ -1,0 +1,531 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-MoE SwiGLU forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole path (route, permute, gather, gate/up GEMM
++ SwiGLU, down GEMM, combine) over one batch of seeded synthetic inputs that
+are already resident in HBM.  The K timed steps are one captured CUDA graph
+(K forwards back to back, stage events inside), bracketed by a barrier and
+a device synchronise; the time is the max over ranks.  Every step re-reads
+all expert weights (1.6-3.8 GB), more than the 126 MB L2, so no L2 flush is
+needed between steps.
+
+Metric: routed tokens/s = live tokens processed per second (whole job).
+Extra keys: `roofline` for the dominant kernel (algorithmic bytes or FLOPs
+per launch / its CUDA-event duration, against MEASURED_PEAKS.json), `e2e`
+(same metric through the C ABI with pinned host buffers, copies inside the
+timed region), `cpu_baseline` (the CPU oracle on a bounded sample, rank 0,
+N=1), `clocks` (NVML samples during the timed region), `gpu_launches`.
+
+With --gpus N > 1 (launched by torch.distributed.run) every rank runs an
+independent replica of the workload on its own GPU (tokens are independent,
+so the path shards by token with no data-path collective): weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+KERNELS_PER_FORWARD = 8  # route, hist, scan, scatter, gather, gemm gate/up, gemm down, combine
+STAGES = ("route", "permute", "gather", "gemm_gate_up", "gemm_down", "combine")
+DEFAULT_STEPS = {"tiny": 200, "decode": 200, "prefill": 30, "mxfp8": 50, "sweep": 20}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=tuple(workloads.WORKLOADS), default="decode")
+    ap.add_argument("--live", type=int, default=None, help="live rows (default: the workload's largest)")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    a = ap.parse_args()
+    if a.steps is None:
+        a.steps = DEFAULT_STEPS[a.workload]
+    if a.warmup < 3:
+        a.warmup = 3
+    return a
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+
+class Dist:
+    def __init__(self, n_gpus):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+        elif torch.cuda.is_available():
+            torch.cuda.set_device(0)
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if self.pg is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Polls NVML (SM clock, max clock, clock-event reasons) on a thread."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as exc:  # no NVML: report that, keep going
+            self.err = str(exc)
+        self._stop = threading.Event()
+        self._t = None
+        self.window = (0.0, 0.0)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+            time.sleep(0.01)
+
+    def stop(self):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        t0, t1 = self.window
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside and self.samples:  # very short region: nearest samples
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:2]
+        mhz = [s[1] for s in inside]
+        bits = 0
+        for s in inside:
+            bits |= int(s[2])
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in self.REASONS.items() if bits & b], "samples": len(inside)}
+
+
+# ---------------------------------------------------------------- peaks / traffic
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+KERNEL_SOURCES = {
+    "gemm_gate_up": ["routed_moe_swiglu_b200/csrc/gemm_bf16.cu", "routed_moe_swiglu_b200/csrc/ptx.cuh",
+                     "routed_moe_swiglu_b200/csrc/moe_internal.cuh"],
+    "gemm_down": ["routed_moe_swiglu_b200/csrc/gemm_bf16.cu", "routed_moe_swiglu_b200/csrc/ptx.cuh",
+                  "routed_moe_swiglu_b200/csrc/moe_internal.cuh"],
+    "combine": ["routed_moe_swiglu_b200/csrc/permute.cu", "routed_moe_swiglu_b200/csrc/moe_internal.cuh"],
+}
+
+
+def source_hash(stage):
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES.get(stage, []):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(stage, workload):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's
+    sources are unchanged since it was taken (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    rec = d.get(f"{stage}@{workload}")
+    if not rec or rec.get("source_sha") != source_hash(stage):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- the CUDA arm
+
+
+def run_ours(a, dist: Dist):
+    import routed_moe_swiglu_b200 as rm
+
+    w = workloads.WORKLOADS[a.workload]
+    live = a.live or w.max_live
+    x, logits = workloads.make_activations(w)
+    wg, wu, wd = workloads.make_weights(w)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    plan = rm.moe_plan_create(hidden=w.hidden, ffn=w.ffn, num_experts=w.num_experts, top_k=w.top_k,
+                              capacity=w.capacity, precision=w.precision)
+    wbuf = rm.alloc_weight_buffer(plan, dev)
+    rm.moe_prepare_weights(plan, wg.to(dev), wu.to(dev), wd.to(dev), wbuf)
+    ws = rm.alloc_workspace(plan, dev)
+    xd, ld = x.to(dev), logits.to(dev)
+    out = torch.zeros((w.capacity, w.hidden), dtype=torch.float32, device=dev)
+    live_d = torch.tensor([live], dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+    K, W = a.steps, a.warmup
+    # one-step graph (warm-up, e2e) and a K-step graph with stage events (timed)
+    with torch.cuda.stream(stream):
+        rm.moe_forward(plan, xd, wbuf, live_d, out, ws, logits=ld)  # first call outside capture
+    stream.synchronize()
+    g1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1, stream=stream):
+        rm.moe_forward(plan, xd, wbuf, live_d, out, ws, logits=ld)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(K)]
+    gk = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gk, stream=stream):
+        for i in range(K):
+            rm.moe_forward_with_events(plan, xd, wbuf, live_d, out, ws, events[i], logits=ld)
+
+    with torch.cuda.stream(stream):
+        for _ in range(W):
+            g1.replay()
+    stream.synchronize()
+
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    h0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        gk.replay()
+        t_end.record(stream)
+    torch.cuda.synchronize()
+    h1 = time.perf_counter()
+    dist.barrier()
+    clocks.window = (h0, h1)
+    clocks.stop()
+    ms_total = dist.max(t_start.elapsed_time(t_end))
+    ms_step = ms_total / K
+
+    stage_ms = {s: [] for s in STAGES}
+    for ev in events:
+        for j, s in enumerate(STAGES):
+            stage_ms[s].append(ev[j].elapsed_time(ev[j + 1]))
+    stage_avg = {s: sum(v) / len(v) for s, v in stage_ms.items()}
+    status = rm.moe_get_device_status(ws)
+
+    # routing statistics of this batch, read from the library's own workspace
+    views = rm.moe_get_workspace_views(plan, ws)
+    off = views["offsets"] - views["base"]
+    offsets = ws[off:off + 4 * (w.num_experts + 1)].view(torch.int32).cpu()
+    counts = (offsets[1:] - offsets[:-1]).tolist()
+    touched = sum(1 for c in counts if c > 0)
+    routes = int(offsets[-1])
+
+    res = {
+        "ms_per_step": ms_step,
+        "value": dist.world * live / (ms_step / 1e3),
+        "stage_ms": stage_avg,
+        "clocks": clocks.summary(),
+        "timed_s": ms_total / 1e3,
+        "touched": touched,
+        "routes": routes,
+        "status": status,
+        "max_rows_per_expert": max(counts),
+    }
+
+    # ---------------- end to end through the C ABI with pinned host buffers
+    if not a.no_e2e:
+        x_pin = x[:live].contiguous().pin_memory()
+        l_pin = logits[:live].contiguous().pin_memory()
+        n_pin = torch.tensor([live], dtype=torch.int32).pin_memory()
+        o_pin = torch.empty((live, w.hidden), dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            xd[:live].copy_(x_pin, non_blocking=True)
+            ld[:live].copy_(l_pin, non_blocking=True)
+            live_d.copy_(n_pin, non_blocking=True)
+            g1.replay()
+            o_pin.copy_(out[:live], non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(W):
+                e2e_step()
+        stream.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(K):
+                e2e_step()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+        e_ms = dist.max(e0.elapsed_time(e1)) / K
+        res["e2e"] = {"value": dist.world * live / (e_ms / 1e3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": x_pin.numel() * 2 + l_pin.numel() * 4 + 4,
+                      "d2h_bytes_per_step": o_pin.numel() * 4, "ms_per_step": e_ms}
+    del gk, g1
+    return w, live, res
+
+
+def roofline(w, res, peaks):
+    """Roofline of the dominant kernel (largest share of the step)."""
+    st = res["stage_ms"]
+    dom = max(st, key=lambda s: st[s])
+    ms = st[dom]
+    H, F, k = w.hidden, w.ffn, w.top_k
+    R = res["routes"]
+    bpe = 1 if w.precision == "mxfp8" else 2
+    sustained = res["timed_s"] > 1.0
+    tflops_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    out = {"kernel": dom}
+    if dom in ("gemm_gate_up", "gemm_down"):
+        if dom == "gemm_gate_up":
+            flops = 4.0 * R * H * F
+            wbytes = res["touched"] * 2 * F * H * bpe
+            abytes = R * H * bpe + R * F * bpe
+        else:
+            flops = 2.0 * R * H * F
+            wbytes = res["touched"] * H * F * bpe
+            abytes = R * F * bpe + R * H * 4
+        bytes_ = wbytes + abytes
+        t_hbm = bytes_ / (peaks["hbm_gbs"] * 1e9)
+        t_tc = flops / (tflops_peak * 1e12 * (2.0 if w.precision == "mxfp8" else 1.0))
+        if t_hbm >= t_tc:
+            ach = bytes_ / (ms / 1e3) / 1e9
+            out.update(bound="hbm", achieved=ach, peak=peaks["hbm_gbs"], unit="GB/s",
+                       algorithmic_per_launch=bytes_)
+        else:
+            ach = flops / (ms / 1e3) / 1e12
+            pk = tflops_peak * (2.0 if w.precision == "mxfp8" else 1.0)
+            out.update(bound="tensor", achieved=ach, peak=pk, unit="TFLOP/s", algorithmic_per_launch=flops,
+                       peak_kind=("sustained" if sustained else "burst")
+                       + (" bf16 x2 (fp8 nominal ratio)" if w.precision == "mxfp8" else " bf16"))
+    else:
+        # memory-bound helper kernels: bytes they must move
+        if dom == "combine":
+            bytes_ = R * H * 4 + res["live"] * H * 4 + R * 8
+        elif dom == "gather":
+            bytes_ = res["live"] * H * 2 + R * H * bpe
+        else:
+            bytes_ = res["live"] * w.num_experts * 4
+        out.update(bound="hbm", achieved=bytes_ / (ms / 1e3) / 1e9, peak=peaks["hbm_gbs"], unit="GB/s",
+                   algorithmic_per_launch=bytes_)
+    out["frac"] = out["achieved"] / out["peak"]
+    out["peak_source"] = peaks["source"]
+    out["kernel_ms"] = ms
+    tr = recorded_traffic(dom, w.name)
+    out["traffic"] = tr
+    return out
+
+
+# ---------------------------------------------------------------- the oracle (CPU) arm
+
+
+def oracle_tokens_per_s(w, x, logits, weights, live, budget_s, min_tokens=8):
+    """Time the oracle (as it stands) on the host cores over a bounded sample
+    of the live tokens: route all live rows, then the expert forward of a
+    growing prefix of a seeded token sample until ~budget_s of work."""
+    import oracle
+
+    wq = oracle.quantize_weights_mxfp8(*weights) if w.precision == "mxfp8" else None
+    toks = workloads.sample_tokens(live, live, w.seed).numpy()
+    t0 = time.perf_counter()
+    ids, probs = oracle.route(logits[:live].numpy(), w.top_k)
+    route_s = time.perf_counter() - t0
+    done, spent, n = 0, 0.0, min_tokens
+    while spent < budget_s:
+        sel = toks[(done + __import__("numpy").arange(n)) % live]
+        t0 = time.perf_counter()
+        if w.precision == "mxfp8":
+            oracle.forward_mxfp8(x[:live], ids, probs, wq, tokens=sel)
+        else:
+            oracle.forward_bf16(x[:live], ids, probs, *weights, tokens=sel)
+        dt = time.perf_counter() - t0
+        spent += dt
+        done += n
+        per_tok = dt / n
+        n = max(1, min(4 * n, int((budget_s - spent) / max(per_tok, 1e-9)) + 1))
+    per_token = spent / done + route_s / live
+    return 1.0 / per_token, done, oracle.threads()
+
+
+def run_reference(a, dist: Dist):
+    """The oracle as the reference arm: K timed steps, each the oracle's
+    forward over a bounded token sample of the same workload."""
+    w = workloads.WORKLOADS[a.workload]
+    live = a.live or w.max_live
+    if dist.rank != 0:
+        return None
+    import numpy as np
+
+    import oracle
+
+    x, logits = workloads.make_activations(w)
+    weights = workloads.make_weights(w)
+    wq = oracle.quantize_weights_mxfp8(*weights) if w.precision == "mxfp8" else None
+    ids, probs = oracle.route(logits[:live].numpy(), w.top_k)
+    toks = workloads.sample_tokens(live, live, w.seed).numpy()
+
+    def step(n, start):
+        sel = toks[(start + np.arange(n)) % live]
+        if wq is not None:
+            oracle.forward_mxfp8(x[:live], ids, probs, wq, tokens=sel)
+        else:
+            oracle.forward_bf16(x[:live], ids, probs, *weights, tokens=sel)
+
+    t0 = time.perf_counter()
+    step(4, 0)
+    per_tok = (time.perf_counter() - t0) / 4
+    budget = 150.0  # whole run
+    n = max(1, int(budget / (a.steps + a.warmup) / max(per_tok, 1e-9)))
+    n = min(n, live)
+    for i in range(a.warmup):
+        step(n, i * n)
+    t0 = time.perf_counter()
+    for i in range(a.steps):
+        step(n, (a.warmup + i) * n)
+    el = time.perf_counter() - t0
+    value = n * a.steps / el
+    return w, live, {"value": value, "ms_per_step": el / a.steps * 1e3, "sample": n}
+
+
+# ---------------------------------------------------------------- main
+
+
+def workload_config(w, live):
+    return {
+        "workload": f"{w.name}: {w.precision} H={w.hidden} F={w.ffn} E={w.num_experts} top-{w.top_k}, "
+                    f"{live} live rows of a {w.capacity}-row buffer",
+        "hidden": w.hidden, "ffn": w.ffn, "experts": w.num_experts, "top_k": w.top_k,
+        "capacity": w.capacity, "live_rows": live, "seed": w.seed,
+        "l2": "no flush: every step re-reads all expert weights (> 126 MB L2)",
+        "graph": "one CUDA graph of K forwards; live count read on the device",
+    }
+
+
+def main():
+    a = parse_args()
+    dist = Dist(a.gpus)
+    if a.impl == "reference":
+        r = run_reference(a, dist)
+        if dist.rank == 0 and r is not None:
+            w, live, res = r
+            import oracle
+
+            line = {
+                "impl": "reference", "metric": "routed tokens/s", "value": res["value"], "unit": "tokens/s",
+                "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup, "ms_per_step": res["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": w.precision if w.precision != "mxfp8" else "mxfp8", "data": "synthetic",
+                "config": workload_config(w, live),
+                "cpu_baseline": {"value": res["value"], "unit": "tokens/s", "cores": oracle.threads(),
+                                 "kind": "oracle",
+                                 "sample": f"{res['sample']} tokens per step of the {w.name} workload"},
+                "e2e": {"value": res["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0},
+            }
+            print(json.dumps(line), flush=True)
+        dist.close()
+        return
+
+    w, live, res = run_ours(a, dist)
+    res["live"] = live
+    peaks = measured_peaks()
+    line = {
+        "metric": "routed tokens/s", "value": res["value"], "unit": "tokens/s", "n_gpus": dist.world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.precision, "data": "synthetic",
+        "config": workload_config(w, live),
+        "roofline": roofline(w, res, peaks),
+        "stage_ms": {k: round(v, 5) for k, v in res["stage_ms"].items()},
+        "clocks": res["clocks"],
+        "gpu_launches": KERNELS_PER_FORWARD * a.steps,
+        "device_status": res["status"],
+        "routing": {"routes": res["routes"], "experts_touched": res["touched"],
+                    "max_rows_per_expert": res["max_rows_per_expert"]},
+    }
+    if "e2e" in res:
+        line["e2e"] = res["e2e"]
+    if dist.rank == 0 and dist.world == 1 and not a.no_cpu_baseline:
+        x, logits = workloads.make_activations(w)
+        weights = workloads.make_weights(w)
+        v, n, cores = oracle_tokens_per_s(w, x, logits, weights, live, a.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": f"{n} tokens of the {w.name} workload (route of all {live} live rows "
+                                          f"+ expert forward of the sample), ~{a.cpu_seconds:.0f} s"}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+if __name__ == "__main__":
+    main()

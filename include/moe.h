@@ -163,6 +163,22 @@ moe_status moe_forward(const moe_plan* plan, const void* x, const float* logits,
                        const float* probs, const void* kernel_buf, const int* live_count_dev,
                        float* out, void* workspace, size_t ws_bytes, void* stream);
 
+/* Stages of moe_forward, in launch order: route (or canonicalise the
+ * caller's routes), permute (histogram, scan, scatter), gather of x rows
+ * (and their MXFP8 quantisation), gate/up GEMM with SwiGLU, down GEMM,
+ * combine. */
+#define MOE_NUM_STAGES 6
+
+/* moe_forward that also records stage_events[i] (cudaEvent_t passed as void*,
+ * MOE_NUM_STAGES + 1 of them, created by the caller with timing enabled) on
+ * `stream` before stage i, and stage_events[MOE_NUM_STAGES] after the last
+ * stage; for measuring each stage's device time.  Same results as
+ * moe_forward. */
+moe_status moe_forward_with_events(const moe_plan* plan, const void* x, const float* logits, const int* ids,
+                                   const float* probs, const void* kernel_buf, const int* live_count_dev,
+                                   float* out, void* workspace, size_t ws_bytes, void* stream,
+                                   void* const* stage_events);
+
 /* Views into a workspace after a forward (device pointers into it), for
  * tests and diagnostics:
  *   route_ids/route_probs [max_live, k]: canonical routes of the last forward
@@ -193,7 +209,8 @@ moe_status moe_get_workspace_views(const moe_plan* plan, const void* workspace,
 /* Copy the workspace's device status word to *flags_host.  Synchronises
  * `stream` (the only call that does). */
 moe_status moe_get_device_status(const void* workspace, unsigned* flags_host, void* stream);
-/* Zero the status word (enqueued on `stream`). */
+/* Zero the status word (enqueued on `stream`).  A newly allocated workspace
+ * holds an undefined status word: clear it once before the first read. */
 moe_status moe_clear_device_status(void* workspace, void* stream);
 
 /* Static string for a status code. */

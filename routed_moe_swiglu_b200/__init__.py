@@ -1,0 +1,257 @@
+"""routed_moe_swiglu_b200 -- B200 (sm_100a) routed-MoE SwiGLU expert forward.
+
+A thin ctypes binding over the C ABI of ``libroutedmoe.so`` (declared in
+``include/moe.h``).  Every function here only marshals arguments: torch
+tensors become device pointers, the current torch CUDA stream becomes the
+``stream`` argument.  All computation runs in the library's CUDA kernels;
+there is no CPU path, and calling any entry point without the built library
+raises.
+
+Typical use::
+
+    import routed_moe_swiglu_b200 as rm
+    plan = rm.moe_plan_create(hidden=2048, ffn=1024, num_experts=128, top_k=8,
+                              capacity=65536, precision="bf16")
+    wbuf = rm.alloc_weight_buffer(plan)
+    rm.moe_prepare_weights(plan, w_gate, w_up, w_down, wbuf)
+    ws = rm.alloc_workspace(plan)
+    rm.moe_forward(plan, x, wbuf, live_count, out, ws, logits=logits)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "MoeError", "Plan", "load_library", "library_path", "moe_version", "moe_plan_create", "moe_plan_destroy",
+    "moe_weight_buffer_bytes", "moe_workspace_bytes", "alloc_weight_buffer", "alloc_workspace",
+    "moe_prepare_weights", "mxfp8_quantize_block32", "moe_route_topk", "moe_forward", "moe_forward_with_events",
+    "MOE_NUM_STAGES", "STAGE_NAMES",
+    "moe_get_workspace_views", "moe_get_device_status", "moe_clear_device_status",
+    "MOE_DEV_LIVE_CLAMPED", "MOE_DEV_BAD_ROUTE", "MOE_DEV_TIMEOUT",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG, "libroutedmoe.so")
+
+MOE_OK = 0
+MOE_DEV_LIVE_CLAMPED = 0x1
+MOE_DEV_BAD_ROUTE = 0x2
+MOE_DEV_TIMEOUT = 0x4
+_PRECISION = {"bf16": 0, "mxfp8": 1}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {_status_string(code)} (status {code})")
+
+
+class _Desc(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("ffn", ctypes.c_int), ("num_experts", ctypes.c_int),
+                ("top_k", ctypes.c_int), ("capacity", ctypes.c_longlong), ("max_live_rows", ctypes.c_longlong),
+                ("precision", ctypes.c_int)]
+
+
+class _Views(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("route_ids", "route_probs", "offsets", "perm", "inv", "pad_offsets",
+                                                 "h", "h_scales", "xq", "xq_scales")] + [
+        ("rows_padded", ctypes.c_longlong), ("status", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load_library():
+    """Load libroutedmoe.so (built by ``python -m routed_moe_swiglu_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise RuntimeError(f"routed_moe_swiglu_b200: CUDA library not built ({library_path} missing); "
+                           "run `python -m routed_moe_swiglu_b200.build`")
+    lib = ctypes.CDLL(library_path)
+    P, I, LL, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t
+    sig = {
+        "moe_plan_create": ([ctypes.POINTER(_Desc), ctypes.POINTER(P)], I),
+        "moe_plan_destroy": ([P], None),
+        "moe_plan_get_desc": ([P, ctypes.POINTER(_Desc)], I),
+        "moe_weight_buffer_bytes": ([P], SZ),
+        "moe_workspace_bytes": ([P], SZ),
+        "moe_prepare_weights": ([P, P, P, P, P, SZ, P], I),
+        "mxfp8_quantize_block32": ([P, LL, I, LL, P, P, P, P], I),
+        "moe_route_topk": ([P, P, P, P, P, P], I),
+        "moe_forward": ([P, P, P, P, P, P, P, P, P, SZ, P], I),
+        "moe_forward_with_events": ([P, P, P, P, P, P, P, P, P, SZ, P, ctypes.POINTER(P)], I),
+        "moe_get_workspace_views": ([P, P, ctypes.POINTER(_Views)], I),
+        "moe_get_device_status": ([P, ctypes.POINTER(ctypes.c_uint), P], I),
+        "moe_clear_device_status": ([P, P], I),
+        "moe_status_string": ([I], ctypes.c_char_p),
+        "moe_version": ([], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def _status_string(code: int) -> str:
+    try:
+        return load_library().moe_status_string(code).decode()
+    except Exception:  # the library itself failed to load
+        return "unknown"
+
+
+def _check(code: int, what: str) -> None:
+    if code != MOE_OK:
+        raise MoeError(code, what)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("routed_moe_swiglu_b200 takes device tensors only")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def moe_version() -> str:
+    return load_library().moe_version().decode()
+
+
+class Plan:
+    """Owns a host-side moe_plan handle (immutable once created)."""
+
+    def __init__(self, handle, desc: _Desc):
+        self._h = handle
+        self.hidden = desc.hidden
+        self.ffn = desc.ffn
+        self.num_experts = desc.num_experts
+        self.top_k = desc.top_k
+        self.capacity = desc.capacity
+        self.max_live_rows = desc.max_live_rows
+        self.precision = {v: k for k, v in _PRECISION.items()}[desc.precision]
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if self._h is not None and _lib is not None:
+            _lib.moe_plan_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def moe_plan_create(hidden: int, ffn: int, num_experts: int, top_k: int, capacity: int,
+                    precision: str = "bf16", max_live_rows: int = 0) -> Plan:
+    lib = load_library()
+    d = _Desc(hidden, ffn, num_experts, top_k, capacity, max_live_rows, _PRECISION[precision])
+    h = ctypes.c_void_p()
+    _check(lib.moe_plan_create(ctypes.byref(d), ctypes.byref(h)), "moe_plan_create")
+    out = _Desc()
+    _check(lib.moe_plan_get_desc(h, ctypes.byref(out)), "moe_plan_get_desc")
+    return Plan(h, out)
+
+
+def moe_plan_destroy(plan: Plan) -> None:
+    plan.close()
+
+
+def moe_weight_buffer_bytes(plan: Plan) -> int:
+    return int(load_library().moe_weight_buffer_bytes(plan.handle))
+
+
+def moe_workspace_bytes(plan: Plan) -> int:
+    return int(load_library().moe_workspace_bytes(plan.handle))
+
+
+def alloc_weight_buffer(plan: Plan, device=None):
+    import torch
+
+    return torch.empty(moe_weight_buffer_bytes(plan), dtype=torch.uint8, device=device or "cuda")
+
+
+def alloc_workspace(plan: Plan, device=None):
+    """A workspace for one stream, with its device status word cleared."""
+    import torch
+
+    ws = torch.empty(moe_workspace_bytes(plan), dtype=torch.uint8, device=device or "cuda")
+    moe_clear_device_status(ws)
+    return ws
+
+
+def moe_prepare_weights(plan: Plan, w_gate, w_up, w_down, kernel_buf, stream=None) -> None:
+    _check(load_library().moe_prepare_weights(plan.handle, _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(kernel_buf),
+                                              kernel_buf.numel() * kernel_buf.element_size(), _stream(stream)),
+           "moe_prepare_weights")
+
+
+def mxfp8_quantize_block32(x, q, scales, live_rows=None, stream=None) -> None:
+    rows, cols = x.shape
+    _check(load_library().mxfp8_quantize_block32(_ptr(x), rows, cols, x.stride(0), _ptr(q), _ptr(scales),
+                                                 _ptr(live_rows), _stream(stream)), "mxfp8_quantize_block32")
+
+
+def moe_route_topk(plan: Plan, logits, live_count, ids, probs, stream=None) -> None:
+    _check(load_library().moe_route_topk(plan.handle, _ptr(logits), _ptr(live_count), _ptr(ids), _ptr(probs),
+                                         _stream(stream)), "moe_route_topk")
+
+
+def moe_forward(plan: Plan, x, kernel_buf, live_count, out, workspace, logits=None, ids=None, probs=None,
+                stream=None) -> None:
+    _check(load_library().moe_forward(plan.handle, _ptr(x), _ptr(logits), _ptr(ids), _ptr(probs), _ptr(kernel_buf),
+                                      _ptr(live_count), _ptr(out), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)), "moe_forward")
+
+
+MOE_NUM_STAGES = 6
+STAGE_NAMES = ("route", "permute", "gather", "gemm_gate_up", "gemm_down", "combine")
+
+
+def moe_forward_with_events(plan: Plan, x, kernel_buf, live_count, out, workspace, events, logits=None, ids=None,
+                            probs=None, stream=None) -> None:
+    """moe_forward recording torch.cuda.Event objects `events` (MOE_NUM_STAGES + 1,
+    enable_timing=True) around each stage."""
+    if len(events) != MOE_NUM_STAGES + 1:
+        raise ValueError("need MOE_NUM_STAGES + 1 events")
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(load_library().moe_forward_with_events(plan.handle, _ptr(x), _ptr(logits), _ptr(ids), _ptr(probs),
+                                                  _ptr(kernel_buf), _ptr(live_count), _ptr(out), _ptr(workspace),
+                                                  workspace.numel() * workspace.element_size(), _stream(stream),
+                                                  arr), "moe_forward_with_events")
+
+
+def moe_get_workspace_views(plan: Plan, workspace) -> dict:
+    v = _Views()
+    _check(load_library().moe_get_workspace_views(plan.handle, _ptr(workspace), ctypes.byref(v)),
+           "moe_get_workspace_views")
+    d = {n: getattr(v, n) for n, _ in _Views._fields_}
+    d["base"] = workspace.data_ptr()
+    return d
+
+
+def moe_get_device_status(workspace, stream=None) -> int:
+    flags = ctypes.c_uint(0)
+    _check(load_library().moe_get_device_status(_ptr(workspace), ctypes.byref(flags), _stream(stream)),
+           "moe_get_device_status")
+    return int(flags.value)
+
+
+def moe_clear_device_status(workspace, stream=None) -> None:
+    _check(load_library().moe_clear_device_status(_ptr(workspace), _stream(stream)), "moe_clear_device_status")

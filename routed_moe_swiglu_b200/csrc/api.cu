@@ -1,0 +1,391 @@
+// api.cu -- the C ABI declared in include/moe.h: plan validation, buffer
+// layouts, TMA descriptors and the launch sequence of the forward.
+#include <cudaTypedefs.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------- device info
+
+int num_sms() {
+    static int cached[64];
+    static bool have[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!have[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+        have[dev] = true;
+    }
+    return cached[dev];
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool get_tensor_map_encoder() {
+    if (g_encode != nullptr) return true;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return false;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return true;
+}
+
+bool make_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                     const unsigned long long* dims, const unsigned long long* strides_bytes, const unsigned* box,
+                     CUtensorMapSwizzle swizzle) {
+    if (!get_tensor_map_encoder()) return false;
+    cuuint64_t gdim[5];
+    cuuint64_t gstride[4];
+    cuuint32_t bdim[5];
+    cuuint32_t estride[5];
+    for (int i = 0; i < rank; ++i) {
+        gdim[i] = dims[i];
+        bdim[i] = box[i];
+        estride[i] = 1;
+        if (i + 1 < rank) gstride[i] = strides_bytes[i];
+    }
+    const CUresult r = g_encode(map, dtype, (cuuint32_t)rank, const_cast<void*>(base), gdim, gstride, bdim, estride,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static void compute_layouts(moe_plan* p) {
+    const size_t H = (size_t)p->d.hidden, F = (size_t)p->d.ffn, E = (size_t)p->d.num_experts;
+    const size_t k = (size_t)p->d.top_k;
+    const size_t L = (size_t)p->max_live;
+    const size_t R = (size_t)p->rows_pad;
+    const bool fp8 = p->d.precision == MOE_MXFP8;
+    WsLayout& w = p->ws;
+    size_t off = 0;
+    auto take = [&off](size_t bytes) {
+        const size_t at = off;
+        off += align256(bytes);
+        return at;
+    };
+    w.status = take(kStWords * 4);
+    w.r_ids = take(L * k * 4);
+    w.r_probs = take(L * k * 4);
+    w.blkcnt = take((size_t)p->nblk * E * 4);
+    w.offsets = take((E + 1) * 4);
+    w.padoff = take((E + 1) * 4);
+    w.tiles = take((size_t)p->max_m_tiles * 16);
+    w.perm = take(L * k * 4);
+    w.inv = take(L * k * 4);
+    if (fp8) {
+        w.xq = take(R * H);
+        w.xs = take(R * (H / 32));
+        w.h = take(R * F);
+        w.hs = take(R * (F / 32));
+    } else {
+        w.xq = take(R * H * 2);
+        w.xs = 0;
+        w.h = take(R * F * 2);
+        w.hs = 0;
+    }
+    w.y = take(R * H * 4);
+    w.total = off;
+
+    WbufLayout& b = p->wb;
+    off = 0;
+    if (fp8) {
+        b.w1 = take(E * 2 * F * H);
+        b.w1s = take(E * 2 * F * (H / 32));
+        b.w2 = take(E * H * F);
+        b.w2s = take(E * H * (F / 32));
+    } else {
+        b.w1 = take(E * 2 * F * H * 2);
+        b.w1s = 0;
+        b.w2 = take(E * H * F * 2);
+        b.w2s = 0;
+    }
+    b.total = off;
+}
+
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_version(void) { return "0.1.0"; }
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+        case MOE_ERR_ALIGNMENT: return "pointer or stride not aligned";
+        case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace or weight buffer too small";
+        case MOE_ERR_CUDA: return "CUDA runtime error";
+        case MOE_ERR_NOT_PREPARED: return "weight buffer not prepared";
+    }
+    return "unknown status";
+}
+
+moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
+    if (desc == nullptr || plan_out == nullptr) return MOE_ERR_INVALID_ARG;
+    *plan_out = nullptr;
+    const moe_desc& d = *desc;
+    if (d.precision != MOE_BF16 && d.precision != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
+    if (d.hidden <= 0 || d.ffn <= 0 || d.num_experts <= 0 || d.top_k <= 0 || d.capacity <= 0)
+        return MOE_ERR_UNSUPPORTED;
+    const int mult = d.precision == MOE_MXFP8 ? 32 : 8;
+    if (d.hidden % mult != 0 || d.ffn % mult != 0) return MOE_ERR_UNSUPPORTED;
+    if (d.hidden > 16384 || d.ffn > 16384) return MOE_ERR_UNSUPPORTED;
+    if (d.num_experts > kMaxExperts || d.top_k > kMaxTopK || d.top_k > d.num_experts) return MOE_ERR_UNSUPPORTED;
+    if (d.capacity > (1ll << 24)) return MOE_ERR_UNSUPPORTED;
+    if (d.max_live_rows < 0 || d.max_live_rows > d.capacity) return MOE_ERR_UNSUPPORTED;
+    if (d.precision == MOE_MXFP8) return MOE_ERR_UNSUPPORTED;  // enabled with the MXFP8 GEMMs
+    moe_plan* p = new (std::nothrow) moe_plan();
+    if (p == nullptr) return MOE_ERR_INVALID_ARG;
+    p->d = d;
+    p->max_live = d.max_live_rows > 0 ? d.max_live_rows : d.capacity;
+    p->d.max_live_rows = p->max_live;
+    p->max_routes = p->max_live * d.top_k;
+    p->max_m_tiles = (p->max_routes + kBM - 1) / kBM + d.num_experts;
+    p->rows_pad = p->max_m_tiles * kBM;
+    p->nblk = (int)((p->max_live + kTokPerBlk - 1) / kTokPerBlk);
+    compute_layouts(p);
+    *plan_out = p;
+    return MOE_OK;
+}
+
+void moe_plan_destroy(moe_plan* plan) { delete plan; }
+
+moe_status moe_plan_get_desc(const moe_plan* plan, moe_desc* desc_out) {
+    if (plan == nullptr || desc_out == nullptr) return MOE_ERR_INVALID_ARG;
+    *desc_out = plan->d;
+    return MOE_OK;
+}
+
+size_t moe_weight_buffer_bytes(const moe_plan* plan) { return plan ? plan->wb.total : 0; }
+size_t moe_workspace_bytes(const moe_plan* plan) { return plan ? plan->ws.total : 0; }
+
+moe_status moe_prepare_weights(const moe_plan* plan, const void* w_gate, const void* w_up, const void* w_down,
+                               void* kernel_buf, size_t buf_bytes, void* stream) {
+    if (plan == nullptr || w_gate == nullptr || w_up == nullptr || w_down == nullptr || kernel_buf == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (buf_bytes < plan->wb.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned(w_gate, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) || !aligned(kernel_buf, 256))
+        return MOE_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const auto* g = static_cast<const __nv_bfloat16*>(w_gate);
+    const auto* u = static_cast<const __nv_bfloat16*>(w_up);
+    const auto* dn = static_cast<const __nv_bfloat16*>(w_down);
+    const cudaError_t e = plan->d.precision == MOE_MXFP8 ? launch_prepare_mxfp8(plan, g, u, dn, kernel_buf, s)
+                                                          : launch_prepare_bf16(plan, g, u, dn, kernel_buf, s);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status mxfp8_quantize_block32(const void* in, long long rows, int cols, long long ld_in, uint8_t* q,
+                                  uint8_t* scales, const int* live_rows_dev, void* stream) {
+    if (in == nullptr || q == nullptr || scales == nullptr) return MOE_ERR_INVALID_ARG;
+    if (rows < 0 || cols <= 0 || ld_in < cols) return MOE_ERR_INVALID_ARG;
+    if (cols % 32 != 0) return MOE_ERR_UNSUPPORTED;
+    if (ld_in % 8 != 0 || !aligned(in, 16) || !aligned(q, 8)) return MOE_ERR_ALIGNMENT;
+    if (rows == 0) return MOE_OK;
+    const cudaError_t e = launch_quantize_rows(static_cast<const __nv_bfloat16*>(in), rows, cols, ld_in, q, scales,
+                                               live_rows_dev, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_route_topk(const moe_plan* plan, const float* logits, const int* live_count_dev, int* ids,
+                          float* probs, void* stream) {
+    if (plan == nullptr || logits == nullptr || live_count_dev == nullptr || ids == nullptr || probs == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    const cudaError_t e = launch_route_topk(logits, live_count_dev, (int)plan->max_live, plan->d.num_experts,
+                                            plan->d.top_k, ids, probs, nullptr, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // extern "C"
+
+namespace {
+
+static moe_status forward_impl(const moe_plan* plan, const void* x, const float* logits, const int* ids,
+                               const float* probs, const void* kernel_buf, const int* live_count_dev, float* out,
+                               void* workspace, size_t ws_bytes, void* stream, void* const* stage_events) {
+    if (plan == nullptr || x == nullptr || kernel_buf == nullptr || live_count_dev == nullptr || out == nullptr ||
+        workspace == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    const bool have_logits = logits != nullptr;
+    const bool have_routes = ids != nullptr && probs != nullptr;
+    if (have_logits == have_routes || ((ids == nullptr) != (probs == nullptr))) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < plan->ws.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned(x, 16) || !aligned(out, 16) || !aligned(workspace, 256) || !aligned(kernel_buf, 256))
+        return MOE_ERR_ALIGNMENT;
+    if (plan->d.precision != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto mark = [&](int i) -> bool {
+        return stage_events == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), s) == cudaSuccess;
+    };
+    const int H = plan->d.hidden, F = plan->d.ffn, E = plan->d.num_experts, k = plan->d.top_k;
+    const int max_live = (int)plan->max_live;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const uint8_t* wb = static_cast<const uint8_t*>(kernel_buf);
+    const WsLayout& L = plan->ws;
+    unsigned* status = reinterpret_cast<unsigned*>(ws + L.status);
+    int* r_ids = reinterpret_cast<int*>(ws + L.r_ids);
+    float* r_probs = reinterpret_cast<float*>(ws + L.r_probs);
+
+    // TMA descriptors for this call's buffers (host-side encoding only)
+    CUtensorMap tA1, tB1, tA2, tB2;
+    const unsigned long long R = (unsigned long long)plan->rows_pad;
+    {
+        const unsigned long long dA[2] = {(unsigned long long)H, R};
+        const unsigned long long sA[1] = {(unsigned long long)H * 2};
+        const unsigned bA[2] = {kBK, 32};
+        const unsigned long long dB[4] = {(unsigned long long)H, (unsigned long long)F, 2ull, (unsigned long long)E};
+        const unsigned long long sB[3] = {(unsigned long long)H * 2, (unsigned long long)F * H * 2,
+                                          2ull * F * H * 2};
+        const unsigned bB[4] = {kBK, (unsigned)kG1BN, 1, 1};
+        const unsigned long long dA2[2] = {(unsigned long long)F, R};
+        const unsigned long long sA2[1] = {(unsigned long long)F * 2};
+        const unsigned long long dB2[3] = {(unsigned long long)F, (unsigned long long)H, (unsigned long long)E};
+        const unsigned long long sB2[2] = {(unsigned long long)F * 2, (unsigned long long)H * F * 2};
+        const unsigned bB2[3] = {kBK, (unsigned)kG2BN, 1};
+        if (!make_tensor_map(&tA1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + L.xq, dA, sA, bA,
+                             CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tB1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, wb + plan->wb.w1, dB, sB, bB,
+                             CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tA2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + L.h, dA2, sA2, bA,
+                             CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tB2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, wb + plan->wb.w2, dB2, sB2, bB2,
+                             CU_TENSOR_MAP_SWIZZLE_128B))
+            return MOE_ERR_CUDA;
+    }
+
+    cudaError_t e;
+    if (!mark(0)) return MOE_ERR_CUDA;
+    if (have_logits)
+        e = launch_route_topk(logits, live_count_dev, max_live, E, k, r_ids, r_probs, status, s);
+    else
+        e = launch_canon_routes(ids, probs, live_count_dev, max_live, E, k, r_ids, r_probs, status, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+
+    if (!mark(1)) return MOE_ERR_CUDA;
+    int* perm = reinterpret_cast<int*>(ws + L.perm);
+    int* inv = reinterpret_cast<int*>(ws + L.inv);
+    int4* tiles = reinterpret_cast<int4*>(ws + L.tiles);
+    e = launch_permute(plan, live_count_dev, r_ids, reinterpret_cast<int*>(ws + L.blkcnt),
+                       reinterpret_cast<int*>(ws + L.offsets), reinterpret_cast<int*>(ws + L.padoff), tiles, perm, inv,
+                       status, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+
+    if (!mark(2)) return MOE_ERR_CUDA;
+    e = launch_gather_bf16(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, k, inv,
+                           reinterpret_cast<__nv_bfloat16*>(ws + L.xq), s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+
+    const long long m_tiles = plan->max_m_tiles;
+    GemmParams g1{};
+    g1.tiles = tiles;
+    g1.status_words = status;
+    g1.status_flags = status + kStFlags;
+    g1.out = ws + L.h;
+    g1.out_scales = nullptr;
+    g1.out_ld = F;
+    g1.out_cols = F;
+    g1.n_tiles = (F + kG1BN - 1) / kG1BN;
+    g1.k_blocks = (H + kBK - 1) / kBK;
+    g1.wait_limit_ns = kWaitLimitNs;
+    const int sms = num_sms();
+    long long grid1 = m_tiles * g1.n_tiles;
+    if (grid1 > sms) grid1 = sms;
+    if (!mark(3)) return MOE_ERR_CUDA;
+    e = launch_gemm1_bf16(tA1, tB1, g1, (int)grid1, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+
+    GemmParams g2 = g1;
+    g2.out = ws + L.y;
+    g2.out_ld = H;
+    g2.out_cols = H;
+    g2.n_tiles = (H + kG2BN - 1) / kG2BN;
+    g2.k_blocks = (F + kBK - 1) / kBK;
+    long long grid2 = m_tiles * g2.n_tiles;
+    if (grid2 > sms) grid2 = sms;
+    if (!mark(4)) return MOE_ERR_CUDA;
+    e = launch_gemm2_bf16(tA2, tB2, g2, (int)grid2, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (!mark(5)) return MOE_ERR_CUDA;
+
+    e = launch_combine(reinterpret_cast<const float*>(ws + L.y), inv, r_probs, live_count_dev, max_live, H, k, out, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    return mark(6) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_forward(const moe_plan* plan, const void* x, const float* logits, const int* ids, const float* probs,
+                       const void* kernel_buf, const int* live_count_dev, float* out, void* workspace,
+                       size_t ws_bytes, void* stream) {
+    return forward_impl(plan, x, logits, ids, probs, kernel_buf, live_count_dev, out, workspace, ws_bytes, stream,
+                        nullptr);
+}
+
+moe_status moe_forward_with_events(const moe_plan* plan, const void* x, const float* logits, const int* ids,
+                                   const float* probs, const void* kernel_buf, const int* live_count_dev, float* out,
+                                   void* workspace, size_t ws_bytes, void* stream, void* const* stage_events) {
+    if (stage_events == nullptr) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i <= MOE_NUM_STAGES; ++i)
+        if (stage_events[i] == nullptr) return MOE_ERR_INVALID_ARG;
+    return forward_impl(plan, x, logits, ids, probs, kernel_buf, live_count_dev, out, workspace, ws_bytes, stream,
+                        stage_events);
+}
+
+moe_status moe_get_workspace_views(const moe_plan* plan, const void* workspace, moe_workspace_views* v) {
+    if (plan == nullptr || workspace == nullptr || v == nullptr) return MOE_ERR_INVALID_ARG;
+    const uint8_t* ws = static_cast<const uint8_t*>(workspace);
+    const WsLayout& L = plan->ws;
+    std::memset(v, 0, sizeof(*v));
+    v->route_ids = reinterpret_cast<const int*>(ws + L.r_ids);
+    v->route_probs = reinterpret_cast<const float*>(ws + L.r_probs);
+    v->offsets = reinterpret_cast<const int*>(ws + L.offsets);
+    v->perm = reinterpret_cast<const int*>(ws + L.perm);
+    v->inv = reinterpret_cast<const int*>(ws + L.inv);
+    v->pad_offsets = reinterpret_cast<const int*>(ws + L.padoff);
+    v->h = ws + L.h;
+    v->h_scales = plan->d.precision == MOE_MXFP8 ? ws + L.hs : nullptr;
+    v->xq = ws + L.xq;
+    v->xq_scales = plan->d.precision == MOE_MXFP8 ? ws + L.xs : nullptr;
+    v->rows_padded = plan->rows_pad;
+    v->status = reinterpret_cast<const unsigned*>(ws + L.status);
+    return MOE_OK;
+}
+
+moe_status moe_get_device_status(const void* workspace, unsigned* flags_host, void* stream) {
+    if (workspace == nullptr || flags_host == nullptr) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(flags_host, workspace, sizeof(unsigned), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return cudaStreamSynchronize(s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_clear_device_status(void* workspace, void* stream) {
+    if (workspace == nullptr) return MOE_ERR_INVALID_ARG;
+    return cudaMemsetAsync(workspace, 0, sizeof(unsigned), static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,112 @@
+// moe_internal.cuh -- shared definitions of the routed-MoE library: tile
+// constants, the plan, the workspace / weight-buffer layouts and the
+// launchers each .cu file provides.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "moe.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- tiling
+constexpr int kBM = 128;           // permuted rows (routes) per M tile
+constexpr int kBK = 64;            // bf16 K elements per pipeline stage (128-byte rows)
+constexpr int kBK8 = 128;          // E4M3 K elements per pipeline stage (128-byte rows)
+constexpr int kG1BN = 128;         // f values per gate/up tile (128 gate + 128 up MMA columns)
+constexpr int kG2BN = 256;         // output columns per down tile
+constexpr int kTokPerBlk = 256;    // tokens per histogram / scatter block
+constexpr int kMaxTopK = 16;
+constexpr int kMaxExperts = 1024;
+
+// Status word layout (uint32 words at the start of the workspace).
+enum : int { kStFlags = 0, kStNumMTiles = 1, kStTotalRoutes = 2, kStWords = 64 };
+
+// Default bound of any on-device wait before the kernel gives up (ns).
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;
+
+struct WsLayout {
+    size_t status, r_ids, r_probs, blkcnt, offsets, padoff, tiles, perm, inv;
+    size_t xq, xs, h, hs, y;
+    size_t total;
+};
+
+struct WbufLayout {
+    size_t w1, w1s, w2, w2s;
+    size_t total;
+};
+
+}  // namespace moe
+
+struct moe_plan {
+    moe_desc d;
+    long long max_live;
+    long long max_routes;   // max_live * k
+    long long max_m_tiles;  // upper bound on M tiles: ceil(routes / BM) + E
+    long long rows_pad;     // max_m_tiles * BM: rows of the padded intermediates
+    int nblk;               // ceil(max_live / kTokPerBlk)
+    moe::WsLayout ws;
+    moe::WbufLayout wb;
+};
+
+namespace moe {
+
+struct GemmParams {
+    const int4* tiles;              // {expert, first padded row, valid rows, 0} per M tile
+    const unsigned* status_words;   // [kStNumMTiles] = number of M tiles
+    unsigned* status_flags;         // sticky MOE_DEV_* bits
+    void* out;                      // h (bf16 / E4M3) or y (fp32)
+    uint8_t* out_scales;            // E8M0 scales of h (MXFP8), else null
+    long long out_ld;               // row stride of out, elements
+    int out_cols;                   // valid output columns (F or H)
+    int n_tiles;                    // N tiles per M tile
+    int k_blocks;                   // pipeline stages per tile
+    unsigned long long wait_limit_ns;
+};
+
+// ---------------------------------------------------------------- launchers
+int num_sms();
+bool get_tensor_map_encoder();
+bool make_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                     const unsigned long long* dims, const unsigned long long* strides_bytes,
+                     const unsigned* box, CUtensorMapSwizzle swizzle);
+
+cudaError_t launch_route_topk(const float* logits, const int* live, int max_live, int E, int k, int* ids,
+                              float* probs, unsigned* status, cudaStream_t s);
+cudaError_t launch_canon_routes(const int* ids_in, const float* probs_in, const int* live, int max_live, int E,
+                                int k, int* ids_out, float* probs_out, unsigned* status, cudaStream_t s);
+cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* blkcnt, int* offsets,
+                           int* padoff, int4* tiles, int* perm, int* inv, unsigned* status_words,
+                           cudaStream_t s);
+cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_live, int H, int k,
+                               const int* inv, __nv_bfloat16* xp, cudaStream_t s);
+cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int k,
+                                const int* inv, uint8_t* xq, uint8_t* xs, long long rows_pad, cudaStream_t s);
+cudaError_t launch_combine(const float* y, const int* inv, const float* probs, const int* live, int max_live,
+                           int H, int k, float* out, cudaStream_t s);
+cudaError_t launch_gemm1_bf16(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& gp, int grid,
+                              cudaStream_t s);
+cudaError_t launch_gemm2_bf16(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& gp, int grid,
+                              cudaStream_t s);
+cudaError_t launch_gemm1_mxfp8(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sfa,
+                               const CUtensorMap& sfb, const GemmParams& gp, int grid, cudaStream_t s);
+cudaError_t launch_gemm2_mxfp8(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sfa,
+                               const CUtensorMap& sfb, const GemmParams& gp, int grid, cudaStream_t s);
+cudaError_t launch_prepare_bf16(const moe_plan* p, const __nv_bfloat16* wg, const __nv_bfloat16* wu,
+                                const __nv_bfloat16* wd, void* buf, cudaStream_t s);
+cudaError_t launch_prepare_mxfp8(const moe_plan* p, const __nv_bfloat16* wg, const __nv_bfloat16* wu,
+                                 const __nv_bfloat16* wd, void* buf, cudaStream_t s);
+cudaError_t launch_quantize_rows(const __nv_bfloat16* in, long long rows, int cols, long long ld_in, uint8_t* q,
+                                 uint8_t* scales, const int* live_rows, cudaStream_t s);
+
+__device__ __forceinline__ int clamp_live(const int* live, int max_live) {
+    int n = __ldg(live);
+    return n < 0 ? 0 : (n > max_live ? max_live : n);
+}
+
+}  // namespace moe

@@ -1,0 +1,176 @@
+// route.cu -- router top-k and canonical route order.
+//
+// Router: "core.transformer.moe.training_matches_inference" API doc, `_route`
+// ([tokens, topk] probabilities and expert ids); Megatron-LM PR #7830,
+// "1. Mega backend for generation" (a token's expert ids are put in a
+// canonical sorted order before the combine).  Per token: softmax over the
+// E experts, the k largest (ties to the lower id), probabilities
+// renormalised over the k, emitted in ascending expert id.
+#include <cfloat>
+#include <cmath>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+// One warp per token.  Logit `id` lives in lane id % 32, slot id / 32.
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits,
+                                                         const int* __restrict__ live, int max_live, int E,
+                                                         int k, int* __restrict__ ids,
+                                                         float* __restrict__ probs, unsigned* status) {
+    int n = __ldg(live);
+    if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0 && (n < 0 || n > max_live))
+        atomicOr(status, MOE_DEV_LIVE_CLAMPED);
+    n = n < 0 ? 0 : (n > max_live ? max_live : n);
+
+    const int lane = threadIdx.x & 31;
+    const int warps_per_block = blockDim.x >> 5;
+    const int nslots = (E + 31) >> 5;
+    for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < n; t += gridDim.x * warps_per_block) {
+        const float* row = logits + (size_t)t * E;
+        float v[32];
+        uint32_t taken = 0;
+#pragma unroll
+        for (int s = 0; s < 32; ++s) {
+            const int id = lane + 32 * s;
+            float x = -INFINITY;
+            if (s < nslots && id < E) {
+                x = __ldg(row + id);
+                if (x != x) x = -INFINITY;  // NaN never wins over a number
+            } else {
+                taken |= 1u << s;
+            }
+            v[s] = x;
+        }
+        float sel_v[kMaxTopK];
+        int sel_id[kMaxTopK];
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) {
+            if (j < k) {
+                float bv = 0.0f;
+                int bid = -1;
+#pragma unroll
+                for (int s = 0; s < 32; ++s) {
+                    // ids grow with s inside a lane: strict '>' keeps the lower id on ties
+                    if (s < nslots && !((taken >> s) & 1u) && (bid < 0 || v[s] > bv)) {
+                        bv = v[s];
+                        bid = lane + 32 * s;
+                    }
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                    const int oid = __shfl_xor_sync(0xffffffffu, bid, off);
+                    const bool better = oid >= 0 && (bid < 0 || ov > bv || (ov == bv && oid < bid));
+                    if (better) {
+                        bv = ov;
+                        bid = oid;
+                    }
+                }
+                if ((bid & 31) == lane) taken |= 1u << (bid >> 5);
+                sel_v[j] = bv;
+                sel_id[j] = bid;
+            }
+        }
+        if (lane == 0) {
+            // renormalised softmax over the chosen k: exp(l_j - max) / sum, in double
+            const double m = (double)sel_v[0];
+            double w[kMaxTopK];
+            double z = 0.0;
+#pragma unroll
+            for (int j = 0; j < kMaxTopK; ++j) {
+                if (j < k) {
+                    w[j] = exp((double)sel_v[j] - m);
+                    z += w[j];
+                }
+            }
+            // ascending expert id, probabilities travel with their ids
+            for (int a = 1; a < k; ++a) {
+                const int id = sel_id[a];
+                const double ww = w[a];
+                int b = a - 1;
+                while (b >= 0 && sel_id[b] > id) {
+                    sel_id[b + 1] = sel_id[b];
+                    w[b + 1] = w[b];
+                    --b;
+                }
+                sel_id[b + 1] = id;
+                w[b + 1] = ww;
+            }
+            for (int j = 0; j < k; ++j) {
+                ids[(size_t)t * k + j] = sel_id[j];
+                probs[(size_t)t * k + j] = (float)(w[j] / z);
+            }
+        }
+    }
+}
+
+// Caller-provided routes: sort each token's k (id, prob) pairs by id; a
+// token with an id outside [0, E) or a repeated id is dropped (ids -1, its
+// output row stays zero) and flagged.
+__global__ void __launch_bounds__(256) canon_routes_kernel(const int* __restrict__ ids_in,
+                                                           const float* __restrict__ probs_in,
+                                                           const int* __restrict__ live, int max_live, int E,
+                                                           int k, int* __restrict__ ids_out,
+                                                           float* __restrict__ probs_out, unsigned* status) {
+    int n = __ldg(live);
+    if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0 && (n < 0 || n > max_live))
+        atomicOr(status, MOE_DEV_LIVE_CLAMPED);
+    n = n < 0 ? 0 : (n > max_live ? max_live : n);
+    for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
+        int id[kMaxTopK];
+        float p[kMaxTopK];
+        bool bad = false;
+        for (int j = 0; j < k; ++j) {
+            id[j] = __ldg(ids_in + (size_t)t * k + j);
+            p[j] = __ldg(probs_in + (size_t)t * k + j);
+            if (id[j] < 0 || id[j] >= E) bad = true;
+        }
+        for (int a = 1; a < k; ++a) {
+            const int ia = id[a];
+            const float pa = p[a];
+            int b = a - 1;
+            while (b >= 0 && id[b] > ia) {
+                id[b + 1] = id[b];
+                p[b + 1] = p[b];
+                --b;
+            }
+            id[b + 1] = ia;
+            p[b + 1] = pa;
+        }
+        for (int j = 1; j < k; ++j)
+            if (id[j] == id[j - 1]) bad = true;
+        if (bad && status != nullptr) atomicOr(status, MOE_DEV_BAD_ROUTE);
+        for (int j = 0; j < k; ++j) {
+            ids_out[(size_t)t * k + j] = bad ? -1 : id[j];
+            probs_out[(size_t)t * k + j] = bad ? 0.0f : p[j];
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_route_topk(const float* logits, const int* live, int max_live, int E, int k, int* ids,
+                              float* probs, unsigned* status, cudaStream_t s) {
+    const int warps = 8;
+    long long blocks = ((long long)max_live + warps - 1) / warps;
+    const long long cap = (long long)num_sms() * 16;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    route_topk_kernel<<<(unsigned)blocks, warps * 32, 0, s>>>(logits, live, max_live, E, k, ids, probs, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_canon_routes(const int* ids_in, const float* probs_in, const int* live, int max_live, int E,
+                                int k, int* ids_out, float* probs_out, unsigned* status, cudaStream_t s) {
+    long long blocks = ((long long)max_live + 255) / 256;
+    const long long cap = (long long)num_sms() * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    canon_routes_kernel<<<(unsigned)blocks, 256, 0, s>>>(ids_in, probs_in, live, max_live, E, k, ids_out,
+                                                         probs_out, status);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

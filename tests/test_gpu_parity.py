@@ -1,0 +1,322 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bit-exact: routed expert ids, the permutation (offsets, perm), MXFP8 codes
+and scales.  Floating point: the tolerance of tests/moe_testlib.py.
+Each test fails (never skips) when the library is missing on a GPU machine."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import routed_moe_swiglu_b200 as rm
+import workloads
+from moe_testlib import GpuMoe, assert_close, oracle_forward, workload_problem
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    rm.load_library()  # raises when the CUDA library is missing
+    torch.cuda.init()
+
+
+# ---------------------------------------------------------------- route
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "sweep"])
+def test_route_ids_bit_exact(name):
+    w = workloads.WORKLOADS[name]
+    _, logits = workloads.make_activations(w)
+    live = w.max_live
+    plan = rm.moe_plan_create(hidden=w.hidden, ffn=w.ffn, num_experts=w.num_experts, top_k=w.top_k,
+                              capacity=w.capacity, max_live_rows=w.max_live)
+    lg = logits.cuda()
+    ids = torch.full((w.capacity, w.top_k), -7, dtype=torch.int32, device="cuda")
+    probs = torch.full((w.capacity, w.top_k), -7.0, dtype=torch.float32, device="cuda")
+    lv = torch.tensor([live], dtype=torch.int32, device="cuda")
+    rm.moe_route_topk(plan, lg, lv, ids, probs)
+    torch.cuda.synchronize()
+    ids_h, probs_h = ids.cpu().numpy(), probs.cpu().numpy()
+    ref_ids, ref_probs = oracle.route(logits[:live].numpy(), w.top_k)
+    assert np.array_equal(ids_h[:live], ref_ids)
+    ulp = np.spacing(np.abs(ref_probs))
+    assert np.all(np.abs(probs_h[:live] - ref_probs) <= ulp)
+    if live < w.capacity:  # rows past the live count untouched
+        assert np.all(ids_h[live:live + 64] == -7) and np.all(probs_h[live:live + 64] == -7.0)
+
+
+# ---------------------------------------------------------------- quantize
+
+
+@pytest.mark.parametrize("anchor", [0.0, 1.0, 2.0 ** 20, 2.0 ** -20, 3.0])
+def test_mxfp8_quantize_exhaustive_bf16(anchor):
+    bits = np.arange(65536, dtype=np.uint32)
+    vals = (bits << 16).view(np.float32)
+    vals = vals[np.isfinite(vals)]
+    blocks = np.zeros((vals.size, 32), np.float32)
+    blocks[:, 0] = vals
+    blocks[:, 1] = anchor
+    blocks[:, 7] = -vals * 0.5
+    x = torch.from_numpy(blocks).to(torch.bfloat16)  # exact: every entry is a bf16 value
+    assert np.array_equal(x.float().numpy(), blocks)
+    q = torch.empty((vals.size, 32), dtype=torch.uint8, device="cuda")
+    s = torch.empty((vals.size, 1), dtype=torch.uint8, device="cuda")
+    rm.mxfp8_quantize_block32(x.cuda(), q, s)
+    torch.cuda.synchronize()
+    rq, rs = oracle.mxfp8_quantize(blocks)
+    assert np.array_equal(s.cpu().numpy(), rs)
+    assert np.array_equal(q.cpu().numpy(), rq)
+
+
+def test_mxfp8_quantize_strided_and_live_bound():
+    gen = torch.Generator().manual_seed(3)
+    full = (torch.randn((300, 512), generator=gen) * torch.exp(torch.randn((300, 1), generator=gen) * 4))
+    full = full.to(torch.bfloat16)
+    x = full.cuda()[:, :384]  # row stride 512, 384 columns
+    q = torch.full((300, 384), 0xAB, dtype=torch.uint8, device="cuda")
+    s = torch.full((300, 12), 0xAB, dtype=torch.uint8, device="cuda")
+    live = torch.tensor([257], dtype=torch.int32, device="cuda")
+    rm.mxfp8_quantize_block32(x, q, s, live_rows=live)
+    torch.cuda.synchronize()
+    rq, rs = oracle.mxfp8_quantize_bf16(full[:, :384].contiguous())
+    assert np.array_equal(q.cpu().numpy()[:257], rq[:257])
+    assert np.array_equal(s.cpu().numpy()[:257], rs[:257])
+    assert np.all(q.cpu().numpy()[257:] == 0xAB) and np.all(s.cpu().numpy()[257:] == 0xAB)
+
+
+# ---------------------------------------------------------------- forward, bf16
+
+
+def _check_permutation(m: GpuMoe, ref_ids, E):
+    v = m.views()
+    live, k = ref_ids.shape
+    ids_gpu = m.read_i32(v["route_ids"], live * k).reshape(live, k)
+    assert np.array_equal(ids_gpu, ref_ids)
+    offsets, perm, inv = oracle.permute(ref_ids, E)
+    off_gpu = m.read_i32(v["offsets"], E + 1)
+    assert np.array_equal(off_gpu, offsets.astype(np.int32))
+    perm_gpu = m.read_i32(v["perm"], live * k)
+    assert np.array_equal(perm_gpu, perm)
+    # padded rows: every expert segment starts on a 128-row boundary, order kept
+    pad = m.read_i32(v["pad_offsets"], E + 1)
+    inv_gpu = m.read_i32(v["inv"], live * k).reshape(live, k)
+    e_of = ref_ids
+    rank = inv.astype(np.int64) - offsets[e_of]
+    assert np.array_equal(inv_gpu, (pad[e_of] + rank).astype(np.int32))
+    assert np.all(pad % 128 == 0)
+
+
+def test_forward_tiny_all_tokens():
+    w, x, logits, weights = workload_problem("tiny")
+    m = GpuMoe(w.hidden, w.ffn, w.num_experts, w.top_k, w.capacity, weights)
+    out = m.forward(x.cuda(), w.max_live, logits=logits.cuda())
+    torch.cuda.synchronize()
+    ref_ids, _, ref = oracle_forward(x, logits, weights, w.top_k, w.max_live)
+    assert_close(out.cpu().numpy(), ref, "bf16", "tiny")
+    _check_permutation(m, ref_ids, w.num_experts)
+    assert m.status() == 0
+
+
+@pytest.mark.parametrize("H,F,E,k,T,cap", [
+    (264, 200, 5, 3, 300, 320),     # K tail (264 = 4*64 + 8), N tail, ragged M tiles
+    (512, 384, 16, 4, 1000, 1000),  # several M tiles per expert
+    (128, 136, 1, 1, 130, 256),     # one expert: a dense SwiGLU MLP, 2 M tiles
+    (256, 512, 64, 8, 17, 64),      # more experts than routes: many empty experts
+])
+def test_forward_ragged_shapes(H, F, E, k, T, cap):
+    x, logits, weights = workloads.small_case(H, F, E, k, T, seed=H + F + E, capacity=cap)
+    m = GpuMoe(H, F, E, k, cap, weights)
+    out = m.forward(x.cuda(), T, logits=logits.cuda())
+    torch.cuda.synchronize()
+    ref_ids, _, ref = oracle_forward(x, logits, weights, k, T)
+    o = out.cpu().numpy()
+    assert_close(o[:T], ref, "bf16", f"ragged {H},{F},{E},{k},{T}")
+    assert np.all(np.isnan(o[T:]))  # rows past the live count never written
+    _check_permutation(m, ref_ids, E)
+
+
+@pytest.fixture(scope="module")
+def decode_problem():
+    w, x, logits, weights = workload_problem("decode")
+    m = GpuMoe(w.hidden, w.ffn, w.num_experts, w.top_k, w.capacity, weights)
+    return w, x, logits, weights, m
+
+
+def test_forward_decode_all_live_tokens(decode_problem):
+    w, x, logits, weights, m = decode_problem
+    live = w.max_live
+    out = m.forward(x.cuda(), live, logits=logits.cuda(), sentinel=-12345.0)
+    torch.cuda.synchronize()
+    ref_ids, _, ref = oracle_forward(x, logits, weights, w.top_k, live)
+    o = out.cpu().numpy()
+    assert_close(o[:live], ref, "bf16", "decode")
+    assert np.all(o[live:] == -12345.0)
+    _check_permutation(m, ref_ids, w.num_experts)
+    assert m.status() == 0
+
+
+def test_forward_prefill_subset_and_full_permutation():
+    w, x, logits, weights = workload_problem("prefill")
+    m = GpuMoe(w.hidden, w.ffn, w.num_experts, w.top_k, w.capacity, weights)
+    live = w.max_live
+    out = m.forward(x.cuda(), live, logits=logits.cuda())
+    torch.cuda.synchronize()
+    toks = workloads.sample_tokens(live, 512, w.seed).numpy()
+    ref_ids, _, ref = oracle_forward(x, logits, weights, w.top_k, live, tokens=toks)
+    assert_close(out.cpu().numpy()[toks], ref, "bf16", "prefill subset")
+    _check_permutation(m, ref_ids, w.num_experts)
+    counts = np.bincount(ref_ids.reshape(-1), minlength=w.num_experts)
+    assert counts.max() > 8 * np.median(counts)  # the Zipf bias really skews the loads
+
+
+# ---------------------------------------------------------------- invariance and edge cases
+
+
+def test_batch_invariance_across_live_counts_and_replays(decode_problem):
+    """A token's output is bitwise identical whatever the live count and on
+    every repeat (the live count is only read on the device)."""
+    w, x, logits, weights, m = decode_problem
+    xd, ld = x.cuda(), logits.cuda()
+    outs = {}
+    for live in (1, 7, 64, 200, 256):
+        outs[live] = m.forward(xd, live, logits=ld).cpu()
+    for live in (7, 64, 200, 256):
+        n = min(live, 1)
+        assert torch.equal(outs[live][:n], outs[1][:n])
+    for a, b in ((7, 64), (64, 200), (200, 256)):
+        assert torch.equal(outs[a][:a], outs[b][:a])
+    again = m.forward(xd, 256, logits=ld).cpu()
+    assert torch.equal(again[:256], outs[256][:256])
+
+
+def test_token_order_invariance():
+    H, F, E, k, T = 256, 256, 16, 4, 200
+    x, logits, weights = workloads.small_case(H, F, E, k, T, seed=77)
+    m = GpuMoe(H, F, E, k, T, weights)
+    base = m.forward(x.cuda(), T, logits=logits.cuda()).cpu()
+    p = torch.randperm(T, generator=torch.Generator().manual_seed(1))
+    perm_out = m.forward(x[p].contiguous().cuda(), T, logits=logits[p].contiguous().cuda()).cpu()
+    assert torch.equal(perm_out, base[p])
+
+
+def test_caller_routes_match_router_and_are_canonicalised():
+    H, F, E, k, T = 256, 256, 16, 4, 100
+    x, logits, weights = workloads.small_case(H, F, E, k, T, seed=5)
+    m = GpuMoe(H, F, E, k, T, weights)
+    a = m.forward(x.cuda(), T, logits=logits.cuda()).cpu()
+    ids, probs = oracle.route(logits.numpy(), k)
+    # hand them over reversed: the library must sort them back
+    ids_r = torch.from_numpy(ids[:, ::-1].copy()).cuda()
+    probs_r = torch.from_numpy(probs[:, ::-1].copy()).cuda()
+    b = m.forward(x.cuda(), T, ids=ids_r, probs=probs_r).cpu()
+    assert torch.equal(a, b)
+    assert m.status() == 0
+
+
+def test_bad_routes_are_flagged_and_zeroed():
+    H, F, E, k, T = 256, 256, 8, 2, 10
+    x, logits, weights = workloads.small_case(H, F, E, k, T, seed=6)
+    m = GpuMoe(H, F, E, k, T, weights)
+    ids, probs = oracle.route(logits.numpy(), k)
+    ids[3] = [4, 4]      # repeated expert
+    ids[5, 1] = E + 3    # out of range
+    m.clear_status()
+    out = m.forward(x.cuda(), T, ids=torch.from_numpy(ids).cuda(), probs=torch.from_numpy(probs).cuda()).cpu()
+    assert m.status() & rm.MOE_DEV_BAD_ROUTE
+    assert torch.all(out[3] == 0) and torch.all(out[5] == 0)
+    good = [t for t in range(T) if t not in (3, 5)]
+    ref = oracle.forward_bf16(x[good], ids[good], probs[good], *weights)
+    assert_close(out.numpy()[good], ref, "bf16", "good tokens next to bad ones")
+
+
+def test_live_count_out_of_range_is_clamped_and_flagged():
+    H, F, E, k, cap = 128, 128, 8, 2, 40
+    x, logits, weights = workloads.small_case(H, F, E, k, 32, seed=8, capacity=cap)
+    x[32:] = 0.5  # finite rows past 32 so that a clamp to 40 stays checkable
+    logits[32:] = torch.randn((cap - 32, E), generator=torch.Generator().manual_seed(9))
+    m = GpuMoe(H, F, E, k, cap, weights, max_live=36)
+    m.clear_status()
+    out = m.forward(x.cuda(), -5, logits=logits.cuda())
+    torch.cuda.synchronize()
+    assert m.status() & rm.MOE_DEV_LIVE_CLAMPED
+    assert torch.all(torch.isnan(out))  # clamped to zero rows: nothing written
+    m.clear_status()
+    assert m.status() == 0
+    out = m.forward(x.cuda(), 1000, logits=logits.cuda()).cpu()
+    assert m.status() & rm.MOE_DEV_LIVE_CLAMPED
+    assert not torch.isnan(out[:36]).any() and torch.isnan(out[36:]).all()
+    _, _, ref = oracle_forward(x, logits, weights, k, 36)
+    assert_close(out.numpy()[:36], ref, "bf16", "clamped")
+
+
+def test_zero_live_rows_writes_nothing():
+    H, F, E, k, cap = 128, 128, 8, 2, 64
+    x, logits, weights = workloads.small_case(H, F, E, k, 0, seed=10, capacity=cap)
+    m = GpuMoe(H, F, E, k, cap, weights)
+    out = m.forward(x.cuda(), 0, logits=logits.cuda(), sentinel=3.0)
+    torch.cuda.synchronize()
+    assert torch.all(out == 3.0)
+    assert m.status() == 0
+
+
+def test_refit_negative_control():
+    """A refit without moe_prepare_weights keeps serving the old weights; with
+    it, the result equals a freshly built plan on the new weights."""
+    H, F, E, k, T = 256, 256, 8, 2, 64
+    x, logits, weights = workloads.small_case(H, F, E, k, T, seed=11)
+    _, _, weights_b = workloads.small_case(H, F, E, k, T, seed=12)
+    m = GpuMoe(H, F, E, k, T, weights)
+    wg, wu, wd = (w.cuda() for w in weights)
+    rm.moe_prepare_weights(m.plan, wg, wu, wd, m.wbuf)
+    a = m.forward(x.cuda(), T, logits=logits.cuda()).cpu()
+    for dst, src in zip((wg, wu, wd), weights_b):  # in-place update of the sources only
+        dst.copy_(src.cuda())
+    stale = m.forward(x.cuda(), T, logits=logits.cuda()).cpu()
+    assert torch.equal(stale, a)
+    rm.moe_prepare_weights(m.plan, wg, wu, wd, m.wbuf)
+    refit = m.forward(x.cuda(), T, logits=logits.cuda()).cpu()
+    fresh = GpuMoe(H, F, E, k, T, weights_b).forward(x.cuda(), T, logits=logits.cuda()).cpu()
+    assert torch.equal(refit, fresh) and not torch.equal(refit, a)
+
+
+def test_graph_capture_replay_with_device_live_counts():
+    """One capture serves every live count: the sweep workload's shapes at a
+    reduced buffer, replayed with live counts written between replays."""
+    w = workloads.WORKLOADS["sweep"]
+    H, F, E, k = w.hidden, w.ffn, w.num_experts, w.top_k
+    cap = 8192
+    x, logits, weights = workloads.small_case(H, F, E, k, 1024, seed=4, capacity=cap)
+    m = GpuMoe(H, F, E, k, cap, weights, max_live=1024)
+    xd, ld = x.cuda(), logits.cuda()
+    out = torch.full((cap, H), float("nan"), device="cuda")
+    live = torch.zeros(1, dtype=torch.int32, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        live.fill_(16)
+        rm.moe_forward(m.plan, xd, m.wbuf, live, out, m.ws, logits=ld)  # warm-up outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        rm.moe_forward(m.plan, xd, m.wbuf, live, out, m.ws, logits=ld)
+    res = {}
+    for n in (1, 64, 1024, 64):
+        out.fill_(float("nan"))
+        live.fill_(n)
+        g.replay()
+        torch.cuda.synchronize()
+        o = out.cpu()
+        assert not torch.isnan(o[:n]).any() and torch.isnan(o[n:]).all()
+        if n in res:
+            assert torch.equal(o[:n], res[n])
+        res[n] = o[:n].clone()
+    assert torch.equal(res[64][:1], res[1]) and torch.equal(res[1024][:64], res[64])
+    toks = workloads.sample_tokens(1024, 48, 4).numpy()
+    _, _, ref = oracle_forward(x, logits, weights, k, 1024, tokens=toks)
+    assert_close(res[1024].numpy()[toks], ref, "bf16", "graph replay")
+    del g

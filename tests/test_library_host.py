@@ -1,0 +1,114 @@
+"""Host-side checks of the C-ABI library (no GPU needed): it loads, exports
+every entry point include/moe.h declares, and rejects bad arguments before
+launching anything."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import routed_moe_swiglu_b200 as rm
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    txt = open(os.path.join(ROOT, "include", "moe.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*([a-z][a-z0-9_]*)\s*\(", txt, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = rm.load_library()
+    names = _declared_functions()
+    assert len(names) >= 14, names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/moe.h but not exported"
+
+
+def test_version_and_status_strings():
+    assert rm.moe_version().count(".") == 2
+    lib = rm.load_library()
+    for code in range(7):
+        assert lib.moe_status_string(code).decode() not in ("", "unknown status")
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(hidden=2050), 2),                # not a multiple of 8
+    (dict(ffn=0), 2),
+    (dict(top_k=17), 2),                   # k > 16
+    (dict(num_experts=4, top_k=5), 2),     # k > E
+    (dict(num_experts=1025), 2),
+    (dict(capacity=0), 2),
+    (dict(max_live_rows=10 ** 9), 2),      # above capacity
+    (dict(hidden=2056, precision="mxfp8"), 2),  # MXFP8 needs multiples of 32
+])
+def test_plan_rejects_unsupported(kw, code):
+    args = dict(hidden=2048, ffn=1024, num_experts=128, top_k=8, capacity=1024, precision="bf16")
+    args.update(kw)
+    with pytest.raises(rm.MoeError) as ei:
+        rm.moe_plan_create(**args)
+    assert ei.value.code == code
+
+
+def test_plan_sizes():
+    p = rm.moe_plan_create(hidden=2048, ffn=1024, num_experts=128, top_k=8, capacity=65536, max_live_rows=256)
+    assert p.max_live_rows == 256
+    # weight buffer: gate+up+down bf16, each 256-byte aligned region
+    assert rm.moe_weight_buffer_bytes(p) >= 3 * 128 * 2048 * 1024 * 2
+    ws = rm.moe_workspace_bytes(p)
+    rows_pad = (256 * 8 // 128 + 128) * 128
+    assert ws >= rows_pad * (2048 * 2 + 1024 * 2 + 2048 * 4)
+    q = rm.moe_plan_create(hidden=2048, ffn=1024, num_experts=128, top_k=8, capacity=65536)
+    assert q.max_live_rows == 65536 and rm.moe_workspace_bytes(q) > ws
+
+
+def test_forward_rejects_bad_arguments_before_launch():
+    lib = rm.load_library()
+    p = rm.moe_plan_create(hidden=256, ffn=512, num_experts=8, top_k=2, capacity=64)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    ws = rm.moe_workspace_bytes(p)
+    null = None
+    # no routing input at all
+    assert lib.moe_forward(p.handle, fake, null, null, null, fake, fake, fake, fake, ws, null) == 1
+    # both logits and ids/probs
+    assert lib.moe_forward(p.handle, fake, fake, fake, fake, fake, fake, fake, fake, ws, null) == 1
+    # ids without probs
+    assert lib.moe_forward(p.handle, fake, null, fake, null, fake, fake, fake, fake, ws, null) == 1
+    # workspace too small
+    assert lib.moe_forward(p.handle, fake, fake, null, null, fake, fake, fake, fake, ws - 1, null) == 4
+    # misaligned x
+    bad = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.moe_forward(p.handle, bad, fake, null, null, fake, fake, fake, fake, ws, null) == 3
+    # null plan / null out
+    assert lib.moe_forward(None, fake, fake, null, null, fake, fake, fake, fake, ws, null) == 1
+    assert lib.moe_forward(p.handle, fake, fake, null, null, fake, fake, null, fake, ws, null) == 1
+
+
+def test_prepare_and_quantize_reject_bad_arguments():
+    lib = rm.load_library()
+    p = rm.moe_plan_create(hidden=256, ffn=512, num_experts=8, top_k=2, capacity=64)
+    fake = ctypes.c_void_p(1 << 20)
+    nb = rm.moe_weight_buffer_bytes(p)
+    assert lib.moe_prepare_weights(p.handle, fake, fake, fake, fake, nb - 1, None) == 4
+    assert lib.moe_prepare_weights(p.handle, None, fake, fake, fake, nb, None) == 1
+    assert lib.moe_prepare_weights(p.handle, fake, fake, fake, ctypes.c_void_p((1 << 20) + 16), nb, None) == 3
+    # cols not a multiple of 32
+    assert lib.mxfp8_quantize_block32(fake, 4, 48, 48, fake, fake, None, None) == 2
+    # ld_in < cols
+    assert lib.mxfp8_quantize_block32(fake, 4, 64, 32, fake, fake, None, None) == 1
+    # zero rows is a no-op success
+    assert lib.mxfp8_quantize_block32(fake, 0, 64, 64, fake, fake, None, None) == 0
+
+
+def test_product_path_does_not_touch_the_oracle():
+    """The package must not import, load or reference the oracle."""
+    pkg = os.path.join(ROOT, "routed_moe_swiglu_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "moe_oracle" not in txt and "from oracle" not in txt, f
