@@ -57,6 +57,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--capacity", type=int, default=None,
+                    help="override the buffer rows (profiling captures only; not a benchmark configuration)")
     a = ap.parse_args()
     if a.steps is None:
         a.steps = DEFAULT_STEPS[a.workload]
@@ -119,7 +121,13 @@ class ClockSampler:
 
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.h = None
+            try:  # map the CUDA device to NVML by PCI bus id (CUDA_VISIBLE_DEVICES may renumber)
+                pr = torch.cuda.get_device_properties(device_index)
+                bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
         except Exception as exc:  # no NVML: report that, keep going
@@ -219,7 +227,12 @@ def run_ours(a, dist: Dist):
     import routed_moe_swiglu_b200 as rm
 
     w = workloads.WORKLOADS[a.workload]
-    live = a.live or w.max_live
+    if a.capacity is not None:
+        import dataclasses
+
+        w = dataclasses.replace(w, capacity=a.capacity, live=tuple(min(v, a.capacity) for v in w.live),
+                                nan_past_live=True)
+    live = min(a.live or w.max_live, w.capacity)
     x, logits = workloads.make_activations(w)
     wg, wu, wd = workloads.make_weights(w)
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -243,6 +256,11 @@ def run_ours(a, dist: Dist):
     with torch.cuda.graph(g1, stream=stream):
         rm.moe_forward(plan, xd, wbuf, live_d, out, ws, logits=ld)
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(K)]
+    with torch.cuda.stream(stream):  # torch creates the CUDA event on its first record
+        for ev in events:
+            for e in ev:
+                e.record(stream)
+    stream.synchronize()
     gk = torch.cuda.CUDAGraph()
     with torch.cuda.graph(gk, stream=stream):
         for i in range(K):
@@ -394,6 +412,8 @@ def oracle_tokens_per_s(w, x, logits, weights, live, budget_s, min_tokens=8):
     """Time the oracle (as it stands) on the host cores over a bounded sample
     of the live tokens: route all live rows, then the expert forward of a
     growing prefix of a seeded token sample until ~budget_s of work."""
+    import numpy as np
+
     import oracle
 
     wq = oracle.quantize_weights_mxfp8(*weights) if w.precision == "mxfp8" else None
@@ -403,7 +423,7 @@ def oracle_tokens_per_s(w, x, logits, weights, live, budget_s, min_tokens=8):
     route_s = time.perf_counter() - t0
     done, spent, n = 0, 0.0, min_tokens
     while spent < budget_s:
-        sel = toks[(done + __import__("numpy").arange(n)) % live]
+        sel = toks[(done + np.arange(n)) % live]
         t0 = time.perf_counter()
         if w.precision == "mxfp8":
             oracle.forward_mxfp8(x[:live], ids, probs, wq, tokens=sel)

@@ -230,6 +230,8 @@ def moe_forward_with_events(plan: Plan, x, kernel_buf, live_count, out, workspac
     enable_timing=True) around each stage."""
     if len(events) != MOE_NUM_STAGES + 1:
         raise ValueError("need MOE_NUM_STAGES + 1 events")
+    if any(e.cuda_event == 0 for e in events):
+        raise ValueError("events must exist on the device (record each once before use)")
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _check(load_library().moe_forward_with_events(plan.handle, _ptr(x), _ptr(logits), _ptr(ids), _ptr(probs),
                                                   _ptr(kernel_buf), _ptr(live_count), _ptr(out), _ptr(workspace),

@@ -235,7 +235,10 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     auto mark = [&](int i) -> bool {
-        return stage_events == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), s) == cudaSuccess;
+        // "external" so that, under stream capture, the graph gets a real event-record node
+        return stage_events == nullptr ||
+               cudaEventRecordWithFlags(static_cast<cudaEvent_t>(stage_events[i]), s, cudaEventRecordExternal) ==
+                   cudaSuccess;
     };
     const int H = plan->d.hidden, F = plan->d.ffn, E = plan->d.num_experts, k = plan->d.top_k;
     const int max_live = (int)plan->max_live;

@@ -61,8 +61,8 @@ def test_mxfp8_quantize_exhaustive_bf16(anchor):
     blocks[:, 0] = vals
     blocks[:, 1] = anchor
     blocks[:, 7] = -vals * 0.5
-    x = torch.from_numpy(blocks).to(torch.bfloat16)  # exact: every entry is a bf16 value
-    assert np.array_equal(x.float().numpy(), blocks)
+    x = torch.from_numpy(blocks).to(torch.bfloat16)
+    blocks = x.float().numpy()  # the bf16 values both sides quantise
     q = torch.empty((vals.size, 32), dtype=torch.uint8, device="cuda")
     s = torch.empty((vals.size, 1), dtype=torch.uint8, device="cuda")
     rm.mxfp8_quantize_block32(x.cuda(), q, s)
