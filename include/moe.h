@@ -186,9 +186,14 @@ moe_status moe_forward_with_events(const moe_plan* plan, const void* x, const fl
  *   perm    int32 [routes]: permuted row r holds route t*k + j
  *   inv     int32 [max_live, k]: padded intermediate row of route (t, j)
  *   pad_offsets int32 [E+1]: first padded intermediate row of each expert
- *   h       intermediate rows (bf16 [rows_padded, F], or E4M3 codes)
- *   h_scales E8M0 scale bytes of h in the GEMM's scale layout (MXFP8) or NULL
- *   xq / xq_scales permuted quantised x rows (MXFP8) or NULL */
+ *   h       intermediate rows (bf16 [rows_padded, F], or E4M3 codes
+ *           [rows_padded, F] in MXFP8)
+ *   xq      permuted x rows (bf16 [rows_padded, H], or E4M3 codes)
+ *   h_scales, xq_scales  MXFP8 only (else NULL): E8M0 bytes in blocks of
+ *           512 bytes, one per (128-row tile, K stage of 128 elements),
+ *           block index tile * ceil(K/128) + stage; inside a block the byte
+ *           of (row r of the tile, 32-element group g of the stage) is at
+ *           (r % 32) * 16 + (r / 32) * 4 + g.  K = F for h, H for x. */
 typedef struct {
     const int* route_ids;
     const float* route_probs;

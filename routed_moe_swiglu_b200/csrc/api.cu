@@ -86,11 +86,12 @@ static void compute_layouts(moe_plan* p) {
     w.tiles = take((size_t)p->max_m_tiles * 16);
     w.perm = take(L * k * 4);
     w.inv = take(L * k * 4);
+    const size_t mtiles = (size_t)p->max_m_tiles;
     if (fp8) {
         w.xq = take(R * H);
-        w.xs = take(R * (H / 32));
+        w.xs = take(mtiles * p->ks1 * kSfBlock);
         w.h = take(R * F);
-        w.hs = take(R * (F / 32));
+        w.hs = take(mtiles * p->ks2 * kSfBlock);
     } else {
         w.xq = take(R * H * 2);
         w.xs = 0;
@@ -104,9 +105,9 @@ static void compute_layouts(moe_plan* p) {
     off = 0;
     if (fp8) {
         b.w1 = take(E * 2 * F * H);
-        b.w1s = take(E * 2 * F * (H / 32));
+        b.w1s = take(E * p->nt1 * p->ks1 * kSfBlock);
         b.w2 = take(E * H * F);
-        b.w2s = take(E * H * (F / 32));
+        b.w2s = take(E * p->nt2 * p->ks2 * kSfBlock);
     } else {
         b.w1 = take(E * 2 * F * H * 2);
         b.w1s = 0;
@@ -152,7 +153,6 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     if (d.num_experts > kMaxExperts || d.top_k > kMaxTopK || d.top_k > d.num_experts) return MOE_ERR_UNSUPPORTED;
     if (d.capacity > (1ll << 24)) return MOE_ERR_UNSUPPORTED;
     if (d.max_live_rows < 0 || d.max_live_rows > d.capacity) return MOE_ERR_UNSUPPORTED;
-    if (d.precision == MOE_MXFP8) return MOE_ERR_UNSUPPORTED;  // enabled with the MXFP8 GEMMs
     moe_plan* p = new (std::nothrow) moe_plan();
     if (p == nullptr) return MOE_ERR_INVALID_ARG;
     p->d = d;
@@ -162,6 +162,17 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     p->max_m_tiles = (p->max_routes + kBM - 1) / kBM + d.num_experts;
     p->rows_pad = p->max_m_tiles * kBM;
     p->nblk = (int)((p->max_live + kTokPerBlk - 1) / kTokPerBlk);
+    if (d.precision == MOE_MXFP8) {
+        p->ks1 = (d.hidden + kBK8 - 1) / kBK8;
+        p->ks2 = (d.ffn + kBK8 - 1) / kBK8;
+        p->nt1 = (d.ffn + kG1BN8 - 1) / kG1BN8;
+        p->nt2 = (d.hidden + kG2BN8 - 1) / kG2BN8;
+    } else {
+        p->ks1 = (d.hidden + kBK - 1) / kBK;
+        p->ks2 = (d.ffn + kBK - 1) / kBK;
+        p->nt1 = (d.ffn + kG1BN - 1) / kG1BN;
+        p->nt2 = (d.hidden + kG2BN - 1) / kG2BN;
+    }
     compute_layouts(p);
     *plan_out = p;
     return MOE_OK;
@@ -231,7 +242,6 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     if (ws_bytes < plan->ws.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     if (!aligned(x, 16) || !aligned(out, 16) || !aligned(workspace, 256) || !aligned(kernel_buf, 256))
         return MOE_ERR_ALIGNMENT;
-    if (plan->d.precision != MOE_BF16) return MOE_ERR_UNSUPPORTED;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     auto mark = [&](int i) -> bool {
@@ -250,28 +260,35 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     float* r_probs = reinterpret_cast<float*>(ws + L.r_probs);
 
     // TMA descriptors for this call's buffers (host-side encoding only)
-    CUtensorMap tA1, tB1, tA2, tB2;
+    const bool fp8 = plan->d.precision == MOE_MXFP8;
     const unsigned long long R = (unsigned long long)plan->rows_pad;
+    const unsigned long long uH = (unsigned long long)H, uF = (unsigned long long)F, uE = (unsigned long long)E;
+    const unsigned long long eb = fp8 ? 1ull : 2ull;  // bytes per operand element
+    const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const unsigned bk = fp8 ? (unsigned)kBK8 : (unsigned)kBK;  // 128-byte rows either way
+    const unsigned g1_rows = fp8 ? (unsigned)kG1BN8 : (unsigned)kG1BN;
+    const unsigned g2_rows = fp8 ? (unsigned)kG2BN8 : (unsigned)kG2BN;
+    CUtensorMap tA1, tB1, tA2, tB2, tY;
     {
-        const unsigned long long dA[2] = {(unsigned long long)H, R};
-        const unsigned long long sA[1] = {(unsigned long long)H * 2};
-        const unsigned bA[2] = {kBK, 32};
-        const unsigned long long dB[4] = {(unsigned long long)H, (unsigned long long)F, 2ull, (unsigned long long)E};
-        const unsigned long long sB[3] = {(unsigned long long)H * 2, (unsigned long long)F * H * 2,
-                                          2ull * F * H * 2};
-        const unsigned bB[4] = {kBK, (unsigned)kG1BN, 1, 1};
-        const unsigned long long dA2[2] = {(unsigned long long)F, R};
-        const unsigned long long sA2[1] = {(unsigned long long)F * 2};
-        const unsigned long long dB2[3] = {(unsigned long long)F, (unsigned long long)H, (unsigned long long)E};
-        const unsigned long long sB2[2] = {(unsigned long long)F * 2, (unsigned long long)H * F * 2};
-        const unsigned bB2[3] = {kBK, (unsigned)kG2BN, 1};
-        if (!make_tensor_map(&tA1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + L.xq, dA, sA, bA,
-                             CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tB1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, wb + plan->wb.w1, dB, sB, bB,
-                             CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tA2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + L.h, dA2, sA2, bA,
-                             CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tB2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, wb + plan->wb.w2, dB2, sB2, bB2,
+        const unsigned long long dA[2] = {uH, R};
+        const unsigned long long sA[1] = {uH * eb};
+        const unsigned bA[2] = {bk, 32};
+        const unsigned long long dB[4] = {uH, uF, 2ull, uE};
+        const unsigned long long sB[3] = {uH * eb, uF * uH * eb, 2ull * uF * uH * eb};
+        const unsigned bB[4] = {bk, g1_rows, 1, 1};
+        const unsigned long long dA2[2] = {uF, R};
+        const unsigned long long sA2[1] = {uF * eb};
+        const unsigned long long dB2[3] = {uF, uH, uE};
+        const unsigned long long sB2[2] = {uF * eb, uH * uF * eb};
+        const unsigned bB2[3] = {bk, g2_rows, 1};
+        const unsigned long long dY[2] = {uH, R};
+        const unsigned long long sY[1] = {uH * 4};
+        const unsigned bY[2] = {32, 32};
+        if (!make_tensor_map(&tA1, dt, 2, ws + L.xq, dA, sA, bA, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tB1, dt, 4, wb + plan->wb.w1, dB, sB, bB, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tA2, dt, 2, ws + L.h, dA2, sA2, bA, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tB2, dt, 3, wb + plan->wb.w2, dB2, sB2, bB2, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ws + L.y, dY, sY, bY,
                              CU_TENSOR_MAP_SWIZZLE_128B))
             return MOE_ERR_CUDA;
     }
@@ -294,8 +311,12 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 
     if (!mark(2)) return MOE_ERR_CUDA;
-    e = launch_gather_bf16(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, k, inv,
-                           reinterpret_cast<__nv_bfloat16*>(ws + L.xq), s);
+    if (fp8)
+        e = launch_gather_mxfp8(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, k, inv, ws + L.xq,
+                                ws + L.xs, s);
+    else
+        e = launch_gather_bf16(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, k, inv,
+                               reinterpret_cast<__nv_bfloat16*>(ws + L.xq), s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 
     const long long m_tiles = plan->max_m_tiles;
@@ -307,26 +328,33 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g1.out_scales = nullptr;
     g1.out_ld = F;
     g1.out_cols = F;
-    g1.n_tiles = (F + kG1BN - 1) / kG1BN;
-    g1.k_blocks = (H + kBK - 1) / kBK;
+    g1.n_tiles = plan->nt1;
+    g1.k_blocks = plan->ks1;
     g1.wait_limit_ns = kWaitLimitNs;
+    g1.sfa = ws + L.xs;
+    g1.sfb = wb + plan->wb.w1s;
+    g1.out_scales = fp8 ? ws + L.hs : nullptr;
+    g1.sf_ks_out = plan->ks2;
     const int sms = num_sms();
     long long grid1 = m_tiles * g1.n_tiles;
     if (grid1 > sms) grid1 = sms;
     if (!mark(3)) return MOE_ERR_CUDA;
-    e = launch_gemm1_bf16(tA1, tB1, g1, (int)grid1, s);
+    e = fp8 ? launch_gemm1_mxfp8(tA1, tB1, tY, g1, (int)grid1, s) : launch_gemm1_bf16(tA1, tB1, tY, g1, (int)grid1, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 
     GemmParams g2 = g1;
     g2.out = ws + L.y;
     g2.out_ld = H;
     g2.out_cols = H;
-    g2.n_tiles = (H + kG2BN - 1) / kG2BN;
-    g2.k_blocks = (F + kBK - 1) / kBK;
+    g2.n_tiles = plan->nt2;
+    g2.k_blocks = plan->ks2;
+    g2.sfa = ws + L.hs;
+    g2.sfb = wb + plan->wb.w2s;
+    g2.out_scales = nullptr;
     long long grid2 = m_tiles * g2.n_tiles;
     if (grid2 > sms) grid2 = sms;
     if (!mark(4)) return MOE_ERR_CUDA;
-    e = launch_gemm2_bf16(tA2, tB2, g2, (int)grid2, s);
+    e = fp8 ? launch_gemm2_mxfp8(tA2, tB2, tY, g2, (int)grid2, s) : launch_gemm2_bf16(tA2, tB2, tY, g2, (int)grid2, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     if (!mark(5)) return MOE_ERR_CUDA;
 

@@ -37,7 +37,9 @@ constexpr uint32_t kABoxBytes = kABoxRows * kBK * 2;    // 4 KB
 constexpr uint32_t kBBytes = 256 * kBK * 2;             // 32 KB per stage
 constexpr uint32_t kAccCols = 256;                      // fp32 columns per accumulator buffer
 constexpr uint32_t kTmemCols = 512;
-constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + kStages * (kABytes + kBBytes) + 256 /*barriers*/;
+constexpr uint32_t kStageOutBytes = 32 * 128;           // one 32-row x 128-byte output box
+constexpr uint32_t kOutBytes = 4 * 2 * kStageOutBytes;  // 4 epilogue warps x 2 buffers
+constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + kStages * (kABytes + kBBytes) + kOutBytes + 256 /*barriers*/;
 
 struct __align__(8) Barriers {
     uint64_t full[kStages];
@@ -61,14 +63,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 template <int kMode>  // 0: gate/up + SwiGLU -> bf16 h;  1: down -> fp32 y
-__global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             const GemmParams p) {
+__device__ __forceinline__ void grouped_gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                                  const CUtensorMap& tmOut, const GemmParams& p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStages * kABytes;
-    Barriers* bars = reinterpret_cast<Barriers*>(sB + kStages * kBBytes);
+    uint8_t* sOut = sB + kStages * kBBytes;  // 1024-aligned
+    Barriers* bars = reinterpret_cast<Barriers*>(sOut + kOutBytes);
     volatile int* abort_flag = &bars->abort_flag;
 
     const int warp = threadIdx.x >> 5;
@@ -205,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp & 3;
         const int r = quad * 32 + lane;  // row inside the tile
         int it = 0;
+        uint32_t out_chunk = 0;  // output boxes this warp has staged (mode 1)
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
             const int buf = it & 1;
             const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
@@ -251,22 +254,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             } else {
-                float* out_row = reinterpret_cast<float*>(p.out) + (size_t)(ti.y + r) * (size_t)p.out_ld;
+                // fp32 rows leave through shared memory: each warp stages its 32 rows x 32
+                // columns in the 128-byte-swizzled box layout and one lane issues a TMA
+                // store.  Only warps whose 32-row slice holds valid rows store; rows past
+                // the expert's count inside a slice land in its own padding rows.
+                const bool slice_live = quad * 32 < ti.z;
+                uint8_t* my_out = sOut + (size_t)quad * 2 * kStageOutBytes;
 #pragma unroll 1
                 for (int c = 0; c < kG2BN / 32; ++c) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(taddr + c * 32, v);
                     tmem_ld_wait();
                     const int c0 = nt * kG2BN + c * 32;
-                    if (valid) {
+                    if (slice_live && c0 < p.out_cols) {
+                        uint8_t* box = my_out + (out_chunk & 1) * kStageOutBytes;
+                        if (lane == 0) bulk_wait_group_read<1>();  // the store that used this buffer has read it
+                        __syncwarp();
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
-                            if (c0 + q * 4 < p.out_cols) {
-                                *reinterpret_cast<float4*>(out_row + c0 + q * 4) =
-                                    make_float4(__uint_as_float(v[q * 4]), __uint_as_float(v[q * 4 + 1]),
-                                                __uint_as_float(v[q * 4 + 2]), __uint_as_float(v[q * 4 + 3]));
-                            }
+                            const uint32_t off = (uint32_t)lane * 128u + (uint32_t)((q ^ (lane & 7)) * 16);
+                            *reinterpret_cast<uint4*>(box + off) = make_uint4(v[q * 4], v[q * 4 + 1], v[q * 4 + 2], v[q * 4 + 3]);
                         }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmOut, box, c0, ti.y + quad * 32);
+                            bulk_commit_group();
+                        }
+                        ++out_chunk;
                     }
                 }
             }
@@ -274,6 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
         }
+        if (kMode == 1 && lane == 0) bulk_wait_group<0>();  // stores complete before the CTA exits
+        __syncwarp();
     }
 
     // ---------------- teardown: every role is done (or gave up); free TMEM
@@ -285,33 +302,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int kMode>
-cudaError_t launch_impl(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& gp, int grid,
-                        cudaStream_t s) {
-    static int configured_device = -1;
+// Distinct names so profilers can tell the two GEMMs apart.
+__global__ void __launch_bounds__(kThreads, 1)
+    moe_gemm_gate_up_swiglu_bf16(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                                 const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
+    grouped_gemm_body<0>(tmA, tmB, tmOut, p);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    moe_gemm_down_bf16(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
+    grouped_gemm_body<1>(tmA, tmB, tmOut, p);
+}
+
+using GemmKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
+
+cudaError_t launch_impl(GemmKernel kern, int* configured_device, const CUtensorMap& a, const CUtensorMap& b,
+                        const CUtensorMap& o, const GemmParams& gp, int grid, cudaStream_t s) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    if (configured_device != dev) {
-        err = cudaFuncSetAttribute(grouped_gemm_bf16_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)kSmemBytes);
+    if (*configured_device != dev) {
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
         if (err != cudaSuccess) return err;
-        configured_device = dev;
+        *configured_device = dev;
     }
-    grouped_gemm_bf16_kernel<kMode><<<grid, kThreads, kSmemBytes, s>>>(a, b, gp);
+    kern<<<grid, kThreads, kSmemBytes, s>>>(a, b, o, gp);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_gemm1_bf16(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& gp, int grid,
-                              cudaStream_t s) {
-    return launch_impl<0>(a, b, gp, grid, s);
+cudaError_t launch_gemm1_bf16(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& gp,
+                              int grid, cudaStream_t s) {
+    static int configured = -1;
+    return launch_impl(moe_gemm_gate_up_swiglu_bf16, &configured, a, b, o, gp, grid, s);
 }
 
-cudaError_t launch_gemm2_bf16(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& gp, int grid,
-                              cudaStream_t s) {
-    return launch_impl<1>(a, b, gp, grid, s);
+cudaError_t launch_gemm2_bf16(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& gp,
+                              int grid, cudaStream_t s) {
+    static int configured = -1;
+    return launch_impl(moe_gemm_down_bf16, &configured, a, b, o, gp, grid, s);
 }
 
 }  // namespace moe

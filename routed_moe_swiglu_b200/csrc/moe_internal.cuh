@@ -20,6 +20,9 @@ constexpr int kBK = 64;            // bf16 K elements per pipeline stage (128-by
 constexpr int kBK8 = 128;          // E4M3 K elements per pipeline stage (128-byte rows)
 constexpr int kG1BN = 128;         // f values per gate/up tile (128 gate + 128 up MMA columns)
 constexpr int kG2BN = 256;         // output columns per down tile
+constexpr int kG1BN8 = 64;         // MXFP8: f values per gate/up tile (64 gate + 64 up MMA columns)
+constexpr int kG2BN8 = 128;        // MXFP8: output columns per down tile
+constexpr int kSfBlock = 512;      // MXFP8 scales of 128 rows x 4 k-groups, [row%32][row/32][k-group]
 constexpr int kTokPerBlk = 256;    // tokens per histogram / scatter block
 constexpr int kMaxTopK = 16;
 constexpr int kMaxExperts = 1024;
@@ -50,6 +53,8 @@ struct moe_plan {
     long long max_m_tiles;  // upper bound on M tiles: ceil(routes / BM) + E
     long long rows_pad;     // max_m_tiles * BM: rows of the padded intermediates
     int nblk;               // ceil(max_live / kTokPerBlk)
+    int ks1, ks2;           // MXFP8 K stages (128 elements) of the gate/up and down GEMMs
+    int nt1, nt2;           // N tiles of the gate/up and down GEMMs
     moe::WsLayout ws;
     moe::WbufLayout wb;
 };
@@ -67,6 +72,12 @@ struct GemmParams {
     int n_tiles;                    // N tiles per M tile
     int k_blocks;                   // pipeline stages per tile
     unsigned long long wait_limit_ns;
+    // MXFP8 only: scale blocks of A ([M tile][K stage][512 B]) and of B
+    // ([expert][N tile][K stage][512 B]); K stages of the down GEMM (the gate/up
+    // epilogue writes h's scales for it).
+    const uint8_t* sfa;
+    const uint8_t* sfb;
+    int sf_ks_out;
 };
 
 // ---------------------------------------------------------------- launchers
@@ -86,23 +97,29 @@ cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* 
 cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_live, int H, int k,
                                const int* inv, __nv_bfloat16* xp, cudaStream_t s);
 cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int k,
-                                const int* inv, uint8_t* xq, uint8_t* xs, long long rows_pad, cudaStream_t s);
+                                const int* inv, uint8_t* xq, uint8_t* xs, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const int* inv, const float* probs, const int* live, int max_live,
                            int H, int k, float* out, cudaStream_t s);
-cudaError_t launch_gemm1_bf16(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& gp, int grid,
-                              cudaStream_t s);
-cudaError_t launch_gemm2_bf16(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& gp, int grid,
-                              cudaStream_t s);
-cudaError_t launch_gemm1_mxfp8(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sfa,
-                               const CUtensorMap& sfb, const GemmParams& gp, int grid, cudaStream_t s);
-cudaError_t launch_gemm2_mxfp8(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& sfa,
-                               const CUtensorMap& sfb, const GemmParams& gp, int grid, cudaStream_t s);
+cudaError_t launch_gemm1_bf16(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& gp,
+                              int grid, cudaStream_t s);
+cudaError_t launch_gemm2_bf16(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& gp,
+                              int grid, cudaStream_t s);
+cudaError_t launch_gemm1_mxfp8(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o,
+                               const GemmParams& gp, int grid, cudaStream_t s);
+cudaError_t launch_gemm2_mxfp8(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o,
+                               const GemmParams& gp, int grid, cudaStream_t s);
 cudaError_t launch_prepare_bf16(const moe_plan* p, const __nv_bfloat16* wg, const __nv_bfloat16* wu,
                                 const __nv_bfloat16* wd, void* buf, cudaStream_t s);
 cudaError_t launch_prepare_mxfp8(const moe_plan* p, const __nv_bfloat16* wg, const __nv_bfloat16* wu,
                                  const __nv_bfloat16* wd, void* buf, cudaStream_t s);
 cudaError_t launch_quantize_rows(const __nv_bfloat16* in, long long rows, int cols, long long ld_in, uint8_t* q,
                                  uint8_t* scales, const int* live_rows, cudaStream_t s);
+
+// Byte offset of (row within a 128-row tile, k-group within a 4-group K
+// stage) inside one 512-byte MXFP8 scale block.
+__host__ __device__ __forceinline__ uint32_t sf_block_offset(int row, int kg) {
+    return (uint32_t)((row & 31) * 16 + ((row >> 5) & 3) * 4 + kg);
+}
 
 __device__ __forceinline__ int clamp_live(const int* live, int max_live) {
     int n = __ldg(live);

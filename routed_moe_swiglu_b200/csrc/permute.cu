@@ -15,6 +15,7 @@
 //            same expert (popcount of the lower lanes plus the earlier warps)
 // and a gather that copies x rows into their padded route rows.
 #include "moe_internal.cuh"
+#include "mxfp8.cuh"
 
 namespace moe {
 namespace {
@@ -155,63 +156,119 @@ __global__ void __launch_bounds__(kTokPerBlk) route_scatter_kernel(
     }
 }
 
-// One warp per token: read the token's x row once, write it to each of its
-// k padded route rows (16-byte chunks, coalesced).
-__global__ void __launch_bounds__(256) gather_rows_bf16_kernel(const uint4* __restrict__ x,
-                                                               const int* __restrict__ live, int max_live,
-                                                               int H, int k, const int* __restrict__ inv,
-                                                               uint4* __restrict__ xp) {
+// One 128-thread block per token (grid-stride): read the token's x row once,
+// write it to each of its k padded route rows; every thread keeps all of its
+// 16-byte loads in flight before storing.
+constexpr int kRowThreads = 128;
+
+__global__ void __launch_bounds__(kRowThreads) gather_rows_bf16_kernel(const uint4* __restrict__ x,
+                                                                       const int* __restrict__ live, int max_live,
+                                                                       int H, int k, const int* __restrict__ inv,
+                                                                       uint4* __restrict__ xp) {
+    __shared__ int s_prow[kMaxTopK];
     const int n = clamp_live(live, max_live);
-    const int lane = threadIdx.x & 31;
-    const int wpb = blockDim.x >> 5;
     const int chunks = H / 8;  // 8 bf16 per 16 bytes
-    for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < n; t += gridDim.x * wpb) {
-        const int mine = lane < k ? __ldg(inv + (size_t)t * k + lane) : -1;
-        int prow[kMaxTopK];
-#pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j) prow[j] = __shfl_sync(0xffffffffu, mine, j);
+    for (int t = blockIdx.x; t < n; t += gridDim.x) {
+        __syncthreads();
+        if (threadIdx.x < k) s_prow[threadIdx.x] = __ldg(inv + (size_t)t * k + threadIdx.x);
+        __syncthreads();
         const uint4* src = x + (size_t)t * chunks;
-        for (int c = lane; c < chunks; c += 32) {
+#pragma unroll 4
+        for (int c = threadIdx.x; c < chunks; c += kRowThreads) {
             const uint4 v = __ldg(src + c);
-#pragma unroll
-            for (int j = 0; j < kMaxTopK; ++j)
-                if (j < k && prow[j] >= 0) xp[(size_t)prow[j] * chunks + c] = v;
+            for (int j = 0; j < k; ++j) {
+                const int pr = s_prow[j];
+                if (pr >= 0) xp[(size_t)pr * chunks + c] = v;
+            }
         }
     }
 }
 
-// One warp per token: out[t] = sum_j p_j * y[inv[t,j]] as fp32 FMAs from
-// zero, j in ascending expert id (Megatron-LM PR #7798, "What is changed":
-// the unpermute adds a token's routes as fp32 fused multiply-adds of
-// probability and row, from zero, in a fixed order; PR #8367: fp32 result).
-__global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ y, const int* __restrict__ inv,
-                                                      const float* __restrict__ probs,
-                                                      const int* __restrict__ live, int max_live, int H, int k,
-                                                      float4* __restrict__ out) {
+// MXFP8 gather: one 128-thread block per token quantises the token's x row
+// once (blocks of 32 along H, 4 threads per block) and writes the E4M3 codes
+// to each of its k padded route rows and the E8M0 bytes into the scale
+// blocks of those rows' M tiles ([tile][K stage][512 B]).
+__global__ void __launch_bounds__(kRowThreads) gather_rows_mxfp8_kernel(const uint4* __restrict__ x,
+                                                                        const int* __restrict__ live, int max_live,
+                                                                        int H, int k, int ks1,
+                                                                        const int* __restrict__ inv,
+                                                                        uint2* __restrict__ xq,
+                                                                        uint8_t* __restrict__ xs) {
+    __shared__ int s_prow[kMaxTopK];
     const int n = clamp_live(live, max_live);
-    const int lane = threadIdx.x & 31;
-    const int wpb = blockDim.x >> 5;
-    const int chunks = H / 4;
-    for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < n; t += gridDim.x * wpb) {
-        const int mine = lane < k ? __ldg(inv + (size_t)t * k + lane) : -1;
-        const float pmine = lane < k ? __ldg(probs + (size_t)t * k + lane) : 0.0f;
-        int prow[kMaxTopK];
-        float pj[kMaxTopK];
-#pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j) {
-            prow[j] = __shfl_sync(0xffffffffu, mine, j);
-            pj[j] = __shfl_sync(0xffffffffu, pmine, j);
+    const int chunks = H / 8;
+    for (int t = blockIdx.x; t < n; t += gridDim.x) {
+        __syncthreads();
+        if (threadIdx.x < k) s_prow[threadIdx.x] = __ldg(inv + (size_t)t * k + threadIdx.x);
+        __syncthreads();
+        const uint4* src = x + (size_t)t * chunks;
+        for (int c0 = 0; c0 < chunks; c0 += kRowThreads) {  // uniform trip count: shuffles inside
+            const int c = c0 + threadIdx.x;
+            const bool active = c < chunks;  // H % 32 == 0: 4-thread groups are all in or all out
+            const uint4 v = active ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            uint8_t sb;
+            const uint2 codes = mxfp8_quantize_8(v, &sb);
+            if (active) {
+                const int g = c >> 2;  // 32-element block index along H
+                for (int j = 0; j < k; ++j) {
+                    const int pr = s_prow[j];
+                    if (pr < 0) continue;
+                    xq[(size_t)pr * chunks + c] = codes;
+                    if ((c & 3) == 0)
+                        xs[((size_t)(pr / kBM) * ks1 + g / 4) * kSfBlock + sf_block_offset(pr % kBM, g % 4)] = sb;
+                }
+            }
         }
-        for (int c = lane; c < chunks; c += 32) {
+        // k-group slots past H/32 in the last K stage: scale byte 0 (their codes are TMA zero fill)
+        if (threadIdx.x < k) {
+            const int pr = s_prow[threadIdx.x];
+            if (pr >= 0)
+                for (int g = H / 32; g < 4 * ks1; ++g)
+                    xs[((size_t)(pr / kBM) * ks1 + g / 4) * kSfBlock + sf_block_offset(pr % kBM, g % 4)] = 0;
+        }
+    }
+}
+
+// One 128-thread block per token: out[t] = sum_j p_j * y[inv[t,j]] as fp32
+// FMAs from zero, j in ascending expert id (Megatron-LM PR #7798, "What is
+// changed": the unpermute adds a token's routes as fp32 fused multiply-adds
+// of probability and row, from zero, in a fixed order; PR #8367: fp32
+// result).  The k rows' loads of a chunk are all issued before the FMA chain.
+__global__ void __launch_bounds__(kRowThreads) combine_kernel(const float4* __restrict__ y,
+                                                              const int* __restrict__ inv,
+                                                              const float* __restrict__ probs,
+                                                              const int* __restrict__ live, int max_live, int H,
+                                                              int k, float4* __restrict__ out) {
+    __shared__ int s_prow[kMaxTopK];
+    __shared__ float s_p[kMaxTopK];
+    const int n = clamp_live(live, max_live);
+    const int chunks = H / 4;
+    for (int t = blockIdx.x; t < n; t += gridDim.x) {
+        __syncthreads();
+        if (threadIdx.x < k) {
+            s_prow[threadIdx.x] = __ldg(inv + (size_t)t * k + threadIdx.x);
+            s_p[threadIdx.x] = __ldg(probs + (size_t)t * k + threadIdx.x);
+        }
+        __syncthreads();
+        for (int c = threadIdx.x; c < chunks; c += kRowThreads) {
+            // loads of up to 8 routes in flight at once, then their FMAs in order
             float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            for (int j0 = 0; j0 < k; j0 += 8) {
+                float4 v[8];
 #pragma unroll
-            for (int j = 0; j < kMaxTopK; ++j) {
-                if (j < k && prow[j] >= 0) {
-                    const float4 v = __ldg(y + (size_t)prow[j] * chunks + c);
-                    acc.x = __fmaf_rn(pj[j], v.x, acc.x);
-                    acc.y = __fmaf_rn(pj[j], v.y, acc.y);
-                    acc.z = __fmaf_rn(pj[j], v.z, acc.z);
-                    acc.w = __fmaf_rn(pj[j], v.w, acc.w);
+                for (int jj = 0; jj < 8; ++jj) {
+                    const int pr = j0 + jj < k ? s_prow[j0 + jj] : -1;
+                    v[jj] = pr >= 0 ? __ldg(y + (size_t)pr * chunks + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    if (j0 + jj < k && s_prow[j0 + jj] >= 0) {
+                        const float p = s_p[j0 + jj];
+                        acc.x = __fmaf_rn(p, v[jj].x, acc.x);
+                        acc.y = __fmaf_rn(p, v[jj].y, acc.y);
+                        acc.z = __fmaf_rn(p, v[jj].z, acc.z);
+                        acc.w = __fmaf_rn(p, v[jj].w, acc.w);
+                    }
                 }
             }
             out[(size_t)t * chunks + c] = acc;
@@ -262,16 +319,24 @@ cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* 
 
 cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_live, int H, int k,
                                const int* inv, __nv_bfloat16* xp, cudaStream_t s) {
-    const int grid = grid_for_warps(max_live, 8, 8);
-    gather_rows_bf16_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(x), live, max_live, H, k, inv,
+    const int grid = grid_for_warps(max_live, 1, 16);
+    gather_rows_bf16_kernel<<<grid, kRowThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), live, max_live, H, k, inv,
                                                  reinterpret_cast<uint4*>(xp));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int k,
+                                const int* inv, uint8_t* xq, uint8_t* xs, cudaStream_t s) {
+    const int grid = grid_for_warps(max_live, 1, 16);
+    gather_rows_mxfp8_kernel<<<grid, kRowThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), live, max_live, H, k,
+                                                          (H + kBK8 - 1) / kBK8, inv, reinterpret_cast<uint2*>(xq), xs);
     return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const float* y, const int* inv, const float* probs, const int* live, int max_live,
                            int H, int k, float* out, cudaStream_t s) {
-    const int grid = grid_for_warps(max_live, 8, 8);
-    combine_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(y), inv, probs, live, max_live, H, k,
+    const int grid = grid_for_warps(max_live, 1, 16);
+    combine_kernel<<<grid, kRowThreads, 0, s>>>(reinterpret_cast<const float4*>(y), inv, probs, live, max_live, H, k,
                                         reinterpret_cast<float4*>(out));
     return cudaGetLastError();
 }

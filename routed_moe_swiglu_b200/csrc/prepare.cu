@@ -8,6 +8,7 @@
 // A gate/up tile loads the same 128 f rows from W1[e][0] and W1[e][1] into
 // one 256-row B operand, so gate and up of one f meet in one accumulator row.
 #include "moe_internal.cuh"
+#include "mxfp8.cuh"
 
 namespace moe {
 namespace {
@@ -46,10 +47,76 @@ cudaError_t launch_prepare_bf16(const moe_plan* p, const __nv_bfloat16* wg, cons
 }  // namespace moe
 
 namespace moe {
-// MXFP8 weight preparation is built with the MXFP8 GEMMs; until then plans
-// reject MXFP8 and this is never reached.
-cudaError_t launch_prepare_mxfp8(const moe_plan*, const __nv_bfloat16*, const __nv_bfloat16*, const __nv_bfloat16*,
-                                 void*, cudaStream_t) {
-    return cudaErrorNotSupported;
+namespace {
+
+// MXFP8 weights: one 128-thread block per weight row (grid-stride), blocks of
+// 32 along the row (the GEMM's K), codes in place of the bf16 layout and
+// scale bytes in the GEMMs' B scale blocks:
+//   gate/up row (e, g/u, f): N tile f / 64, tile row g/u * 64 + f % 64
+//   down row (e, c):         N tile c / 128, tile row c % 128
+__global__ void __launch_bounds__(128) prepare_mxfp8_kernel(const uint4* __restrict__ wg, const uint4* __restrict__ wu,
+                                                            const uint4* __restrict__ wd, uint2* __restrict__ w1q,
+                                                            uint8_t* __restrict__ w1s, uint2* __restrict__ w2q,
+                                                            uint8_t* __restrict__ w2s, int E, int F, int H, int nt1,
+                                                            int ks1, int nt2, int ks2) {
+    const long long rows1 = (long long)E * 2 * F;
+    const long long rows2 = (long long)E * H;
+    for (long long row = blockIdx.x; row < rows1 + rows2; row += gridDim.x) {
+        const uint4* src;
+        uint2* dst;
+        uint8_t* sf_tile;  // the K-stage-0 scale block of this row's N tile
+        int len, trow;
+        if (row < rows1) {
+            const long long e = row / (2 * F);
+            const int rem = (int)(row - e * 2 * F);
+            const int gu = rem / F, f = rem - gu * F;
+            src = (gu ? wu : wg) + ((size_t)e * F + f) * (H / 8);
+            dst = w1q + (size_t)row * (H / 8);
+            len = H;
+            trow = gu * (kG1BN8) + f % kG1BN8;
+            sf_tile = w1s + ((size_t)e * nt1 + f / kG1BN8) * ks1 * kSfBlock;
+        } else {
+            const long long r2 = row - rows1;
+            const long long e = r2 / H;
+            const int c = (int)(r2 - e * H);
+            src = wd + (size_t)r2 * (F / 8);
+            dst = w2q + (size_t)r2 * (F / 8);
+            len = F;
+            trow = c % kG2BN8;
+            sf_tile = w2s + ((size_t)e * nt2 + c / kG2BN8) * ks2 * kSfBlock;
+        }
+        const int chunks = len / 8;
+        for (int c0 = 0; c0 < chunks; c0 += blockDim.x) {
+            const int c = c0 + threadIdx.x;
+            const bool active = c < chunks;
+            const uint4 v = active ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            uint8_t sb;
+            const uint2 codes = mxfp8_quantize_8(v, &sb);
+            if (active) {
+                dst[c] = codes;
+                const int g = c >> 2;
+                if ((c & 3) == 0) sf_tile[(size_t)(g / 4) * kSfBlock + sf_block_offset(trow, g % 4)] = sb;
+            }
+        }
+    }
 }
+
+}  // namespace
+
+cudaError_t launch_prepare_mxfp8(const moe_plan* p, const __nv_bfloat16* wg, const __nv_bfloat16* wu,
+                                 const __nv_bfloat16* wd, void* buf, cudaStream_t s) {
+    uint8_t* base = static_cast<uint8_t*>(buf);
+    const int E = p->d.num_experts, F = p->d.ffn, H = p->d.hidden;
+    // padding rows and k-groups of the scale blocks hold byte 0 (scale 2^-127)
+    cudaError_t err = cudaMemsetAsync(base + p->wb.w1s, 0, p->wb.w2 - p->wb.w1s, s);
+    if (err != cudaSuccess) return err;
+    err = cudaMemsetAsync(base + p->wb.w2s, 0, p->wb.total - p->wb.w2s, s);
+    if (err != cudaSuccess) return err;
+    prepare_mxfp8_kernel<<<num_sms() * 16, 128, 0, s>>>(
+        reinterpret_cast<const uint4*>(wg), reinterpret_cast<const uint4*>(wu), reinterpret_cast<const uint4*>(wd),
+        reinterpret_cast<uint2*>(base + p->wb.w1), base + p->wb.w1s, reinterpret_cast<uint2*>(base + p->wb.w2),
+        base + p->wb.w2s, E, F, H, p->nt1, p->ks1, p->nt2, p->ks2);
+    return cudaGetLastError();
+}
+
 }  // namespace moe

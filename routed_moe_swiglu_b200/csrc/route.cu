@@ -14,7 +14,10 @@
 namespace moe {
 namespace {
 
-// One warp per token.  Logit `id` lives in lane id % 32, slot id / 32.
+// One warp per token.  Logit `id` lives in lane id % 32, slot id / 32;
+// kSlots = ceil(E / 32) is a template parameter so the per-lane scans are
+// fully unrolled over registers.
+template <int kSlots>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits,
                                                          const int* __restrict__ live, int max_live, int E,
                                                          int k, int* __restrict__ ids,
@@ -26,16 +29,15 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
 
     const int lane = threadIdx.x & 31;
     const int warps_per_block = blockDim.x >> 5;
-    const int nslots = (E + 31) >> 5;
     for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < n; t += gridDim.x * warps_per_block) {
         const float* row = logits + (size_t)t * E;
-        float v[32];
+        float v[kSlots];
         uint32_t taken = 0;
 #pragma unroll
-        for (int s = 0; s < 32; ++s) {
+        for (int s = 0; s < kSlots; ++s) {
             const int id = lane + 32 * s;
             float x = -INFINITY;
-            if (s < nslots && id < E) {
+            if (id < E) {
                 x = __ldg(row + id);
                 if (x != x) x = -INFINITY;  // NaN never wins over a number
             } else {
@@ -43,65 +45,52 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
             }
             v[s] = x;
         }
-        float sel_v[kMaxTopK];
-        int sel_id[kMaxTopK];
+        // k rounds of a warp arg-max on (value desc, id asc); every lane ends
+        // each round with the winner, lane j keeps round j's winner
+        float first_v = 0.0f, my_v = 0.0f;
+        int my_id = 0x7fffffff;
+        for (int j = 0; j < k; ++j) {
+            float bv = 0.0f;
+            int bid = -1;
 #pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j) {
-            if (j < k) {
-                float bv = 0.0f;
-                int bid = -1;
-#pragma unroll
-                for (int s = 0; s < 32; ++s) {
-                    // ids grow with s inside a lane: strict '>' keeps the lower id on ties
-                    if (s < nslots && !((taken >> s) & 1u) && (bid < 0 || v[s] > bv)) {
-                        bv = v[s];
-                        bid = lane + 32 * s;
-                    }
+            for (int s = 0; s < kSlots; ++s) {
+                // ids grow with s inside a lane: strict '>' keeps the lower id on ties
+                if (!((taken >> s) & 1u) && (bid < 0 || v[s] > bv)) {
+                    bv = v[s];
+                    bid = lane + 32 * s;
                 }
+            }
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                    const int oid = __shfl_xor_sync(0xffffffffu, bid, off);
-                    const bool better = oid >= 0 && (bid < 0 || ov > bv || (ov == bv && oid < bid));
-                    if (better) {
-                        bv = ov;
-                        bid = oid;
-                    }
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oid = __shfl_xor_sync(0xffffffffu, bid, off);
+                const bool better = oid >= 0 && (bid < 0 || ov > bv || (ov == bv && oid < bid));
+                if (better) {
+                    bv = ov;
+                    bid = oid;
                 }
-                if ((bid & 31) == lane) taken |= 1u << (bid >> 5);
-                sel_v[j] = bv;
-                sel_id[j] = bid;
+            }
+            if ((bid & 31) == lane) taken |= 1u << (bid >> 5);
+            if (j == 0) first_v = bv;
+            if (j == lane) {
+                my_v = bv;
+                my_id = bid;
             }
         }
-        if (lane == 0) {
-            // renormalised softmax over the chosen k: exp(l_j - max) / sum, in double
-            const double m = (double)sel_v[0];
-            double w[kMaxTopK];
-            double z = 0.0;
-#pragma unroll
-            for (int j = 0; j < kMaxTopK; ++j) {
-                if (j < k) {
-                    w[j] = exp((double)sel_v[j] - m);
-                    z += w[j];
-                }
-            }
-            // ascending expert id, probabilities travel with their ids
-            for (int a = 1; a < k; ++a) {
-                const int id = sel_id[a];
-                const double ww = w[a];
-                int b = a - 1;
-                while (b >= 0 && sel_id[b] > id) {
-                    sel_id[b + 1] = sel_id[b];
-                    w[b + 1] = w[b];
-                    --b;
-                }
-                sel_id[b + 1] = id;
-                w[b + 1] = ww;
-            }
-            for (int j = 0; j < k; ++j) {
-                ids[(size_t)t * k + j] = sel_id[j];
-                probs[(size_t)t * k + j] = (float)(w[j] / z);
-            }
+        // Renormalised softmax over the chosen k: exp(l_j - max) / sum, in
+        // double, summed in selection order (the same order in every lane).
+        const double w = lane < k ? exp((double)my_v - (double)first_v) : 0.0;
+        double z = 0.0;
+        for (int j = 0; j < k; ++j) z += __shfl_sync(0xffffffffu, w, j);
+        // rank of route j among the k in ascending expert id
+        int rank = 0;
+        for (int j = 0; j < k; ++j) {
+            const int other = __shfl_sync(0xffffffffu, my_id, j);
+            rank += other < my_id ? 1 : 0;
+        }
+        if (lane < k) {
+            ids[(size_t)t * k + rank] = my_id;
+            probs[(size_t)t * k + rank] = (float)(w / z);
         }
     }
 }
@@ -158,7 +147,15 @@ cudaError_t launch_route_topk(const float* logits, const int* live, int max_live
     const long long cap = (long long)num_sms() * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    route_topk_kernel<<<(unsigned)blocks, warps * 32, 0, s>>>(logits, live, max_live, E, k, ids, probs, status);
+    const int slots = (E + 31) / 32;
+    if (slots <= 4)
+        route_topk_kernel<4><<<(unsigned)blocks, warps * 32, 0, s>>>(logits, live, max_live, E, k, ids, probs, status);
+    else if (slots <= 8)
+        route_topk_kernel<8><<<(unsigned)blocks, warps * 32, 0, s>>>(logits, live, max_live, E, k, ids, probs, status);
+    else if (slots <= 16)
+        route_topk_kernel<16><<<(unsigned)blocks, warps * 32, 0, s>>>(logits, live, max_live, E, k, ids, probs, status);
+    else
+        route_topk_kernel<32><<<(unsigned)blocks, warps * 32, 0, s>>>(logits, live, max_live, E, k, ids, probs, status);
     return cudaGetLastError();
 }
 

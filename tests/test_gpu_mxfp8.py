@@ -1,0 +1,156 @@
+"""MXFP8 path vs the oracle: weight and activation quantisation inside
+prepare/forward bit-exact, the SwiGLU intermediate's codes equal the
+oracle's up to last-bit accumulation-order effects, outputs within the MXFP8
+tolerance (max |d| <= 5e-2 * RMS)."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import routed_moe_swiglu_b200 as rm
+import workloads
+from moe_testlib import GpuMoe, assert_close, oracle_forward, workload_problem
+
+pytestmark = pytest.mark.gpu
+
+SF_BLOCK = 512
+
+
+def sf_offset(row, g):
+    row = np.asarray(row)
+    return (row % 32) * 16 + ((row // 32) % 4) * 4 + g
+
+
+def decode_scales(blob: np.ndarray, rows: np.ndarray, K: int) -> np.ndarray:
+    """Scale bytes [len(rows), K/32] of padded rows from the [tile][stage][512] layout."""
+    ks = (K + 127) // 128
+    out = np.empty((rows.size, K // 32), np.uint8)
+    for g in range(K // 32):
+        idx = ((rows // 128) * ks + g // 4) * SF_BLOCK + sf_offset(rows % 128, g % 4)
+        out[:, g] = blob[idx]
+    return out
+
+
+def _ws_bytes(m: GpuMoe, ptr, nbytes):
+    off = ptr - m.ws.data_ptr()
+    return m.ws[off:off + nbytes].cpu().numpy()
+
+
+def test_prepare_weights_bit_exact():
+    H, F, E = 256, 192, 3  # F not a multiple of 128: partial N tile and K stage
+    gen = torch.Generator().manual_seed(31)
+    wg = (torch.randn((E, F, H), generator=gen) * torch.exp(torch.randn((E, F, 1), generator=gen))).bfloat16()
+    wu = (torch.randn((E, F, H), generator=gen) * 0.1).bfloat16()
+    wd = (torch.randn((E, H, F), generator=gen) * torch.exp(torch.randn((E, H, 1), generator=gen) * 3)).bfloat16()
+    plan = rm.moe_plan_create(hidden=H, ffn=F, num_experts=E, top_k=2, capacity=16, precision="mxfp8")
+    buf = rm.alloc_weight_buffer(plan)
+    rm.moe_prepare_weights(plan, wg.cuda(), wu.cuda(), wd.cuda(), buf)
+    torch.cuda.synchronize()
+    b = buf.cpu().numpy()
+    gq, gs, uq, us, dq, ds = oracle.quantize_weights_mxfp8(wg, wu, wd)
+    n1 = E * 2 * F * H
+    w1 = b[:n1].reshape(E, 2, F, H)
+    assert np.array_equal(w1[:, 0], gq) and np.array_equal(w1[:, 1], uq)
+    al = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    nt1, ks1 = (F + 63) // 64, (H + 127) // 128
+    off_w1s = al(n1)
+    w1s = b[off_w1s:off_w1s + E * nt1 * ks1 * SF_BLOCK]
+    for e in range(E):
+        for gu, ref in ((0, gs), (1, us)):
+            f = np.arange(F)
+            for g in range(H // 32):
+                idx = ((e * nt1 + f // 64) * ks1 + g // 4) * SF_BLOCK + sf_offset(gu * 64 + f % 64, g % 4)
+                assert np.array_equal(w1s[idx], ref[e, :, g]), (e, gu, g)
+    off_w2 = off_w1s + al(E * nt1 * ks1 * SF_BLOCK)
+    w2 = b[off_w2:off_w2 + E * H * F].reshape(E, H, F)
+    assert np.array_equal(w2, dq)
+    nt2, ks2 = (H + 127) // 128, (F + 127) // 128
+    off_w2s = off_w2 + al(E * H * F)
+    w2s = b[off_w2s:off_w2s + E * nt2 * ks2 * SF_BLOCK]
+    c = np.arange(H)
+    for e in range(E):
+        for g in range(F // 32):
+            idx = ((e * nt2 + c // 128) * ks2 + g // 4) * SF_BLOCK + sf_offset(c % 128, g % 4)
+            assert np.array_equal(w2s[idx], ds[e, :, g]), (e, g)
+        # k-group slots past F/32 in the last stage are scale byte 0
+        for g in range(F // 32, 4 * ks2):
+            idx = ((e * nt2 + c // 128) * ks2 + g // 4) * SF_BLOCK + sf_offset(c % 128, g % 4)
+            assert np.all(w2s[idx] == 0)
+
+
+def _check_intermediates(m: GpuMoe, x, ids, H, F, toks, h_ref):
+    v = m.views()
+    live, k = ids.shape
+    inv = m.read_i32(v["inv"], live * k).reshape(live, k)
+    rows = inv[toks].reshape(-1).astype(np.int64)
+    R = v["rows_padded"]
+    # x codes and scales of every sampled route row equal the oracle's quantisation of x[t]
+    xq_all = _ws_bytes(m, v["xq"], R * H).reshape(R, H)
+    xs_blob = _ws_bytes(m, v["xq_scales"], (R // 128) * ((H + 127) // 128) * SF_BLOCK)
+    ref_q, ref_s = oracle.mxfp8_quantize_bf16(x[torch.from_numpy(np.repeat(toks, k))].contiguous())
+    assert np.array_equal(xq_all[rows], ref_q)
+    assert np.array_equal(decode_scales(xs_blob, rows, H), ref_s)
+    # h: codes/scales equal the oracle's wherever the fp32 pre-quantisation value agrees
+    hq_all = _ws_bytes(m, v["h"], R * F).reshape(R, F)
+    hs_blob = _ws_bytes(m, v["h_scales"], (R // 128) * ((F + 127) // 128) * SF_BLOCK)
+    hq_ref, hs_ref, _ = h_ref
+    got_q = hq_all[rows].reshape(len(toks), k, F)
+    got_s = decode_scales(hs_blob, rows, F).reshape(len(toks), k, F // 32)
+    frac_s = np.mean(got_s == hs_ref)
+    frac_q = np.mean(got_q == hq_ref)
+    assert frac_s > 0.995 and frac_q > 0.995, (frac_s, frac_q)
+    # where a code differs with the same scale it is a neighbouring grid point
+    same_s = np.repeat(got_s == hs_ref, 32, axis=2)
+    diff = (got_q != hq_ref) & same_s
+    a = got_q[diff].astype(np.int32)
+    b = hq_ref[diff].astype(np.int32)
+    mag = lambda c: np.where(c & 0x80, -(c & 0x7F), c & 0x7F)  # noqa: E731
+    assert np.all(np.abs(mag(a) - mag(b)) <= 1), np.stack([a, b])[:, :10]
+
+
+@pytest.mark.parametrize("H,F,E,k,T", [(256, 256, 8, 2, 64), (320, 224, 6, 3, 200), (512, 1024, 16, 4, 300)])
+def test_forward_mxfp8_small(H, F, E, k, T):
+    x, logits, weights = workloads.small_case(H, F, E, k, T, seed=H + F, capacity=T + 16)
+    m = GpuMoe(H, F, E, k, T + 16, weights, precision="mxfp8")
+    out = m.forward(x.cuda(), T, logits=logits.cuda())
+    torch.cuda.synchronize()
+    ids, probs = oracle.route(logits[:T].numpy(), k)
+    wq = oracle.quantize_weights_mxfp8(*weights)
+    ref, h_ref = oracle.forward_mxfp8(x[:T], ids, probs, wq, want_h=True)
+    o = out.cpu().numpy()
+    assert_close(o[:T], ref, "mxfp8", f"mxfp8 {H},{F},{E},{k},{T}")
+    assert np.all(np.isnan(o[T:]))
+    _check_intermediates(m, x, ids, H, F, np.arange(T), h_ref)
+    assert m.status() == 0
+
+
+def test_forward_mxfp8_workload_subset():
+    w, x, logits, weights = workload_problem("mxfp8")
+    m = GpuMoe(w.hidden, w.ffn, w.num_experts, w.top_k, w.capacity, weights, precision="mxfp8")
+    live = w.max_live
+    out = m.forward(x.cuda(), live, logits=logits.cuda())
+    torch.cuda.synchronize()
+    toks = workloads.sample_tokens(live, 256, w.seed).numpy()
+    ids, probs = oracle.route(logits[:live].numpy(), w.top_k)
+    wq = oracle.quantize_weights_mxfp8(*weights)
+    ref, h_ref = oracle.forward_mxfp8(x[:live], ids, probs, wq, tokens=toks, want_h=True)
+    assert_close(out.cpu().numpy()[toks], ref, "mxfp8", "mxfp8 workload subset")
+    _check_intermediates(m, x, ids, w.hidden, w.ffn, toks, h_ref)
+    # the MXFP8 result stays a few percent from the bf16 oracle (the pages report ~4%)
+    ref_bf16 = oracle.forward_bf16(x[:live], ids, probs, *weights, tokens=toks)
+    d = np.linalg.norm(out.cpu().numpy()[toks] - ref_bf16) / np.linalg.norm(ref_bf16)
+    assert 0.01 < d < 0.08, d
+
+
+def test_mxfp8_batch_invariance():
+    H, F, E, k = 512, 512, 16, 4
+    x, logits, weights = workloads.small_case(H, F, E, k, 600, seed=41)
+    m = GpuMoe(H, F, E, k, 600, weights, precision="mxfp8")
+    xd, ld = x.cuda(), logits.cuda()
+    a = m.forward(xd, 600, logits=ld).cpu()
+    for n in (1, 33, 300):
+        b = m.forward(xd, n, logits=ld).cpu()
+        assert torch.equal(b[:n], a[:n])
+    assert torch.equal(m.forward(xd, 600, logits=ld).cpu(), a)
