@@ -163,6 +163,33 @@ moe_status moe_forward(const moe_plan* plan, const void* x, const float* logits,
                        const float* probs, const void* kernel_buf, const int* live_count_dev,
                        float* out, void* workspace, size_t ws_bytes, void* stream);
 
+/* moe_forward for callers that cannot allocate device memory (no
+ * counterpart in the pages: an addition of this library).  Some callers get
+ * only their input and output pointers and have no allocator to call -- a
+ * plug-in living inside another engine's memory budget, or code that must not
+ * call cudaMalloc because it would synchronise the device or is not allowed
+ * under the caller's stream capture.  This entry point takes no workspace:
+ * its scratch is one fixed array of MOE_NOALLOC_SCRATCH_BYTES (64 MiB) in
+ * the library's device memory, which every GPU that loads this part of the
+ * library holds until the process exits.  It calls no cudaMalloc, cudaFree
+ * or other allocating routine.
+ *   - Arguments as moe_forward, minus the workspace.
+ *   - Plans whose moe_workspace_bytes exceeds MOE_NOALLOC_SCRATCH_BYTES are
+ *     rejected with MOE_ERR_WORKSPACE_TOO_SMALL before anything runs (use a
+ *     smaller max_live_rows, or moe_forward with your own workspace).
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call, on every stream, shares the one array, which keeps the
+ *     last call's contents: calls that overlap on the GPU race with each
+ *     other.  Serialise them (one stream, or events).
+ *   - The device status word lives in the shared array and is cleared at the
+ *     start of each call; it cannot be read back through this entry point.
+ *   - Same results as moe_forward on the same inputs. */
+#define MOE_NOALLOC_SCRATCH_BYTES (64ull << 20)
+moe_status moe_forward_noalloc(const moe_plan* plan, const void* x, const float* logits, const int* ids,
+                               const float* probs, const void* kernel_buf, const int* live_count_dev,
+                               float* out, void* stream);
+
 /* Stages of moe_forward, in launch order: route (or canonicalise the
  * caller's routes), permute (histogram, scan, scatter), gather of x rows
  * (and their MXFP8 quantisation), gate/up GEMM with SwiGLU, down GEMM,

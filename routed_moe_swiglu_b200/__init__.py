@@ -26,6 +26,7 @@ __all__ = [
     "MoeError", "Plan", "load_library", "library_path", "moe_version", "moe_plan_create", "moe_plan_destroy",
     "moe_weight_buffer_bytes", "moe_workspace_bytes", "alloc_weight_buffer", "alloc_workspace",
     "moe_prepare_weights", "mxfp8_quantize_block32", "moe_route_topk", "moe_forward", "moe_forward_with_events",
+    "moe_forward_noalloc", "MOE_NOALLOC_SCRATCH_BYTES",
     "MOE_NUM_STAGES", "STAGE_NAMES",
     "moe_get_workspace_views", "moe_get_device_status", "moe_clear_device_status",
     "MOE_DEV_LIVE_CLAMPED", "MOE_DEV_BAD_ROUTE", "MOE_DEV_TIMEOUT",
@@ -83,6 +84,7 @@ def load_library():
         "moe_route_topk": ([P, P, P, P, P, P], I),
         "moe_forward": ([P, P, P, P, P, P, P, P, P, SZ, P], I),
         "moe_forward_with_events": ([P, P, P, P, P, P, P, P, P, SZ, P, ctypes.POINTER(P)], I),
+        "moe_forward_noalloc": ([P, P, P, P, P, P, P, P, P], I),
         "moe_get_workspace_views": ([P, P, ctypes.POINTER(_Views)], I),
         "moe_get_device_status": ([P, ctypes.POINTER(ctypes.c_uint), P], I),
         "moe_clear_device_status": ([P, P], I),
@@ -218,6 +220,20 @@ def moe_forward(plan: Plan, x, kernel_buf, live_count, out, workspace, logits=No
     _check(load_library().moe_forward(plan.handle, _ptr(x), _ptr(logits), _ptr(ids), _ptr(probs), _ptr(kernel_buf),
                                       _ptr(live_count), _ptr(out), _ptr(workspace),
                                       workspace.numel() * workspace.element_size(), _stream(stream)), "moe_forward")
+
+
+MOE_NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def moe_forward_noalloc(plan: Plan, x, kernel_buf, live_count, out, logits=None, ids=None, probs=None,
+                        stream=None) -> None:
+    """moe_forward without a workspace, for callers that cannot allocate device
+    memory: the library's own fixed scratch array (MOE_NOALLOC_SCRATCH_BYTES)
+    serves every call, so calls must not overlap on the GPU.  Make the first
+    call on a device outside any stream capture."""
+    _check(load_library().moe_forward_noalloc(plan.handle, _ptr(x), _ptr(logits), _ptr(ids), _ptr(probs),
+                                              _ptr(kernel_buf), _ptr(live_count), _ptr(out), _stream(stream)),
+           "moe_forward_noalloc")
 
 
 MOE_NUM_STAGES = 6
