@@ -190,9 +190,9 @@ def measured_peaks():
 
 
 KERNEL_SOURCES = {
-    "gemm_gate_up": ["routed_moe_swiglu_b200/csrc/gemm_bf16.cu", "routed_moe_swiglu_b200/csrc/ptx.cuh",
+    "gemm_gate_up": ["routed_moe_swiglu_b200/csrc/gemm_bf16_pair.cu", "routed_moe_swiglu_b200/csrc/ptx.cuh",
                      "routed_moe_swiglu_b200/csrc/moe_internal.cuh"],
-    "gemm_down": ["routed_moe_swiglu_b200/csrc/gemm_bf16.cu", "routed_moe_swiglu_b200/csrc/ptx.cuh",
+    "gemm_down": ["routed_moe_swiglu_b200/csrc/gemm_bf16_pair.cu", "routed_moe_swiglu_b200/csrc/ptx.cuh",
                   "routed_moe_swiglu_b200/csrc/moe_internal.cuh"],
     "combine": ["routed_moe_swiglu_b200/csrc/permute.cu", "routed_moe_swiglu_b200/csrc/moe_internal.cuh"],
 }
@@ -316,6 +316,29 @@ def run_ours(a, dist: Dist):
         "status": status,
         "max_rows_per_expert": max(counts),
     }
+
+    # ---------------- live-count sweep: the same one-step graph, device live counts
+    if len(w.live) > 1 and a.live is None:
+        sweep = []
+        reps = max(3, min(20, K))
+        for n in w.live:
+            live_d.fill_(n)
+            with torch.cuda.stream(stream):
+                g1.replay()
+            stream.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(reps):
+                    g1.replay()
+                e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            sweep.append({"live": n, "ms_per_step": ms, "tokens_per_s": n / (ms / 1e3)})
+        live_d.fill_(live)
+        torch.cuda.synchronize()
+        res["sweep"] = sweep
 
     # ---------------- end to end through the C ABI with pinned host buffers
     if not a.no_e2e:
@@ -535,6 +558,8 @@ def main():
     }
     if "e2e" in res:
         line["e2e"] = res["e2e"]
+    if "sweep" in res:
+        line["sweep"] = res["sweep"]
     if dist.rank == 0 and dist.world == 1 and not a.no_cpu_baseline:
         x, logits = workloads.make_activations(w)
         weights = workloads.make_weights(w)

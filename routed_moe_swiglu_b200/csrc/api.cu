@@ -159,8 +159,9 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     p->max_live = d.max_live_rows > 0 ? d.max_live_rows : d.capacity;
     p->d.max_live_rows = p->max_live;
     p->max_routes = p->max_live * d.top_k;
-    p->max_m_tiles = (p->max_routes + kBM - 1) / kBM + d.num_experts;
-    p->rows_pad = p->max_m_tiles * kBM;
+    p->tile_rows = d.precision == MOE_MXFP8 ? kBM : 2 * kBM;
+    p->max_m_tiles = (p->max_routes + p->tile_rows - 1) / p->tile_rows + d.num_experts;
+    p->rows_pad = p->max_m_tiles * p->tile_rows;
     p->nblk = (int)((p->max_live + kTokPerBlk - 1) / kTokPerBlk);
     if (d.precision == MOE_MXFP8) {
         p->ks1 = (d.hidden + kBK8 - 1) / kBK8;
@@ -244,11 +245,15 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
         return MOE_ERR_ALIGNMENT;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // Under stream capture the events are recorded as "external" so that the
+    // graph gets real event-record nodes; outside capture a plain record.
+    cudaStreamCaptureStatus capturing = cudaStreamCaptureStatusNone;
+    if (stage_events != nullptr && cudaStreamIsCapturing(s, &capturing) != cudaSuccess) return MOE_ERR_CUDA;
+    const unsigned record_flags =
+        capturing == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
     auto mark = [&](int i) -> bool {
-        // "external" so that, under stream capture, the graph gets a real event-record node
         return stage_events == nullptr ||
-               cudaEventRecordWithFlags(static_cast<cudaEvent_t>(stage_events[i]), s, cudaEventRecordExternal) ==
-                   cudaSuccess;
+               cudaEventRecordWithFlags(static_cast<cudaEvent_t>(stage_events[i]), s, record_flags) == cudaSuccess;
     };
     const int H = plan->d.hidden, F = plan->d.ffn, E = plan->d.num_experts, k = plan->d.top_k;
     const int max_live = (int)plan->max_live;
@@ -267,12 +272,13 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const unsigned bk = fp8 ? (unsigned)kBK8 : (unsigned)kBK;  // 128-byte rows either way
     const unsigned g1_rows = fp8 ? (unsigned)kG1BN8 : (unsigned)kG1BN;
-    const unsigned g2_rows = fp8 ? (unsigned)kG2BN8 : (unsigned)kG2BN;
-    CUtensorMap tA1, tB1, tA2, tB2, tY;
+    const unsigned g2_rows = fp8 ? (unsigned)kG2BN8 : (unsigned)(kG2BN / 2);  // bf16: one CTA's half of N
+    CUtensorMap tA1, tB1, tA2, tB2, tY, tA1f, tA2f;  // tA*f: A with full 128-row boxes
     {
         const unsigned long long dA[2] = {uH, R};
         const unsigned long long sA[1] = {uH * eb};
         const unsigned bA[2] = {bk, 32};
+        const unsigned bAf[2] = {bk, 128};
         const unsigned long long dB[4] = {uH, uF, 2ull, uE};
         const unsigned long long sB[3] = {uH * eb, uF * uH * eb, 2ull * uF * uH * eb};
         const unsigned bB[4] = {bk, g1_rows, 1, 1};
@@ -289,7 +295,9 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
             !make_tensor_map(&tA2, dt, 2, ws + L.h, dA2, sA2, bA, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_tensor_map(&tB2, dt, 3, wb + plan->wb.w2, dB2, sB2, bB2, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_tensor_map(&tY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ws + L.y, dY, sY, bY,
-                             CU_TENSOR_MAP_SWIZZLE_128B))
+                             CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tA1f, dt, 2, ws + L.xq, dA, sA, bAf, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tA2f, dt, 2, ws + L.h, dA2, sA2, bAf, CU_TENSOR_MAP_SWIZZLE_128B))
             return MOE_ERR_CUDA;
     }
 
@@ -339,7 +347,8 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     long long grid1 = m_tiles * g1.n_tiles;
     if (grid1 > sms) grid1 = sms;
     if (!mark(3)) return MOE_ERR_CUDA;
-    e = fp8 ? launch_gemm1_mxfp8(tA1, tB1, tY, g1, (int)grid1, s) : launch_gemm1_bf16(tA1, tB1, tY, g1, (int)grid1, s);
+    e = fp8 ? launch_gemm1_mxfp8(tA1, tB1, tY, g1, (int)grid1, s)
+            : launch_gemm1_bf16_pair(tA1, tA1f, tB1, tY, g1, m_tiles * g1.n_tiles, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 
     GemmParams g2 = g1;
@@ -354,7 +363,8 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     long long grid2 = m_tiles * g2.n_tiles;
     if (grid2 > sms) grid2 = sms;
     if (!mark(4)) return MOE_ERR_CUDA;
-    e = fp8 ? launch_gemm2_mxfp8(tA2, tB2, tY, g2, (int)grid2, s) : launch_gemm2_bf16(tA2, tB2, tY, g2, (int)grid2, s);
+    e = fp8 ? launch_gemm2_mxfp8(tA2, tB2, tY, g2, (int)grid2, s)
+            : launch_gemm2_bf16_pair(tA2, tA2f, tB2, tY, g2, m_tiles * g2.n_tiles, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     if (!mark(5)) return MOE_ERR_CUDA;
 

@@ -50,10 +50,11 @@ struct moe_plan {
     moe_desc d;
     long long max_live;
     long long max_routes;   // max_live * k
-    long long max_m_tiles;  // upper bound on M tiles: ceil(routes / BM) + E
-    long long rows_pad;     // max_m_tiles * BM: rows of the padded intermediates
+    long long max_m_tiles;  // upper bound on M tiles: ceil(routes / tile_rows) + E
+    long long rows_pad;     // max_m_tiles * tile_rows: rows of the padded intermediates
     int nblk;               // ceil(max_live / kTokPerBlk)
-    int ks1, ks2;           // MXFP8 K stages (128 elements) of the gate/up and down GEMMs
+    int tile_rows;          // rows of an M tile: 256 (bf16, CTA pairs) or 128 (MXFP8)
+    int ks1, ks2;           // K stages of the gate/up and down GEMMs
     int nt1, nt2;           // N tiles of the gate/up and down GEMMs
     moe::WsLayout ws;
     moe::WbufLayout wb;
@@ -62,7 +63,7 @@ struct moe_plan {
 namespace moe {
 
 struct GemmParams {
-    const int4* tiles;              // {expert, first padded row, valid rows, 0} per M tile
+    const int4* tiles;              // {expert, first padded row, valid rows, 0} per M tile (tile_rows rows)
     const unsigned* status_words;   // [kStNumMTiles] = number of M tiles
     unsigned* status_flags;         // sticky MOE_DEV_* bits
     void* out;                      // h (bf16 / E4M3) or y (fp32)
@@ -104,6 +105,10 @@ cudaError_t launch_gemm1_bf16(const CUtensorMap& a, const CUtensorMap& b, const 
                               int grid, cudaStream_t s);
 cudaError_t launch_gemm2_bf16(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& gp,
                               int grid, cudaStream_t s);
+cudaError_t launch_gemm1_bf16_pair(const CUtensorMap& a, const CUtensorMap& a128, const CUtensorMap& b,
+                                   const CUtensorMap& o, const GemmParams& gp, long long max_tiles, cudaStream_t s);
+cudaError_t launch_gemm2_bf16_pair(const CUtensorMap& a, const CUtensorMap& a128, const CUtensorMap& b,
+                                   const CUtensorMap& o, const GemmParams& gp, long long max_tiles, cudaStream_t s);
 cudaError_t launch_gemm1_mxfp8(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o,
                                const GemmParams& gp, int grid, cudaStream_t s);
 cudaError_t launch_gemm2_mxfp8(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o,

@@ -320,3 +320,22 @@ def test_graph_capture_replay_with_device_live_counts():
     _, _, ref = oracle_forward(x, logits, weights, k, 1024, tokens=toks)
     assert_close(res[1024].numpy()[toks], ref, "bf16", "graph replay")
     del g
+
+
+def test_stage_events_eager_and_same_result():
+    """moe_forward_with_events works outside graph capture, records ordered
+    events and gives the same bits as moe_forward."""
+    H, F, E, k, T = 256, 256, 8, 2, 50
+    x, logits, weights = workloads.small_case(H, F, E, k, T, seed=21)
+    m = GpuMoe(H, F, E, k, T, weights)
+    a = m.forward(x.cuda(), T, logits=logits.cuda()).cpu()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(rm.MOE_NUM_STAGES + 1)]
+    for e in evs:
+        e.record()
+    out = torch.full((T, H), float("nan"), device="cuda")
+    m.live.fill_(T)
+    rm.moe_forward_with_events(m.plan, x.cuda(), m.wbuf, m.live, out, m.ws, evs, logits=logits.cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(out.cpu(), a)
+    times = [evs[i].elapsed_time(evs[i + 1]) for i in range(rm.MOE_NUM_STAGES)]
+    assert all(t >= 0.0 for t in times)
