@@ -93,9 +93,9 @@ static void compute_layouts(moe_plan* p) {
         w.h = take(R * F);
         w.hs = take(mtiles * p->ks2 * kSfBlock);
     } else {
-        w.xq = take(R * H * 2);
+        w.xq = take(R * (size_t)p->hp * 2);
         w.xs = 0;
-        w.h = take(R * F * 2);
+        w.h = take(R * (size_t)p->fp * 2);
         w.hs = 0;
     }
     w.y = take(R * H * 4);
@@ -109,9 +109,9 @@ static void compute_layouts(moe_plan* p) {
         b.w2 = take(E * H * F);
         b.w2s = take(E * p->nt2 * p->ks2 * kSfBlock);
     } else {
-        b.w1 = take(E * 2 * F * H * 2);
+        b.w1 = take(E * 2 * F * (size_t)p->hp * 2);
         b.w1s = 0;
-        b.w2 = take(E * H * F * 2);
+        b.w2 = take(E * H * (size_t)p->fp * 2);
         b.w2s = 0;
     }
     b.total = off;
@@ -169,11 +169,13 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
         p->nt1 = (d.ffn + kG1BN8 - 1) / kG1BN8;
         p->nt2 = (d.hidden + kG2BN8 - 1) / kG2BN8;
     } else {
-        p->ks1 = (d.hidden + kBK - 1) / kBK;
-        p->ks2 = (d.ffn + kBK - 1) / kBK;
+        p->ks1 = (d.hidden + 2 * kBK - 1) / (2 * kBK);  // K stages of 128 elements
+        p->ks2 = (d.ffn + 2 * kBK - 1) / (2 * kBK);
         p->nt1 = (d.ffn + kG1BN - 1) / kG1BN;
         p->nt2 = (d.hidden + kG2BN - 1) / kG2BN;
     }
+    p->hp = d.precision == MOE_MXFP8 ? d.hidden : (long long)p->ks1 * 2 * kBK;
+    p->fp = d.precision == MOE_MXFP8 ? d.ffn : (long long)p->ks2 * 2 * kBK;
     compute_layouts(p);
     *plan_out = p;
     return MOE_OK;
@@ -268,25 +270,23 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     const bool fp8 = plan->d.precision == MOE_MXFP8;
     const unsigned long long R = (unsigned long long)plan->rows_pad;
     const unsigned long long uH = (unsigned long long)H, uF = (unsigned long long)F, uE = (unsigned long long)E;
-    const unsigned long long eb = fp8 ? 1ull : 2ull;  // bytes per operand element
     const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    const unsigned bk = fp8 ? (unsigned)kBK8 : (unsigned)kBK;  // 128-byte rows either way
-    const unsigned g1_rows = fp8 ? (unsigned)kG1BN8 : (unsigned)kG1BN;
-    const unsigned g2_rows = fp8 ? (unsigned)kG2BN8 : (unsigned)(kG2BN / 2);  // bf16: one CTA's half of N
-    CUtensorMap tA1, tB1, tA2, tB2, tY, tA1f, tA2f;  // tA*f: A with full 128-row boxes
-    {
+    CUtensorMap tA1, tB1, tA2, tB2, tY, tA1f, tA2f;
+    if (fp8) {
+        // MXFP8 (one CTA per tile): 2-D A maps with 32-row boxes, B in 64/128-row boxes,
+        // K stage = 128 E4M3 elements (one 128-byte swizzle atom)
+        const unsigned bk = (unsigned)kBK8;
         const unsigned long long dA[2] = {uH, R};
-        const unsigned long long sA[1] = {uH * eb};
+        const unsigned long long sA[1] = {uH};
         const unsigned bA[2] = {bk, 32};
-        const unsigned bAf[2] = {bk, 128};
         const unsigned long long dB[4] = {uH, uF, 2ull, uE};
-        const unsigned long long sB[3] = {uH * eb, uF * uH * eb, 2ull * uF * uH * eb};
-        const unsigned bB[4] = {bk, g1_rows, 1, 1};
+        const unsigned long long sB[3] = {uH, uF * uH, 2ull * uF * uH};
+        const unsigned bB[4] = {bk, (unsigned)kG1BN8, 1, 1};
         const unsigned long long dA2[2] = {uF, R};
-        const unsigned long long sA2[1] = {uF * eb};
+        const unsigned long long sA2[1] = {uF};
         const unsigned long long dB2[3] = {uF, uH, uE};
-        const unsigned long long sB2[2] = {uF * eb, uH * uF * eb};
-        const unsigned bB2[3] = {bk, g2_rows, 1};
+        const unsigned long long sB2[2] = {uF, uH * uF};
+        const unsigned bB2[3] = {bk, (unsigned)kG2BN8, 1};
         const unsigned long long dY[2] = {uH, R};
         const unsigned long long sY[1] = {uH * 4};
         const unsigned bY[2] = {32, 32};
@@ -295,10 +295,34 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
             !make_tensor_map(&tA2, dt, 2, ws + L.h, dA2, sA2, bA, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_tensor_map(&tB2, dt, 3, wb + plan->wb.w2, dB2, sB2, bB2, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_tensor_map(&tY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ws + L.y, dY, sY, bY,
-                             CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tA1f, dt, 2, ws + L.xq, dA, sA, bAf, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tA2f, dt, 2, ws + L.h, dA2, sA2, bAf, CU_TENSOR_MAP_SWIZZLE_128B))
+                             CU_TENSOR_MAP_SWIZZLE_128B))
             return MOE_ERR_CUDA;
+    } else {
+        // bf16 (CTA pairs): K stage = 128 elements = two 64-element swizzle atoms.  Every
+        // operand buffer has its K pitch padded to 128 (hp, fp) with zeros, and the maps
+        // address an element k of a row as (k % 64, row, k / 64, ...): the box's third
+        // dimension walks the two atoms, so a box lands as [atom][row][64 elements].
+        const unsigned long long hp = (unsigned long long)plan->hp, fpp = (unsigned long long)plan->fp;
+        const unsigned long long dA[3] = {64ull, R, hp / 64};
+        const unsigned long long sA[2] = {hp * 2, 128ull};
+        const unsigned bA32[3] = {64, 32, 1};   // 32 rows of one atom (sparse tiles)
+        const unsigned bAf[3] = {64, 128, 2};   // 128 rows x both atoms (full tiles)
+        const unsigned long long dA2[3] = {64ull, R, fpp / 64};
+        const unsigned long long sA2[2] = {fpp * 2, 128ull};
+        const unsigned long long dB[5] = {64ull, uF, hp / 64, 2ull, uE};
+        const unsigned long long sB[4] = {hp * 2, 128ull, uF * hp * 2, 2ull * uF * hp * 2};
+        const unsigned bB[5] = {64, 128, 2, 1, 1};
+        const unsigned long long dB2[4] = {64ull, uH, fpp / 64, uE};
+        const unsigned long long sB2[3] = {fpp * 2, 128ull, uH * fpp * 2};
+        const unsigned bB2[4] = {64, 128, 2, 1};
+        if (!make_tensor_map(&tA1, dt, 3, ws + L.xq, dA, sA, bA32, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tA1f, dt, 3, ws + L.xq, dA, sA, bAf, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tA2, dt, 3, ws + L.h, dA2, sA2, bA32, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tA2f, dt, 3, ws + L.h, dA2, sA2, bAf, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tB1, dt, 5, wb + plan->wb.w1, dB, sB, bB, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tB2, dt, 4, wb + plan->wb.w2, dB2, sB2, bB2, CU_TENSOR_MAP_SWIZZLE_128B))
+            return MOE_ERR_CUDA;
+        tY = tB2;  // unused by the pair kernels (y leaves through the LSU)
     }
 
     cudaError_t e;
@@ -323,7 +347,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
         e = launch_gather_mxfp8(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, k, inv, ws + L.xq,
                                 ws + L.xs, s);
     else
-        e = launch_gather_bf16(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, k, inv,
+        e = launch_gather_bf16(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, (int)plan->hp, k, inv,
                                reinterpret_cast<__nv_bfloat16*>(ws + L.xq), s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -334,7 +358,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g1.status_flags = status + kStFlags;
     g1.out = ws + L.h;
     g1.out_scales = nullptr;
-    g1.out_ld = F;
+    g1.out_ld = plan->fp;  // h rows: F values + zero padding to the down GEMM's K pitch
     g1.out_cols = F;
     g1.n_tiles = plan->nt1;
     g1.k_blocks = plan->ks1;

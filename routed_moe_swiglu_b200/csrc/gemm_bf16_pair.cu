@@ -12,12 +12,15 @@
 //   down:     A = h rows, B rows = W_down[e, c0:c0+256] (128 per CTA), fp32 y
 //             rows out through a shared-memory transpose and coalesced stores.
 //
-// Per SM and K stage each CTA loads 16 KB of A and 16 KB of B (instead of
-// 16 + 32 KB for a one-CTA 128x256 tile), so the pipeline can be deeper.
-// A CTA whose 128 rows are all valid loads its A stage with one 128-row TMA
-// box; a sparser one (decode: a few routes per expert) loads only the 32-row
-// boxes that hold valid rows.  Issuing a TMA instruction costs the producer
-// thread ~100+ cycles, so full tiles must not use four boxes where one does.
+// Each CTA loads half of B (the other half feeds the same MMA from the peer),
+// so per SM and MMA FLOP the operand traffic is 2/3 of a one-CTA 128x256
+// tile.  Issuing a TMA copy costs the producer thread on the order of a
+// hundred cycles at these rates, so a K stage is 128 elements (two 128-byte
+// swizzle atoms, 8 MMAs) and each operand of a stage is one 32 KB box: a
+// 3-D (A) or 4-/5-D (B) tensor map whose third dimension walks the atoms of
+// a row (the K row pitch of every bf16 operand buffer is padded to 128 with
+// zeros).  A CTA with fewer than 128 valid rows (decode: a few routes per
+// expert) loads only the 32-row boxes that hold valid rows.
 //
 // Roles (10 warps per CTA): warp 0 issues TMA loads in both CTAs (the
 // completion of both halves is counted on CTA 0's "full" barrier); warp 1
@@ -40,15 +43,18 @@ namespace {
 // Pipeline depth per mode: the gate/up epilogue stores h straight from
 // registers, so its shared memory all goes to stages; the down epilogue keeps
 // one 4 KB transpose box per epilogue warp.
-constexpr int kStagesGateUp = 7;
-constexpr int kStagesDown = 6;
+constexpr int kStagesGateUp = 3;
+constexpr int kStagesDown = 3;
 constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
 constexpr int kPairRows = 256;                          // M of the pair tile
+constexpr int kAtoms = 2;                               // 64-element (128-byte) swizzle atoms per K stage
+constexpr int kStageK = kAtoms * kBK;                   // 128 K elements per stage
+constexpr uint32_t kAtomBytes = 128 * kBK * 2;          // 16 KB: 128 rows x 128 bytes
 constexpr int kABoxRows = 32;
-constexpr uint32_t kABytes = 128 * kBK * 2;             // 16 KB: this CTA's 128 rows
-constexpr uint32_t kABoxBytes = kABoxRows * kBK * 2;    // 4 KB
-constexpr uint32_t kBBytes = 128 * kBK * 2;             // 16 KB: this CTA's half of N = 256
+constexpr uint32_t kABytes = kAtoms * kAtomBytes;       // 32 KB: this CTA's 128 rows
+constexpr uint32_t kABoxBytes = kABoxRows * kBK * 2;    // 4 KB: 32 rows of one atom
+constexpr uint32_t kBBytes = kAtoms * kAtomBytes;       // 32 KB: this CTA's half of N = 256
 constexpr uint32_t kAccCols = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kStageOutBytes = 32 * 128;
@@ -148,7 +154,7 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
                 const int box0 = (rows_of(ti.z, 0) + kABoxRows - 1) / kABoxRows;
                 const int box1 = (rows_of(ti.z, 1) + kABoxRows - 1) / kABoxRows;
                 const int my_boxes = leader ? box0 : box1;
-                const uint32_t tx = (uint32_t)(box0 + box1) * kABoxBytes + 2 * kBBytes;
+                const uint32_t tx = (uint32_t)(box0 + box1) * kAtoms * kABoxBytes + 2 * kBBytes;
                 const int my_row0 = ti.y + 128 * (int)rank;
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!mbar_wait_bounded(&bars->empty[stage], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
@@ -160,17 +166,20 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
                         last_phase[stage] = (int)phase;
                     }
                     const uint32_t full0 = map_to_cta(smem_u32(&bars->full[stage]), 0);
+                    // operands as [atom][row][64 elements]; a box spans both atoms of the stage
                     uint8_t* a_dst = sA + stage * kABytes;
-                    if (my_boxes == 128 / kABoxRows)  // full tile: one TMA instruction
-                        tma_load_2d_pair(a_dst, &tmA128, full0, kb * kBK, my_row0);
+                    if (my_boxes == 128 / kABoxRows)  // full tile: one TMA instruction, 32 KB
+                        tma_load_3d_pair(a_dst, &tmA128, full0, 0, my_row0, kb * kAtoms);
                     else
-                        for (int i = 0; i < my_boxes; ++i)
-                            tma_load_2d_pair(a_dst + i * kABoxBytes, &tmA, full0, kb * kBK, my_row0 + i * kABoxRows);
+                        for (int a = 0; a < kAtoms; ++a)
+                            for (int i = 0; i < my_boxes; ++i)
+                                tma_load_3d_pair(a_dst + a * kAtomBytes + i * kABoxBytes, &tmA, full0, 0,
+                                                 my_row0 + i * kABoxRows, kb * kAtoms + a);
                     uint8_t* b_dst = sB + stage * kBBytes;
                     if (kMode == 0)  // CTA 0: gate rows, CTA 1: up rows of the same 128 f
-                        tma_load_4d_pair(b_dst, &tmB, full0, kb * kBK, nt * kG1BN, (int)rank, ti.x);
+                        tma_load_5d_pair(b_dst, &tmB, full0, 0, nt * kG1BN, kb * kAtoms, (int)rank, ti.x);
                     else
-                        tma_load_3d_pair(b_dst, &tmB, full0, kb * kBK, nt * kG2BN + 128 * (int)rank, ti.x);
+                        tma_load_4d_pair(b_dst, &tmB, full0, 0, nt * kG2BN + 128 * (int)rank, kb * kAtoms, ti.x);
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -216,9 +225,11 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
                     const uint32_t a_addr = smem_u32(sA + stage * kABytes);
                     const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-                        mma_bf16_pair(d_tmem, sdesc_kmajor_sw128(a_addr + kk * 32), sdesc_kmajor_sw128(b_addr + kk * 32),
-                                      idesc, (kb | kk) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < kStageK / 16; ++kk) {
+                        const uint32_t off = (uint32_t)(kk >> 2) * kAtomBytes + (uint32_t)(kk & 3) * 32;
+                        mma_bf16_pair(d_tmem, sdesc_kmajor_sw128(a_addr + off), sdesc_kmajor_sw128(b_addr + off), idesc,
+                                      (kb | kk) != 0 ? 1u : 0u);
+                    }
                     mma_commit_pair_multicast(&bars->empty[stage], 0x3);  // both CTAs may refill the stage
                     if (++stage == kStages) {
                         stage = 0;
@@ -280,7 +291,7 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
                     if (valid) {
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            if (f0 + q * 8 < p.out_cols) {
+                            {  // f >= F are zero-weight rows: h = 0, which pads h's K pitch to 128
                                 uint32_t w[4];
 #pragma unroll
                                 for (int i = 0; i < 4; ++i) {

@@ -54,6 +54,8 @@ struct moe_plan {
     long long rows_pad;     // max_m_tiles * tile_rows: rows of the padded intermediates
     int nblk;               // ceil(max_live / kTokPerBlk)
     int tile_rows;          // rows of an M tile: 256 (bf16, CTA pairs) or 128 (MXFP8)
+    long long hp, fp;       // K row pitch (elements) of x / gate-up rows and of h / down rows:
+                            // bf16 pads H and F to multiples of 128 with zeros; MXFP8 keeps H, F
     int ks1, ks2;           // K stages of the gate/up and down GEMMs
     int nt1, nt2;           // N tiles of the gate/up and down GEMMs
     moe::WsLayout ws;
@@ -95,7 +97,7 @@ cudaError_t launch_canon_routes(const int* ids_in, const float* probs_in, const 
 cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* blkcnt, int* offsets,
                            int* padoff, int4* tiles, int* perm, int* inv, unsigned* status_words,
                            cudaStream_t s);
-cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_live, int H, int k,
+cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
                                const int* inv, __nv_bfloat16* xp, cudaStream_t s);
 cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int k,
                                 const int* inv, uint8_t* xq, uint8_t* xs, cudaStream_t s);

@@ -164,22 +164,24 @@ constexpr int kRowThreads = 128;
 
 __global__ void __launch_bounds__(kRowThreads) gather_rows_bf16_kernel(const uint4* __restrict__ x,
                                                                        const int* __restrict__ live, int max_live,
-                                                                       int H, int k, const int* __restrict__ inv,
+                                                                       int H, int hp, int k,
+                                                                       const int* __restrict__ inv,
                                                                        uint4* __restrict__ xp) {
     __shared__ int s_prow[kMaxTopK];
     const int n = clamp_live(live, max_live);
-    const int chunks = H / 8;  // 8 bf16 per 16 bytes
+    const int chunks = H / 8;       // 8 bf16 per 16 bytes
+    const int chunks_out = hp / 8;  // destination rows are padded to hp with zeros
     for (int t = blockIdx.x; t < n; t += gridDim.x) {
         __syncthreads();
         if (threadIdx.x < k) s_prow[threadIdx.x] = __ldg(inv + (size_t)t * k + threadIdx.x);
         __syncthreads();
         const uint4* src = x + (size_t)t * chunks;
 #pragma unroll 4
-        for (int c = threadIdx.x; c < chunks; c += kRowThreads) {
-            const uint4 v = __ldg(src + c);
+        for (int c = threadIdx.x; c < chunks_out; c += kRowThreads) {
+            const uint4 v = c < chunks ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
             for (int j = 0; j < k; ++j) {
                 const int pr = s_prow[j];
-                if (pr >= 0) xp[(size_t)pr * chunks + c] = v;
+                if (pr >= 0) xp[(size_t)pr * chunks_out + c] = v;
             }
         }
     }
@@ -319,11 +321,11 @@ cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* 
     return cudaGetLastError();
 }
 
-cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_live, int H, int k,
+cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
                                const int* inv, __nv_bfloat16* xp, cudaStream_t s) {
     const int grid = grid_for_warps(max_live, 1, 16);
-    gather_rows_bf16_kernel<<<grid, kRowThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), live, max_live, H, k, inv,
-                                                 reinterpret_cast<uint4*>(xp));
+    gather_rows_bf16_kernel<<<grid, kRowThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), live, max_live, H, hp, k,
+                                                         inv, reinterpret_cast<uint4*>(xp));
     return cudaGetLastError();
 }
 

@@ -3,8 +3,9 @@
 // refresh_mega_weights(), which rewrites the kernel's own copy of the
 // weights; no allocation, no teardown).
 //
-// bf16 layout:  W1 [E][2][F][H]  (gate rows, then up rows of each expert),
-//               W2 [E][H][F]     (down projection).
+// bf16 layout:  W1 [E][2][F][hp]  (gate rows, then up rows of each expert),
+//               W2 [E][H][fp]     (down projection),
+// with the K pitches hp, fp = H, F rounded up to 128 and the padding zero.
 // A gate/up tile loads the same 128 f rows from W1[e][0] and W1[e][1] into
 // one 256-row B operand, so gate and up of one f meet in one accumulator row.
 #include "moe_internal.cuh"
@@ -15,18 +16,27 @@ namespace {
 
 __global__ void __launch_bounds__(256) prepare_bf16_kernel(const uint4* __restrict__ wg, const uint4* __restrict__ wu,
                                                            const uint4* __restrict__ wd, uint4* __restrict__ w1,
-                                                           uint4* __restrict__ w2, long long fh_chunks,
-                                                           long long hf_chunks, int E) {
-    const long long n1 = (long long)E * 2 * fh_chunks;
-    const long long n2 = (long long)E * hf_chunks;
+                                                           uint4* __restrict__ w2, int E, int F, int H, int hp, int fp) {
+    // 16-byte chunks of the destination; rows are padded with zeros to hp / fp
+    const long long c1 = hp / 8, c2 = fp / 8;
+    const long long n1 = (long long)E * 2 * F * c1;
+    const long long n2 = (long long)E * H * c2;
     const long long stride = (long long)gridDim.x * blockDim.x;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n1 + n2; i += stride) {
         if (i < n1) {
-            const long long e = i / (2 * fh_chunks);
-            const long long r = i - e * 2 * fh_chunks;
-            w1[i] = r < fh_chunks ? __ldg(wg + e * fh_chunks + r) : __ldg(wu + e * fh_chunks + (r - fh_chunks));
+            const long long row = i / c1;  // (e * 2 + g) * F + f
+            const int c = (int)(i - row * c1);
+            const long long e = row / (2 * F);
+            const int g = (int)((row / F) & 1);
+            const long long f = row - (e * 2 + g) * F;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (c * 8 < H) v = __ldg((g ? wu : wg) + (e * F + f) * (H / 8) + c);
+            w1[i] = v;
         } else {
-            w2[i - n1] = __ldg(wd + (i - n1));
+            const long long j = i - n1;
+            const long long row = j / c2;  // e * H + h
+            const int c = (int)(j - row * c2);
+            w2[j] = c * 8 < F ? __ldg(wd + row * (F / 8) + c) : make_uint4(0u, 0u, 0u, 0u);
         }
     }
 }
@@ -39,8 +49,8 @@ cudaError_t launch_prepare_bf16(const moe_plan* p, const __nv_bfloat16* wg, cons
     uint8_t* base = static_cast<uint8_t*>(buf);
     prepare_bf16_kernel<<<num_sms() * 8, 256, 0, s>>>(
         reinterpret_cast<const uint4*>(wg), reinterpret_cast<const uint4*>(wu), reinterpret_cast<const uint4*>(wd),
-        reinterpret_cast<uint4*>(base + p->wb.w1), reinterpret_cast<uint4*>(base + p->wb.w2), F * H / 8, H * F / 8,
-        (int)E);
+        reinterpret_cast<uint4*>(base + p->wb.w1), reinterpret_cast<uint4*>(base + p->wb.w2), (int)E, (int)F, (int)H,
+        (int)p->hp, (int)p->fp);
     return cudaGetLastError();
 }
 
