@@ -212,10 +212,12 @@ moe_status moe_forward_with_events(const moe_plan* plan, const void* x, const fl
  *   offsets int32 [E+1]: first row of each expert in the permuted order
  *   perm    int32 [routes]: permuted row r holds route t*k + j
  *   inv     int32 [max_live, k]: padded intermediate row of route (t, j)
- *   pad_offsets int32 [E+1]: first padded intermediate row of each expert
- *   h       intermediate rows (bf16 [rows_padded, F], or E4M3 codes
- *           [rows_padded, F] in MXFP8)
- *   xq      permuted x rows (bf16 [rows_padded, H], or E4M3 codes)
+ *   pad_offsets int32 [E+1]: first padded intermediate row of each expert,
+ *           a multiple of 32 (bf16) or 128 (MXFP8)
+ *   h       intermediate rows (bf16 [rows_padded, ceil(F/128)*128], the
+ *           columns past F zero; or E4M3 codes [rows_padded, F] in MXFP8)
+ *   xq      permuted x rows (bf16 [rows_padded, ceil(H/128)*128], the
+ *           columns past H zero; or E4M3 codes [rows_padded, H])
  *   h_scales, xq_scales  MXFP8 only (else NULL): E8M0 bytes in blocks of
  *           512 bytes, one per (128-row tile, K stage of 128 elements),
  *           block index tile * ceil(K/128) + stage; inside a block the byte

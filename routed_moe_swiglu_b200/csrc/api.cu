@@ -109,7 +109,7 @@ static void compute_layouts(moe_plan* p) {
         b.w2 = take(E * H * F);
         b.w2s = take(E * p->nt2 * p->ks2 * kSfBlock);
     } else {
-        b.w1 = take(E * 2 * F * (size_t)p->hp * 2);
+        b.w1 = take(E * 2 * (size_t)p->fp * (size_t)p->hp * 2);
         b.w1s = 0;
         b.w2 = take(E * H * (size_t)p->fp * 2);
         b.w2s = 0;
@@ -159,9 +159,12 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     p->max_live = d.max_live_rows > 0 ? d.max_live_rows : d.capacity;
     p->d.max_live_rows = p->max_live;
     p->max_routes = p->max_live * d.top_k;
-    p->tile_rows = d.precision == MOE_MXFP8 ? kBM : 2 * kBM;
+    p->tile_rows = d.precision == MOE_MXFP8 ? kBM : kRouteTile;
+    p->row_align = d.precision == MOE_MXFP8 ? kBM : kRouteAlign;
     p->max_m_tiles = (p->max_routes + p->tile_rows - 1) / p->tile_rows + d.num_experts;
-    p->rows_pad = p->max_m_tiles * p->tile_rows;
+    // every expert's rows are padded to row_align: at most routes + E * row_align rows
+    p->rows_pad = d.precision == MOE_MXFP8 ? p->max_m_tiles * p->tile_rows
+                                           : p->max_routes + (long long)d.num_experts * p->row_align;
     p->nblk = (int)((p->max_live + kTokPerBlk - 1) / kTokPerBlk);
     if (d.precision == MOE_MXFP8) {
         p->ks1 = (d.hidden + kBK8 - 1) / kBK8;
@@ -171,7 +174,7 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     } else {
         p->ks1 = (d.hidden + 2 * kBK - 1) / (2 * kBK);  // K stages of 128 elements
         p->ks2 = (d.ffn + 2 * kBK - 1) / (2 * kBK);
-        p->nt1 = (d.ffn + kG1BN - 1) / kG1BN;
+        p->nt1 = p->ks2;  // f tiles of 128 cover the padded F (fp); h's padding columns come out zero
         p->nt2 = (d.hidden + kG2BN - 1) / kG2BN;
     }
     p->hp = d.precision == MOE_MXFP8 ? d.hidden : (long long)p->ks1 * 2 * kBK;
@@ -271,7 +274,8 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     const unsigned long long R = (unsigned long long)plan->rows_pad;
     const unsigned long long uH = (unsigned long long)H, uF = (unsigned long long)F, uE = (unsigned long long)E;
     const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    CUtensorMap tA1, tB1, tA2, tB2, tY, tA1f, tA2f;
+    CUtensorMap tA1, tB1, tA2, tB2, tY;
+    BoxMaps8 rB1, rB2;  // bf16: route-row operands (x rows, h rows)
     if (fp8) {
         // MXFP8 (one CTA per tile): 2-D A maps with 32-row boxes, B in 64/128-row boxes,
         // K stage = 128 E4M3 elements (one 128-byte swizzle atom)
@@ -300,29 +304,26 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     } else {
         // bf16 (CTA pairs): K stage = 128 elements = two 64-element swizzle atoms.  Every
         // operand buffer has its K pitch padded to 128 (hp, fp) with zeros, and the maps
-        // address an element k of a row as (k % 64, row, k / 64, ...): the box's third
-        // dimension walks the two atoms, so a box lands as [atom][row][64 elements].
+        // address an element k of a row as (k % 64, row, k / 64): the box's third dimension
+        // walks the two atoms, so a box lands as [atom][row][64 elements].  Weights (A) load
+        // 128 rows per CTA; route rows (B) load N/2 rows, one map per N/2 in {16, ..., 128}.
         const unsigned long long hp = (unsigned long long)plan->hp, fpp = (unsigned long long)plan->fp;
-        const unsigned long long dA[3] = {64ull, R, hp / 64};
-        const unsigned long long sA[2] = {hp * 2, 128ull};
-        const unsigned bA32[3] = {64, 32, 1};   // 32 rows of one atom (sparse tiles)
-        const unsigned bAf[3] = {64, 128, 2};   // 128 rows x both atoms (full tiles)
-        const unsigned long long dA2[3] = {64ull, R, fpp / 64};
-        const unsigned long long sA2[2] = {fpp * 2, 128ull};
-        const unsigned long long dB[5] = {64ull, uF, hp / 64, 2ull, uE};
-        const unsigned long long sB[4] = {hp * 2, 128ull, uF * hp * 2, 2ull * uF * hp * 2};
-        const unsigned bB[5] = {64, 128, 2, 1, 1};
-        const unsigned long long dB2[4] = {64ull, uH, fpp / 64, uE};
-        const unsigned long long sB2[3] = {fpp * 2, 128ull, uH * fpp * 2};
-        const unsigned bB2[4] = {64, 128, 2, 1};
-        if (!make_tensor_map(&tA1, dt, 3, ws + L.xq, dA, sA, bA32, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tA1f, dt, 3, ws + L.xq, dA, sA, bAf, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tA2, dt, 3, ws + L.h, dA2, sA2, bA32, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tA2f, dt, 3, ws + L.h, dA2, sA2, bAf, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tB1, dt, 5, wb + plan->wb.w1, dB, sB, bB, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tB2, dt, 4, wb + plan->wb.w2, dB2, sB2, bB2, CU_TENSOR_MAP_SWIZZLE_128B))
+        const unsigned box128[3] = {64, 128, 2};
+        const unsigned long long dW1[3] = {64ull, uE * 2ull * fpp, hp / 64};
+        const unsigned long long sW1[2] = {hp * 2, 128ull};
+        const unsigned long long dW2[3] = {64ull, uE * uH, fpp / 64};
+        const unsigned long long sW2[2] = {fpp * 2, 128ull};
+        const unsigned long long dX[3] = {64ull, R, hp / 64};
+        const unsigned long long dH[3] = {64ull, R, fpp / 64};
+        if (!make_tensor_map(&tA1, dt, 3, wb + plan->wb.w1, dW1, sW1, box128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tA2, dt, 3, wb + plan->wb.w2, dW2, sW2, box128, CU_TENSOR_MAP_SWIZZLE_128B))
             return MOE_ERR_CUDA;
-        tY = tB2;  // unused by the pair kernels (y leaves through the LSU)
+        for (int i = 0; i < 8; ++i) {
+            const unsigned box[3] = {64, 16u * (unsigned)(i + 1), 2};
+            if (!make_tensor_map(&rB1.m[i], dt, 3, ws + L.xq, dX, sW1, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+                !make_tensor_map(&rB2.m[i], dt, 3, ws + L.h, dH, sW2, box, CU_TENSOR_MAP_SWIZZLE_128B))
+                return MOE_ERR_CUDA;
+        }
     }
 
     cudaError_t e;
@@ -359,7 +360,8 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g1.out = ws + L.h;
     g1.out_scales = nullptr;
     g1.out_ld = plan->fp;  // h rows: F values + zero padding to the down GEMM's K pitch
-    g1.out_cols = F;
+    g1.out_cols = fp8 ? F : (int)plan->fp;
+    g1.a_rows = 2 * plan->fp;  // bf16 W1: gate and up rows of an expert, padded F
     g1.n_tiles = plan->nt1;
     g1.k_blocks = plan->ks1;
     g1.wait_limit_ns = kWaitLimitNs;
@@ -372,7 +374,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     if (grid1 > sms) grid1 = sms;
     if (!mark(3)) return MOE_ERR_CUDA;
     e = fp8 ? launch_gemm1_mxfp8(tA1, tB1, tY, g1, (int)grid1, s)
-            : launch_gemm1_bf16_pair(tA1, tA1f, tB1, tY, g1, m_tiles * g1.n_tiles, s);
+            : launch_gemm1_bf16_pair(tA1, rB1, g1, m_tiles * g1.n_tiles, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 
     GemmParams g2 = g1;
@@ -381,6 +383,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g2.out_cols = H;
     g2.n_tiles = plan->nt2;
     g2.k_blocks = plan->ks2;
+    g2.a_rows = H;
     g2.sfa = ws + L.hs;
     g2.sfb = wb + plan->wb.w2s;
     g2.out_scales = nullptr;
@@ -388,7 +391,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     if (grid2 > sms) grid2 = sms;
     if (!mark(4)) return MOE_ERR_CUDA;
     e = fp8 ? launch_gemm2_mxfp8(tA2, tB2, tY, g2, (int)grid2, s)
-            : launch_gemm2_bf16_pair(tA2, tA2f, tB2, tY, g2, m_tiles * g2.n_tiles, s);
+            : launch_gemm2_bf16_pair(tA2, rB2, g2, m_tiles * g2.n_tiles, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     if (!mark(5)) return MOE_ERR_CUDA;
 

@@ -1,72 +1,72 @@
 // gemm_bf16_pair.cu -- the two grouped expert GEMMs in bf16, each tile
-// computed by a pair of CTAs on two SMs with one tcgen05 MMA (cta_group::2).
+// computed by a pair of CTAs on two SMs with one tcgen05 MMA (cta_group::2),
+// expert weights as the MMA's M operand and routes as its N operand.
 //
-//   gate/up:  M tile = 256 route rows of expert e (CTA r holds rows
-//             128r..128r+127), N = 256: B rows 0..127 = W_gate[e, f0:f0+128]
-//             in CTA 0's shared memory, rows 128..255 = W_up[e, f0:f0+128] in
-//             CTA 1's.  Each CTA's TMEM receives its 128 rows x 256 columns,
-//             so gate and up of one f sit in columns c and 128+c of the same
-//             row; the epilogue forms h = silu(g) * u and stores bf16
+// Why weights are M: a tile holds the routes of one expert, and experts get
+// very different numbers of routes (a Zipf-skewed router sends a few rows to
+// most experts).  M of a pair MMA is fixed at 256, N may be any multiple of
+// 16 up to 256; with routes along N the last tile of an expert costs its
+// route count rounded up to 32, not a full 256-row tile.
+//
+//   gate/up:  A = 128 f values of expert e as 256 weight rows, 64 f per CTA,
+//             B = N route rows of x.  The prepared W1 interleaves gate and up
+//             so that each 32-lane TMEM quarter q of CTA r holds 16 f: lane
+//             32q+i the gate value of f = f0 + 64r + 16q + i, lane 32q+16+i
+//             the up value of the same f.  The warp reading a quarter swaps
+//             half of its columns across the half-warps (shfl.xor 16), so
+//             every lane forms h = silu(g) * u for 16 routes of one f, bf16
 //             (Megatron-LM PR #7798, "Background": the activation is fused
 //             into the FC1 epilogue).
-//   down:     A = h rows, B rows = W_down[e, c0:c0+256] (128 per CTA), fp32 y
-//             rows out through a shared-memory transpose and coalesced stores.
+//   down:     A = 256 rows of W_down[e] (output columns c0..c0+255, 128 per
+//             CTA), B = N route rows of h; fp32 y out.
 //
-// Each CTA loads half of B (the other half feeds the same MMA from the peer),
-// so per SM and MMA FLOP the operand traffic is 2/3 of a one-CTA 128x256
-// tile.  Issuing a TMA copy costs the producer thread on the order of a
-// hundred cycles at these rates, so a K stage is 128 elements (two 128-byte
-// swizzle atoms, 8 MMAs) and each operand of a stage is one 32 KB box: a
-// 3-D (A) or 4-/5-D (B) tensor map whose third dimension walks the atoms of
-// a row (the K row pitch of every bf16 operand buffer is padded to 128 with
-// zeros).  A CTA with fewer than 128 valid rows (decode: a few routes per
-// expert) loads only the 32-row boxes that hold valid rows.
+// Both epilogues transpose through shared memory so that y and h rows leave
+// as coalesced 16-byte stores (one route row per store group).
+//
+// A K stage is 128 elements (two 128-byte swizzle atoms, 8 MMAs) and each
+// operand of a stage is one TMA instruction: A is a 128-row x 2-atom box, B a
+// (N/2)-row x 2-atom box, one tensor map per N/2 in {16, 32, ..., 128}.  The K
+// row pitch of every bf16 operand buffer is padded to 128 with zeros.
 //
 // Roles (10 warps per CTA): warp 0 issues TMA loads in both CTAs (the
 // completion of both halves is counted on CTA 0's "full" barrier); warp 1
 // owns TMEM in both CTAs and, in CTA 0 only, issues the pair MMAs, whose
 // completion is signalled to both CTAs' barriers (commit with a CTA mask);
-// warps 2-9 drain the accumulators (lane quarter warp % 4, column half
-// (warp - 2) / 4) and release each accumulator on CTA 0's barrier.
-// Two accumulators of 256 fp32 columns (512 TMEM columns) per CTA.
+// warps 2-9 drain the accumulators and release each accumulator on CTA 0's
+// barrier.  Two accumulators of 256 fp32 columns (512 TMEM columns) per CTA.
 //
-// Every wait is bounded; the pair meets in cluster barriers only at start-up
-// and before TMEM is released.  Each output row depends only on its own A row
-// with one instruction shape and K order, so results do not depend on the
-// tile a row lands in or on the live count.
+// Every mbarrier wait is bounded; the pair meets in cluster barriers only at
+// start-up and before TMEM is released.  Each output element is one route's
+// dot product over K in a fixed order with one instruction shape, so results
+// do not depend on the tile or column a route lands in or on the live count.
 #include "moe_internal.cuh"
 #include "ptx.cuh"
 
 namespace moe {
 namespace {
 
-// Pipeline depth per mode: the gate/up epilogue stores h straight from
-// registers, so its shared memory all goes to stages; the down epilogue keeps
-// one 4 KB transpose box per epilogue warp.
-constexpr int kStagesGateUp = 3;
-constexpr int kStagesDown = 3;
+constexpr int kStages = 3;
 constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
-constexpr int kPairRows = 256;                          // M of the pair tile
+constexpr int kPairM = 256;                             // M of the pair MMA (weight rows)
 constexpr int kAtoms = 2;                               // 64-element (128-byte) swizzle atoms per K stage
 constexpr int kStageK = kAtoms * kBK;                   // 128 K elements per stage
 constexpr uint32_t kAtomBytes = 128 * kBK * 2;          // 16 KB: 128 rows x 128 bytes
-constexpr int kABoxRows = 32;
-constexpr uint32_t kABytes = kAtoms * kAtomBytes;       // 32 KB: this CTA's 128 rows
-constexpr uint32_t kABoxBytes = kABoxRows * kBK * 2;    // 4 KB: 32 rows of one atom
-constexpr uint32_t kBBytes = kAtoms * kAtomBytes;       // 32 KB: this CTA's half of N = 256
+constexpr uint32_t kABytes = kAtoms * kAtomBytes;       // 32 KB: this CTA's 128 weight rows
+constexpr uint32_t kBBytes = kAtoms * kAtomBytes;       // up to 32 KB: this CTA's N/2 <= 128 route rows
 constexpr uint32_t kAccCols = 256;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kStageOutBytes = 32 * 128;
+constexpr uint32_t kHTBytes = 32 * 16 * 2 + 64;         // gate/up: h of 32 routes x 16 f, bf16 (+ bank offset)
+constexpr uint32_t kYTBytes = 32 * 32 * 4;              // down: y of 32 routes x 32 c, fp32
+
 template <int kMode>
 struct PairCfg {
-    static constexpr int kStages = kMode == 0 ? kStagesGateUp : kStagesDown;
-    static constexpr uint32_t kOutBytes = kMode == 0 ? 0u : kEpiWarps * kStageOutBytes;
-    static constexpr size_t kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kOutBytes + 256;
+    // one transpose box per epilogue warp
+    static constexpr uint32_t kEpiBytes = kEpiWarps * (kMode == 0 ? kHTBytes : kYTBytes);
+    static constexpr size_t kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kEpiBytes + 256;
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
-template <int kStages>
 struct __align__(8) Barriers {
     uint64_t full[kStages];   // CTA 0's counts both CTAs' loads of a stage
     uint64_t empty[kStages];  // each CTA's: its stage may be refilled
@@ -77,30 +77,20 @@ struct __align__(8) Barriers {
     int abort_flag;
 };
 
-__device__ __forceinline__ float silu_f(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&v);
-}
-
-__device__ __forceinline__ int rows_of(int nvalid, uint32_t rank) {
-    const int r = nvalid - 128 * (int)rank;
-    return r < 0 ? 0 : (r > 128 ? 128 : r);
-}
+// Routes of a tile rounded up to the MMA's N granularity (both CTAs hold N/2 rows of B).
+__device__ __forceinline__ int tile_n(int nvalid) { return (nvalid + 31) & ~31; }
 
 template <int kMode>  // 0: gate/up + SwiGLU -> bf16 h;  1: down -> fp32 y
-__device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmA128,
-                                               const CUtensorMap& tmB, const CUtensorMap& tmOut,
-                                               const GemmParams& p) {
-    constexpr int kStages = PairCfg<kMode>::kStages;
-    constexpr uint32_t kOutBytes = PairCfg<kMode>::kOutBytes;
+__device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const BoxMaps8& tmB, const GemmParams& p) {
+    constexpr uint32_t kEpiBytes = PairCfg<kMode>::kEpiBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStages * kABytes;
-    uint8_t* sOut = sB + kStages * kBBytes;
-    Barriers<kStages>* bars = reinterpret_cast<Barriers<kStages>*>(sOut + kOutBytes);
+    uint8_t* sEpi = sB + kStages * kBBytes;
+    Barriers* bars = reinterpret_cast<Barriers*>(sEpi + kEpiBytes);
     volatile int* abort_flag = &bars->abort_flag;
 
     const int warp = threadIdx.x >> 5;
@@ -141,8 +131,6 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
         if (lane == 0) {
             // ---------------- TMA producer (both CTAs)
             tma_prefetch_desc(&tmA);
-            tma_prefetch_desc(&tmA128);
-            tma_prefetch_desc(&tmB);
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -151,11 +139,11 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
             for (int t = pair; t < total_tiles && ok; t += npairs) {
                 const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
                 const int4 ti = __ldg(p.tiles + mt);
-                const int box0 = (rows_of(ti.z, 0) + kABoxRows - 1) / kABoxRows;
-                const int box1 = (rows_of(ti.z, 1) + kABoxRows - 1) / kABoxRows;
-                const int my_boxes = leader ? box0 : box1;
-                const uint32_t tx = (uint32_t)(box0 + box1) * kAtoms * kABoxBytes + 2 * kBBytes;
-                const int my_row0 = ti.y + 128 * (int)rank;
+                const int hb = tile_n(ti.z) >> 1;  // route rows of B in each CTA
+                const CUtensorMap* mapB = &tmB.m[(hb >> 4) - 1];
+                const uint32_t tx = 2u * (kABytes + (uint32_t)hb * (kAtoms * 128u));
+                const int a_row = (int)((long long)ti.x * p.a_rows) + nt * kPairM + 128 * (int)rank;
+                const int b_row = ti.y + hb * (int)rank;
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!mbar_wait_bounded(&bars->empty[stage], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
                         ok = false;
@@ -166,20 +154,9 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
                         last_phase[stage] = (int)phase;
                     }
                     const uint32_t full0 = map_to_cta(smem_u32(&bars->full[stage]), 0);
-                    // operands as [atom][row][64 elements]; a box spans both atoms of the stage
-                    uint8_t* a_dst = sA + stage * kABytes;
-                    if (my_boxes == 128 / kABoxRows)  // full tile: one TMA instruction, 32 KB
-                        tma_load_3d_pair(a_dst, &tmA128, full0, 0, my_row0, kb * kAtoms);
-                    else
-                        for (int a = 0; a < kAtoms; ++a)
-                            for (int i = 0; i < my_boxes; ++i)
-                                tma_load_3d_pair(a_dst + a * kAtomBytes + i * kABoxBytes, &tmA, full0, 0,
-                                                 my_row0 + i * kABoxRows, kb * kAtoms + a);
-                    uint8_t* b_dst = sB + stage * kBBytes;
-                    if (kMode == 0)  // CTA 0: gate rows, CTA 1: up rows of the same 128 f
-                        tma_load_5d_pair(b_dst, &tmB, full0, 0, nt * kG1BN, kb * kAtoms, (int)rank, ti.x);
-                    else
-                        tma_load_4d_pair(b_dst, &tmB, full0, 0, nt * kG2BN + 128 * (int)rank, kb * kAtoms, ti.x);
+                    // boxes land as [atom][row][64 elements]
+                    tma_load_3d_pair(sA + stage * kABytes, &tmA, full0, 0, a_row, kb * kAtoms);
+                    tma_load_3d_pair(sB + stage * kBBytes, mapB, full0, 0, b_row, kb * kAtoms);
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -202,7 +179,6 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // ---------------- pair MMA issuer (CTA 0)
-            constexpr uint32_t idesc = idesc_bf16_f32(kPairRows, 256);
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -210,6 +186,10 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
             for (int t = pair; t < total_tiles && ok; t += npairs, ++it) {
                 const int buf = it & 1;
                 const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+                const int mt = t / p.n_tiles;
+                const int n = tile_n(__ldg(&p.tiles[mt].z));
+                const uint32_t idesc = idesc_bf16_f32(kPairM, n);
+                const uint32_t b_atom = (uint32_t)(n >> 1) * 128u;  // bytes of one atom of this CTA's B rows
                 if (!mbar_wait_bounded(&bars->acc_empty[buf], acc_phase ^ 1u, abort_flag, p.wait_limit_ns)) {
                     ok = false;
                     break;
@@ -226,8 +206,9 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
                     const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
 #pragma unroll
                     for (int kk = 0; kk < kStageK / 16; ++kk) {
-                        const uint32_t off = (uint32_t)(kk >> 2) * kAtomBytes + (uint32_t)(kk & 3) * 32;
-                        mma_bf16_pair(d_tmem, sdesc_kmajor_sw128(a_addr + off), sdesc_kmajor_sw128(b_addr + off), idesc,
+                        const uint32_t koff = (uint32_t)(kk & 3) * 32;
+                        mma_bf16_pair(d_tmem, sdesc_kmajor_sw128(a_addr + (uint32_t)(kk >> 2) * kAtomBytes + koff),
+                                      sdesc_kmajor_sw128(b_addr + (uint32_t)(kk >> 2) * b_atom + koff), idesc,
                                       (kb | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit_pair_multicast(&bars->empty[stage], 0x3);  // both CTAs may refill the stage
@@ -252,19 +233,17 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
         // ---------------- epilogue: warps 2..9
         const int ew = warp - 2;
         const int quad = warp & 3;   // TMEM lane quarter this warp may read
-        const int half = ew >> 2;    // column half
-        const int r = quad * 32 + lane;
+        const int half = ew >> 2;    // this warp takes the 32-route chunks c with c % 2 == half
         const uint32_t acc_empty0[2] = {map_to_cta(smem_u32(&bars->acc_empty[0]), 0),
                                         map_to_cta(smem_u32(&bars->acc_empty[1]), 0)};
-        uint8_t* my_out = sOut + (size_t)ew * kStageOutBytes;
+        uint8_t* tbuf = sEpi + (size_t)ew * (kMode == 0 ? kHTBytes : kYTBytes);
         int it = 0;
         for (int t = pair; t < total_tiles; t += npairs, ++it) {
             const int buf = it & 1;
             const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
             const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
             const int4 ti = __ldg(p.tiles + mt);
-            const int my_rows = rows_of(ti.z, rank);
-            const int my_row0 = ti.y + 128 * (int)rank;
+            const int nch = tile_n(ti.z) >> 5;
             const bool got = __all_sync(0xffffffffu,
                                         mbar_wait_bounded(&bars->acc_full[buf], acc_phase, abort_flag, p.wait_limit_ns));
             if (!got) {
@@ -275,67 +254,66 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
                 break;
             }
             tc_fence_after_sync();
-            const bool valid = r < my_rows;
             const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)buf * kAccCols;
             if (kMode == 0) {
-                __nv_bfloat16* out_row =
-                    reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)(my_row0 + r) * (size_t)p.out_ld;
+                // f of this lane: f_base + (lane & 15); lanes < 16 hold gate, the others up
+                const int f_base = nt * 128 + 64 * (int)rank + 16 * quad;
+                const bool lo = lane < 16;
+                // transpose box: route r at r * 32 bytes, routes 16..31 shifted by 64 bytes so that
+                // the two half-warps' rows fall in different banks
+                __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
 #pragma unroll 1
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int c = half * 2 + cc;
-                    uint32_t g[32], u[32];
-                    tmem_ld_32x32b_x32(taddr + c * 32, g);
-                    tmem_ld_32x32b_x32(taddr + kG1BN + c * 32, u);
-                    tmem_ld_wait();
-                    const int f0 = nt * kG1BN + c * 32;
-                    if (valid) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            {  // f >= F are zero-weight rows: h = 0, which pads h's K pitch to 128
-                                uint32_t w[4];
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    const int a = q * 8 + 2 * i;
-                                    const float h0 = silu_f(__uint_as_float(g[a])) * __uint_as_float(u[a]);
-                                    const float h1 = silu_f(__uint_as_float(g[a + 1])) * __uint_as_float(u[a + 1]);
-                                    w[i] = pack_bf16x2(h0, h1);
-                                }
-                                *reinterpret_cast<uint4*>(out_row + f0 + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
-                            }
-                        }
-                    }
-                }
-            } else {
-                // fp32 rows leave through the LSU, not the TMA engine (which the
-                // operand loads saturate): the warp stages its 32 rows x 32
-                // columns in a swizzled 4 KB box, reads it back transposed and
-                // writes 4 rows x 128 bytes per instruction, valid rows only.
-                const bool slice_live = quad * 32 < my_rows;
-                float* y = reinterpret_cast<float*>(p.out);
-#pragma unroll 1
-                for (int cc = 0; cc < 4; ++cc) {
-                    const int c = half * 4 + cc;
+                for (int c = half; c < nch; c += 2) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(taddr + c * 32, v);
                     tmem_ld_wait();
-                    const int c0 = nt * kG2BN + c * 32;
-                    if (slice_live && c0 < p.out_cols) {
+                    // lanes < 16 keep their gate values of routes 0..15 and receive the up values;
+                    // lanes >= 16 keep their up values of routes 16..31 and receive the gate values
+                    uint8_t* row0 = tbuf + (lo ? 0 : 16 * 32 + 64) + (lane & 15) * 2;
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const uint32_t off = (uint32_t)lane * 128u + (uint32_t)((q ^ (lane & 7)) * 16);
-                            *reinterpret_cast<uint4*>(my_out + off) =
-                                make_uint4(v[q * 4], v[q * 4 + 1], v[q * 4 + 2], v[q * 4 + 3]);
-                        }
+                    for (int j = 0; j < 16; ++j) {
+                        const uint32_t mine = lo ? v[j] : v[16 + j];
+                        const uint32_t other = __shfl_xor_sync(0xffffffffu, lo ? v[16 + j] : v[j], 16);
+                        const float g = __uint_as_float(lo ? mine : other);
+                        const float u = __uint_as_float(lo ? other : mine);
+                        *reinterpret_cast<__nv_bfloat16*>(row0 + j * 32) = __float2bfloat16_rn(silu_f(g) * u);
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const int r = i * 16 + (lane >> 1);
+                        const int route = c * 32 + r;
+                        const uint4 w = *reinterpret_cast<const uint4*>(tbuf + r * 32 + (r >= 16 ? 64 : 0) +
+                                                                        (lane & 1) * 16);
+                        if (route < ti.z)
+                            *reinterpret_cast<uint4*>(h + (size_t)(ti.y + route) * (size_t)p.out_ld + f_base +
+                                                      (lane & 1) * 8) = w;
+                    }
+                    __syncwarp();
+                }
+            } else {
+                // output columns of this warp: nt*256 + 128*rank + 32*quad + lane
+                const int c_base = nt * kPairM + 128 * (int)rank + 32 * quad;
+                float* y = reinterpret_cast<float*>(p.out);
+                if (c_base < p.out_cols) {
+                    const bool col_ok = c_base + (lane & 7) * 4 < p.out_cols;
+#pragma unroll 1
+                    for (int c = half; c < nch; c += 2) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(taddr + c * 32, v);
+                        tmem_ld_wait();
+                        // transpose: [route][32 c] fp32, 128 bytes per route
+#pragma unroll
+                        for (int r = 0; r < 32; ++r) *reinterpret_cast<uint32_t*>(tbuf + r * 128 + lane * 4) = v[r];
                         __syncwarp();
-                        const int q = lane & 7;
-                        const bool col_ok = c0 + q * 4 < p.out_cols;
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            const int row = i * 4 + (lane >> 3);
-                            const uint4 w = *reinterpret_cast<const uint4*>(my_out + row * 128 + ((q ^ (row & 7)) * 16));
-                            if (col_ok && quad * 32 + row < my_rows)
-                                *reinterpret_cast<uint4*>(y + (size_t)(my_row0 + quad * 32 + row) * (size_t)p.out_ld + c0 +
-                                                          q * 4) = w;
+                            const int r = i * 4 + (lane >> 3);
+                            const int route = c * 32 + r;
+                            const uint4 w = *reinterpret_cast<const uint4*>(tbuf + r * 128 + (lane & 7) * 16);
+                            if (col_ok && route < ti.z)
+                                *reinterpret_cast<uint4*>(y + (size_t)(ti.y + route) * (size_t)p.out_ld + c_base +
+                                                          (lane & 7) * 4) = w;
                         }
                         __syncwarp();
                     }
@@ -358,20 +336,18 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    moe_gemm_gate_up_swiglu_bf16_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA128,
-                                      const __grid_constant__ CUtensorMap tmB,
-                                      const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
-    pair_gemm_body<0>(tmA, tmA128, tmB, tmOut, p);
+    moe_gemm_gate_up_swiglu_bf16_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BoxMaps8 tmB,
+                                      const GemmParams p) {
+    pair_gemm_body<0>(tmA, tmB, p);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    moe_gemm_down_bf16_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA128,
-                            const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmOut,
+    moe_gemm_down_bf16_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BoxMaps8 tmB,
                             const GemmParams p) {
-    pair_gemm_body<1>(tmA, tmA128, tmB, tmOut, p);
+    pair_gemm_body<1>(tmA, tmB, p);
 }
 
-using GemmKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
+using GemmKernel = void (*)(CUtensorMap, BoxMaps8, GemmParams);
 
 struct PairLaunchCache {
     size_t smem = 0;
@@ -379,9 +355,8 @@ struct PairLaunchCache {
     int pairs = 0;
 };
 
-cudaError_t launch_pair(GemmKernel kern, PairLaunchCache* cache, const CUtensorMap& a, const CUtensorMap& a128,
-                        const CUtensorMap& b, const CUtensorMap& o, const GemmParams& gp, long long max_tiles,
-                        cudaStream_t s) {
+cudaError_t launch_pair(GemmKernel kern, PairLaunchCache* cache, const CUtensorMap& a, const BoxMaps8& b,
+                        const GemmParams& gp, long long max_tiles, cudaStream_t s) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
@@ -412,23 +387,23 @@ cudaError_t launch_pair(GemmKernel kern, PairLaunchCache* cache, const CUtensorM
     if (pairs > max_tiles) pairs = max_tiles;
     if (pairs < 1) pairs = 1;
     cfg.gridDim = dim3((unsigned)(2 * pairs));
-    err = cudaLaunchKernelEx(&cfg, kern, a, a128, b, o, gp);
+    err = cudaLaunchKernelEx(&cfg, kern, a, b, gp);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_gemm1_bf16_pair(const CUtensorMap& a, const CUtensorMap& a128, const CUtensorMap& b,
-                                   const CUtensorMap& o, const GemmParams& gp, long long max_tiles, cudaStream_t s) {
+cudaError_t launch_gemm1_bf16_pair(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
+                                   cudaStream_t s) {
     static PairLaunchCache cache{PairCfg<0>::kSmemBytes};
-    return launch_pair(moe_gemm_gate_up_swiglu_bf16_pair, &cache, a, a128, b, o, gp, max_tiles, s);
+    return launch_pair(moe_gemm_gate_up_swiglu_bf16_pair, &cache, a, b, gp, max_tiles, s);
 }
 
-cudaError_t launch_gemm2_bf16_pair(const CUtensorMap& a, const CUtensorMap& a128, const CUtensorMap& b,
-                                   const CUtensorMap& o, const GemmParams& gp, long long max_tiles, cudaStream_t s) {
+cudaError_t launch_gemm2_bf16_pair(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
+                                   cudaStream_t s) {
     static PairLaunchCache cache{PairCfg<1>::kSmemBytes};
-    return launch_pair(moe_gemm_down_bf16_pair, &cache, a, a128, b, o, gp, max_tiles, s);
+    return launch_pair(moe_gemm_down_bf16_pair, &cache, a, b, gp, max_tiles, s);
 }
 
 }  // namespace moe

@@ -15,11 +15,13 @@
 namespace moe {
 
 // ---------------------------------------------------------------- tiling
-constexpr int kBM = 128;           // permuted rows (routes) per M tile
+constexpr int kBM = 128;           // MXFP8: routes per M tile (and the row alignment of its scale blocks)
 constexpr int kBK = 64;            // bf16 K elements per pipeline stage (128-byte rows)
 constexpr int kBK8 = 128;          // E4M3 K elements per pipeline stage (128-byte rows)
-constexpr int kG1BN = 128;         // f values per gate/up tile (128 gate + 128 up MMA columns)
-constexpr int kG2BN = 256;         // output columns per down tile
+constexpr int kG1BN = 128;         // bf16: f values per gate/up weight tile (256 weight rows, gate and up)
+constexpr int kG2BN = 256;         // bf16: output columns per down weight tile
+constexpr int kRouteTile = 256;    // bf16: most routes per tile (N of a pair MMA)
+constexpr int kRouteAlign = 32;    // bf16: route rows of an expert start on a multiple of this
 constexpr int kG1BN8 = 64;         // MXFP8: f values per gate/up tile (64 gate + 64 up MMA columns)
 constexpr int kG2BN8 = 128;        // MXFP8: output columns per down tile
 constexpr int kSfBlock = 512;      // MXFP8 scales of 128 rows x 4 k-groups, [row%32][row/32][k-group]
@@ -50,30 +52,39 @@ struct moe_plan {
     moe_desc d;
     long long max_live;
     long long max_routes;   // max_live * k
-    long long max_m_tiles;  // upper bound on M tiles: ceil(routes / tile_rows) + E
-    long long rows_pad;     // max_m_tiles * tile_rows: rows of the padded intermediates
+    long long max_m_tiles;  // upper bound on route tiles: ceil(routes / tile_rows) + E
+    long long rows_pad;     // rows of the padded intermediates (an upper bound on the padded route space)
     int nblk;               // ceil(max_live / kTokPerBlk)
-    int tile_rows;          // rows of an M tile: 256 (bf16, CTA pairs) or 128 (MXFP8)
+    int tile_rows;          // most routes per tile: 256 (bf16, N of a pair MMA) or 128 (MXFP8, M of the MMA)
+    int row_align;          // each expert's route rows start on a multiple of this: 32 (bf16) or 128 (MXFP8)
     long long hp, fp;       // K row pitch (elements) of x / gate-up rows and of h / down rows:
                             // bf16 pads H and F to multiples of 128 with zeros; MXFP8 keeps H, F
     int ks1, ks2;           // K stages of the gate/up and down GEMMs
-    int nt1, nt2;           // N tiles of the gate/up and down GEMMs
+    int nt1, nt2;           // weight (bf16) / N (MXFP8) tiles of the gate/up and down GEMMs
     moe::WsLayout ws;
     moe::WbufLayout wb;
 };
 
 namespace moe {
 
+// Tensor maps of one route-row operand with box heights 16, 32, ..., 128 rows
+// (entry i: 16 * (i + 1) rows), so that a tile of N routes loads its N/2 rows
+// per CTA of a pair with one TMA instruction.
+struct BoxMaps8 {
+    CUtensorMap m[8];
+};
+
 struct GemmParams {
-    const int4* tiles;              // {expert, first padded row, valid rows, 0} per M tile (tile_rows rows)
+    const int4* tiles;              // {expert, first padded row, valid rows, 0} per route tile
     const unsigned* status_words;   // [kStNumMTiles] = number of M tiles
     unsigned* status_flags;         // sticky MOE_DEV_* bits
     void* out;                      // h (bf16 / E4M3) or y (fp32)
     uint8_t* out_scales;            // E8M0 scales of h (MXFP8), else null
     long long out_ld;               // row stride of out, elements
     int out_cols;                   // valid output columns (F or H)
-    int n_tiles;                    // N tiles per M tile
+    int n_tiles;                    // weight tiles per route tile
     int k_blocks;                   // pipeline stages per tile
+    long long a_rows;               // bf16: rows of one expert in the weight operand's tensor map
     unsigned long long wait_limit_ns;
     // MXFP8 only: scale blocks of A ([M tile][K stage][512 B]) and of B
     // ([expert][N tile][K stage][512 B]); K stages of the down GEMM (the gate/up
@@ -103,14 +114,10 @@ cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max
                                 const int* inv, uint8_t* xq, uint8_t* xs, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const int* inv, const float* probs, const int* live, int max_live,
                            int H, int k, float* out, cudaStream_t s);
-cudaError_t launch_gemm1_bf16(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& gp,
-                              int grid, cudaStream_t s);
-cudaError_t launch_gemm2_bf16(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o, const GemmParams& gp,
-                              int grid, cudaStream_t s);
-cudaError_t launch_gemm1_bf16_pair(const CUtensorMap& a, const CUtensorMap& a128, const CUtensorMap& b,
-                                   const CUtensorMap& o, const GemmParams& gp, long long max_tiles, cudaStream_t s);
-cudaError_t launch_gemm2_bf16_pair(const CUtensorMap& a, const CUtensorMap& a128, const CUtensorMap& b,
-                                   const CUtensorMap& o, const GemmParams& gp, long long max_tiles, cudaStream_t s);
+cudaError_t launch_gemm1_bf16_pair(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
+                                   cudaStream_t s);
+cudaError_t launch_gemm2_bf16_pair(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
+                                   cudaStream_t s);
 cudaError_t launch_gemm1_mxfp8(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o,
                                const GemmParams& gp, int grid, cudaStream_t s);
 cudaError_t launch_gemm2_mxfp8(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o,

@@ -8,8 +8,9 @@
 //   hist     per 256-token block, per-expert route counts (shared-memory
 //            counters: a count does not depend on the order of increments)
 //   scan     one CTA: per-expert prefix over blocks, exclusive scan over
-//            experts -> offsets[E+1]; the same over ceil(count/tile_rows) ->
-//            the padded row space the GEMM tiles live in, and the M-tile list
+//            experts -> offsets[E+1]; the same over the counts rounded up to
+//            row_align -> the padded row space the GEMMs read, and over
+//            ceil(count / tile_rows) -> the list of route tiles
 //   scatter  per block: one 32-bit lane mask per (warp, expert) gives every
 //            route its rank among earlier tokens of the block routed to the
 //            same expert (popcount of the lower lanes plus the earlier warps)
@@ -69,7 +70,7 @@ __device__ __forceinline__ int block_exclusive_scan_1024(int v, int* s_warp, int
 }
 
 __global__ void __launch_bounds__(1024) route_scan_kernel(const int* __restrict__ live, int max_live, int E,
-                                                          int tile_rows, int* __restrict__ blkcnt,
+                                                          int tile_rows, int row_align, int* __restrict__ blkcnt,
                                                           int* __restrict__ offsets,
                                                           int* __restrict__ padoff, int4* __restrict__ tiles,
                                                           unsigned* __restrict__ status_words) {
@@ -86,20 +87,22 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int* __restrict_
         }
     }
     const int mt = (tot + tile_rows - 1) / tile_rows;
-    int sum_tot, sum_mt;
+    const int padded = (tot + row_align - 1) / row_align * row_align;
+    int sum_tot, sum_mt, sum_pad;
     const int ex_tot = block_exclusive_scan_1024(tot, s_warp, &sum_tot);
     const int ex_mt = block_exclusive_scan_1024(mt, s_warp, &sum_mt);
+    const int ex_pad = block_exclusive_scan_1024(padded, s_warp, &sum_pad);
     if (e < E) {
         offsets[e] = ex_tot;
-        padoff[e] = ex_mt * tile_rows;
+        padoff[e] = ex_pad;
         for (int i = 0; i < mt; ++i) {
             const int rows = tot - i * tile_rows;
-            tiles[ex_mt + i] = make_int4(e, (ex_mt + i) * tile_rows, rows < tile_rows ? rows : tile_rows, 0);
+            tiles[ex_mt + i] = make_int4(e, ex_pad + i * tile_rows, rows < tile_rows ? rows : tile_rows, 0);
         }
     }
     if (e == 0) {
         offsets[E] = sum_tot;
-        padoff[E] = sum_mt * tile_rows;
+        padoff[E] = sum_pad;
         status_words[kStNumMTiles] = (unsigned)sum_mt;
         status_words[kStTotalRoutes] = (unsigned)sum_tot;
     }
@@ -298,8 +301,8 @@ cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* 
     route_hist_kernel<<<nblk, kTokPerBlk, E * sizeof(int), s>>>(r_ids, live, max_live, E, k, blkcnt);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    route_scan_kernel<<<1, 1024, 0, s>>>(live, max_live, E, p->tile_rows, blkcnt, offsets, padoff, tiles,
-                                         status_words);
+    route_scan_kernel<<<1, 1024, 0, s>>>(live, max_live, E, p->tile_rows, p->row_align, blkcnt, offsets, padoff,
+                                         tiles, status_words);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     const size_t smem = (size_t)(kTokPerBlk / 32) * E * 8;

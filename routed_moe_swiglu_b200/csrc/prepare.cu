@@ -3,11 +3,14 @@
 // refresh_mega_weights(), which rewrites the kernel's own copy of the
 // weights; no allocation, no teardown).
 //
-// bf16 layout:  W1 [E][2][F][hp]  (gate rows, then up rows of each expert),
-//               W2 [E][H][fp]     (down projection),
-// with the K pitches hp, fp = H, F rounded up to 128 and the padding zero.
-// A gate/up tile loads the same 128 f rows from W1[e][0] and W1[e][1] into
-// one 256-row B operand, so gate and up of one f meet in one accumulator row.
+// bf16 layout:  W1 [E][fp/64][4][2][16][hp]  (per block of 64 f, per group of
+//                                           16 f: the 16 gate rows, then the
+//                                           16 up rows of the same f),
+//               W2 [E][H][fp]               (down projection),
+// with the K pitches hp, fp = H, F rounded up to 128 and the padding zero
+// (rows of f >= F too).  A gate/up weight tile is two consecutive blocks, one
+// per CTA of a pair; a group of 32 rows is one 32-lane TMEM quarter, so gate
+// and up of one f land in the same warp's reach.
 #include "moe_internal.cuh"
 #include "mxfp8.cuh"
 
@@ -19,18 +22,20 @@ __global__ void __launch_bounds__(256) prepare_bf16_kernel(const uint4* __restri
                                                            uint4* __restrict__ w2, int E, int F, int H, int hp, int fp) {
     // 16-byte chunks of the destination; rows are padded with zeros to hp / fp
     const long long c1 = hp / 8, c2 = fp / 8;
-    const long long n1 = (long long)E * 2 * F * c1;
+    const long long rows1 = 2ll * fp;  // W1 rows per expert
+    const long long n1 = (long long)E * rows1 * c1;
     const long long n2 = (long long)E * H * c2;
     const long long stride = (long long)gridDim.x * blockDim.x;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n1 + n2; i += stride) {
         if (i < n1) {
-            const long long row = i / c1;  // (e * 2 + g) * F + f
+            const long long row = i / c1;  // e * 2fp + block * 128 + group * 32 + g * 16 + f % 16
             const int c = (int)(i - row * c1);
-            const long long e = row / (2 * F);
-            const int g = (int)((row / F) & 1);
-            const long long f = row - (e * 2 + g) * F;
+            const long long e = row / rows1;
+            const int rem = (int)(row - e * rows1);
+            const int g = (rem >> 4) & 1;
+            const int f = (rem >> 7) * 64 + ((rem >> 5) & 3) * 16 + (rem & 15);
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (c * 8 < H) v = __ldg((g ? wu : wg) + (e * F + f) * (H / 8) + c);
+            if (f < F && c * 8 < H) v = __ldg((g ? wu : wg) + (e * F + f) * (H / 8) + c);
             w1[i] = v;
         } else {
             const long long j = i - n1;

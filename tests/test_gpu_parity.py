@@ -91,7 +91,7 @@ def test_mxfp8_quantize_strided_and_live_bound():
 # ---------------------------------------------------------------- forward, bf16
 
 
-def _check_permutation(m: GpuMoe, ref_ids, E):
+def _check_permutation(m: GpuMoe, ref_ids, E, align=32):
     v = m.views()
     live, k = ref_ids.shape
     ids_gpu = m.read_i32(v["route_ids"], live * k).reshape(live, k)
@@ -101,13 +101,13 @@ def _check_permutation(m: GpuMoe, ref_ids, E):
     assert np.array_equal(off_gpu, offsets.astype(np.int32))
     perm_gpu = m.read_i32(v["perm"], live * k)
     assert np.array_equal(perm_gpu, perm)
-    # padded rows: every expert segment starts on a 128-row boundary, order kept
+    # padded rows: every expert segment starts on a 32-row (bf16) / 128-row (MXFP8) boundary, order kept
     pad = m.read_i32(v["pad_offsets"], E + 1)
     inv_gpu = m.read_i32(v["inv"], live * k).reshape(live, k)
     e_of = ref_ids
     rank = inv.astype(np.int64) - offsets[e_of]
     assert np.array_equal(inv_gpu, (pad[e_of] + rank).astype(np.int32))
-    assert np.all(pad % 128 == 0)
+    assert np.all(pad % align == 0)
 
 
 def test_forward_tiny_all_tokens():
@@ -171,6 +171,29 @@ def test_forward_prefill_subset_and_full_permutation():
     _check_permutation(m, ref_ids, w.num_experts)
     counts = np.bincount(ref_ids.reshape(-1), minlength=w.num_experts)
     assert counts.max() > 8 * np.median(counts)  # the Zipf bias really skews the loads
+
+
+def test_every_tile_width():
+    """Caller routes that give experts 1..513 routes: every route-tile width
+    (N = 32..256 in steps of 32), full tiles followed by a tail of 1, 31, 32
+    or 33 rows, and K and output-column tails (H = 320, F = 200)."""
+    H, F, E, k = 320, 200, 20, 2
+    counts = np.array([1, 15, 16, 17, 31, 32, 33, 63, 64, 65, 100, 127, 128, 129, 200, 255, 256, 257, 300, 513])
+    T = int(counts.sum()) // k
+    x, _, weights = workloads.small_case(H, F, E, k, T, seed=77)
+    gen = np.random.default_rng(77)
+    experts = np.repeat(np.arange(E), counts)  # route list by expert; token t gets entries t and t + T
+    ids = np.stack([experts[:T], experts[T:]], axis=1)
+    ids = ids[gen.permutation(T)].astype(np.int32)
+    assert np.all(ids[:, 0] != ids[:, 1])
+    p = gen.uniform(0.1, 1.0, size=(T, k))
+    probs = (p / p.sum(axis=1, keepdims=True)).astype(np.float32)
+    m = GpuMoe(H, F, E, k, T, weights)
+    out = m.forward(x.cuda(), T, ids=torch.from_numpy(ids).cuda(), probs=torch.from_numpy(probs).cuda())
+    torch.cuda.synchronize()
+    ref = oracle.forward_bf16(x, ids, probs, *weights)
+    assert_close(out.cpu().numpy(), ref, "bf16", "every tile width")
+    assert m.status() == 0
 
 
 # ---------------------------------------------------------------- invariance and edge cases

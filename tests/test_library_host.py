@@ -60,7 +60,7 @@ def test_plan_sizes():
     # weight buffer: gate+up+down bf16, each 256-byte aligned region
     assert rm.moe_weight_buffer_bytes(p) >= 3 * 128 * 2048 * 1024 * 2
     ws = rm.moe_workspace_bytes(p)
-    rows_pad = (256 * 8 // 128 + 128) * 128
+    rows_pad = 256 * 8 + 128 * 32  # routes + experts x the 32-row segment alignment
     assert ws >= rows_pad * (2048 * 2 + 1024 * 2 + 2048 * 4)
     q = rm.moe_plan_create(hidden=2048, ffn=1024, num_experts=128, top_k=8, capacity=65536)
     assert q.max_live_rows == 65536 and rm.moe_workspace_bytes(q) > ws
