@@ -104,7 +104,7 @@ static void compute_layouts(moe_plan* p) {
     WbufLayout& b = p->wb;
     off = 0;
     if (fp8) {
-        b.w1 = take(E * 2 * F * H);
+        b.w1 = take(E * 2 * ((F + 63) / 64 * 64) * H);  // W1 rows padded to whole 64-f blocks
         b.w1s = take(E * p->nt1 * p->ks1 * kSfBlock);
         b.w2 = take(E * H * F);
         b.w2s = take(E * p->nt2 * p->ks2 * kSfBlock);
@@ -274,33 +274,29 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     const unsigned long long R = (unsigned long long)plan->rows_pad;
     const unsigned long long uH = (unsigned long long)H, uF = (unsigned long long)F, uE = (unsigned long long)E;
     const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    CUtensorMap tA1, tB1, tA2, tB2, tY;
-    BoxMaps8 rB1, rB2;  // bf16: route-row operands (x rows, h rows)
+    CUtensorMap tA1, tA2;  // weight operands
+    BoxMaps8 rB1, rB2;     // route-row operands (x rows, h rows)
     if (fp8) {
-        // MXFP8 (one CTA per tile): 2-D A maps with 32-row boxes, B in 64/128-row boxes,
-        // K stage = 128 E4M3 elements (one 128-byte swizzle atom)
-        const unsigned bk = (unsigned)kBK8;
-        const unsigned long long dA[2] = {uH, R};
-        const unsigned long long sA[1] = {uH};
-        const unsigned bA[2] = {bk, 32};
-        const unsigned long long dB[4] = {uH, uF, 2ull, uE};
-        const unsigned long long sB[3] = {uH, uF * uH, 2ull * uF * uH};
-        const unsigned bB[4] = {bk, (unsigned)kG1BN8, 1, 1};
-        const unsigned long long dA2[2] = {uF, R};
-        const unsigned long long sA2[1] = {uF};
-        const unsigned long long dB2[3] = {uF, uH, uE};
-        const unsigned long long sB2[2] = {uF, uH * uF};
-        const unsigned bB2[3] = {bk, (unsigned)kG2BN8, 1};
-        const unsigned long long dY[2] = {uH, R};
-        const unsigned long long sY[1] = {uH * 4};
-        const unsigned bY[2] = {32, 32};
-        if (!make_tensor_map(&tA1, dt, 2, ws + L.xq, dA, sA, bA, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tB1, dt, 4, wb + plan->wb.w1, dB, sB, bB, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tA2, dt, 2, ws + L.h, dA2, sA2, bA, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tB2, dt, 3, wb + plan->wb.w2, dB2, sB2, bB2, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ws + L.y, dY, sY, bY,
-                             CU_TENSOR_MAP_SWIZZLE_128B))
+        // MXFP8 (one CTA per tile): weights (A) load 128 rows, route rows (B) N <= 128 rows,
+        // one map per N in {32, 64, 96, 128}; K stage = 128 E4M3 elements (one 128-byte swizzle
+        // atom); K past H / F is the maps' zero fill
+        const unsigned long long f64 = (uF + 63) / 64 * 64;
+        const unsigned box128[2] = {(unsigned)kBK8, 128};
+        const unsigned long long dW1[2] = {uH, uE * 2ull * f64};
+        const unsigned long long sW1[1] = {uH};
+        const unsigned long long dW2[2] = {uF, uE * uH};
+        const unsigned long long sW2[1] = {uF};
+        const unsigned long long dX[2] = {uH, R};
+        const unsigned long long dH[2] = {uF, R};
+        if (!make_tensor_map(&tA1, dt, 2, wb + plan->wb.w1, dW1, sW1, box128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tA2, dt, 2, wb + plan->wb.w2, dW2, sW2, box128, CU_TENSOR_MAP_SWIZZLE_128B))
             return MOE_ERR_CUDA;
+        for (int i = 0; i < 4; ++i) {
+            const unsigned box[2] = {(unsigned)kBK8, 32u * (unsigned)(i + 1)};
+            if (!make_tensor_map(&rB1.m[i], dt, 2, ws + L.xq, dX, sW1, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+                !make_tensor_map(&rB2.m[i], dt, 2, ws + L.h, dH, sW2, box, CU_TENSOR_MAP_SWIZZLE_128B))
+                return MOE_ERR_CUDA;
+        }
     } else {
         // bf16 (CTA pairs): K stage = 128 elements = two 64-element swizzle atoms.  Every
         // operand buffer has its K pitch padded to 128 (hp, fp) with zeros, and the maps
@@ -361,19 +357,16 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g1.out_scales = nullptr;
     g1.out_ld = plan->fp;  // h rows: F values + zero padding to the down GEMM's K pitch
     g1.out_cols = fp8 ? F : (int)plan->fp;
-    g1.a_rows = 2 * plan->fp;  // bf16 W1: gate and up rows of an expert, padded F
+    g1.a_rows = fp8 ? 2 * ((F + 63) / 64 * 64) : 2 * plan->fp;  // W1 rows of an expert (padded F)
     g1.n_tiles = plan->nt1;
     g1.k_blocks = plan->ks1;
     g1.wait_limit_ns = kWaitLimitNs;
-    g1.sfa = ws + L.xs;
-    g1.sfb = wb + plan->wb.w1s;
+    g1.sfa = wb + plan->wb.w1s;  // MXFP8: A = weights, B = route rows
+    g1.sfb = ws + L.xs;
     g1.out_scales = fp8 ? ws + L.hs : nullptr;
     g1.sf_ks_out = plan->ks2;
-    const int sms = num_sms();
-    long long grid1 = m_tiles * g1.n_tiles;
-    if (grid1 > sms) grid1 = sms;
     if (!mark(3)) return MOE_ERR_CUDA;
-    e = fp8 ? launch_gemm1_mxfp8(tA1, tB1, tY, g1, (int)grid1, s)
+    e = fp8 ? launch_gemm1_mxfp8(tA1, rB1, g1, m_tiles * g1.n_tiles, s)
             : launch_gemm1_bf16_pair(tA1, rB1, g1, m_tiles * g1.n_tiles, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -384,13 +377,11 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g2.n_tiles = plan->nt2;
     g2.k_blocks = plan->ks2;
     g2.a_rows = H;
-    g2.sfa = ws + L.hs;
-    g2.sfb = wb + plan->wb.w2s;
+    g2.sfa = wb + plan->wb.w2s;
+    g2.sfb = ws + L.hs;
     g2.out_scales = nullptr;
-    long long grid2 = m_tiles * g2.n_tiles;
-    if (grid2 > sms) grid2 = sms;
     if (!mark(4)) return MOE_ERR_CUDA;
-    e = fp8 ? launch_gemm2_mxfp8(tA2, tB2, tY, g2, (int)grid2, s)
+    e = fp8 ? launch_gemm2_mxfp8(tA2, rB2, g2, m_tiles * g2.n_tiles, s)
             : launch_gemm2_bf16_pair(tA2, rB2, g2, m_tiles * g2.n_tiles, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     if (!mark(5)) return MOE_ERR_CUDA;

@@ -1,32 +1,40 @@
 // gemm_mxfp8.cu -- the two grouped expert GEMMs in MXFP8 (E4M3 operands with
 // one E8M0 scale per 32 K elements per row), block-scaled tcgen05 MMAs with
-// the scale factors in TMEM.
+// the scale factors in TMEM, expert weights as the MMA's M operand and routes
+// as its N operand (as in the bf16 kernels: the last tile of an expert costs
+// its route count rounded up to 32, not a full tile).
 //
 // Megatron-LM PR #7798, "Background": the FC1 epilogue fuses the activation
 // and the FC2-input quantisation; probabilities are applied after FC2.
 // Megatron-LM PR #7830 / cudnn-frontend PR #448: MXFP8 blocks are 32
 // elements along K.
 //
-//   gate/up:  M tile = 128 route rows, N tile = 64 f values (B rows 0..63
-//             W_gate[e, f0:f0+64], rows 64..127 W_up[e, f0:f0+64]), K stage
-//             = 128 E4M3 elements = 4 MMAs of K=32.  The epilogue forms
-//             h = silu(g) * u in fp32 and re-quantises it to MXFP8 (blocks of
-//             32 along F): E4M3 codes to h, E8M0 bytes straight into the
-//             scale layout the down GEMM reads.
-//   down:     A = h codes + scales, B = W_down[e, c0:c0+128], fp32 y out.
+//   gate/up:  A = 128 rows of W1 = 64 f values: TMEM lane quarter q holds
+//             the gate rows of f = f0 + 16q + i in lanes 32q+i and the up
+//             rows of the same f in lanes 32q+16+i (the prepared W1 is
+//             interleaved so); B = N <= 128 route rows of x codes.  The
+//             epilogue forms h = silu(g) * u in fp32 (half-warps swap gate
+//             and up with shfl.xor 16), stages 32 routes x 64 f in shared
+//             memory, and two threads per (route, 32-f block) re-quantise it
+//             to MXFP8: E4M3 codes to h, E8M0 bytes into the scale layout the
+//             down GEMM reads.
+//   down:     A = 128 rows of W_down[e] (output columns), B = N route rows of
+//             h codes; fp32 y rows leave through a shared-memory transpose.
 //
-// Scale factors: for each 128-row operand tile and K stage, 512 bytes laid
-// out as [row % 32][row / 32][k-group] (16 bytes per 32-row lane group),
-// which one tcgen05.cp (32x128b, replicated to the 4 lane quarters) moves to
-// 4 TMEM columns; MMA k-group kk selects byte kk of each 32-bit cell.  Both
-// the weights (at prepare time) and the activations (gather, epilogue) are
-// written in that layout, so a stage's scales arrive with one bulk copy.
+// Scale factors: for each 128-row operand tile (a weight tile, or the 128
+// padded route rows a route tile lies in) and K stage of 128 elements, 512
+// bytes laid out as [row % 32][row / 32][k-group], which one tcgen05.cp
+// (32x128b, replicated to the 4 lane quarters) moves to 4 TMEM columns; MMA
+// k-group kk selects byte kk of each 32-bit cell.  The blocks of 8
+// consecutive K stages of a tile are contiguous, so they arrive with one
+// bulk copy per operand into a double-buffered shared-memory area, and the
+// MMA thread moves each stage's blocks to TMEM just before its MMAs.
 //
-// Pipeline as in the bf16 kernel: persistent CTA per SM, warp 0 TMA,
-// warp 1 MMA + TMEM owner, warps 2-5 epilogue; 5 stages; two 128-column
-// accumulators; one scale-factor TMEM slot per stage (a slot is rewritten
-// only after the MMAs that read it have completed, which the producer's wait
-// on that stage's "empty" barrier already implies).
+// Pipeline: persistent CTA per SM, warp 0 TMA, warp 1 MMA + TMEM owner,
+// warps 2-5 epilogue; two 128-column accumulators; one scale-factor TMEM
+// slot per stage (rewritten only after the MMAs that read it have completed,
+// which the producer's wait on that stage's "empty" barrier already
+// implies).  Every wait is bounded.
 #include "moe_internal.cuh"
 #include "mxfp8.cuh"
 #include "ptx.cuh"
@@ -34,28 +42,33 @@
 namespace moe {
 namespace {
 
-constexpr int kStages = 5;
+constexpr int kStages = 6;
 constexpr int kThreads = 192;
-constexpr int kBN = 128;                               // MMA N (both GEMMs)
-constexpr int kABoxRows = 32;
-constexpr uint32_t kABytes = kBM * kBK8;               // 16 KB
-constexpr uint32_t kABoxBytes = kABoxRows * kBK8;      // 4 KB
-constexpr uint32_t kBBytes = kBN * kBK8;               // 16 KB
-constexpr uint32_t kSfBytes = kSfBlock;
-constexpr uint32_t kStageBytes = kABytes + kBBytes + 2 * kSfBytes;
-constexpr uint32_t kAccCols = kBN;
-constexpr uint32_t kSfCol0 = 2 * kAccCols;             // first scale-factor column
+constexpr int kTileM = 128;                            // weight rows per tile
+constexpr int kMaxN = 128;                             // routes per tile
+constexpr uint32_t kABytes = kTileM * kBK8;            // 16 KB
+constexpr uint32_t kBBytes = kMaxN * kBK8;             // up to 16 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr int kSfGroup = 8;                            // K stages per scale-factor bulk copy
+constexpr uint32_t kSfGroupBytes = kSfGroup * kSfBlock;
+constexpr uint32_t kSfBytes = 2 * 2 * kSfGroupBytes;   // [buffer][A/B][8 stages][512 B]
+constexpr uint32_t kAccCols = kMaxN;
+constexpr uint32_t kSfCol0 = 2 * kAccCols;             // first scale-factor TMEM column
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kStageOutBytes = 32 * 128;
-constexpr uint32_t kOutBytes = 4 * 2 * kStageOutBytes;
-constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kOutBytes + 256;
-static_assert(kSfCol0 + 16 * kStages <= kTmemCols, "TMEM budget");
+constexpr uint32_t kStageHBytes = 32 * 64 * 4;         // gate/up: fp32 h of 32 routes x 64 f
+constexpr uint32_t kYTBytes = 32 * 32 * 4;             // down: fp32 y of 32 routes x 32 columns, per warp
+constexpr uint32_t kEpiBytes = 2 * kStageHBytes > 4 * kYTBytes ? 2 * kStageHBytes : 4 * kYTBytes;
+constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kSfBytes + kEpiBytes + 256;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kSfCol0 + 8 * kStages <= kTmemCols, "TMEM budget");
+constexpr uint32_t kEpiBar = 1;                        // named barrier of the 4 epilogue warps
 
 struct __align__(8) Barriers {
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
+    uint64_t sf_empty[2];
     uint64_t done;
     uint32_t tmem_base;
     int abort_flag;
@@ -87,21 +100,22 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                  : "memory");
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
+// Routes of a tile rounded up to the MMA's N granularity.
+__device__ __forceinline__ int tile_n(int nvalid) { return (nvalid + 31) & ~31; }
 
 template <int kMode>  // 0: gate/up + SwiGLU -> MXFP8 h;  1: down -> fp32 y
-__device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const CUtensorMap& tmB,
-                                                const CUtensorMap& tmOut, const GemmParams& p) {
+__device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const BoxMaps8& tmB, const GemmParams& p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sOut = smem + kStages * kStageBytes;  // 1024-aligned (kStageBytes is a multiple of 1024)
-    Barriers* bars = reinterpret_cast<Barriers*>(sOut + kOutBytes);
+    uint8_t* sSf = smem + kStages * kStageBytes;  // [buffer][A/B][8][512]
+    uint8_t* sEpi = sSf + kSfBytes;
+    Barriers* bars = reinterpret_cast<Barriers*>(sEpi + kEpiBytes);
     volatile int* abort_flag = &bars->abort_flag;
     auto stage_a = [&](int s) { return smem + s * kStageBytes; };
     auto stage_b = [&](int s) { return smem + s * kStageBytes + kABytes; };
-    auto stage_sfa = [&](int s) { return smem + s * kStageBytes + kABytes + kBBytes; };
-    auto stage_sfb = [&](int s) { return smem + s * kStageBytes + kABytes + kBBytes + kSfBytes; };
+    auto sf_buf = [&](int b, int ab) { return sSf + (size_t)(b * 2 + ab) * kSfGroupBytes; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -114,6 +128,7 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const CU
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars->acc_full[b], 1);
             mbar_init(&bars->acc_empty[b], 4);
+            mbar_init(&bars->sf_empty[b], 1);
         }
         mbar_init(&bars->done, 1);
         bars->abort_flag = 0;
@@ -136,38 +151,51 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const CU
         if (lane == 0) {
             // ---------------- TMA producer
             tma_prefetch_desc(&tmA);
-            tma_prefetch_desc(&tmB);
             int stage = 0;
             uint32_t phase = 0;
+            uint32_t groups = 0;  // scale-factor groups issued so far
             bool ok = true;
             int last_phase[kStages];
             for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
                 const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
                 const int4 ti = __ldg(p.tiles + mt);
-                const int n_abox = (ti.z + kABoxRows - 1) / kABoxRows;
-                const uint32_t tx = (uint32_t)n_abox * kABoxBytes + kBBytes + 2 * kSfBytes;
-                const uint8_t* sfa_src = p.sfa + ((size_t)(ti.y / kBM) * kb_count) * kSfBytes;
-                const uint8_t* sfb_src = p.sfb + ((size_t)ti.x * p.n_tiles + nt) * kb_count * kSfBytes;
+                const int n = tile_n(ti.z);
+                const CUtensorMap* mapB = &tmB.m[(n >> 5) - 1];
+                const int a_row = (int)((long long)ti.x * p.a_rows) + nt * kTileM;
+                const uint8_t* sfa_src = p.sfa + ((size_t)ti.x * p.n_tiles + nt) * kb_count * kSfBlock;
+                const uint8_t* sfb_src = p.sfb + (size_t)(ti.y / kBM) * kb_count * kSfBlock;
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!mbar_wait_bounded(&bars->empty[stage], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
                         ok = false;
                         break;
                     }
+                    uint32_t tx = kABytes + (uint32_t)n * kBK8;
+                    int gs = 0;
+                    if (kb % kSfGroup == 0) {
+                        // the scale blocks of this stage and the next gs-1 stages, once the MMAs
+                        // that read this buffer two groups ago are done
+                        const int sb = (int)(groups & 1u);
+                        if (!mbar_wait_bounded(&bars->sf_empty[sb], ((groups >> 1) & 1u) ^ 1u, abort_flag,
+                                               p.wait_limit_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        gs = kb_count - kb < kSfGroup ? kb_count - kb : kSfGroup;
+                        tx += 2u * (uint32_t)gs * kSfBlock;
+                    }
                     mbar_arrive_expect_tx(&bars->full[stage], tx);
                     last_phase[stage] = (int)phase;
-                    for (int i = 0; i < n_abox; ++i)
-                        tma_load_2d(stage_a(stage) + i * kABoxBytes, &tmA, &bars->full[stage], kb * kBK8,
-                                    ti.y + i * kABoxRows);
-                    if (kMode == 0) {
-                        tma_load_4d(stage_b(stage), &tmB, &bars->full[stage], kb * kBK8, nt * (kBN / 2), 0, ti.x);
-                        tma_load_4d(stage_b(stage) + kBBytes / 2, &tmB, &bars->full[stage], kb * kBK8, nt * (kBN / 2),
-                                    1, ti.x);
-                    } else {
-                        tma_load_3d(stage_b(stage), &tmB, &bars->full[stage], kb * kBK8, nt * kBN, ti.x);
+                    tma_load_2d(stage_a(stage), &tmA, &bars->full[stage], kb * kBK8, a_row);
+                    tma_load_2d(stage_b(stage), mapB, &bars->full[stage], kb * kBK8, ti.y);
+                    if (gs > 0) {
+                        const int sb = (int)(groups & 1u);
+                        bulk_load(sf_buf(sb, 0), sfa_src + (size_t)kb * kSfBlock, (uint32_t)gs * kSfBlock,
+                                  &bars->full[stage]);
+                        bulk_load(sf_buf(sb, 1), sfb_src + (size_t)kb * kSfBlock, (uint32_t)gs * kSfBlock,
+                                  &bars->full[stage]);
+                        ++groups;
                     }
-                    bulk_load(stage_sfa(stage), sfa_src + (size_t)kb * kSfBytes, kSfBytes, &bars->full[stage]);
-                    bulk_load(stage_sfb(stage), sfb_src + (size_t)kb * kSfBytes, kSfBytes, &bars->full[stage]);
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -190,11 +218,14 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const CU
             // ---------------- MMA issuer
             int stage = 0;
             uint32_t phase = 0;
+            uint32_t groups = 0;
             bool ok = true;
             int it = 0;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++it) {
                 const int buf = it & 1;
                 const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+                const int mt = t / p.n_tiles;
+                const int n = tile_n(__ldg(&p.tiles[mt].z));
                 if (!mbar_wait_bounded(&bars->acc_empty[buf], acc_phase ^ 1u, abort_flag, p.wait_limit_ns)) {
                     ok = false;
                     break;
@@ -207,19 +238,25 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const CU
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t sfa_t = tmem_base + kSfCol0 + (uint32_t)stage * 16u;
-                    const uint32_t sfb_t = sfa_t + 8u;
-                    tmem_cp_32x128b_warpx4(sfa_t, sdesc_sf(smem_u32(stage_sfa(stage))));
-                    tmem_cp_32x128b_warpx4(sfb_t, sdesc_sf(smem_u32(stage_sfb(stage))));
+                    const int sb = (int)(groups & 1u);
+                    const int gi = kb % kSfGroup;
+                    const uint32_t sfa_t = tmem_base + kSfCol0 + (uint32_t)stage * 8u;
+                    const uint32_t sfb_t = sfa_t + 4u;
+                    tmem_cp_32x128b_warpx4(sfa_t, sdesc_sf(smem_u32(sf_buf(sb, 0) + gi * kSfBlock)));
+                    tmem_cp_32x128b_warpx4(sfb_t, sdesc_sf(smem_u32(sf_buf(sb, 1) + gi * kSfBlock)));
                     const uint32_t a_addr = smem_u32(stage_a(stage));
                     const uint32_t b_addr = smem_u32(stage_b(stage));
 #pragma unroll
                     for (int kk = 0; kk < kBK8 / 32; ++kk) {
                         mma_mxf8_ss(d_tmem, sdesc_kmajor_sw128(a_addr + kk * 32), sdesc_kmajor_sw128(b_addr + kk * 32),
-                                    idesc_mxf8(128, kBN, (uint32_t)kk, (uint32_t)kk), sfa_t, sfb_t,
+                                    idesc_mxf8(kTileM, n, (uint32_t)kk, (uint32_t)kk), sfa_t, sfb_t,
                                     (kb | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit(&bars->empty[stage]);
+                    if (gi == kSfGroup - 1 || kb == kb_count - 1) {  // the group's scale blocks are consumed
+                        mma_commit(&bars->sf_empty[sb]);
+                        ++groups;
+                    }
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -238,18 +275,21 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const CU
         }
         __syncwarp();
     } else {
-        // ---------------- epilogue: warps 2..5, TMEM lane quadrant = warp % 4
+        // ---------------- epilogue: warps 2..5, TMEM lane quarter = warp % 4
         const int quad = warp & 3;
-        const int r = quad * 32 + lane;
+        const int et = threadIdx.x - 64;  // 0..127
         int it = 0;
-        uint32_t out_chunk = 0;
+        uint32_t chunk_count = 0;  // chunks staged so far (the staging buffer alternates)
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
             const int buf = it & 1;
             const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
             const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
             const int4 ti = __ldg(p.tiles + mt);
-            const bool got = __all_sync(0xffffffffu,
-                                        mbar_wait_bounded(&bars->acc_full[buf], acc_phase, abort_flag, p.wait_limit_ns));
+            const int nch = tile_n(ti.z) >> 5;
+            bool got = __all_sync(0xffffffffu,
+                                  mbar_wait_bounded(&bars->acc_full[buf], acc_phase, abort_flag, p.wait_limit_ns));
+            // the four warps decide together: the gate/up epilogue meets in a named barrier per chunk
+            if (kMode == 0) got = named_bar_and(kEpiBar, 128, got);
             if (!got) {
                 if (lane == 0) {
                     *abort_flag = 1;
@@ -258,71 +298,94 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const CU
                 break;
             }
             tc_fence_after_sync();
-            const bool valid = r < ti.z;
             const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)buf * kAccCols;
             if (kMode == 0) {
-                uint8_t* h_row = reinterpret_cast<uint8_t*>(p.out) + (size_t)(ti.y + r) * (size_t)p.out_ld;
-                uint8_t* hs_tile = p.out_scales + (size_t)(ti.y / kBM) * p.sf_ks_out * kSfBytes;
+                const bool lo = lane < 16;
+                const int fl = 16 * quad + (lane & 15);  // this lane's f within the tile's 64
+                uint8_t* hq = reinterpret_cast<uint8_t*>(p.out);
+                uint8_t* hs_tile = p.out_scales + (size_t)(ti.y / kBM) * p.sf_ks_out * kSfBlock;
+                // quantisation role: route qr of the chunk, 32-f block qb, half qh (16 f)
+                const int qr = et >> 2, qb = (et >> 1) & 1, qh = et & 1;
+                const int f_blk = nt * 64 + qb * 32;  // first f of the 32-f block
 #pragma unroll 1
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t g[32], u[32];
-                    tmem_ld_32x32b_x32(taddr + c * 32, g);
-                    tmem_ld_32x32b_x32(taddr + kBN / 2 + c * 32, u);
-                    tmem_ld_wait();
-                    const int f0 = nt * (kBN / 2) + c * 32;  // one MXFP8 block of h
-                    float h[32];
-                    float amax = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        h[i] = silu_f(__uint_as_float(g[i])) * __uint_as_float(u[i]);
-                        amax = fmaxf(amax, fabsf(h[i]));
-                    }
-                    float inv;
-                    const uint8_t sbyte = mxfp8_block_scale(amax, &inv);
-                    if (valid) {
-                        if (f0 < p.out_cols) {
-                            uint32_t w[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                w[i] = e4m3x2(h[4 * i + 1] * inv, h[4 * i] * inv) |
-                                       (e4m3x2(h[4 * i + 3] * inv, h[4 * i + 2] * inv) << 16);
-                            *reinterpret_cast<uint4*>(h_row + f0) = make_uint4(w[0], w[1], w[2], w[3]);
-                            *reinterpret_cast<uint4*>(h_row + f0 + 16) = make_uint4(w[4], w[5], w[6], w[7]);
-                        }
-                        hs_tile[(size_t)(f0 / 128) * kSfBytes + sf_block_offset(r, (f0 % 128) / 32)] = sbyte;
-                    }
-                }
-                // k-group slots of the down GEMM's last K stage that no gate/up tile covers hold scale 0
-                if (valid && nt == p.n_tiles - 1) {
-                    for (int g = 2 * p.n_tiles; g < 4 * p.sf_ks_out; ++g)
-                        hs_tile[(size_t)(g / 4) * kSfBytes + sf_block_offset(r, g % 4)] = 0;
-                }
-            } else {
-                const bool slice_live = quad * 32 < ti.z;
-                uint8_t* my_out = sOut + (size_t)quad * 2 * kStageOutBytes;
-#pragma unroll 1
-                for (int c = 0; c < kBN / 32; ++c) {
+                for (int c = 0; c < nch; ++c, ++chunk_count) {
+                    float* st = reinterpret_cast<float*>(sEpi + (chunk_count & 1u) * kStageHBytes);
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(taddr + c * 32, v);
                     tmem_ld_wait();
-                    const int c0 = nt * kBN + c * 32;
-                    if (slice_live && c0 < p.out_cols) {
-                        uint8_t* box = my_out + (out_chunk & 1) * kStageOutBytes;
-                        if (lane == 0) bulk_wait_group_read<1>();
+                    // h of (route (lo ? j : 16 + j), f = fl) into st[route][64 f]; the f index of
+                    // routes 16..31 is xor-ed with 16 so that the two half-warps hit different banks
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const uint32_t mine = lo ? v[j] : v[16 + j];
+                        const uint32_t other = __shfl_xor_sync(0xffffffffu, lo ? v[16 + j] : v[j], 16);
+                        const float g = __uint_as_float(lo ? mine : other);
+                        const float u = __uint_as_float(lo ? other : mine);
+                        const int route = lo ? j : 16 + j;
+                        st[route * 64 + (fl ^ (lo ? 0 : 16))] = silu_f(g) * u;
+                    }
+                    named_bar_sync(kEpiBar, 128);
+                    // quantise: 16 values of (route qr, block qb); the block's other half is lane ^ 1
+                    const float4* src =
+                        reinterpret_cast<const float4*>(st + qr * 64 + ((qb * 32 + qh * 16) ^ (qr >= 16 ? 16 : 0)));
+                    float h[16];
+                    float amax = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float4 w = src[i];
+                        h[4 * i] = w.x;
+                        h[4 * i + 1] = w.y;
+                        h[4 * i + 2] = w.z;
+                        h[4 * i + 3] = w.w;
+                        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(w.x), fabsf(w.y)), fmaxf(fabsf(w.z), fabsf(w.w))));
+                    }
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                    float inv;
+                    const uint8_t sbyte = mxfp8_block_scale(amax, &inv);
+                    const int route = c * 32 + qr;
+                    if (route < ti.z && f_blk < p.out_cols) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            w[i] = e4m3x2(h[4 * i + 1] * inv, h[4 * i] * inv) |
+                                   (e4m3x2(h[4 * i + 3] * inv, h[4 * i + 2] * inv) << 16);
+                        *reinterpret_cast<uint4*>(hq + (size_t)(ti.y + route) * (size_t)p.out_ld + f_blk + qh * 16) =
+                            make_uint4(w[0], w[1], w[2], w[3]);
+                        if (qh == 0)
+                            hs_tile[(size_t)(f_blk / 128) * kSfBlock + sf_block_offset(route, (f_blk % 128) / 32)] =
+                                sbyte;
+                    }
+                    // k-group slots of the down GEMM's last K stage that no f block covers hold scale 0
+                    if (route < ti.z && nt == p.n_tiles - 1 && qb == 0 && qh == 0) {
+                        for (int g = p.out_cols / 32; g < 4 * p.sf_ks_out; ++g)
+                            hs_tile[(size_t)(g / 4) * kSfBlock + sf_block_offset(route, g % 4)] = 0;
+                    }
+                }
+            } else {
+                // output columns of this warp: nt*128 + 32*quad + lane
+                const int c_base = nt * kTileM + 32 * quad;
+                float* y = reinterpret_cast<float*>(p.out);
+                uint8_t* tbuf = sEpi + (size_t)quad * kYTBytes;
+                if (c_base < p.out_cols) {
+                    const bool col_ok = c_base + (lane & 7) * 4 < p.out_cols;
+#pragma unroll 1
+                    for (int c = 0; c < nch; ++c) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(taddr + c * 32, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int r = 0; r < 32; ++r) *reinterpret_cast<uint32_t*>(tbuf + r * 128 + lane * 4) = v[r];
                         __syncwarp();
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const uint32_t off = (uint32_t)lane * 128u + (uint32_t)((q ^ (lane & 7)) * 16);
-                            *reinterpret_cast<uint4*>(box + off) =
-                                make_uint4(v[q * 4], v[q * 4 + 1], v[q * 4 + 2], v[q * 4 + 3]);
+                        for (int i = 0; i < 8; ++i) {
+                            const int r = i * 4 + (lane >> 3);
+                            const int route = c * 32 + r;
+                            const uint4 w = *reinterpret_cast<const uint4*>(tbuf + r * 128 + (lane & 7) * 16);
+                            if (col_ok && route < ti.z)
+                                *reinterpret_cast<uint4*>(y + (size_t)(ti.y + route) * (size_t)p.out_ld + c_base +
+                                                          (lane & 7) * 4) = w;
                         }
-                        fence_proxy_async_smem();
                         __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d(&tmOut, box, c0, ti.y + quad * 32);
-                            bulk_commit_group();
-                        }
-                        ++out_chunk;
                     }
                 }
             }
@@ -330,8 +393,6 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const CU
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
         }
-        if (kMode == 1 && lane == 0) bulk_wait_group<0>();
-        __syncwarp();
     }
 
     tc_fence_before_sync();
@@ -343,21 +404,21 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const CU
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    moe_gemm_gate_up_swiglu_mxfp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                                  const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
-    gemm_mxfp8_body<0>(tmA, tmB, tmOut, p);
+    moe_gemm_gate_up_swiglu_mxfp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BoxMaps8 tmB,
+                                  const GemmParams p) {
+    gemm_mxfp8_body<0>(tmA, tmB, p);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    moe_gemm_down_mxfp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
-    gemm_mxfp8_body<1>(tmA, tmB, tmOut, p);
+    moe_gemm_down_mxfp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BoxMaps8 tmB,
+                        const GemmParams p) {
+    gemm_mxfp8_body<1>(tmA, tmB, p);
 }
 
-using GemmKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, GemmParams);
+using GemmKernel = void (*)(CUtensorMap, BoxMaps8, GemmParams);
 
-cudaError_t launch_impl(GemmKernel kern, int* configured_device, const CUtensorMap& a, const CUtensorMap& b,
-                        const CUtensorMap& o, const GemmParams& gp, int grid, cudaStream_t s) {
+cudaError_t launch_impl(GemmKernel kern, int* configured_device, const CUtensorMap& a, const BoxMaps8& b,
+                        const GemmParams& gp, long long max_tiles, cudaStream_t s) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
@@ -366,22 +427,25 @@ cudaError_t launch_impl(GemmKernel kern, int* configured_device, const CUtensorM
         if (err != cudaSuccess) return err;
         *configured_device = dev;
     }
-    kern<<<grid, kThreads, kSmemBytes, s>>>(a, b, o, gp);
+    long long grid = num_sms();  // persistent: one CTA per SM
+    if (grid > max_tiles) grid = max_tiles;
+    if (grid < 1) grid = 1;
+    kern<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(a, b, gp);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_gemm1_mxfp8(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o,
-                               const GemmParams& gp, int grid, cudaStream_t s) {
+cudaError_t launch_gemm1_mxfp8(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
+                               cudaStream_t s) {
     static int configured = -1;
-    return launch_impl(moe_gemm_gate_up_swiglu_mxfp8, &configured, a, b, o, gp, grid, s);
+    return launch_impl(moe_gemm_gate_up_swiglu_mxfp8, &configured, a, b, gp, max_tiles, s);
 }
 
-cudaError_t launch_gemm2_mxfp8(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o,
-                               const GemmParams& gp, int grid, cudaStream_t s) {
+cudaError_t launch_gemm2_mxfp8(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
+                               cudaStream_t s) {
     static int configured = -1;
-    return launch_impl(moe_gemm_down_mxfp8, &configured, a, b, o, gp, grid, s);
+    return launch_impl(moe_gemm_down_mxfp8, &configured, a, b, gp, max_tiles, s);
 }
 
 }  // namespace moe

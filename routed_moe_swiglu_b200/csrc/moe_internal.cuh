@@ -67,9 +67,10 @@ struct moe_plan {
 
 namespace moe {
 
-// Tensor maps of one route-row operand with box heights 16, 32, ..., 128 rows
-// (entry i: 16 * (i + 1) rows), so that a tile of N routes loads its N/2 rows
-// per CTA of a pair with one TMA instruction.
+// Tensor maps of one route-row operand with several box heights, so that a
+// tile of N routes loads its rows with one TMA instruction: bf16 (CTA pairs)
+// entry i has 16 * (i + 1) rows (N/2 per CTA), MXFP8 entry i < 4 has
+// 32 * (i + 1) rows.
 struct BoxMaps8 {
     CUtensorMap m[8];
 };
@@ -86,9 +87,9 @@ struct GemmParams {
     int k_blocks;                   // pipeline stages per tile
     long long a_rows;               // bf16: rows of one expert in the weight operand's tensor map
     unsigned long long wait_limit_ns;
-    // MXFP8 only: scale blocks of A ([M tile][K stage][512 B]) and of B
-    // ([expert][N tile][K stage][512 B]); K stages of the down GEMM (the gate/up
-    // epilogue writes h's scales for it).
+    // MXFP8 only: scale blocks of A, the weights ([expert][weight tile][K stage][512 B]),
+    // and of B, the route rows ([128-row tile][K stage][512 B]); K stages of the down
+    // GEMM (the gate/up epilogue writes h's scales for it).
     const uint8_t* sfa;
     const uint8_t* sfb;
     int sf_ks_out;
@@ -118,10 +119,10 @@ cudaError_t launch_gemm1_bf16_pair(const CUtensorMap& a, const BoxMaps8& b, cons
                                    cudaStream_t s);
 cudaError_t launch_gemm2_bf16_pair(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
                                    cudaStream_t s);
-cudaError_t launch_gemm1_mxfp8(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o,
-                               const GemmParams& gp, int grid, cudaStream_t s);
-cudaError_t launch_gemm2_mxfp8(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o,
-                               const GemmParams& gp, int grid, cudaStream_t s);
+cudaError_t launch_gemm1_mxfp8(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
+                               cudaStream_t s);
+cudaError_t launch_gemm2_mxfp8(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
+                               cudaStream_t s);
 cudaError_t launch_prepare_bf16(const moe_plan* p, const __nv_bfloat16* wg, const __nv_bfloat16* wu,
                                 const __nv_bfloat16* wd, void* buf, cudaStream_t s);
 cudaError_t launch_prepare_mxfp8(const moe_plan* p, const __nv_bfloat16* wg, const __nv_bfloat16* wu,

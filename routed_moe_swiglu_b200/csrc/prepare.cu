@@ -65,10 +65,13 @@ namespace moe {
 namespace {
 
 // MXFP8 weights: one 128-thread block per weight row (grid-stride), blocks of
-// 32 along the row (the GEMM's K), codes in place of the bf16 layout and
-// scale bytes in the GEMMs' B scale blocks:
-//   gate/up row (e, g/u, f): N tile f / 64, tile row g/u * 64 + f % 64
-//   down row (e, c):         N tile c / 128, tile row c % 128
+// 32 along the row (the GEMM's K).  Codes:
+//   W1 [E][ceil(F/64)][4][2][16][H]  (as the bf16 W1: per 16 f the gate rows,
+//                                     then the up rows; 64 f per weight tile)
+//   W2 [E][H][F]
+// and scale bytes in the GEMMs' weight scale blocks ([tile][K stage][512 B]):
+//   gate/up row (e, g/u, f): tile f / 64, tile row (f % 64 / 16) * 32 + g/u * 16 + f % 16
+//   down row (e, c):         tile c / 128, tile row c % 128
 __global__ void __launch_bounds__(128) prepare_mxfp8_kernel(const uint4* __restrict__ wg, const uint4* __restrict__ wu,
                                                             const uint4* __restrict__ wd, uint2* __restrict__ w1q,
                                                             uint8_t* __restrict__ w1s, uint2* __restrict__ w2q,
@@ -86,9 +89,9 @@ __global__ void __launch_bounds__(128) prepare_mxfp8_kernel(const uint4* __restr
             const int rem = (int)(row - e * 2 * F);
             const int gu = rem / F, f = rem - gu * F;
             src = (gu ? wu : wg) + ((size_t)e * F + f) * (H / 8);
-            dst = w1q + (size_t)row * (H / 8);
+            trow = ((f % kG1BN8) >> 4) * 32 + gu * 16 + (f & 15);
+            dst = w1q + ((size_t)(e * nt1 + f / kG1BN8) * 128 + trow) * (H / 8);
             len = H;
-            trow = gu * (kG1BN8) + f % kG1BN8;
             sf_tile = w1s + ((size_t)e * nt1 + f / kG1BN8) * ks1 * kSfBlock;
         } else {
             const long long r2 = row - rows1;
@@ -122,8 +125,11 @@ cudaError_t launch_prepare_mxfp8(const moe_plan* p, const __nv_bfloat16* wg, con
                                  const __nv_bfloat16* wd, void* buf, cudaStream_t s) {
     uint8_t* base = static_cast<uint8_t*>(buf);
     const int E = p->d.num_experts, F = p->d.ffn, H = p->d.hidden;
-    // padding rows and k-groups of the scale blocks hold byte 0 (scale 2^-127)
+    // padding rows and k-groups of the scale blocks hold byte 0 (scale 2^-127), and the W1
+    // rows of f >= F (when F is not a multiple of 64) hold code 0
     cudaError_t err = cudaMemsetAsync(base + p->wb.w1s, 0, p->wb.w2 - p->wb.w1s, s);
+    if (err != cudaSuccess) return err;
+    if (F % kG1BN8 != 0) err = cudaMemsetAsync(base + p->wb.w1, 0, p->wb.w1s - p->wb.w1, s);
     if (err != cudaSuccess) return err;
     err = cudaMemsetAsync(base + p->wb.w2s, 0, p->wb.total - p->wb.w2s, s);
     if (err != cudaSuccess) return err;

@@ -38,30 +38,38 @@ def _ws_bytes(m: GpuMoe, ptr, nbytes):
     return m.ws[off:off + nbytes].cpu().numpy()
 
 
-def test_prepare_weights_bit_exact():
-    H, F, E = 256, 192, 3  # F not a multiple of 128: partial N tile and K stage
+@pytest.mark.parametrize("F", [192, 160])  # 160: a partial 64-f weight tile (zero rows) and K stage
+def test_prepare_weights_bit_exact(F):
+    H, E = 256, 3
     gen = torch.Generator().manual_seed(31)
     wg = (torch.randn((E, F, H), generator=gen) * torch.exp(torch.randn((E, F, 1), generator=gen))).bfloat16()
     wu = (torch.randn((E, F, H), generator=gen) * 0.1).bfloat16()
     wd = (torch.randn((E, H, F), generator=gen) * torch.exp(torch.randn((E, H, 1), generator=gen) * 3)).bfloat16()
     plan = rm.moe_plan_create(hidden=H, ffn=F, num_experts=E, top_k=2, capacity=16, precision="mxfp8")
     buf = rm.alloc_weight_buffer(plan)
+    buf.fill_(0x5A)  # stale contents: padding rows and scale slots must be rewritten
     rm.moe_prepare_weights(plan, wg.cuda(), wu.cuda(), wd.cuda(), buf)
     torch.cuda.synchronize()
     b = buf.cpu().numpy()
     gq, gs, uq, us, dq, ds = oracle.quantize_weights_mxfp8(wg, wu, wd)
-    n1 = E * 2 * F * H
-    w1 = b[:n1].reshape(E, 2, F, H)
-    assert np.array_equal(w1[:, 0], gq) and np.array_equal(w1[:, 1], uq)
+    # W1 codes: per 64-f tile, per 16 f, the 16 gate rows then the 16 up rows
+    f64 = (F + 63) // 64 * 64
+    n1 = E * 2 * f64 * H
+    w1 = b[:n1].reshape(E, f64 // 64, 4, 2, 16, H)
+    f = np.arange(F)
+    assert np.array_equal(w1[:, f // 64, (f % 64) // 16, 0, f % 16], gq)
+    assert np.array_equal(w1[:, f // 64, (f % 64) // 16, 1, f % 16], uq)
+    fpad = np.arange(F, f64)
+    assert np.all(w1[:, fpad // 64, (fpad % 64) // 16, :, fpad % 16] == 0)
     al = lambda x: (x + 255) // 256 * 256  # noqa: E731
     nt1, ks1 = (F + 63) // 64, (H + 127) // 128
     off_w1s = al(n1)
     w1s = b[off_w1s:off_w1s + E * nt1 * ks1 * SF_BLOCK]
     for e in range(E):
         for gu, ref in ((0, gs), (1, us)):
-            f = np.arange(F)
+            trow = ((f % 64) // 16) * 32 + gu * 16 + f % 16
             for g in range(H // 32):
-                idx = ((e * nt1 + f // 64) * ks1 + g // 4) * SF_BLOCK + sf_offset(gu * 64 + f % 64, g % 4)
+                idx = ((e * nt1 + f // 64) * ks1 + g // 4) * SF_BLOCK + sf_offset(trow, g % 4)
                 assert np.array_equal(w1s[idx], ref[e, :, g]), (e, gu, g)
     off_w2 = off_w1s + al(E * nt1 * ks1 * SF_BLOCK)
     w2 = b[off_w2:off_w2 + E * H * F].reshape(E, H, F)
@@ -123,6 +131,34 @@ def test_forward_mxfp8_small(H, F, E, k, T):
     assert_close(o[:T], ref, "mxfp8", f"mxfp8 {H},{F},{E},{k},{T}")
     assert np.all(np.isnan(o[T:]))
     _check_intermediates(m, x, ids, H, F, np.arange(T), h_ref)
+    assert m.status() == 0
+
+
+def test_mxfp8_every_tile_width():
+    """Caller routes that give experts 1..257 routes: every route-tile width
+    (N = 32..128 in steps of 32), full tiles followed by tails of 1, 31, 32 or
+    33 rows, a K tail (H = 320) and a partial 64-f weight tile (F = 224)."""
+    H, F, E, k = 320, 224, 17, 2
+    counts = np.array([1, 31, 32, 33, 63, 64, 65, 95, 96, 97, 127, 128, 129, 201, 255, 256, 257])
+    T = int(counts.sum()) // k
+    x, _, weights = workloads.small_case(H, F, E, k, T, seed=78)
+    gen = np.random.default_rng(78)
+    experts = np.repeat(np.arange(E), counts)
+    ids = np.stack([experts[:T], experts[T:]], axis=1)
+    ids = ids[gen.permutation(T)].astype(np.int32)
+    assert np.all(ids[:, 0] != ids[:, 1])
+    p = gen.uniform(0.1, 1.0, size=(T, k))
+    probs = (p / p.sum(axis=1, keepdims=True)).astype(np.float32)
+    m = GpuMoe(H, F, E, k, T, weights, precision="mxfp8")
+    out = m.forward(x.cuda(), T, ids=torch.from_numpy(ids).cuda(), probs=torch.from_numpy(probs).cuda())
+    torch.cuda.synchronize()
+    ids_c = np.sort(ids, axis=1)
+    order = np.argsort(ids, axis=1)
+    probs_c = np.take_along_axis(probs, order, axis=1)
+    wq = oracle.quantize_weights_mxfp8(*weights)
+    ref, h_ref = oracle.forward_mxfp8(x, ids_c, probs_c, wq, want_h=True)
+    assert_close(out.cpu().numpy(), ref, "mxfp8", "mxfp8 every tile width")
+    _check_intermediates(m, x, ids_c, H, F, np.arange(T), h_ref)
     assert m.status() == 0
 
 
