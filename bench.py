@@ -189,24 +189,28 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+_CSRC = "routed_moe_swiglu_b200/csrc/"
 KERNEL_SOURCES = {
-    "gemm_gate_up": ["routed_moe_swiglu_b200/csrc/gemm_bf16_pair.cu", "routed_moe_swiglu_b200/csrc/ptx.cuh",
-                     "routed_moe_swiglu_b200/csrc/moe_internal.cuh"],
-    "gemm_down": ["routed_moe_swiglu_b200/csrc/gemm_bf16_pair.cu", "routed_moe_swiglu_b200/csrc/ptx.cuh",
-                  "routed_moe_swiglu_b200/csrc/moe_internal.cuh"],
-    "combine": ["routed_moe_swiglu_b200/csrc/permute.cu", "routed_moe_swiglu_b200/csrc/moe_internal.cuh"],
+    ("gemm_gate_up", "bf16"): [_CSRC + "gemm_bf16_pair.cu", _CSRC + "ptx.cuh", _CSRC + "moe_internal.cuh"],
+    ("gemm_down", "bf16"): [_CSRC + "gemm_bf16_pair.cu", _CSRC + "ptx.cuh", _CSRC + "moe_internal.cuh"],
+    ("gemm_gate_up", "mxfp8"): [_CSRC + "gemm_mxfp8.cu", _CSRC + "mxfp8.cuh", _CSRC + "ptx.cuh",
+                                _CSRC + "moe_internal.cuh"],
+    ("gemm_down", "mxfp8"): [_CSRC + "gemm_mxfp8.cu", _CSRC + "mxfp8.cuh", _CSRC + "ptx.cuh",
+                             _CSRC + "moe_internal.cuh"],
+    ("combine", "bf16"): [_CSRC + "permute.cu", _CSRC + "moe_internal.cuh"],
+    ("combine", "mxfp8"): [_CSRC + "permute.cu", _CSRC + "moe_internal.cuh"],
 }
 
 
-def source_hash(stage):
+def source_hash(stage, precision):
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES.get(stage, []):
+    for rel in KERNEL_SOURCES.get((stage, precision), []):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(stage, workload):
+def recorded_traffic(stage, workload, precision):
     """DRAM bytes per launch from a committed ncu summary, if the kernel's
     sources are unchanged since it was taken (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -215,7 +219,7 @@ def recorded_traffic(stage, workload):
     with open(p) as f:
         d = json.load(f)
     rec = d.get(f"{stage}@{workload}")
-    if not rec or rec.get("source_sha") != source_hash(stage):
+    if not rec or rec.get("source_sha") != source_hash(stage, precision):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -423,7 +427,7 @@ def roofline(w, res, peaks):
     out["frac"] = out["achieved"] / out["peak"]
     out["peak_source"] = peaks["source"]
     out["kernel_ms"] = ms
-    tr = recorded_traffic(dom, w.name)
+    tr = recorded_traffic(dom, w.name, w.precision)
     out["traffic"] = tr
     return out
 
