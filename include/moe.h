@@ -214,10 +214,10 @@ moe_status moe_forward_with_events(const moe_plan* plan, const void* x, const fl
  *   inv     int32 [max_live, k]: padded intermediate row of route (t, j)
  *   pad_offsets int32 [E+1]: first padded intermediate row of each expert,
  *           a multiple of 32 (bf16) or 128 (MXFP8)
- *   h       intermediate rows (bf16 [rows_padded, ceil(F/128)*128], the
- *           columns past F zero; or E4M3 codes [rows_padded, F] in MXFP8)
- *   xq      permuted x rows (bf16 [rows_padded, ceil(H/128)*128], the
- *           columns past H zero; or E4M3 codes [rows_padded, H])
+ *   h       intermediate rows [rows_padded, ceil(F/128)*128], bf16 or
+ *           E4M3 codes, the columns past F zero
+ *   xq      permuted x rows [rows_padded, ceil(H/128)*128], bf16 or E4M3
+ *           codes, the columns past H zero
  *   h_scales, xq_scales  MXFP8 only (else NULL): E8M0 bytes in blocks of
  *           512 bytes, one per (128-row tile, K stage of 128 elements),
  *           block index tile * ceil(K/128) + stage; inside a block the byte

@@ -65,7 +65,7 @@ bool make_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, cons
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 static void compute_layouts(moe_plan* p) {
-    const size_t H = (size_t)p->d.hidden, F = (size_t)p->d.ffn, E = (size_t)p->d.num_experts;
+    const size_t H = (size_t)p->d.hidden, E = (size_t)p->d.num_experts;
     const size_t k = (size_t)p->d.top_k;
     const size_t L = (size_t)p->max_live;
     const size_t R = (size_t)p->rows_pad;
@@ -88,9 +88,9 @@ static void compute_layouts(moe_plan* p) {
     w.inv = take(L * k * 4);
     const size_t mtiles = (size_t)p->max_m_tiles;
     if (fp8) {
-        w.xq = take(R * H);
+        w.xq = take(R * (size_t)p->hp);
         w.xs = take(mtiles * p->ks1 * kSfBlock);
-        w.h = take(R * F);
+        w.h = take(R * (size_t)p->fp);
         w.hs = take(mtiles * p->ks2 * kSfBlock);
     } else {
         w.xq = take(R * (size_t)p->hp * 2);
@@ -104,9 +104,9 @@ static void compute_layouts(moe_plan* p) {
     WbufLayout& b = p->wb;
     off = 0;
     if (fp8) {
-        b.w1 = take(E * 2 * ((F + 63) / 64 * 64) * H);  // W1 rows padded to whole 64-f blocks
+        b.w1 = take(E * 2 * (size_t)p->fp * (size_t)p->hp);
         b.w1s = take(E * p->nt1 * p->ks1 * kSfBlock);
-        b.w2 = take(E * H * F);
+        b.w2 = take(E * H * (size_t)p->fp);
         b.w2s = take(E * p->nt2 * p->ks2 * kSfBlock);
     } else {
         b.w1 = take(E * 2 * (size_t)p->fp * (size_t)p->hp * 2);
@@ -166,19 +166,19 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     p->rows_pad = d.precision == MOE_MXFP8 ? p->max_m_tiles * p->tile_rows
                                            : p->max_routes + (long long)d.num_experts * p->row_align;
     p->nblk = (int)((p->max_live + kTokPerBlk - 1) / kTokPerBlk);
+    // K in blocks of 128 elements (bf16: the GEMMs' K stage; MXFP8: the unit of the scale
+    // blocks, two per K stage); K pitches padded to whole blocks with zeros
+    p->ks1 = (d.hidden + 127) / 128;
+    p->ks2 = (d.ffn + 127) / 128;
+    p->hp = (long long)p->ks1 * 128;
+    p->fp = (long long)p->ks2 * 128;
     if (d.precision == MOE_MXFP8) {
-        p->ks1 = (d.hidden + kBK8 - 1) / kBK8;
-        p->ks2 = (d.ffn + kBK8 - 1) / kBK8;
-        p->nt1 = (d.ffn + kG1BN8 - 1) / kG1BN8;
+        p->nt1 = (int)(p->fp / kG1BN8);  // f tiles of 64 cover fp; h's padding columns come out zero
         p->nt2 = (d.hidden + kG2BN8 - 1) / kG2BN8;
     } else {
-        p->ks1 = (d.hidden + 2 * kBK - 1) / (2 * kBK);  // K stages of 128 elements
-        p->ks2 = (d.ffn + 2 * kBK - 1) / (2 * kBK);
-        p->nt1 = p->ks2;  // f tiles of 128 cover the padded F (fp); h's padding columns come out zero
+        p->nt1 = (int)(p->fp / kG1BN);  // f tiles of 128 cover fp
         p->nt2 = (d.hidden + kG2BN - 1) / kG2BN;
     }
-    p->hp = d.precision == MOE_MXFP8 ? d.hidden : (long long)p->ks1 * 2 * kBK;
-    p->fp = d.precision == MOE_MXFP8 ? d.ffn : (long long)p->ks2 * 2 * kBK;
     compute_layouts(p);
     *plan_out = p;
     return MOE_OK;
@@ -260,7 +260,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
         return stage_events == nullptr ||
                cudaEventRecordWithFlags(static_cast<cudaEvent_t>(stage_events[i]), s, record_flags) == cudaSuccess;
     };
-    const int H = plan->d.hidden, F = plan->d.ffn, E = plan->d.num_experts, k = plan->d.top_k;
+    const int H = plan->d.hidden, E = plan->d.num_experts, k = plan->d.top_k;
     const int max_live = (int)plan->max_live;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const uint8_t* wb = static_cast<const uint8_t*>(kernel_buf);
@@ -272,29 +272,30 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     // TMA descriptors for this call's buffers (host-side encoding only)
     const bool fp8 = plan->d.precision == MOE_MXFP8;
     const unsigned long long R = (unsigned long long)plan->rows_pad;
-    const unsigned long long uH = (unsigned long long)H, uF = (unsigned long long)F, uE = (unsigned long long)E;
+    const unsigned long long uH = (unsigned long long)H, uE = (unsigned long long)E;
     const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     CUtensorMap tA1, tA2;  // weight operands
     BoxMaps8 rB1, rB2;     // route-row operands (x rows, h rows)
     if (fp8) {
-        // MXFP8 (one CTA per tile): weights (A) load 128 rows, route rows (B) N <= 128 rows,
-        // one map per N in {32, 64, 96, 128}; K stage = 128 E4M3 elements (one 128-byte swizzle
-        // atom); K past H / F is the maps' zero fill
-        const unsigned long long f64 = (uF + 63) / 64 * 64;
-        const unsigned box128[2] = {(unsigned)kBK8, 128};
-        const unsigned long long dW1[2] = {uH, uE * 2ull * f64};
-        const unsigned long long sW1[1] = {uH};
-        const unsigned long long dW2[2] = {uF, uE * uH};
-        const unsigned long long sW2[1] = {uF};
-        const unsigned long long dX[2] = {uH, R};
-        const unsigned long long dH[2] = {uF, R};
-        if (!make_tensor_map(&tA1, dt, 2, wb + plan->wb.w1, dW1, sW1, box128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tA2, dt, 2, wb + plan->wb.w2, dW2, sW2, box128, CU_TENSOR_MAP_SWIZZLE_128B))
+        // MXFP8 (one CTA per tile): K stage = 256 E4M3 elements = two 128-byte swizzle atoms;
+        // the maps address element k of a row as (k % 128, row, k / 128), so a box lands as
+        // [atom][row][128 bytes].  Weights (A) load 128 rows, route rows (B) N <= 128 rows, one
+        // map per N in {32, 64, 96, 128}; the K pitches hp, fp are padded to 128 with zeros.
+        const unsigned long long hp = (unsigned long long)plan->hp, fpp = (unsigned long long)plan->fp;
+        const unsigned box128[3] = {128, 128, 2};
+        const unsigned long long dW1[3] = {128ull, uE * 2ull * fpp, hp / 128};
+        const unsigned long long sW1[2] = {hp, 128ull};
+        const unsigned long long dW2[3] = {128ull, uE * uH, fpp / 128};
+        const unsigned long long sW2[2] = {fpp, 128ull};
+        const unsigned long long dX[3] = {128ull, R, hp / 128};
+        const unsigned long long dH[3] = {128ull, R, fpp / 128};
+        if (!make_tensor_map(&tA1, dt, 3, wb + plan->wb.w1, dW1, sW1, box128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tA2, dt, 3, wb + plan->wb.w2, dW2, sW2, box128, CU_TENSOR_MAP_SWIZZLE_128B))
             return MOE_ERR_CUDA;
         for (int i = 0; i < 4; ++i) {
-            const unsigned box[2] = {(unsigned)kBK8, 32u * (unsigned)(i + 1)};
-            if (!make_tensor_map(&rB1.m[i], dt, 2, ws + L.xq, dX, sW1, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-                !make_tensor_map(&rB2.m[i], dt, 2, ws + L.h, dH, sW2, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            const unsigned box[3] = {128, 32u * (unsigned)(i + 1), 2};
+            if (!make_tensor_map(&rB1.m[i], dt, 3, ws + L.xq, dX, sW1, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+                !make_tensor_map(&rB2.m[i], dt, 3, ws + L.h, dH, sW2, box, CU_TENSOR_MAP_SWIZZLE_128B))
                 return MOE_ERR_CUDA;
         }
     } else {
@@ -341,7 +342,8 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
 
     if (!mark(2)) return MOE_ERR_CUDA;
     if (fp8)
-        e = launch_gather_mxfp8(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, k, inv, ws + L.xq,
+        e = launch_gather_mxfp8(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, (int)plan->hp, k,
+                                inv, ws + L.xq,
                                 ws + L.xs, s);
     else
         e = launch_gather_bf16(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, (int)plan->hp, k, inv,
@@ -356,8 +358,8 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g1.out = ws + L.h;
     g1.out_scales = nullptr;
     g1.out_ld = plan->fp;  // h rows: F values + zero padding to the down GEMM's K pitch
-    g1.out_cols = fp8 ? F : (int)plan->fp;
-    g1.a_rows = fp8 ? 2 * ((F + 63) / 64 * 64) : 2 * plan->fp;  // W1 rows of an expert (padded F)
+    g1.out_cols = (int)plan->fp;  // every padded column: f >= F are zero-weight rows, h = 0
+    g1.a_rows = 2 * plan->fp;     // W1 rows of an expert (padded F)
     g1.n_tiles = plan->nt1;
     g1.k_blocks = plan->ks1;
     g1.wait_limit_ns = kWaitLimitNs;

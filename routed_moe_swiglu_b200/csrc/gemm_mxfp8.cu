@@ -21,14 +21,20 @@
 //   down:     A = 128 rows of W_down[e] (output columns), B = N route rows of
 //             h codes; fp32 y rows leave through a shared-memory transpose.
 //
+// A K stage is 256 elements: two 128-byte swizzle atoms, 8 MMAs, and each
+// operand of a stage one TMA instruction (a 3-D map whose third dimension
+// walks the atoms of a row; the K pitches are padded to 128 with zeros).
+// Fewer, larger stages matter here: the per-stage fixed cost (barrier
+// hand-offs, commits, TMA issue) dominated with 128-element stages.
+//
 // Scale factors: for each 128-row operand tile (a weight tile, or the 128
-// padded route rows a route tile lies in) and K stage of 128 elements, 512
+// padded route rows a route tile lies in) and K block of 128 elements, 512
 // bytes laid out as [row % 32][row / 32][k-group], which one tcgen05.cp
 // (32x128b, replicated to the 4 lane quarters) moves to 4 TMEM columns; MMA
 // k-group kk selects byte kk of each 32-bit cell.  The blocks of 8
-// consecutive K stages of a tile are contiguous, so they arrive with one
-// bulk copy per operand into a double-buffered shared-memory area, and the
-// MMA thread moves each stage's blocks to TMEM just before its MMAs.
+// consecutive K blocks (4 stages) of a tile are contiguous, so they arrive
+// with one bulk copy per operand into a double-buffered shared-memory area,
+// and the MMA thread moves each stage's blocks to TMEM just before its MMAs.
 //
 // Pipeline: persistent CTA per SM, warp 0 TMA, warp 1 MMA + TMEM owner,
 // warps 2-5 epilogue; two 128-column accumulators; one scale-factor TMEM
@@ -42,25 +48,29 @@
 namespace moe {
 namespace {
 
-constexpr int kStages = 6;
+constexpr int kStages = 3;
 constexpr int kThreads = 192;
 constexpr int kTileM = 128;                            // weight rows per tile
 constexpr int kMaxN = 128;                             // routes per tile
-constexpr uint32_t kABytes = kTileM * kBK8;            // 16 KB
-constexpr uint32_t kBBytes = kMaxN * kBK8;             // up to 16 KB
+constexpr int kAtoms = 2;                              // 128-element K blocks (swizzle atoms) per stage
+constexpr uint32_t kAtomBytesA = kTileM * kBK8;        // 16 KB
+constexpr uint32_t kABytes = kAtoms * kAtomBytesA;     // 32 KB
+constexpr uint32_t kBBytes = kAtoms * kMaxN * kBK8;    // up to 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr int kSfGroup = 8;                            // K stages per scale-factor bulk copy
+constexpr int kSfGroup = 8;                            // K blocks per scale-factor bulk copy (4 stages)
+constexpr int kStagesPerGroup = kSfGroup / kAtoms;
 constexpr uint32_t kSfGroupBytes = kSfGroup * kSfBlock;
-constexpr uint32_t kSfBytes = 2 * 2 * kSfGroupBytes;   // [buffer][A/B][8 stages][512 B]
+constexpr uint32_t kSfBytes = 2 * 2 * kSfGroupBytes;   // [buffer][A/B][8 blocks][512 B]
 constexpr uint32_t kAccCols = kMaxN;
 constexpr uint32_t kSfCol0 = 2 * kAccCols;             // first scale-factor TMEM column
+constexpr uint32_t kSfColsPerStage = 16;               // per atom: A 4 columns, B 4 columns
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kStageHBytes = 32 * 64 * 4;         // gate/up: fp32 h of 32 routes x 64 f
 constexpr uint32_t kYTBytes = 32 * 32 * 4;             // down: fp32 y of 32 routes x 32 columns, per warp
 constexpr uint32_t kEpiBytes = 2 * kStageHBytes > 4 * kYTBytes ? 2 * kStageHBytes : 4 * kYTBytes;
 constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kSfBytes + kEpiBytes + 256;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kSfCol0 + 8 * kStages <= kTmemCols, "TMEM budget");
+static_assert(kSfCol0 + kSfColsPerStage * kStages <= kTmemCols, "TMEM budget");
 constexpr uint32_t kEpiBar = 1;                        // named barrier of the 4 epilogue warps
 
 struct __align__(8) Barriers {
@@ -145,7 +155,8 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
 
     const int num_m = (int)p.status_words[kStNumMTiles];
     const int total_tiles = num_m * p.n_tiles;
-    const int kb_count = p.k_blocks;
+    const int nblk = p.k_blocks;               // K blocks of 128
+    const int kb_count = (nblk + 1) / kAtoms;  // stages of 256 (the last may hold one block)
 
     if (warp == 0) {
         if (lane == 0) {
@@ -163,16 +174,18 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                 const int n = tile_n(ti.z);
                 const CUtensorMap* mapB = &tmB.m[(n >> 5) - 1];
                 const int a_row = (int)((long long)ti.x * p.a_rows) + nt * kTileM;
-                const uint8_t* sfa_src = p.sfa + ((size_t)ti.x * p.n_tiles + nt) * kb_count * kSfBlock;
-                const uint8_t* sfb_src = p.sfb + (size_t)(ti.y / kBM) * kb_count * kSfBlock;
+                const uint8_t* sfa_src = p.sfa + ((size_t)ti.x * p.n_tiles + nt) * nblk * kSfBlock;
+                const uint8_t* sfb_src = p.sfb + (size_t)(ti.y / kBM) * nblk * kSfBlock;
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!mbar_wait_bounded(&bars->empty[stage], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
                         ok = false;
                         break;
                     }
-                    uint32_t tx = kABytes + (uint32_t)n * kBK8;
+                    // both atoms' bytes count even where the second lies past K (zero fill)
+                    uint32_t tx = kABytes + (uint32_t)n * (kAtoms * kBK8);
                     int gs = 0;
-                    if (kb % kSfGroup == 0) {
+                    const int blk0 = kb * kAtoms;
+                    if (kb % kStagesPerGroup == 0) {
                         // the scale blocks of this stage and the next gs-1 stages, once the MMAs
                         // that read this buffer two groups ago are done
                         const int sb = (int)(groups & 1u);
@@ -181,18 +194,18 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                             ok = false;
                             break;
                         }
-                        gs = kb_count - kb < kSfGroup ? kb_count - kb : kSfGroup;
+                        gs = nblk - blk0 < kSfGroup ? nblk - blk0 : kSfGroup;
                         tx += 2u * (uint32_t)gs * kSfBlock;
                     }
                     mbar_arrive_expect_tx(&bars->full[stage], tx);
                     last_phase[stage] = (int)phase;
-                    tma_load_2d(stage_a(stage), &tmA, &bars->full[stage], kb * kBK8, a_row);
-                    tma_load_2d(stage_b(stage), mapB, &bars->full[stage], kb * kBK8, ti.y);
+                    tma_load_3d(stage_a(stage), &tmA, &bars->full[stage], 0, a_row, blk0);
+                    tma_load_3d(stage_b(stage), mapB, &bars->full[stage], 0, ti.y, blk0);
                     if (gs > 0) {
                         const int sb = (int)(groups & 1u);
-                        bulk_load(sf_buf(sb, 0), sfa_src + (size_t)kb * kSfBlock, (uint32_t)gs * kSfBlock,
+                        bulk_load(sf_buf(sb, 0), sfa_src + (size_t)blk0 * kSfBlock, (uint32_t)gs * kSfBlock,
                                   &bars->full[stage]);
-                        bulk_load(sf_buf(sb, 1), sfb_src + (size_t)kb * kSfBlock, (uint32_t)gs * kSfBlock,
+                        bulk_load(sf_buf(sb, 1), sfb_src + (size_t)blk0 * kSfBlock, (uint32_t)gs * kSfBlock,
                                   &bars->full[stage]);
                         ++groups;
                     }
@@ -239,21 +252,28 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                     }
                     tc_fence_after_sync();
                     const int sb = (int)(groups & 1u);
-                    const int gi = kb % kSfGroup;
-                    const uint32_t sfa_t = tmem_base + kSfCol0 + (uint32_t)stage * 8u;
-                    const uint32_t sfb_t = sfa_t + 4u;
-                    tmem_cp_32x128b_warpx4(sfa_t, sdesc_sf(smem_u32(sf_buf(sb, 0) + gi * kSfBlock)));
-                    tmem_cp_32x128b_warpx4(sfb_t, sdesc_sf(smem_u32(sf_buf(sb, 1) + gi * kSfBlock)));
+                    const int blk0 = kb * kAtoms;
+                    const int nb = nblk - blk0 < kAtoms ? nblk - blk0 : kAtoms;  // K blocks in this stage
                     const uint32_t a_addr = smem_u32(stage_a(stage));
                     const uint32_t b_addr = smem_u32(stage_b(stage));
+                    const uint32_t b_atom = (uint32_t)n * kBK8;  // bytes of one atom of the B box
+                    for (int h = 0; h < nb; ++h) {
+                        const int gi = (blk0 + h) % kSfGroup;
+                        const uint32_t sfa_t = tmem_base + kSfCol0 + (uint32_t)stage * kSfColsPerStage + (uint32_t)h * 8u;
+                        const uint32_t sfb_t = sfa_t + 4u;
+                        tmem_cp_32x128b_warpx4(sfa_t, sdesc_sf(smem_u32(sf_buf(sb, 0) + gi * kSfBlock)));
+                        tmem_cp_32x128b_warpx4(sfb_t, sdesc_sf(smem_u32(sf_buf(sb, 1) + gi * kSfBlock)));
+                        const uint32_t a_h = a_addr + (uint32_t)h * kAtomBytesA;
+                        const uint32_t b_h = b_addr + (uint32_t)h * b_atom;
 #pragma unroll
-                    for (int kk = 0; kk < kBK8 / 32; ++kk) {
-                        mma_mxf8_ss(d_tmem, sdesc_kmajor_sw128(a_addr + kk * 32), sdesc_kmajor_sw128(b_addr + kk * 32),
-                                    idesc_mxf8(kTileM, n, (uint32_t)kk, (uint32_t)kk), sfa_t, sfb_t,
-                                    (kb | kk) != 0 ? 1u : 0u);
+                        for (int kk = 0; kk < kBK8 / 32; ++kk) {
+                            mma_mxf8_ss(d_tmem, sdesc_kmajor_sw128(a_h + kk * 32), sdesc_kmajor_sw128(b_h + kk * 32),
+                                        idesc_mxf8(kTileM, n, (uint32_t)kk, (uint32_t)kk), sfa_t, sfb_t,
+                                        (kb | h | kk) != 0 ? 1u : 0u);
+                        }
                     }
                     mma_commit(&bars->empty[stage]);
-                    if (gi == kSfGroup - 1 || kb == kb_count - 1) {  // the group's scale blocks are consumed
+                    if (kb % kStagesPerGroup == kStagesPerGroup - 1 || kb == kb_count - 1) {  // group consumed
                         mma_commit(&bars->sf_empty[sb]);
                         ++groups;
                     }
@@ -354,11 +374,6 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                         if (qh == 0)
                             hs_tile[(size_t)(f_blk / 128) * kSfBlock + sf_block_offset(route, (f_blk % 128) / 32)] =
                                 sbyte;
-                    }
-                    // k-group slots of the down GEMM's last K stage that no f block covers hold scale 0
-                    if (route < ti.z && nt == p.n_tiles - 1 && qb == 0 && qh == 0) {
-                        for (int g = p.out_cols / 32; g < 4 * p.sf_ks_out; ++g)
-                            hs_tile[(size_t)(g / 4) * kSfBlock + sf_block_offset(route, g % 4)] = 0;
                     }
                 }
             } else {

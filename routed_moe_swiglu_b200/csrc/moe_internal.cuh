@@ -58,8 +58,8 @@ struct moe_plan {
     int tile_rows;          // most routes per tile: 256 (bf16, N of a pair MMA) or 128 (MXFP8, M of the MMA)
     int row_align;          // each expert's route rows start on a multiple of this: 32 (bf16) or 128 (MXFP8)
     long long hp, fp;       // K row pitch (elements) of x / gate-up rows and of h / down rows:
-                            // bf16 pads H and F to multiples of 128 with zeros; MXFP8 keeps H, F
-    int ks1, ks2;           // K stages of the gate/up and down GEMMs
+                            // H and F padded to multiples of 128 with zeros
+    int ks1, ks2;           // K blocks of 128 elements of the gate/up and down GEMMs
     int nt1, nt2;           // weight (bf16) / N (MXFP8) tiles of the gate/up and down GEMMs
     moe::WsLayout ws;
     moe::WbufLayout wb;
@@ -111,7 +111,7 @@ cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* 
                            cudaStream_t s);
 cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
                                const int* inv, __nv_bfloat16* xp, cudaStream_t s);
-cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int k,
+cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
                                 const int* inv, uint8_t* xq, uint8_t* xs, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const int* inv, const float* probs, const int* live, int max_live,
                            int H, int k, float* out, cudaStream_t s);

@@ -192,35 +192,37 @@ __global__ void __launch_bounds__(kRowThreads) gather_rows_bf16_kernel(const uin
 
 // MXFP8 gather: one 128-thread block per token quantises the token's x row
 // once (blocks of 32 along H, 4 threads per block) and writes the E4M3 codes
-// to each of its k padded route rows and the E8M0 bytes into the scale
-// blocks of those rows' M tiles ([tile][K stage][512 B]).
+// to each of its k padded route rows (pitch hp, zero codes past H) and the
+// E8M0 bytes into the scale blocks of those rows' 128-row tiles
+// ([tile][K block of 128][512 B]).
 __global__ void __launch_bounds__(kRowThreads) gather_rows_mxfp8_kernel(const uint4* __restrict__ x,
                                                                         const int* __restrict__ live, int max_live,
-                                                                        int H, int k, int ks1,
+                                                                        int H, int hp, int k, int ks1,
                                                                         const int* __restrict__ inv,
                                                                         uint2* __restrict__ xq,
                                                                         uint8_t* __restrict__ xs) {
     __shared__ int s_prow[kMaxTopK];
     const int n = clamp_live(live, max_live);
-    const int chunks = H / 8;
+    const int chunks = H / 8;       // 8 elements per thread and chunk
+    const int chunks_out = hp / 8;  // destination pitch
     for (int t = blockIdx.x; t < n; t += gridDim.x) {
         __syncthreads();
         if (threadIdx.x < k) s_prow[threadIdx.x] = __ldg(inv + (size_t)t * k + threadIdx.x);
         __syncthreads();
         const uint4* src = x + (size_t)t * chunks;
-        for (int c0 = 0; c0 < chunks; c0 += kRowThreads) {  // uniform trip count: shuffles inside
+        for (int c0 = 0; c0 < chunks_out; c0 += kRowThreads) {  // uniform trip count: shuffles inside
             const int c = c0 + threadIdx.x;
             const bool active = c < chunks;  // H % 32 == 0: 4-thread groups are all in or all out
             const uint4 v = active ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
             uint8_t sb;
-            const uint2 codes = mxfp8_quantize_8(v, &sb);
-            if (active) {
+            const uint2 codes = mxfp8_quantize_8(v, &sb);  // zero codes past H
+            if (c < chunks_out) {
                 const int g = c >> 2;  // 32-element block index along H
                 for (int j = 0; j < k; ++j) {
                     const int pr = s_prow[j];
                     if (pr < 0) continue;
-                    xq[(size_t)pr * chunks + c] = codes;
-                    if ((c & 3) == 0)
+                    xq[(size_t)pr * chunks_out + c] = codes;
+                    if (active && (c & 3) == 0)
                         xs[((size_t)(pr / kBM) * ks1 + g / 4) * kSfBlock + sf_block_offset(pr % kBM, g % 4)] = sb;
                 }
             }
@@ -332,11 +334,11 @@ cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_
     return cudaGetLastError();
 }
 
-cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int k,
+cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
                                 const int* inv, uint8_t* xq, uint8_t* xs, cudaStream_t s) {
     const int grid = grid_for_warps(max_live, 1, 16);
-    gather_rows_mxfp8_kernel<<<grid, kRowThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), live, max_live, H, k,
-                                                          (H + kBK8 - 1) / kBK8, inv, reinterpret_cast<uint2*>(xq), xs);
+    gather_rows_mxfp8_kernel<<<grid, kRowThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), live, max_live, H, hp, k,
+                                                          hp / 128, inv, reinterpret_cast<uint2*>(xq), xs);
     return cudaGetLastError();
 }
 

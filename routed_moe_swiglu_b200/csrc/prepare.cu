@@ -65,18 +65,20 @@ namespace moe {
 namespace {
 
 // MXFP8 weights: one 128-thread block per weight row (grid-stride), blocks of
-// 32 along the row (the GEMM's K).  Codes:
-//   W1 [E][ceil(F/64)][4][2][16][H]  (as the bf16 W1: per 16 f the gate rows,
-//                                     then the up rows; 64 f per weight tile)
-//   W2 [E][H][F]
+// 32 along the row (the GEMM's K).  Codes, K pitches hp, fp = H, F rounded up
+// to 128 with zero padding:
+//   W1 [E][fp/64][4][2][16][hp]  (as the bf16 W1: per 16 f the gate rows,
+//                                 then the up rows; 64 f per weight tile;
+//                                 rows of f >= F zero)
+//   W2 [E][H][fp]
 // and scale bytes in the GEMMs' weight scale blocks ([tile][K stage][512 B]):
 //   gate/up row (e, g/u, f): tile f / 64, tile row (f % 64 / 16) * 32 + g/u * 16 + f % 16
 //   down row (e, c):         tile c / 128, tile row c % 128
 __global__ void __launch_bounds__(128) prepare_mxfp8_kernel(const uint4* __restrict__ wg, const uint4* __restrict__ wu,
                                                             const uint4* __restrict__ wd, uint2* __restrict__ w1q,
                                                             uint8_t* __restrict__ w1s, uint2* __restrict__ w2q,
-                                                            uint8_t* __restrict__ w2s, int E, int F, int H, int nt1,
-                                                            int ks1, int nt2, int ks2) {
+                                                            uint8_t* __restrict__ w2s, int E, int F, int H, int hp,
+                                                            int fp, int nt1, int ks1, int nt2, int ks2) {
     const long long rows1 = (long long)E * 2 * F;
     const long long rows2 = (long long)E * H;
     for (long long row = blockIdx.x; row < rows1 + rows2; row += gridDim.x) {
@@ -90,7 +92,7 @@ __global__ void __launch_bounds__(128) prepare_mxfp8_kernel(const uint4* __restr
             const int gu = rem / F, f = rem - gu * F;
             src = (gu ? wu : wg) + ((size_t)e * F + f) * (H / 8);
             trow = ((f % kG1BN8) >> 4) * 32 + gu * 16 + (f & 15);
-            dst = w1q + ((size_t)(e * nt1 + f / kG1BN8) * 128 + trow) * (H / 8);
+            dst = w1q + ((size_t)(e * nt1 + f / kG1BN8) * 128 + trow) * (hp / 8);
             len = H;
             sf_tile = w1s + ((size_t)e * nt1 + f / kG1BN8) * ks1 * kSfBlock;
         } else {
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(128) prepare_mxfp8_kernel(const uint4* __restr
             const long long e = r2 / H;
             const int c = (int)(r2 - e * H);
             src = wd + (size_t)r2 * (F / 8);
-            dst = w2q + (size_t)r2 * (F / 8);
+            dst = w2q + (size_t)r2 * (fp / 8);
             len = F;
             trow = c % kG2BN8;
             sf_tile = w2s + ((size_t)e * nt2 + c / kG2BN8) * ks2 * kSfBlock;
@@ -125,18 +127,20 @@ cudaError_t launch_prepare_mxfp8(const moe_plan* p, const __nv_bfloat16* wg, con
                                  const __nv_bfloat16* wd, void* buf, cudaStream_t s) {
     uint8_t* base = static_cast<uint8_t*>(buf);
     const int E = p->d.num_experts, F = p->d.ffn, H = p->d.hidden;
-    // padding rows and k-groups of the scale blocks hold byte 0 (scale 2^-127), and the W1
-    // rows of f >= F (when F is not a multiple of 64) hold code 0
+    // padding rows and k-groups of the scale blocks hold byte 0 (scale 2^-127); the K padding
+    // of the code rows and the W1 rows of f >= F hold code 0
     cudaError_t err = cudaMemsetAsync(base + p->wb.w1s, 0, p->wb.w2 - p->wb.w1s, s);
     if (err != cudaSuccess) return err;
-    if (F % kG1BN8 != 0) err = cudaMemsetAsync(base + p->wb.w1, 0, p->wb.w1s - p->wb.w1, s);
+    if (H != p->hp || F != p->fp) err = cudaMemsetAsync(base + p->wb.w1, 0, p->wb.w1s - p->wb.w1, s);
+    if (err != cudaSuccess) return err;
+    if (F != p->fp) err = cudaMemsetAsync(base + p->wb.w2, 0, p->wb.w2s - p->wb.w2, s);
     if (err != cudaSuccess) return err;
     err = cudaMemsetAsync(base + p->wb.w2s, 0, p->wb.total - p->wb.w2s, s);
     if (err != cudaSuccess) return err;
     prepare_mxfp8_kernel<<<num_sms() * 16, 128, 0, s>>>(
         reinterpret_cast<const uint4*>(wg), reinterpret_cast<const uint4*>(wu), reinterpret_cast<const uint4*>(wd),
         reinterpret_cast<uint2*>(base + p->wb.w1), base + p->wb.w1s, reinterpret_cast<uint2*>(base + p->wb.w2),
-        base + p->wb.w2s, E, F, H, p->nt1, p->ks1, p->nt2, p->ks2);
+        base + p->wb.w2s, E, F, H, (int)p->hp, (int)p->fp, p->nt1, p->ks1, p->nt2, p->ks2);
     return cudaGetLastError();
 }
 

@@ -52,17 +52,19 @@ def test_prepare_weights_bit_exact(F):
     torch.cuda.synchronize()
     b = buf.cpu().numpy()
     gq, gs, uq, us, dq, ds = oracle.quantize_weights_mxfp8(wg, wu, wd)
-    # W1 codes: per 64-f tile, per 16 f, the 16 gate rows then the 16 up rows
-    f64 = (F + 63) // 64 * 64
-    n1 = E * 2 * f64 * H
-    w1 = b[:n1].reshape(E, f64 // 64, 4, 2, 16, H)
+    # W1 codes: per 64-f tile, per 16 f, the 16 gate rows then the 16 up rows; K pitches
+    # padded to 128 with zeros, rows of f >= F zero
+    hp, fp = (H + 127) // 128 * 128, (F + 127) // 128 * 128
+    n1 = E * 2 * fp * hp
+    w1 = b[:n1].reshape(E, fp // 64, 4, 2, 16, hp)
     f = np.arange(F)
-    assert np.array_equal(w1[:, f // 64, (f % 64) // 16, 0, f % 16], gq)
-    assert np.array_equal(w1[:, f // 64, (f % 64) // 16, 1, f % 16], uq)
-    fpad = np.arange(F, f64)
+    assert np.array_equal(w1[:, f // 64, (f % 64) // 16, 0, f % 16, :H], gq)
+    assert np.array_equal(w1[:, f // 64, (f % 64) // 16, 1, f % 16, :H], uq)
+    assert np.all(w1[..., H:] == 0)
+    fpad = np.arange(F, fp)
     assert np.all(w1[:, fpad // 64, (fpad % 64) // 16, :, fpad % 16] == 0)
     al = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    nt1, ks1 = (F + 63) // 64, (H + 127) // 128
+    nt1, ks1 = fp // 64, (H + 127) // 128
     off_w1s = al(n1)
     w1s = b[off_w1s:off_w1s + E * nt1 * ks1 * SF_BLOCK]
     for e in range(E):
@@ -72,10 +74,11 @@ def test_prepare_weights_bit_exact(F):
                 idx = ((e * nt1 + f // 64) * ks1 + g // 4) * SF_BLOCK + sf_offset(trow, g % 4)
                 assert np.array_equal(w1s[idx], ref[e, :, g]), (e, gu, g)
     off_w2 = off_w1s + al(E * nt1 * ks1 * SF_BLOCK)
-    w2 = b[off_w2:off_w2 + E * H * F].reshape(E, H, F)
-    assert np.array_equal(w2, dq)
+    w2 = b[off_w2:off_w2 + E * H * fp].reshape(E, H, fp)
+    assert np.array_equal(w2[..., :F], dq)
+    assert np.all(w2[..., F:] == 0)
     nt2, ks2 = (H + 127) // 128, (F + 127) // 128
-    off_w2s = off_w2 + al(E * H * F)
+    off_w2s = off_w2 + al(E * H * fp)
     w2s = b[off_w2s:off_w2s + E * nt2 * ks2 * SF_BLOCK]
     c = np.arange(H)
     for e in range(E):
@@ -94,14 +97,19 @@ def _check_intermediates(m: GpuMoe, x, ids, H, F, toks, h_ref):
     inv = m.read_i32(v["inv"], live * k).reshape(live, k)
     rows = inv[toks].reshape(-1).astype(np.int64)
     R = v["rows_padded"]
+    hp, fp = (H + 127) // 128 * 128, (F + 127) // 128 * 128  # row pitches (zero padding)
     # x codes and scales of every sampled route row equal the oracle's quantisation of x[t]
-    xq_all = _ws_bytes(m, v["xq"], R * H).reshape(R, H)
+    xq_all = _ws_bytes(m, v["xq"], R * hp).reshape(R, hp)
+    assert np.all(xq_all[rows][:, H:] == 0)
+    xq_all = xq_all[:, :H]
     xs_blob = _ws_bytes(m, v["xq_scales"], (R // 128) * ((H + 127) // 128) * SF_BLOCK)
     ref_q, ref_s = oracle.mxfp8_quantize_bf16(x[torch.from_numpy(np.repeat(toks, k))].contiguous())
     assert np.array_equal(xq_all[rows], ref_q)
     assert np.array_equal(decode_scales(xs_blob, rows, H), ref_s)
     # h: codes/scales equal the oracle's wherever the fp32 pre-quantisation value agrees
-    hq_all = _ws_bytes(m, v["h"], R * F).reshape(R, F)
+    hq_all = _ws_bytes(m, v["h"], R * fp).reshape(R, fp)
+    assert np.all(hq_all[rows][:, F:] == 0)
+    hq_all = hq_all[:, :F]
     hs_blob = _ws_bytes(m, v["h_scales"], (R // 128) * ((F + 127) // 128) * SF_BLOCK)
     hq_ref, hs_ref, _ = h_ref
     got_q = hq_all[rows].reshape(len(toks), k, F)
