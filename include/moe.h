@@ -192,8 +192,9 @@ moe_status moe_forward_noalloc(const moe_plan* plan, const void* x, const float*
 
 /* Stages of moe_forward, in launch order: route (or canonicalise the
  * caller's routes), permute (histogram, scan, scatter), gather of x rows
- * (and their MXFP8 quantisation), gate/up GEMM with SwiGLU, down GEMM,
- * combine. */
+ * (and their MXFP8 quantisation; bf16 gathers only the rows of route tiles
+ * of more than 32 routes, the gate/up GEMM reads the others from x itself),
+ * gate/up GEMM with SwiGLU, down GEMM, combine. */
 #define MOE_NUM_STAGES 6
 
 /* moe_forward that also records stage_events[i] (cudaEvent_t passed as void*,
@@ -217,7 +218,9 @@ moe_status moe_forward_with_events(const moe_plan* plan, const void* x, const fl
  *   h       intermediate rows [rows_padded, ceil(F/128)*128], bf16 or
  *           E4M3 codes, the columns past F zero
  *   xq      permuted x rows [rows_padded, ceil(H/128)*128], bf16 or E4M3
- *           codes, the columns past H zero
+ *           codes, the columns past H zero; bf16 writes only the rows of
+ *           route tiles of more than 32 routes (the gate/up GEMM reads the
+ *           x rows of smaller tiles in place)
  *   h_scales, xq_scales  MXFP8 only (else NULL): E8M0 bytes in blocks of
  *           512 bytes, one per (128-row tile, K stage of 128 elements),
  *           block index tile * ceil(K/128) + stage; inside a block the byte

@@ -93,7 +93,7 @@ static void compute_layouts(moe_plan* p) {
         w.h = take(R * (size_t)p->fp);
         w.hs = take(mtiles * p->ks2 * kSfBlock);
     } else {
-        w.xq = take(R * (size_t)p->hp * 2);
+        w.xq = take(R * (size_t)p->hp * 2);  // rows of tiles the gate/up GEMM does not gather itself
         w.xs = 0;
         w.h = take(R * (size_t)p->fp * 2);
         w.hs = 0;
@@ -276,6 +276,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     CUtensorMap tA1, tA2;  // weight operands
     BoxMaps8 rB1, rB2;     // route-row operands (x rows, h rows)
+    CUtensorMap tX;        // bf16: x rows, gathered by token
     if (fp8) {
         // MXFP8 (one CTA per tile): K stage = 256 E4M3 elements = two 128-byte swizzle atoms;
         // the maps address element k of a row as (k % 128, row, k / 128), so a box lands as
@@ -299,25 +300,33 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
                 return MOE_ERR_CUDA;
         }
     } else {
-        // bf16 (CTA pairs): K stage = 128 elements = two 64-element swizzle atoms.  Every
-        // operand buffer has its K pitch padded to 128 (hp, fp) with zeros, and the maps
-        // address an element k of a row as (k % 64, row, k / 64): the box's third dimension
-        // walks the two atoms, so a box lands as [atom][row][64 elements].  Weights (A) load
-        // 128 rows per CTA; route rows (B) load N/2 rows, one map per N/2 in {16, ..., 128}.
+        // bf16 (CTA pairs): K stage = 128 elements = two 64-element swizzle atoms.  The
+        // weight buffers and h have their K pitch padded to 128 (hp, fp) with zeros, and
+        // their maps address an element k of a row as (k % 64, row, k / 64): the box's
+        // third dimension walks the two atoms, so a box lands as [atom][row][64 elements].
+        // Weights (A) load 128 rows per CTA; route rows (B) N/2 rows, one map per N/2 in
+        // {16, ..., 128}.  Gate/up tiles of at most kGatherInGemmMax routes instead gather
+        // their B rows straight from x (one-row boxes of one atom, four rows per
+        // instruction; columns past H read as zeros); the gather kernel writes only the
+        // permuted x rows of the larger tiles.
         const unsigned long long hp = (unsigned long long)plan->hp, fpp = (unsigned long long)plan->fp;
         const unsigned box128[3] = {64, 128, 2};
         const unsigned long long dW1[3] = {64ull, uE * 2ull * fpp, hp / 64};
         const unsigned long long sW1[2] = {hp * 2, 128ull};
         const unsigned long long dW2[3] = {64ull, uE * uH, fpp / 64};
         const unsigned long long sW2[2] = {fpp * 2, 128ull};
-        const unsigned long long dX[3] = {64ull, R, hp / 64};
+        const unsigned long long dXP[3] = {64ull, R, hp / 64};
         const unsigned long long dH[3] = {64ull, R, fpp / 64};
+        const unsigned long long dX[2] = {uH, (unsigned long long)plan->d.capacity};
+        const unsigned long long sX[1] = {uH * 2};
+        const unsigned boxX[2] = {64, 1};
         if (!make_tensor_map(&tA1, dt, 3, wb + plan->wb.w1, dW1, sW1, box128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tA2, dt, 3, wb + plan->wb.w2, dW2, sW2, box128, CU_TENSOR_MAP_SWIZZLE_128B))
+            !make_tensor_map(&tA2, dt, 3, wb + plan->wb.w2, dW2, sW2, box128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tX, dt, 2, x, dX, sX, boxX, CU_TENSOR_MAP_SWIZZLE_128B))
             return MOE_ERR_CUDA;
         for (int i = 0; i < 8; ++i) {
             const unsigned box[3] = {64, 16u * (unsigned)(i + 1), 2};
-            if (!make_tensor_map(&rB1.m[i], dt, 3, ws + L.xq, dX, sW1, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            if (!make_tensor_map(&rB1.m[i], dt, 3, ws + L.xq, dXP, sW1, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
                 !make_tensor_map(&rB2.m[i], dt, 3, ws + L.h, dH, sW2, box, CU_TENSOR_MAP_SWIZZLE_128B))
                 return MOE_ERR_CUDA;
         }
@@ -343,10 +352,11 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     if (!mark(2)) return MOE_ERR_CUDA;
     if (fp8)
         e = launch_gather_mxfp8(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, (int)plan->hp, k,
-                                inv, ws + L.xq,
-                                ws + L.xs, s);
+                                inv, ws + L.xq, ws + L.xs, s);
     else
         e = launch_gather_bf16(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, (int)plan->hp, k, inv,
+                               r_ids, reinterpret_cast<const int*>(ws + L.offsets),
+                               reinterpret_cast<const int*>(ws + L.padoff), plan->tile_rows,
                                reinterpret_cast<__nv_bfloat16*>(ws + L.xq), s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -367,9 +377,11 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g1.sfb = ws + L.xs;
     g1.out_scales = fp8 ? ws + L.hs : nullptr;
     g1.sf_ks_out = plan->ks2;
+    g1.perm = perm;
+    g1.top_k = k;
     if (!mark(3)) return MOE_ERR_CUDA;
     e = fp8 ? launch_gemm1_mxfp8(tA1, rB1, g1, m_tiles * g1.n_tiles, s)
-            : launch_gemm1_bf16_pair(tA1, rB1, g1, m_tiles * g1.n_tiles, s);
+            : launch_gemm1_bf16_pair(tA1, tX, rB1, g1, m_tiles * g1.n_tiles, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 
     GemmParams g2 = g1;

@@ -83,7 +83,8 @@ __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + _
 __device__ __forceinline__ int tile_n(int nvalid) { return (nvalid + 31) & ~31; }
 
 template <int kMode>  // 0: gate/up + SwiGLU -> bf16 h;  1: down -> fp32 y
-__device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const BoxMaps8& tmB, const GemmParams& p) {
+__device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUtensorMap* tmX, const BoxMaps8* tmB,
+                                               const GemmParams& p) {
     constexpr uint32_t kEpiBytes = PairCfg<kMode>::kEpiBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -99,6 +100,7 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const Box
     const bool leader = rank == 0;
     const int pair = (int)cluster_id_x();
     const int npairs = (int)cluster_count_x();
+    pdl_trigger();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -122,57 +124,87 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const Box
     cluster_sync();  // both CTAs' barriers and TMEM exist before any cross-CTA traffic
     tc_fence_after_sync();
     const uint32_t tmem_base = bars->tmem_base;
+    pdl_wait();  // the tile list, x / h rows and status words come from earlier kernels
 
     const int num_m = (int)p.status_words[kStNumMTiles];
     const int total_tiles = num_m * p.n_tiles;
     const int kb_count = p.k_blocks;
 
     if (warp == 0) {
+        // ---------------- TMA producer (both CTAs; lane 0 waits and loads A, and B of the down GEMM)
         if (lane == 0) {
-            // ---------------- TMA producer (both CTAs)
             tma_prefetch_desc(&tmA);
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            int last_phase[kStages];
-            for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
-            for (int t = pair; t < total_tiles && ok; t += npairs) {
-                const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
-                const int4 ti = __ldg(p.tiles + mt);
-                const int hb = tile_n(ti.z) >> 1;  // route rows of B in each CTA
-                const CUtensorMap* mapB = &tmB.m[(hb >> 4) - 1];
-                const uint32_t tx = 2u * (kABytes + (uint32_t)hb * (kAtoms * 128u));
-                const int a_row = (int)((long long)ti.x * p.a_rows) + nt * kPairM + 128 * (int)rank;
-                const int b_row = ti.y + hb * (int)rank;
-                for (int kb = 0; kb < kb_count; ++kb) {
-                    if (!mbar_wait_bounded(&bars->empty[stage], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
-                        ok = false;
-                        break;
-                    }
+            if (kMode == 0) tma_prefetch_desc(tmX);
+        }
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        int last_phase[kStages];
+        for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
+        for (int t = pair; t < total_tiles && ok; t += npairs) {
+            const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
+            const int4 ti = __ldg(p.tiles + mt);
+            const int hb = tile_n(ti.z) >> 1;  // route rows of B in each CTA
+            const uint32_t tx = 2u * (kABytes + (uint32_t)hb * (kAtoms * 128u));
+            const int a_row = (int)((long long)ti.x * p.a_rows) + nt * kPairM + 128 * (int)rank;
+            const int b_row = ti.y + hb * (int)rank;
+            // gate/up tiles of at most kGatherInGemmMax routes: lane L gathers this CTA's B
+            // rows 4L..4L+3 from x, the rows of the tokens of routes hb * rank + 4L + q
+            // (rows past the tile's routes repeat its first token: in bounds, and their
+            // output columns are never stored).  Larger tiles load their rows, gathered
+            // by the gather kernel, as one box: a gather moves 512 bytes per TMA
+            // instruction, too few to feed a full tile.
+            int tok[4] = {0, 0, 0, 0};
+            const bool from_x = kMode == 0 && ti.z <= kGatherInGemmMax;
+            const bool gathers = from_x && 4 * lane < hb;
+            if (from_x) {
+                const int first = __ldg(p.perm + ti.w) / p.top_k;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int i = hb * (int)rank + 4 * lane + q;
+                    tok[q] = i < ti.z ? __ldg(p.perm + ti.w + i) / p.top_k : first;
+                }
+            }
+            for (int kb = 0; kb < kb_count; ++kb) {
+                bool got = true;
+                if (lane == 0) got = mbar_wait_bounded(&bars->empty[stage], phase ^ 1u, abort_flag, p.wait_limit_ns);
+                if (!__shfl_sync(0xffffffffu, got, 0)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t full0 = map_to_cta(smem_u32(&bars->full[stage]), 0);
+                if (lane == 0) {
                     if (leader) {
                         mbar_arrive_expect_tx(&bars->full[stage], tx);
                         last_phase[stage] = (int)phase;
                     }
-                    const uint32_t full0 = map_to_cta(smem_u32(&bars->full[stage]), 0);
                     // boxes land as [atom][row][64 elements]
                     tma_load_3d_pair(sA + stage * kABytes, &tmA, full0, 0, a_row, kb * kAtoms);
-                    tma_load_3d_pair(sB + stage * kBBytes, mapB, full0, 0, b_row, kb * kAtoms);
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    if (!from_x)
+                        tma_load_3d_pair(sB + stage * kBBytes, &tmB->m[(hb >> 4) - 1], full0, 0, b_row,
+                                         kb * kAtoms);
+                }
+                if (gathers) {
+#pragma unroll
+                    for (int at = 0; at < kAtoms; ++at)
+                        tma_gather4_pair(sB + stage * kBBytes + (uint32_t)at * (uint32_t)hb * 128u + lane * 512u,
+                                         tmX, full0, kb * kStageK + at * kBK, tok[0], tok[1], tok[2], tok[3]);
+                }
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
-            if (!ok) {
-                *abort_flag = 1;
-                atomicOr(p.status_flags, MOE_DEV_TIMEOUT);
-                if (leader) {  // copies already issued land before shared memory goes away
-                    for (int s = 0; s < kStages; ++s)
-                        if (last_phase[s] >= 0) {
-                            volatile int never = 0;
-                            (void)mbar_wait_bounded(&bars->full[s], (uint32_t)last_phase[s], &never, 100000000ull);
-                        }
-                }
+        }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            atomicOr(p.status_flags, MOE_DEV_TIMEOUT);
+            if (leader) {  // copies already issued land before shared memory goes away
+                for (int s = 0; s < kStages; ++s)
+                    if (last_phase[s] >= 0) {
+                        volatile int never = 0;
+                        (void)mbar_wait_bounded(&bars->full[s], (uint32_t)last_phase[s], &never, 100000000ull);
+                    }
             }
         }
         __syncwarp();
@@ -336,18 +368,17 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const Box
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    moe_gemm_gate_up_swiglu_bf16_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BoxMaps8 tmB,
-                                      const GemmParams p) {
-    pair_gemm_body<0>(tmA, tmB, p);
+    moe_gemm_gate_up_swiglu_bf16_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmX,
+                                      const __grid_constant__ BoxMaps8 tmB, const GemmParams p) {
+    pair_gemm_body<0>(tmA, &tmX, &tmB, p);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     moe_gemm_down_bf16_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BoxMaps8 tmB,
                             const GemmParams p) {
-    pair_gemm_body<1>(tmA, tmB, p);
+    pair_gemm_body<1>(tmA, nullptr, &tmB, p);
 }
 
-using GemmKernel = void (*)(CUtensorMap, BoxMaps8, GemmParams);
 
 struct PairLaunchCache {
     size_t smem = 0;
@@ -355,17 +386,21 @@ struct PairLaunchCache {
     int pairs = 0;
 };
 
-cudaError_t launch_pair(GemmKernel kern, PairLaunchCache* cache, const CUtensorMap& a, const BoxMaps8& b,
-                        const GemmParams& gp, long long max_tiles, cudaStream_t s) {
+template <class... Operands>
+cudaError_t launch_pair(void (*kern)(CUtensorMap, Operands..., GemmParams), PairLaunchCache* cache,
+                        const CUtensorMap& a, const Operands&... b, const GemmParams& gp, long long max_tiles,
+                        cudaStream_t s) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see pdl_wait()
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = cache->smem;
     cfg.stream = s;
@@ -387,23 +422,25 @@ cudaError_t launch_pair(GemmKernel kern, PairLaunchCache* cache, const CUtensorM
     if (pairs > max_tiles) pairs = max_tiles;
     if (pairs < 1) pairs = 1;
     cfg.gridDim = dim3((unsigned)(2 * pairs));
-    err = cudaLaunchKernelEx(&cfg, kern, a, b, gp);
+    cfg.numAttrs = 2;
+    err = cudaLaunchKernelEx(&cfg, kern, a, b..., gp);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_gemm1_bf16_pair(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
-                                   cudaStream_t s) {
+cudaError_t launch_gemm1_bf16_pair(const CUtensorMap& a, const CUtensorMap& x_rows, const BoxMaps8& b,
+                                   const GemmParams& gp, long long max_tiles, cudaStream_t s) {
     static PairLaunchCache cache{PairCfg<0>::kSmemBytes};
-    return launch_pair(moe_gemm_gate_up_swiglu_bf16_pair, &cache, a, b, gp, max_tiles, s);
+    return launch_pair<CUtensorMap, BoxMaps8>(moe_gemm_gate_up_swiglu_bf16_pair, &cache, a, x_rows, b, gp, max_tiles,
+                                              s);
 }
 
 cudaError_t launch_gemm2_bf16_pair(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
                                    cudaStream_t s) {
     static PairLaunchCache cache{PairCfg<1>::kSmemBytes};
-    return launch_pair(moe_gemm_down_bf16_pair, &cache, a, b, gp, max_tiles, s);
+    return launch_pair<BoxMaps8>(moe_gemm_down_bf16_pair, &cache, a, b, gp, max_tiles, s);
 }
 
 }  // namespace moe

@@ -129,6 +129,7 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    pdl_trigger();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -152,6 +153,7 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = bars->tmem_base;
+    pdl_wait();  // the tile list, route rows, scales and status words come from earlier kernels
 
     const int num_m = (int)p.status_words[kStNumMTiles];
     const int total_tiles = num_m * p.n_tiles;
@@ -445,8 +447,7 @@ cudaError_t launch_impl(GemmKernel kern, int* configured_device, const CUtensorM
     long long grid = num_sms();  // persistent: one CTA per SM
     if (grid > max_tiles) grid = max_tiles;
     if (grid < 1) grid = 1;
-    kern<<<(unsigned)grid, kThreads, kSmemBytes, s>>>(a, b, gp);
-    return cudaGetLastError();
+    return launch_dependent(kern, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, a, b, gp);
 }
 
 }  // namespace

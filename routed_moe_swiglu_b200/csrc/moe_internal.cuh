@@ -9,6 +9,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 
 #include "moe.h"
 
@@ -22,6 +23,7 @@ constexpr int kG1BN = 128;         // bf16: f values per gate/up weight tile (25
 constexpr int kG2BN = 256;         // bf16: output columns per down weight tile
 constexpr int kRouteTile = 256;    // bf16: most routes per tile (N of a pair MMA)
 constexpr int kRouteAlign = 32;    // bf16: route rows of an expert start on a multiple of this
+constexpr int kGatherInGemmMax = 32;  // bf16: route tiles of at most this many routes read x rows by token
 constexpr int kG1BN8 = 64;         // MXFP8: f values per gate/up tile (64 gate + 64 up MMA columns)
 constexpr int kG2BN8 = 128;        // MXFP8: output columns per down tile
 constexpr int kSfBlock = 512;      // MXFP8 scales of 128 rows x 4 k-groups, [row%32][row/32][k-group]
@@ -76,7 +78,7 @@ struct BoxMaps8 {
 };
 
 struct GemmParams {
-    const int4* tiles;              // {expert, first padded row, valid rows, 0} per route tile
+    const int4* tiles;              // {expert, first padded row, valid rows, first permuted row} per route tile
     const unsigned* status_words;   // [kStNumMTiles] = number of M tiles
     unsigned* status_flags;         // sticky MOE_DEV_* bits
     void* out;                      // h (bf16 / E4M3) or y (fp32)
@@ -93,6 +95,10 @@ struct GemmParams {
     const uint8_t* sfa;
     const uint8_t* sfb;
     int sf_ks_out;
+    // bf16 gate/up: the B rows are gathered from x by token, route r of the
+    // permuted order being token perm[r] / top_k
+    const int* perm;
+    int top_k;
 };
 
 // ---------------------------------------------------------------- launchers
@@ -110,13 +116,14 @@ cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* 
                            int* padoff, int4* tiles, int* perm, int* inv, unsigned* status_words,
                            cudaStream_t s);
 cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
-                               const int* inv, __nv_bfloat16* xp, cudaStream_t s);
+                               const int* inv, const int* ids, const int* offsets, const int* padoff, int tile_rows,
+                               __nv_bfloat16* xp, cudaStream_t s);
 cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
                                 const int* inv, uint8_t* xq, uint8_t* xs, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const int* inv, const float* probs, const int* live, int max_live,
                            int H, int k, float* out, cudaStream_t s);
-cudaError_t launch_gemm1_bf16_pair(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
-                                   cudaStream_t s);
+cudaError_t launch_gemm1_bf16_pair(const CUtensorMap& a, const CUtensorMap& x_rows, const BoxMaps8& b,
+                                   const GemmParams& gp, long long max_tiles, cudaStream_t s);
 cudaError_t launch_gemm2_bf16_pair(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
                                    cudaStream_t s);
 cudaError_t launch_gemm1_mxfp8(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
@@ -129,6 +136,34 @@ cudaError_t launch_prepare_mxfp8(const moe_plan* p, const __nv_bfloat16* wg, con
                                  const __nv_bfloat16* wd, void* buf, cudaStream_t s);
 cudaError_t launch_quantize_rows(const __nv_bfloat16* in, long long rows, int cols, long long ld_in, uint8_t* q,
                                  uint8_t* scales, const int* live_rows, cudaStream_t s);
+
+// ---------------------------------------------------------------- dependent launches
+// Every kernel of the forward is launched with programmatic stream
+// serialisation: it may be scheduled while its predecessor in the stream is
+// still running, does its set-up (barriers, TMEM, descriptor prefetch), and
+// waits in pdl_wait() until the predecessor has completed and its writes are
+// visible before reading anything another kernel (or the caller) produced.
+// pdl_trigger() lets the next kernel be scheduled; it changes no ordering
+// of memory, so each kernel issues it first thing.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <class... KArgs, class... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Args&&... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    return err != cudaSuccess ? err : cudaGetLastError();
+}
 
 // Byte offset of (row within a 128-row tile, k-group within a 4-group K
 // stage) inside one 512-byte MXFP8 scale block.

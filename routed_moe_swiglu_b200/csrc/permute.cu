@@ -14,7 +14,9 @@
 //   scatter  per block: one 32-bit lane mask per (warp, expert) gives every
 //            route its rank among earlier tokens of the block routed to the
 //            same expert (popcount of the lower lanes plus the earlier warps)
-// and a gather that copies x rows into their padded route rows.
+// and a gather that copies each token's x row into its padded route rows
+// (MXFP8: quantised once per token; bf16: only the rows of route tiles the
+// gate/up GEMM does not gather from x itself).
 #include "moe_internal.cuh"
 #include "mxfp8.cuh"
 
@@ -25,6 +27,8 @@ __global__ void __launch_bounds__(kTokPerBlk) route_hist_kernel(const int* __res
                                                                 const int* __restrict__ live, int max_live,
                                                                 int E, int k, int* __restrict__ blkcnt) {
     extern __shared__ int s_hist[];
+    pdl_trigger();
+    pdl_wait();
     const int n = clamp_live(live, max_live);
     const int t0 = blockIdx.x * kTokPerBlk;
     if (t0 >= n) return;
@@ -75,6 +79,8 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int* __restrict_
                                                           int* __restrict__ padoff, int4* __restrict__ tiles,
                                                           unsigned* __restrict__ status_words) {
     __shared__ int s_warp[32];
+    pdl_trigger();
+    pdl_wait();
     const int n = clamp_live(live, max_live);
     const int nb = (n + kTokPerBlk - 1) / kTokPerBlk;
     const int e = threadIdx.x;
@@ -97,7 +103,8 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int* __restrict_
         padoff[e] = ex_pad;
         for (int i = 0; i < mt; ++i) {
             const int rows = tot - i * tile_rows;
-            tiles[ex_mt + i] = make_int4(e, ex_pad + i * tile_rows, rows < tile_rows ? rows : tile_rows, 0);
+            tiles[ex_mt + i] =
+                make_int4(e, ex_pad + i * tile_rows, rows < tile_rows ? rows : tile_rows, ex_tot + i * tile_rows);
         }
     }
     if (e == 0) {
@@ -113,6 +120,8 @@ __global__ void __launch_bounds__(kTokPerBlk) route_scatter_kernel(
     const int* __restrict__ blkprefix, const int* __restrict__ offsets, const int* __restrict__ padoff,
     int* __restrict__ perm, int* __restrict__ inv) {
     extern __shared__ uint32_t s_mem[];
+    pdl_trigger();
+    pdl_wait();
     const int n = clamp_live(live, max_live);
     const int t0 = blockIdx.x * kTokPerBlk;
     if (t0 >= n) return;
@@ -160,24 +169,39 @@ __global__ void __launch_bounds__(kTokPerBlk) route_scatter_kernel(
     }
 }
 
-// One 128-thread block per token (grid-stride): read the token's x row once,
-// write it to each of its k padded route rows; every thread keeps all of its
-// 16-byte loads in flight before storing.
 constexpr int kRowThreads = 128;
 
-__global__ void __launch_bounds__(kRowThreads) gather_rows_bf16_kernel(const uint4* __restrict__ x,
-                                                                       const int* __restrict__ live, int max_live,
-                                                                       int H, int hp, int k,
-                                                                       const int* __restrict__ inv,
-                                                                       uint4* __restrict__ xp) {
+// bf16 gather: one 128-thread block per token (grid-stride) reads the
+// token's x row once and writes it to those of its k padded route rows that
+// lie in route tiles of more than kGatherInGemmMax routes; the gate/up GEMM
+// reads the rows of smaller tiles straight from x.  Every thread keeps all
+// of its 16-byte loads in flight before storing.
+__global__ void __launch_bounds__(kRowThreads) gather_rows_bf16_kernel(
+    const uint4* __restrict__ x, const int* __restrict__ live, int max_live, int H, int hp, int k,
+    const int* __restrict__ inv, const int* __restrict__ ids, const int* __restrict__ offsets,
+    const int* __restrict__ padoff, int tile_rows, uint4* __restrict__ xp) {
     __shared__ int s_prow[kMaxTopK];
+    pdl_trigger();
+    pdl_wait();
     const int n = clamp_live(live, max_live);
     const int chunks = H / 8;       // 8 bf16 per 16 bytes
     const int chunks_out = hp / 8;  // destination rows are padded to hp with zeros
     for (int t = blockIdx.x; t < n; t += gridDim.x) {
         __syncthreads();
-        if (threadIdx.x < k) s_prow[threadIdx.x] = __ldg(inv + (size_t)t * k + threadIdx.x);
+        if (threadIdx.x < k) {
+            int pr = __ldg(inv + (size_t)t * k + threadIdx.x);
+            if (pr >= 0) {
+                const int e = __ldg(ids + (size_t)t * k + threadIdx.x);
+                const int local = pr - __ldg(padoff + e);
+                const int left = __ldg(offsets + e + 1) - __ldg(offsets + e) - local / tile_rows * tile_rows;
+                if ((left < tile_rows ? left : tile_rows) <= kGatherInGemmMax) pr = -1;
+            }
+            s_prow[threadIdx.x] = pr;
+        }
         __syncthreads();
+        bool any = false;
+        for (int j = 0; j < k; ++j) any |= s_prow[j] >= 0;
+        if (!any) continue;
         const uint4* src = x + (size_t)t * chunks;
 #pragma unroll 4
         for (int c = threadIdx.x; c < chunks_out; c += kRowThreads) {
@@ -202,6 +226,8 @@ __global__ void __launch_bounds__(kRowThreads) gather_rows_mxfp8_kernel(const ui
                                                                         uint2* __restrict__ xq,
                                                                         uint8_t* __restrict__ xs) {
     __shared__ int s_prow[kMaxTopK];
+    pdl_trigger();
+    pdl_wait();
     const int n = clamp_live(live, max_live);
     const int chunks = H / 8;       // 8 elements per thread and chunk
     const int chunks_out = hp / 8;  // destination pitch
@@ -249,6 +275,8 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(const float4* __re
                                                               int k, float4* __restrict__ out) {
     __shared__ int s_prow[kMaxTopK];
     __shared__ float s_p[kMaxTopK];
+    pdl_trigger();
+    pdl_wait();
     const int n = clamp_live(live, max_live);
     const int chunks = H / 4;
     for (int t = blockIdx.x; t < n; t += gridDim.x) {
@@ -300,12 +328,11 @@ cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* 
     const int E = p->d.num_experts, k = p->d.top_k;
     const int max_live = (int)p->max_live;
     const int nblk = p->nblk;
-    route_hist_kernel<<<nblk, kTokPerBlk, E * sizeof(int), s>>>(r_ids, live, max_live, E, k, blkcnt);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_dependent(route_hist_kernel, dim3(nblk), dim3(kTokPerBlk), E * sizeof(int), s, r_ids,
+                                       live, max_live, E, k, blkcnt);
     if (err != cudaSuccess) return err;
-    route_scan_kernel<<<1, 1024, 0, s>>>(live, max_live, E, p->tile_rows, p->row_align, blkcnt, offsets, padoff,
-                                         tiles, status_words);
-    err = cudaGetLastError();
+    err = launch_dependent(route_scan_kernel, dim3(1), dim3(1024), 0, s, live, max_live, E, p->tile_rows,
+                           p->row_align, blkcnt, offsets, padoff, tiles, status_words);
     if (err != cudaSuccess) return err;
     const size_t smem = (size_t)(kTokPerBlk / 32) * E * 8;
     if (smem > 48 * 1024) {
@@ -321,33 +348,32 @@ cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* 
             configured_device = dev;
         }
     }
-    route_scatter_kernel<<<nblk, kTokPerBlk, smem, s>>>(r_ids, live, max_live, E, k, blkcnt, offsets, padoff,
-                                                        perm, inv);
-    return cudaGetLastError();
+    return launch_dependent(route_scatter_kernel, dim3(nblk), dim3(kTokPerBlk), smem, s, r_ids, live, max_live, E, k,
+                            blkcnt, offsets, padoff, perm, inv);
 }
 
 cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
-                               const int* inv, __nv_bfloat16* xp, cudaStream_t s) {
+                               const int* inv, const int* ids, const int* offsets, const int* padoff, int tile_rows,
+                               __nv_bfloat16* xp, cudaStream_t s) {
     const int grid = grid_for_warps(max_live, 1, 16);
-    gather_rows_bf16_kernel<<<grid, kRowThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), live, max_live, H, hp, k,
-                                                         inv, reinterpret_cast<uint4*>(xp));
-    return cudaGetLastError();
+    return launch_dependent(gather_rows_bf16_kernel, dim3(grid), dim3(kRowThreads), 0, s,
+                            reinterpret_cast<const uint4*>(x), live, max_live, H, hp, k, inv, ids, offsets, padoff,
+                            tile_rows, reinterpret_cast<uint4*>(xp));
 }
 
 cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
                                 const int* inv, uint8_t* xq, uint8_t* xs, cudaStream_t s) {
     const int grid = grid_for_warps(max_live, 1, 16);
-    gather_rows_mxfp8_kernel<<<grid, kRowThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), live, max_live, H, hp, k,
-                                                          hp / 128, inv, reinterpret_cast<uint2*>(xq), xs);
-    return cudaGetLastError();
+    return launch_dependent(gather_rows_mxfp8_kernel, dim3(grid), dim3(kRowThreads), 0, s,
+                            reinterpret_cast<const uint4*>(x), live, max_live, H, hp, k, hp / 128, inv,
+                            reinterpret_cast<uint2*>(xq), xs);
 }
 
 cudaError_t launch_combine(const float* y, const int* inv, const float* probs, const int* live, int max_live,
                            int H, int k, float* out, cudaStream_t s) {
     const int grid = grid_for_warps(max_live, 1, 16);
-    combine_kernel<<<grid, kRowThreads, 0, s>>>(reinterpret_cast<const float4*>(y), inv, probs, live, max_live, H, k,
-                                        reinterpret_cast<float4*>(out));
-    return cudaGetLastError();
+    return launch_dependent(combine_kernel, dim3(grid), dim3(kRowThreads), 0, s, reinterpret_cast<const float4*>(y),
+                            inv, probs, live, max_live, H, k, reinterpret_cast<float4*>(out));
 }
 
 }  // namespace moe

@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
                                                          const int* __restrict__ live, int max_live, int E,
                                                          int k, int* __restrict__ ids,
                                                          float* __restrict__ probs, unsigned* status) {
+    pdl_trigger();
+    pdl_wait();
     int n = __ldg(live);
     if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0 && (n < 0 || n > max_live))
         atomicOr(status, MOE_DEV_LIVE_CLAMPED);
@@ -103,6 +105,8 @@ __global__ void __launch_bounds__(256) canon_routes_kernel(const int* __restrict
                                                            const int* __restrict__ live, int max_live, int E,
                                                            int k, int* __restrict__ ids_out,
                                                            float* __restrict__ probs_out, unsigned* status) {
+    pdl_trigger();
+    pdl_wait();
     int n = __ldg(live);
     if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0 && (n < 0 || n > max_live))
         atomicOr(status, MOE_DEV_LIVE_CLAMPED);
@@ -149,14 +153,17 @@ cudaError_t launch_route_topk(const float* logits, const int* live, int max_live
     if (blocks < 1) blocks = 1;
     const int slots = (E + 31) / 32;
     if (slots <= 4)
-        route_topk_kernel<4><<<(unsigned)blocks, warps * 32, 0, s>>>(logits, live, max_live, E, k, ids, probs, status);
+        return launch_dependent(route_topk_kernel<4>, dim3((unsigned)blocks), dim3(warps * 32), 0, s, logits, live,
+                                max_live, E, k, ids, probs, status);
     else if (slots <= 8)
-        route_topk_kernel<8><<<(unsigned)blocks, warps * 32, 0, s>>>(logits, live, max_live, E, k, ids, probs, status);
+        return launch_dependent(route_topk_kernel<8>, dim3((unsigned)blocks), dim3(warps * 32), 0, s, logits, live,
+                                max_live, E, k, ids, probs, status);
     else if (slots <= 16)
-        route_topk_kernel<16><<<(unsigned)blocks, warps * 32, 0, s>>>(logits, live, max_live, E, k, ids, probs, status);
+        return launch_dependent(route_topk_kernel<16>, dim3((unsigned)blocks), dim3(warps * 32), 0, s, logits, live,
+                                max_live, E, k, ids, probs, status);
     else
-        route_topk_kernel<32><<<(unsigned)blocks, warps * 32, 0, s>>>(logits, live, max_live, E, k, ids, probs, status);
-    return cudaGetLastError();
+        return launch_dependent(route_topk_kernel<32>, dim3((unsigned)blocks), dim3(warps * 32), 0, s, logits, live,
+                                max_live, E, k, ids, probs, status);
 }
 
 cudaError_t launch_canon_routes(const int* ids_in, const float* probs_in, const int* live, int max_live, int E,
@@ -165,9 +172,8 @@ cudaError_t launch_canon_routes(const int* ids_in, const float* probs_in, const 
     const long long cap = (long long)num_sms() * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    canon_routes_kernel<<<(unsigned)blocks, 256, 0, s>>>(ids_in, probs_in, live, max_live, E, k, ids_out,
-                                                         probs_out, status);
-    return cudaGetLastError();
+    return launch_dependent(canon_routes_kernel, dim3((unsigned)blocks), dim3(256), 0, s, ids_in, probs_in, live,
+                            max_live, E, k, ids_out, probs_out, status);
 }
 
 }  // namespace moe
