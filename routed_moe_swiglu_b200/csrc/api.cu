@@ -111,7 +111,7 @@ static void compute_layouts(moe_plan* p) {
     } else {
         b.w1 = take(E * 2 * (size_t)p->fp * (size_t)p->hp * 2);
         b.w1s = 0;
-        b.w2 = take(E * H * (size_t)p->fp * 2);
+        b.w2 = take(E * (size_t)p->hr * (size_t)p->fp * 2);
         b.w2s = 0;
     }
     b.total = off;
@@ -172,6 +172,7 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     p->ks2 = (d.ffn + 127) / 128;
     p->hp = (long long)p->ks1 * 128;
     p->fp = (long long)p->ks2 * 128;
+    p->hr = p->hp;
     if (d.precision == MOE_MXFP8) {
         p->nt1 = (int)(p->fp / kG1BN8);  // f tiles of 64 cover fp; h's padding columns come out zero
         p->nt2 = (d.hidden + kG2BN8 - 1) / kG2BN8;
@@ -300,28 +301,32 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
                 return MOE_ERR_CUDA;
         }
     } else {
-        // bf16 (CTA pairs): K stage = 128 elements = two 64-element swizzle atoms.  The
-        // weight buffers and h have their K pitch padded to 128 (hp, fp) with zeros, and
-        // their maps address an element k of a row as (k % 64, row, k / 64): the box's
-        // third dimension walks the two atoms, so a box lands as [atom][row][64 elements].
-        // Weights (A) load 128 rows per CTA; route rows (B) N/2 rows, one map per N/2 in
+        // bf16 (CTA pairs): K stage = 128 elements = two 64-element swizzle atoms, and
+        // every operand box lands as [atom][row][64 elements].  The permuted x rows and h
+        // have their K pitch padded to 128 (hp, fp) with zeros; their maps address element
+        // k of a row as (k % 64, row, k / 64), the box's third dimension walking the two
+        // atoms.  Weights (A) load 128 rows per CTA; route rows (B) N/2 rows, one map per N/2 in
         // {16, ..., 128}.  Gate/up tiles of at most kGatherInGemmMax routes instead gather
         // their B rows straight from x (one-row boxes of one atom, four rows per
         // instruction; columns past H read as zeros); the gather kernel writes only the
         // permuted x rows of the larger tiles.
         const unsigned long long hp = (unsigned long long)plan->hp, fpp = (unsigned long long)plan->fp;
+        // weights: blocks of [2 atoms][128 rows][64 elements], 32 KB contiguous, one per
+        // (expert, 128-row block, K stage); atom a of block b is index 2b + a of the map's
+        // third dimension
         const unsigned box128[3] = {64, 128, 2};
-        const unsigned long long dW1[3] = {64ull, uE * 2ull * fpp, hp / 64};
+        const unsigned long long dW1[3] = {64ull, 128ull, 2ull * (uE * 2ull * fpp / 128) * (hp / 128)};
+        const unsigned long long dW2[3] = {64ull, 128ull, 2ull * (uE * (unsigned long long)plan->hr / 128) * (fpp / 128)};
+        const unsigned long long sWb[2] = {128ull, 128ull * 128ull};
         const unsigned long long sW1[2] = {hp * 2, 128ull};
-        const unsigned long long dW2[3] = {64ull, uE * uH, fpp / 64};
         const unsigned long long sW2[2] = {fpp * 2, 128ull};
         const unsigned long long dXP[3] = {64ull, R, hp / 64};
         const unsigned long long dH[3] = {64ull, R, fpp / 64};
         const unsigned long long dX[2] = {uH, (unsigned long long)plan->d.capacity};
         const unsigned long long sX[1] = {uH * 2};
         const unsigned boxX[2] = {64, 1};
-        if (!make_tensor_map(&tA1, dt, 3, wb + plan->wb.w1, dW1, sW1, box128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tensor_map(&tA2, dt, 3, wb + plan->wb.w2, dW2, sW2, box128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        if (!make_tensor_map(&tA1, dt, 3, wb + plan->wb.w1, dW1, sWb, box128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tensor_map(&tA2, dt, 3, wb + plan->wb.w2, dW2, sWb, box128, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_tensor_map(&tX, dt, 2, x, dX, sX, boxX, CU_TENSOR_MAP_SWIZZLE_128B))
             return MOE_ERR_CUDA;
         for (int i = 0; i < 8; ++i) {
@@ -390,7 +395,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g2.out_cols = H;
     g2.n_tiles = plan->nt2;
     g2.k_blocks = plan->ks2;
-    g2.a_rows = H;
+    g2.a_rows = fp8 ? H : plan->hr;
     g2.sfa = wb + plan->wb.w2s;
     g2.sfb = ws + L.hs;
     g2.out_scales = nullptr;

@@ -23,10 +23,14 @@
 // Both epilogues transpose through shared memory so that y and h rows leave
 // as coalesced 16-byte stores (one route row per store group).
 //
-// A K stage is 128 elements (two 128-byte swizzle atoms, 8 MMAs) and each
-// operand of a stage is one TMA instruction: A is a 128-row x 2-atom box, B a
-// (N/2)-row x 2-atom box, one tensor map per N/2 in {16, 32, ..., 128}.  The K
-// row pitch of every bf16 operand buffer is padded to 128 with zeros.
+// A K stage is 128 elements (two 128-byte swizzle atoms, 8 MMAs).  A is one
+// TMA box of 32 KB that is contiguous in memory: the prepared weights are
+// stored as blocks of [2 atoms][128 rows][64 elements], one per (expert,
+// 128-row block, K stage), so the weight stream reads whole 32 KB runs.  B
+// is an (N/2)-row x 2-atom box of padded route rows (one tensor map per N/2
+// in {16, 32, ..., 128}; K pitches padded to 128 with zeros), except for
+// gate/up tiles of at most 32 routes, which gather their x rows by token
+// with tile::gather4 (four one-atom rows per instruction) instead.
 //
 // Roles (10 warps per CTA): warp 0 issues TMA loads in both CTAs (the
 // completion of both halves is counted on CTA 0's "full" barrier); warp 1
@@ -146,7 +150,10 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
             const int4 ti = __ldg(p.tiles + mt);
             const int hb = tile_n(ti.z) >> 1;  // route rows of B in each CTA
             const uint32_t tx = 2u * (kABytes + (uint32_t)hb * (kAtoms * 128u));
-            const int a_row = (int)((long long)ti.x * p.a_rows) + nt * kPairM + 128 * (int)rank;
+            // this CTA's 128 weight rows: row block a_rb of the blocked weight buffer, whose
+            // K stage kb is atoms 2 * (a_rb * kb_count + kb) and + 1
+            const long long a_rb = ((long long)ti.x * p.a_rows + nt * kPairM + 128 * (int)rank) / 128;
+            const int a_atom0 = (int)(a_rb * kb_count) * kAtoms;
             const int b_row = ti.y + hb * (int)rank;
             // gate/up tiles of at most kGatherInGemmMax routes: lane L gathers this CTA's B
             // rows 4L..4L+3 from x, the rows of the tokens of routes hb * rank + 4L + q
@@ -179,7 +186,7 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
                         last_phase[stage] = (int)phase;
                     }
                     // boxes land as [atom][row][64 elements]
-                    tma_load_3d_pair(sA + stage * kABytes, &tmA, full0, 0, a_row, kb * kAtoms);
+                    tma_load_3d_pair(sA + stage * kABytes, &tmA, full0, 0, 0, a_atom0 + kb * kAtoms);
                     if (!from_x)
                         tma_load_3d_pair(sB + stage * kBBytes, &tmB->m[(hb >> 4) - 1], full0, 0, b_row,
                                          kb * kAtoms);

@@ -61,6 +61,7 @@ struct moe_plan {
     int row_align;          // each expert's route rows start on a multiple of this: 32 (bf16) or 128 (MXFP8)
     long long hp, fp;       // K row pitch (elements) of x / gate-up rows and of h / down rows:
                             // H and F padded to multiples of 128 with zeros
+    long long hr;           // bf16: rows of an expert's down weights, H padded to 128 with zero rows
     int ks1, ks2;           // K blocks of 128 elements of the gate/up and down GEMMs
     int nt1, nt2;           // weight (bf16) / N (MXFP8) tiles of the gate/up and down GEMMs
     moe::WsLayout ws;
@@ -87,7 +88,7 @@ struct GemmParams {
     int out_cols;                   // valid output columns (F or H)
     int n_tiles;                    // weight tiles per route tile
     int k_blocks;                   // pipeline stages per tile
-    long long a_rows;               // bf16: rows of one expert in the weight operand's tensor map
+    long long a_rows;               // bf16: weight rows of one expert (a multiple of 128)
     unsigned long long wait_limit_ns;
     // MXFP8 only: scale blocks of A, the weights ([expert][weight tile][K stage][512 B]),
     // and of B, the route rows ([128-row tile][K stage][512 B]); K stages of the down

@@ -3,14 +3,18 @@
 // refresh_mega_weights(), which rewrites the kernel's own copy of the
 // weights; no allocation, no teardown).
 //
-// bf16 layout:  W1 [E][fp/64][4][2][16][hp]  (per block of 64 f, per group of
-//                                           16 f: the 16 gate rows, then the
-//                                           16 up rows of the same f),
-//               W2 [E][H][fp]               (down projection),
-// with the K pitches hp, fp = H, F rounded up to 128 and the padding zero
-// (rows of f >= F too).  A gate/up weight tile is two consecutive blocks, one
-// per CTA of a pair; a group of 32 rows is one 32-lane TMEM quarter, so gate
-// and up of one f land in the same warp's reach.
+// bf16 layout: every weight matrix is stored as blocks of 32 KB, one per
+// (expert, block of 128 weight rows, K stage of 128 elements), each block
+// [2 atoms][128 rows][64 elements] -- exactly the GEMM's shared-memory image
+// of one operand stage before swizzling, so one TMA box reads 32 KB of
+// contiguous memory:
+//   W1  rows of an expert: 2fp, in the order (per block of 64 f, per group
+//       of 16 f) the 16 gate rows, then the 16 up rows of the same f; K = hp
+//   W2  rows of an expert: hr (H padded to 128); K = fp
+// with hp, fp = H, F rounded up to 128.  Padding (K past H or F, rows of
+// f >= F, rows c >= H) is zero.  A gate/up weight tile is two consecutive
+// row blocks, one per CTA of a pair; a group of 32 rows is one 32-lane TMEM
+// quarter, so gate and up of one f land in the same warp's reach.
 #include "moe_internal.cuh"
 #include "mxfp8.cuh"
 
@@ -19,29 +23,37 @@ namespace {
 
 __global__ void __launch_bounds__(256) prepare_bf16_kernel(const uint4* __restrict__ wg, const uint4* __restrict__ wu,
                                                            const uint4* __restrict__ wd, uint4* __restrict__ w1,
-                                                           uint4* __restrict__ w2, int E, int F, int H, int hp, int fp) {
-    // 16-byte chunks of the destination; rows are padded with zeros to hp / fp
-    const long long c1 = hp / 8, c2 = fp / 8;
-    const long long rows1 = 2ll * fp;  // W1 rows per expert
-    const long long n1 = (long long)E * rows1 * c1;
-    const long long n2 = (long long)E * H * c2;
+                                                           uint4* __restrict__ w2, int E, int F, int H, int hp, int fp,
+                                                           int hr) {
+    // one thread per 16-byte chunk of the destination: block, atom, row, 8-element chunk
+    constexpr long long kBlockChunks = 2 * 128 * 8;  // 32 KB
+    const int kb1 = hp / 128, kb2 = fp / 128;
+    const int rb1 = 2 * fp / 128, rb2 = hr / 128;  // row blocks per expert
+    const long long n1 = (long long)E * rb1 * kb1 * kBlockChunks;
+    const long long n2 = (long long)E * rb2 * kb2 * kBlockChunks;
     const long long stride = (long long)gridDim.x * blockDim.x;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n1 + n2; i += stride) {
-        if (i < n1) {
-            const long long row = i / c1;  // e * 2fp + block * 128 + group * 32 + g * 16 + f % 16
-            const int c = (int)(i - row * c1);
-            const long long e = row / rows1;
-            const int rem = (int)(row - e * rows1);
+        const bool first = i < n1;
+        const long long j = first ? i : i - n1;
+        const long long blk = j / kBlockChunks;
+        const int w = (int)(j - blk * kBlockChunks);
+        const int atom = w >> 10, r = (w >> 3) & 127, c8 = w & 7;
+        const int kbs = first ? kb1 : kb2, rbs = first ? rb1 : rb2;
+        const int kb = (int)(blk % kbs);
+        const long long erb = blk / kbs;
+        const int rb = (int)(erb % rbs);
+        const long long e = erb / rbs;
+        const int k = kb * 128 + atom * 64 + c8 * 8;  // first K element of the chunk
+        const int rem = rb * 128 + r;                 // weight row within the expert
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (first) {
             const int g = (rem >> 4) & 1;
             const int f = (rem >> 7) * 64 + ((rem >> 5) & 3) * 16 + (rem & 15);
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (f < F && c * 8 < H) v = __ldg((g ? wu : wg) + (e * F + f) * (H / 8) + c);
+            if (f < F && k < H) v = __ldg((g ? wu : wg) + ((e * F + f) * H + k) / 8);
             w1[i] = v;
         } else {
-            const long long j = i - n1;
-            const long long row = j / c2;  // e * H + h
-            const int c = (int)(j - row * c2);
-            w2[j] = c * 8 < F ? __ldg(wd + row * (F / 8) + c) : make_uint4(0u, 0u, 0u, 0u);
+            if (rem < H && k < F) v = __ldg(wd + ((e * H + rem) * F + k) / 8);
+            w2[j] = v;
         }
     }
 }
@@ -55,7 +67,7 @@ cudaError_t launch_prepare_bf16(const moe_plan* p, const __nv_bfloat16* wg, cons
     prepare_bf16_kernel<<<num_sms() * 8, 256, 0, s>>>(
         reinterpret_cast<const uint4*>(wg), reinterpret_cast<const uint4*>(wu), reinterpret_cast<const uint4*>(wd),
         reinterpret_cast<uint4*>(base + p->wb.w1), reinterpret_cast<uint4*>(base + p->wb.w2), (int)E, (int)F, (int)H,
-        (int)p->hp, (int)p->fp);
+        (int)p->hp, (int)p->fp, (int)p->hr);
     return cudaGetLastError();
 }
 
