@@ -86,6 +86,7 @@ static void compute_layouts(moe_plan* p) {
     w.tiles = take((size_t)p->max_m_tiles * 16);
     w.perm = take(L * k * 4);
     w.inv = take(L * k * 4);
+    w.xrow = fp8 ? 0 : take(L * k * 4);
     const size_t mtiles = (size_t)p->max_m_tiles;
     if (fp8) {
         w.xq = take(R * (size_t)p->hp);
@@ -349,9 +350,10 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     int* perm = reinterpret_cast<int*>(ws + L.perm);
     int* inv = reinterpret_cast<int*>(ws + L.inv);
     int4* tiles = reinterpret_cast<int4*>(ws + L.tiles);
+    int* xrow = fp8 ? nullptr : reinterpret_cast<int*>(ws + L.xrow);
     e = launch_permute(plan, live_count_dev, r_ids, reinterpret_cast<int*>(ws + L.blkcnt),
                        reinterpret_cast<int*>(ws + L.offsets), reinterpret_cast<int*>(ws + L.padoff), tiles, perm, inv,
-                       status, s);
+                       xrow, status, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 
     if (!mark(2)) return MOE_ERR_CUDA;
@@ -359,9 +361,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
         e = launch_gather_mxfp8(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, (int)plan->hp, k,
                                 inv, ws + L.xq, ws + L.xs, s);
     else
-        e = launch_gather_bf16(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, (int)plan->hp, k, inv,
-                               r_ids, reinterpret_cast<const int*>(ws + L.offsets),
-                               reinterpret_cast<const int*>(ws + L.padoff), plan->tile_rows,
+        e = launch_gather_bf16(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, (int)plan->hp, k, xrow,
                                reinterpret_cast<__nv_bfloat16*>(ws + L.xq), s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 

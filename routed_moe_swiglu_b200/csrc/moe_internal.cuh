@@ -38,7 +38,7 @@ enum : int { kStFlags = 0, kStNumMTiles = 1, kStTotalRoutes = 2, kStWords = 64 }
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;
 
 struct WsLayout {
-    size_t status, r_ids, r_probs, blkcnt, offsets, padoff, tiles, perm, inv;
+    size_t status, r_ids, r_probs, blkcnt, offsets, padoff, tiles, perm, inv, xrow;
     size_t xq, xs, h, hs, y;
     size_t total;
 };
@@ -113,12 +113,13 @@ cudaError_t launch_route_topk(const float* logits, const int* live, int max_live
                               float* probs, unsigned* status, cudaStream_t s);
 cudaError_t launch_canon_routes(const int* ids_in, const float* probs_in, const int* live, int max_live, int E,
                                 int k, int* ids_out, float* probs_out, unsigned* status, cudaStream_t s);
+// xrow (bf16 only, else null): per route, its padded row if the gather kernel
+// writes it (tiles of more than kGatherInGemmMax routes), else -1
 cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* blkcnt, int* offsets,
-                           int* padoff, int4* tiles, int* perm, int* inv, unsigned* status_words,
+                           int* padoff, int4* tiles, int* perm, int* inv, int* xrow, unsigned* status_words,
                            cudaStream_t s);
 cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
-                               const int* inv, const int* ids, const int* offsets, const int* padoff, int tile_rows,
-                               __nv_bfloat16* xp, cudaStream_t s);
+                               const int* xrow, __nv_bfloat16* xp, cudaStream_t s);
 cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
                                 const int* inv, uint8_t* xq, uint8_t* xs, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const int* inv, const float* probs, const int* live, int max_live,

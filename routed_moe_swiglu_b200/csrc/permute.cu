@@ -86,10 +86,18 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int* __restrict_
     const int e = threadIdx.x;
     int tot = 0;
     if (e < E) {
-        for (int b = 0; b < nb; ++b) {
-            const int c = blkcnt[(size_t)b * E + e];
-            blkcnt[(size_t)b * E + e] = tot;  // becomes the exclusive prefix over earlier blocks
-            tot += c;
+        // each block's count becomes the exclusive prefix over earlier blocks; the counts
+        // of 16 blocks are loaded before any is rewritten, so the loads overlap
+        constexpr int kBatch = 16;
+        for (int b0 = 0; b0 < nb; b0 += kBatch) {
+            int c[kBatch];
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) c[i] = b0 + i < nb ? blkcnt[(size_t)(b0 + i) * E + e] : 0;
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+                if (b0 + i < nb) blkcnt[(size_t)(b0 + i) * E + e] = tot;
+                tot += c[i];
+            }
         }
     }
     const int mt = (tot + tile_rows - 1) / tile_rows;
@@ -117,8 +125,8 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int* __restrict_
 
 __global__ void __launch_bounds__(kTokPerBlk) route_scatter_kernel(
     const int* __restrict__ ids, const int* __restrict__ live, int max_live, int E, int k,
-    const int* __restrict__ blkprefix, const int* __restrict__ offsets, const int* __restrict__ padoff,
-    int* __restrict__ perm, int* __restrict__ inv) {
+    const int* __restrict__ blkprefix, const int* __restrict__ offsets, const int* __restrict__ padoff, int tile_rows,
+    int* __restrict__ perm, int* __restrict__ inv, int* __restrict__ xrow) {
     extern __shared__ uint32_t s_mem[];
     pdl_trigger();
     pdl_wait();
@@ -160,10 +168,18 @@ __global__ void __launch_bounds__(kTokPerBlk) route_scatter_kernel(
             const int e = my_e[j];
             if (e < 0) {
                 inv[(size_t)t * k + j] = -1;
+                if (xrow != nullptr) xrow[(size_t)t * k + j] = -1;
             } else {
                 const int row = wbase[w * E + e] + __popc(masks[w * E + e] & lower);
+                const int local = row - offsets[e];
                 perm[row] = t * k + j;
-                inv[(size_t)t * k + j] = padoff[e] + (row - offsets[e]);
+                inv[(size_t)t * k + j] = padoff[e] + local;
+                if (xrow != nullptr) {
+                    // the route's tile holds min(tile_rows, routes of e left from its first row)
+                    const int left = offsets[e + 1] - offsets[e] - local / tile_rows * tile_rows;
+                    xrow[(size_t)t * k + j] =
+                        (left < tile_rows ? left : tile_rows) > kGatherInGemmMax ? padoff[e] + local : -1;
+                }
             }
         }
     }
@@ -171,44 +187,43 @@ __global__ void __launch_bounds__(kTokPerBlk) route_scatter_kernel(
 
 constexpr int kRowThreads = 128;
 
-// bf16 gather: one 128-thread block per token (grid-stride) reads the
-// token's x row once and writes it to those of its k padded route rows that
-// lie in route tiles of more than kGatherInGemmMax routes; the gate/up GEMM
-// reads the rows of smaller tiles straight from x.  Every thread keeps all
-// of its 16-byte loads in flight before storing.
-__global__ void __launch_bounds__(kRowThreads) gather_rows_bf16_kernel(
+// bf16 gather: one warp per token (grid-stride) reads the token's x row
+// once and writes it to those of its k padded route rows that the scatter
+// marked (routes in tiles of more than kGatherInGemmMax routes; the gate/up
+// GEMM reads the x rows of smaller tiles itself).  Each lane keeps up to 8
+// of its 16-byte loads in flight before storing them.
+constexpr int kGatherWarps = 8;
+
+__global__ void __launch_bounds__(kGatherWarps * 32) gather_rows_bf16_kernel(
     const uint4* __restrict__ x, const int* __restrict__ live, int max_live, int H, int hp, int k,
-    const int* __restrict__ inv, const int* __restrict__ ids, const int* __restrict__ offsets,
-    const int* __restrict__ padoff, int tile_rows, uint4* __restrict__ xp) {
-    __shared__ int s_prow[kMaxTopK];
+    const int* __restrict__ xrow, uint4* __restrict__ xp) {
     pdl_trigger();
     pdl_wait();
     const int n = clamp_live(live, max_live);
+    const int lane = threadIdx.x & 31;
     const int chunks = H / 8;       // 8 bf16 per 16 bytes
     const int chunks_out = hp / 8;  // destination rows are padded to hp with zeros
-    for (int t = blockIdx.x; t < n; t += gridDim.x) {
-        __syncthreads();
-        if (threadIdx.x < k) {
-            int pr = __ldg(inv + (size_t)t * k + threadIdx.x);
-            if (pr >= 0) {
-                const int e = __ldg(ids + (size_t)t * k + threadIdx.x);
-                const int local = pr - __ldg(padoff + e);
-                const int left = __ldg(offsets + e + 1) - __ldg(offsets + e) - local / tile_rows * tile_rows;
-                if ((left < tile_rows ? left : tile_rows) <= kGatherInGemmMax) pr = -1;
-            }
-            s_prow[threadIdx.x] = pr;
-        }
-        __syncthreads();
-        bool any = false;
-        for (int j = 0; j < k; ++j) any |= s_prow[j] >= 0;
-        if (!any) continue;
+    const int warps = gridDim.x * kGatherWarps;
+    for (int t = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); t < n; t += warps) {
+        const int my_row = lane < k ? __ldg(xrow + (size_t)t * k + lane) : -1;
+        const unsigned targets = __ballot_sync(0xffffffffu, my_row >= 0);
+        if (targets == 0u) continue;
         const uint4* src = x + (size_t)t * chunks;
-#pragma unroll 4
-        for (int c = threadIdx.x; c < chunks_out; c += kRowThreads) {
-            const uint4 v = c < chunks ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-            for (int j = 0; j < k; ++j) {
-                const int pr = s_prow[j];
-                if (pr >= 0) xp[(size_t)pr * chunks_out + c] = v;
+        for (int c0 = 0; c0 < chunks_out; c0 += 8 * 32) {
+            uint4 v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c = c0 + i * 32 + lane;
+                v[i] = c < chunks ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            }
+            for (unsigned m = targets; m != 0u; m &= m - 1u) {
+                const int pr = __shfl_sync(0xffffffffu, my_row, __ffs(m) - 1);
+                uint4* dst = xp + (size_t)pr * chunks_out;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int c = c0 + i * 32 + lane;
+                    if (c < chunks_out) dst[c] = v[i];
+                }
             }
         }
     }
@@ -323,7 +338,7 @@ int grid_for_warps(long long items, int warps_per_block, int per_sm) {
 }  // namespace
 
 cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* blkcnt, int* offsets,
-                           int* padoff, int4* tiles, int* perm, int* inv, unsigned* status_words,
+                           int* padoff, int4* tiles, int* perm, int* inv, int* xrow, unsigned* status_words,
                            cudaStream_t s) {
     const int E = p->d.num_experts, k = p->d.top_k;
     const int max_live = (int)p->max_live;
@@ -349,16 +364,15 @@ cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* 
         }
     }
     return launch_dependent(route_scatter_kernel, dim3(nblk), dim3(kTokPerBlk), smem, s, r_ids, live, max_live, E, k,
-                            blkcnt, offsets, padoff, perm, inv);
+                            blkcnt, offsets, padoff, p->tile_rows, perm, inv, xrow);
 }
 
 cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
-                               const int* inv, const int* ids, const int* offsets, const int* padoff, int tile_rows,
-                               __nv_bfloat16* xp, cudaStream_t s) {
-    const int grid = grid_for_warps(max_live, 1, 16);
-    return launch_dependent(gather_rows_bf16_kernel, dim3(grid), dim3(kRowThreads), 0, s,
-                            reinterpret_cast<const uint4*>(x), live, max_live, H, hp, k, inv, ids, offsets, padoff,
-                            tile_rows, reinterpret_cast<uint4*>(xp));
+                               const int* xrow, __nv_bfloat16* xp, cudaStream_t s) {
+    const int grid = grid_for_warps(max_live, kGatherWarps, 8);
+    return launch_dependent(gather_rows_bf16_kernel, dim3(grid), dim3(kGatherWarps * 32), 0, s,
+                            reinterpret_cast<const uint4*>(x), live, max_live, H, hp, k, xrow,
+                            reinterpret_cast<uint4*>(xp));
 }
 
 cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,

@@ -14,9 +14,25 @@
 namespace moe {
 namespace {
 
+// Order-preserving map of a logit to an unsigned key: a larger logit gives a
+// larger key; -0 is taken as +0 and NaN as -infinity (a NaN never wins over a
+// number).  Key 0 is below every logit and marks an absent or taken slot.
+__device__ __forceinline__ uint32_t logit_key(float x) {
+    if (x != x) x = -INFINITY;
+    if (x == 0.0f) x = 0.0f;
+    const uint32_t b = __float_as_uint(x);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_logit(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key);
+}
+
 // One warp per token.  Logit `id` lives in lane id % 32, slot id / 32;
 // kSlots = ceil(E / 32) is a template parameter so the per-lane scans are
-// fully unrolled over registers.
+// fully unrolled over registers.  Each of the k rounds takes every lane's
+// best untaken slot (the lower slot, i.e. the lower id, on equal keys), a
+// warp max of the keys and a warp min of the ids holding that key: the
+// largest logit, ties to the lower expert id.
 template <int kSlots>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits,
                                                          const int* __restrict__ live, int max_live, int E,
@@ -33,50 +49,35 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
     const int warps_per_block = blockDim.x >> 5;
     for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < n; t += gridDim.x * warps_per_block) {
         const float* row = logits + (size_t)t * E;
-        float v[kSlots];
-        uint32_t taken = 0;
+        uint32_t key[kSlots];
 #pragma unroll
         for (int s = 0; s < kSlots; ++s) {
             const int id = lane + 32 * s;
-            float x = -INFINITY;
-            if (id < E) {
-                x = __ldg(row + id);
-                if (x != x) x = -INFINITY;  // NaN never wins over a number
-            } else {
-                taken |= 1u << s;
-            }
-            v[s] = x;
+            key[s] = id < E ? logit_key(__ldg(row + id)) : 0u;
         }
-        // k rounds of a warp arg-max on (value desc, id asc); every lane ends
-        // each round with the winner, lane j keeps round j's winner
         float first_v = 0.0f, my_v = 0.0f;
         int my_id = 0x7fffffff;
         for (int j = 0; j < k; ++j) {
-            float bv = 0.0f;
-            int bid = -1;
+            uint32_t best = 0u;
+            int bs = 0;
 #pragma unroll
-            for (int s = 0; s < kSlots; ++s) {
-                // ids grow with s inside a lane: strict '>' keeps the lower id on ties
-                if (!((taken >> s) & 1u) && (bid < 0 || v[s] > bv)) {
-                    bv = v[s];
-                    bid = lane + 32 * s;
+            for (int s = 0; s < kSlots; ++s)
+                if (key[s] > best) {
+                    best = key[s];
+                    bs = s;
                 }
-            }
+            const uint32_t wkey = __reduce_max_sync(0xffffffffu, best);
+            const uint32_t wid = __reduce_min_sync(0xffffffffu, best == wkey ? (uint32_t)(lane + 32 * bs) : 0xffffffffu);
+            if ((int)(wid & 31u) == lane) {
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oid = __shfl_xor_sync(0xffffffffu, bid, off);
-                const bool better = oid >= 0 && (bid < 0 || ov > bv || (ov == bv && oid < bid));
-                if (better) {
-                    bv = ov;
-                    bid = oid;
-                }
+                for (int s = 0; s < kSlots; ++s)
+                    if (s == (int)(wid >> 5)) key[s] = 0u;
             }
-            if ((bid & 31) == lane) taken |= 1u << (bid >> 5);
+            const float bv = key_logit(wkey);
             if (j == 0) first_v = bv;
             if (j == lane) {
                 my_v = bv;
-                my_id = bid;
+                my_id = (int)wid;
             }
         }
         // Renormalised softmax over the chosen k: exp(l_j - max) / sum, in
