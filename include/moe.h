@@ -250,6 +250,21 @@ moe_status moe_get_device_status(const void* workspace, unsigned* flags_host, vo
  * holds an undefined status word: clear it once before the first read. */
 moe_status moe_clear_device_status(void* workspace, void* stream);
 
+/* Diagnostic of the device-side failure detection (no counterpart in the
+ * pages).  Every pipeline wait inside the forward's kernels is bounded: a
+ * wait that runs out sets MOE_DEV_TIMEOUT in the status word, tells the
+ * other roles of its CTA to stop, and the kernel exits without trapping.
+ * This call runs that mechanism on the device without a forward: one CTA
+ * waits on mbarriers that nothing arrives on; the first wait gives up after
+ * `limit_ns` (1 ns .. 10 s) and sets MOE_DEV_TIMEOUT in *status_dev (a
+ * device word the caller owns; bits are OR-ed in), the second wait ends
+ * through the CTA's abort flag.  elapsed_ns_dev (nullable) receives the two
+ * waits' durations in ns, [0] the one that ran out, [1] the one that was
+ * told to stop.  Enqueued on `stream`; returns MOE_ERR_INVALID_ARG for a
+ * null status pointer or a limit outside the range. */
+moe_status moe_check_bounded_wait(unsigned long long limit_ns, unsigned* status_dev,
+                                  unsigned long long* elapsed_ns_dev, void* stream);
+
 /* Static string for a status code. */
 const char* moe_status_string(moe_status s);
 

@@ -36,6 +36,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_PKG, "libroutedmoe.so")
 
 MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
 MOE_DEV_LIVE_CLAMPED = 0x1
 MOE_DEV_BAD_ROUTE = 0x2
 MOE_DEV_TIMEOUT = 0x4
@@ -88,6 +89,7 @@ def load_library():
         "moe_get_workspace_views": ([P, P, ctypes.POINTER(_Views)], I),
         "moe_get_device_status": ([P, ctypes.POINTER(ctypes.c_uint), P], I),
         "moe_clear_device_status": ([P, P], I),
+        "moe_check_bounded_wait": ([ctypes.c_ulonglong, P, P, P], I),
         "moe_status_string": ([I], ctypes.c_char_p),
         "moe_version": ([], ctypes.c_char_p),
     }
@@ -273,3 +275,12 @@ def moe_get_device_status(workspace, stream=None) -> int:
 
 def moe_clear_device_status(workspace, stream=None) -> None:
     _check(load_library().moe_clear_device_status(_ptr(workspace), _stream(stream)), "moe_clear_device_status")
+
+
+def moe_check_bounded_wait(limit_ns: int, status, elapsed_ns=None, stream=None) -> None:
+    """Run the device's bounded-wait check (see include/moe.h): `status` is a
+    device int32 tensor of one element the MOE_DEV_* bits are OR-ed into,
+    `elapsed_ns` an optional device int64 tensor of two elements."""
+    _check(load_library().moe_check_bounded_wait(int(limit_ns), _ptr(status),
+                                                 _ptr(elapsed_ns) if elapsed_ns is not None else None,
+                                                 _stream(stream)), "moe_check_bounded_wait")

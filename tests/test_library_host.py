@@ -112,3 +112,11 @@ def test_product_path_does_not_touch_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in txt and "moe_oracle" not in txt and "from oracle" not in txt, f
+
+
+def test_bounded_wait_check_rejects_bad_arguments_before_launch():
+    lib = rm.load_library()
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    assert lib.moe_check_bounded_wait(0, fake, None, None) == 1
+    assert lib.moe_check_bounded_wait(10_000_000_001, fake, None, None) == 1
+    assert lib.moe_check_bounded_wait(1000, None, None, None) == 1
