@@ -52,10 +52,13 @@ def _load():
     lib.oracle_mxfp8_dequantize.argtypes = [P, P, I64, I64, P]
     lib.oracle_route.argtypes = [P, I64, I, I, P, P]
     lib.oracle_permute.argtypes = [P, I64, I, I, P, P, P]
-    lib.oracle_forward_bf16.argtypes = [P, P, P, P, P, P, I64, I, I, I, I, P, I64, P, P]
-    lib.oracle_forward_mxfp8.argtypes = [P, P, P, P, P, P, P, P, P, I64, I, I, I, I, P, I64, P, P, P, P]
+    D = ctypes.c_double
+    lib.oracle_forward_bf16.argtypes = [P, P, P, P, P, P, I64, I, I, I, I, P, I64, P, P, I, D]
+    lib.oracle_forward_mxfp8.argtypes = [P, P, P, P, P, P, P, P, P, I64, I, I, I, I, P, I64, P, P, P, P, I, D]
+    lib.oracle_round_bf16.argtypes = [P, I64, P]
     for name in ("oracle_mxfp8_quantize", "oracle_mxfp8_quantize_bf16", "oracle_mxfp8_dequantize",
-                 "oracle_route", "oracle_permute", "oracle_forward_bf16", "oracle_forward_mxfp8"):
+                 "oracle_route", "oracle_permute", "oracle_forward_bf16", "oracle_forward_mxfp8",
+                 "oracle_round_bf16"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -146,11 +149,34 @@ def mxfp8_dequantize(q: np.ndarray, s: np.ndarray) -> np.ndarray:
     return out
 
 
-def forward_bf16(x, ids, probs, w_gate, w_up, w_down, tokens=None, want_h=False):
+PROBS_IN_FC1 = 1
+
+
+def _variant(probs_in_fc1, gate_up_clamp):
+    flags = PROBS_IN_FC1 if probs_in_fc1 else 0
+    clamp = float(gate_up_clamp) if gate_up_clamp else 0.0
+    return flags, clamp
+
+
+def round_bf16(out):
+    """The bf16 finalize: fp32 values rounded to bf16 (nearest even); returns
+    the bf16 bit patterns as uint16."""
+    a = np.ascontiguousarray(out, dtype=np.float32)
+    r = np.empty(a.shape, np.uint16)
+    _check(_load().oracle_round_bf16(_ptr(a), a.size, _ptr(r)), "round_bf16")
+    return r
+
+
+def forward_bf16(x, ids, probs, w_gate, w_up, w_down, tokens=None, want_h=False, probs_in_fc1=False,
+                 gate_up_clamp=None):
     """bf16 routed SwiGLU forward for `tokens` (default: all rows of ids).
 
     x [T,H] bf16, ids/probs [T,k], w_gate/w_up [E,F,H] bf16, w_down [E,H,F] bf16.
-    Returns out fp32 [ntok, H] (and h fp32 [ntok, k, F] when want_h)."""
+    Returns out fp32 [ntok, H] (and h fp32 [ntok, k, F] when want_h).
+    probs_in_fc1 / gate_up_clamp select the variants described in
+    moe_oracle.c (probability applied to the SwiGLU row; clamp of the gate
+    and up pre-activations)."""
+    flags, clamp = _variant(probs_in_fc1, gate_up_clamp)
     xb = _bf16_bits(x)
     gb, ub, db = _bf16_bits(w_gate), _bf16_bits(w_up), _bf16_bits(w_down)
     ids = np.ascontiguousarray(ids, dtype=np.int32)
@@ -162,7 +188,8 @@ def forward_bf16(x, ids, probs, w_gate, w_up, w_down, tokens=None, want_h=False)
     out = np.empty((toks.size, H), np.float32)
     h = np.empty((toks.size, k, F), np.float32) if want_h else None
     _check(_load().oracle_forward_bf16(_ptr(xb), _ptr(ids), _ptr(probs), _ptr(gb), _ptr(ub), _ptr(db),
-                                       xb.shape[0], H, F, E, k, _ptr(toks), toks.size, _ptr(out), _ptr(h)),
+                                       xb.shape[0], H, F, E, k, _ptr(toks), toks.size, _ptr(out), _ptr(h),
+                                       flags, clamp),
            "forward_bf16")
     return (out, h) if want_h else out
 
@@ -176,11 +203,13 @@ def quantize_weights_mxfp8(w_gate, w_up, w_down):
     return gq, gs, uq, us, dq, ds
 
 
-def forward_mxfp8(x, ids, probs, wq, tokens=None, want_h=False):
+def forward_mxfp8(x, ids, probs, wq, tokens=None, want_h=False, probs_in_fc1=False, gate_up_clamp=None):
     """MXFP8 routed SwiGLU forward; `wq` = quantize_weights_mxfp8(...) output.
 
     Returns out fp32 [ntok, H] and, when want_h, (h codes [ntok,k,F],
-    h scales [ntok,k,F/32], h pre-quantisation fp32 [ntok,k,F])."""
+    h scales [ntok,k,F/32], h pre-quantisation fp32 [ntok,k,F]).  Variants
+    as in forward_bf16."""
+    flags, clamp = _variant(probs_in_fc1, gate_up_clamp)
     xb = _bf16_bits(x)
     gq, gs, uq, us, dq, ds = wq
     ids = np.ascontiguousarray(ids, dtype=np.int32)
@@ -196,6 +225,6 @@ def forward_mxfp8(x, ids, probs, wq, tokens=None, want_h=False):
         hf = np.empty((toks.size, k, F), np.float32)
     _check(_load().oracle_forward_mxfp8(_ptr(xb), _ptr(ids), _ptr(probs), _ptr(gq), _ptr(gs), _ptr(uq),
                                         _ptr(us), _ptr(dq), _ptr(ds), xb.shape[0], H, F, E, k, _ptr(toks),
-                                        toks.size, _ptr(out), _ptr(hq), _ptr(hs), _ptr(hf)),
+                                        toks.size, _ptr(out), _ptr(hq), _ptr(hs), _ptr(hf), flags, clamp),
            "forward_mxfp8")
     return (out, (hq, hs, hf)) if want_h else out

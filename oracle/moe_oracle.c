@@ -45,6 +45,19 @@
  *   - an all-zero MXFP8 block gets scale byte 0 (2^-127); negative values
  *     that round to zero keep their sign (code 0x80).
  *
+ * Variants (cudnn-frontend PR #448, the MoeEp constructor's options;
+ * Megatron-LM PR #8367 for the finalize's output type), each off by default:
+ *   ORACLE_PROBS_IN_FC1 -- `apply_topk_in_fc1`: the route's probability
+ *       multiplies the SwiGLU row before it is rounded for FC2,
+ *       h_f = round(fp32(p_j * silu(g_f) * u_f)), and the combine adds the
+ *       routes' rows as fp32 additions from 0.0f in ascending id.
+ *   clamp > 0          -- `gate_up_clamp`: the gate and up pre-activations
+ *       (the FC1 accumulator) are clamped to [-clamp, clamp] before SwiGLU.
+ *   oracle_round_bf16  -- a bf16 finalize output: the fp32 sum rounded to
+ *       bf16 (round-to-nearest-even), as the pages' BF16 finalize does.
+ *   The pages name these options but give no formula; the readings above
+ *   are the plainest ones and are listed in the design notes.
+ *
  * Build: gcc -O2 -fopenmp -shared -fPIC (no -ffast-math: fmaf and the
  * double sums must keep IEEE semantics).
  */
@@ -317,6 +330,28 @@ int oracle_permute(const int32_t* ids, int64_t T, int E, int k,
 
 static double silu_d(double z) { return z / (1.0 + exp(-z)); }
 
+#define ORACLE_PROBS_IN_FC1 1
+
+/* The fp32 SwiGLU value of one (route, f) from its double pre-activations:
+ * clamped when clamp > 0, scaled by the route's probability when the
+ * probabilities are applied in FC1. */
+static float swiglu_value(double g, double u, double clamp, int flags, float p) {
+    if (clamp > 0.0) {
+        g = g < -clamp ? -clamp : (g > clamp ? clamp : g);
+        u = u < -clamp ? -clamp : (u > clamp ? clamp : u);
+    }
+    double h = silu_d(g) * u;
+    if (flags & ORACLE_PROBS_IN_FC1) h *= (double)p;
+    return (float)h;
+}
+
+/* out[i] = bf16(in[i]) with round-to-nearest-even, for a bf16 finalize. */
+int oracle_round_bf16(const float* in, int64_t n, uint16_t* out) {
+    if (!in || !out || n < 0) return ORACLE_EINVAL;
+    for (int64_t i = 0; i < n; ++i) out[i] = float_to_bf16_bits_rne(in[i]);
+    return ORACLE_OK;
+}
+
 /* Canonical order of one token's routes: ascending expert id, carrying the
  * probability with its id. */
 static void sort_routes(const int32_t* ids_in, const float* p_in, int k, int* ids, float* p) {
@@ -341,11 +376,13 @@ static void sort_routes(const int32_t* ids_in, const float* p_in, int k, int* id
  *          route, in canonical (ascending id) order.
  * Per route: g_f = sum_c Wg[e,f,c] x_c and u_f likewise (double);
  * h_f = bf16(fp32(silu(g_f) * u_f)); y_c = fp32(sum_f Wd[e,c,f] h_f);
- * out_c = fmaf(p_j, y_c, out_c) over j in ascending id, from 0.0f. */
+ * out_c = fmaf(p_j, y_c, out_c) over j in ascending id, from 0.0f.
+ * flags / clamp select the variants above (0, 0.0: the plain forward). */
 int oracle_forward_bf16(const uint16_t* x, const int32_t* ids, const float* probs,
                         const uint16_t* w_gate, const uint16_t* w_up, const uint16_t* w_down,
                         int64_t T, int H, int F, int E, int k,
-                        const int64_t* toks, int64_t ntok, float* out, float* h_out) {
+                        const int64_t* toks, int64_t ntok, float* out, float* h_out,
+                        int flags, double clamp) {
     if (!x || !ids || !probs || !w_gate || !w_up || !w_down || !toks || !out) return ORACLE_EINVAL;
     if (H <= 0 || F <= 0 || E <= 0 || k <= 0 || k > 64 || ntok < 0) return ORACLE_EINVAL;
     int bad = 0;
@@ -374,7 +411,7 @@ int oracle_forward_bf16(const uint16_t* x, const int32_t* ids, const float* prob
                     g += (double)bf16_bits_to_float(wg[(int64_t)f * H + c]) * xd[c];
                     u += (double)bf16_bits_to_float(wu[(int64_t)f * H + c]) * xd[c];
                 }
-                float hf = (float)(silu_d(g) * u);
+                float hf = swiglu_value(g, u, clamp, flags, sp[j]);
                 float hb = bf16_bits_to_float(float_to_bf16_bits_rne(hf));
                 hd[f] = (double)hb;
                 if (h_out) h_out[(i * k + j) * F + f] = hb;
@@ -382,7 +419,7 @@ int oracle_forward_bf16(const uint16_t* x, const int32_t* ids, const float* prob
             for (int c = 0; c < H; ++c) {
                 double y = 0.0;
                 for (int f = 0; f < F; ++f) y += (double)bf16_bits_to_float(wd[(int64_t)c * F + f]) * hd[f];
-                acc[c] = fmaf(sp[j], (float)y, acc[c]);
+                acc[c] = (flags & ORACLE_PROBS_IN_FC1) ? acc[c] + (float)y : fmaf(sp[j], (float)y, acc[c]);
             }
         }
         free(xd);
@@ -401,14 +438,15 @@ int oracle_forward_bf16(const uint16_t* x, const int32_t* ids, const float* prob
  * path up to its fp32 value, then quantised (blocks of 32 along F) and the
  * dequantised h enters the down GEMM.
  *   h_q_out [ntok, k, F] codes and h_s_out [ntok, k, F/32] (nullable),
- *   h_f32_out [ntok, k, F] pre-quantisation fp32 h (nullable). */
+ *   h_f32_out [ntok, k, F] pre-quantisation fp32 h (nullable).
+ * flags / clamp select the variants above (0, 0.0: the plain forward). */
 int oracle_forward_mxfp8(const uint16_t* x, const int32_t* ids, const float* probs,
                          const uint8_t* wg_q, const uint8_t* wg_s,
                          const uint8_t* wu_q, const uint8_t* wu_s,
                          const uint8_t* wd_q, const uint8_t* wd_s,
                          int64_t T, int H, int F, int E, int k,
                          const int64_t* toks, int64_t ntok, float* out,
-                         uint8_t* h_q_out, uint8_t* h_s_out, float* h_f32_out) {
+                         uint8_t* h_q_out, uint8_t* h_s_out, float* h_f32_out, int flags, double clamp) {
     if (!x || !ids || !probs || !wg_q || !wg_s || !wu_q || !wu_s || !wd_q || !wd_s || !toks || !out)
         return ORACLE_EINVAL;
     if (H <= 0 || F <= 0 || (H % 32) || (F % 32) || E <= 0 || k <= 0 || k > 64 || ntok < 0)
@@ -459,7 +497,7 @@ int oracle_forward_mxfp8(const uint16_t* x, const int32_t* ids, const float* pro
                     g += wgv * xd[c];
                     u += wuv * xd[c];
                 }
-                float hf = (float)(silu_d(g) * u);
+                float hf = swiglu_value(g, u, clamp, flags, sp[j]);
                 hv[f] = (double)hf;
                 if (h_f32_out) h_f32_out[(i * k + j) * F + f] = hf;
             }
@@ -474,7 +512,7 @@ int oracle_forward_mxfp8(const uint16_t* x, const int32_t* ids, const float* pro
                 double y = 0.0;
                 for (int f = 0; f < F; ++f)
                     y += g_e4m3_all[dq[(int64_t)c * F + f]] * g_pow2[ds[(int64_t)c * nbf + f / 32]] * hd[f];
-                acc[c] = fmaf(sp[j], (float)y, acc[c]);
+                acc[c] = (flags & ORACLE_PROBS_IN_FC1) ? acc[c] + (float)y : fmaf(sp[j], (float)y, acc[c]);
             }
         }
         free(xv); free(xd); free(hv); free(hd); free(qb);

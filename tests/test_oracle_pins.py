@@ -405,3 +405,96 @@ def test_forward_mxfp8_close_to_bf16():
     b = oracle.forward_mxfp8(x, ids, probs, oracle.quantize_weights_mxfp8(wg, wu, wd)).astype(np.float64)
     d = np.linalg.norm(b - a) / np.linalg.norm(a)
     assert 0.005 < d < 0.12
+
+
+# ---------------------------------------------------------------- variants (apply_topk_in_fc1, clamp, bf16 out)
+
+
+def _pow2_probs(ids, seed):
+    """Per-route probabilities that are powers of two (1/2, 1/4, 1/8)."""
+    rng = np.random.default_rng(seed)
+    return (2.0 ** -rng.integers(1, 4, size=ids.shape)).astype(np.float32)
+
+
+def test_variant_probs_in_fc1_pow2_probs_equal_plain_forward():
+    # scaling the SwiGLU row by a power of two commutes with the fp32 and bf16
+    # roundings and scales y exactly, and acc + p*y is then the plain fmaf(p, y, acc):
+    # both variants must agree bit for bit (a dropped or doubled probability fails)
+    x, wg, wu, wd, ids, _ = _small_problem(21, T=10, k=3)
+    probs = _pow2_probs(ids, 21)
+    plain = oracle.forward_bf16(x, ids, probs, wg, wu, wd)
+    fc1 = oracle.forward_bf16(x, ids, probs, wg, wu, wd, probs_in_fc1=True)
+    assert np.array_equal(plain, fc1)
+    wq = oracle.quantize_weights_mxfp8(wg, wu, wd)
+    plain8 = oracle.forward_mxfp8(x, ids, probs, wq)
+    fc18 = oracle.forward_mxfp8(x, ids, probs, wq, probs_in_fc1=True)
+    assert np.array_equal(plain8, fc18)
+
+
+def _dense_variant_ref(x, wg, wu, wd, p=None, clamp=None):
+    """torch float64 dense SwiGLU MLP: pre-activations clamped to [-clamp, clamp],
+    the row scaled by p, rounded to fp32 then bf16; y in fp32."""
+    x64 = x.to(torch.float64)
+    g = x64 @ wg.to(torch.float64).T
+    u = x64 @ wu.to(torch.float64).T
+    if clamp is not None:
+        g, u = g.clamp(-clamp, clamp), u.clamp(-clamp, clamp)
+    h = torch.nn.functional.silu(g) * u
+    if p is not None:
+        h = h * p
+    h = h.to(torch.float32).to(torch.bfloat16).to(torch.float64)
+    return (h @ wd.to(torch.float64).T).to(torch.float32)
+
+
+def _single_expert(seed, T=20, H=96, F=160):
+    gen = torch.Generator().manual_seed(seed)
+    x = rand_bf16(gen, (T, H))
+    wg = rand_bf16(gen, (1, F, H), H ** -0.5)
+    wu = rand_bf16(gen, (1, F, H), H ** -0.5)
+    wd = rand_bf16(gen, (1, H, F), F ** -0.5)
+    return x, wg, wu, wd, np.zeros((T, 1), np.int32)
+
+
+def _close_to_dense(out, ref):
+    rms = float(np.sqrt(np.mean(ref.numpy().astype(np.float64) ** 2)))
+    # rare bf16 rounding flips of h where the two double sums differ in the last bit
+    assert np.max(np.abs(out - ref.numpy())) <= 1e-3 * rms
+    assert np.mean(np.abs(out - ref.numpy())) <= 1e-6 * rms
+
+
+def test_variant_probs_in_fc1_is_dense_mlp_times_p_before_rounding():
+    x, wg, wu, wd, ids = _single_expert(22)
+    p = np.full(ids.shape, 0.3, np.float32)
+    out = oracle.forward_bf16(x, ids, p, wg, wu, wd, probs_in_fc1=True)
+    ref = _dense_variant_ref(x, wg[0], wu[0], wd[0], p=float(np.float32(0.3)))
+    _close_to_dense(out, ref)
+    # and not the plain forward (p applied once, after FC2)
+    plain = oracle.forward_bf16(x, ids, p, wg, wu, wd)
+    assert not np.array_equal(out, plain)
+
+
+def test_variant_clamp_matches_dense_reference_and_is_inert_when_wide():
+    x, wg, wu, wd, ids = _single_expert(23)
+    one = np.ones(ids.shape, np.float32)
+    c = 0.25  # |g|, |u| ~ N(0, 1): most pre-activations are clamped
+    out = oracle.forward_bf16(x, ids, one, wg, wu, wd, gate_up_clamp=c)
+    _close_to_dense(out, _dense_variant_ref(x, wg[0], wu[0], wd[0], clamp=c))
+    plain = oracle.forward_bf16(x, ids, one, wg, wu, wd)
+    assert not np.array_equal(out, plain)
+    wide = oracle.forward_bf16(x, ids, one, wg, wu, wd, gate_up_clamp=1e6)
+    assert np.array_equal(wide, plain)
+
+
+def test_round_bf16_matches_torch_cast_including_ties():
+    rng = np.random.default_rng(24)
+    a = (rng.standard_normal(4096) * np.exp(rng.standard_normal(4096) * 4)).astype(np.float32)
+    # exact ties: low 16 bits 0x8000, with even and odd kept halves
+    ties = (rng.integers(0x3F000000, 0x43000000, size=512, dtype=np.uint32) & 0xFFFF0000) | 0x8000
+    a = np.concatenate([a, ties.view(np.float32), -ties.view(np.float32), np.float32([0.0, -0.0])])
+    got = oracle.round_bf16(a)
+    ref = torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, ref)
+    # ties go to the even kept half
+    t = ties.view(np.float32)
+    kept = oracle.round_bf16(t)
+    assert np.all(kept & 1 == 0)
