@@ -83,7 +83,23 @@ typedef struct {
                                 0 means capacity.  The workspace is sized for it;
                                 larger live counts are clamped and flagged.       */
     moe_precision precision; /* MOE_BF16 or MOE_MXFP8                             */
+    unsigned flags;          /* MOE_FLAG_* variants; 0 for the plain forward      */
+    float gate_up_clamp;     /* > 0: gate and up pre-activations clamped to
+                                [-gate_up_clamp, gate_up_clamp] before SwiGLU
+                                (cudnn-frontend PR #448, MoeEp `gate_up_clamp`);
+                                0: no clamp                                       */
 } moe_desc;
+
+/* Variants of the forward the pages' kernels offer (cudnn-frontend PR #448,
+ * the MoeEp constructor; Megatron-LM PR #8367 for the output type):
+ *   MOE_FLAG_PROBS_IN_FC1  `apply_topk_in_fc1`: each route's probability
+ *       multiplies its SwiGLU row before that row is rounded for the down
+ *       GEMM, h = round(p * silu(g) * u); the combine then adds the routes'
+ *       rows as fp32 additions from 0.0f in ascending expert id.
+ *   MOE_FLAG_OUT_BF16      bf16 finalize: out is bf16 [capacity, H], the
+ *       fp32 sum rounded to nearest even (the plain output is fp32). */
+#define MOE_FLAG_PROBS_IN_FC1 0x1u
+#define MOE_FLAG_OUT_BF16 0x2u
 
 typedef struct moe_plan moe_plan; /* opaque, host memory only */
 
@@ -91,7 +107,8 @@ typedef struct moe_plan moe_plan; /* opaque, host memory only */
  * allocation).  Rejected (MOE_ERR_UNSUPPORTED): H or F not a multiple of 8
  * (bf16) or of 32 (MXFP8); k < 1, k > 16 or k > E; E < 1 or E > 1024;
  * capacity < 1 or > 2^24 rows; max_live_rows < 0 or > capacity;
- * H > 16384 or F > 16384. */
+ * H > 16384 or F > 16384.  Rejected (MOE_ERR_INVALID_ARG): unknown flag
+ * bits, a negative or non-finite gate_up_clamp. */
 moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out);
 void moe_plan_destroy(moe_plan* plan);
 /* Copy of the descriptor the plan was made from (max_live_rows resolved). */
@@ -156,12 +173,15 @@ moe_status moe_route_topk(const moe_plan* plan, const float* logits, const int* 
  *            y_j = W_down[e_j] . (silu(W_gate[e_j] . x_t) * (W_up[e_j] . x_t))
  *            with the SwiGLU row rounded to bf16 (or re-quantised to MXFP8)
  *            and y_j kept in fp32.  Rows >= live count are not written.
+ *            The plan's flags change this as MOE_FLAG_* states (bf16 out,
+ *            probabilities applied in FC1), and gate_up_clamp clamps the
+ *            two pre-activations before silu and the product.
  *   workspace  moe_workspace_bytes(plan) bytes, 256-byte aligned.
  * Each token's output is bitwise independent of the live count and of the
  * other tokens in the launch. */
 moe_status moe_forward(const moe_plan* plan, const void* x, const float* logits, const int* ids,
                        const float* probs, const void* kernel_buf, const int* live_count_dev,
-                       float* out, void* workspace, size_t ws_bytes, void* stream);
+                       void* out, void* workspace, size_t ws_bytes, void* stream);
 
 /* moe_forward for callers that cannot allocate device memory (no
  * counterpart in the pages: an addition of this library).  Some callers get
@@ -188,7 +208,7 @@ moe_status moe_forward(const moe_plan* plan, const void* x, const float* logits,
 #define MOE_NOALLOC_SCRATCH_BYTES (64ull << 20)
 moe_status moe_forward_noalloc(const moe_plan* plan, const void* x, const float* logits, const int* ids,
                                const float* probs, const void* kernel_buf, const int* live_count_dev,
-                               float* out, void* stream);
+                               void* out, void* stream);
 
 /* Stages of moe_forward, in launch order: route (or canonicalise the
  * caller's routes), permute (histogram, scan, scatter), gather of x rows
@@ -204,7 +224,7 @@ moe_status moe_forward_noalloc(const moe_plan* plan, const void* x, const float*
  * moe_forward. */
 moe_status moe_forward_with_events(const moe_plan* plan, const void* x, const float* logits, const int* ids,
                                    const float* probs, const void* kernel_buf, const int* live_count_dev,
-                                   float* out, void* workspace, size_t ws_bytes, void* stream,
+                                   void* out, void* workspace, size_t ws_bytes, void* stream,
                                    void* const* stage_events);
 
 /* Views into a workspace after a forward (device pointers into it), for

@@ -40,6 +40,8 @@ MOE_ERR_INVALID_ARG = 1
 MOE_DEV_LIVE_CLAMPED = 0x1
 MOE_DEV_BAD_ROUTE = 0x2
 MOE_DEV_TIMEOUT = 0x4
+MOE_FLAG_PROBS_IN_FC1 = 0x1
+MOE_FLAG_OUT_BF16 = 0x2
 _PRECISION = {"bf16": 0, "mxfp8": 1}
 
 
@@ -52,7 +54,7 @@ class MoeError(RuntimeError):
 class _Desc(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int), ("ffn", ctypes.c_int), ("num_experts", ctypes.c_int),
                 ("top_k", ctypes.c_int), ("capacity", ctypes.c_longlong), ("max_live_rows", ctypes.c_longlong),
-                ("precision", ctypes.c_int)]
+                ("precision", ctypes.c_int), ("flags", ctypes.c_uint), ("gate_up_clamp", ctypes.c_float)]
 
 
 class _Views(ctypes.Structure):
@@ -145,6 +147,9 @@ class Plan:
         self.capacity = desc.capacity
         self.max_live_rows = desc.max_live_rows
         self.precision = {v: k for k, v in _PRECISION.items()}[desc.precision]
+        self.probs_in_fc1 = bool(desc.flags & MOE_FLAG_PROBS_IN_FC1)
+        self.out_dtype = "bf16" if desc.flags & MOE_FLAG_OUT_BF16 else "fp32"
+        self.gate_up_clamp = float(desc.gate_up_clamp)
 
     @property
     def handle(self):
@@ -163,9 +168,17 @@ class Plan:
 
 
 def moe_plan_create(hidden: int, ffn: int, num_experts: int, top_k: int, capacity: int,
-                    precision: str = "bf16", max_live_rows: int = 0) -> Plan:
+                    precision: str = "bf16", max_live_rows: int = 0, out_dtype: str = "fp32",
+                    probs_in_fc1: bool = False, gate_up_clamp: float | None = None) -> Plan:
+    """out_dtype "fp32" or "bf16" (MOE_FLAG_OUT_BF16); probs_in_fc1 applies each
+    route's probability to its SwiGLU row (MOE_FLAG_PROBS_IN_FC1); gate_up_clamp
+    clamps the gate and up pre-activations (None: no clamp)."""
     lib = load_library()
-    d = _Desc(hidden, ffn, num_experts, top_k, capacity, max_live_rows, _PRECISION[precision])
+    if out_dtype not in ("fp32", "bf16"):
+        raise ValueError(f"out_dtype must be 'fp32' or 'bf16', not {out_dtype!r}")
+    flags = (MOE_FLAG_OUT_BF16 if out_dtype == "bf16" else 0) | (MOE_FLAG_PROBS_IN_FC1 if probs_in_fc1 else 0)
+    d = _Desc(hidden, ffn, num_experts, top_k, capacity, max_live_rows, _PRECISION[precision], flags,
+              float(gate_up_clamp) if gate_up_clamp else 0.0)
     h = ctypes.c_void_p()
     _check(lib.moe_plan_create(ctypes.byref(d), ctypes.byref(h)), "moe_plan_create")
     out = _Desc()
@@ -217,8 +230,17 @@ def moe_route_topk(plan: Plan, logits, live_count, ids, probs, stream=None) -> N
                                          _stream(stream)), "moe_route_topk")
 
 
+def _check_out(plan: Plan, out) -> None:
+    import torch
+
+    want = torch.bfloat16 if plan.out_dtype == "bf16" else torch.float32
+    if out.dtype != want:
+        raise ValueError(f"out must be {want} for this plan, not {out.dtype}")
+
+
 def moe_forward(plan: Plan, x, kernel_buf, live_count, out, workspace, logits=None, ids=None, probs=None,
                 stream=None) -> None:
+    _check_out(plan, out)
     _check(load_library().moe_forward(plan.handle, _ptr(x), _ptr(logits), _ptr(ids), _ptr(probs), _ptr(kernel_buf),
                                       _ptr(live_count), _ptr(out), _ptr(workspace),
                                       workspace.numel() * workspace.element_size(), _stream(stream)), "moe_forward")
@@ -233,6 +255,7 @@ def moe_forward_noalloc(plan: Plan, x, kernel_buf, live_count, out, logits=None,
     memory: the library's own fixed scratch array (MOE_NOALLOC_SCRATCH_BYTES)
     serves every call, so calls must not overlap on the GPU.  Make the first
     call on a device outside any stream capture."""
+    _check_out(plan, out)
     _check(load_library().moe_forward_noalloc(plan.handle, _ptr(x), _ptr(logits), _ptr(ids), _ptr(probs),
                                               _ptr(kernel_buf), _ptr(live_count), _ptr(out), _stream(stream)),
            "moe_forward_noalloc")
@@ -246,6 +269,7 @@ def moe_forward_with_events(plan: Plan, x, kernel_buf, live_count, out, workspac
                             probs=None, stream=None) -> None:
     """moe_forward recording torch.cuda.Event objects `events` (MOE_NUM_STAGES + 1,
     enable_timing=True) around each stage."""
+    _check_out(plan, out)
     if len(events) != MOE_NUM_STAGES + 1:
         raise ValueError("need MOE_NUM_STAGES + 1 events")
     if any(e.cuda_event == 0 for e in events):

@@ -154,6 +154,8 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     if (d.num_experts > kMaxExperts || d.top_k > kMaxTopK || d.top_k > d.num_experts) return MOE_ERR_UNSUPPORTED;
     if (d.capacity > (1ll << 24)) return MOE_ERR_UNSUPPORTED;
     if (d.max_live_rows < 0 || d.max_live_rows > d.capacity) return MOE_ERR_UNSUPPORTED;
+    if ((d.flags & ~(MOE_FLAG_PROBS_IN_FC1 | MOE_FLAG_OUT_BF16)) != 0) return MOE_ERR_INVALID_ARG;
+    if (!(d.gate_up_clamp >= 0.0f) || d.gate_up_clamp > 3.0e38f) return MOE_ERR_INVALID_ARG;
     moe_plan* p = new (std::nothrow) moe_plan();
     if (p == nullptr) return MOE_ERR_INVALID_ARG;
     p->d = d;
@@ -239,7 +241,7 @@ moe_status moe_route_topk(const moe_plan* plan, const float* logits, const int* 
 namespace {
 
 static moe_status forward_impl(const moe_plan* plan, const void* x, const float* logits, const int* ids,
-                               const float* probs, const void* kernel_buf, const int* live_count_dev, float* out,
+                               const float* probs, const void* kernel_buf, const int* live_count_dev, void* out,
                                void* workspace, size_t ws_bytes, void* stream, void* const* stage_events) {
     if (plan == nullptr || x == nullptr || kernel_buf == nullptr || live_count_dev == nullptr || out == nullptr ||
         workspace == nullptr)
@@ -384,6 +386,9 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g1.sf_ks_out = plan->ks2;
     g1.perm = perm;
     g1.top_k = k;
+    const bool probs_in_fc1 = (plan->d.flags & MOE_FLAG_PROBS_IN_FC1) != 0;
+    g1.route_probs = probs_in_fc1 ? r_probs : nullptr;
+    g1.clamp = plan->d.gate_up_clamp;
     if (!mark(3)) return MOE_ERR_CUDA;
     e = fp8 ? launch_gemm1_mxfp8(tA1, rB1, g1, m_tiles * g1.n_tiles, s)
             : launch_gemm1_bf16_pair(tA1, tX, rB1, g1, m_tiles * g1.n_tiles, s);
@@ -405,7 +410,9 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     if (!mark(5)) return MOE_ERR_CUDA;
 
-    e = launch_combine(reinterpret_cast<const float*>(ws + L.y), inv, r_probs, live_count_dev, max_live, H, k, out, s);
+    // the probabilities were applied in the gate/up epilogue: the combine adds the rows
+    e = launch_combine(reinterpret_cast<const float*>(ws + L.y), inv, probs_in_fc1 ? nullptr : r_probs,
+                       live_count_dev, max_live, H, k, out, (plan->d.flags & MOE_FLAG_OUT_BF16) != 0, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     return mark(6) ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -415,14 +422,14 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
 extern "C" {
 
 moe_status moe_forward(const moe_plan* plan, const void* x, const float* logits, const int* ids, const float* probs,
-                       const void* kernel_buf, const int* live_count_dev, float* out, void* workspace,
+                       const void* kernel_buf, const int* live_count_dev, void* out, void* workspace,
                        size_t ws_bytes, void* stream) {
     return forward_impl(plan, x, logits, ids, probs, kernel_buf, live_count_dev, out, workspace, ws_bytes, stream,
                         nullptr);
 }
 
 moe_status moe_forward_with_events(const moe_plan* plan, const void* x, const float* logits, const int* ids,
-                                   const float* probs, const void* kernel_buf, const int* live_count_dev, float* out,
+                                   const float* probs, const void* kernel_buf, const int* live_count_dev, void* out,
                                    void* workspace, size_t ws_bytes, void* stream, void* const* stage_events) {
     if (stage_events == nullptr) return MOE_ERR_INVALID_ARG;
     for (int i = 0; i <= MOE_NUM_STAGES; ++i)

@@ -83,6 +83,16 @@ struct __align__(8) Barriers {
 
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
+// silu(g) * u, the two pre-activations first clamped to [-clamp, clamp] when clamp > 0
+// (the MoeEp `gate_up_clamp` option of cudnn-frontend PR #448)
+__device__ __forceinline__ float swiglu_value(float g, float u, float clamp) {
+    if (clamp > 0.0f) {
+        g = fminf(fmaxf(g, -clamp), clamp);
+        u = fminf(fmaxf(u, -clamp), clamp);
+    }
+    return silu_f(g) * u;
+}
+
 // Routes of a tile rounded up to the MMA's N granularity (both CTAs hold N/2 rows of B).
 __device__ __forceinline__ int tile_n(int nvalid) { return (nvalid + 31) & ~31; }
 
@@ -305,6 +315,10 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
                 for (int c = half; c < nch; c += 2) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(taddr + c * 32, v);
+                    // apply_topk_in_fc1: lane l fetches the probability of route 32c + l
+                    float pv = 1.0f;
+                    if (p.route_probs != nullptr && c * 32 + lane < ti.z)
+                        pv = __ldg(p.route_probs + __ldg(p.perm + ti.w + c * 32 + lane));
                     tmem_ld_wait();
                     // lanes < 16 keep their gate values of routes 0..15 and receive the up values;
                     // lanes >= 16 keep their up values of routes 16..31 and receive the gate values
@@ -315,7 +329,9 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
                         const uint32_t other = __shfl_xor_sync(0xffffffffu, lo ? v[16 + j] : v[j], 16);
                         const float g = __uint_as_float(lo ? mine : other);
                         const float u = __uint_as_float(lo ? other : mine);
-                        *reinterpret_cast<__nv_bfloat16*>(row0 + j * 32) = __float2bfloat16_rn(silu_f(g) * u);
+                        float hv = swiglu_value(g, u, p.clamp);
+                        if (p.route_probs != nullptr) hv *= __shfl_sync(0xffffffffu, pv, lo ? j : 16 + j);
+                        *reinterpret_cast<__nv_bfloat16*>(row0 + j * 32) = __float2bfloat16_rn(hv);
                     }
                     __syncwarp();
 #pragma unroll

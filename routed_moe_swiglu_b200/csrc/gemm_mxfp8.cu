@@ -112,6 +112,16 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
+// silu(g) * u, the two pre-activations first clamped to [-clamp, clamp] when clamp > 0
+// (the MoeEp `gate_up_clamp` option of cudnn-frontend PR #448)
+__device__ __forceinline__ float swiglu_value(float g, float u, float clamp) {
+    if (clamp > 0.0f) {
+        g = fminf(fmaxf(g, -clamp), clamp);
+        u = fminf(fmaxf(u, -clamp), clamp);
+    }
+    return silu_f(g) * u;
+}
+
 // Routes of a tile rounded up to the MMA's N granularity.
 __device__ __forceinline__ int tile_n(int nvalid) { return (nvalid + 31) & ~31; }
 
@@ -334,6 +344,10 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                     float* st = reinterpret_cast<float*>(sEpi + (chunk_count & 1u) * kStageHBytes);
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(taddr + c * 32, v);
+                    // apply_topk_in_fc1: lane l fetches the probability of route 32c + l
+                    float pv = 1.0f;
+                    if (p.route_probs != nullptr && c * 32 + lane < ti.z)
+                        pv = __ldg(p.route_probs + __ldg(p.perm + ti.w + c * 32 + lane));
                     tmem_ld_wait();
                     // h of (route (lo ? j : 16 + j), f = fl) into st[route][64 f]; the f index of
                     // routes 16..31 is xor-ed with 16 so that the two half-warps hit different banks
@@ -344,7 +358,9 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                         const float g = __uint_as_float(lo ? mine : other);
                         const float u = __uint_as_float(lo ? other : mine);
                         const int route = lo ? j : 16 + j;
-                        st[route * 64 + (fl ^ (lo ? 0 : 16))] = silu_f(g) * u;
+                        float hv = swiglu_value(g, u, p.clamp);
+                        if (p.route_probs != nullptr) hv *= __shfl_sync(0xffffffffu, pv, route);
+                        st[route * 64 + (fl ^ (lo ? 0 : 16))] = hv;
                     }
                     named_bar_sync(kEpiBar, 128);
                     // quantise: 16 values of (route qr, block qb); the block's other half is lane ^ 1

@@ -100,6 +100,11 @@ struct GemmParams {
     // permuted order being token perm[r] / top_k
     const int* perm;
     int top_k;
+    // gate/up epilogue variants: route_probs (canonical [max_live, k], or null)
+    // scales each route's SwiGLU row by its probability; clamp > 0 clamps the
+    // gate and up pre-activations to [-clamp, clamp]
+    const float* route_probs;
+    float clamp;
 };
 
 // ---------------------------------------------------------------- launchers
@@ -122,8 +127,10 @@ cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_
                                const int* xrow, __nv_bfloat16* xp, cudaStream_t s);
 cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
                                 const int* inv, uint8_t* xq, uint8_t* xs, cudaStream_t s);
+// probs null: every route's weight is 1 (the probabilities were applied in FC1);
+// out_bf16: out is bf16 (the fp32 sum rounded to nearest even), else fp32
 cudaError_t launch_combine(const float* y, const int* inv, const float* probs, const int* live, int max_live,
-                           int H, int k, float* out, cudaStream_t s);
+                           int H, int k, void* out, bool out_bf16, cudaStream_t s);
 cudaError_t launch_gemm1_bf16_pair(const CUtensorMap& a, const CUtensorMap& x_rows, const BoxMaps8& b,
                                    const GemmParams& gp, long long max_tiles, cudaStream_t s);
 cudaError_t launch_gemm2_bf16_pair(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,

@@ -42,7 +42,7 @@ moe_status scratch_address(void** out) {
 
 extern "C" moe_status moe_forward_noalloc(const moe_plan* plan, const void* x, const float* logits, const int* ids,
                                           const float* probs, const void* kernel_buf, const int* live_count_dev,
-                                          float* out, void* stream) {
+                                          void* out, void* stream) {
     if (plan == nullptr) return MOE_ERR_INVALID_ARG;
     if (plan->ws.total > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE_TOO_SMALL;
     void* scratch = nullptr;

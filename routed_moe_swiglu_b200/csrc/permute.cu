@@ -283,11 +283,15 @@ __global__ void __launch_bounds__(kRowThreads) gather_rows_mxfp8_kernel(const ui
 // changed": the unpermute adds a token's routes as fp32 fused multiply-adds
 // of probability and row, from zero, in a fixed order; PR #8367: fp32
 // result).  The k rows' loads of a chunk are all issued before the FMA chain.
+// probs == nullptr: the probabilities were applied in the gate/up epilogue
+// and every weight is 1 (fma(1, y, acc) is the plain fp32 sum).  kBf16Out:
+// the sum is rounded to bf16, nearest even (the pages' BF16 finalize).
+template <bool kBf16Out>
 __global__ void __launch_bounds__(kRowThreads) combine_kernel(const float4* __restrict__ y,
                                                               const int* __restrict__ inv,
                                                               const float* __restrict__ probs,
                                                               const int* __restrict__ live, int max_live, int H,
-                                                              int k, float4* __restrict__ out) {
+                                                              int k, void* __restrict__ out) {
     __shared__ int s_prow[kMaxTopK];
     __shared__ float s_p[kMaxTopK];
     pdl_trigger();
@@ -298,7 +302,7 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(const float4* __re
         __syncthreads();
         if (threadIdx.x < k) {
             s_prow[threadIdx.x] = __ldg(inv + (size_t)t * k + threadIdx.x);
-            s_p[threadIdx.x] = __ldg(probs + (size_t)t * k + threadIdx.x);
+            s_p[threadIdx.x] = probs != nullptr ? __ldg(probs + (size_t)t * k + threadIdx.x) : 1.0f;
         }
         __syncthreads();
         for (int c = threadIdx.x; c < chunks; c += kRowThreads) {
@@ -322,7 +326,16 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(const float4* __re
                     }
                 }
             }
-            out[(size_t)t * chunks + c] = acc;
+            if (kBf16Out) {
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+                const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+                uint2 w;
+                w.x = *reinterpret_cast<const uint32_t*>(&lo);
+                w.y = *reinterpret_cast<const uint32_t*>(&hi);
+                reinterpret_cast<uint2*>(out)[(size_t)t * chunks + c] = w;
+            } else {
+                reinterpret_cast<float4*>(out)[(size_t)t * chunks + c] = acc;
+            }
         }
     }
 }
@@ -384,10 +397,13 @@ cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max
 }
 
 cudaError_t launch_combine(const float* y, const int* inv, const float* probs, const int* live, int max_live,
-                           int H, int k, float* out, cudaStream_t s) {
+                           int H, int k, void* out, bool out_bf16, cudaStream_t s) {
     const int grid = grid_for_warps(max_live, 1, 16);
-    return launch_dependent(combine_kernel, dim3(grid), dim3(kRowThreads), 0, s, reinterpret_cast<const float4*>(y),
-                            inv, probs, live, max_live, H, k, reinterpret_cast<float4*>(out));
+    if (out_bf16)
+        return launch_dependent(combine_kernel<true>, dim3(grid), dim3(kRowThreads), 0, s,
+                                reinterpret_cast<const float4*>(y), inv, probs, live, max_live, H, k, out);
+    return launch_dependent(combine_kernel<false>, dim3(grid), dim3(kRowThreads), 0, s,
+                            reinterpret_cast<const float4*>(y), inv, probs, live, max_live, H, k, out);
 }
 
 }  // namespace moe

@@ -37,9 +37,9 @@ def assert_close(gpu: np.ndarray, ref: np.ndarray, precision: str, what: str = "
 class GpuMoe:
     """A plan + prepared weight buffer + workspace on cuda:0."""
 
-    def __init__(self, hidden, ffn, experts, top_k, capacity, weights, precision="bf16", max_live=0):
+    def __init__(self, hidden, ffn, experts, top_k, capacity, weights, precision="bf16", max_live=0, **variant):
         self.plan = rm.moe_plan_create(hidden=hidden, ffn=ffn, num_experts=experts, top_k=top_k,
-                                       capacity=capacity, precision=precision, max_live_rows=max_live)
+                                       capacity=capacity, precision=precision, max_live_rows=max_live, **variant)
         self.H, self.F, self.E, self.k, self.cap = hidden, ffn, experts, top_k, capacity
         self.precision = precision
         self.wbuf = rm.alloc_weight_buffer(self.plan)
@@ -54,7 +54,8 @@ class GpuMoe:
 
     def forward(self, x, live, logits=None, ids=None, probs=None, out=None, sentinel=float("nan")):
         if out is None:
-            out = torch.full((self.cap, self.H), sentinel, dtype=torch.float32, device="cuda")
+            dt = torch.bfloat16 if self.plan.out_dtype == "bf16" else torch.float32
+            out = torch.full((self.cap, self.H), sentinel, dtype=dt, device="cuda")
         self.live.fill_(int(live))
         rm.moe_forward(self.plan, x, self.wbuf, self.live, out, self.ws, logits=logits, ids=ids, probs=probs)
         return out

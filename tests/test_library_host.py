@@ -120,3 +120,15 @@ def test_bounded_wait_check_rejects_bad_arguments_before_launch():
     assert lib.moe_check_bounded_wait(0, fake, None, None) == 1
     assert lib.moe_check_bounded_wait(10_000_000_001, fake, None, None) == 1
     assert lib.moe_check_bounded_wait(1000, None, None, None) == 1
+
+
+def test_plan_rejects_unknown_flags_and_bad_clamp():
+    lib = rm.load_library()
+    base = dict(hidden=256, ffn=512, num_experts=8, top_k=2, capacity=64, max_live_rows=0, precision=0)
+    for flags, clamp in ((0x4, 0.0), (0x80000000, 0.0), (0, -1.0), (0, float("nan")), (0, float("inf"))):
+        d = rm._Desc(*base.values(), flags, clamp)
+        h = ctypes.c_void_p()
+        assert lib.moe_plan_create(ctypes.byref(d), ctypes.byref(h)) == 1, (flags, clamp)
+    p = rm.moe_plan_create(hidden=256, ffn=512, num_experts=8, top_k=2, capacity=64, out_dtype="bf16",
+                           probs_in_fc1=True, gate_up_clamp=3.5)
+    assert p.out_dtype == "bf16" and p.probs_in_fc1 and p.gate_up_clamp == 3.5
