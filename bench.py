@@ -57,6 +57,10 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--probs-in-fc1", action="store_true",
+                    help="variant: router probabilities applied to the SwiGLU row (apply_topk_in_fc1)")
+    ap.add_argument("--gate-up-clamp", type=float, default=None, help="variant: clamp of the gate/up pre-activations")
+    ap.add_argument("--out-bf16", action="store_true", help="variant: bf16 finalize output")
     ap.add_argument("--capacity", type=int, default=None,
                     help="override the buffer rows (profiling captures only; not a benchmark configuration)")
     a = ap.parse_args()
@@ -241,12 +245,24 @@ def run_ours(a, dist: Dist):
     wg, wu, wd = workloads.make_weights(w)
     dev = torch.device("cuda", torch.cuda.current_device())
     plan = rm.moe_plan_create(hidden=w.hidden, ffn=w.ffn, num_experts=w.num_experts, top_k=w.top_k,
-                              capacity=w.capacity, precision=w.precision)
+                              capacity=w.capacity, precision=w.precision, probs_in_fc1=a.probs_in_fc1,
+                              gate_up_clamp=a.gate_up_clamp, out_dtype="bf16" if a.out_bf16 else "fp32")
     wbuf = rm.alloc_weight_buffer(plan, dev)
-    rm.moe_prepare_weights(plan, wg.to(dev), wu.to(dev), wd.to(dev), wbuf)
+    wgd, wud, wdd = wg.to(dev), wu.to(dev), wd.to(dev)
+    rm.moe_prepare_weights(plan, wgd, wud, wdd, wbuf)
+    # the kernel-layout rebuild a refit runs (moe_prepare_weights), timed warm
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record()
+    for _ in range(3):
+        rm.moe_prepare_weights(plan, wgd, wud, wdd, wbuf)
+    p1.record()
+    torch.cuda.synchronize()
+    prepare_ms = p0.elapsed_time(p1) / 3
+    del wgd, wud, wdd
     ws = rm.alloc_workspace(plan, dev)
     xd, ld = x.to(dev), logits.to(dev)
-    out = torch.zeros((w.capacity, w.hidden), dtype=torch.float32, device=dev)
+    out_dt = torch.bfloat16 if a.out_bf16 else torch.float32
+    out = torch.zeros((w.capacity, w.hidden), dtype=out_dt, device=dev)
     live_d = torch.tensor([live], dtype=torch.int32, device=dev)
     torch.cuda.synchronize()
 
@@ -324,6 +340,7 @@ def run_ours(a, dist: Dist):
         "ms_per_step": ms_step,
         "value": dist.world * live / (ms_step / 1e3),
         "stage_ms": stage_avg,
+        "prepare_ms": prepare_ms,
         "ms_per_step_with_stage_events": ms_step_events,
         "clocks": clocks.summary(),
         "timed_s": ms_total / 1e3,
@@ -361,7 +378,7 @@ def run_ours(a, dist: Dist):
         x_pin = x[:live].contiguous().pin_memory()
         l_pin = logits[:live].contiguous().pin_memory()
         n_pin = torch.tensor([live], dtype=torch.int32).pin_memory()
-        o_pin = torch.empty((live, w.hidden), dtype=torch.float32).pin_memory()
+        o_pin = torch.empty((live, w.hidden), dtype=out_dt).pin_memory()
 
         def e2e_step():
             xd[:live].copy_(x_pin, non_blocking=True)
@@ -388,7 +405,7 @@ def run_ours(a, dist: Dist):
         e_ms = dist.max(e0.elapsed_time(e1)) / K
         res["e2e"] = {"value": dist.world * live / (e_ms / 1e3), "unit": "tokens/s",
                       "h2d_bytes_per_step": x_pin.numel() * 2 + l_pin.numel() * 4 + 4,
-                      "d2h_bytes_per_step": o_pin.numel() * 4, "ms_per_step": e_ms}
+                      "d2h_bytes_per_step": o_pin.numel() * o_pin.element_size(), "ms_per_step": e_ms}
     del gk, ge, g1
     return w, live, res
 
@@ -447,7 +464,13 @@ def roofline(w, res, peaks):
 # ---------------------------------------------------------------- the oracle (CPU) arm
 
 
-def oracle_tokens_per_s(w, x, logits, weights, live, budget_s, min_tokens=8):
+def oracle_variant(a):
+    """The oracle's options for the variant the CUDA arm runs (the bf16
+    output rounding costs nothing next to the expert forward)."""
+    return {"probs_in_fc1": bool(a.probs_in_fc1), "gate_up_clamp": a.gate_up_clamp}
+
+
+def oracle_tokens_per_s(w, x, logits, weights, live, budget_s, min_tokens=8, variant=None):
     """Time the oracle (as it stands) on the host cores over a bounded sample
     of the live tokens: route all live rows, then the expert forward of a
     growing prefix of a seeded token sample until ~budget_s of work."""
@@ -465,9 +488,9 @@ def oracle_tokens_per_s(w, x, logits, weights, live, budget_s, min_tokens=8):
         sel = toks[(done + np.arange(n)) % live]
         t0 = time.perf_counter()
         if w.precision == "mxfp8":
-            oracle.forward_mxfp8(x[:live], ids, probs, wq, tokens=sel)
+            oracle.forward_mxfp8(x[:live], ids, probs, wq, tokens=sel, **(variant or {}))
         else:
-            oracle.forward_bf16(x[:live], ids, probs, *weights, tokens=sel)
+            oracle.forward_bf16(x[:live], ids, probs, *weights, tokens=sel, **(variant or {}))
         dt = time.perf_counter() - t0
         spent += dt
         done += n
@@ -493,13 +516,14 @@ def run_reference(a, dist: Dist):
     wq = oracle.quantize_weights_mxfp8(*weights) if w.precision == "mxfp8" else None
     ids, probs = oracle.route(logits[:live].numpy(), w.top_k)
     toks = workloads.sample_tokens(live, live, w.seed).numpy()
+    variant = oracle_variant(a)
 
     def step(n, start):
         sel = toks[(start + np.arange(n)) % live]
         if wq is not None:
-            oracle.forward_mxfp8(x[:live], ids, probs, wq, tokens=sel)
+            oracle.forward_mxfp8(x[:live], ids, probs, wq, tokens=sel, **(variant or {}))
         else:
-            oracle.forward_bf16(x[:live], ids, probs, *weights, tokens=sel)
+            oracle.forward_bf16(x[:live], ids, probs, *weights, tokens=sel, **(variant or {}))
 
     t0 = time.perf_counter()
     step(4, 0)
@@ -520,8 +544,16 @@ def run_reference(a, dist: Dist):
 # ---------------------------------------------------------------- main
 
 
-def workload_config(w, live):
+def workload_config(w, live, a=None):
+    variant = []
+    if a is not None and a.probs_in_fc1:
+        variant.append("probs applied in FC1")
+    if a is not None and a.gate_up_clamp:
+        variant.append(f"gate/up clamp {a.gate_up_clamp:g}")
+    if a is not None and a.out_bf16:
+        variant.append("bf16 output")
     return {
+        "variant": ", ".join(variant) if variant else "plain (fp32 output, probabilities in the combine)",
         "workload": f"{w.name}: {w.precision} H={w.hidden} F={w.ffn} E={w.num_experts} top-{w.top_k}, "
                     f"{live} live rows of a {w.capacity}-row buffer",
         "hidden": w.hidden, "ffn": w.ffn, "experts": w.num_experts, "top_k": w.top_k,
@@ -545,7 +577,7 @@ def main():
                 "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup, "ms_per_step": res["ms_per_step"],
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": w.precision if w.precision != "mxfp8" else "mxfp8", "data": "synthetic",
-                "config": workload_config(w, live),
+                "config": workload_config(w, live, a),
                 "cpu_baseline": {"value": res["value"], "unit": "tokens/s", "cores": oracle.threads(),
                                  "kind": "oracle",
                                  "sample": f"{res['sample']} tokens per step of the {w.name} workload"},
@@ -563,10 +595,11 @@ def main():
         "metric": "routed tokens/s", "value": res["value"], "unit": "tokens/s", "n_gpus": dist.world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.precision, "data": "synthetic",
-        "config": workload_config(w, live),
+        "config": workload_config(w, live, a),
         "roofline": roofline(w, res, peaks),
         "stage_ms": {k: round(v, 5) for k, v in res["stage_ms"].items()},
         "ms_per_step_with_stage_events": round(res["ms_per_step_with_stage_events"], 5),
+        "prepare_weights_ms": round(res["prepare_ms"], 4),
         "clocks": res["clocks"],
         "gpu_launches": KERNELS_PER_FORWARD * a.steps,
         "device_status": res["status"],
@@ -580,7 +613,7 @@ def main():
     if dist.rank == 0 and dist.world == 1 and not a.no_cpu_baseline:
         x, logits = workloads.make_activations(w)
         weights = workloads.make_weights(w)
-        v, n, cores = oracle_tokens_per_s(w, x, logits, weights, live, a.cpu_seconds)
+        v, n, cores = oracle_tokens_per_s(w, x, logits, weights, live, a.cpu_seconds, variant=oracle_variant(a))
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                 "sample": f"{n} tokens of the {w.name} workload (route of all {live} live rows "
                                           f"+ expert forward of the sample), ~{a.cpu_seconds:.0f} s"}
