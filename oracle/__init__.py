@@ -150,10 +150,11 @@ def mxfp8_dequantize(q: np.ndarray, s: np.ndarray) -> np.ndarray:
 
 
 PROBS_IN_FC1 = 1
+SQUARED_RELU = 2
 
 
-def _variant(probs_in_fc1, gate_up_clamp):
-    flags = PROBS_IN_FC1 if probs_in_fc1 else 0
+def _variant(probs_in_fc1, gate_up_clamp, squared_relu=False):
+    flags = (PROBS_IN_FC1 if probs_in_fc1 else 0) | (SQUARED_RELU if squared_relu else 0)
     clamp = float(gate_up_clamp) if gate_up_clamp else 0.0
     return flags, clamp
 
@@ -168,17 +169,19 @@ def round_bf16(out):
 
 
 def forward_bf16(x, ids, probs, w_gate, w_up, w_down, tokens=None, want_h=False, probs_in_fc1=False,
-                 gate_up_clamp=None):
+                 gate_up_clamp=None, squared_relu=False):
     """bf16 routed SwiGLU forward for `tokens` (default: all rows of ids).
 
     x [T,H] bf16, ids/probs [T,k], w_gate/w_up [E,F,H] bf16, w_down [E,H,F] bf16.
     Returns out fp32 [ntok, H] (and h fp32 [ntok, k, F] when want_h).
     probs_in_fc1 / gate_up_clamp select the variants described in
     moe_oracle.c (probability applied to the SwiGLU row; clamp of the gate
-    and up pre-activations)."""
-    flags, clamp = _variant(probs_in_fc1, gate_up_clamp)
+    and up pre-activations); squared_relu: experts h = relu(w_gate . x)^2,
+    w_up unused (None)."""
+    flags, clamp = _variant(probs_in_fc1, gate_up_clamp, squared_relu)
     xb = _bf16_bits(x)
-    gb, ub, db = _bf16_bits(w_gate), _bf16_bits(w_up), _bf16_bits(w_down)
+    gb, db = _bf16_bits(w_gate), _bf16_bits(w_down)
+    ub = None if squared_relu else _bf16_bits(w_up)
     ids = np.ascontiguousarray(ids, dtype=np.int32)
     probs = np.ascontiguousarray(probs, dtype=np.float32)
     T, k = ids.shape

@@ -55,6 +55,11 @@
  *       (the FC1 accumulator) are clamped to [-clamp, clamp] before SwiGLU.
  *   oracle_round_bf16  -- a bf16 finalize output: the fp32 sum rounded to
  *       bf16 (round-to-nearest-even), as the pages' BF16 finalize does.
+ *   ORACLE_SQUARED_RELU -- squared-ReLU experts (the Nano-v3 shapes of
+ *       Megatron-LM PR #8367's measurements and the nvfp4-squared_relu
+ *       recipe of its tests): one FC1 projection W1 = w_gate [E, F, H], no
+ *       up projection, h_f = round(fp32(relu(g_f)^2)); the clamp and the
+ *       probability in FC1 act on g_f and on the row as above.
  *   The pages name these options but give no formula; the readings above
  *   are the plainest ones and are listed in the design notes.
  *
@@ -331,16 +336,24 @@ int oracle_permute(const int32_t* ids, int64_t T, int E, int k,
 static double silu_d(double z) { return z / (1.0 + exp(-z)); }
 
 #define ORACLE_PROBS_IN_FC1 1
+#define ORACLE_SQUARED_RELU 2
 
-/* The fp32 SwiGLU value of one (route, f) from its double pre-activations:
- * clamped when clamp > 0, scaled by the route's probability when the
- * probabilities are applied in FC1. */
+/* The fp32 activation value of one (route, f) from its double
+ * pre-activations: clamped when clamp > 0, silu(g) * u (or relu(g)^2 for
+ * squared-ReLU experts, u unused), scaled by the route's probability when
+ * the probabilities are applied in FC1. */
 static float swiglu_value(double g, double u, double clamp, int flags, float p) {
     if (clamp > 0.0) {
         g = g < -clamp ? -clamp : (g > clamp ? clamp : g);
         u = u < -clamp ? -clamp : (u > clamp ? clamp : u);
     }
-    double h = silu_d(g) * u;
+    double h;
+    if (flags & ORACLE_SQUARED_RELU) {
+        const double r = g > 0.0 ? g : 0.0;
+        h = r * r;
+    } else {
+        h = silu_d(g) * u;
+    }
     if (flags & ORACLE_PROBS_IN_FC1) h *= (double)p;
     return (float)h;
 }
@@ -383,7 +396,8 @@ int oracle_forward_bf16(const uint16_t* x, const int32_t* ids, const float* prob
                         int64_t T, int H, int F, int E, int k,
                         const int64_t* toks, int64_t ntok, float* out, float* h_out,
                         int flags, double clamp) {
-    if (!x || !ids || !probs || !w_gate || !w_up || !w_down || !toks || !out) return ORACLE_EINVAL;
+    const int relu2 = (flags & ORACLE_SQUARED_RELU) != 0;
+    if (!x || !ids || !probs || !w_gate || (!w_up && !relu2) || !w_down || !toks || !out) return ORACLE_EINVAL;
     if (H <= 0 || F <= 0 || E <= 0 || k <= 0 || k > 64 || ntok < 0) return ORACLE_EINVAL;
     int bad = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
@@ -403,13 +417,13 @@ int oracle_forward_bf16(const uint16_t* x, const int32_t* ids, const float* prob
             int e = sid[j];
             if (e < 0 || e >= E) { bad = 1; break; }
             const uint16_t* wg = w_gate + (int64_t)e * F * H;
-            const uint16_t* wu = w_up + (int64_t)e * F * H;
+            const uint16_t* wu = relu2 ? NULL : w_up + (int64_t)e * F * H;
             const uint16_t* wd = w_down + (int64_t)e * H * F;
             for (int f = 0; f < F; ++f) {
                 double g = 0.0, u = 0.0;
                 for (int c = 0; c < H; ++c) {
                     g += (double)bf16_bits_to_float(wg[(int64_t)f * H + c]) * xd[c];
-                    u += (double)bf16_bits_to_float(wu[(int64_t)f * H + c]) * xd[c];
+                    if (!relu2) u += (double)bf16_bits_to_float(wu[(int64_t)f * H + c]) * xd[c];
                 }
                 float hf = swiglu_value(g, u, clamp, flags, sp[j]);
                 float hb = bf16_bits_to_float(float_to_bf16_bits_rne(hf));

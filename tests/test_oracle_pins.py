@@ -498,3 +498,54 @@ def test_round_bf16_matches_torch_cast_including_ties():
     t = ties.view(np.float32)
     kept = oracle.round_bf16(t)
     assert np.all(kept & 1 == 0)
+
+
+# ---------------------------------------------------------------- squared-ReLU experts
+
+
+def _dense_relu2_ref(x, w1, wd, p=None, clamp=None):
+    """torch float64 dense squared-ReLU MLP: relu(W1 x)^2 (pre-activation clamped,
+    row scaled by p), rounded to fp32 then bf16; y in fp32."""
+    g = x.to(torch.float64) @ w1.to(torch.float64).T
+    if clamp is not None:
+        g = g.clamp(-clamp, clamp)
+    h = torch.relu(g) ** 2
+    if p is not None:
+        h = h * p
+    h = h.to(torch.float32).to(torch.bfloat16).to(torch.float64)
+    return (h @ wd.to(torch.float64).T).to(torch.float32)
+
+
+def test_squared_relu_single_expert_is_dense_relu2_mlp():
+    x, wg, _, wd, ids = _single_expert(41)
+    one = np.ones(ids.shape, np.float32)
+    out = oracle.forward_bf16(x, ids, one, wg, None, wd, squared_relu=True)
+    _close_to_dense(out, _dense_relu2_ref(x, wg[0], wd[0]))
+    # with the variants: probability in FC1 and a clamp on the one pre-activation
+    p = np.full(ids.shape, 0.3, np.float32)
+    out = oracle.forward_bf16(x, ids, p, wg, None, wd, squared_relu=True, probs_in_fc1=True, gate_up_clamp=0.5)
+    _close_to_dense(out, _dense_relu2_ref(x, wg[0], wd[0], p=float(np.float32(0.3)), clamp=0.5))
+
+
+def test_squared_relu_negative_preactivations_give_zero():
+    gen = torch.Generator().manual_seed(42)
+    T, H, F, E, k = 8, 64, 96, 4, 2
+    x = rand_bf16(gen, (T, H)).abs()
+    w1 = -rand_bf16(gen, (E, F, H), 0.1).abs()  # x >= 0, W1 <= 0: every pre-activation <= 0
+    wd = rand_bf16(gen, (E, H, F), 0.1)
+    ids, probs = oracle.route(np.random.default_rng(42).standard_normal((T, E)).astype(np.float32), k)
+    out = oracle.forward_bf16(x, ids, probs, w1, None, wd, squared_relu=True)
+    assert np.all(out == 0.0)
+    # the same weights as SwiGLU gate and up give a nonzero output: the flag selects the activation
+    out_swiglu = oracle.forward_bf16(x, ids, probs, w1, w1, wd)
+    assert np.any(out_swiglu != 0.0)
+
+
+def test_squared_relu_ignores_probs_scaling_by_pow2_like_plain():
+    # the combine rules do not depend on the activation: power-of-two probabilities give the
+    # same bits with the probability applied in FC1 or in the combine
+    x, wg, _, wd, ids, _ = _small_problem(43, T=10, k=3)
+    probs = _pow2_probs(ids, 43)
+    a = oracle.forward_bf16(x, ids, probs, wg, None, wd, squared_relu=True)
+    b = oracle.forward_bf16(x, ids, probs, wg, None, wd, squared_relu=True, probs_in_fc1=True)
+    assert np.array_equal(a, b)
