@@ -61,6 +61,7 @@ def parse_args():
                     help="variant: router probabilities applied to the SwiGLU row (apply_topk_in_fc1)")
     ap.add_argument("--gate-up-clamp", type=float, default=None, help="variant: clamp of the gate/up pre-activations")
     ap.add_argument("--out-bf16", action="store_true", help="variant: bf16 finalize output")
+    ap.add_argument("--squared-relu", action="store_true", help="variant: squared-ReLU experts (bf16 only)")
     ap.add_argument("--capacity", type=int, default=None,
                     help="override the buffer rows (profiling captures only; not a benchmark configuration)")
     a = ap.parse_args()
@@ -246,7 +247,8 @@ def run_ours(a, dist: Dist):
     dev = torch.device("cuda", torch.cuda.current_device())
     plan = rm.moe_plan_create(hidden=w.hidden, ffn=w.ffn, num_experts=w.num_experts, top_k=w.top_k,
                               capacity=w.capacity, precision=w.precision, probs_in_fc1=a.probs_in_fc1,
-                              gate_up_clamp=a.gate_up_clamp, out_dtype="bf16" if a.out_bf16 else "fp32")
+                              gate_up_clamp=a.gate_up_clamp, out_dtype="bf16" if a.out_bf16 else "fp32",
+                              squared_relu=a.squared_relu)
     wbuf = rm.alloc_weight_buffer(plan, dev)
     wgd, wud, wdd = wg.to(dev), wu.to(dev), wd.to(dev)
     rm.moe_prepare_weights(plan, wgd, wud, wdd, wbuf)
@@ -341,6 +343,7 @@ def run_ours(a, dist: Dist):
         "value": dist.world * live / (ms_step / 1e3),
         "stage_ms": stage_avg,
         "prepare_ms": prepare_ms,
+        "fc1_projections": 1 if a.squared_relu else 2,
         "ms_per_step_with_stage_events": ms_step_events,
         "clocks": clocks.summary(),
         "timed_s": ms_total / 1e3,
@@ -423,8 +426,9 @@ def roofline(w, res, peaks):
     out = {"kernel": dom}
     if dom in ("gemm_gate_up", "gemm_down"):
         if dom == "gemm_gate_up":
-            flops = 4.0 * R * H * F
-            wbytes = res["touched"] * 2 * F * H * bpe
+            nproj = res.get("fc1_projections", 2)  # gate and up, or the one squared-ReLU projection
+            flops = 2.0 * nproj * R * H * F
+            wbytes = res["touched"] * nproj * F * H * bpe
             abytes = R * H * bpe + R * F * bpe
         else:
             flops = 2.0 * R * H * F
@@ -467,7 +471,10 @@ def roofline(w, res, peaks):
 def oracle_variant(a):
     """The oracle's options for the variant the CUDA arm runs (the bf16
     output rounding costs nothing next to the expert forward)."""
-    return {"probs_in_fc1": bool(a.probs_in_fc1), "gate_up_clamp": a.gate_up_clamp}
+    v = {"probs_in_fc1": bool(a.probs_in_fc1), "gate_up_clamp": a.gate_up_clamp}
+    if a.squared_relu:
+        v["squared_relu"] = True
+    return v
 
 
 def oracle_tokens_per_s(w, x, logits, weights, live, budget_s, min_tokens=8, variant=None):
@@ -552,6 +559,8 @@ def workload_config(w, live, a=None):
         variant.append(f"gate/up clamp {a.gate_up_clamp:g}")
     if a is not None and a.out_bf16:
         variant.append("bf16 output")
+    if a is not None and a.squared_relu:
+        variant.append("squared-ReLU experts")
     return {
         "variant": ", ".join(variant) if variant else "plain (fp32 output, probabilities in the combine)",
         "workload": f"{w.name}: {w.precision} H={w.hidden} F={w.ffn} E={w.num_experts} top-{w.top_k}, "

@@ -100,6 +100,12 @@ typedef struct {
  *       fp32 sum rounded to nearest even (the plain output is fp32). */
 #define MOE_FLAG_PROBS_IN_FC1 0x1u
 #define MOE_FLAG_OUT_BF16 0x2u
+/*   MOE_FLAG_SQUARED_RELU  squared-ReLU experts (the Nano-v3 shapes of
+ *       Megatron-LM PR #8367's measurements): one FC1 projection,
+ *       h = relu(W_gate[e] . x)^2; W_up is not used.  bf16 plans only
+ *       (MXFP8 plans with it are MOE_ERR_UNSUPPORTED).  The clamp and the
+ *       probability in FC1 act on the one pre-activation and on the row. */
+#define MOE_FLAG_SQUARED_RELU 0x4u
 
 typedef struct moe_plan moe_plan; /* opaque, host memory only */
 
@@ -107,7 +113,7 @@ typedef struct moe_plan moe_plan; /* opaque, host memory only */
  * allocation).  Rejected (MOE_ERR_UNSUPPORTED): H or F not a multiple of 8
  * (bf16) or of 32 (MXFP8); k < 1, k > 16 or k > E; E < 1 or E > 1024;
  * capacity < 1 or > 2^24 rows; max_live_rows < 0 or > capacity;
- * H > 16384 or F > 16384.  Rejected (MOE_ERR_INVALID_ARG): unknown flag
+ * H > 16384 or F > 16384; MOE_FLAG_SQUARED_RELU with MOE_MXFP8.  Rejected (MOE_ERR_INVALID_ARG): unknown flag
  * bits, a negative or non-finite gate_up_clamp. */
 moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out);
 void moe_plan_destroy(moe_plan* plan);
@@ -123,7 +129,10 @@ size_t moe_workspace_bytes(const moe_plan* plan);
 /* Rebuild the kernel-layout weight buffer in place from the experts' bf16
  * weights ([P1] "refresh_mega_weights": a refit rewrites the same buffer; no
  * allocation, no teardown).  Inputs (device, bf16, row-major):
- *   w_gate [E, F, H], w_up [E, F, H]  (gate and up projections)
+ *   w_gate [E, F, H], w_up [E, F, H]  (gate and up projections; for
+ *                                      MOE_FLAG_SQUARED_RELU plans w_gate is
+ *                                      the one FC1 projection and w_up is not
+ *                                      read and may be NULL)
  *   w_down [E, H, F]                  (down projection)
  * In MXFP8 the weights are quantised here (blocks of 32 along each GEMM's K:
  * H for gate/up, F for down).  Enqueued on `stream`; forwards enqueued later

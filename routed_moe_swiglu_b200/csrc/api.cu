@@ -110,7 +110,7 @@ static void compute_layouts(moe_plan* p) {
         b.w2 = take(E * H * (size_t)p->fp);
         b.w2s = take(E * p->nt2 * p->ks2 * kSfBlock);
     } else {
-        b.w1 = take(E * 2 * (size_t)p->fp * (size_t)p->hp * 2);
+        b.w1 = take(E * (size_t)p->w1r * (size_t)p->hp * 2);
         b.w1s = 0;
         b.w2 = take(E * (size_t)p->hr * (size_t)p->fp * 2);
         b.w2s = 0;
@@ -154,7 +154,9 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     if (d.num_experts > kMaxExperts || d.top_k > kMaxTopK || d.top_k > d.num_experts) return MOE_ERR_UNSUPPORTED;
     if (d.capacity > (1ll << 24)) return MOE_ERR_UNSUPPORTED;
     if (d.max_live_rows < 0 || d.max_live_rows > d.capacity) return MOE_ERR_UNSUPPORTED;
-    if ((d.flags & ~(MOE_FLAG_PROBS_IN_FC1 | MOE_FLAG_OUT_BF16)) != 0) return MOE_ERR_INVALID_ARG;
+    if ((d.flags & ~(MOE_FLAG_PROBS_IN_FC1 | MOE_FLAG_OUT_BF16 | MOE_FLAG_SQUARED_RELU)) != 0)
+        return MOE_ERR_INVALID_ARG;
+    if ((d.flags & MOE_FLAG_SQUARED_RELU) && d.precision == MOE_MXFP8) return MOE_ERR_UNSUPPORTED;
     if (!(d.gate_up_clamp >= 0.0f) || d.gate_up_clamp > 3.0e38f) return MOE_ERR_INVALID_ARG;
     moe_plan* p = new (std::nothrow) moe_plan();
     if (p == nullptr) return MOE_ERR_INVALID_ARG;
@@ -176,11 +178,14 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     p->hp = (long long)p->ks1 * 128;
     p->fp = (long long)p->ks2 * 128;
     p->hr = p->hp;
+    // bf16 FC1 rows per expert: gate and up interleaved (2 fp), or one projection padded to
+    // whole pair tiles of 256 rows (squared-ReLU experts)
+    p->w1r = (d.flags & MOE_FLAG_SQUARED_RELU) ? (p->fp + 255) / 256 * 256 : 2 * p->fp;
     if (d.precision == MOE_MXFP8) {
         p->nt1 = (int)(p->fp / kG1BN8);  // f tiles of 64 cover fp; h's padding columns come out zero
         p->nt2 = (d.hidden + kG2BN8 - 1) / kG2BN8;
     } else {
-        p->nt1 = (int)(p->fp / kG1BN);  // f tiles of 128 cover fp
+        p->nt1 = (int)(p->w1r / 256);  // pair tiles of 256 FC1 rows (SwiGLU: 128 f of gate and up)
         p->nt2 = (d.hidden + kG2BN - 1) / kG2BN;
     }
     compute_layouts(p);
@@ -201,10 +206,13 @@ size_t moe_workspace_bytes(const moe_plan* plan) { return plan ? plan->ws.total 
 
 moe_status moe_prepare_weights(const moe_plan* plan, const void* w_gate, const void* w_up, const void* w_down,
                                void* kernel_buf, size_t buf_bytes, void* stream) {
-    if (plan == nullptr || w_gate == nullptr || w_up == nullptr || w_down == nullptr || kernel_buf == nullptr)
+    const bool relu2 = plan != nullptr && (plan->d.flags & MOE_FLAG_SQUARED_RELU) != 0;
+    if (plan == nullptr || w_gate == nullptr || (w_up == nullptr && !relu2) || w_down == nullptr ||
+        kernel_buf == nullptr)
         return MOE_ERR_INVALID_ARG;
     if (buf_bytes < plan->wb.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
-    if (!aligned(w_gate, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) || !aligned(kernel_buf, 256))
+    if (!aligned(w_gate, 16) || !aligned(relu2 ? w_gate : w_up, 16) || !aligned(w_down, 16) ||
+        !aligned(kernel_buf, 256))
         return MOE_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const auto* g = static_cast<const __nv_bfloat16*>(w_gate);
@@ -318,7 +326,8 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
         // (expert, 128-row block, K stage); atom a of block b is index 2b + a of the map's
         // third dimension
         const unsigned box128[3] = {64, 128, 2};
-        const unsigned long long dW1[3] = {64ull, 128ull, 2ull * (uE * 2ull * fpp / 128) * (hp / 128)};
+        const unsigned long long dW1[3] = {64ull, 128ull,
+                                           2ull * (uE * (unsigned long long)plan->w1r / 128) * (hp / 128)};
         const unsigned long long dW2[3] = {64ull, 128ull, 2ull * (uE * (unsigned long long)plan->hr / 128) * (fpp / 128)};
         const unsigned long long sWb[2] = {128ull, 128ull * 128ull};
         const unsigned long long sW1[2] = {hp * 2, 128ull};
@@ -376,7 +385,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g1.out_scales = nullptr;
     g1.out_ld = plan->fp;  // h rows: F values + zero padding to the down GEMM's K pitch
     g1.out_cols = (int)plan->fp;  // every padded column: f >= F are zero-weight rows, h = 0
-    g1.a_rows = 2 * plan->fp;     // W1 rows of an expert (padded F)
+    g1.a_rows = fp8 ? 2 * plan->fp : plan->w1r;  // FC1 weight rows of an expert
     g1.n_tiles = plan->nt1;
     g1.k_blocks = plan->ks1;
     g1.wait_limit_ns = kWaitLimitNs;
@@ -389,6 +398,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     const bool probs_in_fc1 = (plan->d.flags & MOE_FLAG_PROBS_IN_FC1) != 0;
     g1.route_probs = probs_in_fc1 ? r_probs : nullptr;
     g1.clamp = plan->d.gate_up_clamp;
+    g1.relu2 = (plan->d.flags & MOE_FLAG_SQUARED_RELU) != 0;
     if (!mark(3)) return MOE_ERR_CUDA;
     e = fp8 ? launch_gemm1_mxfp8(tA1, rB1, g1, m_tiles * g1.n_tiles, s)
             : launch_gemm1_bf16_pair(tA1, tX, rB1, g1, m_tiles * g1.n_tiles, s);

@@ -61,12 +61,14 @@ constexpr uint32_t kBBytes = kAtoms * kAtomBytes;       // up to 32 KB: this CTA
 constexpr uint32_t kAccCols = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kHTBytes = 32 * 16 * 2 + 64;         // gate/up: h of 32 routes x 16 f, bf16 (+ bank offset)
+constexpr uint32_t kRTBytes = 32 * 32 * 2;              // squared ReLU: h of 32 routes x 32 f, bf16
+constexpr uint32_t kH0Bytes = kHTBytes > kRTBytes ? kHTBytes : kRTBytes;  // gate/up epilogue box per warp
 constexpr uint32_t kYTBytes = 32 * 32 * 4;              // down: y of 32 routes x 32 c, fp32
 
 template <int kMode>
 struct PairCfg {
     // one transpose box per epilogue warp
-    static constexpr uint32_t kEpiBytes = kEpiWarps * (kMode == 0 ? kHTBytes : kYTBytes);
+    static constexpr uint32_t kEpiBytes = kEpiWarps * (kMode == 0 ? kH0Bytes : kYTBytes);
     static constexpr size_t kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kEpiBytes + 256;
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -285,7 +287,7 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
         const int half = ew >> 2;    // this warp takes the 32-route chunks c with c % 2 == half
         const uint32_t acc_empty0[2] = {map_to_cta(smem_u32(&bars->acc_empty[0]), 0),
                                         map_to_cta(smem_u32(&bars->acc_empty[1]), 0)};
-        uint8_t* tbuf = sEpi + (size_t)ew * (kMode == 0 ? kHTBytes : kYTBytes);
+        uint8_t* tbuf = sEpi + (size_t)ew * (kMode == 0 ? kH0Bytes : kYTBytes);
         int it = 0;
         for (int t = pair; t < total_tiles; t += npairs, ++it) {
             const int buf = it & 1;
@@ -304,7 +306,43 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
             }
             tc_fence_after_sync();
             const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)buf * kAccCols;
-            if (kMode == 0) {
+            if (kMode == 0 && p.relu2) {
+                // squared-ReLU experts: lane = f (this warp's 32 f from f0), register j = route
+                // 32c + j; h = relu(g)^2 goes through a [route][32 f] bf16 box to 64-byte rows
+                const int f0 = nt * kPairM + 128 * (int)rank + 32 * quad;
+                __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
+                if (f0 < p.out_cols) {
+#pragma unroll 1
+                    for (int c = half; c < nch; c += 2) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(taddr + c * 32, v);
+                        float pv = 1.0f;
+                        if (p.route_probs != nullptr && c * 32 + lane < ti.z)
+                            pv = __ldg(p.route_probs + __ldg(p.perm + ti.w + c * 32 + lane));
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            float g = __uint_as_float(v[j]);
+                            if (p.clamp > 0.0f) g = fminf(fmaxf(g, -p.clamp), p.clamp);
+                            const float r = fmaxf(g, 0.0f);
+                            float hv = r * r;
+                            if (p.route_probs != nullptr) hv *= __shfl_sync(0xffffffffu, pv, j);
+                            *reinterpret_cast<__nv_bfloat16*>(tbuf + j * 64 + lane * 2) = __float2bfloat16_rn(hv);
+                        }
+                        __syncwarp();
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int r = i * 8 + (lane >> 2);
+                            const int route = c * 32 + r;
+                            const uint4 w = *reinterpret_cast<const uint4*>(tbuf + r * 64 + (lane & 3) * 16);
+                            if (route < ti.z)
+                                *reinterpret_cast<uint4*>(h + (size_t)(ti.y + route) * (size_t)p.out_ld + f0 +
+                                                          (lane & 3) * 8) = w;
+                        }
+                        __syncwarp();
+                    }
+                }
+            } else if (kMode == 0) {
                 // f of this lane: f_base + (lane & 15); lanes < 16 hold gate, the others up
                 const int f_base = nt * 128 + 64 * (int)rank + 16 * quad;
                 const bool lo = lane < 16;

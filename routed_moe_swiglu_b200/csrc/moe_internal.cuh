@@ -62,6 +62,8 @@ struct moe_plan {
     long long hp, fp;       // K row pitch (elements) of x / gate-up rows and of h / down rows:
                             // H and F padded to multiples of 128 with zeros
     long long hr;           // bf16: rows of an expert's down weights, H padded to 128 with zero rows
+    long long w1r;          // bf16: rows of an expert's FC1 weights: 2 * fp (gate and up interleaved),
+                            // or fp rounded up to 256 (squared-ReLU experts), zero rows past F
     int ks1, ks2;           // K blocks of 128 elements of the gate/up and down GEMMs
     int nt1, nt2;           // weight (bf16) / N (MXFP8) tiles of the gate/up and down GEMMs
     moe::WsLayout ws;
@@ -105,6 +107,7 @@ struct GemmParams {
     // gate and up pre-activations to [-clamp, clamp]
     const float* route_probs;
     float clamp;
+    int relu2;                      // bf16 gate/up GEMM: squared-ReLU experts (A = one FC1 projection)
 };
 
 // ---------------------------------------------------------------- launchers

@@ -10,6 +10,8 @@
 // contiguous memory:
 //   W1  rows of an expert: 2fp, in the order (per block of 64 f, per group
 //       of 16 f) the 16 gate rows, then the 16 up rows of the same f; K = hp
+//       (squared-ReLU experts: the one projection's rows in f order, padded
+//       to a multiple of 256)
 //   W2  rows of an expert: hr (H padded to 128); K = fp
 // with hp, fp = H, F rounded up to 128.  Padding (K past H or F, rows of
 // f >= F, rows c >= H) is zero.  A gate/up weight tile is two consecutive
@@ -24,11 +26,11 @@ namespace {
 __global__ void __launch_bounds__(256) prepare_bf16_kernel(const uint4* __restrict__ wg, const uint4* __restrict__ wu,
                                                            const uint4* __restrict__ wd, uint4* __restrict__ w1,
                                                            uint4* __restrict__ w2, int E, int F, int H, int hp, int fp,
-                                                           int hr) {
+                                                           int hr, int w1r, int relu2) {
     // one thread per 16-byte chunk of the destination: block, atom, row, 8-element chunk
     constexpr long long kBlockChunks = 2 * 128 * 8;  // 32 KB
     const int kb1 = hp / 128, kb2 = fp / 128;
-    const int rb1 = 2 * fp / 128, rb2 = hr / 128;  // row blocks per expert
+    const int rb1 = w1r / 128, rb2 = hr / 128;  // row blocks per expert
     const long long n1 = (long long)E * rb1 * kb1 * kBlockChunks;
     const long long n2 = (long long)E * rb2 * kb2 * kBlockChunks;
     const long long stride = (long long)gridDim.x * blockDim.x;
@@ -47,8 +49,9 @@ __global__ void __launch_bounds__(256) prepare_bf16_kernel(const uint4* __restri
         const int rem = rb * 128 + r;                 // weight row within the expert
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (first) {
-            const int g = (rem >> 4) & 1;
-            const int f = (rem >> 7) * 64 + ((rem >> 5) & 3) * 16 + (rem & 15);
+            // squared-ReLU experts: row = f; SwiGLU: the 16-row gate / up interleave
+            const int g = relu2 ? 0 : (rem >> 4) & 1;
+            const int f = relu2 ? rem : (rem >> 7) * 64 + ((rem >> 5) & 3) * 16 + (rem & 15);
             if (f < F && k < H) v = __ldg((g ? wu : wg) + ((e * F + f) * H + k) / 8);
             w1[i] = v;
         } else {
@@ -67,7 +70,7 @@ cudaError_t launch_prepare_bf16(const moe_plan* p, const __nv_bfloat16* wg, cons
     prepare_bf16_kernel<<<num_sms() * 8, 256, 0, s>>>(
         reinterpret_cast<const uint4*>(wg), reinterpret_cast<const uint4*>(wu), reinterpret_cast<const uint4*>(wd),
         reinterpret_cast<uint4*>(base + p->wb.w1), reinterpret_cast<uint4*>(base + p->wb.w2), (int)E, (int)F, (int)H,
-        (int)p->hp, (int)p->fp, (int)p->hr);
+        (int)p->hp, (int)p->fp, (int)p->hr, (int)p->w1r, (p->d.flags & MOE_FLAG_SQUARED_RELU) ? 1 : 0);
     return cudaGetLastError();
 }
 

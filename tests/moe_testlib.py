@@ -34,6 +34,26 @@ def assert_close(gpu: np.ndarray, ref: np.ndarray, precision: str, what: str = "
     return stats
 
 
+def assert_close_bf16_out(gpu16: np.ndarray, ref32: np.ndarray, precision: str, what: str = "") -> dict:
+    """A bf16 output against the oracle's fp32 output: the fp32 tolerance above
+    plus half a bf16 ulp of each reference value (2^-8 relative), the rounding
+    the output itself adds."""
+    gpu = np.asarray(gpu16, dtype=np.float64)
+    ref = np.asarray(ref32, dtype=np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite GPU output"
+    d = np.abs(gpu - ref)
+    rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
+    t = TOL[precision]
+    excess = d - (t["max_rms"] * rms + 2.0 ** -8 * np.abs(ref))
+    stats = dict(max_abs=float(d.max()) if d.size else 0.0, rms=rms, max_excess=float(excess.max()) if d.size else 0.0,
+                 mean_rel=float(d.mean() / max(np.abs(ref).mean(), 1e-30)) if d.size else 0.0)
+    assert stats["max_excess"] <= 0.0, f"{what}: {stats}"
+    if t["mean_rel"] is not None:
+        assert stats["mean_rel"] <= t["mean_rel"] + 2.0 ** -9, f"{what}: {stats}"
+    return stats
+
+
 class GpuMoe:
     """A plan + prepared weight buffer + workspace on cuda:0."""
 

@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import workloads
-from moe_testlib import GpuMoe, assert_close
+from moe_testlib import GpuMoe, assert_close, assert_close_bf16_out
 
 pytestmark = pytest.mark.gpu
 
@@ -89,8 +89,8 @@ def test_bf16_output_is_the_fp32_output_rounded(precision):
     # the same fp32 sums, rounded to nearest even: bit for bit
     rounded = oracle.round_bf16(out32.cpu().numpy())
     assert np.array_equal(out16.view(torch.int16).cpu().numpy().view(np.uint16), rounded)
-    ref = oracle.round_bf16(_oracle(precision, x, ids, probs, weights)).astype(np.uint32) << 16
-    assert_close(out16.float().cpu().numpy(), ref.view(np.float32), precision, f"bf16 out ({precision})")
+    assert_close_bf16_out(out16.float().cpu().numpy(), _oracle(precision, x, ids, probs, weights), precision,
+                          f"bf16 out ({precision})")
 
 
 def test_all_variants_together_on_the_decode_workload():
@@ -106,7 +106,42 @@ def test_all_variants_together_on_the_decode_workload():
     ids, probs = oracle.route(logits[:live].numpy(), w.top_k)
     toks = np.arange(0, live, 7)
     ref = oracle.forward_bf16(x[:live], ids, probs, *weights, tokens=toks, probs_in_fc1=True, gate_up_clamp=2.0)
-    ref16 = (oracle.round_bf16(ref).astype(np.uint32) << 16).view(np.float32)
-    assert_close(out[toks].float().cpu().numpy(), ref16, "bf16", "decode, all variants")
+    assert_close_bf16_out(out[toks].float().cpu().numpy(), ref, "bf16", "decode, all variants")
     # rows past the live count are untouched (NaN sentinel)
     assert torch.isnan(out[live:].float()).all()
+
+
+
+# ---------------------------------------------------------------- squared-ReLU experts (bf16)
+
+
+def test_squared_relu_matches_oracle():
+    x, logits, weights, ids, probs = _case(35)
+    wg, _, wd = weights
+    H, F, E, k, T = (SHAPE[c] for c in "HFEkT")
+    m = GpuMoe(H, F, E, k, T, (wg, wg, wd), squared_relu=True)
+    out = m.forward(x.cuda(), T, logits=logits.cuda())
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    ref = oracle.forward_bf16(x, ids, probs, wg, None, wd, squared_relu=True)
+    assert_close(out.cpu().numpy(), ref, "bf16", "squared ReLU")
+
+
+def test_squared_relu_with_variants_on_nano_shapes():
+    # H = 2688, F = 1856: F pads to 1920 columns of h and to 2048 FC1 rows, so the last pair
+    # tile's second CTA holds only padding rows and must store nothing
+    H, F, E, k, T = 2688, 1856, 128, 6, 600
+    x, logits, weights = workloads.small_case(H, F, E, k, T, seed=36)
+    wg, _, wd = weights
+    import routed_moe_swiglu_b200 as rm
+    m = GpuMoe(H, F, E, k, T, weights, squared_relu=True, probs_in_fc1=True, gate_up_clamp=1.5,
+               out_dtype="bf16")
+    rm.moe_prepare_weights(m.plan, wg.cuda(), None, wd.cuda(), m.wbuf)  # w_up is not read
+    out = m.forward(x.cuda(), T, logits=logits.cuda())
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    ids, probs = oracle.route(logits.numpy(), k)
+    toks = np.arange(0, T, 5)
+    ref = oracle.forward_bf16(x, ids, probs, wg, None, wd, tokens=toks, squared_relu=True, probs_in_fc1=True,
+                              gate_up_clamp=1.5)
+    assert_close_bf16_out(out[toks].float().cpu().numpy(), ref, "bf16", "squared ReLU, Nano shapes, all variants")

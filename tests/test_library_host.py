@@ -125,10 +125,29 @@ def test_bounded_wait_check_rejects_bad_arguments_before_launch():
 def test_plan_rejects_unknown_flags_and_bad_clamp():
     lib = rm.load_library()
     base = dict(hidden=256, ffn=512, num_experts=8, top_k=2, capacity=64, max_live_rows=0, precision=0)
-    for flags, clamp in ((0x4, 0.0), (0x80000000, 0.0), (0, -1.0), (0, float("nan")), (0, float("inf"))):
+    for flags, clamp in ((0x8, 0.0), (0x80000000, 0.0), (0, -1.0), (0, float("nan")), (0, float("inf"))):
         d = rm._Desc(*base.values(), flags, clamp)
         h = ctypes.c_void_p()
         assert lib.moe_plan_create(ctypes.byref(d), ctypes.byref(h)) == 1, (flags, clamp)
     p = rm.moe_plan_create(hidden=256, ffn=512, num_experts=8, top_k=2, capacity=64, out_dtype="bf16",
                            probs_in_fc1=True, gate_up_clamp=3.5)
     assert p.out_dtype == "bf16" and p.probs_in_fc1 and p.gate_up_clamp == 3.5
+
+
+
+def test_squared_relu_plans():
+    lib = rm.load_library()
+    with pytest.raises(rm.MoeError) as ei:
+        rm.moe_plan_create(hidden=256, ffn=512, num_experts=8, top_k=2, capacity=64, precision="mxfp8",
+                           squared_relu=True)
+    assert ei.value.code == 2
+    p = rm.moe_plan_create(hidden=256, ffn=200, num_experts=8, top_k=2, capacity=64, squared_relu=True)
+    assert p.squared_relu
+    # one FC1 projection: rows padded to 256 per expert, K padded to 256
+    assert rm.moe_weight_buffer_bytes(p) >= 8 * 256 * 256 * 2 + 8 * 256 * 256 * 2
+    fake = ctypes.c_void_p(1 << 20)
+    nb = rm.moe_weight_buffer_bytes(p)
+    # w_up may be NULL for squared-ReLU plans (validation then proceeds to the buffer size)
+    assert lib.moe_prepare_weights(p.handle, fake, None, fake, fake, nb - 1, None) == 4
+    q = rm.moe_plan_create(hidden=256, ffn=200, num_experts=8, top_k=2, capacity=64)
+    assert lib.moe_prepare_weights(q.handle, fake, None, fake, fake, rm.moe_weight_buffer_bytes(q), None) == 1
