@@ -206,13 +206,15 @@ def quantize_weights_mxfp8(w_gate, w_up, w_down):
     return gq, gs, uq, us, dq, ds
 
 
-def forward_mxfp8(x, ids, probs, wq, tokens=None, want_h=False, probs_in_fc1=False, gate_up_clamp=None):
+def forward_mxfp8(x, ids, probs, wq, tokens=None, want_h=False, probs_in_fc1=False, gate_up_clamp=None,
+                  squared_relu=False):
     """MXFP8 routed SwiGLU forward; `wq` = quantize_weights_mxfp8(...) output.
 
     Returns out fp32 [ntok, H] and, when want_h, (h codes [ntok,k,F],
     h scales [ntok,k,F/32], h pre-quantisation fp32 [ntok,k,F]).  Variants
-    as in forward_bf16."""
-    flags, clamp = _variant(probs_in_fc1, gate_up_clamp)
+    as in forward_bf16 (squared_relu: the gate codes are the one FC1
+    projection, the up codes are not read)."""
+    flags, clamp = _variant(probs_in_fc1, gate_up_clamp, squared_relu)
     xb = _bf16_bits(x)
     gq, gs, uq, us, dq, ds = wq
     ids = np.ascontiguousarray(ids, dtype=np.int32)

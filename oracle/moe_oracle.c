@@ -461,7 +461,8 @@ int oracle_forward_mxfp8(const uint16_t* x, const int32_t* ids, const float* pro
                          int64_t T, int H, int F, int E, int k,
                          const int64_t* toks, int64_t ntok, float* out,
                          uint8_t* h_q_out, uint8_t* h_s_out, float* h_f32_out, int flags, double clamp) {
-    if (!x || !ids || !probs || !wg_q || !wg_s || !wu_q || !wu_s || !wd_q || !wd_s || !toks || !out)
+    const int relu2 = (flags & ORACLE_SQUARED_RELU) != 0;
+    if (!x || !ids || !probs || !wg_q || !wg_s || (!relu2 && (!wu_q || !wu_s)) || !wd_q || !wd_s || !toks || !out)
         return ORACLE_EINVAL;
     if (H <= 0 || F <= 0 || (H % 32) || (F % 32) || E <= 0 || k <= 0 || k > 64 || ntok < 0)
         return ORACLE_EINVAL;
@@ -499,17 +500,19 @@ int oracle_forward_mxfp8(const uint16_t* x, const int32_t* ids, const float* pro
             if (e < 0 || e >= E) { bad = 1; break; }
             const uint8_t* gq = wg_q + (int64_t)e * F * H;
             const uint8_t* gs = wg_s + (int64_t)e * F * nbh;
-            const uint8_t* uq = wu_q + (int64_t)e * F * H;
-            const uint8_t* us = wu_s + (int64_t)e * F * nbh;
+            const uint8_t* uq = relu2 ? NULL : wu_q + (int64_t)e * F * H;
+            const uint8_t* us = relu2 ? NULL : wu_s + (int64_t)e * F * nbh;
             const uint8_t* dq = wd_q + (int64_t)e * H * F;
             const uint8_t* ds = wd_s + (int64_t)e * H * nbf;
             for (int f = 0; f < F; ++f) {
                 double g = 0.0, u = 0.0;
                 for (int c = 0; c < H; ++c) {
                     double wgv = g_e4m3_all[gq[(int64_t)f * H + c]] * g_pow2[gs[(int64_t)f * nbh + c / 32]];
-                    double wuv = g_e4m3_all[uq[(int64_t)f * H + c]] * g_pow2[us[(int64_t)f * nbh + c / 32]];
                     g += wgv * xd[c];
-                    u += wuv * xd[c];
+                    if (!relu2) {
+                        double wuv = g_e4m3_all[uq[(int64_t)f * H + c]] * g_pow2[us[(int64_t)f * nbh + c / 32]];
+                        u += wuv * xd[c];
+                    }
                 }
                 float hf = swiglu_value(g, u, clamp, flags, sp[j]);
                 hv[f] = (double)hf;

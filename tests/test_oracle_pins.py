@@ -549,3 +549,28 @@ def test_squared_relu_ignores_probs_scaling_by_pow2_like_plain():
     a = oracle.forward_bf16(x, ids, probs, wg, None, wd, squared_relu=True)
     b = oracle.forward_bf16(x, ids, probs, wg, None, wd, squared_relu=True, probs_in_fc1=True)
     assert np.array_equal(a, b)
+
+
+def test_squared_relu_mxfp8_single_expert_is_dense_relu2_mlp():
+    gen = torch.Generator().manual_seed(44)
+    T, H, F = 16, 128, 96
+    x = rand_bf16(gen, (T, H))
+    w1 = rand_bf16(gen, (1, F, H), H ** -0.5)
+    wd = rand_bf16(gen, (1, H, F), F ** -0.5)
+    wq = oracle.quantize_weights_mxfp8(w1, w1, wd)
+    # the up codes are not read: poison them, the result must not change
+    gq, gs, uq, us, dq, ds = wq
+    poisoned = (gq, gs, np.full_like(uq, 0x7F), np.full_like(us, 0xFE), dq, ds)
+    ids = np.zeros((T, 1), np.int32)
+    probs = np.ones((T, 1), np.float32)
+    out, (hq, hs, hf) = oracle.forward_mxfp8(x, ids, probs, poisoned, want_h=True, squared_relu=True)
+    # independent pipeline: numpy scales + torch e4m3 cast
+    xq = indep_dequant(*indep_mxfp8(x.double().numpy()))
+    g = xq @ indep_dequant(*indep_mxfp8(w1[0].double().numpy())).T
+    h32 = (np.maximum(g, 0.0) ** 2).astype(np.float32)
+    assert np.mean(h32 != hf[:, 0, :]) < 2e-2
+    ref = (indep_dequant(*indep_mxfp8(h32.astype(np.float64))) @ indep_dequant(*indep_mxfp8(wd[0].double().numpy())).T)
+    ref = ref.astype(np.float32)
+    rms = float(np.sqrt(np.mean(ref.astype(np.float64) ** 2)))
+    assert np.max(np.abs(out - ref)) <= 5e-2 * rms
+    assert np.mean(np.abs(out - ref)) <= 2e-3 * np.mean(np.abs(ref))
