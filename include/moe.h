@@ -102,8 +102,7 @@ typedef struct {
 #define MOE_FLAG_OUT_BF16 0x2u
 /*   MOE_FLAG_SQUARED_RELU  squared-ReLU experts (the Nano-v3 shapes of
  *       Megatron-LM PR #8367's measurements): one FC1 projection,
- *       h = relu(W_gate[e] . x)^2; W_up is not used.  bf16 plans only
- *       (MXFP8 plans with it are MOE_ERR_UNSUPPORTED).  The clamp and the
+ *       h = relu(W_gate[e] . x)^2; W_up is not used.  The clamp and the
  *       probability in FC1 act on the one pre-activation and on the row. */
 #define MOE_FLAG_SQUARED_RELU 0x4u
 
@@ -113,7 +112,7 @@ typedef struct moe_plan moe_plan; /* opaque, host memory only */
  * allocation).  Rejected (MOE_ERR_UNSUPPORTED): H or F not a multiple of 8
  * (bf16) or of 32 (MXFP8); k < 1, k > 16 or k > E; E < 1 or E > 1024;
  * capacity < 1 or > 2^24 rows; max_live_rows < 0 or > capacity;
- * H > 16384 or F > 16384; MOE_FLAG_SQUARED_RELU with MOE_MXFP8.  Rejected (MOE_ERR_INVALID_ARG): unknown flag
+ * H > 16384 or F > 16384.  Rejected (MOE_ERR_INVALID_ARG): unknown flag
  * bits, a negative or non-finite gate_up_clamp. */
 moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out);
 void moe_plan_destroy(moe_plan* plan);

@@ -105,7 +105,7 @@ static void compute_layouts(moe_plan* p) {
     WbufLayout& b = p->wb;
     off = 0;
     if (fp8) {
-        b.w1 = take(E * 2 * (size_t)p->fp * (size_t)p->hp);
+        b.w1 = take(E * (size_t)p->w1r * (size_t)p->hp);
         b.w1s = take(E * p->nt1 * p->ks1 * kSfBlock);
         b.w2 = take(E * H * (size_t)p->fp);
         b.w2s = take(E * p->nt2 * p->ks2 * kSfBlock);
@@ -156,7 +156,6 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     if (d.max_live_rows < 0 || d.max_live_rows > d.capacity) return MOE_ERR_UNSUPPORTED;
     if ((d.flags & ~(MOE_FLAG_PROBS_IN_FC1 | MOE_FLAG_OUT_BF16 | MOE_FLAG_SQUARED_RELU)) != 0)
         return MOE_ERR_INVALID_ARG;
-    if ((d.flags & MOE_FLAG_SQUARED_RELU) && d.precision == MOE_MXFP8) return MOE_ERR_UNSUPPORTED;
     if (!(d.gate_up_clamp >= 0.0f) || d.gate_up_clamp > 3.0e38f) return MOE_ERR_INVALID_ARG;
     moe_plan* p = new (std::nothrow) moe_plan();
     if (p == nullptr) return MOE_ERR_INVALID_ARG;
@@ -178,11 +177,12 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     p->hp = (long long)p->ks1 * 128;
     p->fp = (long long)p->ks2 * 128;
     p->hr = p->hp;
-    // bf16 FC1 rows per expert: gate and up interleaved (2 fp), or one projection padded to
-    // whole pair tiles of 256 rows (squared-ReLU experts)
-    p->w1r = (d.flags & MOE_FLAG_SQUARED_RELU) ? (p->fp + 255) / 256 * 256 : 2 * p->fp;
+    // FC1 rows per expert: gate and up interleaved (2 fp), or one projection (squared-ReLU
+    // experts), padded to whole weight tiles (bf16: pair tiles of 256 rows; MXFP8: 128)
+    const bool relu2 = (d.flags & MOE_FLAG_SQUARED_RELU) != 0;
+    p->w1r = !relu2 ? 2 * p->fp : (d.precision == MOE_MXFP8 ? p->fp : (p->fp + 255) / 256 * 256);
     if (d.precision == MOE_MXFP8) {
-        p->nt1 = (int)(p->fp / kG1BN8);  // f tiles of 64 cover fp; h's padding columns come out zero
+        p->nt1 = (int)(p->w1r / 128);  // weight tiles of 128 rows; h's padding columns come out zero
         p->nt2 = (d.hidden + kG2BN8 - 1) / kG2BN8;
     } else {
         p->nt1 = (int)(p->w1r / 256);  // pair tiles of 256 FC1 rows (SwiGLU: 128 f of gate and up)
@@ -296,7 +296,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
         // map per N in {32, 64, 96, 128}; the K pitches hp, fp are padded to 128 with zeros.
         const unsigned long long hp = (unsigned long long)plan->hp, fpp = (unsigned long long)plan->fp;
         const unsigned box128[3] = {128, 128, 2};
-        const unsigned long long dW1[3] = {128ull, uE * 2ull * fpp, hp / 128};
+        const unsigned long long dW1[3] = {128ull, uE * (unsigned long long)plan->w1r, hp / 128};
         const unsigned long long sW1[2] = {hp, 128ull};
         const unsigned long long dW2[3] = {128ull, uE * uH, fpp / 128};
         const unsigned long long sW2[2] = {fpp, 128ull};
@@ -385,7 +385,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g1.out_scales = nullptr;
     g1.out_ld = plan->fp;  // h rows: F values + zero padding to the down GEMM's K pitch
     g1.out_cols = (int)plan->fp;  // every padded column: f >= F are zero-weight rows, h = 0
-    g1.a_rows = fp8 ? 2 * plan->fp : plan->w1r;  // FC1 weight rows of an expert
+    g1.a_rows = plan->w1r;  // FC1 weight rows of an expert
     g1.n_tiles = plan->nt1;
     g1.k_blocks = plan->ks1;
     g1.wait_limit_ns = kWaitLimitNs;

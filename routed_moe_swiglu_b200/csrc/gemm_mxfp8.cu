@@ -71,6 +71,7 @@ constexpr uint32_t kEpiBytes = 2 * kStageHBytes > 4 * kYTBytes ? 2 * kStageHByte
 constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kSfBytes + kEpiBytes + 256;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kSfCol0 + kSfColsPerStage * kStages <= kTmemCols, "TMEM budget");
+static_assert(kEpiBytes >= 4 * 32 * 32 * 4, "squared-ReLU epilogue boxes");
 constexpr uint32_t kEpiBar = 1;                        // named barrier of the 4 epilogue warps
 
 struct __align__(8) Barriers {
@@ -331,7 +332,59 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
             }
             tc_fence_after_sync();
             const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)buf * kAccCols;
-            if (kMode == 0) {
+            if (kMode == 0 && p.relu2) {
+                // squared-ReLU experts: lane = f (this warp's 32 f from f0, one 32-f block),
+                // register j = route 32c + j.  h = relu(g)^2 goes through a per-warp box
+                // [route][32 f] fp32 (column rotated by the route against bank conflicts); then
+                // lane l quantises route 32c + l's block: amax, E8M0 scale, 32 E4M3 codes.
+                const int f0 = nt * kTileM + 32 * quad;
+                uint8_t* hq = reinterpret_cast<uint8_t*>(p.out);
+                uint8_t* hs_tile = p.out_scales + (size_t)(ti.y / kBM) * p.sf_ks_out * kSfBlock;
+                float* box = reinterpret_cast<float*>(sEpi + (size_t)quad * 32 * 32 * 4);
+                if (f0 < p.out_cols) {
+#pragma unroll 1
+                    for (int c = 0; c < nch; ++c) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(taddr + c * 32, v);
+                        float pv = 1.0f;
+                        if (p.route_probs != nullptr && c * 32 + lane < ti.z)
+                            pv = __ldg(p.route_probs + __ldg(p.perm + ti.w + c * 32 + lane));
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            float g = __uint_as_float(v[j]);
+                            if (p.clamp > 0.0f) g = fminf(fmaxf(g, -p.clamp), p.clamp);
+                            const float r = fmaxf(g, 0.0f);
+                            float hv = r * r;
+                            if (p.route_probs != nullptr) hv *= __shfl_sync(0xffffffffu, pv, j);
+                            box[j * 32 + ((lane + j) & 31)] = hv;
+                        }
+                        __syncwarp();
+                        float hv[32];
+                        float amax = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            hv[i] = box[lane * 32 + ((i + lane) & 31)];
+                            amax = fmaxf(amax, fabsf(hv[i]));
+                        }
+                        __syncwarp();
+                        float inv;
+                        const uint8_t sbyte = mxfp8_block_scale(amax, &inv);
+                        const int route = c * 32 + lane;
+                        if (route < ti.z) {
+                            uint32_t w[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                w[i] = e4m3x2(hv[4 * i + 1] * inv, hv[4 * i] * inv) |
+                                       (e4m3x2(hv[4 * i + 3] * inv, hv[4 * i + 2] * inv) << 16);
+                            uint4* dst = reinterpret_cast<uint4*>(hq + (size_t)(ti.y + route) * (size_t)p.out_ld + f0);
+                            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                            hs_tile[(size_t)(f0 / 128) * kSfBlock + sf_block_offset(route, (f0 % 128) / 32)] = sbyte;
+                        }
+                    }
+                }
+            } else if (kMode == 0) {
                 const bool lo = lane < 16;
                 const int fl = 16 * quad + (lane & 15);  // this lane's f within the tile's 64
                 uint8_t* hq = reinterpret_cast<uint8_t*>(p.out);

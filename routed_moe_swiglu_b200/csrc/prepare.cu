@@ -93,8 +93,8 @@ __global__ void __launch_bounds__(128) prepare_mxfp8_kernel(const uint4* __restr
                                                             const uint4* __restrict__ wd, uint2* __restrict__ w1q,
                                                             uint8_t* __restrict__ w1s, uint2* __restrict__ w2q,
                                                             uint8_t* __restrict__ w2s, int E, int F, int H, int hp,
-                                                            int fp, int nt1, int ks1, int nt2, int ks2) {
-    const long long rows1 = (long long)E * 2 * F;
+                                                            int fp, int nt1, int ks1, int nt2, int ks2, int relu2) {
+    const long long rows1 = (long long)E * (relu2 ? 1 : 2) * F;
     const long long rows2 = (long long)E * H;
     for (long long row = blockIdx.x; row < rows1 + rows2; row += gridDim.x) {
         const uint4* src;
@@ -102,14 +102,18 @@ __global__ void __launch_bounds__(128) prepare_mxfp8_kernel(const uint4* __restr
         uint8_t* sf_tile;  // the K-stage-0 scale block of this row's N tile
         int len, trow;
         if (row < rows1) {
-            const long long e = row / (2 * F);
-            const int rem = (int)(row - e * 2 * F);
+            const int per_e = relu2 ? F : 2 * F;
+            const long long e = row / per_e;
+            const int rem = (int)(row - e * per_e);
             const int gu = rem / F, f = rem - gu * F;
             src = (gu ? wu : wg) + ((size_t)e * F + f) * (H / 8);
-            trow = ((f % kG1BN8) >> 4) * 32 + gu * 16 + (f & 15);
-            dst = w1q + ((size_t)(e * nt1 + f / kG1BN8) * 128 + trow) * (hp / 8);
+            // SwiGLU: 64 f per 128-row tile, gate / up interleaved in groups of 16;
+            // squared-ReLU experts: 128 f per tile in f order
+            const int tile = relu2 ? f / 128 : f / kG1BN8;
+            trow = relu2 ? f % 128 : ((f % kG1BN8) >> 4) * 32 + gu * 16 + (f & 15);
+            dst = w1q + ((size_t)(e * nt1 + tile) * 128 + trow) * (hp / 8);
             len = H;
-            sf_tile = w1s + ((size_t)e * nt1 + f / kG1BN8) * ks1 * kSfBlock;
+            sf_tile = w1s + ((size_t)e * nt1 + tile) * ks1 * kSfBlock;
         } else {
             const long long r2 = row - rows1;
             const long long e = r2 / H;
@@ -155,7 +159,8 @@ cudaError_t launch_prepare_mxfp8(const moe_plan* p, const __nv_bfloat16* wg, con
     prepare_mxfp8_kernel<<<num_sms() * 16, 128, 0, s>>>(
         reinterpret_cast<const uint4*>(wg), reinterpret_cast<const uint4*>(wu), reinterpret_cast<const uint4*>(wd),
         reinterpret_cast<uint2*>(base + p->wb.w1), base + p->wb.w1s, reinterpret_cast<uint2*>(base + p->wb.w2),
-        base + p->wb.w2s, E, F, H, (int)p->hp, (int)p->fp, p->nt1, p->ks1, p->nt2, p->ks2);
+        base + p->wb.w2s, E, F, H, (int)p->hp, (int)p->fp, p->nt1, p->ks1, p->nt2, p->ks2,
+        (p->d.flags & MOE_FLAG_SQUARED_RELU) ? 1 : 0);
     return cudaGetLastError();
 }
 

@@ -115,16 +115,21 @@ def test_all_variants_together_on_the_decode_workload():
 # ---------------------------------------------------------------- squared-ReLU experts (bf16)
 
 
-def test_squared_relu_matches_oracle():
+@pytest.mark.parametrize("precision", ["bf16", "mxfp8"])
+def test_squared_relu_matches_oracle(precision):
     x, logits, weights, ids, probs = _case(35)
     wg, _, wd = weights
     H, F, E, k, T = (SHAPE[c] for c in "HFEkT")
-    m = GpuMoe(H, F, E, k, T, (wg, wg, wd), squared_relu=True)
+    m = GpuMoe(H, F, E, k, T, (wg, wg, wd), precision=precision, squared_relu=True)
     out = m.forward(x.cuda(), T, logits=logits.cuda())
     torch.cuda.synchronize()
     assert m.status() == 0
-    ref = oracle.forward_bf16(x, ids, probs, wg, None, wd, squared_relu=True)
-    assert_close(out.cpu().numpy(), ref, "bf16", "squared ReLU")
+    if precision == "bf16":
+        ref = oracle.forward_bf16(x, ids, probs, wg, None, wd, squared_relu=True)
+    else:
+        # the oracle's MXFP8 path quantises W1 as its gate rows; the up rows are not used
+        ref = oracle.forward_mxfp8(x, ids, probs, oracle.quantize_weights_mxfp8(wg, wg, wd), squared_relu=True)
+    assert_close(out.cpu().numpy(), ref, precision, f"squared ReLU ({precision})")
 
 
 def test_squared_relu_with_variants_on_nano_shapes():

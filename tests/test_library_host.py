@@ -137,10 +137,11 @@ def test_plan_rejects_unknown_flags_and_bad_clamp():
 
 def test_squared_relu_plans():
     lib = rm.load_library()
-    with pytest.raises(rm.MoeError) as ei:
-        rm.moe_plan_create(hidden=256, ffn=512, num_experts=8, top_k=2, capacity=64, precision="mxfp8",
+    m = rm.moe_plan_create(hidden=256, ffn=512, num_experts=8, top_k=2, capacity=64, precision="mxfp8",
                            squared_relu=True)
-    assert ei.value.code == 2
+    # MXFP8: one projection of F rows per expert (codes) instead of gate and up
+    assert rm.moe_weight_buffer_bytes(m) < rm.moe_weight_buffer_bytes(
+        rm.moe_plan_create(hidden=256, ffn=512, num_experts=8, top_k=2, capacity=64, precision="mxfp8"))
     p = rm.moe_plan_create(hidden=256, ffn=200, num_experts=8, top_k=2, capacity=64, squared_relu=True)
     assert p.squared_relu
     # one FC1 projection: rows padded to 256 per expert, K padded to 256
