@@ -76,19 +76,28 @@ def parse_args():
 
 
 class Dist:
-    def __init__(self, n_gpus):
+    """One process per GPU (RANK / LOCAL_RANK / WORLD_SIZE from the launcher).
+    The path shards by token with replicated weights, so the only collectives
+    are the barrier around the timed region and the max over ranks of its
+    time.  backend: "nccl" on GPUs; "gloo" runs the same steps on CPU (tests)."""
+
+    def __init__(self, n_gpus, backend: str | None = None):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
         self.pg = None
         if self.world > 1:
             import datetime
 
             import torch.distributed as dist
 
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                    device_id=torch.device("cuda", self.local))
+            if self.backend == "nccl":
+                torch.cuda.set_device(self.local)
+                dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                        device_id=torch.device("cuda", self.local))
+            else:
+                dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=60))
             self.pg = dist
         elif torch.cuda.is_available():
             torch.cuda.set_device(0)
@@ -100,7 +109,8 @@ class Dist:
     def max(self, v: float) -> float:
         if self.pg is None:
             return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dev = "cuda" if self.backend == "nccl" else "cpu"
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
