@@ -86,15 +86,15 @@ static void compute_layouts(moe_plan* p) {
     w.tiles = take((size_t)p->max_m_tiles * 16);
     w.perm = take(L * k * 4);
     w.inv = take(L * k * 4);
-    w.xrow = fp8 ? 0 : take(L * k * 4);
     const size_t mtiles = (size_t)p->max_m_tiles;
+    w.ready = fp8 ? 0 : take(mtiles * 4);
     if (fp8) {
         w.xq = take(R * (size_t)p->hp);
         w.xs = take(mtiles * p->ks1 * kSfBlock);
         w.h = take(R * (size_t)p->fp);
         w.hs = take(mtiles * p->ks2 * kSfBlock);
     } else {
-        w.xq = take(R * (size_t)p->hp * 2);  // rows of tiles the gate/up GEMM does not gather itself
+        w.xq = take(R * (size_t)p->hp * 2);  // x rows of tiles of more than kGatherInGemmMax routes
         w.xs = 0;
         w.h = take(R * (size_t)p->fp * 2);
         w.hs = 0;
@@ -319,8 +319,8 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
         // atoms.  Weights (A) load 128 rows per CTA; route rows (B) N/2 rows, one map per N/2 in
         // {16, ..., 128}.  Gate/up tiles of at most kGatherInGemmMax routes instead gather
         // their B rows straight from x (one-row boxes of one atom, four rows per
-        // instruction; columns past H read as zeros); the gather kernel writes only the
-        // permuted x rows of the larger tiles.
+        // instruction; columns past H read as zeros); the gate/up GEMM's copy warps write
+        // the permuted x rows of the larger tiles ahead of their loads.
         const unsigned long long hp = (unsigned long long)plan->hp, fpp = (unsigned long long)plan->fp;
         // weights: blocks of [2 atoms][128 rows][64 elements], 32 KB contiguous, one per
         // (expert, 128-row block, K stage); atom a of block b is index 2b + a of the map's
@@ -361,20 +361,18 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     int* perm = reinterpret_cast<int*>(ws + L.perm);
     int* inv = reinterpret_cast<int*>(ws + L.inv);
     int4* tiles = reinterpret_cast<int4*>(ws + L.tiles);
-    int* xrow = fp8 ? nullptr : reinterpret_cast<int*>(ws + L.xrow);
+    int* ready = fp8 ? nullptr : reinterpret_cast<int*>(ws + L.ready);
     e = launch_permute(plan, live_count_dev, r_ids, reinterpret_cast<int*>(ws + L.blkcnt),
                        reinterpret_cast<int*>(ws + L.offsets), reinterpret_cast<int*>(ws + L.padoff), tiles, perm, inv,
-                       xrow, status, s);
+                       ready, status, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 
     if (!mark(2)) return MOE_ERR_CUDA;
-    if (fp8)
+    if (fp8) {  // bf16: the gate/up GEMM copies the x rows itself
         e = launch_gather_mxfp8(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, (int)plan->hp, k,
                                 inv, ws + L.xq, ws + L.xs, s);
-    else
-        e = launch_gather_bf16(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, (int)plan->hp, k, xrow,
-                               reinterpret_cast<__nv_bfloat16*>(ws + L.xq), s);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
 
     const long long m_tiles = plan->max_m_tiles;
     GemmParams g1{};
@@ -399,6 +397,13 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g1.route_probs = probs_in_fc1 ? r_probs : nullptr;
     g1.clamp = plan->d.gate_up_clamp;
     g1.relu2 = (plan->d.flags & MOE_FLAG_SQUARED_RELU) != 0;
+    g1.x = static_cast<const uint8_t*>(x);
+    g1.x_pitch = (long long)H * 2;
+    g1.x_bytes = H * 2;
+    g1.xg = ws + L.xq;
+    g1.xg_pitch = plan->hp * 2;
+    g1.ready = ready;
+    g1.copy_next = status + kStCopyNext;
     if (!mark(3)) return MOE_ERR_CUDA;
     e = fp8 ? launch_gemm1_mxfp8(tA1, rB1, g1, m_tiles * g1.n_tiles, s)
             : launch_gemm1_bf16_pair(tA1, tX, rB1, g1, m_tiles * g1.n_tiles, s);

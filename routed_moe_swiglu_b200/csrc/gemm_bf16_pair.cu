@@ -38,6 +38,13 @@
 // completion is signalled to both CTAs' barriers (commit with a CTA mask);
 // warps 2-9 drain the accumulators and release each accumulator on CTA 0's
 // barrier.  Two accumulators of 256 fp32 columns (512 TMEM columns) per CTA.
+// The gate/up kernel has four more warps that copy the x rows of tiles of
+// more than 32 routes into their padded route rows while the MMAs run (the
+// dispatch fused into the GEMM: no separate gather pass over HBM).  They
+// claim 8-route chunks in tile order from a global counter and count each
+// finished chunk in its tile's ready counter; a producer acquires that count
+// before the tile's first route-row load.  The copy warps wait on nothing,
+// and every CTA of the persistent grid is resident, so those waits end.
 //
 // Every mbarrier wait is bounded; the pair meets in cluster barriers only at
 // start-up and before TMEM is released.  Each output element is one route's
@@ -50,8 +57,8 @@ namespace moe {
 namespace {
 
 constexpr int kStages = 3;
-constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
+constexpr int kCopyWarps = 4;                           // gate/up: x rows of large tiles into their route rows
 constexpr int kPairM = 256;                             // M of the pair MMA (weight rows)
 constexpr int kAtoms = 2;                               // 64-element (128-byte) swizzle atoms per K stage
 constexpr int kStageK = kAtoms * kBK;                   // 128 K elements per stage
@@ -67,6 +74,7 @@ constexpr uint32_t kYTBytes = 32 * 32 * 4;              // down: y of 32 routes 
 
 template <int kMode>
 struct PairCfg {
+    static constexpr int kThreads = (2 + kEpiWarps + (kMode == 0 ? kCopyWarps : 0)) * 32;
     // one transpose box per epilogue warp
     static constexpr uint32_t kEpiBytes = kEpiWarps * (kMode == 0 ? kH0Bytes : kYTBytes);
     static constexpr size_t kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kEpiBytes + 256;
@@ -170,12 +178,26 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
             // gate/up tiles of at most kGatherInGemmMax routes: lane L gathers this CTA's B
             // rows 4L..4L+3 from x, the rows of the tokens of routes hb * rank + 4L + q
             // (rows past the tile's routes repeat its first token: in bounds, and their
-            // output columns are never stored).  Larger tiles load their rows, gathered
-            // by the gather kernel, as one box: a gather moves 512 bytes per TMA
-            // instruction, too few to feed a full tile.
+            // output columns are never stored).  Larger tiles load their rows, written by
+            // the copy warps, as one box: a gather moves 512 bytes per TMA instruction, too
+            // few to feed a full tile.
             int tok[4] = {0, 0, 0, 0};
             const bool from_x = kMode == 0 && ti.z <= kGatherInGemmMax;
             const bool gathers = from_x && 4 * lane < hb;
+            if (kMode == 0 && !from_x) {
+                // the copy warps (of any CTA) have written all of this tile's route rows:
+                // acquire their counts, then order them before this thread's TMA reads
+                bool rdy = true;
+                if (lane == 0) {
+                    rdy = wait_count_bounded(p.ready + mt, (ti.z + kCopyChunk - 1) / kCopyChunk, abort_flag,
+                                             p.wait_limit_ns);
+                    fence_proxy_async_global();
+                }
+                if (!__shfl_sync(0xffffffffu, rdy, 0)) {
+                    ok = false;
+                    break;
+                }
+            }
             if (from_x) {
                 const int first = __ldg(p.perm + ti.w) / p.top_k;
 #pragma unroll
@@ -280,7 +302,7 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
             (void)mbar_wait_bounded(&bars->done, 0, &never, 100000000ull);
         }
         __syncwarp();
-    } else {
+    } else if (warp < 2 + kEpiWarps) {
         // ---------------- epilogue: warps 2..9
         const int ew = warp - 2;
         const int quad = warp & 3;   // TMEM lane quarter this warp may read
@@ -416,6 +438,60 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty0[buf]);  // release on CTA 0's barrier
         }
+    } else if constexpr (kMode == 0) {
+        // ---------------- copy warps (gate/up): the x rows of tiles of more than
+        // kGatherInGemmMax routes into their padded route rows, one 8-route chunk at a
+        // time, claimed in tile order so that the first tiles the producers load are
+        // the first complete.  A chunk's rows are made visible (and ordered before TMA
+        // reads) before it is counted in ready[tile].
+        const unsigned units = (unsigned)num_m * kChunksPerTile;
+        const int chunks_in = p.x_bytes >> 4;  // 16-byte chunks of an x row
+        const int chunks_out = (int)(p.xg_pitch >> 4);
+        while (true) {
+            unsigned u = 0;
+            if (lane == 0) u = atomicAdd(p.copy_next, 1u);
+            u = __shfl_sync(0xffffffffu, u, 0);
+            if (u >= units || *abort_flag != 0) break;
+            const int mt = (int)(u / kChunksPerTile);
+            const int r0 = (int)(u % kChunksPerTile) * kCopyChunk;
+            const int4 ti = __ldg(p.tiles + mt);
+            if (ti.z <= kGatherInGemmMax || r0 >= ti.z) continue;
+            const int nrows = min(kCopyChunk, ti.z - r0);
+            const int my_tok = lane < nrows ? __ldg(p.perm + ti.w + r0 + lane) / p.top_k : 0;
+            // two rows at a time: 16 loads of 16 bytes in flight per lane
+#pragma unroll 1
+            for (int i = 0; i < nrows; i += 2) {
+                const bool two = i + 1 < nrows;
+                const int tok0 = __shfl_sync(0xffffffffu, my_tok, i);
+                const int tok1 = __shfl_sync(0xffffffffu, my_tok, two ? i + 1 : i);
+                const uint4* src0 = reinterpret_cast<const uint4*>(p.x + (size_t)tok0 * (size_t)p.x_pitch);
+                const uint4* src1 = reinterpret_cast<const uint4*>(p.x + (size_t)tok1 * (size_t)p.x_pitch);
+                uint4* dst0 = reinterpret_cast<uint4*>(p.xg + (size_t)(ti.y + r0 + i) * (size_t)p.xg_pitch);
+                uint4* dst1 = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dst0) + p.xg_pitch);
+                for (int c0 = 0; c0 < chunks_out; c0 += 8 * 32) {
+                    uint4 v0[8], v1[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int ch = c0 + j * 32 + lane;
+                        const bool in = ch < chunks_in;
+                        v0[j] = in ? __ldg(src0 + ch) : make_uint4(0u, 0u, 0u, 0u);
+                        v1[j] = in && two ? __ldg(src1 + ch) : make_uint4(0u, 0u, 0u, 0u);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int ch = c0 + j * 32 + lane;
+                        if (ch < chunks_out) {
+                            dst0[ch] = v0[j];
+                            if (two) dst1[ch] = v1[j];
+                        }
+                    }
+                }
+            }
+            fence_proxy_async_global();
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) red_release_gpu_add(p.ready + mt, 1);
+        }
     }
 
     // ---------------- teardown: no pair MMA is in flight once CTA 0 has seen "done"
@@ -428,13 +504,13 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(PairCfg<0>::kThreads, 1)
     moe_gemm_gate_up_swiglu_bf16_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmX,
                                       const __grid_constant__ BoxMaps8 tmB, const GemmParams p) {
     pair_gemm_body<0>(tmA, &tmX, &tmB, p);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(PairCfg<1>::kThreads, 1)
     moe_gemm_down_bf16_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BoxMaps8 tmB,
                             const GemmParams p) {
     pair_gemm_body<1>(tmA, nullptr, &tmB, p);
@@ -443,6 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 struct PairLaunchCache {
     size_t smem = 0;
+    int threads = 0;
     int device = -1;
     int pairs = 0;
 };
@@ -462,7 +539,7 @@ cudaError_t launch_pair(void (*kern)(CUtensorMap, Operands..., GemmParams), Pair
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see pdl_wait()
     attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(cache->threads);
     cfg.dynamicSmemBytes = cache->smem;
     cfg.stream = s;
     cfg.attrs = attr;
@@ -493,14 +570,14 @@ cudaError_t launch_pair(void (*kern)(CUtensorMap, Operands..., GemmParams), Pair
 
 cudaError_t launch_gemm1_bf16_pair(const CUtensorMap& a, const CUtensorMap& x_rows, const BoxMaps8& b,
                                    const GemmParams& gp, long long max_tiles, cudaStream_t s) {
-    static PairLaunchCache cache{PairCfg<0>::kSmemBytes};
+    static PairLaunchCache cache{PairCfg<0>::kSmemBytes, PairCfg<0>::kThreads};
     return launch_pair<CUtensorMap, BoxMaps8>(moe_gemm_gate_up_swiglu_bf16_pair, &cache, a, x_rows, b, gp, max_tiles,
                                               s);
 }
 
 cudaError_t launch_gemm2_bf16_pair(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
                                    cudaStream_t s) {
-    static PairLaunchCache cache{PairCfg<1>::kSmemBytes};
+    static PairLaunchCache cache{PairCfg<1>::kSmemBytes, PairCfg<1>::kThreads};
     return launch_pair<BoxMaps8>(moe_gemm_down_bf16_pair, &cache, a, b, gp, max_tiles, s);
 }
 

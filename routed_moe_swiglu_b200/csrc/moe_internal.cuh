@@ -24,6 +24,8 @@ constexpr int kG2BN = 256;         // bf16: output columns per down weight tile
 constexpr int kRouteTile = 256;    // bf16: most routes per tile (N of a pair MMA)
 constexpr int kRouteAlign = 32;    // bf16: route rows of an expert start on a multiple of this
 constexpr int kGatherInGemmMax = 32;  // bf16: route tiles of at most this many routes read x rows by token
+constexpr int kCopyChunk = 8;         // bf16: routes per chunk the gate/up GEMM's copy warps claim
+constexpr int kChunksPerTile = kRouteTile / kCopyChunk;
 constexpr int kG1BN8 = 64;         // MXFP8: f values per gate/up tile (64 gate + 64 up MMA columns)
 constexpr int kG2BN8 = 128;        // MXFP8: output columns per down tile
 constexpr int kSfBlock = 512;      // MXFP8 scales of 128 rows x 4 k-groups, [row%32][row/32][k-group]
@@ -32,13 +34,13 @@ constexpr int kMaxTopK = 16;
 constexpr int kMaxExperts = 1024;
 
 // Status word layout (uint32 words at the start of the workspace).
-enum : int { kStFlags = 0, kStNumMTiles = 1, kStTotalRoutes = 2, kStWords = 64 };
+enum : int { kStFlags = 0, kStNumMTiles = 1, kStTotalRoutes = 2, kStCopyNext = 3, kStWords = 64 };
 
 // Default bound of any on-device wait before the kernel gives up (ns).
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;
 
 struct WsLayout {
-    size_t status, r_ids, r_probs, blkcnt, offsets, padoff, tiles, perm, inv, xrow;
+    size_t status, r_ids, r_probs, blkcnt, offsets, padoff, tiles, perm, inv, ready;
     size_t xq, xs, h, hs, y;
     size_t total;
 };
@@ -108,6 +110,17 @@ struct GemmParams {
     const float* route_probs;
     float clamp;
     int relu2;                      // bf16 gate/up GEMM: squared-ReLU experts (A = one FC1 projection)
+    // bf16 gate/up: the copy warps write the x rows of tiles of more than
+    // kGatherInGemmMax routes into their padded route rows xg (pitch xg_pitch
+    // bytes, zeros from x_bytes to the pitch), counting each 32-route chunk in
+    // ready[tile]; copy_next (zeroed with the tile list) hands out the chunks
+    const uint8_t* x;
+    long long x_pitch;              // bytes between x rows
+    int x_bytes;                    // bytes of one x row (H * 2)
+    uint8_t* xg;
+    long long xg_pitch;
+    int* ready;
+    unsigned* copy_next;
 };
 
 // ---------------------------------------------------------------- launchers
@@ -121,13 +134,11 @@ cudaError_t launch_route_topk(const float* logits, const int* live, int max_live
                               float* probs, unsigned* status, cudaStream_t s);
 cudaError_t launch_canon_routes(const int* ids_in, const float* probs_in, const int* live, int max_live, int E,
                                 int k, int* ids_out, float* probs_out, unsigned* status, cudaStream_t s);
-// xrow (bf16 only, else null): per route, its padded row if the gather kernel
-// writes it (tiles of more than kGatherInGemmMax routes), else -1
+// ready (bf16 only, else null): one counter per route tile, zeroed with the
+// tile list; the gate/up GEMM's copy warps count the tile's copied chunks in it
 cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* blkcnt, int* offsets,
-                           int* padoff, int4* tiles, int* perm, int* inv, int* xrow, unsigned* status_words,
+                           int* padoff, int4* tiles, int* perm, int* inv, int* ready, unsigned* status_words,
                            cudaStream_t s);
-cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
-                               const int* xrow, __nv_bfloat16* xp, cudaStream_t s);
 cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
                                 const int* inv, uint8_t* xq, uint8_t* xs, cudaStream_t s);
 // probs null: every route's weight is 1 (the probabilities were applied in FC1);

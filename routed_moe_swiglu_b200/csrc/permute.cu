@@ -14,9 +14,10 @@
 //   scatter  per block: one 32-bit lane mask per (warp, expert) gives every
 //            route its rank among earlier tokens of the block routed to the
 //            same expert (popcount of the lower lanes plus the earlier warps)
-// and a gather that copies each token's x row into its padded route rows
-// (MXFP8: quantised once per token; bf16: only the rows of route tiles the
-// gate/up GEMM does not gather from x itself).
+//            The scan also zeroes the per-tile counters and the chunk counter
+//            through which the bf16 gate/up GEMM copies x rows itself.
+// and, for MXFP8, a gather that quantises each token's x row once and writes
+// it to its padded route rows.
 #include "moe_internal.cuh"
 #include "mxfp8.cuh"
 
@@ -77,6 +78,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int* __restrict_
                                                           int tile_rows, int row_align, int* __restrict__ blkcnt,
                                                           int* __restrict__ offsets,
                                                           int* __restrict__ padoff, int4* __restrict__ tiles,
+                                                          int* __restrict__ ready,
                                                           unsigned* __restrict__ status_words) {
     __shared__ int s_warp[32];
     pdl_trigger();
@@ -113,6 +115,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int* __restrict_
             const int rows = tot - i * tile_rows;
             tiles[ex_mt + i] =
                 make_int4(e, ex_pad + i * tile_rows, rows < tile_rows ? rows : tile_rows, ex_tot + i * tile_rows);
+            if (ready != nullptr) ready[ex_mt + i] = 0;
         }
     }
     if (e == 0) {
@@ -120,13 +123,14 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int* __restrict_
         padoff[E] = sum_pad;
         status_words[kStNumMTiles] = (unsigned)sum_mt;
         status_words[kStTotalRoutes] = (unsigned)sum_tot;
+        status_words[kStCopyNext] = 0u;
     }
 }
 
 __global__ void __launch_bounds__(kTokPerBlk) route_scatter_kernel(
     const int* __restrict__ ids, const int* __restrict__ live, int max_live, int E, int k,
-    const int* __restrict__ blkprefix, const int* __restrict__ offsets, const int* __restrict__ padoff, int tile_rows,
-    int* __restrict__ perm, int* __restrict__ inv, int* __restrict__ xrow) {
+    const int* __restrict__ blkprefix, const int* __restrict__ offsets, const int* __restrict__ padoff,
+    int* __restrict__ perm, int* __restrict__ inv) {
     extern __shared__ uint32_t s_mem[];
     pdl_trigger();
     pdl_wait();
@@ -168,66 +172,16 @@ __global__ void __launch_bounds__(kTokPerBlk) route_scatter_kernel(
             const int e = my_e[j];
             if (e < 0) {
                 inv[(size_t)t * k + j] = -1;
-                if (xrow != nullptr) xrow[(size_t)t * k + j] = -1;
             } else {
                 const int row = wbase[w * E + e] + __popc(masks[w * E + e] & lower);
-                const int local = row - offsets[e];
                 perm[row] = t * k + j;
-                inv[(size_t)t * k + j] = padoff[e] + local;
-                if (xrow != nullptr) {
-                    // the route's tile holds min(tile_rows, routes of e left from its first row)
-                    const int left = offsets[e + 1] - offsets[e] - local / tile_rows * tile_rows;
-                    xrow[(size_t)t * k + j] =
-                        (left < tile_rows ? left : tile_rows) > kGatherInGemmMax ? padoff[e] + local : -1;
-                }
+                inv[(size_t)t * k + j] = padoff[e] + row - offsets[e];
             }
         }
     }
 }
 
 constexpr int kRowThreads = 128;
-
-// bf16 gather: one warp per token (grid-stride) reads the token's x row
-// once and writes it to those of its k padded route rows that the scatter
-// marked (routes in tiles of more than kGatherInGemmMax routes; the gate/up
-// GEMM reads the x rows of smaller tiles itself).  Each lane keeps up to 8
-// of its 16-byte loads in flight before storing them.
-constexpr int kGatherWarps = 8;
-
-__global__ void __launch_bounds__(kGatherWarps * 32) gather_rows_bf16_kernel(
-    const uint4* __restrict__ x, const int* __restrict__ live, int max_live, int H, int hp, int k,
-    const int* __restrict__ xrow, uint4* __restrict__ xp) {
-    pdl_trigger();
-    pdl_wait();
-    const int n = clamp_live(live, max_live);
-    const int lane = threadIdx.x & 31;
-    const int chunks = H / 8;       // 8 bf16 per 16 bytes
-    const int chunks_out = hp / 8;  // destination rows are padded to hp with zeros
-    const int warps = gridDim.x * kGatherWarps;
-    for (int t = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); t < n; t += warps) {
-        const int my_row = lane < k ? __ldg(xrow + (size_t)t * k + lane) : -1;
-        const unsigned targets = __ballot_sync(0xffffffffu, my_row >= 0);
-        if (targets == 0u) continue;
-        const uint4* src = x + (size_t)t * chunks;
-        for (int c0 = 0; c0 < chunks_out; c0 += 8 * 32) {
-            uint4 v[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int c = c0 + i * 32 + lane;
-                v[i] = c < chunks ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-            }
-            for (unsigned m = targets; m != 0u; m &= m - 1u) {
-                const int pr = __shfl_sync(0xffffffffu, my_row, __ffs(m) - 1);
-                uint4* dst = xp + (size_t)pr * chunks_out;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int c = c0 + i * 32 + lane;
-                    if (c < chunks_out) dst[c] = v[i];
-                }
-            }
-        }
-    }
-}
 
 // MXFP8 gather: one 128-thread block per token quantises the token's x row
 // once (blocks of 32 along H, 4 threads per block) and writes the E4M3 codes
@@ -351,7 +305,7 @@ int grid_for_warps(long long items, int warps_per_block, int per_sm) {
 }  // namespace
 
 cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* blkcnt, int* offsets,
-                           int* padoff, int4* tiles, int* perm, int* inv, int* xrow, unsigned* status_words,
+                           int* padoff, int4* tiles, int* perm, int* inv, int* ready, unsigned* status_words,
                            cudaStream_t s) {
     const int E = p->d.num_experts, k = p->d.top_k;
     const int max_live = (int)p->max_live;
@@ -360,7 +314,7 @@ cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* 
                                        live, max_live, E, k, blkcnt);
     if (err != cudaSuccess) return err;
     err = launch_dependent(route_scan_kernel, dim3(1), dim3(1024), 0, s, live, max_live, E, p->tile_rows,
-                           p->row_align, blkcnt, offsets, padoff, tiles, status_words);
+                           p->row_align, blkcnt, offsets, padoff, tiles, ready, status_words);
     if (err != cudaSuccess) return err;
     const size_t smem = (size_t)(kTokPerBlk / 32) * E * 8;
     if (smem > 48 * 1024) {
@@ -377,15 +331,7 @@ cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* 
         }
     }
     return launch_dependent(route_scatter_kernel, dim3(nblk), dim3(kTokPerBlk), smem, s, r_ids, live, max_live, E, k,
-                            blkcnt, offsets, padoff, p->tile_rows, perm, inv, xrow);
-}
-
-cudaError_t launch_gather_bf16(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
-                               const int* xrow, __nv_bfloat16* xp, cudaStream_t s) {
-    const int grid = grid_for_warps(max_live, kGatherWarps, 8);
-    return launch_dependent(gather_rows_bf16_kernel, dim3(grid), dim3(kGatherWarps * 32), 0, s,
-                            reinterpret_cast<const uint4*>(x), live, max_live, H, hp, k, xrow,
-                            reinterpret_cast<uint4*>(xp));
+                            blkcnt, offsets, padoff, perm, inv);
 }
 
 cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,

@@ -145,6 +145,31 @@ __device__ __forceinline__ void bulk_wait_group() {
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// The same for global memory: generic-proxy writes (this thread's, or ones
+// it acquired from another thread) before later TMA reads of them.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(int* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Wait until *counter >= target (acquire), giving up after limit_ns or when
+// *abort_flag is raised; returns whether the count was reached.
+__device__ __forceinline__ bool wait_count_bounded(const int* counter, int target, volatile int* abort_flag,
+                                                   unsigned long long limit_ns) {
+    if (ld_acquire_gpu(counter) >= target) return true;
+    const unsigned long long t0 = global_timer_ns();
+    while (true) {
+        __nanosleep(128);
+        if (ld_acquire_gpu(counter) >= target) return true;
+        if (*abort_flag != 0 || global_timer_ns() - t0 > limit_ns) return false;
+    }
+}
 
 // ---------------------------------------------------------------- tcgen05
 
