@@ -56,9 +56,14 @@ def _load():
     lib.oracle_forward_bf16.argtypes = [P, P, P, P, P, P, I64, I, I, I, I, P, I64, P, P, I, D]
     lib.oracle_forward_mxfp8.argtypes = [P, P, P, P, P, P, P, P, P, I64, I, I, I, I, P, I64, P, P, P, P, I, D]
     lib.oracle_round_bf16.argtypes = [P, I64, P]
+    lib.oracle_nvfp4_quantize.argtypes = [P, I64, I64, I, P, P, P]
+    lib.oracle_nvfp4_quantize_bf16.argtypes = [P, I64, I64, I, P, P, P]
+    lib.oracle_nvfp4_dequantize.argtypes = [P, P, P, I64, I64, I, P]
+    lib.oracle_forward_nvfp4.argtypes = [P, P, P, P, P, P, P, P, P, I64, I, I, I, I, P, I64, P, P, P, P, P, I, D]
     for name in ("oracle_mxfp8_quantize", "oracle_mxfp8_quantize_bf16", "oracle_mxfp8_dequantize",
                  "oracle_route", "oracle_permute", "oracle_forward_bf16", "oracle_forward_mxfp8",
-                 "oracle_round_bf16"):
+                 "oracle_round_bf16", "oracle_nvfp4_quantize", "oracle_nvfp4_quantize_bf16",
+                 "oracle_nvfp4_dequantize", "oracle_forward_nvfp4"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -233,3 +238,88 @@ def forward_mxfp8(x, ids, probs, wq, tokens=None, want_h=False, probs_in_fc1=Fal
                                         toks.size, _ptr(out), _ptr(hq), _ptr(hs), _ptr(hf), flags, clamp),
            "forward_mxfp8")
     return (out, (hq, hs, hf)) if want_h else out
+
+
+def nvfp4_quantize(values, per_row: bool = True):
+    """NVFP4 (the per-token recipe) of an fp32 [rows, cols] matrix (cols % 16 == 0), or of a
+    bf16 tensor / uint16 bit array.  Returns (codes uint8 [rows, cols/2], element 2i in the
+    low nibble; E4M3 block scales uint8 [rows, cols/16]; second-level scales fp32 [rows]
+    when per_row, else [1] for the whole matrix)."""
+    bf16 = not (isinstance(values, np.ndarray) and values.dtype != np.uint16)
+    v = _bf16_bits(values) if bf16 else np.ascontiguousarray(values, dtype=np.float32)
+    rows, cols = v.shape
+    q = np.empty((rows, cols // 2), np.uint8)
+    s = np.empty((rows, cols // 16), np.uint8)
+    g = np.empty(rows if per_row else 1, np.float32)
+    fn = _load().oracle_nvfp4_quantize_bf16 if bf16 else _load().oracle_nvfp4_quantize
+    _check(fn(_ptr(v), rows, cols, 1 if per_row else 0, _ptr(q), _ptr(s), _ptr(g)), "nvfp4_quantize")
+    return q, s, g
+
+
+def nvfp4_dequantize(q, s, g, per_row: bool = True) -> np.ndarray:
+    """float64 [rows, cols] values of NVFP4 codes, block scales and second-level scales."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    s = np.ascontiguousarray(s, dtype=np.uint8)
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    rows, half = q.shape
+    out = np.empty((rows, 2 * half), np.float64)
+    _check(_load().oracle_nvfp4_dequantize(_ptr(q), _ptr(s), _ptr(g), rows, 2 * half, 1 if per_row else 0,
+                                           _ptr(out)), "nvfp4_dequantize")
+    return out
+
+
+def quantize_weights_nvfp4(w_gate, w_up, w_down):
+    """NVFP4 expert weights with one second-level scale per expert matrix: W1[e] = the gate
+    rows then the up rows (w_up None: squared-ReLU experts, gate rows only), blocks along
+    H; W_down[e] blocks along F.  Returns (w1_q [E,R1,H/2], w1_s [E,R1,H/16], g1 [E],
+    wd_q [E,H,F/2], wd_s [E,H,F/16], g2 [E])."""
+    import torch  # plain CPU tensor handling only
+
+    gb = _bf16_bits(w_gate)
+    E, F, H = gb.shape
+    w1 = gb if w_up is None else np.concatenate([gb, _bf16_bits(w_up)], axis=1)
+    db = _bf16_bits(w_down)
+    R1 = w1.shape[1]
+    w1_q = np.empty((E, R1, H // 2), np.uint8)
+    w1_s = np.empty((E, R1, H // 16), np.uint8)
+    wd_q = np.empty((E, H, F // 2), np.uint8)
+    wd_s = np.empty((E, H, F // 16), np.uint8)
+    g1 = np.empty(E, np.float32)
+    g2 = np.empty(E, np.float32)
+    for e in range(E):
+        w1_q[e], w1_s[e], g = nvfp4_quantize(np.ascontiguousarray(w1[e]), per_row=False)
+        g1[e] = g[0]
+        wd_q[e], wd_s[e], g = nvfp4_quantize(np.ascontiguousarray(db[e]), per_row=False)
+        g2[e] = g[0]
+    del torch
+    return w1_q, w1_s, g1, wd_q, wd_s, g2
+
+
+def forward_nvfp4(x, ids, probs, wq, tokens=None, want_h=False, probs_in_fc1=False, gate_up_clamp=None,
+                  squared_relu=False):
+    """NVFP4 routed SwiGLU forward (per-token recipe); `wq` = quantize_weights_nvfp4(...).
+
+    Returns out fp32 [ntok, H] and, when want_h, (h codes [ntok,k,F/2], h block scales
+    [ntok,k,F/16], h second-level scales [ntok,k], h pre-quantisation fp32 [ntok,k,F])."""
+    flags, clamp = _variant(probs_in_fc1, gate_up_clamp, squared_relu)
+    xb = _bf16_bits(x)
+    w1_q, w1_s, g1, wd_q, wd_s, g2 = wq
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    probs = np.ascontiguousarray(probs, dtype=np.float32)
+    T, k = ids.shape
+    E, H, half_f = wd_q.shape
+    F = 2 * half_f
+    toks = np.arange(T, dtype=np.int64) if tokens is None else np.ascontiguousarray(tokens, dtype=np.int64)
+    out = np.empty((toks.size, H), np.float32)
+    hq = hs = hg = hf = None
+    if want_h:
+        hq = np.empty((toks.size, k, F // 2), np.uint8)
+        hs = np.empty((toks.size, k, F // 16), np.uint8)
+        hg = np.empty((toks.size, k), np.float32)
+        hf = np.empty((toks.size, k, F), np.float32)
+    _check(_load().oracle_forward_nvfp4(_ptr(xb), _ptr(ids), _ptr(probs), _ptr(w1_q), _ptr(w1_s), _ptr(g1),
+                                        _ptr(wd_q), _ptr(wd_s), _ptr(g2), xb.shape[0], H, F, E, k, _ptr(toks),
+                                        toks.size, _ptr(out), _ptr(hq), _ptr(hs), _ptr(hg), _ptr(hf), flags,
+                                        clamp),
+           "forward_nvfp4")
+    return (out, (hq, hs, hg, hf)) if want_h else out

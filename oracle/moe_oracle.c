@@ -25,6 +25,15 @@
  *                         one E8M0 power-of-two scale per 32 elements along
  *                         K, the OCP MX rule scale = 2^(floor(log2 amax)-8),
  *                         round-to-nearest-even, saturating to +-448.
+ *   oracle_nvfp4_*     -- Megatron-LM PR #7798, "Per-token NVFP4" and
+ *                         "Core metric" (TE's per-token recipe:
+ *                         NVFP4BlockScaling with row-scaled activations, 1-D
+ *                         blocks, no Hadamard transform, no stochastic
+ *                         rounding): E2M1 elements, one E4M3 scale per 16
+ *                         elements along K, and an fp32 second-level scale
+ *                         per activation row (per weight matrix for weights).
+ *                         The pages give the recipe's name, not its formulas;
+ *                         the reading taken is written out at nvfp4_row().
  *   oracle_forward_*   -- Megatron-LM PR #7798, "Background" (activation
  *                         fused into FC1, probabilities applied after FC2)
  *                         and "What is changed" (a token's routes summed as
@@ -191,6 +200,85 @@ static void mxfp8_block(const double* v, int n, uint8_t* q, uint8_t* sbyte) {
     *sbyte = sb;
 }
 
+/* E2M1 (FP4: 1 sign, 2 exponent, 1 mantissa bit, bias 1): code c = 0..7
+ * of a magnitude from the format definition: subnormal 0.5 * m when the
+ * exponent field is 0, else (1 + m / 2) * 2^(e - 1); no infinities, no NaN. */
+static double e2m1_code_value(int code) {
+    int ef = (code >> 1) & 3, mf = code & 1;
+    double mag = ef == 0 ? 0.5 * mf : ldexp(1.0 + 0.5 * mf, ef - 1);
+    return (code & 8) ? -mag : mag;
+}
+
+/* Round a real value onto the E2M1 grid: nearest magnitude, ties to the
+ * code with an even mantissa bit, magnitudes beyond 6 (and NaN) saturate to
+ * 6, the sign is kept (so -tiny -> code 8). */
+static uint8_t e2m1_encode_rne_sat(double v) {
+    int neg = signbit(v) ? 1 : 0;
+    double a = fabs(v);
+    int code;
+    if (!(a < 6.0)) {
+        code = 7;
+    } else {
+        int lo = 0, hi = 7;
+        while (hi - lo > 1) {
+            int mid = (lo + hi) / 2;
+            if (e2m1_code_value(mid) <= a) lo = mid; else hi = mid;
+        }
+        double dlo = a - e2m1_code_value(lo), dhi = e2m1_code_value(hi) - a;
+        if (dlo < dhi) code = lo;
+        else if (dhi < dlo) code = hi;
+        else code = (lo & 1) ? hi : lo; /* tie: even mantissa */
+    }
+    return (uint8_t)(code | (neg << 3));
+}
+
+/* Second-level NVFP4 scale of a row (or matrix) from its largest
+ * magnitude: g = amax / (6 * 448) in fp32, so that the largest block scale
+ * is at most E4M3's 448 and the largest element at most E2M1's 6; an
+ * all-zero (or underflowing) amax gives g = 1. */
+static float nvfp4_global(float amax) {
+    float g = amax / 2688.0f;
+    return (amax > 0.0f && g > 0.0f) ? g : 1.0f;
+}
+
+/* NVFP4 quantisation of n values (n a multiple of 16) under the second-
+ * level scale g.  Per block of 16: s = E4M3((amax_b / g) / 6) (fp32
+ * divisions in that order, the E4M3 rounding to nearest-even and
+ * saturating); the block's divisor d = value(s) * g (fp32); each element
+ * v -> E2M1(v / d) (fp32 division, then the E2M1 rounding), or the signed
+ * zero code when d is 0.  Codes are packed two per byte, element 2i in the
+ * low nibble.  Dequantised: value(code) * value(s) * g. */
+static void nvfp4_row(const float* v, int n, float g, uint8_t* q, uint8_t* s) {
+    for (int b = 0; b < n / 16; ++b) {
+        float amax = 0.0f;
+        for (int i = 0; i < 16; ++i) {
+            float a = fabsf(v[b * 16 + i]);
+            if (a > amax) amax = a;
+        }
+        float sf = (amax / g) / 6.0f;
+        uint8_t sb = e4m3_encode_rne_sat((double)sf);
+        float d = (float)g_e4m3_all[sb] * g;
+        s[b] = sb;
+        for (int i = 0; i < 16; i += 2) {
+            uint8_t c[2];
+            for (int h = 0; h < 2; ++h) {
+                float x = v[b * 16 + i + h];
+                c[h] = d != 0.0f ? e2m1_encode_rne_sat((double)(x / d)) : (uint8_t)(signbit(x) ? 8 : 0);
+            }
+            q[(b * 16 + i) / 2] = (uint8_t)(c[0] | (c[1] << 4));
+        }
+    }
+}
+
+static float row_amax(const float* v, int64_t n) {
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float a = fabsf(v[i]);
+        if (a > amax) amax = a;
+    }
+    return amax;
+}
+
 /* ------------------------------------------------------------------ */
 /* Public entry points (called through ctypes by the tests)           */
 /* ------------------------------------------------------------------ */
@@ -252,6 +340,51 @@ int oracle_mxfp8_dequantize(const uint8_t* q, const uint8_t* s, int64_t rows, in
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t c = 0; c < cols; ++c)
             out[r * cols + c] = (float)(g_e4m3_all[q[r * cols + c]] * g_pow2[s[r * nb + c / 32]]);
+    return ORACLE_OK;
+}
+
+/* NVFP4 quantisation of a row-major fp32 matrix [rows, cols] (cols a
+ * multiple of 16): codes [rows, cols/2], E4M3 block scales [rows, cols/16]
+ * and the second-level scale: per row (per_row = 1, g_out[rows]) or one for
+ * the whole matrix (per_row = 0, g_out[1]). */
+int oracle_nvfp4_quantize(const float* in, int64_t rows, int64_t cols, int per_row,
+                          uint8_t* q, uint8_t* s, float* g_out) {
+    if (!in || !q || !s || !g_out || rows < 0 || cols <= 0 || (cols % 16)) return ORACLE_EINVAL;
+    build_tables();
+    float g_all = per_row ? 0.0f : nvfp4_global(row_amax(in, rows * cols));
+    if (!per_row) g_out[0] = g_all;
+    for (int64_t r = 0; r < rows; ++r) {
+        float g = per_row ? nvfp4_global(row_amax(in + r * cols, cols)) : g_all;
+        if (per_row) g_out[r] = g;
+        nvfp4_row(in + r * cols, (int)cols, g, q + r * (cols / 2), s + r * (cols / 16));
+    }
+    return ORACLE_OK;
+}
+
+/* Same, for a matrix given as bf16 bit patterns. */
+int oracle_nvfp4_quantize_bf16(const uint16_t* in, int64_t rows, int64_t cols, int per_row,
+                               uint8_t* q, uint8_t* s, float* g_out) {
+    if (!in || rows < 0 || cols <= 0) return ORACLE_EINVAL;
+    float* f = (float*)malloc(sizeof(float) * (size_t)(rows * cols > 0 ? rows * cols : 1));
+    if (!f) return ORACLE_ENOMEM;
+    for (int64_t i = 0; i < rows * cols; ++i) f[i] = bf16_bits_to_float(in[i]);
+    int rc = oracle_nvfp4_quantize(f, rows, cols, per_row, q, s, g_out);
+    free(f);
+    return rc;
+}
+
+/* Dequantise: out[r,c] = value(code) * value(s[r,c/16]) * g, in double
+ * (exact: at most 2 + 4 + 24 significant bits). */
+int oracle_nvfp4_dequantize(const uint8_t* q, const uint8_t* s, const float* g, int64_t rows, int64_t cols,
+                            int per_row, double* out) {
+    if (!q || !s || !g || !out || rows < 0 || cols <= 0 || (cols % 16)) return ORACLE_EINVAL;
+    build_tables();
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            int code = (q[r * (cols / 2) + c / 2] >> ((c & 1) * 4)) & 15;
+            out[r * cols + c] = e2m1_code_value(code) * g_e4m3_all[s[r * (cols / 16) + c / 16]] *
+                                (double)g[per_row ? r : 0];
+        }
     return ORACLE_OK;
 }
 
@@ -533,6 +666,103 @@ int oracle_forward_mxfp8(const uint16_t* x, const int32_t* ids, const float* pro
             }
         }
         free(xv); free(xd); free(hv); free(hd); free(qb);
+    }
+    return bad ? ORACLE_EINVAL : ORACLE_OK;
+}
+
+/* NVFP4 forward for a list of tokens (the per-token recipe above).  The
+ * weights arrive quantised, as oracle_nvfp4_quantize makes them from the
+ * bf16 weights with one second-level scale per expert matrix:
+ *   w1_q [E, 2F, H/2], w1_s [E, 2F, H/16], g1 [E]: rows 0..F-1 the gate
+ *       projection, F..2F-1 the up projection (one matrix, one scale);
+ *       squared-ReLU experts (flags) have only the F gate rows;
+ *   wd_q [E, H, F/2],  wd_s [E, H, F/16],  g2 [E].
+ * x rows are quantised here from their bf16 values with a scale per token.
+ * The GEMMs use the dequantised operands exactly; h is formed as in the
+ * bf16 path up to its fp32 value, then quantised with a scale per route row
+ * (blocks of 16 along F), and the dequantised h enters the down GEMM.
+ *   h_q_out [ntok, k, F/2], h_s_out [ntok, k, F/16], h_g_out [ntok, k] and
+ *   h_f32_out [ntok, k, F] (each nullable). */
+int oracle_forward_nvfp4(const uint16_t* x, const int32_t* ids, const float* probs,
+                         const uint8_t* w1_q, const uint8_t* w1_s, const float* g1,
+                         const uint8_t* wd_q, const uint8_t* wd_s, const float* g2,
+                         int64_t T, int H, int F, int E, int k,
+                         const int64_t* toks, int64_t ntok, float* out,
+                         uint8_t* h_q_out, uint8_t* h_s_out, float* h_g_out, float* h_f32_out, int flags,
+                         double clamp) {
+    const int relu2 = (flags & ORACLE_SQUARED_RELU) != 0;
+    const int R1 = relu2 ? F : 2 * F;
+    if (!x || !ids || !probs || !w1_q || !w1_s || !g1 || !wd_q || !wd_s || !g2 || !toks || !out)
+        return ORACLE_EINVAL;
+    if (H <= 0 || F <= 0 || (H % 16) || (F % 16) || E <= 0 || k <= 0 || k > 64 || ntok < 0)
+        return ORACLE_EINVAL;
+    build_tables();
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t i = 0; i < ntok; ++i) {
+        int64_t t = toks[i];
+        if (t < 0 || t >= T) { bad = 1; continue; }
+        float* xf = (float*)malloc(sizeof(float) * (size_t)H);
+        double* xd = (double*)malloc(sizeof(double) * (size_t)H);
+        float* hf = (float*)malloc(sizeof(float) * (size_t)F);
+        double* hd = (double*)malloc(sizeof(double) * (size_t)F);
+        uint8_t* qb = (uint8_t*)malloc((size_t)(H > F ? H : F));
+        uint8_t* sb = (uint8_t*)malloc((size_t)(H > F ? H : F) / 16);
+        float* acc = out + i * H;
+        int sid[64];
+        float sp[64];
+        if (!xf || !xd || !hf || !hd || !qb || !sb) {
+            free(xf); free(xd); free(hf); free(hd); free(qb); free(sb);
+            bad = 1;
+            continue;
+        }
+        /* x: bf16 -> NVFP4 with this token's scale -> dequantised values */
+        for (int c = 0; c < H; ++c) xf[c] = bf16_bits_to_float(x[t * H + c]);
+        float gx = nvfp4_global(row_amax(xf, H));
+        nvfp4_row(xf, H, gx, qb, sb);
+        for (int c = 0; c < H; ++c)
+            xd[c] = e2m1_code_value((qb[c / 2] >> ((c & 1) * 4)) & 15) * g_e4m3_all[sb[c / 16]] * (double)gx;
+        for (int c = 0; c < H; ++c) acc[c] = 0.0f;
+        sort_routes(ids + t * k, probs + t * k, k, sid, sp);
+        for (int j = 0; j < k; ++j) {
+            int e = sid[j];
+            if (e < 0 || e >= E) { bad = 1; break; }
+            const uint8_t* q1 = w1_q + (int64_t)e * R1 * (H / 2);
+            const uint8_t* s1 = w1_s + (int64_t)e * R1 * (H / 16);
+            const uint8_t* q2 = wd_q + (int64_t)e * H * (F / 2);
+            const uint8_t* s2 = wd_s + (int64_t)e * H * (F / 16);
+            for (int f = 0; f < F; ++f) {
+                double gsum = 0.0, usum = 0.0;
+                for (int c = 0; c < H; ++c) {
+                    int64_t rg = f, ru = F + f;
+                    double wg = e2m1_code_value((q1[rg * (H / 2) + c / 2] >> ((c & 1) * 4)) & 15) *
+                                g_e4m3_all[s1[rg * (H / 16) + c / 16]] * (double)g1[e];
+                    gsum += wg * xd[c];
+                    if (!relu2) {
+                        double wu = e2m1_code_value((q1[ru * (H / 2) + c / 2] >> ((c & 1) * 4)) & 15) *
+                                    g_e4m3_all[s1[ru * (H / 16) + c / 16]] * (double)g1[e];
+                        usum += wu * xd[c];
+                    }
+                }
+                hf[f] = swiglu_value(gsum, usum, clamp, flags, sp[j]);
+                if (h_f32_out) h_f32_out[(i * k + j) * F + f] = hf[f];
+            }
+            float gh = nvfp4_global(row_amax(hf, F));
+            nvfp4_row(hf, F, gh, qb, sb);
+            for (int f = 0; f < F; ++f)
+                hd[f] = e2m1_code_value((qb[f / 2] >> ((f & 1) * 4)) & 15) * g_e4m3_all[sb[f / 16]] * (double)gh;
+            if (h_q_out) memcpy(h_q_out + (i * k + j) * (F / 2), qb, (size_t)(F / 2));
+            if (h_s_out) memcpy(h_s_out + (i * k + j) * (F / 16), sb, (size_t)(F / 16));
+            if (h_g_out) h_g_out[i * k + j] = gh;
+            for (int c = 0; c < H; ++c) {
+                double y = 0.0;
+                for (int f = 0; f < F; ++f)
+                    y += e2m1_code_value((q2[(int64_t)c * (F / 2) + f / 2] >> ((f & 1) * 4)) & 15) *
+                         g_e4m3_all[s2[(int64_t)c * (F / 16) + f / 16]] * (double)g2[e] * hd[f];
+                acc[c] = (flags & ORACLE_PROBS_IN_FC1) ? acc[c] + (float)y : fmaf(sp[j], (float)y, acc[c]);
+            }
+        }
+        free(xf); free(xd); free(hf); free(hd); free(qb); free(sb);
     }
     return bad ? ORACLE_EINVAL : ORACLE_OK;
 }

@@ -19,6 +19,12 @@ Which plausible mistake each pin catches:
              in ascending expert id (checked against exact rational
              arithmetic); token order and duplication invariance;
              MXFP8 E=1 dense check with the independent quantiser.
+  nvfp4      a worked row fixes the E2M1 grid, every tie, saturation and the
+             sign of zero; random rows over many binades (fp32 and bf16,
+             scale per row and per matrix) equal an independent quantiser
+             (numpy fp32 divisions, torch's E4M3 cast, E2M1 by distance to
+             all eight values); closed forms: g = amax / 2688, all-zero rows,
+             power-of-two invariance, the error bound; E=1 dense check.
 """
 from __future__ import annotations
 
@@ -574,3 +580,173 @@ def test_squared_relu_mxfp8_single_expert_is_dense_relu2_mlp():
     rms = float(np.sqrt(np.mean(ref.astype(np.float64) ** 2)))
     assert np.max(np.abs(out - ref)) <= 5e-2 * rms
     assert np.mean(np.abs(out - ref)) <= 2e-3 * np.mean(np.abs(ref))
+
+
+# ---------------------------------------------------------------- nvfp4 (per-token recipe)
+
+E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def indep_e2m1(x64: np.ndarray) -> np.ndarray:
+    """E2M1 codes by distance to all eight magnitudes, ties to the even code."""
+    d = np.abs(np.abs(x64)[..., None] - E2M1_GRID) + 1e-12 * (np.arange(8) & 1)
+    return (np.argmin(d, axis=-1) | (np.signbit(x64).astype(np.int64) << 3)).astype(np.uint8)
+
+
+def indep_nvfp4(v, per_row=True):
+    """Independent NVFP4 quantiser of fp32 rows [rows, cols]: numpy float32
+    arithmetic for the scales and quotients, torch's float8_e4m3fn cast for
+    the block scales.  Returns packed codes, scale bytes, second-level scales."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    rows, cols = v.shape
+    amax = np.abs(v).max(axis=1) if per_row else np.full(rows, np.abs(v).max(), np.float32)
+    with np.errstate(divide="ignore", invalid="ignore", under="ignore"):
+        g = (amax / np.float32(2688.0)).astype(np.float32)
+        g = np.where((amax > 0) & (g > 0), g, np.float32(1.0)).astype(np.float32)
+        blocks = v.reshape(rows, cols // 16, 16)
+        amax_b = np.abs(blocks).max(axis=2)
+        sf = ((amax_b / g[:, None]).astype(np.float32) / np.float32(6.0)).astype(np.float32)
+        sbytes = torch.from_numpy(np.minimum(sf, np.float32(448.0))).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        sval = torch_e4m3_table()[sbytes].astype(np.float32)
+        d = (sval * g[:, None]).astype(np.float32)
+        quot = (blocks / d[:, :, None]).astype(np.float32)
+    codes = np.where(d[:, :, None] != 0, indep_e2m1(quot.astype(np.float64)),
+                     (np.signbit(blocks).astype(np.uint8) << 3)).reshape(rows, cols).astype(np.uint8)
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    return packed, sbytes.astype(np.uint8), (g if per_row else g[:1])
+
+
+def indep_nvfp4_dequant(q, s, g, per_row=True) -> np.ndarray:
+    rows, half = q.shape
+    codes = np.empty((rows, 2 * half), np.int64)
+    codes[:, 0::2] = q & 15
+    codes[:, 1::2] = q >> 4
+    mag = E2M1_GRID[codes & 7] * np.where(codes & 8, -1.0, 1.0)
+    gg = g.astype(np.float64) if per_row else np.full(rows, float(g[0]))
+    return (mag.reshape(rows, -1, 16) * torch_e4m3_table()[s][:, :, None] * gg[:, None, None]).reshape(rows, -1)
+
+
+def test_nvfp4_grid_ties_saturation_and_sign():
+    # amax 2688 fixes g = 1; a block with amax 6 has scale 1.0 (E4M3 0x38), so its codes are E2M1(v)
+    row = np.zeros((1, 48), np.float32)
+    row[0, 0] = 2688.0
+    row[0, 16:32] = [0, 0.25, 0.5, 0.75, 1, 1.25, 1.5, 1.75, 2, 2.5, 3, 3.5, 4, 5, 6, -0.1]
+    row[0, 32:48] = [6, -6, 0.2499, 0.2501, 5.01, -4.99, 2.51, -2.49, 0, 0, 0, 0, 0, 0, 0, -0.0]
+    q, s, g = oracle.nvfp4_quantize(row)
+    assert g[0] == 1.0 and s[0, 0] == 0x7E and s[0, 1] == 0x38 and s[0, 2] == 0x38
+    codes = np.empty(48, np.int64)
+    codes[0::2], codes[1::2] = q[0] & 15, q[0] >> 4
+    # ties to even: 0.25 -> 0, 0.75 -> 1, 1.25 -> 1, 1.75 -> 2, 2.5 -> 2, 3.5 -> 4, 5 -> 4; -0.1 -> -0
+    assert list(codes[16:32]) == [0, 0, 1, 2, 2, 2, 3, 4, 4, 4, 5, 6, 6, 6, 7, 8]
+    assert list(codes[32:40]) == [7, 15, 0, 1, 7, 14, 5, 12]
+    assert codes[47] == 8 and codes[0] == 7  # -0.0 keeps its sign; 2688 / 448 = 6
+    # beyond 6 saturates: a block whose scale is capped at 448 by the row's g
+    row = np.zeros((1, 16), np.float32)
+    row[0, :2] = [2688.0, -2688.0]
+    q, s, g = oracle.nvfp4_quantize(row)
+    assert (q[0, 0] & 15) == 7 and (q[0, 0] >> 4) == 15
+
+
+@pytest.mark.parametrize("per_row", [True, False])
+def test_nvfp4_matches_independent_quantiser(per_row):
+    gen = np.random.default_rng(17)
+    rows = []
+    for mag in (1e-30, 1e-6, 1e-2, 1.0, 37.0, 1e4, 1e30):
+        rows.append(gen.standard_normal((6, 64)) * mag)
+    v = np.concatenate(rows).astype(np.float32)
+    v[3, 5:21] = 0.0          # a whole block of zeros next to live ones
+    v[10] = 0.0               # an all-zero row
+    v[20, ::7] *= 1000.0      # a few outliers
+    q, s, g = oracle.nvfp4_quantize(v, per_row=per_row)
+    q2, s2, g2 = indep_nvfp4(v, per_row=per_row)
+    assert np.array_equal(g, g2) and np.array_equal(s, s2) and np.array_equal(q, q2)
+    # bf16 entry equals the fp32 entry on the same values
+    xb = torch.from_numpy(v).to(torch.bfloat16)
+    qa, sa, ga = oracle.nvfp4_quantize(xb, per_row=per_row)
+    qb, sb, gb = oracle.nvfp4_quantize(xb.float().numpy(), per_row=per_row)
+    assert np.array_equal(qa, qb) and np.array_equal(sa, sb) and np.array_equal(ga, gb)
+    assert np.array_equal(oracle.nvfp4_dequantize(q, s, g, per_row), indep_nvfp4_dequant(q2, s2, g2, per_row))
+
+
+def test_nvfp4_closed_forms():
+    gen = np.random.default_rng(5)
+    v = gen.standard_normal((8, 128)).astype(np.float32)
+    q, s, g = oracle.nvfp4_quantize(v)
+    amax = np.abs(v).max(axis=1)
+    assert np.array_equal(g, (amax / np.float32(2688.0)).astype(np.float32))
+    # all-zero row: g = 1, scale bytes 0, codes 0
+    qz, sz, gz = oracle.nvfp4_quantize(np.zeros((1, 32), np.float32))
+    assert gz[0] == 1.0 and np.all(sz == 0) and np.all(qz == 0)
+    # scaling a row by 2^j scales g by 2^j exactly and leaves codes and block scales unchanged
+    for j in (-20, -3, 5, 40):
+        qj, sj, gj = oracle.nvfp4_quantize(v * np.float32(2.0 ** j))
+        assert np.array_equal(qj, q) and np.array_equal(sj, s) and np.array_equal(gj, g * np.float32(2.0 ** j))
+    # error bound: every element is within one block divisor value(s) * g of its value
+    deq = oracle.nvfp4_dequantize(q, s, g)
+    div = (torch_e4m3_table()[s] * g[:, None].astype(np.float64))
+    assert np.all(np.abs(deq - v).reshape(8, 8, 16) <= div[:, :, None] * (1 + 1e-12))
+    # and the block amax is reproduced within a quarter of itself (E2M1 step at 4..6, E4M3 rounding)
+    amax_b = np.abs(v).reshape(8, 8, 16).max(axis=2)
+    amax_dq = np.abs(deq).reshape(8, 8, 16).max(axis=2)
+    assert np.all(np.abs(amax_dq - amax_b) <= 0.25 * amax_b)
+
+
+def _nvfp4_dense_ref(x, wg, wu, wd):
+    """Independent NVFP4 pipeline for one expert (E=1, k=1, p=1): independent
+    quantisers, float64 matmuls, fp32 h quantised per row."""
+    xq = indep_nvfp4_dequant(*indep_nvfp4(x.float().numpy()))
+    w1 = np.concatenate([wg[0].float().numpy(), wu[0].float().numpy()])
+    w1d = indep_nvfp4_dequant(*indep_nvfp4(w1, per_row=False), per_row=False)
+    wdd = indep_nvfp4_dequant(*indep_nvfp4(wd[0].float().numpy(), per_row=False), per_row=False)
+    F = wg.shape[1]
+    g = xq @ w1d[:F].T
+    u = xq @ w1d[F:].T
+    h32 = (scipy.special.expit(g) * g * u).astype(np.float32)
+    return h32, (indep_nvfp4_dequant(*indep_nvfp4(h32)) @ wdd.T).astype(np.float32)
+
+
+def test_forward_nvfp4_k1_single_expert_is_dense_mlp():
+    gen = torch.Generator().manual_seed(31)
+    T, H, F = 16, 128, 96
+    x = rand_bf16(gen, (T, H))
+    wg = rand_bf16(gen, (1, F, H), H ** -0.5)
+    wu = rand_bf16(gen, (1, F, H), H ** -0.5)
+    wd = rand_bf16(gen, (1, H, F), F ** -0.5)
+    wq = oracle.quantize_weights_nvfp4(wg, wu, wd)
+    ids = np.zeros((T, 1), np.int32)
+    probs = np.ones((T, 1), np.float32)
+    out, (hq, hs, hg, hf) = oracle.forward_nvfp4(x, ids, probs, wq, want_h=True)
+    h32, ref = _nvfp4_dense_ref(x, wg, wu, wd)
+    assert np.mean(h32 != hf[:, 0, :]) < 2e-2  # double-sum order may flip a last fp32 bit
+    q2, s2, g2 = indep_nvfp4(hf[:, 0, :])    # quantiser consistency on the oracle's own h
+    assert np.array_equal(q2, hq[:, 0, :]) and np.array_equal(s2, hs[:, 0, :]) and np.array_equal(g2, hg[:, 0])
+    rms = float(np.sqrt(np.mean(ref.astype(np.float64) ** 2)))
+    assert np.max(np.abs(out - ref)) <= 5e-2 * rms
+    assert np.mean(np.abs(out - ref)) <= 5e-3 * np.mean(np.abs(ref))
+
+
+def test_forward_nvfp4_weight_scales_are_per_expert_matrix():
+    x, wg, wu, wd, ids, probs = _small_problem(33, H=64, F=32, E=3)
+    w1_q, w1_s, g1, wd_q, wd_s, g2 = oracle.quantize_weights_nvfp4(wg, wu, wd)
+    for e in range(3):
+        a1 = max(float(wg[e].float().abs().max()), float(wu[e].float().abs().max()))
+        assert g1[e] == np.float32(np.float32(a1) / np.float32(2688.0))
+        assert g2[e] == np.float32(np.float32(float(wd[e].float().abs().max())) / np.float32(2688.0))
+
+
+def test_forward_nvfp4_zero_gate_gives_zero():
+    x, wg, wu, wd, ids, probs = _small_problem(34, H=64, F=64)
+    out = oracle.forward_nvfp4(x, ids, probs, oracle.quantize_weights_nvfp4(torch.zeros_like(wg), wu, wd))
+    assert np.all(out == 0.0)
+
+
+def test_forward_nvfp4_close_to_bf16():
+    """NVFP4 and bf16 forwards of the same problem differ by some percent: more
+    than MXFP8 (3 bits of element precision instead of 4, scales to 1/16)."""
+    x, wg, wu, wd, ids, probs = _small_problem(35, T=32, H=256, F=128, E=4, k=2)
+    a = oracle.forward_bf16(x, ids, probs, wg, wu, wd).astype(np.float64)
+    b = oracle.forward_nvfp4(x, ids, probs, oracle.quantize_weights_nvfp4(wg, wu, wd)).astype(np.float64)
+    c = oracle.forward_mxfp8(x, ids, probs, oracle.quantize_weights_mxfp8(wg, wu, wd)).astype(np.float64)
+    d4 = np.linalg.norm(b - a) / np.linalg.norm(a)
+    d8 = np.linalg.norm(c - a) / np.linalg.norm(a)
+    assert 0.02 < d4 < 0.3 and d8 < d4
