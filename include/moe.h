@@ -64,7 +64,7 @@ typedef enum {
     MOE_ERR_NOT_PREPARED = 6          /* reserved: weight buffer not prepared    */
 } moe_status;
 
-typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1 } moe_precision;
+typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1, MOE_NVFP4 = 2 } moe_precision;
 
 /* Device status bits (sticky until moe_clear_device_status). */
 #define MOE_DEV_LIVE_CLAMPED 0x1u  /* live count < 0 or > max live rows: clamped    */
@@ -82,7 +82,7 @@ typedef struct {
     long long max_live_rows; /* largest live count a call will pass (<= capacity);
                                 0 means capacity.  The workspace is sized for it;
                                 larger live counts are clamped and flagged.       */
-    moe_precision precision; /* MOE_BF16 or MOE_MXFP8                             */
+    moe_precision precision; /* MOE_BF16, MOE_MXFP8 or MOE_NVFP4                  */
     unsigned flags;          /* MOE_FLAG_* variants; 0 for the plain forward      */
     float gate_up_clamp;     /* > 0: gate and up pre-activations clamped to
                                 [-gate_up_clamp, gate_up_clamp] before SwiGLU
@@ -156,6 +156,24 @@ moe_status moe_prepare_weights(const moe_plan* plan, const void* w_gate, const v
 moe_status mxfp8_quantize_block32(const void* in, long long rows, int cols, long long ld_in,
                                   uint8_t* q, uint8_t* scales, const int* live_rows_dev,
                                   void* stream);
+
+/* NVFP4 quantisation of bf16 rows as the per-token recipe does it ([P2]
+ * "Per-token NVFP4": TE's NVFP4BlockScaling with row-scaled activations,
+ * 1-D blocks, no Hadamard transform, no stochastic rounding).  Per row:
+ *   g = amax(row) / 2688 in fp32 (1 for an all-zero row), row_scales[r];
+ *   per 16 elements: s = E4M3((amax_16 / g) / 6) (fp32 divisions, round to
+ *   nearest even, saturating at 448), scales[r, c/16];
+ *   each element: E2M1(v / (value(s) * g)) (fp32, round to nearest even,
+ *   saturating at 6; signed zero when the divisor is 0), packed two per
+ *   byte with element 2i in the low nibble, q[r, c/2].
+ * The value of an element is E2M1 * value(s) * g.  in bf16 [rows, ld_in];
+ * q uint8 [rows, cols/2], scales uint8 [rows, cols/16], row_scales fp32
+ * [rows], all row-major, device pointers.  live_rows_dev as for
+ * mxfp8_quantize_block32.  cols a positive multiple of 32, ld_in >= cols and
+ * a multiple of 8, `in` 16-byte aligned, q and row_scales 4-byte aligned. */
+moe_status nvfp4_quantize_block16(const void* in, long long rows, int cols, long long ld_in,
+                                  uint8_t* q, uint8_t* scales, float* row_scales,
+                                  const int* live_rows_dev, void* stream);
 
 /* Router ([P4] `_route`): for each live row t of logits (fp32 [capacity, E]),
  * softmax over the E experts, the k largest (ties: lower expert id), the k
@@ -242,18 +260,27 @@ moe_status moe_forward_with_events(const moe_plan* plan, const void* x, const fl
  *   perm    int32 [routes]: permuted row r holds route t*k + j
  *   inv     int32 [max_live, k]: padded intermediate row of route (t, j)
  *   pad_offsets int32 [E+1]: first padded intermediate row of each expert,
- *           a multiple of 32 (bf16) or 128 (MXFP8)
+ *           a multiple of 32 (bf16) or 128 (MXFP8, NVFP4)
  *   h       intermediate rows [rows_padded, ceil(F/128)*128], bf16 or
  *           E4M3 codes, the columns past F zero
  *   xq      permuted x rows [rows_padded, ceil(H/128)*128], bf16 or E4M3
  *           codes, the columns past H zero; bf16 writes only the rows of
  *           route tiles of more than 32 routes (the gate/up GEMM reads the
  *           x rows of smaller tiles in place)
- *   h_scales, xq_scales  MXFP8 only (else NULL): E8M0 bytes in blocks of
- *           512 bytes, one per (128-row tile, K stage of 128 elements),
- *           block index tile * ceil(K/128) + stage; inside a block the byte
- *           of (row r of the tile, 32-element group g of the stage) is at
- *           (r % 32) * 16 + (r / 32) * 4 + g.  K = F for h, H for x. */
+ *   h_scales, xq_scales  MXFP8 and NVFP4 (else NULL).  MXFP8: E8M0 bytes
+ *           in blocks of 512 bytes, one per (128-row tile, K stage of 128
+ *           elements), block index tile * ceil(K/128) + stage; inside a block
+ *           the byte of (row r of the tile, 32-element group g of the stage)
+ *           is at (r % 32) * 16 + (r / 32) * 4 + g.  K = F for h, H for x.
+ *           NVFP4: E4M3 bytes, four 512-byte blocks per (128-row tile, K
+ *           block of 256 elements), block index (tile * ceil(K/256) + K
+ *           block) * 4 + (64-element step within it); inside a block the
+ *           byte of (row r, 16-element block b of the step) is at
+ *           (r % 32) * 16 + (r / 32) * 4 + b.  NVFP4 h and xq are codes two
+ *           per byte ([rows_padded, ceil(K/256)*128] bytes).
+ *   xq_row_scales, h_row_scales  NVFP4 only: fp32 second-level scale per
+ *           padded row;  h_fp32  NVFP4 only: the gate/up GEMM's fp32 h rows
+ *           [rows_padded, ceil(F/256)*256] before quantisation. */
 typedef struct {
     const int* route_ids;
     const float* route_probs;
@@ -267,6 +294,9 @@ typedef struct {
     const uint8_t* xq_scales;
     long long rows_padded; /* rows of the padded intermediate buffers */
     const unsigned* status; /* device status word */
+    const float* xq_row_scales;
+    const float* h_row_scales;
+    const float* h_fp32;
 } moe_workspace_views;
 moe_status moe_get_workspace_views(const moe_plan* plan, const void* workspace,
                                    moe_workspace_views* views);

@@ -25,7 +25,7 @@ import os
 __all__ = [
     "MoeError", "Plan", "load_library", "library_path", "moe_version", "moe_plan_create", "moe_plan_destroy",
     "moe_weight_buffer_bytes", "moe_workspace_bytes", "alloc_weight_buffer", "alloc_workspace",
-    "moe_prepare_weights", "mxfp8_quantize_block32", "moe_route_topk", "moe_forward", "moe_forward_with_events",
+    "moe_prepare_weights", "mxfp8_quantize_block32", "nvfp4_quantize_block16", "moe_route_topk", "moe_forward", "moe_forward_with_events",
     "moe_forward_noalloc", "MOE_NOALLOC_SCRATCH_BYTES",
     "MOE_NUM_STAGES", "STAGE_NAMES",
     "moe_get_workspace_views", "moe_get_device_status", "moe_clear_device_status",
@@ -43,7 +43,7 @@ MOE_DEV_TIMEOUT = 0x4
 MOE_FLAG_PROBS_IN_FC1 = 0x1
 MOE_FLAG_OUT_BF16 = 0x2
 MOE_FLAG_SQUARED_RELU = 0x4
-_PRECISION = {"bf16": 0, "mxfp8": 1}
+_PRECISION = {"bf16": 0, "mxfp8": 1, "nvfp4": 2}
 
 
 class MoeError(RuntimeError):
@@ -61,7 +61,8 @@ class _Desc(ctypes.Structure):
 class _Views(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("route_ids", "route_probs", "offsets", "perm", "inv", "pad_offsets",
                                                  "h", "h_scales", "xq", "xq_scales")] + [
-        ("rows_padded", ctypes.c_longlong), ("status", ctypes.c_void_p)]
+        ("rows_padded", ctypes.c_longlong), ("status", ctypes.c_void_p), ("xq_row_scales", ctypes.c_void_p),
+        ("h_row_scales", ctypes.c_void_p), ("h_fp32", ctypes.c_void_p)]
 
 
 _lib = None
@@ -85,6 +86,7 @@ def load_library():
         "moe_workspace_bytes": ([P], SZ),
         "moe_prepare_weights": ([P, P, P, P, P, SZ, P], I),
         "mxfp8_quantize_block32": ([P, LL, I, LL, P, P, P, P], I),
+        "nvfp4_quantize_block16": ([P, LL, I, LL, P, P, P, P, P], I),
         "moe_route_topk": ([P, P, P, P, P, P], I),
         "moe_forward": ([P, P, P, P, P, P, P, P, P, SZ, P], I),
         "moe_forward_with_events": ([P, P, P, P, P, P, P, P, P, SZ, P, ctypes.POINTER(P)], I),
@@ -228,6 +230,15 @@ def mxfp8_quantize_block32(x, q, scales, live_rows=None, stream=None) -> None:
     rows, cols = x.shape
     _check(load_library().mxfp8_quantize_block32(_ptr(x), rows, cols, x.stride(0), _ptr(q), _ptr(scales),
                                                  _ptr(live_rows), _stream(stream)), "mxfp8_quantize_block32")
+
+
+def nvfp4_quantize_block16(x, q, scales, row_scales, live_rows=None, stream=None) -> None:
+    """x bf16 [rows, cols] (row stride in elements a multiple of 8) -> q uint8 [rows, cols/2],
+    scales uint8 [rows, cols/16], row_scales fp32 [rows] (the per-token NVFP4 recipe)."""
+    rows, cols = x.shape
+    _check(load_library().nvfp4_quantize_block16(_ptr(x), rows, cols, x.stride(0), _ptr(q), _ptr(scales),
+                                                 _ptr(row_scales), _ptr(live_rows), _stream(stream)),
+           "nvfp4_quantize_block16")
 
 
 def moe_route_topk(plan: Plan, logits, live_count, ids, probs, stream=None) -> None:

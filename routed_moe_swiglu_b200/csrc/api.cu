@@ -87,8 +87,19 @@ static void compute_layouts(moe_plan* p) {
     w.perm = take(L * k * 4);
     w.inv = take(L * k * 4);
     const size_t mtiles = (size_t)p->max_m_tiles;
-    w.ready = fp8 ? 0 : take(mtiles * 4);
-    if (fp8) {
+    const bool fp4 = p->d.precision == MOE_NVFP4;
+    w.ready = fp8 || fp4 ? 0 : take(mtiles * 4);
+    w.xg = w.hf = w.hg = 0;
+    if (fp4) {
+        // codes two per byte; four 512-byte scale blocks per 128-row tile and K block of 256
+        w.xq = take(R * (size_t)p->hp / 2);
+        w.xs = take(mtiles * p->ks1 * 4 * kSfBlock);
+        w.xg = take(R * 4);
+        w.hf = take(R * (size_t)p->fp * 4);
+        w.h = take(R * (size_t)p->fp / 2);
+        w.hs = take(mtiles * p->ks2 * 4 * kSfBlock);
+        w.hg = take(R * 4);
+    } else if (fp8) {
         w.xq = take(R * (size_t)p->hp);
         w.xs = take(mtiles * p->ks1 * kSfBlock);
         w.h = take(R * (size_t)p->fp);
@@ -104,7 +115,14 @@ static void compute_layouts(moe_plan* p) {
 
     WbufLayout& b = p->wb;
     off = 0;
-    if (fp8) {
+    b.wg = 0;
+    if (fp4) {
+        b.w1 = take(E * (size_t)p->w1r * (size_t)p->hp / 2);
+        b.w1s = take(E * p->nt1 * p->ks1 * 4 * kSfBlock);
+        b.w2 = take(E * H * (size_t)p->fp / 2);
+        b.w2s = take(E * p->nt2 * p->ks2 * 4 * kSfBlock);
+        b.wg = take(E * 2 * 4);
+    } else if (fp8) {
         b.w1 = take(E * (size_t)p->w1r * (size_t)p->hp);
         b.w1s = take(E * p->nt1 * p->ks1 * kSfBlock);
         b.w2 = take(E * H * (size_t)p->fp);
@@ -145,10 +163,11 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     if (desc == nullptr || plan_out == nullptr) return MOE_ERR_INVALID_ARG;
     *plan_out = nullptr;
     const moe_desc& d = *desc;
-    if (d.precision != MOE_BF16 && d.precision != MOE_MXFP8) return MOE_ERR_INVALID_ARG;
+    if (d.precision != MOE_BF16 && d.precision != MOE_MXFP8 && d.precision != MOE_NVFP4) return MOE_ERR_INVALID_ARG;
+    const bool blockscaled = d.precision != MOE_BF16;  // MXFP8 or NVFP4: one CTA, 128-row tiles
     if (d.hidden <= 0 || d.ffn <= 0 || d.num_experts <= 0 || d.top_k <= 0 || d.capacity <= 0)
         return MOE_ERR_UNSUPPORTED;
-    const int mult = d.precision == MOE_MXFP8 ? 32 : 8;
+    const int mult = blockscaled ? 32 : 8;
     if (d.hidden % mult != 0 || d.ffn % mult != 0) return MOE_ERR_UNSUPPORTED;
     if (d.hidden > 16384 || d.ffn > 16384) return MOE_ERR_UNSUPPORTED;
     if (d.num_experts > kMaxExperts || d.top_k > kMaxTopK || d.top_k > d.num_experts) return MOE_ERR_UNSUPPORTED;
@@ -163,25 +182,27 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     p->max_live = d.max_live_rows > 0 ? d.max_live_rows : d.capacity;
     p->d.max_live_rows = p->max_live;
     p->max_routes = p->max_live * d.top_k;
-    p->tile_rows = d.precision == MOE_MXFP8 ? kBM : kRouteTile;
-    p->row_align = d.precision == MOE_MXFP8 ? kBM : kRouteAlign;
+    p->tile_rows = blockscaled ? kBM : kRouteTile;
+    p->row_align = blockscaled ? kBM : kRouteAlign;
     p->max_m_tiles = (p->max_routes + p->tile_rows - 1) / p->tile_rows + d.num_experts;
     // every expert's rows are padded to row_align: at most routes + E * row_align rows
-    p->rows_pad = d.precision == MOE_MXFP8 ? p->max_m_tiles * p->tile_rows
+    p->rows_pad = blockscaled ? p->max_m_tiles * p->tile_rows
                                            : p->max_routes + (long long)d.num_experts * p->row_align;
     p->nblk = (int)((p->max_live + kTokPerBlk - 1) / kTokPerBlk);
     // K in blocks of 128 elements (bf16: the GEMMs' K stage; MXFP8: the unit of the scale
     // blocks, two per K stage); K pitches padded to whole blocks with zeros
-    p->ks1 = (d.hidden + 127) / 128;
-    p->ks2 = (d.ffn + 127) / 128;
-    p->hp = (long long)p->ks1 * 128;
-    p->fp = (long long)p->ks2 * 128;
+    // (NVFP4: K blocks of 256 elements, which are 128 bytes of codes as in MXFP8)
+    const int kblk = d.precision == MOE_NVFP4 ? 256 : 128;
+    p->ks1 = (d.hidden + kblk - 1) / kblk;
+    p->ks2 = (d.ffn + kblk - 1) / kblk;
+    p->hp = (long long)p->ks1 * kblk;
+    p->fp = (long long)p->ks2 * kblk;
     p->hr = p->hp;
     // FC1 rows per expert: gate and up interleaved (2 fp), or one projection (squared-ReLU
     // experts), padded to whole weight tiles (bf16: pair tiles of 256 rows; MXFP8: 128)
     const bool relu2 = (d.flags & MOE_FLAG_SQUARED_RELU) != 0;
-    p->w1r = !relu2 ? 2 * p->fp : (d.precision == MOE_MXFP8 ? p->fp : (p->fp + 255) / 256 * 256);
-    if (d.precision == MOE_MXFP8) {
+    p->w1r = !relu2 ? 2 * p->fp : (blockscaled ? p->fp : (p->fp + 255) / 256 * 256);
+    if (blockscaled) {
         p->nt1 = (int)(p->w1r / 128);  // weight tiles of 128 rows; h's padding columns come out zero
         p->nt2 = (d.hidden + kG2BN8 - 1) / kG2BN8;
     } else {
@@ -218,8 +239,9 @@ moe_status moe_prepare_weights(const moe_plan* plan, const void* w_gate, const v
     const auto* g = static_cast<const __nv_bfloat16*>(w_gate);
     const auto* u = static_cast<const __nv_bfloat16*>(w_up);
     const auto* dn = static_cast<const __nv_bfloat16*>(w_down);
-    const cudaError_t e = plan->d.precision == MOE_MXFP8 ? launch_prepare_mxfp8(plan, g, u, dn, kernel_buf, s)
-                                                          : launch_prepare_bf16(plan, g, u, dn, kernel_buf, s);
+    const cudaError_t e = plan->d.precision == MOE_MXFP8   ? launch_prepare_mxfp8(plan, g, u, dn, kernel_buf, s)
+                          : plan->d.precision == MOE_NVFP4 ? launch_prepare_nvfp4(plan, g, u, dn, kernel_buf, s)
+                                                           : launch_prepare_bf16(plan, g, u, dn, kernel_buf, s);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -232,6 +254,19 @@ moe_status mxfp8_quantize_block32(const void* in, long long rows, int cols, long
     if (rows == 0) return MOE_OK;
     const cudaError_t e = launch_quantize_rows(static_cast<const __nv_bfloat16*>(in), rows, cols, ld_in, q, scales,
                                                live_rows_dev, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status nvfp4_quantize_block16(const void* in, long long rows, int cols, long long ld_in, uint8_t* q,
+                                  uint8_t* scales, float* row_scales, const int* live_rows_dev, void* stream) {
+    if (in == nullptr || q == nullptr || scales == nullptr || row_scales == nullptr) return MOE_ERR_INVALID_ARG;
+    if (rows < 0 || cols <= 0 || ld_in < cols) return MOE_ERR_INVALID_ARG;
+    if (cols % 32 != 0) return MOE_ERR_UNSUPPORTED;
+    if (ld_in % 8 != 0 || !aligned(in, 16) || !aligned(q, 4) || !aligned(row_scales, 4)) return MOE_ERR_ALIGNMENT;
+    if (rows == 0) return MOE_OK;
+    const cudaError_t e = launch_nvfp4_quantize_rows(static_cast<const __nv_bfloat16*>(in), rows, cols, ld_in, q,
+                                                     scales, row_scales, live_rows_dev,
+                                                     static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -283,18 +318,21 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
 
     // TMA descriptors for this call's buffers (host-side encoding only)
     const bool fp8 = plan->d.precision == MOE_MXFP8;
+    const bool fp4 = plan->d.precision == MOE_NVFP4;
     const unsigned long long R = (unsigned long long)plan->rows_pad;
     const unsigned long long uH = (unsigned long long)H, uE = (unsigned long long)E;
-    const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const CUtensorMapDataType dt = fp8 || fp4 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     CUtensorMap tA1, tA2;  // weight operands
     BoxMaps8 rB1, rB2;     // route-row operands (x rows, h rows)
     CUtensorMap tX;        // bf16: x rows, gathered by token
-    if (fp8) {
-        // MXFP8 (one CTA per tile): K stage = 256 E4M3 elements = two 128-byte swizzle atoms;
-        // the maps address element k of a row as (k % 128, row, k / 128), so a box lands as
-        // [atom][row][128 bytes].  Weights (A) load 128 rows, route rows (B) N <= 128 rows, one
-        // map per N in {32, 64, 96, 128}; the K pitches hp, fp are padded to 128 with zeros.
-        const unsigned long long hp = (unsigned long long)plan->hp, fpp = (unsigned long long)plan->fp;
+    if (fp8 || fp4) {
+        // MXFP8 / NVFP4 (one CTA per tile): K stage = 256 bytes of codes (256 E4M3 or 512
+        // E2M1 elements) = two 128-byte swizzle atoms; the maps address byte b of a row as
+        // (b % 128, row, b / 128), so a box lands as [atom][row][128 bytes].  Weights (A) load
+        // 128 rows, route rows (B) N <= 128 rows, one map per N in {32, 64, 96, 128}; the
+        // K pitches (hp, fp elements) are whole 128-byte blocks padded with zero codes.
+        const unsigned long long hp = (unsigned long long)(fp4 ? plan->hp / 2 : plan->hp);
+        const unsigned long long fpp = (unsigned long long)(fp4 ? plan->fp / 2 : plan->fp);
         const unsigned box128[3] = {128, 128, 2};
         const unsigned long long dW1[3] = {128ull, uE * (unsigned long long)plan->w1r, hp / 128};
         const unsigned long long sW1[2] = {hp, 128ull};
@@ -361,7 +399,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     int* perm = reinterpret_cast<int*>(ws + L.perm);
     int* inv = reinterpret_cast<int*>(ws + L.inv);
     int4* tiles = reinterpret_cast<int4*>(ws + L.tiles);
-    int* ready = fp8 ? nullptr : reinterpret_cast<int*>(ws + L.ready);
+    int* ready = fp8 || fp4 ? nullptr : reinterpret_cast<int*>(ws + L.ready);  // bf16 only
     e = launch_permute(plan, live_count_dev, r_ids, reinterpret_cast<int*>(ws + L.blkcnt),
                        reinterpret_cast<int*>(ws + L.offsets), reinterpret_cast<int*>(ws + L.padoff), tiles, perm, inv,
                        ready, status, s);
@@ -372,6 +410,10 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
         e = launch_gather_mxfp8(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, (int)plan->hp, k,
                                 inv, ws + L.xq, ws + L.xs, s);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
+    } else if (fp4) {
+        e = launch_gather_nvfp4(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, (int)plan->hp, k,
+                                inv, ws + L.xq, ws + L.xs, reinterpret_cast<float*>(ws + L.xg), s);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
 
     const long long m_tiles = plan->max_m_tiles;
@@ -379,7 +421,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g1.tiles = tiles;
     g1.status_words = status;
     g1.status_flags = status + kStFlags;
-    g1.out = ws + L.h;
+    g1.out = fp4 ? ws + L.hf : ws + L.h;  // NVFP4: fp32 h rows for the per-row quantisation pass
     g1.out_scales = nullptr;
     g1.out_ld = plan->fp;  // h rows: F values + zero padding to the down GEMM's K pitch
     g1.out_cols = (int)plan->fp;  // every padded column: f >= F are zero-weight rows, h = 0
@@ -404,10 +446,18 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g1.xg_pitch = plan->hp * 2;
     g1.ready = ready;
     g1.copy_next = status + kStCopyNext;
+    g1.row_scale = fp4 ? reinterpret_cast<const float*>(ws + L.xg) : nullptr;
+    g1.w_scale = fp4 ? reinterpret_cast<const float*>(wb + plan->wb.wg) : nullptr;
     if (!mark(3)) return MOE_ERR_CUDA;
-    e = fp8 ? launch_gemm1_mxfp8(tA1, rB1, g1, m_tiles * g1.n_tiles, s)
-            : launch_gemm1_bf16_pair(tA1, tX, rB1, g1, m_tiles * g1.n_tiles, s);
+    e = fp8   ? launch_gemm1_mxfp8(tA1, rB1, g1, m_tiles * g1.n_tiles, s)
+        : fp4 ? launch_gemm1_nvfp4(tA1, rB1, g1, m_tiles * g1.n_tiles, s)
+              : launch_gemm1_bf16_pair(tA1, tX, rB1, g1, m_tiles * g1.n_tiles, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (fp4) {  // h rows -> NVFP4 with a scale per row (timed with the gate/up stage)
+        e = launch_quantize_h_nvfp4(reinterpret_cast<const float*>(ws + L.hf), live_count_dev, max_live, k,
+                                    (int)plan->fp, inv, ws + L.h, ws + L.hs, reinterpret_cast<float*>(ws + L.hg), s);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
 
     GemmParams g2 = g1;
     g2.out = ws + L.y;
@@ -415,13 +465,15 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g2.out_cols = H;
     g2.n_tiles = plan->nt2;
     g2.k_blocks = plan->ks2;
-    g2.a_rows = fp8 ? H : plan->hr;
+    g2.a_rows = fp8 || fp4 ? H : plan->hr;
     g2.sfa = wb + plan->wb.w2s;
     g2.sfb = ws + L.hs;
     g2.out_scales = nullptr;
+    g2.row_scale = fp4 ? reinterpret_cast<const float*>(ws + L.hg) : nullptr;
     if (!mark(4)) return MOE_ERR_CUDA;
-    e = fp8 ? launch_gemm2_mxfp8(tA2, rB2, g2, m_tiles * g2.n_tiles, s)
-            : launch_gemm2_bf16_pair(tA2, rB2, g2, m_tiles * g2.n_tiles, s);
+    e = fp8   ? launch_gemm2_mxfp8(tA2, rB2, g2, m_tiles * g2.n_tiles, s)
+        : fp4 ? launch_gemm2_nvfp4(tA2, rB2, g2, m_tiles * g2.n_tiles, s)
+              : launch_gemm2_bf16_pair(tA2, rB2, g2, m_tiles * g2.n_tiles, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     if (!mark(5)) return MOE_ERR_CUDA;
 
@@ -465,9 +517,14 @@ moe_status moe_get_workspace_views(const moe_plan* plan, const void* workspace, 
     v->inv = reinterpret_cast<const int*>(ws + L.inv);
     v->pad_offsets = reinterpret_cast<const int*>(ws + L.padoff);
     v->h = ws + L.h;
-    v->h_scales = plan->d.precision == MOE_MXFP8 ? ws + L.hs : nullptr;
+    const bool scaled = plan->d.precision != MOE_BF16;
+    const bool fp4 = plan->d.precision == MOE_NVFP4;
+    v->h_scales = scaled ? ws + L.hs : nullptr;
     v->xq = ws + L.xq;
-    v->xq_scales = plan->d.precision == MOE_MXFP8 ? ws + L.xs : nullptr;
+    v->xq_scales = scaled ? ws + L.xs : nullptr;
+    v->xq_row_scales = fp4 ? reinterpret_cast<const float*>(ws + L.xg) : nullptr;
+    v->h_row_scales = fp4 ? reinterpret_cast<const float*>(ws + L.hg) : nullptr;
+    v->h_fp32 = fp4 ? reinterpret_cast<const float*>(ws + L.hf) : nullptr;
     v->rows_padded = plan->rows_pad;
     v->status = reinterpret_cast<const unsigned*>(ws + L.status);
     return MOE_OK;

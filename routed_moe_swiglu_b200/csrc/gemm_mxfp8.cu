@@ -43,6 +43,7 @@
 // implies).  Every wait is bounded.
 #include "moe_internal.cuh"
 #include "mxfp8.cuh"
+#include "nvfp4.cuh"
 #include "ptx.cuh"
 
 namespace moe {
@@ -57,20 +58,28 @@ constexpr uint32_t kAtomBytesA = kTileM * kBK8;        // 16 KB
 constexpr uint32_t kABytes = kAtoms * kAtomBytesA;     // 32 KB
 constexpr uint32_t kBBytes = kAtoms * kMaxN * kBK8;    // up to 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr int kSfGroup = 8;                            // K blocks per scale-factor bulk copy (4 stages)
-constexpr int kStagesPerGroup = kSfGroup / kAtoms;
-constexpr uint32_t kSfGroupBytes = kSfGroup * kSfBlock;
-constexpr uint32_t kSfBytes = 2 * 2 * kSfGroupBytes;   // [buffer][A/B][8 blocks][512 B]
+// Scale blocks: MXFP8 (kFmt 0) has one 512-byte block per operand and 128-byte K block
+// (4 MMAs, a byte each); NVFP4 (kFmt 1) has one per 64-element MMA step, four per K block.
+template <int kFmt>
+struct SfCfg {
+    static constexpr int kPerKb = kFmt == 0 ? 1 : 4;               // scale blocks per K block
+    static constexpr int kGroup = kFmt == 0 ? 8 : 2;               // K blocks per bulk copy (4 stages / 1)
+    static constexpr int kStagesPerGroup = kGroup / kAtoms;
+    static constexpr uint32_t kGroupBytes = (uint32_t)(kGroup * kPerKb) * kSfBlock;  // 4 KB either way
+    static constexpr uint32_t kColsPerStage = (uint32_t)(kAtoms * kPerKb) * 8u;     // A 4 + B 4 per block
+};
+constexpr uint32_t kSfGroupBytes = SfCfg<0>::kGroupBytes;
+static_assert(SfCfg<1>::kGroupBytes == kSfGroupBytes, "one scale staging size for both formats");
+constexpr uint32_t kSfBytes = 2 * 2 * kSfGroupBytes;   // [buffer][A/B][group][512 B blocks]
 constexpr uint32_t kAccCols = kMaxN;
 constexpr uint32_t kSfCol0 = 2 * kAccCols;             // first scale-factor TMEM column
-constexpr uint32_t kSfColsPerStage = 16;               // per atom: A 4 columns, B 4 columns
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kStageHBytes = 32 * 64 * 4;         // gate/up: fp32 h of 32 routes x 64 f
 constexpr uint32_t kYTBytes = 32 * 32 * 4;             // down: fp32 y of 32 routes x 32 columns, per warp
 constexpr uint32_t kEpiBytes = 2 * kStageHBytes > 4 * kYTBytes ? 2 * kStageHBytes : 4 * kYTBytes;
 constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kSfBytes + kEpiBytes + 256;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kSfCol0 + kSfColsPerStage * kStages <= kTmemCols, "TMEM budget");
+static_assert(kSfCol0 + SfCfg<1>::kColsPerStage * kStages <= kTmemCols, "TMEM budget");
 static_assert(kEpiBytes >= 4 * 32 * 32 * 4, "squared-ReLU epilogue boxes");
 constexpr uint32_t kEpiBar = 1;                        // named barrier of the 4 epilogue warps
 
@@ -92,6 +101,26 @@ __host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, uint32_t sfa_id,
            | (1u << 23)                    // scale type: E8M0
            | ((uint32_t)(M >> 4) << 24)    // M / 16
            | (sfa_id << 29);               // A scale-factor byte
+}
+
+// NVFP4: E2M1 x E2M1 (kind::mxf4nvf4), E4M3 scales, one per 16 K elements
+// (scale_vec::4X: an MMA of K = 64 reads a whole 32-bit scale cell per row).
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+    return (1u << 7) | (1u << 10)          // A, B: E2M1
+           | ((uint32_t)(N >> 3) << 17)    // N / 8
+           | (0u << 23)                    // scale type: E4M3
+           | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+__device__ __forceinline__ void mma_nvf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
 }
 
 // Descriptor of a 32-row x 16-byte scale block in shared memory (no
@@ -126,8 +155,11 @@ __device__ __forceinline__ float swiglu_value(float g, float u, float clamp) {
 // Routes of a tile rounded up to the MMA's N granularity.
 __device__ __forceinline__ int tile_n(int nvalid) { return (nvalid + 31) & ~31; }
 
-template <int kMode>  // 0: gate/up + SwiGLU -> MXFP8 h;  1: down -> fp32 y
+// kMode 0: gate/up + SwiGLU -> h (MXFP8 codes, or NVFP4's fp32 rows for a second pass);
+// kMode 1: down -> fp32 y.  kFmt 0: MXFP8; 1: NVFP4.
+template <int kMode, int kFmt>
 __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const BoxMaps8& tmB, const GemmParams& p) {
+    using Sf = SfCfg<kFmt>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sSf = smem + kStages * kStageBytes;  // [buffer][A/B][8][512]
@@ -187,8 +219,8 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                 const int n = tile_n(ti.z);
                 const CUtensorMap* mapB = &tmB.m[(n >> 5) - 1];
                 const int a_row = (int)((long long)ti.x * p.a_rows) + nt * kTileM;
-                const uint8_t* sfa_src = p.sfa + ((size_t)ti.x * p.n_tiles + nt) * nblk * kSfBlock;
-                const uint8_t* sfb_src = p.sfb + (size_t)(ti.y / kBM) * nblk * kSfBlock;
+                const uint8_t* sfa_src = p.sfa + ((size_t)ti.x * p.n_tiles + nt) * nblk * Sf::kPerKb * kSfBlock;
+                const uint8_t* sfb_src = p.sfb + (size_t)(ti.y / kBM) * nblk * Sf::kPerKb * kSfBlock;
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!mbar_wait_bounded(&bars->empty[stage], phase ^ 1u, abort_flag, p.wait_limit_ns)) {
                         ok = false;
@@ -198,7 +230,7 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                     uint32_t tx = kABytes + (uint32_t)n * (kAtoms * kBK8);
                     int gs = 0;
                     const int blk0 = kb * kAtoms;
-                    if (kb % kStagesPerGroup == 0) {
+                    if (kb % Sf::kStagesPerGroup == 0) {
                         // the scale blocks of this stage and the next gs-1 stages, once the MMAs
                         // that read this buffer two groups ago are done
                         const int sb = (int)(groups & 1u);
@@ -207,8 +239,8 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                             ok = false;
                             break;
                         }
-                        gs = nblk - blk0 < kSfGroup ? nblk - blk0 : kSfGroup;
-                        tx += 2u * (uint32_t)gs * kSfBlock;
+                        gs = nblk - blk0 < Sf::kGroup ? nblk - blk0 : Sf::kGroup;
+                        tx += 2u * (uint32_t)(gs * Sf::kPerKb) * kSfBlock;
                     }
                     mbar_arrive_expect_tx(&bars->full[stage], tx);
                     last_phase[stage] = (int)phase;
@@ -216,9 +248,10 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                     tma_load_3d(stage_b(stage), mapB, &bars->full[stage], 0, ti.y, blk0);
                     if (gs > 0) {
                         const int sb = (int)(groups & 1u);
-                        bulk_load(sf_buf(sb, 0), sfa_src + (size_t)blk0 * kSfBlock, (uint32_t)gs * kSfBlock,
+                        const uint32_t sf_bytes = (uint32_t)(gs * Sf::kPerKb) * kSfBlock;
+                        bulk_load(sf_buf(sb, 0), sfa_src + (size_t)blk0 * Sf::kPerKb * kSfBlock, sf_bytes,
                                   &bars->full[stage]);
-                        bulk_load(sf_buf(sb, 1), sfb_src + (size_t)blk0 * kSfBlock, (uint32_t)gs * kSfBlock,
+                        bulk_load(sf_buf(sb, 1), sfb_src + (size_t)blk0 * Sf::kPerKb * kSfBlock, sf_bytes,
                                   &bars->full[stage]);
                         ++groups;
                     }
@@ -271,22 +304,38 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                     const uint32_t b_addr = smem_u32(stage_b(stage));
                     const uint32_t b_atom = (uint32_t)n * kBK8;  // bytes of one atom of the B box
                     for (int h = 0; h < nb; ++h) {
-                        const int gi = (blk0 + h) % kSfGroup;
-                        const uint32_t sfa_t = tmem_base + kSfCol0 + (uint32_t)stage * kSfColsPerStage + (uint32_t)h * 8u;
-                        const uint32_t sfb_t = sfa_t + 4u;
-                        tmem_cp_32x128b_warpx4(sfa_t, sdesc_sf(smem_u32(sf_buf(sb, 0) + gi * kSfBlock)));
-                        tmem_cp_32x128b_warpx4(sfb_t, sdesc_sf(smem_u32(sf_buf(sb, 1) + gi * kSfBlock)));
+                        const int gi = (blk0 + h) % Sf::kGroup;
                         const uint32_t a_h = a_addr + (uint32_t)h * kAtomBytesA;
                         const uint32_t b_h = b_addr + (uint32_t)h * b_atom;
+                        const uint32_t sf_t0 = tmem_base + kSfCol0 + (uint32_t)stage * Sf::kColsPerStage +
+                                               (uint32_t)(h * Sf::kPerKb) * 8u;
+                        if constexpr (kFmt == 0) {
+                            // one scale block per operand: MMA kk reads byte kk of each cell
+                            tmem_cp_32x128b_warpx4(sf_t0, sdesc_sf(smem_u32(sf_buf(sb, 0) + gi * kSfBlock)));
+                            tmem_cp_32x128b_warpx4(sf_t0 + 4u, sdesc_sf(smem_u32(sf_buf(sb, 1) + gi * kSfBlock)));
 #pragma unroll
-                        for (int kk = 0; kk < kBK8 / 32; ++kk) {
-                            mma_mxf8_ss(d_tmem, sdesc_kmajor_sw128(a_h + kk * 32), sdesc_kmajor_sw128(b_h + kk * 32),
-                                        idesc_mxf8(kTileM, n, (uint32_t)kk, (uint32_t)kk), sfa_t, sfb_t,
-                                        (kb | h | kk) != 0 ? 1u : 0u);
+                            for (int kk = 0; kk < kBK8 / 32; ++kk) {
+                                mma_mxf8_ss(d_tmem, sdesc_kmajor_sw128(a_h + kk * 32),
+                                            sdesc_kmajor_sw128(b_h + kk * 32),
+                                            idesc_mxf8(kTileM, n, (uint32_t)kk, (uint32_t)kk), sf_t0, sf_t0 + 4u,
+                                            (kb | h | kk) != 0 ? 1u : 0u);
+                            }
+                        } else {
+                            // one scale block per operand and 64-element MMA step (32 bytes of K)
+#pragma unroll
+                            for (int kk = 0; kk < kBK8 / 32; ++kk) {
+                                const uint32_t sfa_t = sf_t0 + (uint32_t)kk * 8u;
+                                const uint32_t src = (uint32_t)(gi * Sf::kPerKb + kk) * kSfBlock;
+                                tmem_cp_32x128b_warpx4(sfa_t, sdesc_sf(smem_u32(sf_buf(sb, 0) + src)));
+                                tmem_cp_32x128b_warpx4(sfa_t + 4u, sdesc_sf(smem_u32(sf_buf(sb, 1) + src)));
+                                mma_nvf4_ss(d_tmem, sdesc_kmajor_sw128(a_h + kk * 32),
+                                            sdesc_kmajor_sw128(b_h + kk * 32), idesc_nvf4(kTileM, n), sfa_t,
+                                            sfa_t + 4u, (kb | h | kk) != 0 ? 1u : 0u);
+                            }
                         }
                     }
                     mma_commit(&bars->empty[stage]);
-                    if (kb % kStagesPerGroup == kStagesPerGroup - 1 || kb == kb_count - 1) {  // group consumed
+                    if (kb % Sf::kStagesPerGroup == Sf::kStagesPerGroup - 1 || kb == kb_count - 1) {  // group consumed
                         mma_commit(&bars->sf_empty[sb]);
                         ++groups;
                     }
@@ -332,7 +381,74 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
             }
             tc_fence_after_sync();
             const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)buf * kAccCols;
-            if (kMode == 0 && p.relu2) {
+            if constexpr (kMode == 0 && kFmt == 1) {
+                // NVFP4: the accumulator times g_x(route) * g_w1(expert) is the pre-activation;
+                // h leaves as fp32 rows (pitch out_ld) for the per-row quantisation pass.
+                float* hf = reinterpret_cast<float*>(p.out);
+                const float gw = __ldg(p.w_scale + 2 * ti.x);
+                if (p.relu2) {
+                    // squared-ReLU experts: lane = f (32 f from f0), register j = route 32c + j
+                    const int f0 = nt * kTileM + 32 * quad;
+#pragma unroll 1
+                    for (int c = 0; c < nch; ++c) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(taddr + c * 32, v);
+                        float pv = 1.0f, sc = 0.0f;
+                        if (c * 32 + lane < ti.z) {
+                            sc = __ldg(p.row_scale + ti.y + c * 32 + lane) * gw;
+                            if (p.route_probs != nullptr) pv = __ldg(p.route_probs + __ldg(p.perm + ti.w + c * 32 + lane));
+                        }
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            float g = __uint_as_float(v[j]) * __shfl_sync(0xffffffffu, sc, j);
+                            if (p.clamp > 0.0f) g = fminf(fmaxf(g, -p.clamp), p.clamp);
+                            const float r = fmaxf(g, 0.0f);
+                            float hv = r * r;
+                            if (p.route_probs != nullptr) hv *= __shfl_sync(0xffffffffu, pv, j);
+                            if (c * 32 + j < ti.z && f0 < p.out_cols)
+                                hf[(size_t)(ti.y + c * 32 + j) * (size_t)p.out_ld + f0 + lane] = hv;
+                        }
+                    }
+                } else {
+                    const bool lo = lane < 16;
+                    const int fl = 16 * quad + (lane & 15);  // this lane's f within the tile's 64
+                    const int qr = et >> 2, qf = (et & 3) * 16;  // store role: route qr, f qf..qf+15
+#pragma unroll 1
+                    for (int c = 0; c < nch; ++c, ++chunk_count) {
+                        float* st = reinterpret_cast<float*>(sEpi + (chunk_count & 1u) * kStageHBytes);
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(taddr + c * 32, v);
+                        float pv = 1.0f, sc = 0.0f;
+                        if (c * 32 + lane < ti.z) {
+                            sc = __ldg(p.row_scale + ti.y + c * 32 + lane) * gw;
+                            if (p.route_probs != nullptr) pv = __ldg(p.route_probs + __ldg(p.perm + ti.w + c * 32 + lane));
+                        }
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const uint32_t mine = lo ? v[j] : v[16 + j];
+                            const uint32_t other = __shfl_xor_sync(0xffffffffu, lo ? v[16 + j] : v[j], 16);
+                            const int route = lo ? j : 16 + j;
+                            const float rs = __shfl_sync(0xffffffffu, sc, route);
+                            const float g = __uint_as_float(lo ? mine : other) * rs;
+                            const float u = __uint_as_float(lo ? other : mine) * rs;
+                            float hv = swiglu_value(g, u, p.clamp);
+                            if (p.route_probs != nullptr) hv *= __shfl_sync(0xffffffffu, pv, route);
+                            st[route * 64 + (fl ^ (lo ? 0 : 16))] = hv;
+                        }
+                        named_bar_sync(kEpiBar, 128);
+                        const int route = c * 32 + qr;
+                        const int fb = nt * 64 + qf;
+                        if (route < ti.z && fb < p.out_cols) {
+                            const float4* src = reinterpret_cast<const float4*>(st + qr * 64 + (qf ^ (qr >= 16 ? 16 : 0)));
+                            float4* dst = reinterpret_cast<float4*>(hf + (size_t)(ti.y + route) * (size_t)p.out_ld + fb);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) dst[i] = src[i];
+                        }
+                    }
+                }
+            } else if (kMode == 0 && p.relu2) {
                 // squared-ReLU experts: lane = f (this warp's 32 f from f0, one 32-f block),
                 // register j = route 32c + j.  h = relu(g)^2 goes through a per-warp box
                 // [route][32 f] fp32 (column rotated by the route against bank conflicts); then
@@ -458,7 +574,15 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                     for (int c = 0; c < nch; ++c) {
                         uint32_t v[32];
                         tmem_ld_32x32b_x32(taddr + c * 32, v);
+                        float sc = 0.0f;  // NVFP4: g_h(route 32c + lane) * g_w2(expert)
+                        if (kFmt == 1 && c * 32 + lane < ti.z)
+                            sc = __ldg(p.row_scale + ti.y + c * 32 + lane) * __ldg(p.w_scale + 2 * ti.x + 1);
                         tmem_ld_wait();
+                        if constexpr (kFmt == 1) {
+#pragma unroll
+                            for (int r = 0; r < 32; ++r)
+                                v[r] = __float_as_uint(__uint_as_float(v[r]) * __shfl_sync(0xffffffffu, sc, r));
+                        }
 #pragma unroll
                         for (int r = 0; r < 32; ++r) *reinterpret_cast<uint32_t*>(tbuf + r * 128 + lane * 4) = v[r];
                         __syncwarp();
@@ -492,13 +616,25 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
 __global__ void __launch_bounds__(kThreads, 1)
     moe_gemm_gate_up_swiglu_mxfp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BoxMaps8 tmB,
                                   const GemmParams p) {
-    gemm_mxfp8_body<0>(tmA, tmB, p);
+    gemm_mxfp8_body<0, 0>(tmA, tmB, p);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     moe_gemm_down_mxfp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BoxMaps8 tmB,
                         const GemmParams p) {
-    gemm_mxfp8_body<1>(tmA, tmB, p);
+    gemm_mxfp8_body<1, 0>(tmA, tmB, p);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    moe_gemm_gate_up_swiglu_nvfp4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BoxMaps8 tmB,
+                                  const GemmParams p) {
+    gemm_mxfp8_body<0, 1>(tmA, tmB, p);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    moe_gemm_down_nvfp4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BoxMaps8 tmB,
+                        const GemmParams p) {
+    gemm_mxfp8_body<1, 1>(tmA, tmB, p);
 }
 
 using GemmKernel = void (*)(CUtensorMap, BoxMaps8, GemmParams);
@@ -531,6 +667,18 @@ cudaError_t launch_gemm2_mxfp8(const CUtensorMap& a, const BoxMaps8& b, const Ge
                                cudaStream_t s) {
     static int configured = -1;
     return launch_impl(moe_gemm_down_mxfp8, &configured, a, b, gp, max_tiles, s);
+}
+
+cudaError_t launch_gemm1_nvfp4(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
+                               cudaStream_t s) {
+    static int configured = -1;
+    return launch_impl(moe_gemm_gate_up_swiglu_nvfp4, &configured, a, b, gp, max_tiles, s);
+}
+
+cudaError_t launch_gemm2_nvfp4(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
+                               cudaStream_t s) {
+    static int configured = -1;
+    return launch_impl(moe_gemm_down_nvfp4, &configured, a, b, gp, max_tiles, s);
 }
 
 }  // namespace moe

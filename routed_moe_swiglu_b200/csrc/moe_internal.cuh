@@ -42,11 +42,13 @@ constexpr unsigned long long kWaitLimitNs = 4000000000ull;
 struct WsLayout {
     size_t status, r_ids, r_probs, blkcnt, offsets, padoff, tiles, perm, inv, ready;
     size_t xq, xs, h, hs, y;
+    size_t xg, hf, hg;  // NVFP4: per-row scales of x and h, the fp32 h rows
     size_t total;
 };
 
 struct WbufLayout {
     size_t w1, w1s, w2, w2s;
+    size_t wg;  // NVFP4: second-level scales [E][2] (W1, W2)
     size_t total;
 };
 
@@ -121,6 +123,10 @@ struct GemmParams {
     long long xg_pitch;
     int* ready;
     unsigned* copy_next;
+    // NVFP4: second-level scales of the B rows (fp32 per padded route row: x for the
+    // gate/up GEMM, h for the down GEMM) and of the weights ([E][2]: W1, W2)
+    const float* row_scale;
+    const float* w_scale;
 };
 
 // ---------------------------------------------------------------- launchers
@@ -153,6 +159,18 @@ cudaError_t launch_gemm1_mxfp8(const CUtensorMap& a, const BoxMaps8& b, const Ge
                                cudaStream_t s);
 cudaError_t launch_gemm2_mxfp8(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
                                cudaStream_t s);
+cudaError_t launch_gemm1_nvfp4(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
+                               cudaStream_t s);
+cudaError_t launch_gemm2_nvfp4(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
+                               cudaStream_t s);
+cudaError_t launch_nvfp4_quantize_rows(const __nv_bfloat16* in, long long rows, int cols, long long ld_in,
+                                       uint8_t* q, uint8_t* scales, float* g, const int* live_rows, cudaStream_t s);
+cudaError_t launch_gather_nvfp4(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
+                                const int* inv, uint8_t* xq, uint8_t* xs, float* xg, cudaStream_t s);
+cudaError_t launch_quantize_h_nvfp4(const float* hf, const int* live, int max_live, int k, int fp, const int* inv,
+                                    uint8_t* hq, uint8_t* hs, float* hg, cudaStream_t s);
+cudaError_t launch_prepare_nvfp4(const moe_plan* p, const __nv_bfloat16* wg, const __nv_bfloat16* wu,
+                                 const __nv_bfloat16* wd, void* buf, cudaStream_t s);
 cudaError_t launch_prepare_bf16(const moe_plan* p, const __nv_bfloat16* wg, const __nv_bfloat16* wu,
                                 const __nv_bfloat16* wd, void* buf, cudaStream_t s);
 cudaError_t launch_prepare_mxfp8(const moe_plan* p, const __nv_bfloat16* wg, const __nv_bfloat16* wu,

@@ -15,7 +15,8 @@ import oracle
 import routed_moe_swiglu_b200 as rm
 import workloads
 
-TOL = {"bf16": dict(max_rms=2e-2, mean_rel=2e-3), "mxfp8": dict(max_rms=5e-2, mean_rel=None)}
+TOL = {"bf16": dict(max_rms=2e-2, mean_rel=2e-3), "mxfp8": dict(max_rms=5e-2, mean_rel=None),
+       "nvfp4": dict(max_rms=5e-2, mean_rel=None)}
 
 
 def assert_close(gpu: np.ndarray, ref: np.ndarray, precision: str, what: str = "") -> dict:
@@ -105,6 +106,10 @@ def oracle_forward(x_cpu, logits_cpu, weights, k, live, tokens=None, precision="
     toks = np.arange(live) if tokens is None else np.asarray(tokens)
     if precision == "bf16":
         out = oracle.forward_bf16(x_cpu[:live], ids, probs, *weights, tokens=toks)
+    elif precision == "nvfp4":
+        if wq is None:
+            wq = oracle.quantize_weights_nvfp4(*weights)
+        out = oracle.forward_nvfp4(x_cpu[:live], ids, probs, wq, tokens=toks)
     else:
         if wq is None:
             wq = oracle.quantize_weights_mxfp8(*weights)

@@ -21,6 +21,9 @@ describes them; weights are random-init, there are no trained checkpoints):
             expert loads are heavily skewed.
   mxfp8     T=4,096, same shapes and routing distribution as prefill, seed 3,
             run in MXFP8.
+  nvfp4     T=4,096, same shapes and routing distribution as prefill, seed 5,
+            run in NVFP4 (the per-token recipe).
+  decode_nvfp4  the decode workload's shapes and buffer, seed 6, in NVFP4.
   sweep     H=2688, F=1856, E=128, top-6, a 262,144-row buffer, seed 4; live
             counts {1, 64, 1024, 8192} are written on the device between
             replays of one captured graph.  Rows at or past the largest live
@@ -47,7 +50,7 @@ class Workload:
     capacity: int  # rows in the preallocated buffer
     live: tuple  # live row counts this workload runs with
     seed: int
-    precision: str  # "bf16" or "mxfp8"
+    precision: str  # "bf16", "mxfp8" or "nvfp4"
     zipf_bias: bool = False
     distinct_logits_gap: float = 0.0
     nan_past_live: bool = False
@@ -75,6 +78,8 @@ WORKLOADS = {
     "decode": Workload("decode", 2048, 1024, 128, 8, 65536, (256,), 1, "bf16", nan_past_live=True),
     "prefill": Workload("prefill", 2048, 1024, 128, 8, 16384, (16384,), 2, "bf16", zipf_bias=True),
     "mxfp8": Workload("mxfp8", 2048, 1024, 128, 8, 4096, (4096,), 3, "mxfp8", zipf_bias=True),
+    "nvfp4": Workload("nvfp4", 2048, 1024, 128, 8, 4096, (4096,), 5, "nvfp4", zipf_bias=True),
+    "decode_nvfp4": Workload("decode_nvfp4", 2048, 1024, 128, 8, 65536, (256,), 6, "nvfp4", nan_past_live=True),
     "sweep": Workload("sweep", 2688, 1856, 128, 6, 262144, (1, 64, 1024, 8192), 4, "bf16",
                       nan_past_live=True),
 }
