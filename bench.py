@@ -4,7 +4,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One step = one pass of the whole path (route, permute, gather, gate/up GEMM
-+ SwiGLU, down GEMM, combine) over one batch of seeded synthetic inputs that
++ SwiGLU, down GEMM, combine; NVFP4 also quantises h between the GEMMs, timed
+with the gate/up stage) over one batch of seeded synthetic inputs that
 are already resident in HBM.  The K timed steps are one captured CUDA graph
 (K forwards back to back, stage events inside), bracketed by a barrier and
 a device synchronise; the time is the max over ranks.  Every step re-reads
@@ -41,9 +42,16 @@ import torch  # noqa: E402
 
 import workloads  # noqa: E402
 
-KERNELS_PER_FORWARD = 8  # route, hist, scan, scatter, gather, gemm gate/up, gemm down, combine
+def kernels_per_forward(precision: str, max_live: int) -> int:
+    """Library kernels one forward launches: route, the permute (hist, scan, scatter; one
+    kernel for plans of at most 1,024 live rows), the x gather (MXFP8, NVFP4: bf16 copies
+    the rows inside its gate/up GEMM), gate/up GEMM, NVFP4's h quantisation, down GEMM,
+    combine."""
+    permute = 1 if max_live <= 1024 else 3
+    return 1 + permute + (precision != "bf16") + 1 + (precision == "nvfp4") + 1 + 1
 STAGES = ("route", "permute", "gather", "gemm_gate_up", "gemm_down", "combine")
-DEFAULT_STEPS = {"tiny": 200, "decode": 200, "prefill": 30, "mxfp8": 50, "sweep": 20}
+DEFAULT_STEPS = {"tiny": 200, "decode": 200, "prefill": 30, "mxfp8": 50, "nvfp4": 50, "decode_nvfp4": 200,
+                 "sweep": 20}
 
 
 def parse_args():
@@ -214,6 +222,11 @@ KERNEL_SOURCES = {
                              _CSRC + "moe_internal.cuh"],
     ("combine", "bf16"): [_CSRC + "permute.cu", _CSRC + "moe_internal.cuh"],
     ("combine", "mxfp8"): [_CSRC + "permute.cu", _CSRC + "moe_internal.cuh"],
+    ("gemm_gate_up", "nvfp4"): [_CSRC + "gemm_mxfp8.cu", _CSRC + "mxfp8.cuh", _CSRC + "nvfp4.cuh", _CSRC + "nvfp4.cu",
+                                _CSRC + "ptx.cuh", _CSRC + "moe_internal.cuh"],
+    ("gemm_down", "nvfp4"): [_CSRC + "gemm_mxfp8.cu", _CSRC + "mxfp8.cuh", _CSRC + "nvfp4.cuh", _CSRC + "ptx.cuh",
+                             _CSRC + "moe_internal.cuh"],
+    ("combine", "nvfp4"): [_CSRC + "permute.cu", _CSRC + "moe_internal.cuh"],
 }
 
 
@@ -430,7 +443,10 @@ def roofline(w, res, peaks):
     ms = st[dom]
     H, F, k = w.hidden, w.ffn, w.top_k
     R = res["routes"]
-    bpe = 1 if w.precision == "mxfp8" else 2
+    # bytes per element of the operands, block scales included: E4M3 + an E8M0 per 32,
+    # E2M1 + an E4M3 per 16, bf16
+    bpe = {"mxfp8": 1 + 1 / 32, "nvfp4": 0.5 + 1 / 16}.get(w.precision, 2)
+    tc_ratio = {"mxfp8": 2.0, "nvfp4": 4.0}.get(w.precision, 1.0)  # nominal dense peak over bf16
     sustained = res["timed_s"] > 1.0
     tflops_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     out = {"kernel": dom}
@@ -446,17 +462,18 @@ def roofline(w, res, peaks):
             abytes = R * F * bpe + R * H * 4
         bytes_ = wbytes + abytes
         t_hbm = bytes_ / (peaks["hbm_gbs"] * 1e9)
-        t_tc = flops / (tflops_peak * 1e12 * (2.0 if w.precision == "mxfp8" else 1.0))
+        t_tc = flops / (tflops_peak * 1e12 * tc_ratio)
         if t_hbm >= t_tc:
             ach = bytes_ / (ms / 1e3) / 1e9
             out.update(bound="hbm", achieved=ach, peak=peaks["hbm_gbs"], unit="GB/s",
                        algorithmic_per_launch=bytes_)
         else:
             ach = flops / (ms / 1e3) / 1e12
-            pk = tflops_peak * (2.0 if w.precision == "mxfp8" else 1.0)
+            pk = tflops_peak * tc_ratio
             out.update(bound="tensor", achieved=ach, peak=pk, unit="TFLOP/s", algorithmic_per_launch=flops,
                        peak_kind=("sustained" if sustained else "burst")
-                       + (" bf16 x2 (fp8 nominal ratio)" if w.precision == "mxfp8" else " bf16"))
+                       + {"mxfp8": " bf16 x2 (fp8 nominal ratio)", "nvfp4": " bf16 x4 (fp4 nominal ratio)"}.get(
+                           w.precision, " bf16"))
     else:
         # memory-bound helper kernels: bytes they must move
         if dom == "combine":
@@ -487,6 +504,28 @@ def oracle_variant(a):
     return v
 
 
+def oracle_weights(w, weights, variant):
+    """The oracle's quantised weights for a block-scaled workload (None for bf16)."""
+    import oracle
+
+    if w.precision == "mxfp8":
+        return oracle.quantize_weights_mxfp8(*weights)
+    if w.precision == "nvfp4":
+        relu2 = bool((variant or {}).get("squared_relu"))
+        return oracle.quantize_weights_nvfp4(weights[0], None if relu2 else weights[1], weights[2])
+    return None
+
+
+def oracle_forward_tokens(w, x, ids, probs, weights, wq, sel, variant):
+    import oracle
+
+    if w.precision == "mxfp8":
+        return oracle.forward_mxfp8(x, ids, probs, wq, tokens=sel, **(variant or {}))
+    if w.precision == "nvfp4":
+        return oracle.forward_nvfp4(x, ids, probs, wq, tokens=sel, **(variant or {}))
+    return oracle.forward_bf16(x, ids, probs, *weights, tokens=sel, **(variant or {}))
+
+
 def oracle_tokens_per_s(w, x, logits, weights, live, budget_s, min_tokens=8, variant=None):
     """Time the oracle (as it stands) on the host cores over a bounded sample
     of the live tokens: route all live rows, then the expert forward of a
@@ -495,7 +534,7 @@ def oracle_tokens_per_s(w, x, logits, weights, live, budget_s, min_tokens=8, var
 
     import oracle
 
-    wq = oracle.quantize_weights_mxfp8(*weights) if w.precision == "mxfp8" else None
+    wq = oracle_weights(w, weights, variant)
     toks = workloads.sample_tokens(live, live, w.seed).numpy()
     t0 = time.perf_counter()
     ids, probs = oracle.route(logits[:live].numpy(), w.top_k)
@@ -504,10 +543,7 @@ def oracle_tokens_per_s(w, x, logits, weights, live, budget_s, min_tokens=8, var
     while spent < budget_s:
         sel = toks[(done + np.arange(n)) % live]
         t0 = time.perf_counter()
-        if w.precision == "mxfp8":
-            oracle.forward_mxfp8(x[:live], ids, probs, wq, tokens=sel, **(variant or {}))
-        else:
-            oracle.forward_bf16(x[:live], ids, probs, *weights, tokens=sel, **(variant or {}))
+        oracle_forward_tokens(w, x[:live], ids, probs, weights, wq, sel, variant)
         dt = time.perf_counter() - t0
         spent += dt
         done += n
@@ -530,17 +566,14 @@ def run_reference(a, dist: Dist):
 
     x, logits = workloads.make_activations(w)
     weights = workloads.make_weights(w)
-    wq = oracle.quantize_weights_mxfp8(*weights) if w.precision == "mxfp8" else None
+    variant = oracle_variant(a)
+    wq = oracle_weights(w, weights, variant)
     ids, probs = oracle.route(logits[:live].numpy(), w.top_k)
     toks = workloads.sample_tokens(live, live, w.seed).numpy()
-    variant = oracle_variant(a)
 
     def step(n, start):
         sel = toks[(start + np.arange(n)) % live]
-        if wq is not None:
-            oracle.forward_mxfp8(x[:live], ids, probs, wq, tokens=sel, **(variant or {}))
-        else:
-            oracle.forward_bf16(x[:live], ids, probs, *weights, tokens=sel, **(variant or {}))
+        oracle_forward_tokens(w, x[:live], ids, probs, weights, wq, sel, variant)
 
     t0 = time.perf_counter()
     step(4, 0)
@@ -595,7 +628,7 @@ def main():
                 "impl": "reference", "metric": "routed tokens/s", "value": res["value"], "unit": "tokens/s",
                 "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup, "ms_per_step": res["ms_per_step"],
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": w.precision if w.precision != "mxfp8" else "mxfp8", "data": "synthetic",
+                "dtype": w.precision, "data": "synthetic",
                 "config": workload_config(w, live, a),
                 "cpu_baseline": {"value": res["value"], "unit": "tokens/s", "cores": oracle.threads(),
                                  "kind": "oracle",
@@ -620,7 +653,7 @@ def main():
         "ms_per_step_with_stage_events": round(res["ms_per_step_with_stage_events"], 5),
         "prepare_weights_ms": round(res["prepare_ms"], 4),
         "clocks": res["clocks"],
-        "gpu_launches": KERNELS_PER_FORWARD * a.steps,
+        "gpu_launches": kernels_per_forward(w.precision, w.capacity) * a.steps,
         "device_status": res["status"],
         "routing": {"routes": res["routes"], "experts_touched": res["touched"],
                     "max_rows_per_expert": res["max_rows_per_expert"]},
