@@ -142,9 +142,10 @@ def test_forward_ragged_shapes(H, F, E, k, T, cap):
 @pytest.mark.parametrize("precision", ["bf16", "mxfp8"])
 def test_small_plan_permute_matches_three_pass_permute(precision):
     """Plans of at most 1,024 live rows permute in one block; larger plans in
-    three passes (per-block histogram, scan, per-block scatter).  The same
-    routes through both give the same permutation, padded rows, tile list and
-    output, bit for bit, on a skewed load with a ragged last chunk."""
+    three passes (per-block histogram, scan, per-block scatter).  Both forms
+    give the oracle's permutation, and the same tokens the same output bit for
+    bit, on a skewed load with a ragged last chunk; the three-pass plan keeps
+    the shared tokens' outputs bit for bit across live counts 1,000..1,100."""
     H, F, E, k, T = 256, 192, 24, 4, 1000
     x, logits, weights = workloads.small_case(H, F, E, k, T, seed=2024, capacity=4096, zipf=True)
     small = GpuMoe(H, F, E, k, 4096, weights, precision=precision, max_live=1024)
@@ -161,6 +162,17 @@ def test_small_plan_permute_matches_three_pass_permute(precision):
         assert np.array_equal(small.read_i32(vs[name], count), large.read_i32(vl[name], count)), name
     ref_ids, _ = oracle.route(logits[:T].numpy(), k)
     _check_permutation(small, ref_ids, E, align=32 if precision == "bf16" else 128)
+    # the three-pass plan across live counts around the one-block plans' limit: the shared
+    # tokens' outputs agree bit for bit and every permutation is the oracle's
+    x2, logits2, _ = workloads.small_case(H, F, E, k, 1100, seed=2024, capacity=4096, zipf=True)
+    outs = {}
+    for n in (1000, 1024, 1025, 1100):
+        outs[n] = large.forward(x2.cuda(), n, logits=logits2.cuda()).cpu().numpy()
+        assert large.status() == 0
+        ids_n, _ = oracle.route(logits2[:n].numpy(), k)
+        _check_permutation(large, ids_n, E, align=32 if precision == "bf16" else 128)
+    for n in (1024, 1025, 1100):
+        assert np.array_equal(outs[n][:1000], outs[1000][:1000]), n
 
 
 @pytest.fixture(scope="module")
