@@ -25,7 +25,8 @@ import os
 __all__ = [
     "MoeError", "Plan", "load_library", "library_path", "moe_version", "moe_plan_create", "moe_plan_destroy",
     "moe_weight_buffer_bytes", "moe_workspace_bytes", "alloc_weight_buffer", "alloc_workspace",
-    "moe_prepare_weights", "mxfp8_quantize_block32", "nvfp4_quantize_block16", "moe_route_topk", "moe_forward", "moe_forward_with_events",
+    "moe_prepare_weights", "mxfp8_quantize_block32", "nvfp4_quantize_block16", "moe_route_topk", "moe_forward",
+    "moe_forward_with_events",
     "moe_forward_noalloc", "MOE_NOALLOC_SCRATCH_BYTES",
     "MOE_NUM_STAGES", "STAGE_NAMES",
     "moe_get_workspace_views", "moe_get_device_status", "moe_clear_device_status",

@@ -45,6 +45,7 @@ def test_version_and_status_strings():
     (dict(capacity=0), 2),
     (dict(max_live_rows=10 ** 9), 2),      # above capacity
     (dict(hidden=2056, precision="mxfp8"), 2),  # MXFP8 needs multiples of 32
+    (dict(ffn=1040, precision="nvfp4"), 2),     # so does NVFP4
 ])
 def test_plan_rejects_unsupported(kw, code):
     args = dict(hidden=2048, ffn=1024, num_experts=128, top_k=8, capacity=1024, precision="bf16")
@@ -152,3 +153,28 @@ def test_squared_relu_plans():
     assert lib.moe_prepare_weights(p.handle, fake, None, fake, fake, nb - 1, None) == 4
     q = rm.moe_plan_create(hidden=256, ffn=200, num_experts=8, top_k=2, capacity=64)
     assert lib.moe_prepare_weights(q.handle, fake, None, fake, fake, rm.moe_weight_buffer_bytes(q), None) == 1
+
+
+def test_nvfp4_plans_and_quantizer_arguments():
+    lib = rm.load_library()
+    E, H, F = 128, 2048, 1024
+    p4 = rm.moe_plan_create(hidden=H, ffn=F, num_experts=E, top_k=8, capacity=4096, precision="nvfp4")
+    p8 = rm.moe_plan_create(hidden=H, ffn=F, num_experts=E, top_k=8, capacity=4096, precision="mxfp8")
+    assert p4.precision == "nvfp4"
+    # weights: E2M1 codes (half a byte per element) + an E4M3 scale per 16 + fp32 scales [E][2]
+    w4 = rm.moe_weight_buffer_bytes(p4)
+    assert 3 * E * H * F * (0.5 + 1 / 16) <= w4 < 0.6 * rm.moe_weight_buffer_bytes(p8)
+    # workspace: NVFP4 adds the fp32 h rows and per-row scales to MXFP8's buffers
+    assert rm.moe_workspace_bytes(p4) > rm.moe_workspace_bytes(p8)
+    # squared-ReLU NVFP4 plans hold one FC1 projection
+    r4 = rm.moe_plan_create(hidden=H, ffn=F, num_experts=E, top_k=8, capacity=4096, precision="nvfp4",
+                            squared_relu=True)
+    assert rm.moe_weight_buffer_bytes(r4) < w4
+    fake = ctypes.c_void_p(1 << 20)
+    # nvfp4_quantize_block16(in, rows, cols, ld_in, q, scales, row_scales, live, stream)
+    assert lib.nvfp4_quantize_block16(fake, 4, 48, 48, fake, fake, fake, None, None) == 2   # cols % 32
+    assert lib.nvfp4_quantize_block16(fake, 4, 64, 32, fake, fake, fake, None, None) == 1   # ld_in < cols
+    assert lib.nvfp4_quantize_block16(fake, 4, 64, 64, fake, fake, None, None, None) == 1   # no row scales
+    assert lib.nvfp4_quantize_block16(ctypes.c_void_p((1 << 20) + 8), 4, 64, 64, fake, fake, fake, None,
+                                      None) == 3                                             # misaligned in
+    assert lib.nvfp4_quantize_block16(fake, 0, 64, 64, fake, fake, fake, None, None) == 0   # no rows: no-op
