@@ -38,7 +38,7 @@
 // completion is signalled to both CTAs' barriers (commit with a CTA mask);
 // warps 2-9 drain the accumulators and release each accumulator on CTA 0's
 // barrier.  Two accumulators of 256 fp32 columns (512 TMEM columns) per CTA.
-// The gate/up kernel has four more warps that copy the x rows of tiles of
+// The gate/up kernel has two more warps that copy the x rows of tiles of
 // more than 32 routes into their padded route rows while the MMAs run (the
 // dispatch fused into the GEMM: no separate gather pass over HBM).  They
 // claim 8-route chunks in tile order from a global counter and count each
@@ -58,7 +58,7 @@ namespace {
 
 constexpr int kStages = 3;
 constexpr int kEpiWarps = 8;
-constexpr int kCopyWarps = 4;                           // gate/up: x rows of large tiles into their route rows
+constexpr int kCopyWarps = 2;                           // gate/up: x rows of large tiles into their route rows
 constexpr int kPairM = 256;                             // M of the pair MMA (weight rows)
 constexpr int kAtoms = 2;                               // 64-element (128-byte) swizzle atoms per K stage
 constexpr int kStageK = kAtoms * kBK;                   // 128 K elements per stage
