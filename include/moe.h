@@ -16,7 +16,10 @@
  *   [P2] Megatron-LM PR #7798 (moe_training_matches_inference): "Background"
  *        (activation fused into FC1's epilogue, probabilities applied after
  *        FC2) and "What is changed" (a token's routes summed as fp32 fused
- *        multiply-adds of probability and row, from zero, in a fixed order).
+ *        multiply-adds of probability and row, from zero, in a fixed order);
+ *        "Per-token NVFP4" (TE's NVFP4BlockScaling recipe with row-scaled
+ *        activations, 1-D blocks, no Hadamard transform, no stochastic
+ *        rounding).
  *   [P3] Megatron-LM PR #8367 ("bound the FlashInfer MoE expert kernels by
  *        token count"): "Problem" -- the live token count is known only on
  *        the device; results are returned in fp32.
