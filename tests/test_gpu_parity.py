@@ -2,7 +2,7 @@
 
 Bit-exact: routed expert ids, the permutation (offsets, perm), MXFP8 codes
 and scales.  Floating point: the tolerance of tests/moe_testlib.py.
-Each test fails (never skips) when the library is missing on a GPU machine."""
+Each test fails (never skips) when the library is missing on a machine with a GPU."""
 from __future__ import annotations
 
 import numpy as np
