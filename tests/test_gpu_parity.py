@@ -91,6 +91,18 @@ def test_mxfp8_quantize_strided_and_live_bound():
 # ---------------------------------------------------------------- forward, bf16
 
 
+PRECISIONS = ("bf16", "mxfp8", "nvfp4")
+
+
+def _oracle_tokens(precision, x, ids, probs, weights):
+    """The oracle's output for caller routes in the given precision."""
+    if precision == "mxfp8":
+        return oracle.forward_mxfp8(x, ids, probs, oracle.quantize_weights_mxfp8(*weights))
+    if precision == "nvfp4":
+        return oracle.forward_nvfp4(x, ids, probs, oracle.quantize_weights_nvfp4(*weights))
+    return oracle.forward_bf16(x, ids, probs, *weights)
+
+
 def _check_permutation(m: GpuMoe, ref_ids, E, align=32):
     v = m.views()
     live, k = ref_ids.shape
@@ -276,10 +288,11 @@ def test_caller_routes_match_router_and_are_canonicalised():
     assert m.status() == 0
 
 
-def test_bad_routes_are_flagged_and_zeroed():
+@pytest.mark.parametrize("precision", PRECISIONS)
+def test_bad_routes_are_flagged_and_zeroed(precision):
     H, F, E, k, T = 256, 256, 8, 2, 10
     x, logits, weights = workloads.small_case(H, F, E, k, T, seed=6)
-    m = GpuMoe(H, F, E, k, T, weights)
+    m = GpuMoe(H, F, E, k, T, weights, precision=precision)
     ids, probs = oracle.route(logits.numpy(), k)
     ids[3] = [4, 4]      # repeated expert
     ids[5, 1] = E + 3    # out of range
@@ -288,16 +301,17 @@ def test_bad_routes_are_flagged_and_zeroed():
     assert m.status() & rm.MOE_DEV_BAD_ROUTE
     assert torch.all(out[3] == 0) and torch.all(out[5] == 0)
     good = [t for t in range(T) if t not in (3, 5)]
-    ref = oracle.forward_bf16(x[good], ids[good], probs[good], *weights)
-    assert_close(out.numpy()[good], ref, "bf16", "good tokens next to bad ones")
+    ref = _oracle_tokens(precision, x[good], ids[good], probs[good], weights)
+    assert_close(out.numpy()[good], ref, precision, "good tokens next to bad ones")
 
 
-def test_live_count_out_of_range_is_clamped_and_flagged():
+@pytest.mark.parametrize("precision", PRECISIONS)
+def test_live_count_out_of_range_is_clamped_and_flagged(precision):
     H, F, E, k, cap = 128, 128, 8, 2, 40
     x, logits, weights = workloads.small_case(H, F, E, k, 32, seed=8, capacity=cap)
     x[32:] = 0.5  # finite rows past 32 so that a clamp to 40 stays checkable
     logits[32:] = torch.randn((cap - 32, E), generator=torch.Generator().manual_seed(9))
-    m = GpuMoe(H, F, E, k, cap, weights, max_live=36)
+    m = GpuMoe(H, F, E, k, cap, weights, precision=precision, max_live=36)
     m.clear_status()
     out = m.forward(x.cuda(), -5, logits=logits.cuda())
     torch.cuda.synchronize()
@@ -308,14 +322,15 @@ def test_live_count_out_of_range_is_clamped_and_flagged():
     out = m.forward(x.cuda(), 1000, logits=logits.cuda()).cpu()
     assert m.status() & rm.MOE_DEV_LIVE_CLAMPED
     assert not torch.isnan(out[:36]).any() and torch.isnan(out[36:]).all()
-    _, _, ref = oracle_forward(x, logits, weights, k, 36)
-    assert_close(out.numpy()[:36], ref, "bf16", "clamped")
+    _, _, ref = oracle_forward(x, logits, weights, k, 36, precision=precision)
+    assert_close(out.numpy()[:36], ref, precision, "clamped")
 
 
-def test_zero_live_rows_writes_nothing():
+@pytest.mark.parametrize("precision", PRECISIONS)
+def test_zero_live_rows_writes_nothing(precision):
     H, F, E, k, cap = 128, 128, 8, 2, 64
     x, logits, weights = workloads.small_case(H, F, E, k, 0, seed=10, capacity=cap)
-    m = GpuMoe(H, F, E, k, cap, weights)
+    m = GpuMoe(H, F, E, k, cap, weights, precision=precision)
     out = m.forward(x.cuda(), 0, logits=logits.cuda(), sentinel=3.0)
     torch.cuda.synchronize()
     assert torch.all(out == 3.0)
@@ -342,14 +357,17 @@ def test_refit_negative_control():
     assert torch.equal(refit, fresh) and not torch.equal(refit, a)
 
 
-def test_graph_capture_replay_with_device_live_counts():
+@pytest.mark.parametrize("precision", PRECISIONS)
+def test_graph_capture_replay_with_device_live_counts(precision):
     """One capture serves every live count: the sweep workload's shapes at a
     reduced buffer, replayed with live counts written between replays."""
     w = workloads.WORKLOADS["sweep"]
     H, F, E, k = w.hidden, w.ffn, w.num_experts, w.top_k
+    if precision != "bf16":  # smaller shapes: the block-scaled oracles decode every weight element per route
+        H, F, E, k = 512, 512, 32, 4
     cap = 8192
     x, logits, weights = workloads.small_case(H, F, E, k, 1024, seed=4, capacity=cap)
-    m = GpuMoe(H, F, E, k, cap, weights, max_live=1024)
+    m = GpuMoe(H, F, E, k, cap, weights, precision=precision, max_live=1024)
     xd, ld = x.cuda(), logits.cuda()
     out = torch.full((cap, H), float("nan"), device="cuda")
     live = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -376,8 +394,8 @@ def test_graph_capture_replay_with_device_live_counts():
         res[n] = o[:n].clone()
     assert torch.equal(res[64][:1], res[1]) and torch.equal(res[1024][:64], res[64])
     toks = workloads.sample_tokens(1024, 48, 4).numpy()
-    _, _, ref = oracle_forward(x, logits, weights, k, 1024, tokens=toks)
-    assert_close(res[1024].numpy()[toks], ref, "bf16", "graph replay")
+    _, _, ref = oracle_forward(x, logits, weights, k, 1024, tokens=toks, precision=precision)
+    assert_close(res[1024].numpy()[toks], ref, precision, "graph replay")
     del g
 
 
