@@ -99,7 +99,7 @@ def _with_canaries(n_bytes: int, pad: int = 4096):
     return full, full[pad:pad + n_bytes]
 
 
-@pytest.mark.parametrize("precision", ["bf16", "mxfp8"])
+@pytest.mark.parametrize("precision", ["bf16", "mxfp8", "nvfp4"])
 def test_canaries_around_every_written_buffer_survive(precision):
     H, F, E, k, T, cap = 320, 224, 12, 3, 300, 400
     x, logits, weights = workloads.small_case(H, F, E, k, T, seed=52, capacity=cap, zipf=True)
@@ -121,9 +121,10 @@ def test_canaries_around_every_written_buffer_survive(precision):
     assert rm.moe_get_device_status(ws) == 0
 
 
-@pytest.mark.parametrize("precision", ["bf16", "mxfp8"])
+@pytest.mark.parametrize("precision", ["bf16", "mxfp8", "nvfp4"])
 def test_outlier_tokens_match_the_oracle(precision):
-    # the pages' second input distribution: 5% of the tokens scaled by 30
+    # the pages' second input distribution: 5% of the tokens scaled by 30 (NVFP4's scale per
+    # token row keeps the other tokens' resolution)
     H, F, E, k, T = 256, 512, 16, 4, 400
     x, logits, weights = workloads.small_case(H, F, E, k, T, seed=53)
     rng = np.random.default_rng(53)
@@ -137,6 +138,8 @@ def test_outlier_tokens_match_the_oracle(precision):
     ids, probs = oracle.route(logits.numpy(), k)
     if precision == "bf16":
         ref = oracle.forward_bf16(x, ids, probs, *weights)
+    elif precision == "nvfp4":
+        ref = oracle.forward_nvfp4(x, ids, probs, oracle.quantize_weights_nvfp4(*weights))
     else:
         ref = oracle.forward_mxfp8(x, ids, probs, oracle.quantize_weights_mxfp8(*weights))
     got = out.cpu().numpy()
