@@ -113,7 +113,7 @@ typedef struct moe_plan moe_plan; /* opaque, host memory only */
 
 /* Validate `desc` and build a host-side plan (no device work, no device
  * allocation).  Rejected (MOE_ERR_UNSUPPORTED): H or F not a multiple of 8
- * (bf16) or of 32 (MXFP8); k < 1, k > 16 or k > E; E < 1 or E > 1024;
+ * (bf16) or of 32 (MXFP8, NVFP4); k < 1, k > 16 or k > E; E < 1 or E > 1024;
  * capacity < 1 or > 2^24 rows; max_live_rows < 0 or > capacity;
  * H > 16384 or F > 16384.  Rejected (MOE_ERR_INVALID_ARG): unknown flag
  * bits, a negative or non-finite gate_up_clamp. */
@@ -137,7 +137,9 @@ size_t moe_workspace_bytes(const moe_plan* plan);
  *                                      read and may be NULL)
  *   w_down [E, H, F]                  (down projection)
  * In MXFP8 the weights are quantised here (blocks of 32 along each GEMM's K:
- * H for gate/up, F for down).  Enqueued on `stream`; forwards enqueued later
+ * H for gate/up, F for down); in NVFP4 likewise (blocks of 16) with one
+ * second-level scale per expert matrix (W1 = gate and up together, W2), as
+ * nvfp4_quantize_block16 describes.  Enqueued on `stream`; forwards enqueued later
  * on the same stream see the new weights, forwards enqueued earlier finish
  * with the old ones.  Returns MOE_ERR_WORKSPACE_TOO_SMALL if buf_bytes <
  * moe_weight_buffer_bytes. */
@@ -200,8 +202,11 @@ moe_status moe_route_topk(const moe_plan* plan, const float* logits, const int* 
  *            sum over its routes j in ascending expert id of
  *            p_j * y_j as fp32 FMAs from 0.0f, where
  *            y_j = W_down[e_j] . (silu(W_gate[e_j] . x_t) * (W_up[e_j] . x_t))
- *            with the SwiGLU row rounded to bf16 (or re-quantised to MXFP8)
- *            and y_j kept in fp32.  Rows >= live count are not written.
+ *            with the SwiGLU row rounded to bf16 (or re-quantised to MXFP8,
+ *            or to NVFP4 with the row's own scale) and y_j kept in fp32; in
+ *            MXFP8 and NVFP4, x_t and the weights are quantised as their
+ *            quantisation entry points describe.  Rows >= live count are not
+ *            written.
  *            The plan's flags change this as MOE_FLAG_* states (bf16 out,
  *            probabilities applied in FC1), and gate_up_clamp clamps the
  *            two pre-activations before silu and the product.
