@@ -43,7 +43,7 @@ def _noalloc(plan, wbuf, x, logits, live, cap, H):
     return out.cpu()
 
 
-@pytest.mark.parametrize("precision", ["bf16", "mxfp8"])
+@pytest.mark.parametrize("precision", ["bf16", "mxfp8", "nvfp4"])
 def test_noalloc_matches_workspace_forward_on_consecutive_calls(precision):
     H, F, E, k, T, cap = 256, 512, 8, 2, 64, 80
     plan, wbuf, x, logits = _setup(H, F, E, k, T, cap, seed=101, precision=precision)
