@@ -1,7 +1,7 @@
 """GPU parity of the forward's variants (cudnn-frontend PR #448, the MoeEp
 options; Megatron-LM PR #8367, the output type): the router probability
 applied to the SwiGLU row (`apply_topk_in_fc1`), the gate/up clamp, and the
-bf16 finalize output, in bf16 and MXFP8, against the oracle's variants on
+bf16 finalize output, in bf16, MXFP8 and NVFP4, against the oracle's variants on
 the same inputs, with the tolerances of the plain forward.
 """
 from __future__ import annotations
@@ -40,10 +40,12 @@ def _run(precision, weights, x, logits, **variant):
 def _oracle(precision, x, ids, probs, weights, **variant):
     if precision == "bf16":
         return oracle.forward_bf16(x, ids, probs, *weights, **variant)
+    if precision == "nvfp4":
+        return oracle.forward_nvfp4(x, ids, probs, oracle.quantize_weights_nvfp4(*weights), **variant)
     return oracle.forward_mxfp8(x, ids, probs, oracle.quantize_weights_mxfp8(*weights), **variant)
 
 
-@pytest.mark.parametrize("precision", ["bf16", "mxfp8"])
+@pytest.mark.parametrize("precision", ["bf16", "mxfp8", "nvfp4"])
 def test_probs_in_fc1_matches_oracle(precision):
     x, logits, weights, ids, probs = _case(31)
     out = _run(precision, weights, x, logits, probs_in_fc1=True)
@@ -54,9 +56,10 @@ def test_probs_in_fc1_matches_oracle(precision):
     assert np.max(np.abs(ref - plain)) > 0
 
 
-@pytest.mark.parametrize("precision", ["bf16", "mxfp8"])
+@pytest.mark.parametrize("precision", ["bf16", "mxfp8", "nvfp4"])
 def test_probs_in_fc1_with_power_of_two_probs_is_bitwise_the_plain_forward(precision):
-    # scaling h by 2^-n commutes with its rounding / quantisation and scales the
+    # scaling h by 2^-n commutes with its rounding / quantisation (NVFP4: the row's
+    # scale takes the factor exactly, codes and block scales stay) and scales the
     # down GEMM's fp32 sums exactly, and acc + p*y is fmaf(p, y, acc)
     H, F, E, k, T = (SHAPE[c] for c in "HFEkT")
     x, _, weights, ids, _ = _case(32)
@@ -69,7 +72,7 @@ def test_probs_in_fc1_with_power_of_two_probs_is_bitwise_the_plain_forward(preci
     assert torch.equal(outs[0], outs[1])
 
 
-@pytest.mark.parametrize("precision", ["bf16", "mxfp8"])
+@pytest.mark.parametrize("precision", ["bf16", "mxfp8", "nvfp4"])
 def test_gate_up_clamp_matches_oracle(precision):
     x, logits, weights, ids, probs = _case(33)
     c = 0.5
@@ -80,7 +83,7 @@ def test_gate_up_clamp_matches_oracle(precision):
     assert np.max(np.abs(ref - plain)) > 1e-3 * np.sqrt(np.mean(plain.astype(np.float64) ** 2))
 
 
-@pytest.mark.parametrize("precision", ["bf16", "mxfp8"])
+@pytest.mark.parametrize("precision", ["bf16", "mxfp8", "nvfp4"])
 def test_bf16_output_is_the_fp32_output_rounded(precision):
     x, logits, weights, ids, probs = _case(34)
     out32 = _run(precision, weights, x, logits)
@@ -115,7 +118,7 @@ def test_all_variants_together_on_the_decode_workload():
 # ---------------------------------------------------------------- squared-ReLU experts (bf16)
 
 
-@pytest.mark.parametrize("precision", ["bf16", "mxfp8"])
+@pytest.mark.parametrize("precision", ["bf16", "mxfp8", "nvfp4"])
 def test_squared_relu_matches_oracle(precision):
     x, logits, weights, ids, probs = _case(35)
     wg, _, wd = weights
@@ -126,6 +129,9 @@ def test_squared_relu_matches_oracle(precision):
     assert m.status() == 0
     if precision == "bf16":
         ref = oracle.forward_bf16(x, ids, probs, wg, None, wd, squared_relu=True)
+    elif precision == "nvfp4":
+        # one FC1 matrix (the gate rows) with its own second-level scale
+        ref = oracle.forward_nvfp4(x, ids, probs, oracle.quantize_weights_nvfp4(wg, None, wd), squared_relu=True)
     else:
         # the oracle's MXFP8 path quantises W1 as its gate rows; the up rows are not used
         ref = oracle.forward_mxfp8(x, ids, probs, oracle.quantize_weights_mxfp8(wg, wg, wd), squared_relu=True)
