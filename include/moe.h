@@ -261,6 +261,67 @@ moe_status moe_forward_with_events(const moe_plan* plan, const void* x, const fl
                                    void* out, void* workspace, size_t ws_bytes, void* stream,
                                    void* const* stage_events);
 
+/* Expert parallelism ([P2] "What is changed" and "Limitations"; [P5]: a
+ * variable-size all-to-all of route rows, local experts, a top-k combine).
+ * The E experts are split into ep_size equal contiguous ranges; EP rank g
+ * owns experts [g*E/ep_size, (g+1)*E/ep_size).  One step on each rank:
+ *   1. moe_ep_dispatch with the rank's own tokens and its full-E plan: route,
+ *      order the routes by expert, pack one send row per route;
+ *   2. exchange send_counts, then the first sum(send_counts) send rows
+ *      (x, ids, probs) with an all-to-all: the rows for rank g are the g-th
+ *      run of send_counts[g] rows (the caller's collective, e.g. NCCL);
+ *   3. on the receiving rank, moe_forward of a plan with the E/ep_size local
+ *      experts, top_k 1, fp32 output and the same precision, flags (but
+ *      MOE_FLAG_OUT_BF16) and clamp, over the received rows as tokens with
+ *      ids = received ids and probs = received probs: its output rows are
+ *      the routes' expert outputs y (each row a top-1 token whose weight
+ *      multiplies y exactly: 1.0, or its probability under
+ *      MOE_FLAG_PROBS_IN_FC1, which the FC1 epilogue then applies);
+ *   4. return those rows with the reverse all-to-all, so that send row r
+ *      gets back its route's y row at row r;
+ *   5. moe_ep_combine with the full-E plan.
+ * The output of step 5 is bitwise the one-GPU moe_forward's for the same
+ * tokens, whatever ep_size: each y row is one route's arithmetic whatever
+ * launch computes it, and the combine is the same ascending-id fp32 FMA chain
+ * (the pages' generation combine adds per-rank partials and is not
+ * EP-invariant). */
+
+/* Send side (step 1).  plan: the source rank's plan (all E experts).
+ *   ep_size  1 .. 128, dividing E; MOE_ERR_UNSUPPORTED otherwise.
+ *   x, logits / ids + probs, live_count_dev, workspace: as moe_forward.
+ *   send_x       bf16 [max_live_rows * k, H], 16-byte aligned: row r is the
+ *                x row of the r-th live route in expert order (stable by
+ *                token within an expert); rows >= the route count are not
+ *                written.
+ *   send_ids     int32 [max_live_rows * k]: row r's expert id local to its
+ *                owning rank (e mod E/ep_size).
+ *   send_probs   fp32 [max_live_rows * k]: row r's weight in the receiving
+ *                forward: 1.0, or the route's probability under
+ *                MOE_FLAG_PROBS_IN_FC1.
+ *   send_counts  int32 [ep_size]: rows for each destination rank, in rank
+ *                order (they sum to the live route count).
+ *   route_rows   int32 [max_live_rows, k]: the send row of route (t, j) of
+ *                live token t in canonical (ascending id) order; -1 for the
+ *                routes of a dropped token (a caller id out of range or
+ *                repeated, flagged MOE_DEV_BAD_ROUTE).
+ *   route_probs  fp32 [max_live_rows, k]: the route's combine weight (its
+ *                probability, or 1.0 under MOE_FLAG_PROBS_IN_FC1).
+ * All outputs are device memory the caller owns; rows of tokens >= the live
+ * count are not written. */
+moe_status moe_ep_dispatch(const moe_plan* plan, int ep_size, const void* x, const float* logits, const int* ids,
+                           const float* probs, const int* live_count_dev, void* send_x, int* send_ids,
+                           float* send_probs, int* send_counts, int* route_rows, float* route_probs,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* Combine (step 5).  plan: the source rank's plan.  y_rows fp32 [rows, H],
+ * 16-byte aligned, row r = the returned y of send row r.  out (fp32, or bf16
+ * under MOE_FLAG_OUT_BF16) [capacity, H]: row t < live count gets the sum
+ * over j in ascending expert id of route_probs[t,j] * y_rows[route_rows[t,j]]
+ * as fp32 FMAs from 0.0f (routes with row -1 skipped), as moe_forward's
+ * combine; rows >= the live count are not written. */
+moe_status moe_ep_combine(const moe_plan* plan, const float* y_rows, const int* route_rows,
+                          const float* route_probs, const int* live_count_dev, void* out, void* stream);
+
 /* Views into a workspace after a forward (device pointers into it), for
  * tests and diagnostics:
  *   route_ids/route_probs [max_live, k]: canonical routes of the last forward

@@ -27,7 +27,7 @@ __all__ = [
     "moe_weight_buffer_bytes", "moe_workspace_bytes", "alloc_weight_buffer", "alloc_workspace",
     "moe_prepare_weights", "mxfp8_quantize_block32", "nvfp4_quantize_block16", "moe_route_topk", "moe_forward",
     "moe_forward_with_events",
-    "moe_forward_noalloc", "MOE_NOALLOC_SCRATCH_BYTES",
+    "moe_forward_noalloc", "MOE_NOALLOC_SCRATCH_BYTES", "moe_ep_dispatch", "moe_ep_combine",
     "MOE_NUM_STAGES", "STAGE_NAMES",
     "moe_get_workspace_views", "moe_get_device_status", "moe_clear_device_status",
     "MOE_DEV_LIVE_CLAMPED", "MOE_DEV_BAD_ROUTE", "MOE_DEV_TIMEOUT",
@@ -92,6 +92,8 @@ def load_library():
         "moe_forward": ([P, P, P, P, P, P, P, P, P, SZ, P], I),
         "moe_forward_with_events": ([P, P, P, P, P, P, P, P, P, SZ, P, ctypes.POINTER(P)], I),
         "moe_forward_noalloc": ([P, P, P, P, P, P, P, P, P], I),
+        "moe_ep_dispatch": ([P, I, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P], I),
+        "moe_ep_combine": ([P, P, P, P, P, P, P], I),
         "moe_get_workspace_views": ([P, P, ctypes.POINTER(_Views)], I),
         "moe_get_device_status": ([P, ctypes.POINTER(ctypes.c_uint), P], I),
         "moe_clear_device_status": ([P, P], I),
@@ -276,6 +278,25 @@ def moe_forward_noalloc(plan: Plan, x, kernel_buf, live_count, out, logits=None,
     _check(load_library().moe_forward_noalloc(plan.handle, _ptr(x), _ptr(logits), _ptr(ids), _ptr(probs),
                                               _ptr(kernel_buf), _ptr(live_count), _ptr(out), _stream(stream)),
            "moe_forward_noalloc")
+
+
+def moe_ep_dispatch(plan: Plan, ep_size: int, x, live_count, send_x, send_ids, send_probs, send_counts, route_rows,
+                    route_probs, workspace, logits=None, ids=None, probs=None, stream=None) -> None:
+    """Expert-parallel send side (include/moe.h): route, order by expert, pack one
+    send row per live route.  `ep.py` composes it into a whole step."""
+    _check(load_library().moe_ep_dispatch(plan.handle, int(ep_size), _ptr(x), _ptr(logits), _ptr(ids), _ptr(probs),
+                                          _ptr(live_count), _ptr(send_x), _ptr(send_ids), _ptr(send_probs),
+                                          _ptr(send_counts), _ptr(route_rows), _ptr(route_probs), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream(stream)),
+           "moe_ep_dispatch")
+
+
+def moe_ep_combine(plan: Plan, y_rows, route_rows, route_probs, live_count, out, stream=None) -> None:
+    """Expert-parallel combine: out[t] = sum over j (ascending expert id) of
+    route_probs[t, j] * y_rows[route_rows[t, j]] as fp32 FMAs from zero."""
+    _check_out(plan, out)
+    _check(load_library().moe_ep_combine(plan.handle, _ptr(y_rows), _ptr(route_rows), _ptr(route_probs),
+                                         _ptr(live_count), _ptr(out), _stream(stream)), "moe_ep_combine")
 
 
 MOE_NUM_STAGES = 6

@@ -505,6 +505,60 @@ moe_status moe_forward_with_events(const moe_plan* plan, const void* x, const fl
                         stage_events);
 }
 
+// Expert-parallel send side: the forward's route (or canonicalisation) and
+// permute stages into the workspace, then the pack kernel.
+moe_status moe_ep_dispatch(const moe_plan* plan, int ep_size, const void* x, const float* logits, const int* ids,
+                           const float* probs, const int* live_count_dev, void* send_x, int* send_ids,
+                           float* send_probs, int* send_counts, int* route_rows, float* route_probs,
+                           void* workspace, size_t ws_bytes, void* stream) {
+    if (plan == nullptr || x == nullptr || live_count_dev == nullptr || send_x == nullptr || send_ids == nullptr ||
+        send_probs == nullptr || send_counts == nullptr || route_rows == nullptr || route_probs == nullptr ||
+        workspace == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    const bool have_logits = logits != nullptr;
+    const bool have_routes = ids != nullptr && probs != nullptr;
+    if (have_logits == have_routes || ((ids == nullptr) != (probs == nullptr))) return MOE_ERR_INVALID_ARG;
+    const int H = plan->d.hidden, E = plan->d.num_experts, k = plan->d.top_k;
+    if (ep_size < 1 || ep_size > ep_max_size() || E % ep_size != 0) return MOE_ERR_UNSUPPORTED;
+    if (ws_bytes < plan->ws.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned(x, 16) || !aligned(send_x, 16) || !aligned(workspace, 256)) return MOE_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int max_live = (int)plan->max_live;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const WsLayout& L = plan->ws;
+    unsigned* status = reinterpret_cast<unsigned*>(ws + L.status);
+    int* r_ids = reinterpret_cast<int*>(ws + L.r_ids);
+    float* r_probs = reinterpret_cast<float*>(ws + L.r_probs);
+    const bool blockscaled = plan->d.precision != MOE_BF16;
+    cudaError_t e = have_logits ? launch_route_topk(logits, live_count_dev, max_live, E, k, r_ids, r_probs, status, s)
+                                : launch_canon_routes(ids, probs, live_count_dev, max_live, E, k, r_ids, r_probs,
+                                                      status, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    int* inv = reinterpret_cast<int*>(ws + L.inv);
+    int* offsets = reinterpret_cast<int*>(ws + L.offsets);
+    int* padoff = reinterpret_cast<int*>(ws + L.padoff);
+    e = launch_permute(plan, live_count_dev, r_ids, reinterpret_cast<int*>(ws + L.blkcnt), offsets, padoff,
+                       reinterpret_cast<int4*>(ws + L.tiles), reinterpret_cast<int*>(ws + L.perm), inv,
+                       blockscaled ? nullptr : reinterpret_cast<int*>(ws + L.ready), status, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    e = launch_ep_pack(x, live_count_dev, max_live, H, k, r_ids, r_probs, inv, offsets, padoff, E, ep_size,
+                       (plan->d.flags & MOE_FLAG_PROBS_IN_FC1) != 0, send_x, send_ids, send_probs, send_counts,
+                       route_rows, route_probs, s);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_ep_combine(const moe_plan* plan, const float* y_rows, const int* route_rows,
+                          const float* route_probs, const int* live_count_dev, void* out, void* stream) {
+    if (plan == nullptr || y_rows == nullptr || route_rows == nullptr || route_probs == nullptr ||
+        live_count_dev == nullptr || out == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned(y_rows, 16) || !aligned(out, 16)) return MOE_ERR_ALIGNMENT;
+    const cudaError_t e = launch_combine(y_rows, route_rows, route_probs, live_count_dev, (int)plan->max_live,
+                                         plan->d.hidden, plan->d.top_k, out,
+                                         (plan->d.flags & MOE_FLAG_OUT_BF16) != 0, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status moe_get_workspace_views(const moe_plan* plan, const void* workspace, moe_workspace_views* v) {
     if (plan == nullptr || workspace == nullptr || v == nullptr) return MOE_ERR_INVALID_ARG;
     const uint8_t* ws = static_cast<const uint8_t*>(workspace);

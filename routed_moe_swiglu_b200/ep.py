@@ -1,0 +1,178 @@
+"""Expert parallelism: one routed-MoE step over ep_size ranks, each holding the
+weights of E/ep_size contiguous experts.
+
+The sequence (include/moe.h, "Expert parallelism") is:
+  1. ``moe_ep_dispatch`` routes the rank's own tokens and packs one send row per
+     route, in expert order, so the rows for rank g are one run;
+  2. all-to-alls of the counts and then of the rows (x, local expert ids,
+     FC1 weights);
+  3. the rank's own experts run ``moe_forward`` over the received rows as top-1
+     tokens, whose output rows are the routes' expert outputs y;
+  4. the reverse all-to-all brings each y row back to its send row;
+  5. ``moe_ep_combine`` adds each token's routes in ascending expert id.
+
+The result is bitwise the one-GPU forward's, for any EP size (Megatron-LM PR
+#7798, "What is changed": the expert kernel computes every dispatched row as a
+top-1 token with probability 1.0; its "Limitations": generation's combine adds
+rank partials and is not EP-invariant, which the ascending-id combine here
+is).  cudnn-frontend PR #448 (MoeEp API) names the same parts: a variable-size
+all-to-all dispatch, local experts and a top-k combine.
+
+The exchanges are ``torch.distributed`` all-to-alls (NCCL over NVLink between
+GPUs), which need the row counts on the host: step 2 reads them back, as an
+all-to-all dispatcher does.  Every other step is the library's kernels; this
+module only sequences them and moves bytes.
+
+The phases (``dispatch``, ``expert_forward``, ``combine``) are separate so that
+a driver other than ``moe_forward_ep`` can run the exchange itself.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+from . import (MoeError, Plan, alloc_workspace, moe_ep_combine, moe_ep_dispatch, moe_forward, moe_plan_create)
+
+__all__ = ["expert_range", "shard_plan_create", "EpBuffers", "dispatch", "expert_forward", "combine",
+           "exchange_counts", "exchange_rows", "moe_forward_ep"]
+
+
+def expert_range(num_experts: int, ep_size: int, rank: int) -> tuple[int, int]:
+    """(first expert, number of experts) owned by EP rank `rank`."""
+    if ep_size < 1 or num_experts % ep_size != 0:
+        raise ValueError(f"ep_size {ep_size} must divide the {num_experts} experts")
+    if not 0 <= rank < ep_size:
+        raise ValueError(f"rank {rank} outside [0, {ep_size})")
+    per = num_experts // ep_size
+    return rank * per, per
+
+
+def shard_plan_create(plan: Plan, ep_size: int, max_recv_rows: int) -> Plan:
+    """The plan of one rank's experts: E/ep_size experts, top-1 routes, fp32
+    output, the source plan's precision, FC1 flags and clamp; `max_recv_rows`
+    bounds the rows one step may bring to the rank (at most ep_size times the
+    source plan's live rows times k)."""
+    expert_range(plan.num_experts, ep_size, 0)
+    return moe_plan_create(hidden=plan.hidden, ffn=plan.ffn, num_experts=plan.num_experts // ep_size, top_k=1,
+                           capacity=max_recv_rows, precision=plan.precision, out_dtype="fp32",
+                           probs_in_fc1=plan.probs_in_fc1, gate_up_clamp=plan.gate_up_clamp or None,
+                           squared_relu=plan.squared_relu)
+
+
+@dataclass
+class EpBuffers:
+    """Device buffers of one rank's EP step (sizes from the two plans)."""
+    ep_size: int
+    workspace: object      # the source plan's workspace
+    send_x: object         # bf16 [max_live * k, H]
+    send_ids: object       # int32 [max_live * k]
+    send_probs: object     # fp32 [max_live * k]
+    send_counts: object    # int32 [ep_size]
+    route_rows: object     # int32 [max_live, k]
+    route_probs: object    # fp32 [max_live, k]
+    y_back: object         # fp32 [max_live * k, H]
+    recv_x: object         # bf16 [max_recv, H]
+    recv_ids: object       # int32 [max_recv, 1]
+    recv_probs: object     # fp32 [max_recv, 1]
+    recv_y: object         # fp32 [max_recv, H]
+    recv_live: object      # int32 [1]
+    shard_workspace: object
+
+    @classmethod
+    def allocate(cls, plan: Plan, shard: Plan, ep_size: int, device=None) -> "EpBuffers":
+        import torch
+
+        dev = device or "cuda"
+        routes = plan.max_live_rows * plan.top_k
+        recv = shard.capacity
+        H = plan.hidden
+        return cls(ep_size=ep_size, workspace=alloc_workspace(plan, dev),
+                   send_x=torch.empty(routes, H, dtype=torch.bfloat16, device=dev),
+                   send_ids=torch.empty(routes, dtype=torch.int32, device=dev),
+                   send_probs=torch.empty(routes, dtype=torch.float32, device=dev),
+                   send_counts=torch.empty(ep_size, dtype=torch.int32, device=dev),
+                   route_rows=torch.empty(plan.max_live_rows, plan.top_k, dtype=torch.int32, device=dev),
+                   route_probs=torch.empty(plan.max_live_rows, plan.top_k, dtype=torch.float32, device=dev),
+                   y_back=torch.empty(routes, H, dtype=torch.float32, device=dev),
+                   recv_x=torch.empty(recv, H, dtype=torch.bfloat16, device=dev),
+                   recv_ids=torch.empty(recv, 1, dtype=torch.int32, device=dev),
+                   recv_probs=torch.empty(recv, 1, dtype=torch.float32, device=dev),
+                   recv_y=torch.empty(recv, H, dtype=torch.float32, device=dev),
+                   recv_live=torch.zeros(1, dtype=torch.int32, device=dev),
+                   shard_workspace=alloc_workspace(shard, dev))
+
+
+def dispatch(plan: Plan, bufs: EpBuffers, x, live_count, logits=None, ids=None, probs=None, stream=None) -> None:
+    """Step 1: fills send_x / send_ids / send_probs / send_counts / route_rows /
+    route_probs of `bufs` for the rank's live tokens."""
+    moe_ep_dispatch(plan, bufs.ep_size, x, live_count, bufs.send_x, bufs.send_ids, bufs.send_probs, bufs.send_counts,
+                    bufs.route_rows, bufs.route_probs, bufs.workspace, logits=logits, ids=ids, probs=probs,
+                    stream=stream)
+
+
+def expert_forward(shard: Plan, bufs: EpBuffers, shard_wbuf, n_recv: int, stream=None) -> None:
+    """Step 3: the rank's experts over the first `n_recv` rows of recv_x (their
+    local ids and FC1 weights in recv_ids / recv_probs) into recv_y."""
+    if n_recv > shard.capacity:
+        raise MoeError(4, f"{n_recv} received rows exceed the expert plan's {shard.capacity}")
+    bufs.recv_live.fill_(n_recv)
+    moe_forward(shard, bufs.recv_x, shard_wbuf, bufs.recv_live, bufs.recv_y, bufs.shard_workspace,
+                ids=bufs.recv_ids, probs=bufs.recv_probs, stream=stream)
+
+
+def combine(plan: Plan, bufs: EpBuffers, live_count, out, stream=None) -> None:
+    """Step 5: out rows of the rank's live tokens from the returned y rows."""
+    moe_ep_combine(plan, bufs.y_back, bufs.route_rows, bufs.route_probs, live_count, out, stream=stream)
+
+
+def exchange_counts(send_counts, group=None):
+    """All-to-all of one count per rank pair: returns recv_counts, where
+    recv_counts[s] is what rank s sends to this rank."""
+    import torch
+    import torch.distributed as dist
+
+    recv = torch.empty_like(send_counts)
+    dist.all_to_all_single(recv, send_counts, group=group)
+    return recv
+
+
+def exchange_rows(send, send_splits: list[int], recv_splits: list[int], recv, group=None):
+    """All-to-all of rows: send[:sum(send_splits)] goes out in runs of
+    send_splits[g] rows to rank g; the runs from ranks 0, 1, ... land in
+    recv[:sum(recv_splits)] in rank order.  bf16 rows move as their bytes
+    (uint8), which every backend copies as is.  Returns that view of `recv`."""
+    import torch
+    import torch.distributed as dist
+
+    n_out = sum(recv_splits)
+    if n_out > recv.shape[0]:
+        raise MoeError(4, f"{n_out} rows to receive exceed the buffer's {recv.shape[0]}")
+    src = send[:sum(send_splits)]
+    dst = recv[:n_out]
+    if src.dtype == torch.bfloat16:
+        src, dst = src.view(torch.uint8), dst.view(torch.uint8)
+    dist.all_to_all_single(dst, src, output_split_sizes=list(recv_splits), input_split_sizes=list(send_splits),
+                           group=group)
+    return recv[:n_out]
+
+
+def moe_forward_ep(plan: Plan, shard: Plan, bufs: EpBuffers, x, shard_wbuf, live_count, out, group=None,
+                   logits=None, ids=None, probs=None, stream=None) -> None:
+    """One EP step on this rank (every rank of `group` calls it together):
+    `x`, `live_count`, `logits` or `ids` + `probs` and `out` are the rank's own
+    tokens as for ``moe_forward`` with `plan`; `shard_wbuf` holds the rank's
+    experts, prepared with `shard` (``shard_plan_create``)."""
+    import torch.distributed as dist
+
+    if dist.get_world_size(group) != bufs.ep_size:
+        raise ValueError(f"group has {dist.get_world_size(group)} ranks, buffers are for {bufs.ep_size}")
+    dispatch(plan, bufs, x, live_count, logits=logits, ids=ids, probs=probs, stream=stream)
+    recv_counts = exchange_counts(bufs.send_counts, group)
+    send_splits = bufs.send_counts.tolist()  # the host needs the split sizes
+    recv_splits = recv_counts.tolist()
+    n_recv = sum(recv_splits)
+    exchange_rows(bufs.send_x, send_splits, recv_splits, bufs.recv_x, group)
+    exchange_rows(bufs.send_ids, send_splits, recv_splits, bufs.recv_ids.view(-1), group)
+    exchange_rows(bufs.send_probs, send_splits, recv_splits, bufs.recv_probs.view(-1), group)
+    expert_forward(shard, bufs, shard_wbuf, n_recv, stream=stream)
+    exchange_rows(bufs.recv_y, recv_splits, send_splits, bufs.y_back, group)
+    combine(plan, bufs, live_count, out, stream=stream)

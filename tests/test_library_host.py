@@ -178,3 +178,27 @@ def test_nvfp4_plans_and_quantizer_arguments():
     assert lib.nvfp4_quantize_block16(ctypes.c_void_p((1 << 20) + 8), 4, 64, 64, fake, fake, fake, None,
                                       None) == 3                                             # misaligned in
     assert lib.nvfp4_quantize_block16(fake, 0, 64, 64, fake, fake, fake, None, None) == 0   # no rows: no-op
+
+
+def test_ep_entries_reject_bad_arguments_before_launch():
+    lib = rm.load_library()
+    p = rm.moe_plan_create(hidden=256, ffn=512, num_experts=8, top_k=2, capacity=64)
+    f = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    ws = rm.moe_workspace_bytes(p)
+    null = None
+
+    def dispatch(ep=2, x=f, logits=f, ids=null, probs=null, send_x=f, counts=f, wsb=ws):
+        return lib.moe_ep_dispatch(p.handle, ep, x, logits, ids, probs, f, send_x, f, f, counts, f, f, f, wsb, null)
+
+    assert dispatch(ep=3) == 2            # 3 does not divide the 8 experts
+    assert dispatch(ep=0) == 2
+    assert dispatch(ep=16) == 2           # more ranks than experts
+    assert dispatch(logits=null) == 1     # no routing input
+    assert dispatch(ids=f) == 1           # ids without probs, and logits too
+    assert dispatch(counts=null) == 1
+    assert dispatch(wsb=ws - 1) == 4
+    assert dispatch(send_x=ctypes.c_void_p((1 << 20) + 8)) == 3
+    assert dispatch(x=ctypes.c_void_p((1 << 20) + 2)) == 3
+    assert lib.moe_ep_combine(p.handle, f, f, f, f, null, null) == 1
+    assert lib.moe_ep_combine(None, f, f, f, f, f, null) == 1
+    assert lib.moe_ep_combine(p.handle, ctypes.c_void_p((1 << 20) + 4), f, f, f, f, null) == 3
