@@ -188,3 +188,36 @@ def test_ep_caller_routes_with_a_dropped_token():
     assert torch.all(ranks[0].out[17] == 0)
     assert rm.moe_get_device_status(ranks[0].bufs.workspace) & rm.MOE_DEV_BAD_ROUTE
     assert sum(sum(c) for c in counts) == (T - 1) * K
+
+
+def test_ep_step_through_nccl_with_one_rank():
+    """moe_forward_ep itself over a one-rank NCCL group (each all-to-all is a
+    copy to itself): the NCCL calls on device buffers, the host split sizes and
+    the phases in sequence give the one-GPU forward's output bit for bit."""
+    import socket
+
+    import torch.distributed as dist
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True)
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1)
+    try:
+        T = 500
+        x, logits, weights = workloads.small_case(H, F, E, K, T, seed=35, zipf=True)
+        for precision in ("bf16", "mxfp8"):
+            plan = rm.moe_plan_create(hidden=H, ffn=F, num_experts=E, top_k=K, capacity=T, precision=precision)
+            shard = moe_ep.shard_plan_create(plan, 1, T * K)
+            wbuf = rm.alloc_weight_buffer(shard)
+            rm.moe_prepare_weights(shard, *(w.cuda() for w in weights), wbuf)
+            bufs = moe_ep.EpBuffers.allocate(plan, shard, 1)
+            out = torch.full((T, H), float("nan"), device="cuda")
+            live = torch.tensor([T], dtype=torch.int32, device="cuda")
+            moe_ep.moe_forward_ep(plan, shard, bufs, x.cuda(), wbuf, live, out, logits=logits.cuda())
+            torch.cuda.synchronize()
+            ref, _ = _one_gpu(precision, x, logits, weights, T)
+            assert torch.equal(out.view(torch.int32), ref.view(torch.int32)), precision
+            assert bufs.send_counts.tolist() == [T * K]
+    finally:
+        dist.destroy_process_group()
