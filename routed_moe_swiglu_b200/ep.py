@@ -28,6 +28,7 @@ a driver other than ``moe_forward_ep`` can run the exchange itself.
 """
 from __future__ import annotations
 
+import contextlib
 from dataclasses import dataclass
 
 from . import (MoeError, Plan, alloc_workspace, moe_ep_combine, moe_ep_dispatch, moe_forward, moe_plan_create)
@@ -101,6 +102,15 @@ class EpBuffers:
                    shard_workspace=alloc_workspace(shard, dev))
 
 
+def _on(stream):
+    """Context that makes `stream` (a torch.cuda.Stream, or None for the
+    current one) torch's current stream, so that tensor ops and collectives
+    are ordered with the library calls on it."""
+    import torch
+
+    return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+
+
 def dispatch(plan: Plan, bufs: EpBuffers, x, live_count, logits=None, ids=None, probs=None, stream=None) -> None:
     """Step 1: fills send_x / send_ids / send_probs / send_counts / route_rows /
     route_probs of `bufs` for the rank's live tokens."""
@@ -114,7 +124,8 @@ def expert_forward(shard: Plan, bufs: EpBuffers, shard_wbuf, n_recv: int, stream
     local ids and FC1 weights in recv_ids / recv_probs) into recv_y."""
     if n_recv > shard.capacity:
         raise MoeError(4, f"{n_recv} received rows exceed the expert plan's {shard.capacity}")
-    bufs.recv_live.fill_(n_recv)
+    with _on(stream):
+        bufs.recv_live.fill_(n_recv)
     moe_forward(shard, bufs.recv_x, shard_wbuf, bufs.recv_live, bufs.recv_y, bufs.shard_workspace,
                 ids=bufs.recv_ids, probs=bufs.recv_probs, stream=stream)
 
@@ -160,19 +171,21 @@ def moe_forward_ep(plan: Plan, shard: Plan, bufs: EpBuffers, x, shard_wbuf, live
     """One EP step on this rank (every rank of `group` calls it together):
     `x`, `live_count`, `logits` or `ids` + `probs` and `out` are the rank's own
     tokens as for ``moe_forward`` with `plan`; `shard_wbuf` holds the rank's
-    experts, prepared with `shard` (``shard_plan_create``)."""
+    experts, prepared with `shard` (``shard_plan_create``).  `stream`: a
+    torch.cuda.Stream for the whole step (default: the current stream)."""
     import torch.distributed as dist
 
     if dist.get_world_size(group) != bufs.ep_size:
         raise ValueError(f"group has {dist.get_world_size(group)} ranks, buffers are for {bufs.ep_size}")
-    dispatch(plan, bufs, x, live_count, logits=logits, ids=ids, probs=probs, stream=stream)
-    recv_counts = exchange_counts(bufs.send_counts, group)
-    send_splits = bufs.send_counts.tolist()  # the host needs the split sizes
-    recv_splits = recv_counts.tolist()
-    n_recv = sum(recv_splits)
-    exchange_rows(bufs.send_x, send_splits, recv_splits, bufs.recv_x, group)
-    exchange_rows(bufs.send_ids, send_splits, recv_splits, bufs.recv_ids.view(-1), group)
-    exchange_rows(bufs.send_probs, send_splits, recv_splits, bufs.recv_probs.view(-1), group)
-    expert_forward(shard, bufs, shard_wbuf, n_recv, stream=stream)
-    exchange_rows(bufs.recv_y, recv_splits, send_splits, bufs.y_back, group)
-    combine(plan, bufs, live_count, out, stream=stream)
+    with _on(stream):  # every step below on one stream, in order
+        dispatch(plan, bufs, x, live_count, logits=logits, ids=ids, probs=probs)
+        recv_counts = exchange_counts(bufs.send_counts, group)
+        send_splits = bufs.send_counts.tolist()  # the host needs the split sizes
+        recv_splits = recv_counts.tolist()
+        n_recv = sum(recv_splits)
+        exchange_rows(bufs.send_x, send_splits, recv_splits, bufs.recv_x, group)
+        exchange_rows(bufs.send_ids, send_splits, recv_splits, bufs.recv_ids.view(-1), group)
+        exchange_rows(bufs.send_probs, send_splits, recv_splits, bufs.recv_probs.view(-1), group)
+        expert_forward(shard, bufs, shard_wbuf, n_recv)
+        exchange_rows(bufs.recv_y, recv_splits, send_splits, bufs.y_back, group)
+        combine(plan, bufs, live_count, out)
