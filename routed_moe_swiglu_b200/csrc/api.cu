@@ -6,6 +6,7 @@
 #include <cstring>
 #include <new>
 
+#include "ep.cuh"
 #include "moe_internal.cuh"
 
 namespace moe {

@@ -15,6 +15,7 @@
 // chain as the one-GPU forward, so the output does not depend on the EP size
 // (the same PR's "Limitations" names generation's combine, which adds rank
 // partials, as not EP-invariant).
+#include "ep.cuh"
 #include "moe_internal.cuh"
 
 namespace moe {

@@ -151,14 +151,6 @@ cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max
 // out_bf16: out is bf16 (the fp32 sum rounded to nearest even), else fp32
 cudaError_t launch_combine(const float* y, const int* inv, const float* probs, const int* live, int max_live,
                            int H, int k, void* out, bool out_bf16, cudaStream_t s);
-// Expert-parallel send side: x rows of every live route (after the permute) into
-// send_x in expert order, local expert ids and FC1 probabilities per row, rows per
-// destination rank, and each route's send row and combine weight.
-int ep_max_size();
-cudaError_t launch_ep_pack(const void* x, const int* live, int max_live, int H, int k, const int* r_ids,
-                           const float* r_probs, const int* inv, const int* offsets, const int* padoff, int E,
-                           int ep_size, bool probs_in_fc1, void* send_x, int* send_ids, float* send_probs,
-                           int* send_counts, int* route_rows, float* route_probs, cudaStream_t s);
 cudaError_t launch_gemm1_bf16_pair(const CUtensorMap& a, const CUtensorMap& x_rows, const BoxMaps8& b,
                                    const GemmParams& gp, long long max_tiles, cudaStream_t s);
 cudaError_t launch_gemm2_bf16_pair(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
