@@ -307,7 +307,10 @@ moe_status moe_forward_with_events(const moe_plan* plan, const void* x, const fl
  *   route_probs  fp32 [max_live_rows, k]: the route's combine weight (its
  *                probability, or 1.0 under MOE_FLAG_PROBS_IN_FC1).
  * All outputs are device memory the caller owns; rows of tokens >= the live
- * count are not written. */
+ * count are not written.  The workspace holds the routes and the permutation
+ * as in moe_forward: one workspace serves one stream, and a moe_forward on the
+ * same workspace before step 5 would not disturb this step (step 5 reads only
+ * route_rows, route_probs and the returned rows). */
 moe_status moe_ep_dispatch(const moe_plan* plan, int ep_size, const void* x, const float* logits, const int* ids,
                            const float* probs, const int* live_count_dev, void* send_x, int* send_ids,
                            float* send_probs, int* send_counts, int* route_rows, float* route_probs,
