@@ -19,14 +19,18 @@
  *        multiply-adds of probability and row, from zero, in a fixed order);
  *        "Per-token NVFP4" (TE's NVFP4BlockScaling recipe with row-scaled
  *        activations, 1-D blocks, no Hadamard transform, no stochastic
- *        rounding).
+ *        rounding).  "What is changed" also runs every row an all-to-all
+ *        dispatcher delivers as a top-1 token with probability 1.0;
+ *        "Limitations": generation's combine is not EP-invariant.
  *   [P3] Megatron-LM PR #8367 ("bound the FlashInfer MoE expert kernels by
  *        token count"): "Problem" -- the live token count is known only on
  *        the device; results are returned in fp32.
  *   [P4] core.transformer.moe.training_matches_inference API doc: `_route`
  *        ([tokens, topk] probs and ids) and `expert_value_pass` (rows sorted
  *        by local expert).
- *   [P5] cudnn-frontend PR #448 (MoeEp API): MXFP8 uses 32-element blocks.
+ *   [P5] cudnn-frontend PR #448 (MoeEp API): MXFP8 uses 32-element blocks;
+ *        the parts of an EP layer: a variable-size all-to-all dispatch of
+ *        routes, local experts, a top-k combine.
  *
  * Conventions for every entry point:
  *   - Every pointer named *_dev or described as "device" is a device pointer
