@@ -130,3 +130,26 @@ def test_expert_range_splits_contiguously():
         except ValueError:
             continue
         raise AssertionError(f"expert_range{bad} accepted")
+
+
+def test_shard_plan_carries_the_source_plans_arithmetic():
+    """The receiving rank's plan: E/ep experts, top-1, fp32 rows out, and the
+    source plan's precision, FC1 flags and clamp (host-only: plans need no GPU)."""
+    import routed_moe_swiglu_b200 as rm
+    from routed_moe_swiglu_b200 import ep as moe_ep
+
+    src = rm.moe_plan_create(hidden=512, ffn=256, num_experts=16, top_k=4, capacity=100, precision="nvfp4",
+                             out_dtype="bf16", probs_in_fc1=True, gate_up_clamp=2.5, squared_relu=True)
+    shard = moe_ep.shard_plan_create(src, 4, 1600)
+    assert (shard.num_experts, shard.top_k, shard.capacity, shard.hidden, shard.ffn) == (4, 1, 1600, 512, 256)
+    assert shard.precision == "nvfp4" and shard.out_dtype == "fp32"
+    assert shard.probs_in_fc1 and shard.squared_relu and shard.gate_up_clamp == 2.5
+    plain = moe_ep.shard_plan_create(rm.moe_plan_create(hidden=512, ffn=256, num_experts=16, top_k=4,
+                                                        capacity=100), 2, 800)
+    assert not plain.probs_in_fc1 and not plain.squared_relu and plain.gate_up_clamp == 0.0
+    try:
+        moe_ep.shard_plan_create(src, 3, 100)
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("an EP size that does not divide E was accepted")
