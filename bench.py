@@ -77,8 +77,6 @@ def parse_args():
     if a.steps is None:
         a.steps = DEFAULT_STEPS[a.workload]
     if a.warmup is None:
-        # a few hundred forwards bring the step to its steady time (0.287 ms after
-        # 5 warm-up forwards of the decode workload, 0.276-0.283 ms after 200)
         a.warmup = a.steps
     if a.warmup < 3:
         a.warmup = 3
@@ -176,7 +174,7 @@ class ClockSampler:
                 self.samples.append((time.perf_counter(), mhz, reasons))
             except Exception:
                 pass
-            time.sleep(0.002)
+            time.sleep(0.010)  # a handful of samples in a timed region of tens of ms
 
     def start(self):
         if self.ok:
