@@ -112,6 +112,14 @@ typedef struct {
  *       h = relu(W_gate[e] . x)^2; W_up is not used.  The clamp and the
  *       probability in FC1 act on the one pre-activation and on the row. */
 #define MOE_FLAG_SQUARED_RELU 0x4u
+/*   MOE_FLAG_KEEP_H_FP32   MXFP8 only, for checking the fused quantiser: the
+ *       gate/up epilogue also stores the fp32 SwiGLU values it quantises,
+ *       [rows_padded, ceil(F/128)*128], into the workspace (the h_fp32
+ *       view).  The workspace grows by that buffer and every h element costs
+ *       one more 4-byte store; results are unchanged.  NVFP4 plans keep
+ *       these rows always (its quantisation pass reads them); bf16 plans
+ *       reject the flag. */
+#define MOE_FLAG_KEEP_H_FP32 0x8u
 
 typedef struct moe_plan moe_plan; /* opaque, host memory only */
 
@@ -235,8 +243,11 @@ moe_status moe_forward(const moe_plan* plan, const void* x, const float* logits,
  *   - Plans whose moe_workspace_bytes exceeds MOE_NOALLOC_SCRATCH_BYTES are
  *     rejected with MOE_ERR_WORKSPACE_TOO_SMALL before anything runs (use a
  *     smaller max_live_rows, or moe_forward with your own workspace).
- *   - The first call on a device looks up the array's device address (with
- *     that device current); make that first call before any stream capture.
+ *   - Each call outside stream capture looks up the array's device address
+ *     on the current device (so a cudaDeviceReset between calls is safe);
+ *     a call under capture uses the address that the last call outside
+ *     capture found.  Make one call on each device before any stream capture,
+ *     and again after a device reset.
  *   - Every call, on every stream, shares the one array, which keeps the
  *     last call's contents: calls that overlap on the GPU race with each
  *     other.  Serialise them (one stream, or events).
@@ -355,8 +366,10 @@ moe_status moe_ep_combine(const moe_plan* plan, const float* y_rows, const int* 
  *           (r % 32) * 16 + (r / 32) * 4 + b.  NVFP4 h and xq are codes two
  *           per byte ([rows_padded, ceil(K/256)*128] bytes).
  *   xq_row_scales, h_row_scales  NVFP4 only: fp32 second-level scale per
- *           padded row;  h_fp32  NVFP4 only: the gate/up GEMM's fp32 h rows
- *           [rows_padded, ceil(F/256)*256] before quantisation. */
+ *           padded row;  h_fp32  the gate/up GEMM's fp32 h rows before
+ *           quantisation: NVFP4 [rows_padded, ceil(F/256)*256]; MXFP8 plans
+ *           made with MOE_FLAG_KEEP_H_FP32 [rows_padded, ceil(F/128)*128];
+ *           else NULL. */
 typedef struct {
     const int* route_ids;
     const float* route_probs;

@@ -44,6 +44,7 @@ MOE_DEV_TIMEOUT = 0x4
 MOE_FLAG_PROBS_IN_FC1 = 0x1
 MOE_FLAG_OUT_BF16 = 0x2
 MOE_FLAG_SQUARED_RELU = 0x4
+MOE_FLAG_KEEP_H_FP32 = 0x8
 _PRECISION = {"bf16": 0, "mxfp8": 1, "nvfp4": 2}
 
 
@@ -157,6 +158,7 @@ class Plan:
         self.out_dtype = "bf16" if desc.flags & MOE_FLAG_OUT_BF16 else "fp32"
         self.gate_up_clamp = float(desc.gate_up_clamp)
         self.squared_relu = bool(desc.flags & MOE_FLAG_SQUARED_RELU)
+        self.keep_h_fp32 = bool(desc.flags & MOE_FLAG_KEEP_H_FP32)
 
     @property
     def handle(self):
@@ -177,16 +179,18 @@ class Plan:
 def moe_plan_create(hidden: int, ffn: int, num_experts: int, top_k: int, capacity: int,
                     precision: str = "bf16", max_live_rows: int = 0, out_dtype: str = "fp32",
                     probs_in_fc1: bool = False, gate_up_clamp: float | None = None,
-                    squared_relu: bool = False) -> Plan:
+                    squared_relu: bool = False, keep_h_fp32: bool = False) -> Plan:
     """out_dtype "fp32" or "bf16" (MOE_FLAG_OUT_BF16); probs_in_fc1 applies each
     route's probability to its SwiGLU row (MOE_FLAG_PROBS_IN_FC1); gate_up_clamp
     clamps the gate and up pre-activations (None: no clamp); squared_relu makes
-    the experts relu(W1 x)^2 MLPs (MOE_FLAG_SQUARED_RELU; w_up unused)."""
+    the experts relu(W1 x)^2 MLPs (MOE_FLAG_SQUARED_RELU; w_up unused);
+    keep_h_fp32 (MXFP8) also stores the fp32 h the gate/up epilogue quantises,
+    read through the h_fp32 workspace view (MOE_FLAG_KEEP_H_FP32)."""
     lib = load_library()
     if out_dtype not in ("fp32", "bf16"):
         raise ValueError(f"out_dtype must be 'fp32' or 'bf16', not {out_dtype!r}")
     flags = (MOE_FLAG_OUT_BF16 if out_dtype == "bf16" else 0) | (MOE_FLAG_PROBS_IN_FC1 if probs_in_fc1 else 0) | (
-        MOE_FLAG_SQUARED_RELU if squared_relu else 0)
+        MOE_FLAG_SQUARED_RELU if squared_relu else 0) | (MOE_FLAG_KEEP_H_FP32 if keep_h_fp32 else 0)
     d = _Desc(hidden, ffn, num_experts, top_k, capacity, max_live_rows, _PRECISION[precision], flags,
               float(gate_up_clamp) if gate_up_clamp else 0.0)
     h = ctypes.c_void_p()

@@ -105,6 +105,7 @@ static void compute_layouts(moe_plan* p) {
         w.xs = take(mtiles * p->ks1 * kSfBlock);
         w.h = take(R * (size_t)p->fp);
         w.hs = take(mtiles * p->ks2 * kSfBlock);
+        if ((p->d.flags & MOE_FLAG_KEEP_H_FP32) != 0) w.hf = take(R * (size_t)p->fp * 4);
     } else {
         w.xq = take(R * (size_t)p->hp * 2);  // x rows of tiles of more than kGatherInGemmMax routes
         w.xs = 0;
@@ -174,8 +175,9 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** plan_out) {
     if (d.num_experts > kMaxExperts || d.top_k > kMaxTopK || d.top_k > d.num_experts) return MOE_ERR_UNSUPPORTED;
     if (d.capacity > (1ll << 24)) return MOE_ERR_UNSUPPORTED;
     if (d.max_live_rows < 0 || d.max_live_rows > d.capacity) return MOE_ERR_UNSUPPORTED;
-    if ((d.flags & ~(MOE_FLAG_PROBS_IN_FC1 | MOE_FLAG_OUT_BF16 | MOE_FLAG_SQUARED_RELU)) != 0)
+    if ((d.flags & ~(MOE_FLAG_PROBS_IN_FC1 | MOE_FLAG_OUT_BF16 | MOE_FLAG_SQUARED_RELU | MOE_FLAG_KEEP_H_FP32)) != 0)
         return MOE_ERR_INVALID_ARG;
+    if ((d.flags & MOE_FLAG_KEEP_H_FP32) != 0 && d.precision == MOE_BF16) return MOE_ERR_INVALID_ARG;
     if (!(d.gate_up_clamp >= 0.0f) || d.gate_up_clamp > 3.0e38f) return MOE_ERR_INVALID_ARG;
     moe_plan* p = new (std::nothrow) moe_plan();
     if (p == nullptr) return MOE_ERR_INVALID_ARG;
@@ -449,6 +451,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g1.copy_next = status + kStCopyNext;
     g1.row_scale = fp4 ? reinterpret_cast<const float*>(ws + L.xg) : nullptr;
     g1.w_scale = fp4 ? reinterpret_cast<const float*>(wb + plan->wb.wg) : nullptr;
+    g1.h_fp32 = fp8 && L.hf != 0 ? reinterpret_cast<float*>(ws + L.hf) : nullptr;
     if (!mark(3)) return MOE_ERR_CUDA;
     e = fp8   ? launch_gemm1_mxfp8(tA1, rB1, g1, m_tiles * g1.n_tiles, s)
         : fp4 ? launch_gemm1_nvfp4(tA1, rB1, g1, m_tiles * g1.n_tiles, s)
@@ -471,6 +474,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g2.sfb = ws + L.hs;
     g2.out_scales = nullptr;
     g2.row_scale = fp4 ? reinterpret_cast<const float*>(ws + L.hg) : nullptr;
+    g2.h_fp32 = nullptr;
     if (!mark(4)) return MOE_ERR_CUDA;
     e = fp8   ? launch_gemm2_mxfp8(tA2, rB2, g2, m_tiles * g2.n_tiles, s)
         : fp4 ? launch_gemm2_nvfp4(tA2, rB2, g2, m_tiles * g2.n_tiles, s)
@@ -579,7 +583,7 @@ moe_status moe_get_workspace_views(const moe_plan* plan, const void* workspace, 
     v->xq_scales = scaled ? ws + L.xs : nullptr;
     v->xq_row_scales = fp4 ? reinterpret_cast<const float*>(ws + L.xg) : nullptr;
     v->h_row_scales = fp4 ? reinterpret_cast<const float*>(ws + L.hg) : nullptr;
-    v->h_fp32 = fp4 ? reinterpret_cast<const float*>(ws + L.hf) : nullptr;
+    v->h_fp32 = L.hf != 0 ? reinterpret_cast<const float*>(ws + L.hf) : nullptr;
     v->rows_padded = plan->rows_pad;
     v->status = reinterpret_cast<const unsigned*>(ws + L.status);
     return MOE_OK;

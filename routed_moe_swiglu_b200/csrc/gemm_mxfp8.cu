@@ -487,6 +487,11 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                         float inv;
                         const uint8_t sbyte = mxfp8_block_scale(amax, &inv);
                         const int route = c * 32 + lane;
+                        if (p.h_fp32 != nullptr && route < ti.z) {
+                            float4* hd = reinterpret_cast<float4*>(p.h_fp32 + (size_t)(ti.y + route) * (size_t)p.out_ld + f0);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) hd[i] = make_float4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+                        }
                         if (route < ti.z) {
                             uint32_t w[8];
 #pragma unroll
@@ -550,6 +555,12 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                     float inv;
                     const uint8_t sbyte = mxfp8_block_scale(amax, &inv);
                     const int route = c * 32 + qr;
+                    if (p.h_fp32 != nullptr && route < ti.z && f_blk < p.out_cols) {
+                        float4* hd = reinterpret_cast<float4*>(p.h_fp32 + (size_t)(ti.y + route) * (size_t)p.out_ld +
+                                                               f_blk + qh * 16);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) hd[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+                    }
                     if (route < ti.z && f_blk < p.out_cols) {
                         uint32_t w[4];
 #pragma unroll

@@ -42,7 +42,7 @@ constexpr unsigned long long kWaitLimitNs = 4000000000ull;
 struct WsLayout {
     size_t status, r_ids, r_probs, blkcnt, offsets, padoff, tiles, perm, inv, ready;
     size_t xq, xs, h, hs, y;
-    size_t xg, hf, hg;  // NVFP4: per-row scales of x and h, the fp32 h rows
+    size_t xg, hf, hg;  // NVFP4: per-row scales of x and h; the fp32 h rows (NVFP4, or MXFP8 keeping them)
     size_t total;
 };
 
@@ -127,6 +127,9 @@ struct GemmParams {
     // gate/up GEMM, h for the down GEMM) and of the weights ([E][2]: W1, W2)
     const float* row_scale;
     const float* w_scale;
+    // MXFP8 gate/up, plans with MOE_FLAG_KEEP_H_FP32 (else null): the fp32 h values the
+    // epilogue quantises, stored at the codes' positions (pitch out_ld)
+    float* h_fp32;
 };
 
 // ---------------------------------------------------------------- launchers

@@ -1,7 +1,13 @@
 """MXFP8 path vs the oracle: weight and activation quantisation inside
-prepare/forward bit-exact, the SwiGLU intermediate's codes equal the
-oracle's up to last-bit accumulation-order effects, outputs within the MXFP8
-tolerance (max |d| <= 5e-2 * RMS)."""
+prepare/forward bit-exact; the SwiGLU intermediate's codes and scales equal,
+bit for bit, the oracle quantiser applied to the GPU's own fp32 h (kept by
+MOE_FLAG_KEEP_H_FP32), and equal the oracle's own codes up to last-bit
+accumulation-order effects; outputs within the MXFP8 tolerance
+(max |d| <= 5e-2 * RMS).
+
+The fused FC1-epilogue quantisation is Megatron-LM PR #7798, "Background";
+the 32-element block rule is Megatron-LM PR #7830, "1. Mega backend for
+generation" (mxfp8_quantize_per_block_32) and cudnn-frontend PR #448."""
 from __future__ import annotations
 
 import numpy as np
@@ -91,6 +97,36 @@ def test_prepare_weights_bit_exact(F):
             assert np.all(w2s[idx] == 0)
 
 
+def _read_rows_f32(m: GpuMoe, ptr, rows_total, pitch, rows):
+    """fp32 rows `rows` of a [rows_total, pitch] workspace buffer (read on the device)."""
+    off = ptr - m.ws.data_ptr()
+    t = m.ws[off:off + rows_total * pitch * 4].view(torch.float32).view(rows_total, pitch)
+    return t[torch.from_numpy(np.asarray(rows, np.int64)).cuda()].cpu().numpy()
+
+
+def _check_h_own_quantisation(m: GpuMoe, F, rows, hf_ref=None):
+    """The fused epilogue's E4M3 codes and E8M0 scales of h are exactly the
+    oracle quantiser applied to the epilogue's own fp32 h (rows: padded route rows)."""
+    v = m.views()
+    assert v["h_fp32"], "the plan keeps no fp32 h (MOE_FLAG_KEEP_H_FP32)"
+    R = v["rows_padded"]
+    fp = (F + 127) // 128 * 128
+    hf = _read_rows_f32(m, v["h_fp32"], R, fp, rows)
+    assert np.all(hf[:, F:] == 0), "padding columns of h must be exact zeros"
+    own_q, own_s = oracle.mxfp8_quantize(np.ascontiguousarray(hf[:, :F]))
+    hq = _ws_bytes(m, v["h"], R * fp).reshape(R, fp)[rows][:, :F]
+    hs = decode_scales(_ws_bytes(m, v["h_scales"], (R // 128) * (fp // 128) * SF_BLOCK), rows, F)
+    bad_q = np.argwhere(hq != own_q)
+    assert bad_q.size == 0, f"{len(bad_q)} h codes differ from the oracle quantiser, first {bad_q[:4]}"
+    assert np.array_equal(hs, own_s), np.argwhere(hs != own_s)[:4]
+    if hf_ref is not None:
+        # and the fp32 values are the oracle's up to accumulation order
+        got = hf[:, :F].reshape(hf_ref.shape)
+        scale = np.abs(hf_ref).max(axis=-1, keepdims=True) + 1e-30
+        assert np.max(np.abs(got - hf_ref) / scale) < 1e-4
+    return hq.size
+
+
 def _check_intermediates(m: GpuMoe, x, ids, H, F, toks, h_ref):
     v = m.views()
     live, k = ids.shape
@@ -124,12 +160,14 @@ def _check_intermediates(m: GpuMoe, x, ids, H, F, toks, h_ref):
     b = hq_ref[diff].astype(np.int32)
     mag = lambda c: np.where(c & 0x80, -(c & 0x7F), c & 0x7F)  # noqa: E731
     assert np.all(np.abs(mag(a) - mag(b)) <= 1), np.stack([a, b])[:, :10]
+    if m.plan.keep_h_fp32:
+        _check_h_own_quantisation(m, F, rows, h_ref[2])
 
 
 @pytest.mark.parametrize("H,F,E,k,T", [(256, 256, 8, 2, 64), (320, 224, 6, 3, 200), (512, 1024, 16, 4, 300)])
 def test_forward_mxfp8_small(H, F, E, k, T):
     x, logits, weights = workloads.small_case(H, F, E, k, T, seed=H + F, capacity=T + 16)
-    m = GpuMoe(H, F, E, k, T + 16, weights, precision="mxfp8")
+    m = GpuMoe(H, F, E, k, T + 16, weights, precision="mxfp8", keep_h_fp32=True)
     out = m.forward(x.cuda(), T, logits=logits.cuda())
     torch.cuda.synchronize()
     ids, probs = oracle.route(logits[:T].numpy(), k)
@@ -157,7 +195,7 @@ def test_mxfp8_every_tile_width():
     assert np.all(ids[:, 0] != ids[:, 1])
     p = gen.uniform(0.1, 1.0, size=(T, k))
     probs = (p / p.sum(axis=1, keepdims=True)).astype(np.float32)
-    m = GpuMoe(H, F, E, k, T, weights, precision="mxfp8")
+    m = GpuMoe(H, F, E, k, T, weights, precision="mxfp8", keep_h_fp32=True)
     out = m.forward(x.cuda(), T, ids=torch.from_numpy(ids).cuda(), probs=torch.from_numpy(probs).cuda())
     torch.cuda.synchronize()
     ids_c = np.sort(ids, axis=1)
@@ -172,7 +210,7 @@ def test_mxfp8_every_tile_width():
 
 def test_forward_mxfp8_workload_subset():
     w, x, logits, weights = workload_problem("mxfp8")
-    m = GpuMoe(w.hidden, w.ffn, w.num_experts, w.top_k, w.capacity, weights, precision="mxfp8")
+    m = GpuMoe(w.hidden, w.ffn, w.num_experts, w.top_k, w.capacity, weights, precision="mxfp8", keep_h_fp32=True)
     live = w.max_live
     out = m.forward(x.cuda(), live, logits=logits.cuda())
     torch.cuda.synchronize()
@@ -198,3 +236,49 @@ def test_mxfp8_batch_invariance():
         b = m.forward(xd, n, logits=ld).cpu()
         assert torch.equal(b[:n], a[:n])
     assert torch.equal(m.forward(xd, 600, logits=ld).cpu(), a)
+
+
+@pytest.mark.parametrize("variant", [dict(), dict(squared_relu=True), dict(probs_in_fc1=True),
+                                     dict(gate_up_clamp=1.0), dict(squared_relu=True, probs_in_fc1=True,
+                                                                   gate_up_clamp=0.75)])
+def test_fused_h_quantiser_bit_exact_every_epilogue(variant):
+    """Every MXFP8 gate/up epilogue (SwiGLU, squared ReLU, probability in FC1,
+    clamp) quantises h exactly as the oracle quantiser does on the same fp32
+    values: every live route row, every block, bit for bit.  H, F not
+    multiples of 128 and enough tokens for every route-tile width."""
+    H, F, E, k, T = 320, 224, 12, 3, 700
+    x, logits, weights = workloads.small_case(H, F, E, k, T, seed=91, zipf=True)
+    wg, wu, wd = weights
+    relu2 = variant.get("squared_relu", False)
+    m = GpuMoe(H, F, E, k, T, (wg, wg if relu2 else wu, wd), precision="mxfp8", keep_h_fp32=True, **variant)
+    out = m.forward(x.cuda(), T, logits=logits.cuda())
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    ids, probs = oracle.route(logits.numpy(), k)
+    wq = oracle.quantize_weights_mxfp8(wg, wg if relu2 else wu, wd)
+    ref, h_ref = oracle.forward_mxfp8(x, ids, probs, wq, want_h=True, **variant)
+    assert_close(out.cpu().numpy(), ref, "mxfp8", f"mxfp8 {variant}")
+    inv = m.read_i32(m.views()["inv"], T * k).reshape(T, k)
+    n = _check_h_own_quantisation(m, F, inv.reshape(-1).astype(np.int64), h_ref[2])
+    assert n == T * k * F
+
+
+def test_keep_h_fp32_changes_no_result():
+    """The debug flag adds stores only: outputs and h bytes are bitwise those of a plain plan."""
+    H, F, E, k, T = 512, 256, 16, 4, 300
+    x, logits, weights = workloads.small_case(H, F, E, k, T, seed=92)
+    a = GpuMoe(H, F, E, k, T, weights, precision="mxfp8")
+    b = GpuMoe(H, F, E, k, T, weights, precision="mxfp8", keep_h_fp32=True)
+    assert a.views()["h_fp32"] is None and b.views()["h_fp32"]
+    oa = a.forward(x.cuda(), T, logits=logits.cuda())
+    ob = b.forward(x.cuda(), T, logits=logits.cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(oa.view(torch.int32), ob.view(torch.int32))
+    va, vb = a.views(), b.views()
+    R = va["rows_padded"]
+    # the route rows (padding rows between experts are never written)
+    rows = a.read_i32(va["inv"], T * k).astype(np.int64)
+    assert np.array_equal(rows, b.read_i32(vb["inv"], T * k))
+    ha = _ws_bytes(a, va["h"], R * 256).reshape(R, 256)[rows]
+    hb = _ws_bytes(b, vb["h"], R * 256).reshape(R, 256)[rows]
+    assert np.array_equal(ha, hb)
