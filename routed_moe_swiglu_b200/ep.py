@@ -34,7 +34,7 @@ from dataclasses import dataclass
 from . import (MoeError, Plan, alloc_workspace, moe_ep_combine, moe_ep_dispatch, moe_forward, moe_plan_create)
 
 __all__ = ["expert_range", "shard_plan_create", "EpBuffers", "dispatch", "expert_forward", "combine",
-           "exchange_counts", "exchange_rows", "moe_forward_ep"]
+           "exchange_counts", "agree_on_receive_capacity", "exchange_rows", "moe_forward_ep"]
 
 
 def expert_range(num_experts: int, ep_size: int, rank: int) -> tuple[int, int]:
@@ -146,6 +146,22 @@ def exchange_counts(send_counts, group=None):
     return recv
 
 
+def agree_on_receive_capacity(recv_splits: list[int], capacity: int, device, group=None) -> None:
+    """Every rank learns whether any rank would receive more rows than it can
+    hold, before any row moves: a MAX all-reduce of one overflow flag.  All
+    ranks then raise together (MoeError 4) instead of one rank raising while
+    the others wait in the row all-to-all until the group's timeout."""
+    import torch
+    import torch.distributed as dist
+
+    n_recv = sum(recv_splits)
+    flag = torch.tensor([1 if n_recv > capacity else 0], dtype=torch.int32, device=device)
+    dist.all_reduce(flag, op=dist.ReduceOp.MAX, group=group)
+    if int(flag.item()):
+        mine = f"this rank receives {n_recv} rows for {capacity}" if n_recv > capacity else "another rank"
+        raise MoeError(4, f"an EP rank's receive buffer is too small ({mine}); no rows were exchanged")
+
+
 def exchange_rows(send, send_splits: list[int], recv_splits: list[int], recv, group=None):
     """All-to-all of rows: send[:sum(send_splits)] goes out in runs of
     send_splits[g] rows to rank g; the runs from ranks 0, 1, ... land in
@@ -183,6 +199,8 @@ def moe_forward_ep(plan: Plan, shard: Plan, bufs: EpBuffers, x, shard_wbuf, live
         send_splits = bufs.send_counts.tolist()  # the host needs the split sizes
         recv_splits = recv_counts.tolist()
         n_recv = sum(recv_splits)
+        capacity = bufs.recv_x.shape[0] if shard is None else min(bufs.recv_x.shape[0], shard.capacity)
+        agree_on_receive_capacity(recv_splits, capacity, bufs.send_counts.device, group)
         exchange_rows(bufs.send_x, send_splits, recv_splits, bufs.recv_x, group)
         exchange_rows(bufs.send_ids, send_splits, recv_splits, bufs.recv_ids.view(-1), group)
         exchange_rows(bufs.send_probs, send_splits, recv_splits, bufs.recv_probs.view(-1), group)

@@ -103,6 +103,73 @@ def _rank_main(rank: int, world: int, port: int, results) -> None:
         dist.destroy_process_group()
 
 
+def _overflow_rank_main(rank: int, world: int, port: int, results) -> None:
+    """Rank 1's receive buffer holds one row, and rank 0 sends it more: both
+    ranks must raise before any row all-to-all starts."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+
+    from routed_moe_swiglu_b200 import MoeError
+    from routed_moe_swiglu_b200 import ep as moe_ep
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=30))
+    try:
+        row_exchanges = []
+
+        def fake_dispatch(plan, bufs, x, live_count, logits=None, ids=None, probs=None, stream=None):
+            bufs.send_counts[:] = torch.tensor([2, 5] if rank == 0 else [0, 0], dtype=torch.int32)
+
+        real_exchange = moe_ep.exchange_rows
+
+        def counting_exchange(*args, **kwargs):
+            row_exchanges.append(1)
+            return real_exchange(*args, **kwargs)
+
+        moe_ep.dispatch, moe_ep.exchange_rows = fake_dispatch, counting_exchange
+        recv = 64 if rank == 0 else 1
+        bufs = moe_ep.EpBuffers(
+            ep_size=world, workspace=None, send_x=torch.zeros((8, H), dtype=torch.bfloat16),
+            send_ids=torch.zeros(8, dtype=torch.int32), send_probs=torch.zeros(8),
+            send_counts=torch.zeros(world, dtype=torch.int32), route_rows=torch.zeros(4, K, dtype=torch.int32),
+            route_probs=torch.zeros(4, K), y_back=torch.zeros((8, H)),
+            recv_x=torch.zeros((recv, H), dtype=torch.bfloat16), recv_ids=torch.zeros((recv, 1), dtype=torch.int32),
+            recv_probs=torch.zeros(recv, 1), recv_y=torch.zeros((recv, H)), recv_live=torch.zeros(1, dtype=torch.int32),
+            shard_workspace=None)
+        live = torch.tensor([2], dtype=torch.int32)
+        try:
+            moe_ep.moe_forward_ep(None, None, bufs, torch.zeros((4, H), dtype=torch.bfloat16), None, live,
+                                  torch.zeros((4, H)), ids=torch.zeros((4, K), dtype=torch.int32),
+                                  probs=torch.zeros(4, K))
+            results[rank] = ("no error", len(row_exchanges))
+        except MoeError as exc:
+            results[rank] = (f"MoeError {exc.code}", len(row_exchanges))
+        # the group still works: every rank left the step at the same point
+        t = torch.tensor([rank + 1])
+        dist.all_reduce(t)
+        results[f"after{rank}"] = int(t)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_receive_overflow_on_one_rank_raises_on_every_rank():
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        results = mgr.dict()
+        procs = [ctx.Process(target=_overflow_rank_main, args=(r, 2, port, results)) for r in range(2)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+            assert p.exitcode == 0
+        res = dict(results)
+    assert res[0] == ("MoeError 4", 0) and res[1] == ("MoeError 4", 0), res
+    assert res["after0"] == 3 and res["after1"] == 3
+
+
 def test_two_rank_ep_step_exchanges_rows_and_returns_them_in_place():
     port = _free_port()
     ctx = mp.get_context("spawn")
