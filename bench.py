@@ -6,11 +6,18 @@
 One step = one pass of the whole path (route, permute, gather, gate/up GEMM
 + SwiGLU, down GEMM, combine; NVFP4 also quantises h between the GEMMs, timed
 with the gate/up stage) over one batch of seeded synthetic inputs that
-are already resident in HBM.  The K timed steps are one captured CUDA graph
-(K forwards back to back, stage events inside), bracketed by a barrier and
-a device synchronise; the time is the max over ranks.  Every step re-reads
-all expert weights (1.6-3.8 GB), more than the 126 MB L2, so no L2 flush is
-needed between steps.
+are already resident in HBM.  The K timed steps are K replays of a captured
+one-forward CUDA graph (the granularity of the end-to-end loop), bracketed
+by a barrier and a device synchronise; the time is the max over ranks.  The
+stage split comes from a second graph with events between the stages.  Every
+step re-reads all expert weights (1.6-3.8 GB), more than the 126 MB L2, so
+no L2 flush is needed between steps.
+
+The default run (decode headline, one GPU) also measures the other
+configurations in the same process and reports each under `configs`: the
+16,384-token bf16 prefill (tensor-bound), the 4,096-token MXFP8 prefill and
+the live-count sweep (with its bitwise invariance across counts and
+replays).
 
 Metric: routed tokens/s = live tokens processed per second (whole job).
 Extra keys: `roofline` for the dominant kernel (algorithmic bytes or FLOPs
@@ -50,6 +57,9 @@ def kernels_per_forward(precision: str, max_live: int) -> int:
     permute = 1 if max_live <= 1024 else 3
     return 1 + permute + (precision != "bf16") + 1 + (precision == "nvfp4") + 1 + 1
 STAGES = ("route", "permute", "gather", "gemm_gate_up", "gemm_down", "combine")
+# measured after the headline (decode) in the default run: the tensor-bound prefill,
+# the MXFP8 prefill and the live-count sweep
+EXTRA_CONFIGS = ("prefill", "mxfp8", "sweep")
 DEFAULT_STEPS = {"tiny": 200, "decode": 200, "prefill": 30, "mxfp8": 50, "nvfp4": 50, "decode_nvfp4": 200,
                  "sweep": 20}
 
@@ -66,6 +76,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other configurations' records (prefill, mxfp8, sweep) after the decode line")
     ap.add_argument("--probs-in-fc1", action="store_true",
                     help="variant: router probabilities applied to the SwiGLU row (apply_topk_in_fc1)")
     ap.add_argument("--gate-up-clamp", type=float, default=None, help="variant: clamp of the gate/up pre-activations")
@@ -174,7 +186,7 @@ class ClockSampler:
                 self.samples.append((time.perf_counter(), mhz, reasons))
             except Exception:
                 pass
-            time.sleep(0.010)  # a handful of samples in a timed region of tens of ms
+            time.sleep(0.001)  # several samples even in a timed region of a few ms
 
     def start(self):
         if self.ok:
@@ -258,16 +270,23 @@ def recorded_traffic(stage, workload, precision):
 # ---------------------------------------------------------------- the CUDA arm
 
 
-def run_ours(a, dist: Dist):
-    import routed_moe_swiglu_b200 as rm
-
-    w = workloads.WORKLOADS[a.workload]
-    if a.capacity is not None:
+def _workload(a, name):
+    w = workloads.WORKLOADS[name]
+    if a.capacity is not None and name == a.workload:
         import dataclasses
 
         w = dataclasses.replace(w, capacity=a.capacity, live=tuple(min(v, a.capacity) for v in w.live),
                                 nan_past_live=True)
-    live = min(a.live or w.max_live, w.capacity)
+    return w
+
+
+def measure(a, dist: Dist, w, live, K, W, want_e2e=False, want_sweep=False):
+    """One workload on this rank's GPU: K timed forwards (replays of a one-step
+    CUDA graph, the granularity of the end-to-end loop too), their stage split
+    from a second graph with events between the stages, the live-count sweep
+    (when the workload has several live counts) and the end-to-end loop."""
+    import routed_moe_swiglu_b200 as rm
+
     x, logits = workloads.make_activations(w)
     wg, wu, wd = workloads.make_weights(w)
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -295,12 +314,10 @@ def run_ours(a, dist: Dist):
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream(device=dev)
-    K, W = a.steps, a.warmup
-    # one-step graph (warm-up, e2e) and a K-step graph with stage events (timed)
     with torch.cuda.stream(stream):
         rm.moe_forward(plan, xd, wbuf, live_d, out, ws, logits=ld)  # first call outside capture
     stream.synchronize()
-    g1 = torch.cuda.CUDAGraph()
+    g1 = torch.cuda.CUDAGraph()  # one forward: the timed step, the warm-up, the sweep and e2e
     with torch.cuda.graph(g1, stream=stream):
         rm.moe_forward(plan, xd, wbuf, live_d, out, ws, logits=ld)
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(K)]
@@ -309,13 +326,8 @@ def run_ours(a, dist: Dist):
             for e in ev:
                 e.record(stream)
     stream.synchronize()
-    # the timed graph: K plain forwards (the kernels overlap their launches, see
-    # pdl_wait in the library); a second K-step graph with stage events between
-    # the kernels (which serialises them fully) gives the per-stage split
-    gk = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gk, stream=stream):
-        for i in range(K):
-            rm.moe_forward(plan, xd, wbuf, live_d, out, ws, logits=ld)
+    # the stage split: K forwards with an event between every two stages (which
+    # serialises the kernels fully), replayed after the timed region
     ge = torch.cuda.CUDAGraph()
     with torch.cuda.graph(ge, stream=stream):
         for i in range(K):
@@ -335,7 +347,8 @@ def run_ours(a, dist: Dist):
     h0 = time.perf_counter()
     with torch.cuda.stream(stream):
         t_start.record(stream)
-        gk.replay()
+        for _ in range(K):
+            g1.replay()
         t_end.record(stream)
     torch.cuda.synchronize()
     h1 = time.perf_counter()
@@ -361,8 +374,6 @@ def run_ours(a, dist: Dist):
     off = views["offsets"] - views["base"]
     offsets = ws[off:off + 4 * (w.num_experts + 1)].view(torch.int32).cpu()
     counts = (offsets[1:] - offsets[:-1]).tolist()
-    touched = sum(1 for c in counts if c > 0)
-    routes = int(offsets[-1])
 
     res = {
         "ms_per_step": ms_step,
@@ -373,21 +384,25 @@ def run_ours(a, dist: Dist):
         "ms_per_step_with_stage_events": ms_step_events,
         "clocks": clocks.summary(),
         "timed_s": ms_total / 1e3,
-        "touched": touched,
-        "routes": routes,
+        "touched": sum(1 for c in counts if c > 0),
+        "routes": int(offsets[-1]),
         "status": status,
         "max_rows_per_expert": max(counts),
+        "live": live,
     }
 
-    # ---------------- live-count sweep: the same one-step graph, device live counts
-    if len(w.live) > 1 and a.live is None:
-        sweep = []
+    # ---------------- live-count sweep: the same one-step graph, device live counts;
+    # each token's output must be bitwise the same at every count and in every replay
+    if want_sweep and len(w.live) > 1:
+        sweep, kept = [], {}
         reps = max(3, min(20, K))
+        invariant = True
         for n in w.live:
             live_d.fill_(n)
             with torch.cuda.stream(stream):
                 g1.replay()
             stream.synchronize()
+            first = out[:n].clone()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             with torch.cuda.stream(stream):
@@ -397,10 +412,22 @@ def run_ours(a, dist: Dist):
                 e1.record(stream)
             torch.cuda.synchronize()
             ms = e0.elapsed_time(e1) / reps
-            sweep.append({"live": n, "ms_per_step": ms, "tokens_per_s": n / (ms / 1e3)})
+            same_replays = bool(torch.equal(first.view(torch.int32), out[:n].view(torch.int32)))
+            kept[n] = first
+            o_n = ws[off:off + 4 * (w.num_experts + 1)].view(torch.int32).cpu()
+            c_n = o_n[1:] - o_n[:-1]
+            sweep.append({"live": n, "ms_per_step": ms, "tokens_per_s": n / (ms / 1e3),
+                          "routes": int(o_n[-1]), "touched": int((c_n > 0).sum()),
+                          "bitwise_equal_across_replays": same_replays})
+            invariant = invariant and same_replays
+        ns = sorted(kept)
+        for lo, hi in zip(ns, ns[1:]):
+            invariant = invariant and bool(torch.equal(kept[hi][:lo].view(torch.int32), kept[lo].view(torch.int32)))
+        del kept
         live_d.fill_(live)
         torch.cuda.synchronize()
         res["sweep"] = sweep
+        res["sweep_bitwise_invariant"] = invariant
 
     # ---------------- end to end through the C ABI with pinned host buffers
     # Every step copies its inputs (x, logits, live count) in from pinned host
@@ -410,7 +437,7 @@ def run_ours(a, dist: Dist):
     # forwards in order on `stream`; events keep each set's reuse ordered (a
     # set's inputs are rewritten once its last forward is done, its output
     # once it has been read back).
-    if not a.no_e2e:
+    if want_e2e:
         x_pin = x[:live].contiguous().pin_memory()
         l_pin = logits[:live].contiguous().pin_memory()
         n_pin = torch.tensor([live], dtype=torch.int32).pin_memory()
@@ -473,21 +500,39 @@ def run_ours(a, dist: Dist):
                       "d2h_bytes_per_step": o_pins[0].numel() * o_pins[0].element_size(), "ms_per_step": e_ms,
                       "copies": "overlapped with the neighbouring steps' forwards (two buffer sets)"}
         del g1b
-    del gk, ge, g1
+    del ge, g1
+    return res
+
+
+def run_ours(a, dist: Dist):
+    w = _workload(a, a.workload)
+    live = min(a.live or w.max_live, w.capacity)
+    res = measure(a, dist, w, live, a.steps, a.warmup, want_e2e=not a.no_e2e, want_sweep=a.live is None)
     return w, live, res
 
 
+def _bpe(precision):
+    """Bytes per operand element with its block scales: E4M3 + an E8M0 per 32,
+    E2M1 + an E4M3 per 16, bf16."""
+    return {"mxfp8": 1 + 1 / 32, "nvfp4": 0.5 + 1 / 16}.get(precision, 2)
+
+
+def _tc_ratio(precision):
+    return {"mxfp8": 2.0, "nvfp4": 4.0}.get(precision, 1.0)  # nominal dense peak over bf16
+
+
 def roofline(w, res, peaks):
-    """Roofline of the dominant kernel (largest share of the step)."""
+    """Roofline of the dominant kernel (largest share of the step).  The
+    algorithmic work counts only what the method must do (routes * 6 * H * F
+    FLOPs; the touched experts' weights once, x in once per token, out once
+    per token) and not the padded work or the h / y round trips."""
     st = res["stage_ms"]
     dom = max(st, key=lambda s: st[s])
     ms = st[dom]
-    H, F, k = w.hidden, w.ffn, w.top_k
-    R = res["routes"]
-    # bytes per element of the operands, block scales included: E4M3 + an E8M0 per 32,
-    # E2M1 + an E4M3 per 16, bf16
-    bpe = {"mxfp8": 1 + 1 / 32, "nvfp4": 0.5 + 1 / 16}.get(w.precision, 2)
-    tc_ratio = {"mxfp8": 2.0, "nvfp4": 4.0}.get(w.precision, 1.0)  # nominal dense peak over bf16
+    H, F, E = w.hidden, w.ffn, w.num_experts
+    R, n = res["routes"], res["live"]
+    bpe = _bpe(w.precision)
+    tc_ratio = _tc_ratio(w.precision)
     sustained = res["timed_s"] > 1.0
     tflops_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     out = {"kernel": dom}
@@ -495,13 +540,10 @@ def roofline(w, res, peaks):
         if dom == "gemm_gate_up":
             nproj = res.get("fc1_projections", 2)  # gate and up, or the one squared-ReLU projection
             flops = 2.0 * nproj * R * H * F
-            wbytes = res["touched"] * nproj * F * H * bpe
-            abytes = R * H * bpe + R * F * bpe
+            bytes_ = res["touched"] * nproj * F * H * bpe + n * H * bpe  # weights + x, once
         else:
             flops = 2.0 * R * H * F
-            wbytes = res["touched"] * H * F * bpe
-            abytes = R * F * bpe + R * H * 4
-        bytes_ = wbytes + abytes
+            bytes_ = res["touched"] * H * F * bpe  # weights, once
         t_hbm = bytes_ / (peaks["hbm_gbs"] * 1e9)
         t_tc = flops / (tflops_peak * 1e12 * tc_ratio)
         if t_hbm >= t_tc:
@@ -518,19 +560,66 @@ def roofline(w, res, peaks):
     else:
         # memory-bound helper kernels: bytes they must move
         if dom == "combine":
-            bytes_ = R * H * 4 + res["live"] * H * 4 + R * 8
+            bytes_ = R * H * 4 + n * H * 4 + R * 8
         elif dom == "gather":
-            bytes_ = res["live"] * H * 2 + R * H * bpe
+            bytes_ = n * H * 2 + R * H * bpe
         else:
-            bytes_ = res["live"] * w.num_experts * 4
+            bytes_ = n * E * 4
         out.update(bound="hbm", achieved=bytes_ / (ms / 1e3) / 1e9, peak=peaks["hbm_gbs"], unit="GB/s",
                    algorithmic_per_launch=bytes_)
     out["frac"] = out["achieved"] / out["peak"]
     out["peak_source"] = peaks["source"]
     out["kernel_ms"] = ms
-    tr = recorded_traffic(dom, w.name, w.precision)
-    out["traffic"] = tr
+    out["traffic"] = recorded_traffic(dom, w.name, w.precision)
     return out
+
+
+def step_roofline(w, res, peaks, point=None):
+    """The whole step against the roofline of the method's algorithmic work:
+    bytes = the touched experts' weights once + x, logits in and out out per
+    live token; FLOPs = routes * 6 * H * F (squared-ReLU: 4).  frac = the
+    roofline time (the larger of bytes / HBM and FLOPs / tensor peak) over
+    the measured step time.  `point`: a sweep entry (live, routes, touched,
+    ms_per_step) instead of the timed step."""
+    H, F, E = w.hidden, w.ffn, w.num_experts
+    src = res if point is None else point
+    n, R, touched, ms = src["live"], src["routes"], src["touched"], src["ms_per_step"]
+    nproj = res.get("fc1_projections", 2)
+    bpe = _bpe(w.precision)
+    bytes_ = touched * (nproj + 1) * H * F * bpe + n * (H * 2 + E * 4 + H * 4)
+    flops = 2.0 * (nproj + 1) * R * H * F
+    out = {}
+    for kind, tf in (("burst", peaks["bf16_tflops"]), ("sustained", peaks["bf16_tflops_sustained"])):
+        t_b = bytes_ / (peaks["hbm_gbs"] * 1e9)
+        t_f = flops / (tf * 1e12 * _tc_ratio(w.precision))
+        t = max(t_b, t_f)
+        out[f"frac_{kind}"] = t / (ms / 1e3)
+        if kind == "burst":
+            out.update(bound="hbm" if t_b >= t_f else "tensor", bytes=bytes_, flops=flops,
+                       roofline_ms=t * 1e3, hbm_frac=t_b / (ms / 1e3), tensor_frac=t_f / (ms / 1e3))
+    out["peak_source"] = peaks["source"]
+    return out
+
+
+def sub_record(a, dist, name, peaks):
+    """A spec configuration measured in the same process as the headline."""
+    w = _workload(a, name)
+    K = DEFAULT_STEPS[name]
+    res = measure(a, dist, w, w.max_live, K, K, want_e2e=False, want_sweep=True)
+    rec = {"workload": workload_config(w, w.max_live, a)["workload"], "steps": K, "warmup": K,
+           "ms_per_step": res["ms_per_step"], "tokens_per_s": res["value"],
+           "stage_ms": {k: round(v, 5) for k, v in res["stage_ms"].items()},
+           "roofline": roofline(w, res, peaks), "step_roofline": step_roofline(w, res, peaks),
+           "clocks": res["clocks"], "device_status": res["status"],
+           "gpu_launches": kernels_per_forward(w.precision, w.capacity) * K}
+    if "sweep" in res:
+        for e in res["sweep"]:
+            e["step_roofline_frac"] = step_roofline(w, res, peaks, point=e)["frac_burst"]
+        rec["sweep"] = res["sweep"]
+        rec["bitwise_invariant"] = res["sweep_bitwise_invariant"]
+    del res
+    torch.cuda.empty_cache()
+    return rec
 
 
 # ---------------------------------------------------------------- the oracle (CPU) arm
@@ -682,7 +771,6 @@ def main():
         return
 
     w, live, res = run_ours(a, dist)
-    res["live"] = live
     peaks = measured_peaks()
     line = {
         "metric": "routed tokens/s", "value": res["value"], "unit": "tokens/s", "n_gpus": dist.world,
@@ -690,6 +778,7 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": w.precision, "data": "synthetic",
         "config": workload_config(w, live, a),
         "roofline": roofline(w, res, peaks),
+        "step_roofline": step_roofline(w, res, peaks),
         "stage_ms": {k: round(v, 5) for k, v in res["stage_ms"].items()},
         "ms_per_step_with_stage_events": round(res["ms_per_step_with_stage_events"], 5),
         "prepare_weights_ms": round(res["prepare_ms"], 4),
@@ -703,6 +792,10 @@ def main():
         line["e2e"] = res["e2e"]
     if "sweep" in res:
         line["sweep"] = res["sweep"]
+        line["sweep_bitwise_invariant"] = res["sweep_bitwise_invariant"]
+    if dist.world == 1 and not a.no_extra and a.workload == "decode" and a.live is None and a.capacity is None:
+        # the other spec configurations, each timed alone in this process
+        line["configs"] = {name: sub_record(a, dist, name, peaks) for name in EXTRA_CONFIGS}
     if dist.rank == 0 and dist.world == 1 and not a.no_cpu_baseline:
         x, logits = workloads.make_activations(w)
         weights = workloads.make_weights(w)
