@@ -50,12 +50,10 @@ import torch  # noqa: E402
 import workloads  # noqa: E402
 
 def kernels_per_forward(precision: str, max_live: int) -> int:
-    """Library kernels one forward launches: route, the permute (hist, scan, scatter; one
-    kernel for plans of at most 1,024 live rows), the x gather (MXFP8, NVFP4: bf16 copies
-    the rows inside its gate/up GEMM), gate/up GEMM, NVFP4's h quantisation, down GEMM,
-    combine."""
-    permute = 1 if max_live <= 1024 else 3
-    return 1 + permute + (precision != "bf16") + 1 + (precision == "nvfp4") + 1 + 1
+    """Library kernels one forward launches: route, permute, the x gather (MXFP8, NVFP4:
+    bf16 copies the rows inside its gate/up GEMM), gate/up GEMM, NVFP4's h quantisation,
+    down GEMM, combine."""
+    return 1 + 1 + (precision != "bf16") + 1 + (precision == "nvfp4") + 1 + 1
 STAGES = ("route", "permute", "gather", "gemm_gate_up", "gemm_down", "combine")
 # measured after the headline (decode) in the default run: the tensor-bound prefill,
 # the MXFP8 prefill and the live-count sweep

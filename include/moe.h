@@ -78,7 +78,9 @@ typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1, MOE_NVFP4 = 2 } moe_precision;
 #define MOE_DEV_BAD_ROUTE 0x2u     /* caller ids out of [0,E) or repeated in a token:
                                       that token's output row is all zeros          */
 #define MOE_DEV_TIMEOUT 0x4u       /* a bounded on-device wait gave up; outputs of
-                                      that call are not valid                       */
+                                      that call are not valid, and while the bit is
+                                      set, forwards on this workspace write no
+                                      output rows (clear it to run again)           */
 
 typedef struct {
     int hidden;              /* H: model width (K of the gate/up GEMM)            */

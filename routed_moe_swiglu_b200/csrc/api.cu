@@ -81,7 +81,7 @@ static void compute_layouts(moe_plan* p) {
     w.status = take(kStWords * 4);
     w.r_ids = take(L * k * 4);
     w.r_probs = take(L * k * 4);
-    w.blkcnt = take((size_t)p->nblk * E * 4);
+    w.blkcnt = take(((size_t)p->nblk + 1) * E * 4);  // per-chunk counts, then the per-expert totals
     w.offsets = take((E + 1) * 4);
     w.padoff = take((E + 1) * 4);
     w.tiles = take((size_t)p->max_m_tiles * 16);
@@ -411,11 +411,11 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     if (!mark(2)) return MOE_ERR_CUDA;
     if (fp8) {  // bf16: the gate/up GEMM copies the x rows itself
         e = launch_gather_mxfp8(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, (int)plan->hp, k,
-                                inv, ws + L.xq, ws + L.xs, s);
+                                inv, ws + L.xq, ws + L.xs, status, s);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     } else if (fp4) {
         e = launch_gather_nvfp4(static_cast<const __nv_bfloat16*>(x), live_count_dev, max_live, H, (int)plan->hp, k,
-                                inv, ws + L.xq, ws + L.xs, reinterpret_cast<float*>(ws + L.xg), s);
+                                inv, ws + L.xq, ws + L.xs, reinterpret_cast<float*>(ws + L.xg), status, s);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
 
@@ -459,7 +459,8 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     if (fp4) {  // h rows -> NVFP4 with a scale per row (timed with the gate/up stage)
         e = launch_quantize_h_nvfp4(reinterpret_cast<const float*>(ws + L.hf), live_count_dev, max_live, k,
-                                    (int)plan->fp, inv, ws + L.h, ws + L.hs, reinterpret_cast<float*>(ws + L.hg), s);
+                                    (int)plan->fp, inv, ws + L.h, ws + L.hs, reinterpret_cast<float*>(ws + L.hg),
+                                    status, s);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
 
@@ -484,7 +485,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
 
     // the probabilities were applied in the gate/up epilogue: the combine adds the rows
     e = launch_combine(reinterpret_cast<const float*>(ws + L.y), inv, probs_in_fc1 ? nullptr : r_probs,
-                       live_count_dev, max_live, H, k, out, (plan->d.flags & MOE_FLAG_OUT_BF16) != 0, s);
+                       live_count_dev, max_live, H, k, out, (plan->d.flags & MOE_FLAG_OUT_BF16) != 0, status, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     return mark(6) ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -548,7 +549,7 @@ moe_status moe_ep_dispatch(const moe_plan* plan, int ep_size, const void* x, con
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_ep_pack(x, live_count_dev, max_live, H, k, r_ids, r_probs, inv, offsets, padoff, E, ep_size,
                        (plan->d.flags & MOE_FLAG_PROBS_IN_FC1) != 0, send_x, send_ids, send_probs, send_counts,
-                       route_rows, route_probs, s);
+                       route_rows, route_probs, status, s);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -560,7 +561,8 @@ moe_status moe_ep_combine(const moe_plan* plan, const float* y_rows, const int* 
     if (!aligned(y_rows, 16) || !aligned(out, 16)) return MOE_ERR_ALIGNMENT;
     const cudaError_t e = launch_combine(y_rows, route_rows, route_probs, live_count_dev, (int)plan->max_live,
                                          plan->d.hidden, plan->d.top_k, out,
-                                         (plan->d.flags & MOE_FLAG_OUT_BF16) != 0, static_cast<cudaStream_t>(stream));
+                                         (plan->d.flags & MOE_FLAG_OUT_BF16) != 0, nullptr,
+                                         static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

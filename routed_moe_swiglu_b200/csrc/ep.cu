@@ -30,14 +30,16 @@ __global__ void __launch_bounds__(kPackThreads) ep_pack_kernel(
     const int* __restrict__ r_ids, const float* __restrict__ r_probs, const int* __restrict__ inv,
     const int* __restrict__ offsets, const int* __restrict__ padoff, int E, int ep_size, int probs_in_fc1,
     uint4* __restrict__ send_x, int* __restrict__ send_ids, float* __restrict__ send_probs,
-    int* __restrict__ send_counts, int* __restrict__ route_rows, float* __restrict__ route_probs) {
+    int* __restrict__ send_counts, int* __restrict__ route_rows, float* __restrict__ route_probs,
+    const unsigned* status) {
     __shared__ int s_row[kMaxTopK];
     pdl_trigger();
     pdl_wait();
-    const int n = clamp_live(live, max_live);
+    const bool poisoned = forward_poisoned(status);  // a partial permutation sends nothing
+    const int n = poisoned ? 0 : clamp_live(live, max_live);
     const int el = E / ep_size;  // experts per EP rank
     if (blockIdx.x == 0 && (int)threadIdx.x < ep_size)
-        send_counts[threadIdx.x] = offsets[(threadIdx.x + 1) * el] - offsets[threadIdx.x * el];
+        send_counts[threadIdx.x] = poisoned ? 0 : offsets[(threadIdx.x + 1) * el] - offsets[threadIdx.x * el];
     for (int t = blockIdx.x; t < n; t += gridDim.x) {
         __syncthreads();
         if ((int)threadIdx.x < k) {
@@ -75,7 +77,8 @@ int ep_max_size() { return kPackThreads; }
 cudaError_t launch_ep_pack(const void* x, const int* live, int max_live, int H, int k, const int* r_ids,
                            const float* r_probs, const int* inv, const int* offsets, const int* padoff, int E,
                            int ep_size, bool probs_in_fc1, void* send_x, int* send_ids, float* send_probs,
-                           int* send_counts, int* route_rows, float* route_probs, cudaStream_t s) {
+                           int* send_counts, int* route_rows, float* route_probs, const unsigned* status,
+                           cudaStream_t s) {
     long long blocks = max_live;
     const long long cap = (long long)num_sms() * 16;
     if (blocks > cap) blocks = cap;
@@ -83,7 +86,7 @@ cudaError_t launch_ep_pack(const void* x, const int* live, int max_live, int H, 
     return launch_dependent(ep_pack_kernel, dim3((unsigned)blocks), dim3(kPackThreads), 0, s,
                             static_cast<const uint4*>(x), live, max_live, H * 2 / 16, k, r_ids, r_probs, inv, offsets,
                             padoff, E, ep_size, probs_in_fc1 ? 1 : 0, static_cast<uint4*>(send_x), send_ids,
-                            send_probs, send_counts, route_rows, route_probs);
+                            send_probs, send_counts, route_rows, route_probs, status);
 }
 
 }  // namespace moe

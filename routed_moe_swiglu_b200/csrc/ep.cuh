@@ -13,6 +13,7 @@ int ep_max_size();
 cudaError_t launch_ep_pack(const void* x, const int* live, int max_live, int H, int k, const int* r_ids,
                            const float* r_probs, const int* inv, const int* offsets, const int* padoff, int E,
                            int ep_size, bool probs_in_fc1, void* send_x, int* send_ids, float* send_probs,
-                           int* send_counts, int* route_rows, float* route_probs, cudaStream_t s);
+                           int* send_counts, int* route_rows, float* route_probs, const unsigned* status,
+                           cudaStream_t s);
 
 }  // namespace moe

@@ -150,7 +150,7 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
     const uint32_t tmem_base = bars->tmem_base;
     pdl_wait();  // the tile list, x / h rows and status words come from earlier kernels
 
-    const int num_m = (int)p.status_words[kStNumMTiles];
+    const int num_m = forward_poisoned(p.status_words) ? 0 : (int)p.status_words[kStNumMTiles];
     const int total_tiles = num_m * p.n_tiles;
     const int kb_count = p.k_blocks;
 

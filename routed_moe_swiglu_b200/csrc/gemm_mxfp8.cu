@@ -198,7 +198,7 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
     const uint32_t tmem_base = bars->tmem_base;
     pdl_wait();  // the tile list, route rows, scales and status words come from earlier kernels
 
-    const int num_m = (int)p.status_words[kStNumMTiles];
+    const int num_m = forward_poisoned(p.status_words) ? 0 : (int)p.status_words[kStNumMTiles];
     const int total_tiles = num_m * p.n_tiles;
     const int nblk = p.k_blocks;               // K blocks of 128
     const int kb_count = (nblk + 1) / kAtoms;  // stages of 256 (the last may hold one block)

@@ -34,7 +34,9 @@ constexpr int kMaxTopK = 16;
 constexpr int kMaxExperts = 1024;
 
 // Status word layout (uint32 words at the start of the workspace).
-enum : int { kStFlags = 0, kStNumMTiles = 1, kStTotalRoutes = 2, kStCopyNext = 3, kStWords = 64 };
+// kStPermBar: arrivals at the permute's grid-wide barriers, zeroed by the router kernel
+// (route or canonicalise) that precedes the permute in every forward.
+enum : int { kStFlags = 0, kStNumMTiles = 1, kStTotalRoutes = 2, kStCopyNext = 3, kStPermBar = 4, kStWords = 64 };
 
 // Default bound of any on-device wait before the kernel gives up (ns).
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;
@@ -148,12 +150,13 @@ cudaError_t launch_canon_routes(const int* ids_in, const float* probs_in, const 
 cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* blkcnt, int* offsets,
                            int* padoff, int4* tiles, int* perm, int* inv, int* ready, unsigned* status_words,
                            cudaStream_t s);
+// status (the workspace's status words, or null) on the launchers below: see forward_poisoned()
 cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
-                                const int* inv, uint8_t* xq, uint8_t* xs, cudaStream_t s);
+                                const int* inv, uint8_t* xq, uint8_t* xs, const unsigned* status, cudaStream_t s);
 // probs null: every route's weight is 1 (the probabilities were applied in FC1);
 // out_bf16: out is bf16 (the fp32 sum rounded to nearest even), else fp32
 cudaError_t launch_combine(const float* y, const int* inv, const float* probs, const int* live, int max_live,
-                           int H, int k, void* out, bool out_bf16, cudaStream_t s);
+                           int H, int k, void* out, bool out_bf16, const unsigned* status, cudaStream_t s);
 cudaError_t launch_gemm1_bf16_pair(const CUtensorMap& a, const CUtensorMap& x_rows, const BoxMaps8& b,
                                    const GemmParams& gp, long long max_tiles, cudaStream_t s);
 cudaError_t launch_gemm2_bf16_pair(const CUtensorMap& a, const BoxMaps8& b, const GemmParams& gp, long long max_tiles,
@@ -169,9 +172,10 @@ cudaError_t launch_gemm2_nvfp4(const CUtensorMap& a, const BoxMaps8& b, const Ge
 cudaError_t launch_nvfp4_quantize_rows(const __nv_bfloat16* in, long long rows, int cols, long long ld_in,
                                        uint8_t* q, uint8_t* scales, float* g, const int* live_rows, cudaStream_t s);
 cudaError_t launch_gather_nvfp4(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
-                                const int* inv, uint8_t* xq, uint8_t* xs, float* xg, cudaStream_t s);
+                                const int* inv, uint8_t* xq, uint8_t* xs, float* xg, const unsigned* status,
+                                cudaStream_t s);
 cudaError_t launch_quantize_h_nvfp4(const float* hf, const int* live, int max_live, int k, int fp, const int* inv,
-                                    uint8_t* hq, uint8_t* hs, float* hg, cudaStream_t s);
+                                    uint8_t* hq, uint8_t* hs, float* hg, const unsigned* status, cudaStream_t s);
 cudaError_t launch_prepare_nvfp4(const moe_plan* p, const __nv_bfloat16* wg, const __nv_bfloat16* wu,
                                  const __nv_bfloat16* wd, void* buf, cudaStream_t s);
 cudaError_t launch_prepare_bf16(const moe_plan* p, const __nv_bfloat16* wg, const __nv_bfloat16* wu,
@@ -218,6 +222,17 @@ __host__ __device__ __forceinline__ uint32_t sf_block_offset(int row, int kg) {
 __device__ __forceinline__ int clamp_live(const int* live, int max_live) {
     int n = __ldg(live);
     return n < 0 ? 0 : (n > max_live ? max_live : n);
+}
+
+// Whether a bounded wait of this forward (or of an earlier one on the same
+// workspace, until the word is cleared) gave up: the permutation may then be
+// partial, so the kernels after it do no work rather than index memory
+// through it.  status: the workspace's status words (null: not checked).
+__device__ __forceinline__ bool forward_poisoned(const unsigned* status) {
+    return status != nullptr && (*status & MOE_DEV_TIMEOUT) != 0u;
+}
+__device__ __forceinline__ int live_rows(const int* live, int max_live, const unsigned* status) {
+    return forward_poisoned(status) ? 0 : clamp_live(live, max_live);
 }
 
 }  // namespace moe

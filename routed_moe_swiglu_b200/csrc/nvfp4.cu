@@ -97,12 +97,13 @@ __global__ void __launch_bounds__(kQThreads) gather_rows_nvfp4_kernel(const uint
                                                                       const int* __restrict__ inv,
                                                                       uint32_t* __restrict__ xq,
                                                                       uint8_t* __restrict__ xs,
-                                                                      float* __restrict__ xg) {
+                                                                      float* __restrict__ xg,
+                                                                      const unsigned* status) {
     __shared__ int s_prow[kMaxTopK];
     __shared__ float s_red[kQThreads / 32];
     pdl_trigger();
     pdl_wait();
-    const int n = clamp_live(live, max_live);
+    const int n = live_rows(live, max_live, status);
     const int chunks = H / 8, chunks_out = hp / 8;
     for (int t = blockIdx.x; t < n; t += gridDim.x) {
         __syncthreads();
@@ -144,11 +145,12 @@ __global__ void __launch_bounds__(kQThreads) quantize_h_nvfp4_kernel(const float
                                                                      const int* __restrict__ inv,
                                                                      uint32_t* __restrict__ hq,
                                                                      uint8_t* __restrict__ hs,
-                                                                     float* __restrict__ hg) {
+                                                                     float* __restrict__ hg,
+                                                                     const unsigned* status) {
     __shared__ float s_red[kQThreads / 32];
     pdl_trigger();
     pdl_wait();
-    const int n = clamp_live(live, max_live);
+    const int n = live_rows(live, max_live, status);
     const int chunks = fp / 8;
     for (long long i = blockIdx.x; i < (long long)n * k; i += gridDim.x) {
         const int pr = __ldg(inv + i);  // uniform over the block
@@ -281,25 +283,26 @@ cudaError_t launch_nvfp4_quantize_rows(const __nv_bfloat16* in, long long rows, 
 }
 
 cudaError_t launch_gather_nvfp4(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
-                                const int* inv, uint8_t* xq, uint8_t* xs, float* xg, cudaStream_t s) {
+                                const int* inv, uint8_t* xq, uint8_t* xs, float* xg, const unsigned* status,
+                                cudaStream_t s) {
     long long grid = max_live;
     const long long cap = (long long)num_sms() * 16;
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
     return launch_dependent(gather_rows_nvfp4_kernel, dim3((unsigned)grid), dim3(kQThreads), 0, s,
                             reinterpret_cast<const uint4*>(x), live, max_live, H, hp, k, hp / 256, inv,
-                            reinterpret_cast<uint32_t*>(xq), xs, xg);
+                            reinterpret_cast<uint32_t*>(xq), xs, xg, status);
 }
 
 cudaError_t launch_quantize_h_nvfp4(const float* hf, const int* live, int max_live, int k, int fp, const int* inv,
-                                    uint8_t* hq, uint8_t* hs, float* hg, cudaStream_t s) {
+                                    uint8_t* hq, uint8_t* hs, float* hg, const unsigned* status, cudaStream_t s) {
     long long grid = (long long)max_live * k;
     const long long cap = (long long)num_sms() * 16;
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
     return launch_dependent(quantize_h_nvfp4_kernel, dim3((unsigned)grid), dim3(kQThreads), 0, s,
                             reinterpret_cast<const float4*>(hf), live, max_live, k, fp, fp / 256, inv,
-                            reinterpret_cast<uint32_t*>(hq), hs, hg);
+                            reinterpret_cast<uint32_t*>(hq), hs, hg, status);
 }
 
 cudaError_t launch_prepare_nvfp4(const moe_plan* p, const __nv_bfloat16* wg, const __nv_bfloat16* wu,

@@ -4,47 +4,31 @@
 // `expert_value_pass`: "each row is one route, sorted by local expert";
 // Megatron-LM PR #7830: with one rank the dispatch stages are a pass-through).
 //
-// Three deterministic passes, no atomics on positions:
-//   hist     per 256-token block, per-expert route counts (shared-memory
+// One launch, deterministic, no atomics on positions:
+//   hist     per 256-token chunk, per-expert route counts (shared-memory
 //            counters: a count does not depend on the order of increments)
-//   scan     one CTA: per-expert prefix over blocks, exclusive scan over
-//            experts -> offsets[E+1]; the same over the counts rounded up to
-//            row_align -> the padded row space the GEMMs read, and over
-//            ceil(count / tile_rows) -> the list of route tiles
-//   scatter  per block: one 32-bit lane mask per (warp, expert) gives every
-//            route its rank among earlier tokens of the block routed to the
+//   scan     a warp per expert: the counts of the chunks become exclusive
+//            prefixes over earlier chunks, and the expert's total; then every
+//            block scans the totals over experts -> offsets[E+1], the same
+//            over the counts rounded up to row_align -> the padded row space
+//            the GEMMs read, and over ceil(count / tile_rows) -> the list of
+//            route tiles
+//   scatter  per chunk: one 32-bit lane mask per (warp, expert) gives every
+//            route its rank among earlier tokens of the chunk routed to the
 //            same expert (popcount of the lower lanes plus the earlier warps)
-//            The scan also zeroes the per-tile counters and the chunk counter
-//            through which the bf16 gate/up GEMM copies x rows itself.
-// and, for MXFP8, a gather that quantises each token's x row once and writes
-// it to its padded route rows.
+// The three phases meet in two grid-wide barriers (a counter in the
+// workspace's status words, zeroed by the router kernel of the same forward;
+// every wait bounded).  With at most 1,024 live rows one block does all three
+// phases and no barrier is needed.  The scan also zeroes the per-tile
+// counters and the chunk counter through which the bf16 gate/up GEMM copies
+// x rows itself.  For MXFP8, a gather then quantises each token's x row once
+// and writes it to its padded route rows.
 #include "moe_internal.cuh"
 #include "mxfp8.cuh"
+#include "ptx.cuh"
 
 namespace moe {
 namespace {
-
-__global__ void __launch_bounds__(kTokPerBlk) route_hist_kernel(const int* __restrict__ ids,
-                                                                const int* __restrict__ live, int max_live,
-                                                                int E, int k, int* __restrict__ blkcnt) {
-    extern __shared__ int s_hist[];
-    pdl_trigger();
-    pdl_wait();
-    const int n = clamp_live(live, max_live);
-    const int t0 = blockIdx.x * kTokPerBlk;
-    if (t0 >= n) return;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
-    __syncthreads();
-    const int t = t0 + threadIdx.x;
-    if (t < n) {
-        for (int j = 0; j < k; ++j) {
-            const int e = __ldg(ids + (size_t)t * k + j);
-            if (e >= 0) atomicAdd(&s_hist[e], 1);
-        }
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) blkcnt[(size_t)blockIdx.x * E + e] = s_hist[e];
-}
 
 // Exclusive scan of one int per thread over a block of kWarps warps; returns
 // the exclusive prefix and writes the total to *total (all threads see it).
@@ -74,234 +58,246 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
     __syncthreads();
     return warp_prefix + x - v;
 }
-__device__ __forceinline__ int block_exclusive_scan_1024(int v, int* s_warp, int* total) {
-    return block_exclusive_scan<32>(v, s_warp, total);
+
+constexpr int kPermWarps = kTokPerBlk / 32;
+// Plans with at most this many live rows permute in one block, without barriers.
+constexpr int kSmallPermuteTokens = 4 * kTokPerBlk;
+
+struct PermuteArgs {
+    const int* ids;       // canonical routes [max_live, k] (-1: dropped)
+    const int* live;
+    int max_live, E, k, tile_rows, row_align;
+    int* blkcnt;          // [chunks][E]: counts, then exclusive prefixes over chunks
+    int* tot;             // [E]: routes per expert
+    int* offsets;         // [E + 1]
+    int* padoff;          // [E + 1]
+    int4* tiles;
+    int* perm;
+    int* inv;
+    int* ready;           // bf16: per-tile copy counters (zeroed here), else null
+    unsigned* status;     // status words
+    unsigned long long wait_limit_ns;
+};
+
+// Shared memory of the permute block: s_count[E] (count, then the chunk's next
+// free row), s_off[E], s_pad[E], masks[kPermWarps][E], wbase[kPermWarps][E].
+__host__ __device__ constexpr size_t permute_smem_bytes(int E) {
+    return (size_t)(3 + 2 * kPermWarps) * (size_t)E * sizeof(int);
 }
 
-__global__ void __launch_bounds__(1024) route_scan_kernel(const int* __restrict__ live, int max_live, int E,
-                                                          int tile_rows, int row_align, int* __restrict__ blkcnt,
-                                                          int* __restrict__ offsets,
-                                                          int* __restrict__ padoff, int4* __restrict__ tiles,
-                                                          int* __restrict__ ready,
-                                                          unsigned* __restrict__ status_words) {
-    __shared__ int s_warp[32];
-    pdl_trigger();
-    pdl_wait();
-    const int n = clamp_live(live, max_live);
-    const int nb = (n + kTokPerBlk - 1) / kTokPerBlk;
-    const int e = threadIdx.x;
-    int tot = 0;
-    if (e < E) {
-        // each block's count becomes the exclusive prefix over earlier blocks; the counts
-        // of 16 blocks are loaded before any is rewritten, so the loads overlap
-        constexpr int kBatch = 16;
-        for (int b0 = 0; b0 < nb; b0 += kBatch) {
-            int c[kBatch];
-#pragma unroll
-            for (int i = 0; i < kBatch; ++i) c[i] = b0 + i < nb ? blkcnt[(size_t)(b0 + i) * E + e] : 0;
-#pragma unroll
-            for (int i = 0; i < kBatch; ++i) {
-                if (b0 + i < nb) blkcnt[(size_t)(b0 + i) * E + e] = tot;
-                tot += c[i];
+// The scan over experts of per-expert counts c[e] (read through count(e)):
+// offsets, padded offsets and the tile list; thread tid owns experts
+// [tid * q, tid * q + q).  Every thread of the block calls it; s_off / s_pad
+// receive offsets[e] / padoff[e]; when `write`, the globals are written too.
+template <class CountFn>
+__device__ __forceinline__ void scan_experts(const PermuteArgs& a, CountFn count, int* s_off, int* s_pad,
+                                             int* s_warp, bool write) {
+    const int tid = threadIdx.x, E = a.E;
+    const int q = (E + kTokPerBlk - 1) / kTokPerBlk;
+    const int e0 = tid * q, e1 = min(E, e0 + q);
+    int tot = 0, nmt = 0, npad = 0;
+    for (int e = e0; e < e1; ++e) {
+        const int c = count(e);
+        tot += c;
+        nmt += (c + a.tile_rows - 1) / a.tile_rows;
+        npad += (c + a.row_align - 1) / a.row_align * a.row_align;
+    }
+    int sum_tot, sum_mt, sum_pad;
+    int ex_tot = block_exclusive_scan<kPermWarps>(tot, s_warp, &sum_tot);
+    int ex_mt = block_exclusive_scan<kPermWarps>(nmt, s_warp, &sum_mt);
+    int ex_pad = block_exclusive_scan<kPermWarps>(npad, s_warp, &sum_pad);
+    for (int e = e0; e < e1; ++e) {
+        const int c = count(e);
+        const int mt = (c + a.tile_rows - 1) / a.tile_rows;
+        s_off[e] = ex_tot;
+        s_pad[e] = ex_pad;
+        if (write) {
+            a.offsets[e] = ex_tot;
+            a.padoff[e] = ex_pad;
+            for (int i = 0; i < mt; ++i) {
+                const int rows = c - i * a.tile_rows;
+                a.tiles[ex_mt + i] = make_int4(e, ex_pad + i * a.tile_rows, rows < a.tile_rows ? rows : a.tile_rows,
+                                               ex_tot + i * a.tile_rows);
+                if (a.ready != nullptr) a.ready[ex_mt + i] = 0;
             }
         }
+        ex_tot += c;
+        ex_mt += mt;
+        ex_pad += (c + a.row_align - 1) / a.row_align * a.row_align;
     }
-    const int mt = (tot + tile_rows - 1) / tile_rows;
-    const int padded = (tot + row_align - 1) / row_align * row_align;
-    int sum_tot, sum_mt, sum_pad;
-    const int ex_tot = block_exclusive_scan_1024(tot, s_warp, &sum_tot);
-    const int ex_mt = block_exclusive_scan_1024(mt, s_warp, &sum_mt);
-    const int ex_pad = block_exclusive_scan_1024(padded, s_warp, &sum_pad);
-    if (e < E) {
-        offsets[e] = ex_tot;
-        padoff[e] = ex_pad;
-        for (int i = 0; i < mt; ++i) {
-            const int rows = tot - i * tile_rows;
-            tiles[ex_mt + i] =
-                make_int4(e, ex_pad + i * tile_rows, rows < tile_rows ? rows : tile_rows, ex_tot + i * tile_rows);
-            if (ready != nullptr) ready[ex_mt + i] = 0;
-        }
-    }
-    if (e == 0) {
-        offsets[E] = sum_tot;
-        padoff[E] = sum_pad;
-        status_words[kStNumMTiles] = (unsigned)sum_mt;
-        status_words[kStTotalRoutes] = (unsigned)sum_tot;
-        status_words[kStCopyNext] = 0u;
+    if (write && tid == 0) {
+        a.offsets[E] = sum_tot;
+        a.padoff[E] = sum_pad;
+        a.status[kStTotalRoutes] = (unsigned)sum_tot;
+        a.status[kStCopyNext] = 0u;
+        __threadfence();
+        a.status[kStNumMTiles] = (unsigned)sum_mt;
     }
 }
 
-__global__ void __launch_bounds__(kTokPerBlk) route_scatter_kernel(
-    const int* __restrict__ ids, const int* __restrict__ live, int max_live, int E, int k,
-    const int* __restrict__ blkprefix, const int* __restrict__ offsets, const int* __restrict__ padoff,
-    int* __restrict__ perm, int* __restrict__ inv) {
-    extern __shared__ uint32_t s_mem[];
-    pdl_trigger();
-    pdl_wait();
-    const int n = clamp_live(live, max_live);
-    const int t0 = blockIdx.x * kTokPerBlk;
-    if (t0 >= n) return;
-    constexpr int kWarps = kTokPerBlk / 32;
-    uint32_t* masks = s_mem;                                // [kWarps][E]
-    int* wbase = reinterpret_cast<int*>(s_mem + kWarps * E);  // [kWarps][E]
-    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) masks[i] = 0u;
+// Stable scatter of the 256 tokens from t0: each route's row is s_base[e]
+// (the chunk's first free row of expert e) plus its rank in the chunk;
+// s_base[e] is advanced past the chunk.  s_off / s_pad map a row to its
+// padded row.
+__device__ __forceinline__ void scatter_chunk(const PermuteArgs& a, int n, int t0, int* s_base, const int* s_off,
+                                              const int* s_pad, uint32_t* masks, int* wbase) {
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, E = a.E, k = a.k;
+    for (int i = tid; i < kPermWarps * E; i += kTokPerBlk) masks[i] = 0u;
     __syncthreads();
-    const int t = t0 + threadIdx.x;
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = t0 + tid;
     const bool is_live = t < n;
     int my_e[kMaxTopK];
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
         my_e[j] = -1;
         if (j < k && is_live) {
-            my_e[j] = __ldg(ids + (size_t)t * k + j);
+            my_e[j] = __ldg(a.ids + (size_t)t * k + j);
             if (my_e[j] >= 0) atomicOr(&masks[w * E + my_e[j]], 1u << lane);
         }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int base = offsets[e] + blkprefix[(size_t)blockIdx.x * E + e];
+    for (int e = tid; e < E; e += kTokPerBlk) {
+        int base = s_base[e];
 #pragma unroll
-        for (int w2 = 0; w2 < kWarps; ++w2) {
+        for (int w2 = 0; w2 < kPermWarps; ++w2) {
             wbase[w2 * E + e] = base;
             base += __popc(masks[w2 * E + e]);
         }
+        s_base[e] = base;
     }
     __syncthreads();
-    if (!is_live) return;
-    const uint32_t lower = (1u << lane) - 1u;
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-        if (j < k) {
-            const int e = my_e[j];
-            if (e < 0) {
-                inv[(size_t)t * k + j] = -1;
-            } else {
-                const int row = wbase[w * E + e] + __popc(masks[w * E + e] & lower);
-                perm[row] = t * k + j;
-                inv[(size_t)t * k + j] = padoff[e] + row - offsets[e];
-            }
-        }
-    }
-}
-
-// Plans of at most kSmallPermuteTokens live rows: the three passes above in
-// one 256-thread block, one launch instead of three (each dependent launch
-// waits for its predecessor to finish, which at decode sizes costs more than
-// the work).  Tokens are taken in chunks of 256 with a running per-expert
-// base, so every route gets the same row as in the three-pass form.
-constexpr int kSmallPermuteTokens = 4 * kTokPerBlk;
-
-__global__ void __launch_bounds__(kTokPerBlk) route_permute_small_kernel(
-    const int* __restrict__ ids, const int* __restrict__ live, int max_live, int E, int k, int tile_rows,
-    int row_align, int* __restrict__ offsets, int* __restrict__ padoff, int4* __restrict__ tiles,
-    int* __restrict__ perm, int* __restrict__ inv, int* __restrict__ ready, unsigned* __restrict__ status_words) {
-    constexpr int kWarps = kTokPerBlk / 32;
-    extern __shared__ int s_small[];
-    int* s_base = s_small;                                         // [E] count, then next free row
-    int* s_off = s_small + E;                                      // [E] offsets[e]
-    int* s_pad = s_small + 2 * E;                                  // [E] padoff[e]
-    uint32_t* masks = reinterpret_cast<uint32_t*>(s_small + 3 * E);  // [kWarps][E]
-    int* wbase = s_small + (3 + kWarps) * E;                       // [kWarps][E]
-    __shared__ int s_warp[32];
-    pdl_trigger();
-    pdl_wait();
-    const int n = clamp_live(live, max_live);
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-
-    // histogram
-    for (int e = tid; e < E; e += kTokPerBlk) s_base[e] = 0;
-    __syncthreads();
-    for (int i = tid; i < n * k; i += kTokPerBlk) {
-        const int e = __ldg(ids + i);
-        if (e >= 0) atomicAdd(&s_base[e], 1);
-    }
-    __syncthreads();
-
-    // scan: thread tid owns the experts [tid * q, tid * q + q)
-    const int q = (E + kTokPerBlk - 1) / kTokPerBlk;
-    const int e0 = tid * q, e1 = min(E, e0 + q);
-    int tot = 0, nmt = 0, npad = 0;
-    for (int e = e0; e < e1; ++e) {
-        const int c = s_base[e];
-        tot += c;
-        nmt += (c + tile_rows - 1) / tile_rows;
-        npad += (c + row_align - 1) / row_align * row_align;
-    }
-    int sum_tot, sum_mt, sum_pad;
-    int ex_tot = block_exclusive_scan<kWarps>(tot, s_warp, &sum_tot);
-    int ex_mt = block_exclusive_scan<kWarps>(nmt, s_warp, &sum_mt);
-    int ex_pad = block_exclusive_scan<kWarps>(npad, s_warp, &sum_pad);
-    for (int e = e0; e < e1; ++e) {
-        const int c = s_base[e];
-        const int mt = (c + tile_rows - 1) / tile_rows;
-        offsets[e] = ex_tot;
-        padoff[e] = ex_pad;
-        s_off[e] = ex_tot;
-        s_pad[e] = ex_pad;
-        for (int i = 0; i < mt; ++i) {
-            const int rows = c - i * tile_rows;
-            tiles[ex_mt + i] =
-                make_int4(e, ex_pad + i * tile_rows, rows < tile_rows ? rows : tile_rows, ex_tot + i * tile_rows);
-            if (ready != nullptr) ready[ex_mt + i] = 0;
-        }
-        s_base[e] = ex_tot;  // the scatter's next free row of expert e
-        ex_tot += c;
-        ex_mt += mt;
-        ex_pad += (c + row_align - 1) / row_align * row_align;
-    }
-    if (tid == 0) {
-        offsets[E] = sum_tot;
-        padoff[E] = sum_pad;
-        status_words[kStNumMTiles] = (unsigned)sum_mt;
-        status_words[kStTotalRoutes] = (unsigned)sum_tot;
-        status_words[kStCopyNext] = 0u;
-    }
-
-    // stable scatter, 256 tokens at a time (as route_scatter_kernel per block)
-    const uint32_t lower = (1u << lane) - 1u;
-    for (int t0 = 0; t0 < n; t0 += kTokPerBlk) {
-        for (int i = tid; i < kWarps * E; i += kTokPerBlk) masks[i] = 0u;
-        __syncthreads();
-        const int t = t0 + tid;
-        const bool is_live = t < n;
-        int my_e[kMaxTopK];
+    if (is_live) {
+        const uint32_t lower = (1u << lane) - 1u;
 #pragma unroll
         for (int j = 0; j < kMaxTopK; ++j) {
-            my_e[j] = -1;
-            if (j < k && is_live) {
-                my_e[j] = __ldg(ids + (size_t)t * k + j);
-                if (my_e[j] >= 0) atomicOr(&masks[w * E + my_e[j]], 1u << lane);
-            }
-        }
-        __syncthreads();
-        for (int e = tid; e < E; e += kTokPerBlk) {
-            int base = s_base[e];
-#pragma unroll
-            for (int w2 = 0; w2 < kWarps; ++w2) {
-                wbase[w2 * E + e] = base;
-                base += __popc(masks[w2 * E + e]);
-            }
-            s_base[e] = base;
-        }
-        __syncthreads();
-        if (is_live) {
-#pragma unroll
-            for (int j = 0; j < kMaxTopK; ++j) {
-                if (j < k) {
-                    const int e = my_e[j];
-                    if (e < 0) {
-                        inv[(size_t)t * k + j] = -1;
-                    } else {
-                        const int row = wbase[w * E + e] + __popc(masks[w * E + e] & lower);
-                        perm[row] = t * k + j;
-                        inv[(size_t)t * k + j] = s_pad[e] + row - s_off[e];
-                    }
+            if (j < k) {
+                const int e = my_e[j];
+                if (e < 0) {
+                    a.inv[(size_t)t * k + j] = -1;
+                } else {
+                    const int row = wbase[w * E + e] + __popc(masks[w * E + e] & lower);
+                    a.perm[row] = t * k + j;
+                    a.inv[(size_t)t * k + j] = s_pad[e] + row - s_off[e];
                 }
             }
         }
-        __syncthreads();  // masks and wbase are rewritten by the next chunk
     }
+    __syncthreads();  // masks and wbase are rewritten by the next chunk
+}
+
+// Grid-wide barrier of the `parts` participating blocks (all resident: the
+// grid is at most one block per SM and the next kernel is released only after
+// the barriers).  Returns false when the wait ran out (MOE_DEV_TIMEOUT set).
+__device__ __forceinline__ bool permute_grid_barrier(const PermuteArgs& a, int target, int* s_flag) {
+    __syncthreads();  // the block's writes precede the arrival (bar.sync is cumulative)
+    if (threadIdx.x == 0) {
+        int* bar = reinterpret_cast<int*>(a.status + kStPermBar);
+        __threadfence();
+        red_release_gpu_add(bar, 1);
+        volatile int never = 0;
+        const bool ok = wait_count_bounded(bar, target, &never, a.wait_limit_ns);
+        if (!ok) atomicOr(a.status + kStFlags, MOE_DEV_TIMEOUT);
+        __threadfence();
+        *s_flag = ok ? 1 : 0;
+    }
+    __syncthreads();
+    return *s_flag != 0;
+}
+
+__global__ void __launch_bounds__(kTokPerBlk) route_permute_kernel(const PermuteArgs a) {
+    extern __shared__ int s_perm[];
+    __shared__ int s_warp[32];
+    __shared__ int s_flag;
+    const int E = a.E, k = a.k;
+    int* s_count = s_perm;
+    int* s_off = s_perm + E;
+    int* s_pad = s_perm + 2 * E;
+    uint32_t* masks = reinterpret_cast<uint32_t*>(s_perm + 3 * E);
+    int* wbase = s_perm + (3 + kPermWarps) * E;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // No early launch of the next kernel: it is released once every block of
+    // this grid has passed the barriers (see permute_grid_barrier).
+    pdl_wait();
+    const int n = clamp_live(a.live, a.max_live);
+
+    if (n <= kSmallPermuteTokens) {
+        // one block: histogram, scan, scatter in chunks of 256 with a running base
+        if (blockIdx.x == 0) {
+            for (int e = tid; e < E; e += kTokPerBlk) s_count[e] = 0;
+            __syncthreads();
+            for (int i = tid; i < n * k; i += kTokPerBlk) {
+                const int e = __ldg(a.ids + i);
+                if (e >= 0) atomicAdd(&s_count[e], 1);
+            }
+            __syncthreads();
+            scan_experts(a, [&](int e) { return s_count[e]; }, s_off, s_pad, s_warp, true);
+            __syncthreads();
+            for (int e = tid; e < E; e += kTokPerBlk) s_count[e] = s_off[e];  // next free row of expert e
+            __syncthreads();
+            for (int t0 = 0; t0 < n; t0 += kTokPerBlk) scatter_chunk(a, n, t0, s_count, s_off, s_pad, masks, wbase);
+        }
+        pdl_trigger();
+        return;
+    }
+
+    const int nb = (n + kTokPerBlk - 1) / kTokPerBlk;  // chunks of 256 tokens
+    const int parts = (int)gridDim.x < nb ? (int)gridDim.x : nb;
+    if ((int)blockIdx.x >= parts) {
+        pdl_trigger();
+        return;
+    }
+    // phase 1: the histogram of each chunk this block owns
+    for (int c = blockIdx.x; c < nb; c += parts) {
+        for (int e = tid; e < E; e += kTokPerBlk) s_count[e] = 0;
+        __syncthreads();
+        const int t = c * kTokPerBlk + tid;
+        if (t < n)
+            for (int j = 0; j < k; ++j) {
+                const int e = __ldg(a.ids + (size_t)t * k + j);
+                if (e >= 0) atomicAdd(&s_count[e], 1);
+            }
+        __syncthreads();
+        for (int e = tid; e < E; e += kTokPerBlk) a.blkcnt[(size_t)c * E + e] = s_count[e];
+        __syncthreads();
+    }
+    bool ok = permute_grid_barrier(a, parts, &s_flag);
+    // phase 2: a warp per expert turns its column of chunk counts into exclusive
+    // prefixes over earlier chunks (32 chunks per step, in place) and its total
+    if (ok) {
+        for (int e = blockIdx.x * kPermWarps + warp; e < E; e += parts * kPermWarps) {
+            int carry = 0;
+            for (int c0 = 0; c0 < nb; c0 += 32) {
+                const int c = c0 + lane;
+                const int v = c < nb ? __ldcg(a.blkcnt + (size_t)c * E + e) : 0;
+                int x = v;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (lane >= off) x += y;
+                }
+                if (c < nb) a.blkcnt[(size_t)c * E + e] = carry + x - v;
+                carry += __shfl_sync(0xffffffffu, x, 31);
+            }
+            if (lane == 0) a.tot[e] = carry;
+        }
+        ok = permute_grid_barrier(a, 2 * parts, &s_flag);
+    }
+    if (!ok) {
+        // a barrier ran out: the GEMMs get an empty tile list instead of a partial one
+        if (blockIdx.x == 0 && tid == 0) a.status[kStNumMTiles] = 0u;
+        pdl_trigger();
+        return;
+    }
+    // phase 3: every block scans the totals (block 0 writes the results), then
+    // scatters its chunks from their first free rows
+    scan_experts(a, [&](int e) { return __ldcg(a.tot + e); }, s_off, s_pad, s_warp, blockIdx.x == 0);
+    __syncthreads();
+    for (int c = blockIdx.x; c < nb; c += parts) {
+        for (int e = tid; e < E; e += kTokPerBlk) s_count[e] = s_off[e] + __ldcg(a.blkcnt + (size_t)c * E + e);
+        __syncthreads();
+        scatter_chunk(a, n, c * kTokPerBlk, s_count, s_off, s_pad, masks, wbase);
+    }
+    pdl_trigger();
 }
 
 constexpr int kRowThreads = 128;
@@ -316,11 +312,12 @@ __global__ void __launch_bounds__(kRowThreads) gather_rows_mxfp8_kernel(const ui
                                                                         int H, int hp, int k, int ks1,
                                                                         const int* __restrict__ inv,
                                                                         uint2* __restrict__ xq,
-                                                                        uint8_t* __restrict__ xs) {
+                                                                        uint8_t* __restrict__ xs,
+                                                                        const unsigned* status) {
     __shared__ int s_prow[kMaxTopK];
     pdl_trigger();
     pdl_wait();
-    const int n = clamp_live(live, max_live);
+    const int n = live_rows(live, max_live, status);
     const int chunks = H / 8;       // 8 elements per thread and chunk
     const int chunks_out = hp / 8;  // destination pitch
     for (int t = blockIdx.x; t < n; t += gridDim.x) {
@@ -372,12 +369,12 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(const float4* __re
                                                               const int* __restrict__ inv,
                                                               const float* __restrict__ probs,
                                                               const int* __restrict__ live, int max_live, int H,
-                                                              int k, void* __restrict__ out) {
+                                                              int k, void* __restrict__ out, const unsigned* status) {
     __shared__ int s_prow[kMaxTopK];
     __shared__ float s_p[kMaxTopK];
     pdl_trigger();
     pdl_wait();
-    const int n = clamp_live(live, max_live);
+    const int n = live_rows(live, max_live, status);
     const int chunks = H / 4;
     const int max_parts = (chunks + kRowThreads - 1) / kRowThreads;
     int parts = n > 0 ? (int)(gridDim.x / (unsigned)n) : 1;
@@ -441,68 +438,60 @@ int grid_for_warps(long long items, int warps_per_block, int per_sm) {
 cudaError_t launch_permute(const moe_plan* p, const int* live, int* r_ids, int* blkcnt, int* offsets,
                            int* padoff, int4* tiles, int* perm, int* inv, int* ready, unsigned* status_words,
                            cudaStream_t s) {
-    const int E = p->d.num_experts, k = p->d.top_k;
-    const int max_live = (int)p->max_live;
-    const int nblk = p->nblk;
-    cudaError_t err;
-    if (max_live <= kSmallPermuteTokens) {
-        const size_t smem = (size_t)(3 + 2 * (kTokPerBlk / 32)) * E * sizeof(int);
-        if (smem > 48 * 1024) {
-            static int configured_device = -1;  // once per device, at the largest size any plan can ask for
-            int dev = 0;
-            err = cudaGetDevice(&dev);
-            if (err != cudaSuccess) return err;
-            if (configured_device != dev) {
-                err = cudaFuncSetAttribute(route_permute_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)((3 + 2 * (kTokPerBlk / 32)) * kMaxExperts * sizeof(int)));
-                if (err != cudaSuccess) return err;
-                configured_device = dev;
-            }
-        }
-        return launch_dependent(route_permute_small_kernel, dim3(1), dim3(kTokPerBlk), smem, s, r_ids, live,
-                                max_live, E, k, p->tile_rows, p->row_align, offsets, padoff, tiles, perm, inv, ready,
-                                status_words);
-    }
-    err = launch_dependent(route_hist_kernel, dim3(nblk), dim3(kTokPerBlk), E * sizeof(int), s, r_ids,
-                                       live, max_live, E, k, blkcnt);
-    if (err != cudaSuccess) return err;
-    err = launch_dependent(route_scan_kernel, dim3(1), dim3(1024), 0, s, live, max_live, E, p->tile_rows,
-                           p->row_align, blkcnt, offsets, padoff, tiles, ready, status_words);
-    if (err != cudaSuccess) return err;
-    const size_t smem = (size_t)(kTokPerBlk / 32) * E * 8;
+    const int E = p->d.num_experts;
+    PermuteArgs a;
+    a.ids = r_ids;
+    a.live = live;
+    a.max_live = (int)p->max_live;
+    a.E = E;
+    a.k = p->d.top_k;
+    a.tile_rows = p->tile_rows;
+    a.row_align = p->row_align;
+    a.blkcnt = blkcnt;
+    a.tot = blkcnt + (size_t)p->nblk * E;  // the workspace's count area has E ints past the chunks'
+    a.offsets = offsets;
+    a.padoff = padoff;
+    a.tiles = tiles;
+    a.perm = perm;
+    a.inv = inv;
+    a.ready = ready;
+    a.status = status_words;
+    a.wait_limit_ns = kWaitLimitNs;
+    const size_t smem = permute_smem_bytes(E);
     if (smem > 48 * 1024) {
-        // once per device, at the largest size any plan can ask for
-        static int configured_device = -1;
+        static int configured_device = -1;  // once per device, at the largest size any plan can ask for
         int dev = 0;
-        err = cudaGetDevice(&dev);
+        cudaError_t err = cudaGetDevice(&dev);
         if (err != cudaSuccess) return err;
         if (configured_device != dev) {
-            err = cudaFuncSetAttribute(route_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)((kTokPerBlk / 32) * kMaxExperts * 8));
+            err = cudaFuncSetAttribute(route_permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)permute_smem_bytes(kMaxExperts));
             if (err != cudaSuccess) return err;
             configured_device = dev;
         }
     }
-    return launch_dependent(route_scatter_kernel, dim3(nblk), dim3(kTokPerBlk), smem, s, r_ids, live, max_live, E, k,
-                            blkcnt, offsets, padoff, perm, inv);
+    // at most one block per SM: the blocks meet in grid-wide barriers
+    int grid = p->nblk < num_sms() ? p->nblk : num_sms();
+    if (grid < 1) grid = 1;
+    return launch_dependent(route_permute_kernel, dim3((unsigned)grid), dim3(kTokPerBlk), smem, s, a);
 }
 
 cudaError_t launch_gather_mxfp8(const __nv_bfloat16* x, const int* live, int max_live, int H, int hp, int k,
-                                const int* inv, uint8_t* xq, uint8_t* xs, cudaStream_t s) {
+                                const int* inv, uint8_t* xq, uint8_t* xs, const unsigned* status, cudaStream_t s) {
     const int grid = grid_for_warps(max_live, 1, 16);
     return launch_dependent(gather_rows_mxfp8_kernel, dim3(grid), dim3(kRowThreads), 0, s,
                             reinterpret_cast<const uint4*>(x), live, max_live, H, hp, k, hp / 128, inv,
-                            reinterpret_cast<uint2*>(xq), xs);
+                            reinterpret_cast<uint2*>(xq), xs, status);
 }
 
 cudaError_t launch_combine(const float* y, const int* inv, const float* probs, const int* live, int max_live,
-                           int H, int k, void* out, bool out_bf16, cudaStream_t s) {
+                           int H, int k, void* out, bool out_bf16, const unsigned* status, cudaStream_t s) {
     const dim3 grid((unsigned)grid_for_warps((long long)max_live * ((H / 4 + kRowThreads - 1) / kRowThreads), 1, 16));
     if (out_bf16)
         return launch_dependent(combine_kernel<true>, grid, dim3(kRowThreads), 0, s,
-                                reinterpret_cast<const float4*>(y), inv, probs, live, max_live, H, k, out);
+                                reinterpret_cast<const float4*>(y), inv, probs, live, max_live, H, k, out, status);
     return launch_dependent(combine_kernel<false>, grid, dim3(kRowThreads), 0, s,
-                            reinterpret_cast<const float4*>(y), inv, probs, live, max_live, H, k, out);
+                            reinterpret_cast<const float4*>(y), inv, probs, live, max_live, H, k, out, status);
 }
 
 }  // namespace moe

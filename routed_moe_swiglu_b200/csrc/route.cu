@@ -41,8 +41,10 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
     pdl_trigger();
     pdl_wait();
     int n = __ldg(live);
-    if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0 && (n < 0 || n > max_live))
-        atomicOr(status, MOE_DEV_LIVE_CLAMPED);
+    if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+        if (n < 0 || n > max_live) atomicOr(status, MOE_DEV_LIVE_CLAMPED);
+        status[kStPermBar] = 0u;  // the permute that follows meets in barriers on this count
+    }
     n = n < 0 ? 0 : (n > max_live ? max_live : n);
 
     const int lane = threadIdx.x & 31;
@@ -109,8 +111,10 @@ __global__ void __launch_bounds__(256) canon_routes_kernel(const int* __restrict
     pdl_trigger();
     pdl_wait();
     int n = __ldg(live);
-    if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0 && (n < 0 || n > max_live))
-        atomicOr(status, MOE_DEV_LIVE_CLAMPED);
+    if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+        if (n < 0 || n > max_live) atomicOr(status, MOE_DEV_LIVE_CLAMPED);
+        status[kStPermBar] = 0u;  // the permute that follows meets in barriers on this count
+    }
     n = n < 0 ? 0 : (n > max_live ? max_live : n);
     for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
         int id[kMaxTopK];

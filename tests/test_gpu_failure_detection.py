@@ -60,3 +60,28 @@ def test_bounded_wait_rejects_bad_arguments():
         assert ei.value.code == rm.MOE_ERR_INVALID_ARG
     torch.cuda.synchronize()
     assert status.item() == 0
+
+
+@pytest.mark.parametrize("precision", ["bf16", "mxfp8", "nvfp4"])
+def test_forward_does_no_work_while_a_timeout_is_flagged(precision):
+    """A forward whose workspace carries MOE_DEV_TIMEOUT (set here on the host,
+    as a wait that ran out would set it) writes no output rows and reads no
+    permutation: every kernel after the router sees the bit and does nothing.
+    Cleared, the same workspace serves a correct forward again.  Shapes past
+    1,024 live rows, so the permute runs its multi-block form."""
+    H, F, E, k, T = 256, 256, 16, 4, 1500
+    x, logits, weights = workloads.small_case(H, F, E, k, T, seed=77)
+    m = GpuMoe(H, F, E, k, T, weights, precision=precision)
+    m.clear_status()
+    good = m.forward(x.cuda(), T, logits=logits.cuda()).cpu()
+    assert m.status() == 0
+    ws_status = m.ws[:4].view(torch.int32)
+    ws_status.fill_(rm.MOE_DEV_TIMEOUT)
+    out = m.forward(x.cuda(), T, logits=logits.cuda(), sentinel=-5.0)
+    torch.cuda.synchronize()
+    assert torch.all(out == -5.0)
+    assert m.status() & rm.MOE_DEV_TIMEOUT
+    m.clear_status()
+    again = m.forward(x.cuda(), T, logits=logits.cuda()).cpu()
+    assert m.status() == 0
+    assert torch.equal(again.view(torch.int32), good.view(torch.int32))
