@@ -56,7 +56,7 @@
 namespace moe {
 namespace {
 
-constexpr int kStages = 3;
+constexpr int kStagesMax = 5;  // pipeline stages per launch: 3..5, by the widest route tile (see StageCfg)
 constexpr int kEpiWarps = 8;
 constexpr int kCopyWarps = 2;                           // gate/up: x rows of large tiles into their route rows
 constexpr int kPairM = 256;                             // M of the pair MMA (weight rows)
@@ -64,7 +64,7 @@ constexpr int kAtoms = 2;                               // 64-element (128-byte)
 constexpr int kStageK = kAtoms * kBK;                   // 128 K elements per stage
 constexpr uint32_t kAtomBytes = 128 * kBK * 2;          // 16 KB: 128 rows x 128 bytes
 constexpr uint32_t kABytes = kAtoms * kAtomBytes;       // 32 KB: this CTA's 128 weight rows
-constexpr uint32_t kBBytes = kAtoms * kAtomBytes;       // up to 32 KB: this CTA's N/2 <= 128 route rows
+constexpr uint32_t kBBytesMax = kAtoms * kAtomBytes;    // up to 32 KB: this CTA's N/2 <= 128 route rows
 constexpr uint32_t kAccCols = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kHTBytes = 32 * 16 * 2 + 64;         // gate/up: h of 32 routes x 16 f, bf16 (+ bank offset)
@@ -77,13 +77,16 @@ struct PairCfg {
     static constexpr int kThreads = (2 + kEpiWarps + (kMode == 0 ? kCopyWarps : 0)) * 32;
     // one transpose box per epilogue warp
     static constexpr uint32_t kEpiBytes = kEpiWarps * (kMode == 0 ? kH0Bytes : kYTBytes);
-    static constexpr size_t kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kEpiBytes + 256;
+    // the stages: gate/up up to 5 x (32 + 8) KB, down up to 4 x (32 + 16) KB; 3 x (32 + 32) KB at most width
+    static constexpr uint32_t kStageRegion = kMode == 0 ? 5 * (kABytes + 8192) : 4 * (kABytes + 16384);
+    static constexpr size_t kSmemBytes = 1024 + kStageRegion + kEpiBytes + 256;
     static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kStageRegion >= 3 * (kABytes + kBBytesMax), "three full-width stages");
 };
 
 struct __align__(8) Barriers {
-    uint64_t full[kStages];   // CTA 0's counts both CTAs' loads of a stage
-    uint64_t empty[kStages];  // each CTA's: its stage may be refilled
+    uint64_t full[kStagesMax];   // CTA 0's counts both CTAs' loads of a stage
+    uint64_t empty[kStagesMax];  // each CTA's: its stage may be refilled
     uint64_t acc_full[2];     // each CTA's: its accumulator rows are ready
     uint64_t acc_empty[2];    // CTA 0's: both CTAs drained the accumulator
     uint64_t done;
@@ -106,6 +109,23 @@ __device__ __forceinline__ float swiglu_value(float g, float u, float clamp) {
 // Routes of a tile rounded up to the MMA's N granularity (both CTAs hold N/2 rows of B).
 __device__ __forceinline__ int tile_n(int nvalid) { return (nvalid + 31) & ~31; }
 
+// The pipeline of one launch, from the widest route tile of the forward
+// (known after the permute): narrow tiles (decode) leave room for more stages
+// in flight.  Weight slots (kABytes each) come first, at multiples of 32 KB,
+// then the route-row slots.  Every CTA and role of the launch derives the same
+// configuration.
+struct StageCfg {
+    int n;          // stages
+    uint32_t b;     // route-row slot bytes
+};
+template <int kMode>
+__device__ __forceinline__ StageCfg stage_cfg(int widest_tile) {
+    const int hb = tile_n(widest_tile) >> 1;  // route rows per CTA
+    if (kMode == 0 && hb <= 32) return {5, 8192u};
+    if (hb <= 64) return {4, 16384u};
+    return {3, kBBytesMax};
+}
+
 template <int kMode>  // 0: gate/up + SwiGLU -> bf16 h;  1: down -> fp32 y
 __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUtensorMap* tmX, const BoxMaps8* tmB,
                                                const GemmParams& p) {
@@ -113,8 +133,7 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + kStages * kABytes;
-    uint8_t* sEpi = sB + kStages * kBBytes;
+    uint8_t* sEpi = smem + PairCfg<kMode>::kStageRegion;
     Barriers* bars = reinterpret_cast<Barriers*>(sEpi + kEpiBytes);
     volatile int* abort_flag = &bars->abort_flag;
 
@@ -127,7 +146,7 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
     pdl_trigger();
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kStagesMax; ++s) {
             mbar_init(&bars->full[s], 1);
             mbar_init(&bars->empty[s], 1);
         }
@@ -153,6 +172,10 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
     const int num_m = forward_poisoned(p.status_words) ? 0 : (int)p.status_words[kStNumMTiles];
     const int total_tiles = num_m * p.n_tiles;
     const int kb_count = p.k_blocks;
+    const StageCfg sc = stage_cfg<kMode>((int)p.status_words[kStMaxTileRows]);
+    const int kStages = sc.n;
+    const uint32_t kBBytes = sc.b;
+    uint8_t* sB = smem + kStages * kABytes;
 
     if (warp == 0) {
         // ---------------- TMA producer (both CTAs; lane 0 waits and loads A, and B of the down GEMM)
@@ -163,8 +186,8 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        int last_phase[kStages];
-        for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
+        int last_phase[kStagesMax];
+        for (int s = 0; s < kStagesMax; ++s) last_phase[s] = -1;
         for (int t = pair; t < total_tiles && ok; t += npairs) {
             const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
             const int4 ti = __ldg(p.tiles + mt);

@@ -49,7 +49,7 @@
 namespace moe {
 namespace {
 
-constexpr int kStages = 3;
+constexpr int kStagesMax = 4;  // pipeline stages per launch: 3 or 4, by the widest route tile
 constexpr int kThreads = 192;
 constexpr int kTileM = 128;                            // weight rows per tile
 constexpr int kMaxN = 128;                             // routes per tile
@@ -57,7 +57,9 @@ constexpr int kAtoms = 2;                              // 128-element K blocks (
 constexpr uint32_t kAtomBytesA = kTileM * kBK8;        // 16 KB
 constexpr uint32_t kABytes = kAtoms * kAtomBytesA;     // 32 KB
 constexpr uint32_t kBBytes = kAtoms * kMaxN * kBK8;    // up to 32 KB
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
+// the stages: 4 x (32 + 16) KB when every route tile holds at most 64 routes, else 3 x (32 + 32) KB
+constexpr uint32_t kStageRegion = 3 * (kABytes + kBBytes);
+static_assert(kStageRegion == 4 * (kABytes + kBBytes / 2), "both pipelines fill the stage region");
 // Scale blocks: MXFP8 (kFmt 0) has one 512-byte block per operand and 128-byte K block
 // (4 MMAs, a byte each); NVFP4 (kFmt 1) has one per 64-element MMA step, four per K block.
 template <int kFmt>
@@ -77,15 +79,15 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kStageHBytes = 32 * 64 * 4;         // gate/up: fp32 h of 32 routes x 64 f
 constexpr uint32_t kYTBytes = 32 * 32 * 4;             // down: fp32 y of 32 routes x 32 columns, per warp
 constexpr uint32_t kEpiBytes = 2 * kStageHBytes > 4 * kYTBytes ? 2 * kStageHBytes : 4 * kYTBytes;
-constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kSfBytes + kEpiBytes + 256;
+constexpr size_t kSmemBytes = 1024 + kStageRegion + kSfBytes + kEpiBytes + 256;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kSfCol0 + SfCfg<1>::kColsPerStage * kStages <= kTmemCols, "TMEM budget");
+static_assert(kSfCol0 + SfCfg<1>::kColsPerStage * kStagesMax <= kTmemCols, "TMEM budget");
 static_assert(kEpiBytes >= 4 * 32 * 32 * 4, "squared-ReLU epilogue boxes");
 constexpr uint32_t kEpiBar = 1;                        // named barrier of the 4 epilogue warps
 
 struct __align__(8) Barriers {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[kStagesMax];
+    uint64_t empty[kStagesMax];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t sf_empty[2];
@@ -162,12 +164,10 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
     using Sf = SfCfg<kFmt>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sSf = smem + kStages * kStageBytes;  // [buffer][A/B][8][512]
+    uint8_t* sSf = smem + kStageRegion;  // [buffer][A/B][8][512]
     uint8_t* sEpi = sSf + kSfBytes;
     Barriers* bars = reinterpret_cast<Barriers*>(sEpi + kEpiBytes);
     volatile int* abort_flag = &bars->abort_flag;
-    auto stage_a = [&](int s) { return smem + s * kStageBytes; };
-    auto stage_b = [&](int s) { return smem + s * kStageBytes + kABytes; };
     auto sf_buf = [&](int b, int ab) { return sSf + (size_t)(b * 2 + ab) * kSfGroupBytes; };
 
     const int warp = threadIdx.x >> 5;
@@ -175,7 +175,7 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
     pdl_trigger();
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kStagesMax; ++s) {
             mbar_init(&bars->full[s], 1);
             mbar_init(&bars->empty[s], 1);
         }
@@ -199,6 +199,12 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
     pdl_wait();  // the tile list, route rows, scales and status words come from earlier kernels
 
     const int num_m = forward_poisoned(p.status_words) ? 0 : (int)p.status_words[kStNumMTiles];
+    // the pipeline of this launch, from the widest route tile of the forward (every role
+    // derives the same): weight slots first, at multiples of 32 KB, then the route-row slots
+    const int kStages = tile_n((int)p.status_words[kStMaxTileRows]) <= 64 ? 4 : 3;
+    const uint32_t b_slot = kStages == 4 ? kBBytes / 2 : kBBytes;
+    auto stage_a = [&](int s) { return smem + s * kABytes; };
+    auto stage_b = [&](int s) { return smem + kStages * kABytes + s * b_slot; };
     const int total_tiles = num_m * p.n_tiles;
     const int nblk = p.k_blocks;               // K blocks of 128
     const int kb_count = (nblk + 1) / kAtoms;  // stages of 256 (the last may hold one block)
@@ -211,8 +217,8 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
             uint32_t phase = 0;
             uint32_t groups = 0;  // scale-factor groups issued so far
             bool ok = true;
-            int last_phase[kStages];
-            for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
+            int last_phase[kStagesMax];
+            for (int s = 0; s < kStagesMax; ++s) last_phase[s] = -1;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
                 const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
                 const int4 ti = __ldg(p.tiles + mt);

@@ -35,8 +35,17 @@ constexpr int kMaxExperts = 1024;
 
 // Status word layout (uint32 words at the start of the workspace).
 // kStPermBar: arrivals at the permute's grid-wide barriers, zeroed by the router kernel
-// (route or canonicalise) that precedes the permute in every forward.
-enum : int { kStFlags = 0, kStNumMTiles = 1, kStTotalRoutes = 2, kStCopyNext = 3, kStPermBar = 4, kStWords = 64 };
+// (route or canonicalise) that precedes the permute in every forward.  kStMaxTileRows:
+// the most routes in one route tile of this forward (the GEMMs size their pipelines by it).
+enum : int {
+    kStFlags = 0,
+    kStNumMTiles = 1,
+    kStTotalRoutes = 2,
+    kStCopyNext = 3,
+    kStPermBar = 4,
+    kStMaxTileRows = 5,
+    kStWords = 64
+};
 
 // Default bound of any on-device wait before the kernel gives up (ns).
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;

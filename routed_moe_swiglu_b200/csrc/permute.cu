@@ -95,13 +95,21 @@ __device__ __forceinline__ void scan_experts(const PermuteArgs& a, CountFn count
     const int tid = threadIdx.x, E = a.E;
     const int q = (E + kTokPerBlk - 1) / kTokPerBlk;
     const int e0 = tid * q, e1 = min(E, e0 + q);
-    int tot = 0, nmt = 0, npad = 0;
+    int tot = 0, nmt = 0, npad = 0, widest = 0;
     for (int e = e0; e < e1; ++e) {
         const int c = count(e);
         tot += c;
         nmt += (c + a.tile_rows - 1) / a.tile_rows;
         npad += (c + a.row_align - 1) / a.row_align * a.row_align;
+        widest = max(widest, min(c, a.tile_rows));
     }
+    // the widest route tile (a block-wide max, through the scan's scratch)
+    widest = __reduce_max_sync(0xffffffffu, widest);
+    if ((tid & 31) == 0) s_warp[tid >> 5] = widest;
+    __syncthreads();
+    widest = 0;
+    for (int w = 0; w < kPermWarps; ++w) widest = max(widest, s_warp[w]);
+    __syncthreads();
     int sum_tot, sum_mt, sum_pad;
     int ex_tot = block_exclusive_scan<kPermWarps>(tot, s_warp, &sum_tot);
     int ex_mt = block_exclusive_scan<kPermWarps>(nmt, s_warp, &sum_mt);
@@ -130,6 +138,7 @@ __device__ __forceinline__ void scan_experts(const PermuteArgs& a, CountFn count
         a.padoff[E] = sum_pad;
         a.status[kStTotalRoutes] = (unsigned)sum_tot;
         a.status[kStCopyNext] = 0u;
+        a.status[kStMaxTileRows] = (unsigned)widest;
         __threadfence();
         a.status[kStNumMTiles] = (unsigned)sum_mt;
     }
