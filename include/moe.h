@@ -342,6 +342,74 @@ moe_status moe_ep_dispatch(const moe_plan* plan, int ep_size, const void* x, con
 moe_status moe_ep_combine(const moe_plan* plan, const float* y_rows, const int* route_rows,
                           const float* route_probs, const int* live_count_dev, void* out, void* stream);
 
+/* Expert-parallel exchange through peer memory (no counterpart to call in
+ * the pages, which put the EP transport inside their expert kernels:
+ * Megatron-LM PR #7830; the NCCL all-to-all of steps 2 and 4 above reads the
+ * split sizes on the host, Megatron-LM PR #7798, "Performance").  The same
+ * step with the exchange done by the library's kernels over NVLink peer
+ * memory, so that no host read of sizes is needed and one CUDA graph can
+ * capture the whole step.  Every rank owns one region of
+ * moe_ep_region_bytes(plan, ep_size) bytes (device memory, 256-byte aligned,
+ * zero-filled once before the first step) that every other rank maps (e.g.
+ * through moe_ep_ipc_handle / moe_ep_ipc_open); regions_dev is a device array
+ * of ep_size pointers, entry g = rank g's region as this rank addresses it
+ * (entry `rank` its own).  All ranks use plans of the same shape.  One step:
+ *   1. moe_ep_peer_dispatch: route, permute, and store every route's x row,
+ *      local expert id and FC1 weight into its owner's region (slot of this
+ *      source); then raise this source's flag in every owner's region;
+ *   2. moe_ep_peer_receive: wait until every source's flag is raised, then
+ *      compact the received rows into the region's recv_x / recv_ids /
+ *      recv_probs and set *recv_live (views below);
+ *   3. moe_forward of the rank's expert plan (as in step 3 above) with
+ *      x = recv_x, ids = recv_ids, probs = recv_probs, live = recv_live,
+ *      out = recv_y;
+ *   4. moe_ep_peer_return: store each received row's y into its source's
+ *      region at the route's send row; then raise this owner's return flag
+ *      in every source's region;
+ *   5. moe_ep_peer_combine: wait until every owner's return flag is raised,
+ *      then combine as moe_ep_combine.
+ * Every step of every rank runs in stream order; every wait is bounded by
+ * wait_limit_ns (> 0) and on expiry sets MOE_DEV_TIMEOUT in the region's
+ * status word, after which the rank's later kernels of the step do no work
+ * and its return flags stay down, so its sources time out too.  Flags carry
+ * the step number (kept in the region), so no flag needs clearing between
+ * steps.  The output is bitwise the one-GPU moe_forward's.  Not run across
+ * several GPUs in this library's tests (one GPU per test machine): the tests
+ * run every rank's steps in turn on one GPU, all regions in its memory. */
+#define MOE_EP_IPC_HANDLE_BYTES 64
+size_t moe_ep_region_bytes(const moe_plan* plan, int ep_size);
+typedef struct {
+    unsigned* status;  /* MOE_DEV_* bits of this rank's exchange (device word) */
+    int* recv_live;    /* device int: rows received this step (step 2)         */
+    void* recv_x;      /* bf16 [recv_rows, H]                                   */
+    int* recv_ids;     /* int32 [recv_rows]: expert id local to this rank       */
+    float* recv_probs; /* fp32 [recv_rows]: FC1 weight of the row               */
+    float* recv_y;     /* fp32 [recv_rows, H]: the expert forward's output       */
+    float* y_back;     /* fp32 [max_live_rows * k, H]: this rank's routes' y     */
+    long long recv_rows; /* ep_size * max_live_rows * k: the expert plan's capacity */
+} moe_ep_region_views;
+moe_status moe_ep_region_views_get(const moe_plan* plan, int ep_size, void* region, moe_ep_region_views* views);
+/* Step 1.  plan, ep_size, x, logits / ids + probs, live_count_dev,
+ * route_rows, route_probs, workspace: as moe_ep_dispatch; rank: this rank. */
+moe_status moe_ep_peer_dispatch(const moe_plan* plan, int ep_size, int rank, const void* x, const float* logits,
+                                const int* ids, const float* probs, const int* live_count_dev,
+                                void* const* regions_dev, int* route_rows, float* route_probs, void* workspace,
+                                size_t ws_bytes, void* stream);
+/* Step 2.  region: this rank's region. */
+moe_status moe_ep_peer_receive(const moe_plan* plan, int ep_size, void* region, unsigned long long wait_limit_ns,
+                               void* stream);
+/* Step 4. */
+moe_status moe_ep_peer_return(const moe_plan* plan, int ep_size, int rank, void* const* regions_dev, void* stream);
+/* Step 5.  out, route_rows, route_probs, live_count_dev: as moe_ep_combine. */
+moe_status moe_ep_peer_combine(const moe_plan* plan, int ep_size, void* region, const int* route_rows,
+                               const float* route_probs, const int* live_count_dev, void* out,
+                               unsigned long long wait_limit_ns, void* stream);
+/* CUDA IPC of a region between the ranks' processes (host calls, thin
+ * wrappers of the runtime's IPC handles; handle: MOE_EP_IPC_HANDLE_BYTES). */
+moe_status moe_ep_ipc_handle(void* dev_ptr, void* handle_out);
+moe_status moe_ep_ipc_open(const void* handle, void** dev_ptr_out);
+moe_status moe_ep_ipc_close(void* dev_ptr);
+
 /* Views into a workspace after a forward (device pointers into it), for
  * tests and diagnostics:
  *   route_ids/route_probs [max_live, k]: canonical routes of the last forward

@@ -54,6 +54,12 @@ class MoeError(RuntimeError):
         super().__init__(f"{what}: {_status_string(code)} (status {code})")
 
 
+class _EpViews(ctypes.Structure):
+    _fields_ = [("status", ctypes.c_void_p), ("recv_live", ctypes.c_void_p), ("recv_x", ctypes.c_void_p),
+                ("recv_ids", ctypes.c_void_p), ("recv_probs", ctypes.c_void_p), ("recv_y", ctypes.c_void_p),
+                ("y_back", ctypes.c_void_p), ("recv_rows", ctypes.c_longlong)]
+
+
 class _Desc(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int), ("ffn", ctypes.c_int), ("num_experts", ctypes.c_int),
                 ("top_k", ctypes.c_int), ("capacity", ctypes.c_longlong), ("max_live_rows", ctypes.c_longlong),
@@ -95,6 +101,15 @@ def load_library():
         "moe_forward_noalloc": ([P, P, P, P, P, P, P, P, P], I),
         "moe_ep_dispatch": ([P, I, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P], I),
         "moe_ep_combine": ([P, P, P, P, P, P, P], I),
+        "moe_ep_region_bytes": ([P, I], SZ),
+        "moe_ep_region_views_get": ([P, I, P, ctypes.POINTER(_EpViews)], I),
+        "moe_ep_peer_dispatch": ([P, I, I, P, P, P, P, P, P, P, P, P, SZ, P], I),
+        "moe_ep_peer_receive": ([P, I, P, ctypes.c_ulonglong, P], I),
+        "moe_ep_peer_return": ([P, I, I, P, P], I),
+        "moe_ep_peer_combine": ([P, I, P, P, P, P, P, ctypes.c_ulonglong, P], I),
+        "moe_ep_ipc_handle": ([P, P], I),
+        "moe_ep_ipc_open": ([P, ctypes.POINTER(P)], I),
+        "moe_ep_ipc_close": ([P], I),
         "moe_get_workspace_views": ([P, P, ctypes.POINTER(_Views)], I),
         "moe_get_device_status": ([P, ctypes.POINTER(ctypes.c_uint), P], I),
         "moe_clear_device_status": ([P, P], I),
@@ -301,6 +316,87 @@ def moe_ep_combine(plan: Plan, y_rows, route_rows, route_probs, live_count, out,
     _check_out(plan, out)
     _check(load_library().moe_ep_combine(plan.handle, _ptr(y_rows), _ptr(route_rows), _ptr(route_probs),
                                          _ptr(live_count), _ptr(out), _stream(stream)), "moe_ep_combine")
+
+
+# ---------------------------------------------------------------- peer-memory EP exchange
+
+MOE_EP_IPC_HANDLE_BYTES = 64
+EP_WAIT_LIMIT_NS = 4_000_000_000
+
+
+def moe_ep_region_bytes(plan: Plan, ep_size: int) -> int:
+    return int(load_library().moe_ep_region_bytes(plan.handle, int(ep_size)))
+
+
+def moe_ep_region_views(plan: Plan, ep_size: int, region) -> dict:
+    """Device tensors (views of `region`) of one rank's exchange state: status,
+    recv_live, recv_x, recv_ids, recv_probs, recv_y, y_back."""
+    import torch
+
+    v = _EpViews()
+    _check(load_library().moe_ep_region_views_get(plan.handle, int(ep_size), _ptr(region), ctypes.byref(v)),
+           "moe_ep_region_views_get")
+    base = region.data_ptr()
+    rows, H = int(v.recv_rows), plan.hidden
+
+    def view(ptr, n, dtype, shape):
+        off = ptr - base
+        return region[off:off + n * torch.empty((), dtype=dtype).element_size()].view(dtype).view(shape)
+
+    return {"status": view(v.status, 1, torch.int32, (1,)), "recv_live": view(v.recv_live, 1, torch.int32, (1,)),
+            "recv_x": view(v.recv_x, rows * H, torch.bfloat16, (rows, H)),
+            "recv_ids": view(v.recv_ids, rows, torch.int32, (rows, 1)),
+            "recv_probs": view(v.recv_probs, rows, torch.float32, (rows, 1)),
+            "recv_y": view(v.recv_y, rows * H, torch.float32, (rows, H)),
+            "y_back": view(v.y_back, plan.max_live_rows * plan.top_k * H, torch.float32,
+                           (plan.max_live_rows * plan.top_k, H)),
+            "recv_rows": rows}
+
+
+def moe_ep_peer_dispatch(plan: Plan, ep_size: int, rank: int, x, live_count, regions, route_rows, route_probs,
+                         workspace, logits=None, ids=None, probs=None, stream=None) -> None:
+    """Step 1 of the peer-memory EP step (include/moe.h): `regions` is a device
+    int64 tensor of the ep_size region addresses as this rank sees them."""
+    _check(load_library().moe_ep_peer_dispatch(plan.handle, int(ep_size), int(rank), _ptr(x), _ptr(logits), _ptr(ids),
+                                               _ptr(probs), _ptr(live_count), _ptr(regions), _ptr(route_rows),
+                                               _ptr(route_probs), _ptr(workspace),
+                                               workspace.numel() * workspace.element_size(), _stream(stream)),
+           "moe_ep_peer_dispatch")
+
+
+def moe_ep_peer_receive(plan: Plan, ep_size: int, region, wait_limit_ns: int = EP_WAIT_LIMIT_NS, stream=None):
+    _check(load_library().moe_ep_peer_receive(plan.handle, int(ep_size), _ptr(region), int(wait_limit_ns),
+                                              _stream(stream)), "moe_ep_peer_receive")
+
+
+def moe_ep_peer_return(plan: Plan, ep_size: int, rank: int, regions, stream=None) -> None:
+    _check(load_library().moe_ep_peer_return(plan.handle, int(ep_size), int(rank), _ptr(regions), _stream(stream)),
+           "moe_ep_peer_return")
+
+
+def moe_ep_peer_combine(plan: Plan, ep_size: int, region, route_rows, route_probs, live_count, out,
+                        wait_limit_ns: int = EP_WAIT_LIMIT_NS, stream=None) -> None:
+    _check_out(plan, out)
+    _check(load_library().moe_ep_peer_combine(plan.handle, int(ep_size), _ptr(region), _ptr(route_rows),
+                                              _ptr(route_probs), _ptr(live_count), _ptr(out), int(wait_limit_ns),
+                                              _stream(stream)), "moe_ep_peer_combine")
+
+
+def moe_ep_ipc_handle(region) -> bytes:
+    buf = ctypes.create_string_buffer(MOE_EP_IPC_HANDLE_BYTES)
+    _check(load_library().moe_ep_ipc_handle(_ptr(region), buf), "moe_ep_ipc_handle")
+    return buf.raw
+
+
+def moe_ep_ipc_open(handle: bytes) -> int:
+    out = ctypes.c_void_p()
+    _check(load_library().moe_ep_ipc_open(ctypes.create_string_buffer(bytes(handle), MOE_EP_IPC_HANDLE_BYTES),
+                                          ctypes.byref(out)), "moe_ep_ipc_open")
+    return int(out.value)
+
+
+def moe_ep_ipc_close(addr: int) -> None:
+    _check(load_library().moe_ep_ipc_close(ctypes.c_void_p(addr)), "moe_ep_ipc_close")
 
 
 MOE_NUM_STAGES = 6

@@ -566,6 +566,133 @@ moe_status moe_ep_combine(const moe_plan* plan, const float* y_rows, const int* 
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- peer-memory EP exchange
+
+size_t moe_ep_region_bytes(const moe_plan* plan, int ep_size) {
+    if (plan == nullptr || ep_size < 1 || ep_size > kEpMaxRanks) return 0;
+    return ep_region_layout(plan->d.hidden, (int)plan->max_live, plan->d.top_k, ep_size).total;
+}
+
+moe_status moe_ep_region_views_get(const moe_plan* plan, int ep_size, void* region, moe_ep_region_views* v) {
+    if (plan == nullptr || region == nullptr || v == nullptr) return MOE_ERR_INVALID_ARG;
+    if (ep_size < 1 || ep_size > kEpMaxRanks) return MOE_ERR_UNSUPPORTED;
+    const EpRegionLayout l = ep_region_layout(plan->d.hidden, (int)plan->max_live, plan->d.top_k, ep_size);
+    uint8_t* b = static_cast<uint8_t*>(region);
+    std::memset(v, 0, sizeof(*v));
+    v->status = reinterpret_cast<unsigned*>(b) + kEpStatus;
+    v->recv_live = reinterpret_cast<int*>(b) + kEpRecvLive;
+    v->recv_x = b + l.recv_x;
+    v->recv_ids = reinterpret_cast<int*>(b + l.recv_ids);
+    v->recv_probs = reinterpret_cast<float*>(b + l.recv_probs);
+    v->recv_y = reinterpret_cast<float*>(b + l.recv_y);
+    v->y_back = reinterpret_cast<float*>(b + l.y_back);
+    v->recv_rows = l.max_send * ep_size;
+    return MOE_OK;
+}
+
+moe_status moe_ep_peer_dispatch(const moe_plan* plan, int ep_size, int rank, const void* x, const float* logits,
+                                const int* ids, const float* probs, const int* live_count_dev,
+                                void* const* regions_dev, int* route_rows, float* route_probs, void* workspace,
+                                size_t ws_bytes, void* stream) {
+    if (plan == nullptr || x == nullptr || live_count_dev == nullptr || regions_dev == nullptr ||
+        route_rows == nullptr || route_probs == nullptr || workspace == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    const bool have_logits = logits != nullptr;
+    const bool have_routes = ids != nullptr && probs != nullptr;
+    if (have_logits == have_routes || ((ids == nullptr) != (probs == nullptr))) return MOE_ERR_INVALID_ARG;
+    const int H = plan->d.hidden, E = plan->d.num_experts, k = plan->d.top_k;
+    if (ep_size < 1 || ep_size > kEpMaxRanks || E % ep_size != 0) return MOE_ERR_UNSUPPORTED;
+    if (rank < 0 || rank >= ep_size) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < plan->ws.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned(x, 16) || !aligned(workspace, 256) || !aligned(regions_dev, 8)) return MOE_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int max_live = (int)plan->max_live;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const WsLayout& L = plan->ws;
+    unsigned* status = reinterpret_cast<unsigned*>(ws + L.status);
+    int* r_ids = reinterpret_cast<int*>(ws + L.r_ids);
+    float* r_probs = reinterpret_cast<float*>(ws + L.r_probs);
+    const bool blockscaled = plan->d.precision != MOE_BF16;
+    cudaError_t e = have_logits ? launch_route_topk(logits, live_count_dev, max_live, E, k, r_ids, r_probs, status, s)
+                                : launch_canon_routes(ids, probs, live_count_dev, max_live, E, k, r_ids, r_probs,
+                                                      status, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    int* inv = reinterpret_cast<int*>(ws + L.inv);
+    int* offsets = reinterpret_cast<int*>(ws + L.offsets);
+    int* padoff = reinterpret_cast<int*>(ws + L.padoff);
+    e = launch_permute(plan, live_count_dev, r_ids, reinterpret_cast<int*>(ws + L.blkcnt), offsets, padoff,
+                       reinterpret_cast<int4*>(ws + L.tiles), reinterpret_cast<int*>(ws + L.perm), inv,
+                       blockscaled ? nullptr : reinterpret_cast<int*>(ws + L.ready), status, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    const EpRegionLayout lay = ep_region_layout(H, max_live, k, ep_size);
+    e = launch_ep_peer_pack(x, live_count_dev, max_live, H, k, r_ids, r_probs, inv, offsets, padoff, E, ep_size, rank,
+                            (plan->d.flags & MOE_FLAG_PROBS_IN_FC1) != 0, regions_dev, lay, route_rows, route_probs,
+                            status, s);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_ep_peer_receive(const moe_plan* plan, int ep_size, void* region, unsigned long long wait_limit_ns,
+                               void* stream) {
+    if (plan == nullptr || region == nullptr) return MOE_ERR_INVALID_ARG;
+    if (ep_size < 1 || ep_size > kEpMaxRanks || plan->d.num_experts % ep_size != 0) return MOE_ERR_UNSUPPORTED;
+    if (wait_limit_ns == 0 || !aligned(region, 256)) return wait_limit_ns == 0 ? MOE_ERR_INVALID_ARG : MOE_ERR_ALIGNMENT;
+    const EpRegionLayout lay = ep_region_layout(plan->d.hidden, (int)plan->max_live, plan->d.top_k, ep_size);
+    const cudaError_t e = launch_ep_peer_receive(region, ep_size, plan->d.hidden, lay, wait_limit_ns,
+                                                 static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_ep_peer_return(const moe_plan* plan, int ep_size, int rank, void* const* regions_dev, void* stream) {
+    if (plan == nullptr || regions_dev == nullptr) return MOE_ERR_INVALID_ARG;
+    if (ep_size < 1 || ep_size > kEpMaxRanks || plan->d.num_experts % ep_size != 0) return MOE_ERR_UNSUPPORTED;
+    if (rank < 0 || rank >= ep_size) return MOE_ERR_INVALID_ARG;
+    const EpRegionLayout lay = ep_region_layout(plan->d.hidden, (int)plan->max_live, plan->d.top_k, ep_size);
+    const cudaError_t e = launch_ep_peer_return(regions_dev, nullptr, rank, ep_size, plan->d.hidden, lay,
+                                                static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_ep_peer_combine(const moe_plan* plan, int ep_size, void* region, const int* route_rows,
+                               const float* route_probs, const int* live_count_dev, void* out,
+                               unsigned long long wait_limit_ns, void* stream) {
+    if (plan == nullptr || region == nullptr || route_rows == nullptr || route_probs == nullptr ||
+        live_count_dev == nullptr || out == nullptr || wait_limit_ns == 0)
+        return MOE_ERR_INVALID_ARG;
+    if (ep_size < 1 || ep_size > kEpMaxRanks || plan->d.num_experts % ep_size != 0) return MOE_ERR_UNSUPPORTED;
+    if (!aligned(out, 16) || !aligned(region, 256)) return MOE_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const EpRegionLayout lay = ep_region_layout(plan->d.hidden, (int)plan->max_live, plan->d.top_k, ep_size);
+    cudaError_t e = launch_ep_peer_wait_returns(region, ep_size, wait_limit_ns, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    uint8_t* b = static_cast<uint8_t*>(region);
+    e = launch_combine(reinterpret_cast<const float*>(b + lay.y_back), route_rows, route_probs, live_count_dev,
+                       (int)plan->max_live, plan->d.hidden, plan->d.top_k, out,
+                       (plan->d.flags & MOE_FLAG_OUT_BF16) != 0, reinterpret_cast<const unsigned*>(b) + kEpStatus, s);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_ep_ipc_handle(void* dev_ptr, void* handle_out) {
+    if (dev_ptr == nullptr || handle_out == nullptr) return MOE_ERR_INVALID_ARG;
+    static_assert(sizeof(cudaIpcMemHandle_t) == MOE_EP_IPC_HANDLE_BYTES, "IPC handle size");
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, dev_ptr) != cudaSuccess) return MOE_ERR_CUDA;
+    std::memcpy(handle_out, &h, sizeof(h));
+    return MOE_OK;
+}
+
+moe_status moe_ep_ipc_open(const void* handle, void** dev_ptr_out) {
+    if (handle == nullptr || dev_ptr_out == nullptr) return MOE_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle, sizeof(h));
+    return cudaIpcOpenMemHandle(dev_ptr_out, h, cudaIpcMemLazyEnablePeerAccess) == cudaSuccess ? MOE_OK
+                                                                                                : MOE_ERR_CUDA;
+}
+
+moe_status moe_ep_ipc_close(void* dev_ptr) {
+    if (dev_ptr == nullptr) return MOE_ERR_INVALID_ARG;
+    return cudaIpcCloseMemHandle(dev_ptr) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status moe_get_workspace_views(const moe_plan* plan, const void* workspace, moe_workspace_views* v) {
     if (plan == nullptr || workspace == nullptr || v == nullptr) return MOE_ERR_INVALID_ARG;
     const uint8_t* ws = static_cast<const uint8_t*>(workspace);

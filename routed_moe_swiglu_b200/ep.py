@@ -18,10 +18,13 @@ rank partials and is not EP-invariant, which the ascending-id combine here
 is).  cudnn-frontend PR #448 (MoeEp API) names the same parts: a variable-size
 all-to-all dispatch, local experts and a top-k combine.
 
-The exchanges are ``torch.distributed`` all-to-alls (NCCL over NVLink between
-GPUs), which need the row counts on the host: step 2 reads them back, as an
-all-to-all dispatcher does.  Every other step is the library's kernels; this
-module only sequences them and moves bytes.
+``moe_forward_ep`` does the exchanges with ``torch.distributed`` all-to-alls
+(NCCL over NVLink between GPUs), which need the row counts on the host: step 2
+reads them back, as an all-to-all dispatcher does.  ``moe_forward_ep_peer``
+does them with the library's kernels storing rows into the peers' regions
+(``PeerRegions``), flags with bounded waits in place of the host read, so the
+whole step can be captured in one CUDA graph.  Every other step is the
+library's kernels; this module only sequences them and moves bytes.
 
 The phases (``dispatch``, ``expert_forward``, ``combine``) are separate so that
 a driver other than ``moe_forward_ep`` can run the exchange itself.
@@ -34,7 +37,9 @@ from dataclasses import dataclass
 from . import (MoeError, Plan, alloc_workspace, moe_ep_combine, moe_ep_dispatch, moe_forward, moe_plan_create)
 
 __all__ = ["expert_range", "shard_plan_create", "EpBuffers", "dispatch", "expert_forward", "combine",
-           "exchange_counts", "agree_on_receive_capacity", "exchange_rows", "moe_forward_ep"]
+           "exchange_counts", "agree_on_receive_capacity", "exchange_rows", "moe_forward_ep", "PeerRegions",
+           "peer_dispatch", "peer_receive", "peer_expert_forward", "peer_return", "peer_combine",
+           "moe_forward_ep_peer"]
 
 
 def expert_range(num_experts: int, ep_size: int, rank: int) -> tuple[int, int]:
@@ -207,3 +212,112 @@ def moe_forward_ep(plan: Plan, shard: Plan, bufs: EpBuffers, x, shard_wbuf, live
         expert_forward(shard, bufs, shard_wbuf, n_recv)
         exchange_rows(bufs.recv_y, recv_splits, send_splits, bufs.y_back, group)
         combine(plan, bufs, live_count, out)
+
+
+# ---------------------------------------------------------------- the exchange through peer memory
+
+
+class PeerRegions:
+    """One rank's exchange region (include/moe.h, "Expert-parallel exchange
+    through peer memory") and the device table of every rank's region as this
+    rank addresses it.
+
+    With a process group of ep_size ranks (one GPU each), the region's CUDA IPC
+    handle is exchanged through the group once and every peer's region is
+    mapped here.  Without one (`addresses` given), the table is taken as is:
+    the regions of several ranks in one GPU's memory, or ep_size 1."""
+
+    def __init__(self, plan: Plan, ep_size: int, rank: int, group=None, addresses=None, device=None, region=None):
+        import torch
+
+        from . import moe_ep_ipc_handle, moe_ep_ipc_open, moe_ep_region_bytes, moe_ep_region_views
+
+        self.plan, self.ep_size, self.rank = plan, ep_size, rank
+        dev = device or "cuda"
+        # zero-filled once: flags, counters and the step number start at 0
+        if region is None:
+            region = torch.zeros(moe_ep_region_bytes(plan, ep_size), dtype=torch.uint8, device=dev)
+        elif region.numel() < moe_ep_region_bytes(plan, ep_size):
+            raise ValueError("region smaller than moe_ep_region_bytes")
+        self.region = region
+        self._opened = []
+        if addresses is None:
+            if ep_size == 1:
+                addresses = [self.region.data_ptr()]
+            else:
+                import torch.distributed as dist
+
+                mine = torch.frombuffer(bytearray(moe_ep_ipc_handle(self.region)), dtype=torch.uint8)
+                handles = [torch.empty_like(mine) for _ in range(ep_size)]
+                dist.all_gather(handles, mine.to(dev) if dist.get_backend(group) == "nccl" else mine, group=group)
+                addresses = []
+                for g, h in enumerate(handles):
+                    if g == rank:
+                        addresses.append(self.region.data_ptr())
+                    else:
+                        a = moe_ep_ipc_open(bytes(h.cpu().numpy().tobytes()))
+                        self._opened.append(a)
+                        addresses.append(a)
+        self.addresses = list(addresses)
+        self.table = torch.tensor(self.addresses, dtype=torch.int64, device=dev)
+        self.views = moe_ep_region_views(plan, ep_size, self.region)
+
+    def close(self):
+        from . import moe_ep_ipc_close
+
+        for a in self._opened:
+            moe_ep_ipc_close(a)
+        self._opened = []
+
+
+def peer_dispatch(plan: Plan, peer: PeerRegions, x, live_count, route_rows, route_probs, workspace, logits=None,
+                  ids=None, probs=None, stream=None) -> None:
+    from . import moe_ep_peer_dispatch
+
+    moe_ep_peer_dispatch(plan, peer.ep_size, peer.rank, x, live_count, peer.table, route_rows, route_probs, workspace,
+                         logits=logits, ids=ids, probs=probs, stream=stream)
+
+
+def peer_receive(plan: Plan, peer: PeerRegions, wait_limit_ns=None, stream=None) -> None:
+    from . import EP_WAIT_LIMIT_NS, moe_ep_peer_receive
+
+    moe_ep_peer_receive(plan, peer.ep_size, peer.region, wait_limit_ns or EP_WAIT_LIMIT_NS, stream=stream)
+
+
+def peer_expert_forward(shard: Plan, peer: PeerRegions, shard_wbuf, shard_workspace, stream=None) -> None:
+    v = peer.views
+    moe_forward(shard, v["recv_x"], shard_wbuf, v["recv_live"], v["recv_y"], shard_workspace, ids=v["recv_ids"],
+                probs=v["recv_probs"], stream=stream)
+
+
+def peer_return(plan: Plan, peer: PeerRegions, stream=None) -> None:
+    from . import moe_ep_peer_return
+
+    moe_ep_peer_return(plan, peer.ep_size, peer.rank, peer.table, stream=stream)
+
+
+def peer_combine(plan: Plan, peer: PeerRegions, route_rows, route_probs, live_count, out, wait_limit_ns=None,
+                 stream=None) -> None:
+    from . import EP_WAIT_LIMIT_NS, moe_ep_peer_combine
+
+    moe_ep_peer_combine(plan, peer.ep_size, peer.region, route_rows, route_probs, live_count, out,
+                        wait_limit_ns or EP_WAIT_LIMIT_NS, stream=stream)
+
+
+def moe_forward_ep_peer(plan: Plan, shard: Plan, peer: PeerRegions, x, shard_wbuf, shard_workspace, live_count, out,
+                        route_rows, route_probs, workspace, logits=None, ids=None, probs=None, stream=None) -> None:
+    """One EP step on this rank with the exchange through peer memory: no host
+    synchronisation, so a CUDA graph can capture it.  `shard` is the rank's
+    expert plan (shard_plan_create(plan, ep_size, peer.views["recv_rows"]));
+    route_rows [max_live, k] int32 and route_probs [max_live, k] fp32 are the
+    step's scratch.  Every rank of the step calls it together."""
+    if shard.capacity < peer.views["recv_rows"]:
+        raise ValueError(f"the expert plan holds {shard.capacity} rows, the exchange can bring "
+                         f"{peer.views['recv_rows']}")
+    with _on(stream):
+        peer_dispatch(plan, peer, x, live_count, route_rows, route_probs, workspace, logits=logits, ids=ids,
+                      probs=probs)
+        peer_receive(plan, peer)
+        peer_expert_forward(shard, peer, shard_wbuf, shard_workspace)
+        peer_return(plan, peer)
+        peer_combine(plan, peer, route_rows, route_probs, live_count, out)

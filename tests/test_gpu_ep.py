@@ -18,7 +18,7 @@ import torch
 import oracle
 import routed_moe_swiglu_b200 as rm
 import workloads
-from moe_testlib import GpuMoe
+from moe_testlib import GpuMoe, assert_close
 from routed_moe_swiglu_b200 import ep as moe_ep
 
 pytestmark = pytest.mark.gpu
@@ -221,3 +221,20 @@ def test_ep_step_through_nccl_with_one_rank():
             assert bufs.send_counts.tolist() == [T * K]
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("precision", ["bf16", "mxfp8", "nvfp4"])
+def test_ep_output_against_the_oracle(precision):
+    """The EP step at EP 2 against the oracle directly, every token."""
+    T = 120
+    x, logits, weights = workloads.small_case(H, F, E, K, T, seed=33, zipf=True)
+    ranks, _ = _run_ep(precision, 2, x, logits, weights, [0, 70, T])
+    got = torch.cat([ranks[0].out[:70], ranks[1].out[:T - 70]]).float().cpu().numpy()
+    ids, probs = oracle.route(logits[:T].numpy(), K)
+    if precision == "bf16":
+        ref = oracle.forward_bf16(x[:T], ids, probs, *weights)
+    elif precision == "mxfp8":
+        ref = oracle.forward_mxfp8(x[:T], ids, probs, oracle.quantize_weights_mxfp8(*weights))
+    else:
+        ref = oracle.forward_nvfp4(x[:T], ids, probs, oracle.quantize_weights_nvfp4(*weights))
+    assert_close(got, ref, precision, f"EP 2 ({precision}) against the oracle")
