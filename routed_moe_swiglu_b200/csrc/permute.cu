@@ -148,22 +148,24 @@ __device__ __forceinline__ void scan_experts(const PermuteArgs& a, CountFn count
 // (the chunk's first free row of expert e) plus its rank in the chunk;
 // s_base[e] is advanced past the chunk.  s_off / s_pad map a row to its
 // padded row.
-__device__ __forceinline__ void scatter_chunk(const PermuteArgs& a, int n, int t0, int* s_base, const int* s_off,
-                                              const int* s_pad, uint32_t* masks, int* wbase) {
+// The k canonical expert ids of token t (all -1 past the live count), loaded together.
+__device__ __forceinline__ void load_token_ids(const PermuteArgs& a, int t, int n, int (&ids)[kMaxTopK]) {
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) ids[j] = (j < a.k && t < n) ? __ldg(a.ids + (size_t)t * a.k + j) : -1;
+}
+
+// my_e: the ids of this thread's token t0 + threadIdx.x (load_token_ids).
+__device__ __forceinline__ void scatter_chunk(const PermuteArgs& a, int n, int t0, const int (&my_e)[kMaxTopK],
+                                              int* s_base, const int* s_off, const int* s_pad, uint32_t* masks,
+                                              int* wbase) {
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, E = a.E, k = a.k;
     for (int i = tid; i < kPermWarps * E; i += kTokPerBlk) masks[i] = 0u;
     __syncthreads();
     const int t = t0 + tid;
     const bool is_live = t < n;
-    int my_e[kMaxTopK];
 #pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-        my_e[j] = -1;
-        if (j < k && is_live) {
-            my_e[j] = __ldg(a.ids + (size_t)t * k + j);
-            if (my_e[j] >= 0) atomicOr(&masks[w * E + my_e[j]], 1u << lane);
-        }
-    }
+    for (int j = 0; j < kMaxTopK; ++j)
+        if (j < k && my_e[j] >= 0) atomicOr(&masks[w * E + my_e[j]], 1u << lane);
     __syncthreads();
     for (int e = tid; e < E; e += kTokPerBlk) {
         int base = s_base[e];
@@ -217,7 +219,7 @@ __global__ void __launch_bounds__(kTokPerBlk) route_permute_kernel(const Permute
     extern __shared__ int s_perm[];
     __shared__ int s_warp[32];
     __shared__ int s_flag;
-    const int E = a.E, k = a.k;
+    const int E = a.E;
     int* s_count = s_perm;
     int* s_off = s_perm + E;
     int* s_pad = s_perm + 2 * E;
@@ -233,17 +235,38 @@ __global__ void __launch_bounds__(kTokPerBlk) route_permute_kernel(const Permute
         // one block: histogram, scan, scatter in chunks of 256 with a running base
         if (blockIdx.x == 0) {
             for (int e = tid; e < E; e += kTokPerBlk) s_count[e] = 0;
+            // thread tid takes token tid of each chunk; the first chunk's ids stay in
+            // registers for its scatter (decode: the only chunk)
+            int first[kMaxTopK];
+            load_token_ids(a, tid, n, first);
             __syncthreads();
-            for (int i = tid; i < n * k; i += kTokPerBlk) {
-                const int e = __ldg(a.ids + i);
-                if (e >= 0) atomicAdd(&s_count[e], 1);
+            for (int t0 = 0; t0 < n; t0 += kTokPerBlk) {
+                int ids[kMaxTopK];
+                if (t0 == 0) {
+#pragma unroll
+                    for (int j = 0; j < kMaxTopK; ++j) ids[j] = first[j];
+                } else {
+                    load_token_ids(a, t0 + tid, n, ids);
+                }
+#pragma unroll
+                for (int j = 0; j < kMaxTopK; ++j)
+                    if (ids[j] >= 0) atomicAdd(&s_count[ids[j]], 1);
             }
             __syncthreads();
             scan_experts(a, [&](int e) { return s_count[e]; }, s_off, s_pad, s_warp, true);
             __syncthreads();
             for (int e = tid; e < E; e += kTokPerBlk) s_count[e] = s_off[e];  // next free row of expert e
             __syncthreads();
-            for (int t0 = 0; t0 < n; t0 += kTokPerBlk) scatter_chunk(a, n, t0, s_count, s_off, s_pad, masks, wbase);
+            for (int t0 = 0; t0 < n; t0 += kTokPerBlk) {
+                int ids[kMaxTopK];
+                if (t0 == 0) {
+#pragma unroll
+                    for (int j = 0; j < kMaxTopK; ++j) ids[j] = first[j];
+                } else {
+                    load_token_ids(a, t0 + tid, n, ids);
+                }
+                scatter_chunk(a, n, t0, ids, s_count, s_off, s_pad, masks, wbase);
+            }
         }
         pdl_trigger();
         return;
@@ -257,14 +280,13 @@ __global__ void __launch_bounds__(kTokPerBlk) route_permute_kernel(const Permute
     }
     // phase 1: the histogram of each chunk this block owns
     for (int c = blockIdx.x; c < nb; c += parts) {
+        int ids[kMaxTopK];
+        load_token_ids(a, c * kTokPerBlk + tid, n, ids);
         for (int e = tid; e < E; e += kTokPerBlk) s_count[e] = 0;
         __syncthreads();
-        const int t = c * kTokPerBlk + tid;
-        if (t < n)
-            for (int j = 0; j < k; ++j) {
-                const int e = __ldg(a.ids + (size_t)t * k + j);
-                if (e >= 0) atomicAdd(&s_count[e], 1);
-            }
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j)
+            if (ids[j] >= 0) atomicAdd(&s_count[ids[j]], 1);
         __syncthreads();
         for (int e = tid; e < E; e += kTokPerBlk) a.blkcnt[(size_t)c * E + e] = s_count[e];
         __syncthreads();
@@ -302,9 +324,11 @@ __global__ void __launch_bounds__(kTokPerBlk) route_permute_kernel(const Permute
     scan_experts(a, [&](int e) { return __ldcg(a.tot + e); }, s_off, s_pad, s_warp, blockIdx.x == 0);
     __syncthreads();
     for (int c = blockIdx.x; c < nb; c += parts) {
+        int ids[kMaxTopK];
+        load_token_ids(a, c * kTokPerBlk + tid, n, ids);
         for (int e = tid; e < E; e += kTokPerBlk) s_count[e] = s_off[e] + __ldcg(a.blkcnt + (size_t)c * E + e);
         __syncthreads();
-        scatter_chunk(a, n, c * kTokPerBlk, s_count, s_off, s_pad, masks, wbase);
+        scatter_chunk(a, n, c * kTokPerBlk, ids, s_count, s_off, s_pad, masks, wbase);
     }
     pdl_trigger();
 }
