@@ -202,3 +202,38 @@ def test_ep_entries_reject_bad_arguments_before_launch():
     assert lib.moe_ep_combine(p.handle, f, f, f, f, null, null) == 1
     assert lib.moe_ep_combine(None, f, f, f, f, f, null) == 1
     assert lib.moe_ep_combine(p.handle, ctypes.c_void_p((1 << 20) + 4), f, f, f, f, null) == 3
+
+
+def test_ep_peer_region_size_and_argument_checks():
+    """The peer-memory exchange's region: a header, one receive slot per source
+    of max_live * k rows (x, id, weight), the returned y rows, the compacted
+    received rows; host-side checks before any launch."""
+    lib = rm.load_library()
+    H, k, cap = 256, 2, 64
+    p = rm.moe_plan_create(hidden=H, ffn=512, num_experts=8, top_k=k, capacity=cap)
+    send = cap * k
+    sizes = {ep: rm.moe_ep_region_bytes(p, ep) for ep in (1, 2, 4, 8)}
+    for ep, b in sizes.items():
+        # slots ep * send * (2H + 8) + y_back send * 4H + received ep * send * (2H + 8 + 4H + 8)
+        floor = ep * send * (2 * H + 8) + send * 4 * H + ep * send * (2 * H + 4 * H + 16)
+        assert floor <= b <= floor + 4096 + 16 * 256, (ep, b, floor)
+    assert sizes[2] > sizes[1] and sizes[4] > sizes[2]
+    assert rm.moe_ep_region_bytes(p, 0) == 0 and rm.moe_ep_region_bytes(p, 129) == 0
+    f = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    null = None
+    ws = rm.moe_workspace_bytes(p)
+
+    def dispatch(ep=2, rank=0, logits=f, table=f, wsb=ws):
+        return lib.moe_ep_peer_dispatch(p.handle, ep, rank, f, logits, null, null, f, table, f, f, f, wsb, null)
+
+    assert dispatch(ep=3) == 2       # 3 does not divide the 8 experts
+    assert dispatch(rank=2) == 1     # rank outside [0, ep)
+    assert dispatch(rank=-1) == 1
+    assert dispatch(logits=null) == 1
+    assert dispatch(table=null) == 1
+    assert dispatch(wsb=ws - 1) == 4
+    assert lib.moe_ep_peer_receive(p.handle, 2, f, 0, null) == 1                          # no wait limit
+    assert lib.moe_ep_peer_receive(p.handle, 2, ctypes.c_void_p((1 << 20) + 64), 1000, null) == 3
+    assert lib.moe_ep_peer_return(p.handle, 2, 2, f, null) == 1
+    assert lib.moe_ep_peer_combine(p.handle, 2, f, f, f, f, null, 1000, null) == 1
+    assert lib.moe_ep_peer_combine(p.handle, 5, f, f, f, f, f, 1000, null) == 2
