@@ -183,6 +183,11 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
             tma_prefetch_desc(&tmA);
             if (kMode == 0) tma_prefetch_desc(tmX);
         }
+        // When no expert has more than one route tile (decode), every weight tile is read by
+        // one unit only: its lines go first out of L2, which keeps the h and y rows that the
+        // next kernels read resident there instead of written back and read from HBM.
+        const bool weights_once = (int)p.status_words[kStMaxTileRows] < kRouteTile;
+        const uint64_t pol_once = l2_policy_evict_first();
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -243,7 +248,10 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
                         last_phase[stage] = (int)phase;
                     }
                     // boxes land as [atom][row][64 elements]
-                    tma_load_3d_pair(sA + stage * kABytes, &tmA, full0, 0, 0, a_atom0 + kb * kAtoms);
+                    if (weights_once)
+                        tma_load_3d_pair_hint(sA + stage * kABytes, &tmA, full0, 0, 0, a_atom0 + kb * kAtoms, pol_once);
+                    else
+                        tma_load_3d_pair(sA + stage * kABytes, &tmA, full0, 0, 0, a_atom0 + kb * kAtoms);
                     if (!from_x)
                         tma_load_3d_pair(sB + stage * kBBytes, &tmB->m[(hb >> 4) - 1], full0, 0, b_row,
                                          kb * kAtoms);
