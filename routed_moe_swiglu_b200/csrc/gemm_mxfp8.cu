@@ -213,6 +213,10 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
         if (lane == 0) {
             // ---------------- TMA producer
             tma_prefetch_desc(&tmA);
+            // no expert with more than one route tile (decode): each weight tile is read by
+            // one CTA only, and its lines go first out of L2 (the h and y rows stay)
+            const bool weights_once = (int)p.status_words[kStMaxTileRows] < kBM;
+            const uint64_t pol_once = l2_policy_evict_first();
             int stage = 0;
             uint32_t phase = 0;
             uint32_t groups = 0;  // scale-factor groups issued so far
@@ -250,7 +254,10 @@ __device__ __forceinline__ void gemm_mxfp8_body(const CUtensorMap& tmA, const Bo
                     }
                     mbar_arrive_expect_tx(&bars->full[stage], tx);
                     last_phase[stage] = (int)phase;
-                    tma_load_3d(stage_a(stage), &tmA, &bars->full[stage], 0, a_row, blk0);
+                    if (weights_once)
+                        tma_load_3d_hint(stage_a(stage), &tmA, &bars->full[stage], 0, a_row, blk0, pol_once);
+                    else
+                        tma_load_3d(stage_a(stage), &tmA, &bars->full[stage], 0, a_row, blk0);
                     tma_load_3d(stage_b(stage), mapB, &bars->full[stage], 0, ti.y, blk0);
                     if (gs > 0) {
                         const int sb = (int)(groups & 1u);
