@@ -341,6 +341,18 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
         const uint32_t acc_empty0[2] = {map_to_cta(smem_u32(&bars->acc_empty[0]), 0),
                                         map_to_cta(smem_u32(&bars->acc_empty[1]), 0)};
         uint8_t* tbuf = sEpi + (size_t)ew * (kMode == 0 ? kH0Bytes : kYTBytes);
+        // Experts with several route tiles (prefill): the weights and route rows are read
+        // again by other units while h / y (larger than L2) stream out; the output lines go
+        // first out of L2 so that they do not push the operands out.  With one tile per
+        // expert (decode) the outputs stay, for the next kernel to read from L2.
+        const bool out_first = (int)p.status_words[kStMaxTileRows] >= kRouteTile;
+        const uint64_t pol_out = l2_policy_evict_first();
+        auto store_out = [&](void* dst, uint4 w) {
+            if (out_first)
+                st_global_v4_hint(dst, w, pol_out);
+            else
+                *reinterpret_cast<uint4*>(dst) = w;
+        };
         int it = 0;
         for (int t = pair; t < total_tiles; t += npairs, ++it) {
             const int buf = it & 1;
@@ -389,8 +401,7 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
                             const int route = c * 32 + r;
                             const uint4 w = *reinterpret_cast<const uint4*>(tbuf + r * 64 + (lane & 3) * 16);
                             if (route < ti.z)
-                                *reinterpret_cast<uint4*>(h + (size_t)(ti.y + route) * (size_t)p.out_ld + f0 +
-                                                          (lane & 3) * 8) = w;
+                                store_out(h + (size_t)(ti.y + route) * (size_t)p.out_ld + f0 + (lane & 3) * 8, w);
                         }
                         __syncwarp();
                     }
@@ -432,8 +443,7 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
                         const uint4 w = *reinterpret_cast<const uint4*>(tbuf + r * 32 + (r >= 16 ? 64 : 0) +
                                                                         (lane & 1) * 16);
                         if (route < ti.z)
-                            *reinterpret_cast<uint4*>(h + (size_t)(ti.y + route) * (size_t)p.out_ld + f_base +
-                                                      (lane & 1) * 8) = w;
+                            store_out(h + (size_t)(ti.y + route) * (size_t)p.out_ld + f_base + (lane & 1) * 8, w);
                     }
                     __syncwarp();
                 }
@@ -458,8 +468,7 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
                             const int route = c * 32 + r;
                             const uint4 w = *reinterpret_cast<const uint4*>(tbuf + r * 128 + (lane & 7) * 16);
                             if (col_ok && route < ti.z)
-                                *reinterpret_cast<uint4*>(y + (size_t)(ti.y + route) * (size_t)p.out_ld + c_base +
-                                                          (lane & 7) * 4) = w;
+                                store_out(y + (size_t)(ti.y + route) * (size_t)p.out_ld + c_base + (lane & 7) * 4, w);
                         }
                         __syncwarp();
                     }
