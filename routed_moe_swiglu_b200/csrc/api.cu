@@ -449,6 +449,7 @@ static moe_status forward_impl(const moe_plan* plan, const void* x, const float*
     g1.xg_pitch = plan->hp * 2;
     g1.ready = ready;
     g1.copy_next = status + kStCopyNext;
+    g1.tile_started = reinterpret_cast<int*>(status + kStTileStarted);
     g1.row_scale = fp4 ? reinterpret_cast<const float*>(ws + L.xg) : nullptr;
     g1.w_scale = fp4 ? reinterpret_cast<const float*>(wb + plan->wb.wg) : nullptr;
     g1.h_fp32 = fp8 && L.hf != 0 ? reinterpret_cast<float*>(ws + L.hf) : nullptr;

@@ -59,6 +59,7 @@ namespace {
 constexpr int kStagesMax = 5;  // pipeline stages per launch: 3..5, by the widest route tile (see StageCfg)
 constexpr int kEpiWarps = 8;
 constexpr int kCopyWarps = 2;                           // gate/up: x rows of large tiles into their route rows
+constexpr int kCopyAhead = 16;                          // route tiles the copy may run ahead of the producers
 constexpr int kPairM = 256;                             // M of the pair MMA (weight rows)
 constexpr int kAtoms = 2;                               // 64-element (128-byte) swizzle atoms per K stage
 constexpr int kStageK = kAtoms * kBK;                   // 128 K elements per stage
@@ -212,6 +213,7 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
             int tok[4] = {0, 0, 0, 0};
             const bool from_x = kMode == 0 && ti.z <= kGatherInGemmMax;
             const bool gathers = from_x && 4 * lane < hb;
+            if (kMode == 0 && leader && lane == 0) atomicMax(p.tile_started, mt);  // lets the copy warps on
             if (kMode == 0 && !from_x) {
                 // the copy warps (of any CTA) have written all of this tile's route rows:
                 // acquire their counts, then order them before this thread's TMA reads
@@ -496,6 +498,20 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
             const int r0 = (int)(u % kChunksPerTile) * kCopyChunk;
             const int4 ti = __ldg(p.tiles + mt);
             if (ti.z <= kGatherInGemmMax || r0 >= ti.z) continue;
+            // stay at most kCopyAhead tiles ahead of the highest tile a producer has started:
+            // rows copied further ahead would leave L2 before their loads and come back from
+            // HBM.  A producer marks its tile before it waits for the tile's rows, so this
+            // wait ends whenever a producer waits on this chunk.
+            bool go = true;
+            if (lane == 0 && mt > kCopyAhead)
+                go = wait_count_bounded(p.tile_started, mt - kCopyAhead, abort_flag, p.wait_limit_ns);
+            if (!__shfl_sync(0xffffffffu, go, 0)) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    atomicOr(p.status_flags, MOE_DEV_TIMEOUT);
+                }
+                break;
+            }
             const int nrows = min(kCopyChunk, ti.z - r0);
             const int my_tok = lane < nrows ? __ldg(p.perm + ti.w + r0 + lane) / p.top_k : 0;
             // two rows at a time: 16 loads of 16 bytes in flight per lane

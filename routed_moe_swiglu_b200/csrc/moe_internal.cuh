@@ -37,6 +37,8 @@ constexpr int kMaxExperts = 1024;
 // kStPermBar: arrivals at the permute's grid-wide barriers, zeroed by the router kernel
 // (route or canonicalise) that precedes the permute in every forward.  kStMaxTileRows:
 // the most routes in one route tile of this forward (the GEMMs size their pipelines by it).
+// kStTileStarted: the highest route tile a bf16 gate/up producer has started (zeroed with
+// the tile list); the copy warps stay a bounded distance ahead of it.
 enum : int {
     kStFlags = 0,
     kStNumMTiles = 1,
@@ -44,6 +46,7 @@ enum : int {
     kStCopyNext = 3,
     kStPermBar = 4,
     kStMaxTileRows = 5,
+    kStTileStarted = 6,
     kStWords = 64
 };
 
@@ -134,6 +137,7 @@ struct GemmParams {
     long long xg_pitch;
     int* ready;
     unsigned* copy_next;
+    int* tile_started;              // highest route tile whose loads a producer has started
     // NVFP4: second-level scales of the B rows (fp32 per padded route row: x for the
     // gate/up GEMM, h for the down GEMM) and of the weights ([E][2]: W1, W2)
     const float* row_scale;

@@ -138,6 +138,7 @@ __device__ __forceinline__ void scan_experts(const PermuteArgs& a, CountFn count
         a.padoff[E] = sum_pad;
         a.status[kStTotalRoutes] = (unsigned)sum_tot;
         a.status[kStCopyNext] = 0u;
+        a.status[kStTileStarted] = 0u;
         a.status[kStMaxTileRows] = (unsigned)widest;
         __threadfence();
         a.status[kStNumMTiles] = (unsigned)sum_mt;
