@@ -213,7 +213,8 @@ __device__ __forceinline__ void pair_gemm_body(const CUtensorMap& tmA, const CUt
             int tok[4] = {0, 0, 0, 0};
             const bool from_x = kMode == 0 && ti.z <= kGatherInGemmMax;
             const bool gathers = from_x && 4 * lane < hb;
-            if (kMode == 0 && leader && lane == 0) atomicMax(p.tile_started, mt);  // lets the copy warps on
+            // mark this tile as started: the copy warps may now run up to kCopyAhead tiles past it
+            if (kMode == 0 && leader && lane == 0) atomicMax(p.tile_started, mt);
             if (kMode == 0 && !from_x) {
                 // the copy warps (of any CTA) have written all of this tile's route rows:
                 // acquire their counts, then order them before this thread's TMA reads

@@ -334,7 +334,7 @@ __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m
         "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar_cluster), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
-// The same load with an L2 eviction policy (createpolicy below) for its lines.
+// The same load with an L2 eviction policy (l2_policy_evict_first) for its lines.
 __device__ __forceinline__ void tma_load_3d_pair_hint(void* dst, const CUtensorMap* map, uint32_t mbar_cluster,
                                                       int c0, int c1, int c2, uint64_t policy) {
     asm volatile(
@@ -343,8 +343,10 @@ __device__ __forceinline__ void tma_load_3d_pair_hint(void* dst, const CUtensorM
         "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar_cluster), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
         : "memory");
 }
-// L2 policy for data read once: its lines are the first evicted, so that they
-// do not push out lines that are read again (outputs that the next kernel reads).
+// L2 policy whose lines are the first evicted: for data that is not read again
+// soon (a weight tile read by one unit, an output larger than L2), so that it
+// does not push out lines that are (operands read again, outputs the next kernel
+// reads from L2).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
