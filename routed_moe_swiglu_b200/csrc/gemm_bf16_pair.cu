@@ -43,8 +43,11 @@
 // dispatch fused into the GEMM: no separate gather pass over HBM).  They
 // claim 8-route chunks in tile order from a global counter and count each
 // finished chunk in its tile's ready counter; a producer acquires that count
-// before the tile's first route-row load.  The copy warps wait on nothing,
-// and every CTA of the persistent grid is resident, so those waits end.
+// before the tile's first route-row load.  The copy runs at most 16 tiles
+// ahead of the highest tile a producer has started (rows copied further ahead
+// leave L2 before their loads); a producer marks its tile before it waits for
+// the tile's rows, chunks are claimed in tile order, and every CTA of the
+// persistent grid is resident, so every one of these waits ends.
 //
 // Every mbarrier wait is bounded; the pair meets in cluster barriers only at
 // start-up and before TMEM is released.  Each output element is one route's
