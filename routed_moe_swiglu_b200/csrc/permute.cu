@@ -20,8 +20,8 @@
 // workspace's status words, zeroed by the router kernel of the same forward;
 // every wait bounded).  With at most 1,024 live rows one block does all three
 // phases and no barrier is needed.  The scan also zeroes the per-tile
-// counters and the chunk counter through which the bf16 gate/up GEMM copies
-// x rows itself.  For MXFP8, a gather then quantises each token's x row once
+// counters, the chunk counter and the started-tile mark through which the
+// bf16 gate/up GEMM copies x rows itself.  For MXFP8, a gather then quantises each token's x row once
 // and writes it to its padded route rows.
 #include "moe_internal.cuh"
 #include "mxfp8.cuh"
